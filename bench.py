@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Throughput of the QE linear layer on B200: one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the hot path over one batch: every projection of the
+workload's layer set goes through qe_linear_forward. Each forward is router
++ bucket sort, per-token quantization, adapter down-projection, and the int8
+tcgen05 product with its adapter epilogue. Inputs are synthetic and seeded,
+with the shapes of the named model (qe_inputs), and resident in HBM when the
+timed region starts. L2 is flushed between steps, outside the per-step event
+pairs. The step time is the sum of the per-step event pairs. Under torchrun
+each rank runs an independent replica on its own token batch (weak
+scaling, no data-path collective), and the time is the max over ranks.
+
+`--impl reference` times the CPU oracle (a deliberately slow, plain program)
+on a bounded token sample of the same workload, on the host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import qe_inputs as qi  # noqa: E402
+
+WORKLOADS = {
+    # name: (config, T override, description)
+    "qwen2vl2b": ("qwen2vl2b", None, "Qwen2VL-2B-shaped layer set (q,o 1536x1536; gate,up 1536->8960; down 8960->1536), "
+                                     "T=2048, W4A6 g128, r_s=32, N_r=8, r_r=4"),
+    "internvl2_8b": ("internvl2_8b", None, "InternVL2-8B-shaped layer set, T=4096, W4A8 g128"),
+    "qwen2vl72b": ("qwen2vl72b", None, "Qwen2VL-72B-shaped layer set, T=8192, W4A6 g128"),
+    "decode72b_w4a8": ("decode72b_w4a8", 16, "72B decode gate/up/down, T=16, W4A8 g128"),
+    "decode72b_w4a8_t1": ("decode72b_w4a8", 1, "72B decode gate/up/down, T=1, W4A8 g128"),
+    "decode72b_w3a16": ("decode72b_w3a16", 16, "72B decode gate/up/down, T=16, W3A16 g128"),
+    "decode72b_w3a16_t1": ("decode72b_w3a16", 1, "72B decode gate/up/down, T=1, W3A16 g128"),
+}
+METRIC = "QE linear tokens/s and effective TOPS; % of int8-TC / HBM roofline, 1 B200"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2vl2b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=64)
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "bf16_tflops": d.get("bf16_tflops", 1590.0),
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", 1400.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def git_src_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel_file: str, name: str):
+    """Per-launch DRAM bytes from a committed ncu summary (profiles/<name>.md), or None when
+    absent or when the kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", name + ".md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    try:
+        if vals.get("source_hash") != git_src_hash([kernel_file]):
+            return None
+        return float(vals["dram_bytes_per_launch_full_workload"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() in ("active", "1", "yes"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- reference arm (CPU oracle)
+
+def oracle_sample_run(cfg, T_total, sample_tokens, seed_shift=0):
+    """Times the oracle's forward over `sample_tokens` tokens of every projection. Returns seconds."""
+    import oracle
+    prep = []
+    for pi, proj in enumerate(cfg.projections):
+        inp = qi.layer_inputs(cfg, proj, T=sample_tokens, proj_index=pi + seed_shift)
+        codes, scales, _, _ = oracle.quantize_weights(inp["W"], inp["s"], cfg.group, cfg.w_bits)
+        prep.append((inp, codes, scales))
+    t0 = time.perf_counter()
+    for inp, codes, scales in prep:
+        oracle.qe_forward(inp["X"], codes, scales, inp["s_inv"], inp["A_s"], inp["B_s"], inp["A_r"], inp["B_r"],
+                          inp["G"], cfg.group, cfg.a_bits)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, workload):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    cfg_name, t_over, desc = WORKLOADS[workload]
+    cfg = qi.CONFIGS[cfg_name]
+    T = t_over or cfg.T
+    cores = os.cpu_count() or 1
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    sample = max(1, min(args.cpu_sample_tokens, T))
+    for _ in range(args.warmup):
+        oracle_sample_run(cfg, T, min(sample, 4))
+    secs = [oracle_sample_run(cfg, T, sample) for _ in range(args.steps)]
+    tot = sum(secs)
+    value = sample * args.steps / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64", "data": "synthetic",
+        "config": {"workload": workload, "description": desc, "T": T, "sample_tokens_per_step": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{sample} tokens of every projection per step (tokens are independent)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+
+def build_layers(cfg, T, rank, dev):
+    import torch
+    import quantized_gemm_moe_b200 as qe
+    layers = []
+    for pi, proj in enumerate(cfg.projections):
+        inp = qi.layer_inputs(cfg, proj, T=T, proj_index=pi)
+        if rank:
+            # each replica gets its own token batch (same weights)
+            spec = cfg.outlier_spec(proj.d_in)
+            x = qi.outlier_activations(T, proj.d_in, 1000 + 7919 * rank + pi, spec)
+            inp["X"] = qi.to_bf16(x) if cfg.x_dtype == "bf16" else x
+        desc = qe.make_desc(proj.d_in, proj.d_out, cfg.group, cfg.w_bits, cfg.a_bits, cfg.rank_shared, cfg.n_routed,
+                            cfg.rank_routed)
+
+        def c(a):
+            t = torch.from_numpy(np.ascontiguousarray(a)) if isinstance(a, np.ndarray) else a
+            return t.contiguous().to(dev)
+
+        layer = qe.QELayer.from_float(desc, c(inp["W"]), c(inp["s"]), c(inp["A_s"]), c(inp["B_s"]), c(inp["A_r"]),
+                                      c(inp["B_r"]), c(inp["G"]), s_inv=c(inp["s_inv"]))
+        X = c(inp["X"])
+        Y = torch.empty((T, proj.d_out), dtype=torch.bfloat16, device=dev)
+        ws = layer.workspace(T)
+        layers.append(dict(proj=proj, desc=desc, layer=layer, X=X, Y=Y, ws=ws, x_host=inp["X"]))
+        del inp
+    torch.cuda.synchronize()
+    return layers
+
+
+def run_ours(args, workload):
+    import torch
+    import quantized_gemm_moe_b200 as qe
+    from quantized_gemm_moe_b200 import roofline
+
+    rank, local_rank, world = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    qe.load()
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    cfg_name, t_over, desc_txt = WORKLOADS[workload]
+    cfg = qi.CONFIGS[cfg_name]
+    T = t_over or cfg.T
+    layers = build_layers(cfg, T, rank, dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    wonly = cfg.a_bits == 16
+    stages = (qe.QE_STAGE_ROUTE, qe.QE_STAGE_QUANT, qe.QE_STAGE_ADAPTERS, qe.QE_STAGE_PRODUCT)
+
+    def step(record):
+        evs = []
+        for L in layers:
+            if record:
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+                e[0].record(stream)
+                for i, sm in enumerate(stages):
+                    qe.linear_forward_stages(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"], sm)
+                    e[i + 1].record(stream)
+                evs.append(e)
+            else:
+                qe.linear_forward(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"])
+        return evs
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step(False)
+    torch.cuda.synchronize()
+    assert qe.device_error() == 0, "a device wait ran out during warm-up"
+
+    all_evs = []
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            all_evs.append(step(True))
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    err = qe.device_error()
+    assert err == 0, f"device wait ran out (code {err:#x})"
+
+    n_proj = len(layers)
+    stage_ms = np.zeros((args.steps, n_proj, len(stages)))
+    for s_i, evs in enumerate(all_evs):
+        for p_i, e in enumerate(evs):
+            for k in range(len(stages)):
+                stage_ms[s_i, p_i, k] = e[k].elapsed_time(e[k + 1])
+    step_ms = stage_ms.sum(axis=(1, 2))
+    total_ms = float(step_ms.sum())
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    # algorithmic work per step
+    ints = sum(roofline.int_ops(T, L["proj"].d_in, L["proj"].d_out) for L in layers) if not wonly else 0
+    fl = sum(roofline.adapter_flops(T, L["proj"].d_in, L["proj"].d_out, cfg.rank_shared, cfg.n_routed,
+                                    cfg.rank_routed) for L in layers)
+    if wonly:
+        fl += sum(2 * T * L["proj"].d_in * L["proj"].d_out for L in layers)
+    xb = 2 if cfg.x_dtype == "bf16" else 4
+    nbytes = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
+                                      cfg.n_routed, cfg.rank_routed, xb, 2) for L in layers)
+    peaks = load_peaks()
+    prod_ms = stage_ms[:, :, 3].sum(axis=1).mean()  # the product kernels of one step
+    int8_peak = 2.0 * peaks["bf16_tflops"]           # int8 dense = 2x bf16 dense (nominal ratio)
+    decode = T <= 16
+    kernel_file = "quantized_gemm_moe_b200/csrc/k_misc.cu" if wonly else "quantized_gemm_moe_b200/csrc/k_gemm.cu"
+    prod_bytes = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
+                                          cfg.n_routed, cfg.rank_routed, 1 if not wonly else 2, 2) for L in layers)
+    traffic = read_traffic(kernel_file, ("wonly_" if wonly else "qgemm_") + workload)
+    if decode:
+        ach = prod_bytes / (prod_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic,
+                "kernel": "wonly" if wonly else "qgemm", "peak_source": peaks["source"] + " hbm copy"}
+    else:
+        ach = ints / (prod_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": int8_peak, "unit": "TOP/s",
+                "frac": ach / int8_peak, "traffic": traffic, "kernel": "qgemm",
+                "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TF/s x 2 (int8:bf16 nominal ratio)"}
+
+    per_proj = []
+    for p_i, L in enumerate(layers):
+        ms = stage_ms[:, p_i, :].mean(axis=0)
+        K, N = L["proj"].d_in, L["proj"].d_out
+        tot = ms.sum()
+        per_proj.append({
+            "proj": L["proj"].name, "K": K, "N": N, "ms": float(tot),
+            "stage_ms": {"route": float(ms[0]), "quant": float(ms[1]), "adapters": float(ms[2]), "product": float(ms[3])},
+            "product_tops": (roofline.int_ops(T, K, N) / (ms[3] / 1e3) / 1e12) if not wonly else None,
+            "product_gbs": roofline.layer_bytes(T, K, N, cfg.group, cfg.w_bits, cfg.rank_shared, cfg.n_routed,
+                                                cfg.rank_routed, 1 if not wonly else 2, 2) / (ms[3] / 1e3) / 1e9,
+            "layer_tokens_per_s": T / (tot / 1e3),
+        })
+
+    # end to end through the public call with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        xh = [torch.from_numpy(np.ascontiguousarray(L["x_host"])) if isinstance(L["x_host"], np.ndarray)
+              else L["x_host"] for L in layers]
+        xh = [x.contiguous().pin_memory() for x in xh]
+        yh = [torch.empty(L["Y"].shape, dtype=L["Y"].dtype).pin_memory() for L in layers]
+        h2d = sum(x.numel() * x.element_size() for x in xh)
+        d2h = sum(y.numel() * y.element_size() for y in yh)
+        e_ms = 0.0
+        for it in range(args.warmup + args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for L, x, y in zip(layers, xh, yh):
+                L["X"].copy_(x, non_blocking=True)
+                qe.linear_forward(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"])
+                y.copy_(L["Y"], non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= args.warmup:
+                e_ms += e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * T * args.steps / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+        sample = max(1, min(args.cpu_sample_tokens, T))
+        secs = oracle_sample_run(cfg, T, sample)
+        cpu = {"value": sample / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{sample} tokens through every projection of the layer set (tokens are independent)"}
+
+    launches = sum(qe.linear_kernel_launches(L["desc"], T, qe.QE_BF16 if cfg.x_dtype == "bf16" else qe.QE_F32)
+                   for L in layers) * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wonly else "int8", "data": "synthetic",
+        "config": {"workload": workload, "description": desc_txt, "T_per_gpu": T,
+                   "projections": [[L["proj"].name, L["proj"].d_in, L["proj"].d_out] for L in layers],
+                   "l2": "flushed between steps (256 MB write outside the per-step events)",
+                   "parallelism": f"replicas x{world}"},
+        "effective_tops": (ints + fl) / (ms_per_step / 1e3) / 1e12 * world,
+        "hbm_gbs_algorithmic": nbytes / (ms_per_step / 1e3) / 1e9,
+        "roofline": roof,
+        "per_projection": per_proj,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "gpu_launches": launches,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for L in layers:
+        L.clear()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args, args.workload)
+    return run_ours(args, args.workload)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,268 @@
+/*
+ * qe.h -- C ABI of the B200 (sm_100a) Quant Experts (QE) linear-layer library.
+ *
+ * The layer (Quant Experts: Token-aware Adaptive Error Reconstruction with
+ * Mixture of Experts for Large Vision-Language Models Quantization; method
+ * text on the MCISLAB DeepRead summary page, section "Method"; cost model in
+ * Table 7 of the thelatestinai listing):
+ *
+ *   Y = dequant(Q_A(X/s)) . dequant(Q_W(W.s))^T  +  X.A_s.B_s  +  X.A_r[e(t)].B_r[e(t)]
+ *
+ * - W.s / X/s: channel-wise scaling (Method, "Shared Expert"), with s_inv = 1/s
+ *   stored per input channel.
+ * - Q_W: symmetric group RTN, W4 or W3, one fp32 scale per (output row, group).
+ * - Q_A: symmetric per-token RTN, A8 or A6 (a_bits 8/6). a_bits 16 means
+ *   weight-only (W3A16 / W4A16): bf16(x/s) against the dequantized weight.
+ * - A_s.B_s: the shared low-rank expert, applied to every token (Method,
+ *   "Shared Expert").
+ * - A_r[e].B_r[e]: one routed low-rank expert per token (Method, "Routed
+ *   Experts"). e(t) = argmin_e (X.G)[t,e], a router that predicts each
+ *   expert's residual error and takes the smallest. Table 7 prices it at
+ *   s*d*N_r, so it is a single d_in x N_r linear map.
+ *
+ * Conventions for every entry point
+ * - Pointers marked (device) are CUDA device pointers. The caller allocates
+ *   and owns all of them. The library allocates no device memory and keeps
+ *   no device state except one error word (qe_device_error). It never frees
+ *   anything it did not allocate.
+ * - Matrices are row-major. W is [d_out, d_in] (the nn.Linear convention),
+ *   X is [T, d_in] and Y is [T, d_out].
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream). Arguments are validated synchronously before anything
+ *   is launched. On a non-OK return nothing was launched.
+ * - Every device pointer must be 16-byte aligned. d_in must be a multiple of
+ *   the group (64 or 128). Row pitches equal the row width (dense).
+ * - Kernels never trap. A device-side wait that runs out (2 s) records a code
+ *   that qe_device_error() returns. The caller should then treat that call's
+ *   outputs as invalid.
+ * - No exception crosses this ABI.
+ */
+#ifndef QE_H_
+#define QE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QE_API __attribute__((visibility("default")))
+#else
+#define QE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QE_OK = 0,
+  QE_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, inconsistent shape */
+  QE_ERR_UNSUPPORTED = 2,  /* a combination this build does not implement (bits, group, ranks) */
+  QE_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+  QE_ERR_WORKSPACE = 4,    /* workspace pointer null or smaller than qe_linear_workspace_bytes */
+  QE_ERR_CUDA = 5,         /* a CUDA launch or driver call failed (see qe_last_cuda_error) */
+  QE_ERR_TIMEOUT = 6       /* a device wait ran out (returned by qe_device_error) */
+} qe_status;
+
+typedef enum { QE_F32 = 0, QE_BF16 = 1 } qe_dtype;
+
+/* Shape and precision of one QE linear layer. */
+typedef struct {
+  int32_t d_in;         /* K, multiple of group, >= 128                           */
+  int32_t d_out;        /* N, any positive value                                  */
+  int32_t group;        /* weight quantization group along K: 64 or 128           */
+  int32_t w_bits;       /* 4 (W4) or 3 (W3)                                        */
+  int32_t a_bits;       /* 8 (A8), 6 (A6) or 16 (weight-only, bf16 activations)   */
+  int32_t rank_shared;  /* r_s >= 0                                                */
+  int32_t n_routed;     /* N_r in [1, 16]                                          */
+  int32_t rank_routed;  /* r_r >= 0; r_s + N_r*r_r <= 512                          */
+} qe_layer_desc;
+
+/*
+ * Quantized weight storage (library-defined layouts; produced by
+ * qe_quantize_weights, read by qe_linear_forward; safe to save and reload as
+ * bytes on the same library version):
+ *
+ * w_packed (device, qe_packed_weight_bytes bytes): codes in blocks of
+ *   128 output rows x 128 input channels. Block (n, b) with n = o/128 and
+ *   b = k/128 starts at byte (n*ceil(d_in/128) + b) * block_bytes. Rows past
+ *   d_out and channels past d_in hold zero codes.
+ *   W4: block_bytes = 8192. Row r of a block is 64 bytes at r*64: four
+ *     16-byte pieces i = 0..3. In piece i, byte 4w+b of 32-bit word w holds
+ *     code (32i + 4w + b) in its low nibble and code (32i + 16 + 4w + b) in
+ *     its high nibble. Codes are 4-bit two's complement in [-7, 7].
+ *   W3: block_bytes = 6144. Row r of a block is 48 bytes at r*48. Codes are
+ *     stored offset-binary as u = q + 4 in [1, 7]. Bytes 0..31 are eight
+ *     32-bit words of 2-bit fields: word m holds the low two bits of u for
+ *     code 16m + 2p at bits [2p, 2p+2), and for code 16m + 2p + 1 at bits
+ *     [16+2p, 18+2p), p = 0..7. Bytes 32..47 are four 32-bit words of
+ *     high bits: word h holds bit 2 of u for code 32h + 2p at bit p, and for
+ *     code 32h + 2p + 1 at bit 16 + p, p = 0..15.
+ * w_scale (device, fp32 [d_in/group][d_out], group-major): the weight scale of
+ *   (output row o, group j) is w_scale[j*d_out + o].
+ * s_inv (device, fp32 [d_in]): 1/s, the reciprocal channel smoothing factor.
+ * adapters (device, qe_adapter_packed_bytes bytes): produced by
+ *   qe_pack_adapters from the natural-layout adapters and router.
+ */
+typedef struct {
+  const void* w_packed;
+  const float* w_scale;
+  const float* s_inv;
+  const void* adapters;
+} qe_layer_weights;
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Bytes of w_packed for this layer (0 on an invalid desc). */
+QE_API size_t qe_packed_weight_bytes(const qe_layer_desc* desc);
+
+/* Bytes of the packed adapter/router buffer for this layer (0 on an invalid desc). */
+QE_API size_t qe_adapter_packed_bytes(const qe_layer_desc* desc);
+
+/* Bytes of the caller-provided scratch that qe_linear_forward needs for T tokens. */
+QE_API size_t qe_linear_workspace_bytes(const qe_layer_desc* desc, int32_t T);
+
+/* ---------------------------------------------------------------- weight preparation */
+
+/*
+ * Channel-scaled symmetric group quantization of W (Method, "Shared Expert":
+ * weights are multiplied by s; bit widths W4/W3 from Tables 1-3), plus the
+ * importance statistic's weight term w = Meanrow(|W_f|) (Method: per input
+ * channel, the mean over output rows of |W|).
+ *   W        (device) [d_out, d_in], fp32 or bf16 (w_dtype)
+ *   s        (device) fp32 [d_in] smoothing factor (the weights are multiplied by it)
+ *   w_packed (device) out, qe_packed_weight_bytes(desc) bytes
+ *   w_scale  (device) out, fp32 [d_in/group][d_out]
+ *   w_mean   (device) out, fp32 [d_in], may be NULL
+ *   w_colmax (device) out, fp32 [d_in] = max_o |W[o][k]|, may be NULL
+ * For each (o, group j): scale = fl32(max_k |fl32(W[o][k]*s[k])| / qmax) and
+ * code = clamp(rint(fl32(fl32(W*s)/scale)), -qmax, qmax), with ties to
+ * even. A zero scale gives zero codes. qmax = 7 (W4) or 3 (W3). w_mean
+ * is summed in fp64 and rounded once.
+ */
+QE_API qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, qe_dtype w_dtype, const float* s,
+                              void* w_packed, float* w_scale, float* w_mean, float* w_colmax, void* stream);
+
+/*
+ * Packs the shared expert, the routed experts and the router into the
+ * library's adapter layout.
+ *   A_s (device) bf16 [d_in][r_s]      B_s (device) bf16 [r_s][d_out]
+ *   A_r (device) bf16 [N_r][d_in][r_r] B_r (device) bf16 [N_r][r_r][d_out]
+ *   G   (device) bf16 [d_in][N_r]      (router: logits = X.G)
+ *   out (device) qe_adapter_packed_bytes(desc) bytes
+ * A_s/B_s may be NULL when r_s = 0, and A_r/B_r may be NULL when r_r = 0.
+ */
+QE_API qe_status qe_pack_adapters(const qe_layer_desc* desc, const void* A_s, const void* B_s, const void* A_r,
+                           const void* B_r, const void* G, void* out, void* stream);
+
+/* ---------------------------------------------------------------- the hot path */
+
+/*
+ * Token-aware importance statistic (Method: Top-k(|x_t| * w) per token with
+ * w = Meanrow(|W_f|); the channel frequency is counted over tokens).
+ *   X      (device) [T, d_in], fp32 or bf16
+ *   w_mean (device) fp32 [d_in]
+ *   idx    (device) out int32 [T, k]. The k channels with the largest
+ *          score fl32(|x|*w_mean), ordered by (score desc, channel asc).
+ *          Equal scores go to the lower channel.
+ *   hist   (device) int32 [d_in]: hist[c] += number of tokens whose Top-k
+ *          holds c. It is zeroed first unless accumulate_hist != 0. May be NULL.
+ * 1 <= k <= min(d_in, 128). T = 0 is a no-op.
+ */
+QE_API qe_status qe_topk_importance(const void* X, qe_dtype x_dtype, const float* w_mean, int32_t T, int32_t d_in,
+                             int32_t k, int32_t* idx, int32_t* hist, int32_t accumulate_hist, void* stream);
+
+/*
+ * Router and token buckets (Method, "Routed Experts": the router picks the
+ * expert with the smallest predicted residual error; one routed expert
+ * per token).
+ *   X       (device) [T, d_in], fp32 or bf16
+ *   G       (device) bf16 [d_in][n_routed]
+ *   expert  (device) out int32 [T]: argmin_e fl32-accumulated (X.G)[t,e],
+ *           ties -> lowest e
+ *   perm    (device) out int32 [T]: token at sorted position p (stable by t)
+ *   offsets (device) out int32 [n_routed+1]: expert e owns positions
+ *           [offsets[e], offsets[e+1])
+ *   logits  (device) out fp32 [T, n_routed], may be NULL
+ * T <= 1<<20.
+ */
+QE_API qe_status qe_route(const void* X, qe_dtype x_dtype, const void* G, int32_t T, int32_t d_in, int32_t n_routed,
+                   int32_t* expert, int32_t* perm, int32_t* offsets, float* logits, void* stream);
+
+/*
+ * The QE linear layer forward (the formula at the top of this file).
+ *   X         (device) [T, d_in], fp32 or bf16 (x_dtype)
+ *   Y         (device) out [T, d_out], fp32 or bf16 (y_dtype)
+ *   workspace (device) scratch of at least qe_linear_workspace_bytes(desc, T)
+ *             bytes. Contents on entry are ignored. Calls that share a
+ *             workspace must not overlap on the GPU.
+ * Steps (all on the GPU): router + per-token absmax -> stable bucket sort ->
+ * per-token quantization in bucket order -> adapter down-projection
+ * (tensor cores) -> int8 tcgen05 GEMM with per-group scale promotion and the
+ * adapter up-projection in its epilogue -> scatter to token order. With
+ * a_bits = 16 the main product is the weight-only bf16 path.
+ * T = 0 is a no-op.
+ */
+QE_API qe_status qe_linear_forward(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
+                            qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * The same forward split into its steps, for per-step timing: `stages` is a
+ * bitmask of QE_STAGE_* run in the documented order. Running every stage in
+ * separate calls on one stream, with the same workspace, computes exactly
+ * what qe_linear_forward computes. A stage reads what earlier stages left in
+ * the workspace. Unknown bits -> QE_ERR_INVALID_ARG.
+ */
+#define QE_STAGE_ROUTE 1    /* router + per-token absmax, stable bucket sort          */
+#define QE_STAGE_QUANT 2    /* per-token quantization in bucket order                 */
+#define QE_STAGE_ADAPTERS 4 /* adapter down-projection (tensor cores), expert masking  */
+#define QE_STAGE_PRODUCT 8  /* main product with the adapter epilogue, scatter to Y   */
+#define QE_STAGE_ALL 15
+QE_API qe_status qe_linear_forward_stages(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
+                                          qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,
+                                          size_t workspace_bytes, int32_t stages, void* stream);
+
+/* Number of kernels one qe_linear_forward launches for this layer and T (-1 on an invalid desc). */
+QE_API int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype);
+
+/* ---------------------------------------------------------------- status */
+
+QE_API const char* qe_status_string(qe_status s);
+/* The last CUDA error string seen by a call that returned QE_ERR_CUDA (thread-local). */
+QE_API const char* qe_last_cuda_error(void);
+/*
+ * Synchronizes `stream`, then reads the device error word. *code receives 0,
+ * or the code of the first device wait that ran out. clear != 0 resets it.
+ * Returns QE_ERR_TIMEOUT when a code was set, QE_OK otherwise.
+ */
+QE_API qe_status qe_device_error(void* stream, int32_t* code, int32_t clear);
+
+/* ---------------------------------------------------------------- diagnostics (tests) */
+
+/* Unpacks w_packed to int8 codes [d_out, d_in] (device), one code per byte. */
+QE_API qe_status qe_unpack_weights(const qe_layer_desc* desc, const void* w_packed, int8_t* codes, void* stream);
+
+/*
+ * Per-token quantization alone, in token order: codes (device) int8 [T, d_in],
+ * sa (device) fp32 [T]. a_bits 6 or 8.
+ */
+QE_API qe_status qe_act_quant(const void* X, qe_dtype x_dtype, const float* s_inv, int32_t T, int32_t d_in,
+                       int32_t a_bits, int8_t* codes, float* sa, void* stream);
+
+/*
+ * qe_linear_forward with its intermediates exposed (a_bits 6/8 only):
+ *   acc     (device) out int32 [T, d_out, d_in/group]: the exact int32 group
+ *           accumulators sum_{k in group} xq[t][k]*wq[o][k], taken from TMEM.
+ *           For small layers only (T*d_out*d_in/group*4 bytes).
+ *   expert/perm (device) out int32 [T] (as qe_route); sa (device) out fp32 [T]
+ *   in token order. Any of acc/expert/perm/sa may be NULL.
+ */
+QE_API qe_status qe_linear_forward_debug(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
+                                  qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,
+                                  size_t workspace_bytes, int32_t* acc, int32_t* expert, int32_t* perm, float* sa,
+                                  void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QE_H_ */

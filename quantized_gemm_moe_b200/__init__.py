@@ -1,0 +1,275 @@
+"""Python binding of the sm_100a QE linear-layer library (libqe.so, C ABI in include/qe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. PyTorch supplies device memory and the current stream. Importing
+works without a GPU (the tests check the exported symbols on CPU). Every
+compute call raises QEError when the library is missing or a call fails.
+There is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libqe.so")
+
+QE_OK, QE_ERR_INVALID_ARG, QE_ERR_UNSUPPORTED, QE_ERR_ALIGNMENT, QE_ERR_WORKSPACE, QE_ERR_CUDA, QE_ERR_TIMEOUT = range(7)
+QE_F32, QE_BF16 = 0, 1
+
+# Every symbol include/qe.h declares (the tests check that the library exports them).
+EXPORTS = (
+    "qe_packed_weight_bytes", "qe_adapter_packed_bytes", "qe_linear_workspace_bytes", "qe_quantize_weights",
+    "qe_pack_adapters", "qe_topk_importance", "qe_route", "qe_linear_forward", "qe_status_string",
+    "qe_last_cuda_error", "qe_device_error", "qe_unpack_weights", "qe_act_quant", "qe_linear_forward_debug",
+    "qe_linear_forward_stages", "qe_linear_kernel_launches",
+)
+QE_STAGE_ROUTE, QE_STAGE_QUANT, QE_STAGE_ADAPTERS, QE_STAGE_PRODUCT, QE_STAGE_ALL = 1, 2, 4, 8, 15
+
+
+class QEError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str = ""):
+        self.status = status
+        msg = f"{what} failed: status {status}"
+        if _LIB is not None:
+            msg += f" ({_LIB.qe_status_string(status).decode()})"
+        if detail:
+            msg += f": {detail}"
+        super().__init__(msg)
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("w_bits", ctypes.c_int32), ("a_bits", ctypes.c_int32), ("rank_shared", ctypes.c_int32),
+                ("n_routed", ctypes.c_int32), ("rank_routed", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "LayerDesc(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("w_packed", ctypes.c_void_p), ("w_scale", ctypes.c_void_p), ("s_inv", ctypes.c_void_p),
+                ("adapters", ctypes.c_void_p)]
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def load() -> ctypes.CDLL:
+    """Loads libqe.so (built by quantized_gemm_moe_b200.build). Raises when it is missing."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise QEError(-1, "load", f"{LIB_PATH} is missing; build it with `python -m quantized_gemm_moe_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, S = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    D = ctypes.POINTER(LayerDesc)
+    sigs = {
+        "qe_packed_weight_bytes": ([D], S),
+        "qe_adapter_packed_bytes": ([D], S),
+        "qe_linear_workspace_bytes": ([D, I], S),
+        "qe_quantize_weights": ([D, P, I, P, P, P, P, P, P], I),
+        "qe_pack_adapters": ([D, P, P, P, P, P, P, P], I),
+        "qe_topk_importance": ([P, I, P, I, I, I, P, P, I, P], I),
+        "qe_route": ([P, I, P, I, I, I, P, P, P, P, P], I),
+        "qe_linear_forward": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P, S, P], I),
+        "qe_linear_forward_debug": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P, S, P, P, P, P, P], I),
+        "qe_linear_forward_stages": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P, S, I, P], I),
+        "qe_linear_kernel_launches": ([D, I, I], I),
+        "qe_status_string": ([I], ctypes.c_char_p),
+        "qe_last_cuda_error": ([], ctypes.c_char_p),
+        "qe_device_error": ([P, ctypes.POINTER(I), I], I),
+        "qe_unpack_weights": ([D, P, P, P], I),
+        "qe_act_quant": ([P, I, P, I, I, I, P, P, P], I),
+    }
+    for name, (args, res) in sigs.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _LIB = L
+    return L
+
+
+# ---------------------------------------------------------------- marshalling helpers
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _dtype(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return QE_F32
+    if t.dtype == torch.bfloat16:
+        return QE_BF16
+    raise QEError(QE_ERR_INVALID_ARG, "dtype", f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(rc: int, what: str):
+    if rc != QE_OK:
+        detail = load().qe_last_cuda_error().decode() if rc == QE_ERR_CUDA else ""
+        raise QEError(rc, what, detail)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise QEError(QE_ERR_INVALID_ARG, "device", "tensors passed to the QE library must be CUDA tensors")
+        if t is not None and not t.is_contiguous():
+            raise QEError(QE_ERR_INVALID_ARG, "layout", "tensors passed to the QE library must be contiguous")
+
+
+def make_desc(d_in, d_out, group=128, w_bits=4, a_bits=8, rank_shared=32, n_routed=8, rank_routed=4) -> LayerDesc:
+    return LayerDesc(d_in, d_out, group, w_bits, a_bits, rank_shared, n_routed, rank_routed)
+
+
+# ---------------------------------------------------------------- the C ABI, one wrapper per entry point
+
+def packed_weight_bytes(desc: LayerDesc) -> int:
+    return int(load().qe_packed_weight_bytes(ctypes.byref(desc)))
+
+
+def adapter_packed_bytes(desc: LayerDesc) -> int:
+    return int(load().qe_adapter_packed_bytes(ctypes.byref(desc)))
+
+
+def linear_workspace_bytes(desc: LayerDesc, T: int) -> int:
+    return int(load().qe_linear_workspace_bytes(ctypes.byref(desc), T))
+
+
+def quantize_weights(desc, W, s, w_packed, w_scale, w_mean=None, w_colmax=None, stream=None):
+    _need_cuda(W, s, w_packed, w_scale, w_mean, w_colmax)
+    _check(load().qe_quantize_weights(ctypes.byref(desc), _ptr(W), _dtype(W), _ptr(s), _ptr(w_packed),
+                                      _ptr(w_scale), _ptr(w_mean), _ptr(w_colmax), _stream(stream)),
+           "qe_quantize_weights")
+
+
+def pack_adapters(desc, A_s, B_s, A_r, B_r, G, out, stream=None):
+    _need_cuda(A_s, B_s, A_r, B_r, G, out)
+    _check(load().qe_pack_adapters(ctypes.byref(desc), _ptr(A_s), _ptr(B_s), _ptr(A_r), _ptr(B_r), _ptr(G),
+                                   _ptr(out), _stream(stream)), "qe_pack_adapters")
+
+
+def topk_importance(X, w_mean, k, idx, hist=None, accumulate=False, stream=None):
+    _need_cuda(X, w_mean, idx, hist)
+    T, K = X.shape
+    _check(load().qe_topk_importance(_ptr(X), _dtype(X), _ptr(w_mean), T, K, k, _ptr(idx), _ptr(hist),
+                                     1 if accumulate else 0, _stream(stream)), "qe_topk_importance")
+
+
+def route(X, G, expert, perm, offsets, logits=None, stream=None):
+    _need_cuda(X, G, expert, perm, offsets, logits)
+    T, K = X.shape
+    _check(load().qe_route(_ptr(X), _dtype(X), _ptr(G), T, K, G.shape[1], _ptr(expert), _ptr(perm), _ptr(offsets),
+                           _ptr(logits), _stream(stream)), "qe_route")
+
+
+def linear_forward(desc, weights: LayerWeights, X, Y, workspace, stream=None):
+    _need_cuda(X, Y, workspace)
+    _check(load().qe_linear_forward(ctypes.byref(desc), ctypes.byref(weights), _ptr(X), _dtype(X), X.shape[0],
+                                    _ptr(Y), _dtype(Y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)), "qe_linear_forward")
+
+
+def linear_kernel_launches(desc: LayerDesc, T: int, x_dtype: int = QE_BF16) -> int:
+    return int(load().qe_linear_kernel_launches(ctypes.byref(desc), T, x_dtype))
+
+
+def linear_forward_stages(desc, weights: LayerWeights, X, Y, workspace, stages: int, stream=None):
+    _need_cuda(X, Y, workspace)
+    _check(load().qe_linear_forward_stages(ctypes.byref(desc), ctypes.byref(weights), _ptr(X), _dtype(X), X.shape[0],
+                                           _ptr(Y), _dtype(Y), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), stages, _stream(stream)),
+           "qe_linear_forward_stages")
+
+
+def linear_forward_debug(desc, weights, X, Y, workspace, acc=None, expert=None, perm=None, sa=None, stream=None):
+    _need_cuda(X, Y, workspace, acc, expert, perm, sa)
+    _check(load().qe_linear_forward_debug(ctypes.byref(desc), ctypes.byref(weights), _ptr(X), _dtype(X), X.shape[0],
+                                          _ptr(Y), _dtype(Y), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _ptr(acc), _ptr(expert),
+                                          _ptr(perm), _ptr(sa), _stream(stream)), "qe_linear_forward_debug")
+
+
+def unpack_weights(desc, w_packed, codes, stream=None):
+    _need_cuda(w_packed, codes)
+    _check(load().qe_unpack_weights(ctypes.byref(desc), _ptr(w_packed), _ptr(codes), _stream(stream)),
+           "qe_unpack_weights")
+
+
+def act_quant(X, s_inv, a_bits, codes, sa, stream=None):
+    _need_cuda(X, s_inv, codes, sa)
+    T, K = X.shape
+    _check(load().qe_act_quant(_ptr(X), _dtype(X), _ptr(s_inv), T, K, a_bits, _ptr(codes), _ptr(sa),
+                               _stream(stream)), "qe_act_quant")
+
+
+def device_error(clear: bool = True, stream=None) -> int:
+    """Synchronizes the stream and returns the device error word (0 = no device wait ran out)."""
+    code = ctypes.c_int32(0)
+    rc = load().qe_device_error(_stream(stream), ctypes.byref(code), 1 if clear else 0)
+    if rc not in (QE_OK, QE_ERR_TIMEOUT):
+        _check(rc, "qe_device_error")
+    return int(code.value)
+
+
+# ---------------------------------------------------------------- a layer object (device buffers via torch)
+
+class QELayer:
+    """One QE linear layer resident on the GPU: quantized weights, scales and packed adapters.
+
+    Built from full-precision weights with `from_float`. `forward` runs
+    qe_linear_forward on the current stream.
+    """
+
+    def __init__(self, desc: LayerDesc, w_packed, w_scale, s_inv, adapters, w_mean=None, w_colmax=None):
+        self.desc = desc
+        self.w_packed, self.w_scale, self.s_inv, self.adapters = w_packed, w_scale, s_inv, adapters
+        self.w_mean, self.w_colmax = w_mean, w_colmax
+        self.weights = LayerWeights(w_packed.data_ptr(), w_scale.data_ptr(), s_inv.data_ptr(), adapters.data_ptr())
+        self._ws = None
+
+    @classmethod
+    def from_float(cls, desc: LayerDesc, W, s, A_s, B_s, A_r, B_r, G, s_inv=None, stream=None) -> "QELayer":
+        """W [d_out, d_in] (fp32/bf16), s [d_in] fp32, adapters/G bf16 in their natural layouts (CUDA tensors).
+
+        s_inv (fp32 [d_in]) is the stored reciprocal smoothing factor the activations are
+        multiplied by. When omitted, it is fl32(1/s).
+        """
+        import torch
+        dev = W.device
+        K, N = desc.d_in, desc.d_out
+        w_packed = torch.empty(packed_weight_bytes(desc), dtype=torch.uint8, device=dev)
+        w_scale = torch.empty((K // desc.group, N), dtype=torch.float32, device=dev)
+        w_mean = torch.empty(K, dtype=torch.float32, device=dev)
+        w_colmax = torch.empty(K, dtype=torch.float32, device=dev)
+        quantize_weights(desc, W, s, w_packed, w_scale, w_mean, w_colmax, stream)
+        adapters = torch.empty(adapter_packed_bytes(desc), dtype=torch.uint8, device=dev)
+        pack_adapters(desc, A_s, B_s, A_r, B_r, G, adapters, stream)
+        if s_inv is None:
+            s_inv = (torch.ones_like(s) / s).contiguous()
+        return cls(desc, w_packed, w_scale, s_inv.contiguous(), adapters, w_mean, w_colmax)
+
+    def workspace(self, T: int):
+        import torch
+        need = linear_workspace_bytes(self.desc, T)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.w_packed.device)
+        return self._ws
+
+    def forward(self, X, out_dtype=None, Y=None, stream=None):
+        import torch
+        T = X.shape[0]
+        if Y is None:
+            Y = torch.empty((T, self.desc.d_out), dtype=out_dtype or X.dtype, device=X.device)
+        linear_forward(self.desc, self.weights, X, Y, self.workspace(T), stream)
+        return Y

@@ -1,0 +1,560 @@
+// Memory-bound kernels of the QE linear layer: router + per-token absmax,
+// stable token->expert bucket sort, per-token quantization, weight
+// quantization / packing, adapter packing, adapter finalize, split-K reduce.
+#include <cuda_bf16.h>
+
+#include "qe_internal.h"
+
+namespace qe {
+
+// The library's only device state: the error word that bounded waits write.
+__device__ int g_device_error = 0;
+
+int* device_error_ptr() {
+  static int* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cached[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    cached[dev] = static_cast<int*>(p);
+  }
+  return cached[dev];
+}
+
+cudaError_t read_device_error(int* value, bool clear, cudaStream_t st) {
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (clear) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  }
+  return e;
+}
+
+namespace {
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
+  __nv_bfloat16 h = __float2bfloat16_rn(v);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// Loads 8 consecutive elements x[row][k0..k0+8) as fp32 (k0 multiple of 8, row pitch K).
+template <bool BF16>
+__device__ __forceinline__ void load8(const void* X, size_t row, int K, int k0, float (&v)[8]) {
+  if constexpr (BF16) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(X) + row * K + k0));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+      v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(X) + row * K + k0);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ void load8f(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// One symmetric RTN code: clamp(rint(fl32(v / scale)), -qmax, qmax); zero scale -> 0.
+__device__ __forceinline__ int rtn_code(float v, float scale, int qmax) {
+  if (scale == 0.0f) return 0;
+  float r = rintf(__fdiv_rn(v, scale));
+  r = fminf(fmaxf(r, -static_cast<float>(qmax)), static_cast<float>(qmax));
+  return static_cast<int>(r);
+}
+
+// ------------------------------------------------------------------ router + absmax
+// One CTA per token. logits[e] = sum_k x[k]*G[k][e] in fp32; e* = argmin (lowest e on ties);
+// sa = fl32(max_k |fl32(x[k]*s_inv[k])| / qmax).
+template <bool BF16, int NR>
+__global__ void __launch_bounds__(256) k_route_stats(const void* __restrict__ X, const float* __restrict__ s_inv,
+                                                     const uint16_t* __restrict__ G, int T, int K, int n_r,
+                                                     int qmax, int32_t* __restrict__ expert,
+                                                     float* __restrict__ sa, float* __restrict__ logits) {
+  const int t = blockIdx.x;
+  float acc[NR];
+#pragma unroll
+  for (int e = 0; e < NR; ++e) acc[e] = 0.0f;
+  float amax = 0.0f;
+  const bool want_sa = sa != nullptr;
+  for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
+    float xv[8];
+    load8<BF16>(X, t, K, k0, xv);
+    if (want_sa) {
+      float si[8];
+      load8f(s_inv + k0, si);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(__fmul_rn(xv[i], si[i])));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint16_t* g = G + static_cast<size_t>(k0 + i) * n_r;
+      if constexpr (NR == 8) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(g));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[2 * j] = fmaf(xv[i], bf16_bits_to_f32(w[j] & 0xFFFFu), acc[2 * j]);
+          acc[2 * j + 1] = fmaf(xv[i], bf16_bits_to_f32(w[j] >> 16), acc[2 * j + 1]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < NR; ++e)
+          if (e < n_r) acc[e] = fmaf(xv[i], bf16_bits_to_f32(__ldg(g + e)), acc[e]);
+      }
+    }
+  }
+  // block reduction: warp shuffles, then one row per warp in shared memory
+  __shared__ float red[8][NR + 1];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+#pragma unroll
+    for (int e = 0; e < NR; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int e = 0; e < NR; ++e) red[warp][e] = acc[e];
+    red[warp][NR] = amax;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int nw = blockDim.x >> 5;
+    float best = 0.0f;
+    int beste = 0;
+    float am = 0.0f;
+    for (int w = 0; w < nw; ++w) am = fmaxf(am, red[w][NR]);
+    for (int e = 0; e < n_r; ++e) {
+      float L = 0.0f;
+      for (int w = 0; w < nw; ++w) L += red[w][e];
+      if (logits) logits[static_cast<size_t>(t) * n_r + e] = L;
+      if (e == 0 || L < best) {
+        best = L;
+        beste = e;
+      }
+    }
+    if (expert) expert[t] = beste;
+    if (sa) sa[t] = __fdiv_rn(am, static_cast<float>(qmax));
+  }
+}
+
+// ------------------------------------------------------------------ stable bucket sort
+// Single CTA of 1024 threads. Counts per expert, then assigns positions chunk by
+// chunk: warp ballots give each token its rank inside its warp, a scan over the
+// 32 warps gives the warp offsets, and chunks are taken in token order, so
+// the sort is stable.
+__global__ void __launch_bounds__(1024) k_bucket(const int32_t* __restrict__ expert, int T, int n_r,
+                                                 int32_t* __restrict__ perm, int32_t* __restrict__ pos,
+                                                 int32_t* __restrict__ offsets) {
+  __shared__ int cnt[kMaxRouted], base[kMaxRouted];
+  __shared__ int wcnt[32][kMaxRouted], wbase[32][kMaxRouted];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < kMaxRouted) cnt[tid] = 0;
+  __syncthreads();
+  for (int t = tid; t < T; t += blockDim.x) atomicAdd(&cnt[expert[t]], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < n_r; ++e) {
+      base[e] = run;
+      offsets[e] = run;
+      run += cnt[e];
+    }
+    offsets[n_r] = run;
+  }
+  __syncthreads();
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int c0 = 0; c0 < T; c0 += blockDim.x) {
+    const int t = c0 + tid;
+    const int e = (t < T) ? expert[t] : -1;
+    int rank = 0;
+    for (int ee = 0; ee < n_r; ++ee) {
+      const uint32_t m = __ballot_sync(0xffffffffu, e == ee);
+      if (lane == 0) wcnt[warp][ee] = __popc(m);
+      if (e == ee) rank = __popc(m & lt_mask);
+    }
+    __syncthreads();
+    if (tid < n_r) {
+      int run = base[tid];
+      for (int w = 0; w < 32; ++w) {
+        wbase[w][tid] = run;
+        run += wcnt[w][tid];
+      }
+      base[tid] = run;
+    }
+    __syncthreads();
+    if (t < T) {
+      const int p = wbase[warp][e] + rank;
+      perm[p] = t;
+      if (pos) pos[t] = p;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ per-token quantization
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_act_quant(const void* __restrict__ X, const float* __restrict__ s_inv,
+                                                   int T, int K, int qmax, const float* __restrict__ sa_tok,
+                                                   const int32_t* __restrict__ pos, int8_t* __restrict__ codes,
+                                                   float* __restrict__ sa_sorted, uint16_t* __restrict__ act16,
+                                                   uint16_t* __restrict__ xb16) {
+  const int t = blockIdx.x;
+  const size_t p = pos ? static_cast<size_t>(pos[t]) : static_cast<size_t>(t);
+  const float sa = sa_tok ? sa_tok[t] : 0.0f;
+  for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
+    float xv[8], si[8];
+    load8<BF16>(X, t, K, k0, xv);
+    load8f(s_inv + k0, si);
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(xv[i], si[i]);
+    if (codes) {
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        w0 |= (static_cast<uint32_t>(rtn_code(v[i], sa, qmax)) & 0xFFu) << (8 * i);
+        w1 |= (static_cast<uint32_t>(rtn_code(v[4 + i], sa, qmax)) & 0xFFu) << (8 * i);
+      }
+      *reinterpret_cast<uint2*>(codes + p * K + k0) = make_uint2(w0, w1);
+    }
+    if (act16) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w[i] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i])) |
+               (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i + 1])) << 16);
+      *reinterpret_cast<uint4*>(act16 + p * K + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (xb16) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w[i] = static_cast<uint32_t>(f32_to_bf16_bits(xv[2 * i])) |
+               (static_cast<uint32_t>(f32_to_bf16_bits(xv[2 * i + 1])) << 16);
+      *reinterpret_cast<uint4*>(xb16 + static_cast<size_t>(t) * K + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  if (codes && sa_sorted && threadIdx.x == 0) sa_sorted[p] = sa;
+}
+
+// ------------------------------------------------------------------ weight quantization + packing
+// One CTA per (128-row tile, 128-channel block), thread = row. Two passes over
+// the block: group absmax -> scale, then codes, packed 32 codes at a time.
+template <bool BF16, int BITS>
+__global__ void __launch_bounds__(128) k_quant_w(const void* __restrict__ W, const float* __restrict__ s, int N,
+                                                 int K, int group, uint8_t* __restrict__ packed,
+                                                 float* __restrict__ w_scale) {
+  constexpr int qmax = (1 << (BITS - 1)) - 1;
+  const int nt = blockIdx.x, kb = blockIdx.y, r = threadIdx.x;
+  const int o = nt * kTileN + r;
+  const int KB = static_cast<int>(ceil_div(K, kTileK));
+  const int kbase = kb * kTileK;
+  const bool row_ok = o < N;
+  auto wval = [&](int k) -> float {
+    if (!row_ok || k >= K) return 0.0f;
+    const size_t i = static_cast<size_t>(o) * K + k;
+    const float w = BF16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(W)[i]) : static_cast<const float*>(W)[i];
+    return __fmul_rn(w, s[k]);
+  };
+  float sc[2] = {0.0f, 0.0f};
+  const int gpb = kTileK / group;  // groups per block: 1 (g=128) or 2 (g=64)
+  for (int gi = 0; gi < gpb; ++gi) {
+    const int k0 = kbase + gi * group;
+    if (k0 >= K) break;
+    float amax = 0.0f;
+    for (int k = k0; k < k0 + group; ++k) amax = fmaxf(amax, fabsf(wval(k)));
+    sc[gi] = __fdiv_rn(amax, static_cast<float>(qmax));
+    if (row_ok) w_scale[static_cast<size_t>(k0 / group) * N + o] = sc[gi];
+  }
+  const size_t block = static_cast<size_t>(nt) * KB + kb;
+  for (int h = 0; h < 4; ++h) {  // 32 codes at a time
+    int q[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int kl = 32 * h + i;
+      const int k = kbase + kl;
+      q[i] = (k < K) ? rtn_code(wval(k), sc[kl / group], qmax) : 0;
+    }
+    if constexpr (BITS == 4) {
+      uint32_t wd[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t x = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const uint32_t lo = static_cast<uint32_t>(q[4 * w + b]) & 0xFu;
+          const uint32_t hi = static_cast<uint32_t>(q[16 + 4 * w + b]) & 0xFu;
+          x |= (lo | (hi << 4)) << (8 * b);
+        }
+        wd[w] = x;
+      }
+      *reinterpret_cast<uint4*>(packed + block * kW4BlockBytes + r * 64 + h * 16) =
+          make_uint4(wd[0], wd[1], wd[2], wd[3]);
+    } else {
+      uint32_t two[2] = {0u, 0u}, one = 0u;
+#pragma unroll
+      for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const uint32_t u0 = static_cast<uint32_t>(q[16 * mm + 2 * p] + 4);
+          const uint32_t u1 = static_cast<uint32_t>(q[16 * mm + 2 * p + 1] + 4);
+          two[mm] |= ((u0 & 3u) << (2 * p)) | ((u1 & 3u) << (16 + 2 * p));
+        }
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        const uint32_t u0 = static_cast<uint32_t>(q[2 * p] + 4);
+        const uint32_t u1 = static_cast<uint32_t>(q[2 * p + 1] + 4);
+        one |= ((u0 >> 2) & 1u) << p;
+        one |= ((u1 >> 2) & 1u) << (16 + p);
+      }
+      uint8_t* row = packed + block * kW3BlockBytes + r * 48;
+      *reinterpret_cast<uint2*>(row + 8 * h) = make_uint2(two[0], two[1]);
+      *reinterpret_cast<uint32_t*>(row + 32 + 4 * h) = one;
+    }
+  }
+}
+
+// w_mean[k] = (sum_o |W[o][k]| in fp64) / N rounded once; w_colmax[k] = max_o |W[o][k]|.
+template <bool BF16>
+__global__ void __launch_bounds__(64) k_colstats(const void* __restrict__ W, int N, int K,
+                                                 float* __restrict__ w_mean, float* __restrict__ w_colmax) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  double sum = 0.0;
+  float mx = 0.0f;
+  for (int o = 0; o < N; ++o) {
+    const size_t i = static_cast<size_t>(o) * K + k;
+    const float w = BF16 ? bf16_bits_to_f32(__ldg(static_cast<const uint16_t*>(W) + i))
+                         : __ldg(static_cast<const float*>(W) + i);
+    const float a = fabsf(w);
+    sum += static_cast<double>(a);
+    mx = fmaxf(mx, a);
+  }
+  if (w_mean) w_mean[k] = static_cast<float>(sum / static_cast<double>(N));
+  if (w_colmax) w_colmax[k] = mx;
+}
+
+// Inverse of the packing above (diagnostics).
+template <int BITS>
+__global__ void __launch_bounds__(128) k_unpack_w(const uint8_t* __restrict__ packed, int N, int K,
+                                                  int8_t* __restrict__ codes) {
+  const int nt = blockIdx.x, kb = blockIdx.y, r = threadIdx.x;
+  const int o = nt * kTileN + r;
+  if (o >= N) return;
+  const int KB = static_cast<int>(ceil_div(K, kTileK));
+  const size_t block = static_cast<size_t>(nt) * KB + kb;
+  for (int kl = 0; kl < kTileK; ++kl) {
+    const int k = kb * kTileK + kl;
+    if (k >= K) break;
+    int q;
+    if constexpr (BITS == 4) {
+      const int h = kl / 32, i = kl % 32;
+      const int hi = i / 16, w = (i % 16) / 4, b = i % 4;
+      const uint8_t byte = packed[block * kW4BlockBytes + r * 64 + h * 16 + 4 * w + b];
+      const int nib = hi ? (byte >> 4) : (byte & 0xF);
+      q = (nib & 8) ? nib - 16 : nib;
+    } else {
+      const uint8_t* row = packed + block * kW3BlockBytes + r * 48;
+      const int m = kl / 16, p = (kl % 16) / 2, odd = kl & 1;
+      const uint32_t two = *reinterpret_cast<const uint32_t*>(row + 4 * m);
+      const int hword = kl / 32, hp = (kl % 32) / 2;
+      const uint32_t one = *reinterpret_cast<const uint32_t*>(row + 32 + 4 * hword);
+      const uint32_t lo2 = (two >> (odd ? 16 + 2 * p : 2 * p)) & 3u;
+      const uint32_t b2 = (one >> (odd ? 16 + hp : hp)) & 1u;
+      q = static_cast<int>(lo2 | (b2 << 2)) - 4;
+    }
+    codes[static_cast<size_t>(o) * K + k] = static_cast<int8_t>(q);
+  }
+}
+
+// Adapter packing: A_catT [R_pad][K], B_catT [N][R_pad], G copy [K][n_r], all bf16.
+__global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a, int R_pad,
+                                const uint16_t* __restrict__ A_s, const uint16_t* __restrict__ B_s,
+                                const uint16_t* __restrict__ A_r, const uint16_t* __restrict__ B_r,
+                                const uint16_t* __restrict__ G, uint16_t* __restrict__ acat,
+                                uint16_t* __restrict__ bcat, uint16_t* __restrict__ gout) {
+  const size_t n1 = static_cast<size_t>(R_pad) * K, n2 = static_cast<size_t>(N) * R_pad,
+               n3 = static_cast<size_t>(K) * n_r;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n1 + n2 + n3;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    if (i < n1) {
+      const int c = static_cast<int>(i / K), k = static_cast<int>(i % K);
+      uint16_t v = 0;
+      if (c < r_s) v = A_s[static_cast<size_t>(k) * r_s + c];
+      else if (c < R_a) {
+        const int e = (c - r_s) / r_r, j = (c - r_s) % r_r;
+        v = A_r[(static_cast<size_t>(e) * K + k) * r_r + j];
+      }
+      acat[i] = v;
+    } else if (i < n1 + n2) {
+      const size_t ii = i - n1;
+      const int o = static_cast<int>(ii / R_pad), c = static_cast<int>(ii % R_pad);
+      uint16_t v = 0;
+      if (c < r_s) v = B_s[static_cast<size_t>(c) * N + o];
+      else if (c < R_a) {
+        const int e = (c - r_s) / r_r, j = (c - r_s) % r_r;
+        v = B_r[(static_cast<size_t>(e) * r_r + j) * N + o];
+      }
+      bcat[ii] = v;
+    } else {
+      const size_t ii = i - n1 - n2;
+      gout[ii] = G[ii];
+    }
+  }
+}
+
+// U_cat[p][c] = bf16(sum_s P[s][t][c]) with t = perm[p]; routed columns of other experts -> 0.
+__global__ void k_ufinal(const float* __restrict__ partial, int splits, const int32_t* __restrict__ perm,
+                         const int32_t* __restrict__ expert, int T, int R_pad, int r_s, int r_r, int R_a,
+                         uint16_t* __restrict__ ucat) {
+  const int chunks = R_pad / 8;
+  const size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (idx >= static_cast<size_t>(T) * chunks) return;
+  const int p = static_cast<int>(idx / chunks), c0 = static_cast<int>(idx % chunks) * 8;
+  const int t = perm[p];
+  const int e = expert[t];
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+  for (int s = 0; s < splits; ++s) {
+    const float* src = partial + (static_cast<size_t>(s) * T + t) * R_pad + c0;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  }
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = c0 + i;
+    bool keep = c < R_a && (c < r_s || (c - r_s) / r_r == e);
+    if (!keep) v[i] = 0.0f;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i])) | (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i + 1])) << 16);
+  *reinterpret_cast<uint4*>(ucat + static_cast<size_t>(p) * R_pad + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Y[perm[p]][o] = sum_s partial[s][p][o] (fixed order).
+__global__ void k_splitk_reduce(const float* __restrict__ partial, int splits, const int32_t* __restrict__ perm,
+                                int T, int N, void* __restrict__ Y, int y_bf16) {
+  const size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (idx >= static_cast<size_t>(T) * N) return;
+  const int p = static_cast<int>(idx / N), o = static_cast<int>(idx % N);
+  float v = 0.0f;
+  for (int s = 0; s < splits; ++s) v += partial[(static_cast<size_t>(s) * T + p) * N + o];
+  const size_t dst = static_cast<size_t>(perm[p]) * N + o;
+  if (y_bf16) static_cast<uint16_t*>(Y)[dst] = f32_to_bf16_bits(v);
+  else static_cast<float*>(Y)[dst] = v;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_route_stats(const void* X, bool x_bf16, const float* s_inv, const uint16_t* G, int T, int K,
+                               int n_r, int qmax, int32_t* expert, float* sa, float* logits, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+#define QE_ROUTE(B, NR) k_route_stats<B, NR><<<T, 256, 0, st>>>(X, s_inv, G, T, K, n_r, qmax, expert, sa, logits)
+  if (x_bf16) {
+    if (n_r == 8) QE_ROUTE(true, 8);
+    else if (n_r <= 4) QE_ROUTE(true, 4);
+    else QE_ROUTE(true, 16);
+  } else {
+    if (n_r == 8) QE_ROUTE(false, 8);
+    else if (n_r <= 4) QE_ROUTE(false, 4);
+    else QE_ROUTE(false, 16);
+  }
+#undef QE_ROUTE
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bucket(const int32_t* expert, int T, int n_r, int32_t* perm, int32_t* pos, int32_t* offsets,
+                          cudaStream_t st) {
+  k_bucket<<<1, 1024, 0, st>>>(expert, T, n_r, perm, pos, offsets);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
+                             const float* sa_tok, const int32_t* pos, int8_t* codes, float* sa_sorted,
+                             uint16_t* act16, uint16_t* xb16, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (x_bf16)
+    k_act_quant<true><<<T, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16);
+  else
+    k_act_quant<false><<<T, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_weights(const void* W, bool w_bf16, const float* s, int N, int K, int group,
+                                    int w_bits, uint8_t* packed, float* w_scale, cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>(ceil_div(N, kTileN)), static_cast<unsigned>(ceil_div(K, kTileK)));
+  if (w_bits == 4) {
+    if (w_bf16) k_quant_w<true, 4><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale);
+    else k_quant_w<false, 4><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale);
+  } else {
+    if (w_bf16) k_quant_w<true, 3><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale);
+    else k_quant_w<false, 3><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_colstats(const void* W, bool w_bf16, int N, int K, float* w_mean, float* w_colmax,
+                            cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(ceil_div(K, 64));
+  if (w_bf16) k_colstats<true><<<grid, 64, 0, st>>>(W, N, K, w_mean, w_colmax);
+  else k_colstats<false><<<grid, 64, 0, st>>>(W, N, K, w_mean, w_colmax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_weights(const uint8_t* packed, int N, int K, int w_bits, int8_t* codes,
+                                  cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>(ceil_div(N, kTileN)), static_cast<unsigned>(ceil_div(K, kTileK)));
+  if (w_bits == 4) k_unpack_w<4><<<grid, 128, 0, st>>>(packed, N, K, codes);
+  else k_unpack_w<3><<<grid, 128, 0, st>>>(packed, N, K, codes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint16_t* A_s, const uint16_t* B_s,
+                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out,
+                                 cudaStream_t st) {
+  k_pack_adapters<<<592, 256, 0, st>>>(K, N, g.r_s, g.n_r, g.r_r, g.R_a, g.R_pad, A_s, B_s, A_r, B_r, G,
+                                       reinterpret_cast<uint16_t*>(out + g.off_acat),
+                                       reinterpret_cast<uint16_t*>(out + g.off_bcat),
+                                       reinterpret_cast<uint16_t*>(out + g.off_g));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ufinal(const float* partial, int splits, const int32_t* perm, const int32_t* expert, int T,
+                          int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(T) * (R_pad / 8);
+  if (n == 0) return cudaSuccess;
+  k_ufinal<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, st>>>(partial, splits, perm, expert, T, R_pad, r_s,
+                                                                    r_r > 0 ? r_r : 1, R_a, ucat);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_splitk_reduce(const float* partial, int splits, const int32_t* perm, int T, int N, void* Y,
+                                 int y_bf16, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(T) * N;
+  if (n == 0) return cudaSuccess;
+  k_splitk_reduce<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, st>>>(partial, splits, perm, T, N, Y, y_bf16);
+  return cudaGetLastError();
+}
+
+}  // namespace qe

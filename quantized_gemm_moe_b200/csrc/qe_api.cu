@@ -1,0 +1,441 @@
+// Host side of the C ABI declared in include/qe.h: argument validation,
+// workspace planning, TMA tensor-map encoding and the launch sequence of the
+// QE linear layer. Nothing here allocates device memory.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qe.h"
+#include "qe_internal.h"
+
+namespace qe {
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+qe_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", where, cudaGetErrorString(e));
+  return QE_ERR_CUDA;
+}
+
+#define QE_CUDA(call, where)                          \
+  do {                                                \
+    cudaError_t e_ = (call);                          \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qe_status check_desc(const qe_layer_desc* d) {
+  if (!d) return QE_ERR_INVALID_ARG;
+  if (d->d_in <= 0 || d->d_out <= 0 || d->group <= 0) return QE_ERR_INVALID_ARG;
+  if (d->group != 64 && d->group != 128) return QE_ERR_UNSUPPORTED;
+  if (d->d_in % d->group != 0) return QE_ERR_INVALID_ARG;
+  if (d->d_in < 128) return QE_ERR_UNSUPPORTED;
+  if (d->w_bits != 3 && d->w_bits != 4) return QE_ERR_UNSUPPORTED;
+  if (d->a_bits != 6 && d->a_bits != 8 && d->a_bits != 16) return QE_ERR_UNSUPPORTED;
+  if (d->a_bits != 16 && d->w_bits != 4) return QE_ERR_UNSUPPORTED;  // W3 runs weight-only
+  if (d->n_routed < 1 || d->n_routed > kMaxRouted) return QE_ERR_UNSUPPORTED;
+  if (d->rank_shared < 0 || d->rank_routed < 0) return QE_ERR_INVALID_ARG;
+  if (d->rank_shared + int64_t(d->n_routed) * d->rank_routed > 512) return QE_ERR_UNSUPPORTED;
+  if (d->d_in > (1 << 24) || d->d_out > (1 << 24)) return QE_ERR_UNSUPPORTED;
+  return QE_OK;
+}
+
+int qmax_of(int bits) { return (1 << (bits - 1)) - 1; }
+
+size_t packed_bytes(const qe_layer_desc* d) {
+  const size_t blocks = size_t(ceil_div(d->d_out, kTileN)) * size_t(ceil_div(d->d_in, kTileK));
+  return blocks * (d->w_bits == 4 ? kW4BlockBytes : kW3BlockBytes);
+}
+
+AdapterGeom geom_of(const qe_layer_desc* d) {
+  return adapter_geom(d->d_in, d->d_out, d->rank_shared, d->n_routed, d->rank_routed);
+}
+
+// ------------------------------------------------------------------ workspace plan
+struct Plan {
+  int T, K, N;
+  bool has_ad;
+  AdapterGeom g;
+  UgemmPlan up;
+  int bn, msplits, kbps;  // main product
+  size_t off_expert, off_perm, off_pos, off_offsets, off_sa_tok, off_sa_sorted, off_act, off_xb16, off_upart,
+      off_ucat, off_ypart, bytes;
+};
+
+int wonly_splits(int T, int N, int K) {
+  const int64_t ntiles = ceil_div(N, kTileN);
+  const int64_t ttiles = ceil_div(T, 16);
+  const int KB = static_cast<int>(ceil_div(K, kTileK));
+  int splits = static_cast<int>(ceil_div(2 * 148, ntiles * ttiles));
+  splits = std::max(1, std::min(splits, std::max(1, KB / 4)));
+  const int kbps = static_cast<int>(ceil_div(KB, splits));
+  return static_cast<int>(ceil_div(KB, kbps));
+}
+
+Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
+  Plan p{};
+  p.T = T;
+  p.K = d->d_in;
+  p.N = d->d_out;
+  p.g = geom_of(d);
+  p.has_ad = p.g.R_a > 0;
+  const int Tm = std::max(T, 1);
+  p.up = plan_ugemm(Tm, p.K, p.g.R_pad);
+  if (d->a_bits == 16) {
+    p.bn = 0;
+    p.msplits = wonly_splits(Tm, p.N, p.K);
+    p.kbps = 0;
+  } else {
+    p.bn = pick_qgemm_bn(Tm, p.N, p.K, &p.msplits, &p.kbps);
+  }
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  p.off_expert = take(size_t(Tm) * 4);
+  p.off_perm = take(size_t(Tm) * 4);
+  p.off_pos = take(size_t(Tm) * 4);
+  p.off_offsets = take(size_t(kMaxRouted + 1) * 4);
+  p.off_sa_tok = take(size_t(Tm) * 4);
+  p.off_sa_sorted = take(size_t(Tm) * 4);
+  p.off_act = take(size_t(Tm) * p.K * (d->a_bits == 16 ? 2 : 1));
+  p.off_xb16 = (!x_bf16 && p.has_ad) ? take(size_t(Tm) * p.K * 2) : 0;
+  p.off_upart = p.has_ad ? take(size_t(p.up.splits) * Tm * p.g.R_pad * 4) : 0;
+  p.off_ucat = p.has_ad ? take(size_t(Tm) * p.g.R_pad * 2) : 0;
+  p.off_ypart = (p.msplits > 1) ? take(size_t(p.msplits) * Tm * p.N * 4) : 0;
+  p.bytes = o;
+  return p;
+}
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2-D row-major [rows][cols] tensor, box {box_cols, box_rows}, 128-byte swizzle, zero fill out of bounds.
+qe_status make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t cols,
+                    uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
+    return QE_ERR_CUDA;
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", int(r));
+    return QE_ERR_CUDA;
+  }
+  return QE_OK;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const void* X, qe_dtype xd, int32_t T,
+                       void* Y, qe_dtype yd, void* ws, size_t ws_bytes, int32_t* dbg_acc, int32_t* dbg_expert,
+                       int32_t* dbg_perm, float* dbg_sa, int32_t stages, cudaStream_t st) {
+  qe_status s = check_desc(d);
+  if (s != QE_OK) return s;
+  if (!w || !w->w_packed || !w->w_scale || !w->s_inv || !w->adapters) return QE_ERR_INVALID_ARG;
+  if (T < 0 || T > (1 << 20)) return QE_ERR_INVALID_ARG;
+  if (xd != QE_F32 && xd != QE_BF16) return QE_ERR_INVALID_ARG;
+  if (yd != QE_F32 && yd != QE_BF16) return QE_ERR_INVALID_ARG;
+  if (T == 0) return QE_OK;
+  if (!X || !Y) return QE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(w->w_packed) || !aligned16(w->w_scale) ||
+      !aligned16(w->s_inv) || !aligned16(w->adapters))
+    return QE_ERR_ALIGNMENT;
+  const bool x_bf16 = xd == QE_BF16;
+  const Plan p = make_plan(d, T, x_bf16);
+  if (!ws || ws_bytes < p.bytes) return QE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QE_ERR_ALIGNMENT;
+  int* err = device_error_ptr();
+  const uint8_t* ad = static_cast<const uint8_t*>(w->adapters);
+  const uint16_t* acat = reinterpret_cast<const uint16_t*>(ad + p.g.off_acat);
+  const uint16_t* bcat = reinterpret_cast<const uint16_t*>(ad + p.g.off_bcat);
+  const uint16_t* G = reinterpret_cast<const uint16_t*>(ad + p.g.off_g);
+  int32_t* expert = at<int32_t>(ws, p.off_expert);
+  int32_t* perm = at<int32_t>(ws, p.off_perm);
+  int32_t* pos = at<int32_t>(ws, p.off_pos);
+  int32_t* offsets = at<int32_t>(ws, p.off_offsets);
+  float* sa_tok = at<float>(ws, p.off_sa_tok);
+  float* sa_sorted = at<float>(ws, p.off_sa_sorted);
+  const bool wonly = d->a_bits == 16;
+  const int qmax = wonly ? 1 : qmax_of(d->a_bits);
+  const int K = p.K, N = p.N;
+
+  // 1. router + per-token absmax, then the stable bucket sort
+  if (stages & QE_STAGE_ROUTE) {
+    QE_CUDA(launch_route_stats(X, x_bf16, w->s_inv, G, T, K, d->n_routed, qmax, expert, wonly ? nullptr : sa_tok,
+                               nullptr, st),
+            "route_stats");
+    QE_CUDA(launch_bucket(expert, T, d->n_routed, perm, pos, offsets, st), "bucket");
+  }
+  // 3. quantize in bucket order
+  int8_t* codes = wonly ? nullptr : at<int8_t>(ws, p.off_act);
+  uint16_t* act16 = wonly ? at<uint16_t>(ws, p.off_act) : nullptr;
+  uint16_t* xb16 = (!x_bf16 && p.has_ad) ? at<uint16_t>(ws, p.off_xb16) : nullptr;
+  if (stages & QE_STAGE_QUANT)
+    QE_CUDA(launch_act_quant(X, x_bf16, w->s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16, st),
+            "act_quant");
+  // 4. adapter down-projection (tensor cores) -> U_cat in bucket order
+  uint16_t* ucat = p.has_ad ? at<uint16_t>(ws, p.off_ucat) : nullptr;
+  if (p.has_ad && (stages & QE_STAGE_ADAPTERS)) {
+    CUtensorMap tm_x, tm_acat;
+    const void* xsrc = x_bf16 ? X : static_cast<const void*>(xb16);
+    if ((s = make_tmap(&tm_x, xsrc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK) return s;
+    if ((s = make_tmap(&tm_acat, acat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, p.g.R_pad, kAdapterAtom,
+                       p.up.nu)) != QE_OK)
+      return s;
+    float* upart = at<float>(ws, p.off_upart);
+    QE_CUDA(launch_ugemm(tm_x, tm_acat, p.up, T, K, p.g.R_pad, upart, err, st), "ugemm");
+    QE_CUDA(launch_ufinal(upart, p.up.splits, perm, expert, T, p.g.R_pad, d->rank_shared, d->rank_routed, p.g.R_a,
+                          ucat, st),
+            "ufinal");
+  }
+  // 5. main product
+  if (!(stages & QE_STAGE_PRODUCT)) return QE_OK;
+  float* ypart = p.msplits > 1 ? at<float>(ws, p.off_ypart) : nullptr;
+  const int y_bf16 = yd == QE_BF16;
+  if (wonly) {
+    QE_CUDA(launch_wonly(act16, static_cast<const uint8_t*>(w->w_packed), w->w_scale, d->w_bits, ucat, bcat,
+                         p.g.R_pad, p.has_ad ? 1 : 0, perm, T, N, K, d->group, Y, y_bf16, ypart, p.msplits, st),
+            "wonly");
+  } else {
+    CUtensorMap tm_xq, tm_bcat, tm_ucat;
+    if ((s = make_tmap(&tm_xq, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, T, kTileK, p.bn)) != QE_OK) return s;
+    if (p.has_ad) {
+      if ((s = make_tmap(&tm_bcat, bcat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.g.R_pad, N, kAdapterAtom, kTileN)) !=
+          QE_OK)
+        return s;
+      if ((s = make_tmap(&tm_ucat, ucat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.g.R_pad, T, kAdapterAtom, p.bn)) !=
+          QE_OK)
+        return s;
+    } else {
+      tm_bcat = tm_xq;
+      tm_ucat = tm_xq;
+    }
+    QgemmArgs a{};
+    a.w_packed = static_cast<const uint8_t*>(w->w_packed);
+    a.w_scale = w->w_scale;
+    a.sa_sorted = sa_sorted;
+    a.perm = perm;
+    a.T = T;
+    a.N = N;
+    a.K = K;
+    a.group = d->group;
+    a.KB = static_cast<int>(ceil_div(K, kTileK));
+    a.adapter_atoms = p.has_ad ? p.g.R_pad / kAdapterAtom : 0;
+    a.splits = p.msplits;
+    a.kb_per_split = p.kbps;
+    a.Y = Y;
+    a.y_bf16 = y_bf16;
+    a.partial = ypart;
+    a.dbg_acc = dbg_acc;
+    a.err = err;
+    QE_CUDA(launch_qgemm(p.bn, tm_xq, tm_bcat, tm_ucat, a, st), "qgemm");
+  }
+  if (p.msplits > 1) QE_CUDA(launch_splitk_reduce(ypart, p.msplits, perm, T, N, Y, y_bf16, st), "splitk_reduce");
+  if (dbg_expert) QE_CUDA(cudaMemcpyAsync(dbg_expert, expert, size_t(T) * 4, cudaMemcpyDeviceToDevice, st), "copy");
+  if (dbg_perm) QE_CUDA(cudaMemcpyAsync(dbg_perm, perm, size_t(T) * 4, cudaMemcpyDeviceToDevice, st), "copy");
+  if (dbg_sa) QE_CUDA(cudaMemcpyAsync(dbg_sa, sa_tok, size_t(T) * 4, cudaMemcpyDeviceToDevice, st), "copy");
+  return QE_OK;
+}
+
+}  // namespace
+}  // namespace qe
+
+using namespace qe;
+
+extern "C" {
+
+size_t qe_packed_weight_bytes(const qe_layer_desc* desc) {
+  if (check_desc(desc) != QE_OK) return 0;
+  return packed_bytes(desc);
+}
+
+size_t qe_adapter_packed_bytes(const qe_layer_desc* desc) {
+  if (check_desc(desc) != QE_OK) return 0;
+  return geom_of(desc).bytes;
+}
+
+size_t qe_linear_workspace_bytes(const qe_layer_desc* desc, int32_t T) {
+  if (check_desc(desc) != QE_OK || T < 0) return 0;
+  // sized for the larger of the fp32 / bf16 input plans
+  return std::max(make_plan(desc, T, true).bytes, make_plan(desc, T, false).bytes);
+}
+
+qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, qe_dtype w_dtype, const float* s,
+                              void* w_packed, float* w_scale, float* w_mean, float* w_colmax, void* stream) {
+  qe_status st = check_desc(desc);
+  if (st != QE_OK) return st;
+  if (!W || !s || !w_packed || !w_scale) return QE_ERR_INVALID_ARG;
+  if (w_dtype != QE_F32 && w_dtype != QE_BF16) return QE_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(s) || !aligned16(w_packed) || !aligned16(w_scale) ||
+      (w_mean && !aligned16(w_mean)) || (w_colmax && !aligned16(w_colmax)))
+    return QE_ERR_ALIGNMENT;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  QE_CUDA(launch_quantize_weights(W, w_dtype == QE_BF16, s, desc->d_out, desc->d_in, desc->group, desc->w_bits,
+                                  static_cast<uint8_t*>(w_packed), w_scale, cs),
+          "quantize_weights");
+  if (w_mean || w_colmax)
+    QE_CUDA(launch_colstats(W, w_dtype == QE_BF16, desc->d_out, desc->d_in, w_mean, w_colmax, cs), "colstats");
+  return QE_OK;
+}
+
+qe_status qe_pack_adapters(const qe_layer_desc* desc, const void* A_s, const void* B_s, const void* A_r,
+                           const void* B_r, const void* G, void* out, void* stream) {
+  qe_status st = check_desc(desc);
+  if (st != QE_OK) return st;
+  if (!G || !out) return QE_ERR_INVALID_ARG;
+  if (desc->rank_shared > 0 && (!A_s || !B_s)) return QE_ERR_INVALID_ARG;
+  if (desc->rank_routed > 0 && (!A_r || !B_r)) return QE_ERR_INVALID_ARG;
+  if (!aligned16(out)) return QE_ERR_ALIGNMENT;
+  const AdapterGeom g = geom_of(desc);
+  QE_CUDA(launch_pack_adapters(g, desc->d_in, desc->d_out, static_cast<const uint16_t*>(A_s),
+                               static_cast<const uint16_t*>(B_s), static_cast<const uint16_t*>(A_r),
+                               static_cast<const uint16_t*>(B_r), static_cast<const uint16_t*>(G),
+                               static_cast<uint8_t*>(out), static_cast<cudaStream_t>(stream)),
+          "pack_adapters");
+  return QE_OK;
+}
+
+qe_status qe_topk_importance(const void* X, qe_dtype x_dtype, const float* w_mean, int32_t T, int32_t d_in,
+                             int32_t k, int32_t* idx, int32_t* hist, int32_t accumulate_hist, void* stream) {
+  if (T < 0 || d_in <= 0 || k < 1 || k > 128 || k > d_in) return QE_ERR_INVALID_ARG;
+  if (d_in % 8 != 0 || d_in > 32768) return QE_ERR_UNSUPPORTED;
+  if (x_dtype != QE_F32 && x_dtype != QE_BF16) return QE_ERR_INVALID_ARG;
+  if (!w_mean || (T > 0 && (!X || !idx))) return QE_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || !aligned16(w_mean)) return QE_ERR_ALIGNMENT;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (hist && !accumulate_hist) QE_CUDA(cudaMemsetAsync(hist, 0, size_t(d_in) * 4, cs), "memset hist");
+  QE_CUDA(launch_topk(X, x_dtype == QE_BF16, w_mean, T, d_in, k, idx, hist, cs), "topk");
+  return QE_OK;
+}
+
+qe_status qe_route(const void* X, qe_dtype x_dtype, const void* G, int32_t T, int32_t d_in, int32_t n_routed,
+                   int32_t* expert, int32_t* perm, int32_t* offsets, float* logits, void* stream) {
+  if (T < 0 || T > (1 << 20) || d_in <= 0 || n_routed < 1 || n_routed > kMaxRouted) return QE_ERR_INVALID_ARG;
+  if (d_in % 8 != 0) return QE_ERR_UNSUPPORTED;
+  if (x_dtype != QE_F32 && x_dtype != QE_BF16) return QE_ERR_INVALID_ARG;
+  if (!G || !expert || !perm || !offsets || (T > 0 && !X)) return QE_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || !aligned16(G)) return QE_ERR_ALIGNMENT;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // routing alone: no activation scale is computed, so s_inv is not read
+  QE_CUDA(launch_route_stats(X, x_dtype == QE_BF16, nullptr, static_cast<const uint16_t*>(G),
+                             T, d_in, n_routed, 1, expert, nullptr, logits, cs),
+          "route_stats");
+  QE_CUDA(launch_bucket(expert, T, n_routed, perm, nullptr, offsets, cs), "bucket");
+  return QE_OK;
+}
+
+qe_status qe_linear_forward(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
+                            qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return forward_impl(desc, weights, X, x_dtype, T, Y, y_dtype, workspace, workspace_bytes, nullptr, nullptr,
+                      nullptr, nullptr, QE_STAGE_ALL, static_cast<cudaStream_t>(stream));
+}
+
+int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype) {
+  if (check_desc(desc) != QE_OK || T < 0) return -1;
+  if (T == 0) return 0;
+  const Plan p = make_plan(desc, T, x_dtype == QE_BF16);
+  int n = 3;                    // route_stats, bucket, act_quant
+  if (p.has_ad) n += 2;         // ugemm, ufinal
+  n += 1;                       // qgemm or the weight-only product
+  if (p.msplits > 1) n += 1;    // split-K reduce
+  return n;
+}
+
+qe_status qe_linear_forward_stages(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
+                                   qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,
+                                   size_t workspace_bytes, int32_t stages, void* stream) {
+  if (stages & ~QE_STAGE_ALL) return QE_ERR_INVALID_ARG;
+  return forward_impl(desc, weights, X, x_dtype, T, Y, y_dtype, workspace, workspace_bytes, nullptr, nullptr,
+                      nullptr, nullptr, stages, static_cast<cudaStream_t>(stream));
+}
+
+qe_status qe_linear_forward_debug(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
+                                  qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,
+                                  size_t workspace_bytes, int32_t* acc, int32_t* expert, int32_t* perm, float* sa,
+                                  void* stream) {
+  if (desc && desc->a_bits == 16 && acc) return QE_ERR_UNSUPPORTED;
+  return forward_impl(desc, weights, X, x_dtype, T, Y, y_dtype, workspace, workspace_bytes, acc, expert, perm, sa,
+                      QE_STAGE_ALL, static_cast<cudaStream_t>(stream));
+}
+
+qe_status qe_unpack_weights(const qe_layer_desc* desc, const void* w_packed, int8_t* codes, void* stream) {
+  qe_status st = check_desc(desc);
+  if (st != QE_OK) return st;
+  if (!w_packed || !codes) return QE_ERR_INVALID_ARG;
+  QE_CUDA(launch_unpack_weights(static_cast<const uint8_t*>(w_packed), desc->d_out, desc->d_in, desc->w_bits, codes,
+                                static_cast<cudaStream_t>(stream)),
+          "unpack_weights");
+  return QE_OK;
+}
+
+qe_status qe_act_quant(const void* X, qe_dtype x_dtype, const float* s_inv, int32_t T, int32_t d_in, int32_t a_bits,
+                       int8_t* codes, float* sa, void* stream) {
+  if (T < 0 || d_in <= 0 || (a_bits != 6 && a_bits != 8)) return QE_ERR_INVALID_ARG;
+  if (d_in % 8 != 0) return QE_ERR_UNSUPPORTED;
+  if (x_dtype != QE_F32 && x_dtype != QE_BF16) return QE_ERR_INVALID_ARG;
+  if (!s_inv || !sa || (T > 0 && (!X || !codes))) return QE_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || !aligned16(s_inv) || (codes && (reinterpret_cast<uintptr_t>(codes) & 7u)))
+    return QE_ERR_ALIGNMENT;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int qmax = qmax_of(a_bits);
+  QE_CUDA(launch_route_stats(X, x_dtype == QE_BF16, s_inv, nullptr, T, d_in, 0, qmax, nullptr, sa, nullptr, cs),
+          "act_stats");
+  QE_CUDA(launch_act_quant(X, x_dtype == QE_BF16, s_inv, T, d_in, qmax, sa, nullptr, codes, nullptr, nullptr,
+                           nullptr, cs),
+          "act_quant");
+  return QE_OK;
+}
+
+const char* qe_status_string(qe_status s) {
+  switch (s) {
+    case QE_OK: return "ok";
+    case QE_ERR_INVALID_ARG: return "invalid argument";
+    case QE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QE_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case QE_ERR_WORKSPACE: return "workspace missing or too small";
+    case QE_ERR_CUDA: return "CUDA error";
+    case QE_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* qe_last_cuda_error(void) { return g_last_cuda_error; }
+
+qe_status qe_device_error(void* stream, int32_t* code, int32_t clear) {
+  int v = 0;
+  QE_CUDA(read_device_error(&v, clear != 0, static_cast<cudaStream_t>(stream)), "device_error");
+  if (code) *code = v;
+  return v ? QE_ERR_TIMEOUT : QE_OK;
+}
+
+}  // extern "C"

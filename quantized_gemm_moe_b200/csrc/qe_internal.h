@@ -1,0 +1,120 @@
+// Internal declarations shared by the host API (qe_api.cu) and the kernel files.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace qe {
+
+constexpr int kTileN = 128;       // output rows per weight block / GEMM tile (MMA M)
+constexpr int kTileK = 128;       // input channels per weight block / pipeline stage
+constexpr int kW4BlockBytes = 8192;
+constexpr int kW3BlockBytes = 6144;
+constexpr int kMaxRouted = 16;
+constexpr int kAdapterAtom = 64;  // bf16 elements per 128-byte swizzle row
+
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Packed adapter buffer geometry.
+struct AdapterGeom {
+  int r_s, n_r, r_r;
+  int R_a;    // r_s + n_r * r_r
+  int R_pad;  // round_up(R_a, 64), >= 64
+  size_t off_acat, off_bcat, off_g, bytes;
+};
+inline AdapterGeom adapter_geom(int K, int N, int r_s, int n_r, int r_r) {
+  AdapterGeom g;
+  g.r_s = r_s;
+  g.n_r = n_r;
+  g.r_r = r_r;
+  g.R_a = r_s + n_r * r_r;
+  g.R_pad = static_cast<int>(round_up(g.R_a > 0 ? g.R_a : 1, kAdapterAtom));
+  g.off_acat = 0;
+  g.off_bcat = align256(g.off_acat + size_t(g.R_pad) * K * 2);
+  g.off_g = align256(g.off_bcat + size_t(N) * g.R_pad * 2);
+  g.bytes = align256(g.off_g + size_t(K) * n_r * 2);
+  return g;
+}
+
+// ------------------------------------------------------------------ kernel launchers
+// Each returns the launch's cudaError_t. The host API validates before calling.
+
+cudaError_t launch_quantize_weights(const void* W, bool w_bf16, const float* s, int N, int K, int group,
+                                    int w_bits, uint8_t* packed, float* w_scale, cudaStream_t st);
+cudaError_t launch_colstats(const void* W, bool w_bf16, int N, int K, float* w_mean, float* w_colmax,
+                            cudaStream_t st);
+cudaError_t launch_unpack_weights(const uint8_t* packed, int N, int K, int w_bits, int8_t* codes,
+                                  cudaStream_t st);
+cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint16_t* A_s, const uint16_t* B_s,
+                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out,
+                                 cudaStream_t st);
+
+// Router logits + argmin, and (when sa != nullptr) the per-token absmax -> scale.
+cudaError_t launch_route_stats(const void* X, bool x_bf16, const float* s_inv, const uint16_t* G, int T, int K,
+                               int n_r, int qmax, int32_t* expert, float* sa, float* logits, cudaStream_t st);
+// Stable bucket sort of tokens by expert: perm (sorted pos -> token), pos (token -> sorted pos), offsets.
+cudaError_t launch_bucket(const int32_t* expert, int T, int n_r, int32_t* perm, int32_t* pos, int32_t* offsets,
+                          cudaStream_t st);
+// Per-token quantization of x*s_inv with the scale sa_tok[t], written at row pos[t] (pos == nullptr: row t).
+//   codes != nullptr: int8 codes, sa_sorted[pos] = sa_tok[t]
+//   act16 != nullptr: bf16(x*s_inv) (weight-only layers)
+//   xb16  != nullptr: bf16(x) in token order (for fp32 inputs feeding the adapter GEMM)
+cudaError_t launch_act_quant(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
+                             const float* sa_tok, const int32_t* pos, int8_t* codes, float* sa_sorted,
+                             uint16_t* act16, uint16_t* xb16, cudaStream_t st);
+
+// Adapter down-projection partials: P[split][t][c] = sum_{k in split} X[t][k] * A_catT[c][k] (tcgen05, bf16).
+struct UgemmPlan {
+  int splits;
+  int kchunks_per_split;  // 64-wide K chunks per split
+  int nu;                 // N tile (columns of A_catT per CTA), <= 256
+  int ntiles;
+};
+UgemmPlan plan_ugemm(int T, int K, int R_pad);
+cudaError_t launch_ugemm(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, const UgemmPlan& plan, int T,
+                         int K, int R_pad, float* partial, int* err, cudaStream_t st);
+// U_cat[p][c] = bf16(sum_s P[s][perm[p]][c]), routed columns masked to the token's expert.
+cudaError_t launch_ufinal(const float* partial, int splits, const int32_t* perm, const int32_t* expert, int T,
+                          int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, cudaStream_t st);
+
+// Main quantized GEMM (W4 x A8/A6 codes, tcgen05 kind::i8) with per-group promotion,
+// per-token scale, adapter MMA in the epilogue and scatter to token order.
+struct QgemmArgs {
+  const uint8_t* w_packed;
+  const float* w_scale;     // [G][N]
+  const float* sa_sorted;   // [T]
+  const int32_t* perm;      // [T]
+  int T, N, K, group;
+  int KB;                   // ceil(K / 128)
+  int adapter_atoms;        // R_pad / 64, or 0 when the layer has no adapters
+  int splits, kb_per_split;
+  void* Y;                  // [T][N] (splits == 1)
+  int y_bf16;
+  float* partial;           // [splits][T][N] sorted rows (splits > 1)
+  int32_t* dbg_acc;         // [T][N][G] token order, or nullptr
+  int* err;                 // device error word
+};
+int pick_qgemm_bn(int T, int N, int K, int* splits_out, int* kbps_out);
+cudaError_t launch_qgemm(int BN, const CUtensorMap& tm_xq, const CUtensorMap& tm_bcat, const CUtensorMap& tm_ucat,
+                         const QgemmArgs& a, cudaStream_t st);
+cudaError_t launch_splitk_reduce(const float* partial, int splits, const int32_t* perm, int T, int N, void* Y,
+                                 int y_bf16, cudaStream_t st);
+
+// Weight-only (W3A16 / W4A16) product on CUDA cores, token chunks of up to 16.
+cudaError_t launch_wonly(const uint16_t* act16, const uint8_t* w_packed, const float* w_scale, int w_bits,
+                         const uint16_t* ucat, const uint16_t* bcat, int R_pad, int has_adapters,
+                         const int32_t* perm, int T, int N, int K, int group, void* Y, int y_bf16, float* partial,
+                         int splits, cudaStream_t st);
+
+// Device error word (one per device, in the library's own device memory).
+int* device_error_ptr();  // nullptr when the symbol lookup fails
+cudaError_t read_device_error(int* value, bool clear, cudaStream_t st);
+
+// Top-k importance.
+cudaError_t launch_topk(const void* X, bool x_bf16, const float* w_mean, int T, int K, int k, int32_t* idx,
+                        int32_t* hist, cudaStream_t st);
+
+}  // namespace qe

@@ -1,0 +1,107 @@
+"""CPU checks of the C-ABI boundary: the library loads, exports every symbol
+include/qe.h declares, and its host-side sizing and validation behave as the
+header documents. No compute call runs here (there is no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_gemm_moe_b200 as qe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "qe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qe_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_gemm_moe_b200 import build
+    build.build()
+    return qe.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    declared = _declared_symbols()
+    assert declared, "no declarations parsed from include/qe.h"
+    assert sorted(qe.EXPORTS) == declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_sizes_follow_documented_layout(lib):
+    d = qe.make_desc(1536, 8960, 128, 4, 6, 32, 8, 4)
+    assert qe.packed_weight_bytes(d) == (8960 // 128) * (1536 // 128) * 8192
+    d3 = qe.make_desc(8192, 29568, 128, 3, 16, 32, 8, 4)
+    assert qe.packed_weight_bytes(d3) == (29568 // 128) * (8192 // 128) * 6144
+    # ragged d_out pads to whole 128-row blocks
+    dr = qe.make_desc(256, 200, 64, 4, 8, 8, 4, 4)
+    assert qe.packed_weight_bytes(dr) == 2 * 2 * 8192
+    # adapters: A_catT [R_pad][K] + B_catT [N][R_pad] + G [K][N_r], bf16, 256-byte aligned pieces
+    R_pad = 64
+    expect = 0
+    for nbytes in (R_pad * 1536 * 2, 8960 * R_pad * 2, 1536 * 8 * 2):
+        expect = ((expect + nbytes + 255) // 256) * 256
+    assert qe.adapter_packed_bytes(d) == expect
+    assert qe.linear_workspace_bytes(d, 2048) > 2048 * 1536  # at least the int8 codes
+    assert qe.linear_workspace_bytes(d, 0) > 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("group", 32, qe.QE_ERR_UNSUPPORTED),
+    ("d_in", 100, qe.QE_ERR_INVALID_ARG),
+    ("w_bits", 2, qe.QE_ERR_UNSUPPORTED),
+    ("a_bits", 4, qe.QE_ERR_UNSUPPORTED),
+    ("n_routed", 17, qe.QE_ERR_UNSUPPORTED),
+    ("rank_shared", -1, qe.QE_ERR_INVALID_ARG),
+    ("rank_routed", 200, qe.QE_ERR_UNSUPPORTED),  # 8 + 4*200 > 512
+])
+def test_invalid_desc_rejected_before_launch(lib, field, value, status):
+    d = qe.make_desc(256, 256, 64, 4, 8, 8, 4, 4)
+    setattr(d, field, value)
+    assert qe.packed_weight_bytes(d) == 0
+    w = qe.LayerWeights(16, 16, 16, 16)
+    rc = lib.qe_linear_forward(ctypes.byref(d), ctypes.byref(w), 16, 0, 4, 16, 0, 16, 1 << 30, None)
+    assert rc == status
+
+
+def test_forward_argument_checks(lib):
+    d = qe.make_desc(256, 256, 64, 4, 8, 8, 4, 4)
+    w = qe.LayerWeights(16, 16, 16, 16)
+    f = lib.qe_linear_forward
+    assert f(None, ctypes.byref(w), 16, 0, 4, 16, 0, 16, 1 << 30, None) == qe.QE_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), None, 16, 0, 4, 16, 0, 16, 1 << 30, None) == qe.QE_ERR_INVALID_ARG
+    # T = 0 is a no-op that touches nothing
+    assert f(ctypes.byref(d), ctypes.byref(w), None, 0, 0, None, 0, None, 0, None) == qe.QE_OK
+    # misaligned pointer
+    assert f(ctypes.byref(d), ctypes.byref(w), 18, 0, 4, 16, 0, 16, 1 << 30, None) == qe.QE_ERR_ALIGNMENT
+    # workspace too small
+    assert f(ctypes.byref(d), ctypes.byref(w), 16, 0, 4, 16, 0, 16, 8, None) == qe.QE_ERR_WORKSPACE
+    # bad dtype
+    assert f(ctypes.byref(d), ctypes.byref(w), 16, 7, 4, 16, 0, 16, 1 << 30, None) == qe.QE_ERR_INVALID_ARG
+
+
+def test_other_entry_points_validate(lib):
+    assert lib.qe_topk_importance(16, 1, 16, 4, 256, 0, 16, None, 0, None) == qe.QE_ERR_INVALID_ARG  # k = 0
+    assert lib.qe_topk_importance(16, 1, 16, 4, 256, 129, 16, None, 0, None) == qe.QE_ERR_INVALID_ARG  # k > 128
+    assert lib.qe_route(16, 1, 16, 4, 256, 0, 16, 16, 16, None, None) == qe.QE_ERR_INVALID_ARG  # n_routed = 0
+    assert lib.qe_route(16, 1, 16, 4, 256, 17, 16, 16, 16, None, None) == qe.QE_ERR_INVALID_ARG
+    assert lib.qe_act_quant(16, 1, 16, 4, 256, 5, 16, 16, None) == qe.QE_ERR_INVALID_ARG  # a_bits 5
+    d = qe.make_desc(256, 256, 64, 4, 8, 8, 4, 4)
+    assert lib.qe_quantize_weights(ctypes.byref(d), None, 0, 16, 16, 16, None, None, None) == qe.QE_ERR_INVALID_ARG
+    assert lib.qe_quantize_weights(ctypes.byref(d), 8, 0, 16, 16, 16, None, None, None) == qe.QE_ERR_ALIGNMENT
+    assert lib.qe_pack_adapters(ctypes.byref(d), 16, 16, 16, 16, None, 16, None) == qe.QE_ERR_INVALID_ARG
+    for s in range(7):
+        assert lib.qe_status_string(s)
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    d = qe.make_desc(256, 256, 64, 4, 8, 8, 4, 4)
+    with pytest.raises(qe.QEError):
+        qe.quantize_weights(d, torch.zeros(256, 256), torch.ones(256), torch.zeros(10, dtype=torch.uint8),
+                            torch.zeros(4, 256))

@@ -1,0 +1,316 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, on the same seeded inputs.
+
+Integer stages (weight codes and scales, activation codes and scales, int32
+group accumulators, router choices, bucket order, Top-k index sets and
+histograms) must match bit for bit. Router choices may differ only on
+fp32 near-ties. Final fp outputs must be within 2e-3 (gpu_util.rel_err).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qe_inputs as qi
+import quantized_gemm_moe_b200 as qe
+from gpu_util import Case, Y_TOL, check_routing, cuda, f32, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def _cfg(base="tiny", **kw):
+    return qi.CONFIGS[base].with_(**kw)
+
+
+# ---------------------------------------------------------------- weight quantization
+
+@pytest.mark.parametrize("N,K,group,bits,wdt", [
+    (256, 256, 64, 4, "f32"), (200, 384, 64, 4, "bf16"), (1536, 1536, 128, 4, "bf16"),
+    (300, 256, 128, 3, "bf16"), (256, 320, 64, 3, "f32"), (8960, 1536, 128, 4, "bf16"),
+])
+def test_weight_quantization_bit_exact(N, K, group, bits, wdt):
+    cfg = _cfg(group=group, w_bits=bits, a_bits=8 if bits == 4 else 16, x_dtype=wdt)
+    inp = qi.layer_inputs(cfg, qi.Projection("w", K, N), T=4)
+    codes, scales, w_mean, colmax = oracle.quantize_weights(inp["W"], inp["s"], group, bits)
+    desc = qe.make_desc(K, N, group, bits, cfg.a_bits, 8, 4, 4)
+    Wd = cuda(inp["W"])
+    wp = torch.empty(qe.packed_weight_bytes(desc), dtype=torch.uint8, device="cuda")
+    ws = torch.empty((K // group, N), dtype=torch.float32, device="cuda")
+    wm = torch.empty(K, dtype=torch.float32, device="cuda")
+    wc = torch.empty(K, dtype=torch.float32, device="cuda")
+    qe.quantize_weights(desc, Wd, cuda(inp["s"]), wp, ws, wm, wc)
+    got = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    qe.unpack_weights(desc, wp, got)
+    torch.cuda.synchronize()
+    assert (got.cpu().numpy() == codes).all()
+    assert (ws.cpu().numpy().T == scales).all()
+    assert (wc.cpu().numpy() == colmax).all()
+    np.testing.assert_allclose(wm.cpu().numpy(), w_mean, rtol=2e-7, atol=0)
+    # padding rows of the last block hold zero codes (checked through the raw bytes)
+    if N % 128:
+        nb = (K + 127) // 128
+        blk = 8192 if bits == 4 else 6144
+        raw = wp.cpu().numpy().reshape(-1, nb, blk)[-1]
+        rowb = blk // 128
+        pad = raw[:, (N % 128) * rowb:]
+        expect = 0 if bits == 4 else None
+        if bits == 4:
+            assert (pad == expect).all()
+
+
+# ---------------------------------------------------------------- activations, router, buckets
+
+@pytest.mark.parametrize("T,K,bits,xdt", [(1, 256, 8, "f32"), (3, 384, 6, "bf16"), (64, 256, 8, "f32"),
+                                          (129, 1536, 6, "bf16"), (64, 8960, 6, "bf16")])
+def test_activation_quantization_bit_exact(T, K, bits, xdt):
+    cfg = _cfg(x_dtype=xdt, spec="qwen2b" if K >= 1024 else "tiny")
+    inp = qi.layer_inputs(cfg, qi.Projection("x", K, 128), T=T)
+    X = inp["X"]
+    if T > 2:
+        X = X.clone() if isinstance(X, torch.Tensor) else X.copy()
+        X[1] = 0  # all-zero token: zero scale and codes
+    q_ref, sa_ref = oracle.act_quant(X, inp["s_inv"], bits)
+    codes = torch.empty((T, K), dtype=torch.int8, device="cuda")
+    sa = torch.empty(T, dtype=torch.float32, device="cuda")
+    qe.act_quant(cuda(X), cuda(inp["s_inv"]), bits, codes, sa)
+    torch.cuda.synchronize()
+    assert (sa.cpu().numpy() == sa_ref).all()
+    assert (codes.cpu().numpy() == q_ref).all()
+
+
+@pytest.mark.parametrize("T,K,Nr,xdt", [(1, 256, 4, "f32"), (64, 256, 4, "f32"), (300, 1536, 8, "bf16"),
+                                        (2048, 1536, 8, "bf16"), (77, 512, 16, "bf16"), (40, 256, 3, "f32"),
+                                        (33, 256, 1, "bf16")])
+def test_router_and_buckets(T, K, Nr, xdt):
+    cfg = _cfg(x_dtype=xdt, n_routed=Nr, spec="qwen2b" if K >= 1024 else "tiny")
+    inp = qi.layer_inputs(cfg, qi.Projection("x", K, 128), T=T)
+    L_ref, e_ref = oracle.route(inp["X"], inp["G"])
+    expert = torch.empty(T, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(Nr + 1, dtype=torch.int32, device="cuda")
+    logits = torch.empty((T, Nr), dtype=torch.float32, device="cuda")
+    qe.route(cuda(inp["X"]), cuda(inp["G"]), expert, perm, offsets, logits)
+    torch.cuda.synchronize()
+    e = expert.cpu().numpy()
+    check_routing(inp["X"], inp["G"], e, e_ref)
+    np.testing.assert_allclose(logits.cpu().numpy(), L_ref, rtol=1e-4, atol=1e-4 * np.abs(L_ref).max())
+    # buckets are exactly the stable counting sort of the GPU's own choices
+    p_ref, o_ref = oracle.bucket(e, Nr)
+    assert (perm.cpu().numpy() == p_ref).all()
+    assert (offsets.cpu().numpy() == o_ref).all()
+
+
+def test_router_exact_ties_take_lowest_expert():
+    cfg = _cfg()
+    inp = qi.layer_inputs(cfg, qi.Projection("x", 256, 128), T=50)
+    G = inp["G"].clone()
+    G[:, 2] = G[:, 0]  # experts 0 and 2 tie exactly on every token
+    G[:, 3] = G[:, 0]
+    expert = torch.empty(50, dtype=torch.int32, device="cuda")
+    perm = torch.empty(50, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(5, dtype=torch.int32, device="cuda")
+    qe.route(cuda(inp["X"]), cuda(G), expert, perm, offsets)
+    torch.cuda.synchronize()
+    e = expert.cpu().numpy()
+    assert not np.isin(e, [2, 3]).any()
+
+
+# ---------------------------------------------------------------- Top-k importance
+
+@pytest.mark.parametrize("T,K,k,xdt", [(1, 256, 1, "f32"), (64, 256, 8, "f32"), (100, 1536, 32, "bf16"),
+                                       (37, 8960, 64, "bf16"), (5, 512, 128, "bf16"), (9, 29568, 32, "bf16")])
+def test_topk_bit_exact(T, K, k, xdt):
+    cfg = _cfg(x_dtype=xdt, spec="qwen2b" if K >= 1024 else "tiny")
+    inp = qi.layer_inputs(cfg, qi.Projection("x", K, 128), T=T)
+    X = f32(inp["X"]).copy()
+    if T > 3:
+        X[2] = 0.0              # all-zero token: ties everywhere, lowest channels win
+        X[3, : K // 2] = 1.0    # many exact ties
+    _, _, w_mean, _ = oracle.quantize_weights(inp["W"], inp["s"], 64, 4)
+    w_mean = w_mean.copy()
+    w_mean[:8] = w_mean[8]      # equal weights -> equal scores on equal |x|
+    Xs = X if xdt == "f32" else qi.to_bf16(X)
+    idx_ref, hist_ref = oracle.topk(Xs, w_mean, k)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    hist = torch.full((K,), 7, dtype=torch.int32, device="cuda")
+    qe.topk_importance(cuda(Xs), cuda(w_mean), k, idx, hist)
+    torch.cuda.synchronize()
+    assert (idx.cpu().numpy() == idx_ref).all()
+    assert (hist.cpu().numpy() == hist_ref).all()
+    # accumulate mode adds a second pass on top
+    qe.topk_importance(cuda(Xs), cuda(w_mean), k, idx, hist, accumulate=True)
+    torch.cuda.synchronize()
+    assert (hist.cpu().numpy() == 2 * hist_ref).all()
+
+
+def test_topk_full_size_sampled_rows():
+    # 72B-shaped statistic: all 8192 tokens at d = 29568 on the GPU; the oracle checks a
+    # seeded sample of rows, and sum(hist) = T*k, hist == bincount(idx) hold for the whole run.
+    cfg = qi.CONFIGS["qwen2vl72b"]
+    K, T, k = 29568, 8192, 32
+    X = qi.to_bf16(qi.outlier_activations(T, K, 777, cfg.outlier_spec(K)))
+    w_mean = np.abs(qi.gaussian(K, 0.02, 778)).astype(np.float32)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    hist = torch.empty(K, dtype=torch.int32, device="cuda")
+    qe.topk_importance(cuda(X), cuda(w_mean), k, idx, hist)
+    torch.cuda.synchronize()
+    idx_c = idx.cpu().numpy()
+    h = hist.cpu().numpy()
+    assert h.sum() == T * k
+    assert (h == np.bincount(idx_c.ravel(), minlength=K)).all()
+    rows = np.random.default_rng(5).choice(T, 48, replace=False)
+    idx_ref, _ = oracle.topk(X[rows], w_mean, k)
+    assert (idx_c[rows] == idx_ref).all()
+
+
+# ---------------------------------------------------------------- the forward
+
+def _forward_check(case: Case, with_acc=True):
+    Y, acc, expert, perm, sa = case.gpu_debug(with_acc)
+    inp = case.inp
+    _, e_ref = oracle.route(inp["X"], inp["G"])
+    e = expert.cpu().numpy()
+    check_routing(inp["X"], inp["G"], e, e_ref)
+    xq_ref, sa_ref = oracle.act_quant(inp["X"], inp["s_inv"], case.cfg.a_bits) if case.cfg.a_bits != 16 else (None, None)
+    if sa_ref is not None:
+        assert (sa.cpu().numpy() == sa_ref).all()
+    p_ref, _ = oracle.bucket(e, case.cfg.n_routed)
+    assert (perm.cpu().numpy() == p_ref).all()
+    if with_acc:
+        codes, _, _, _ = case.oracle_weights()
+        acc_ref = oracle.group_acc(xq_ref, codes, case.cfg.group)
+        assert (acc.cpu().numpy().astype(np.int64) == acc_ref).all()
+    Y_ref, _ = case.oracle_forward(expert_override=e)
+    err = rel_err(Y.cpu().numpy(), Y_ref)
+    assert err <= Y_TOL, err
+    return Y, Y_ref
+
+
+def test_forward_tiny_layer():
+    cfg = qi.CONFIGS["tiny"]
+    _forward_check(Case(cfg, cfg.projections[0], cfg.T))
+
+
+def test_forward_tiny_layer_with_svd_experts():
+    # adapters built the pages' way (whitened SVD of E = W - W_q) on a calibration draw
+    from oracle import fixtures
+    cfg = qi.CONFIGS["tiny"]
+    proj = cfg.projections[0]
+    inp = qi.layer_inputs(cfg, proj, T=cfg.T)
+    calib = qi.layer_inputs(cfg, proj, T=512, proj_index=9)
+    codes, scales, _, _ = oracle.quantize_weights(inp["W"], inp["s"], cfg.group, cfg.w_bits)
+    _, ec = oracle.route(calib["X"], inp["G"])
+    A_s, B_s, A_r, B_r = fixtures.qe_adapters(inp["W"], codes, scales, inp["s"], cfg.group, calib["X"], ec,
+                                             cfg.rank_shared, cfg.n_routed, cfg.rank_routed)
+    for name, v in (("A_s", A_s), ("B_s", B_s), ("A_r", A_r), ("B_r", B_r)):
+        inp[name] = qi.to_bf16(v)
+    Y, Y_ref = _forward_check(Case(cfg, proj, cfg.T, inp=inp))
+    # and the compensated layer is closer to the full-precision product than RTN alone
+    X = np.asarray(inp["X"], np.float64)
+    Yfp = X @ np.asarray(inp["W"], np.float64).T
+    z = np.zeros_like
+    Yq, _ = oracle.qe_forward(inp["X"], codes, scales, inp["s_inv"], z(A_s), z(B_s), z(A_r), z(B_r), inp["G"],
+                              cfg.group, cfg.a_bits)
+    assert ((Y.cpu().numpy() - Yfp) ** 2).sum() < ((Yq - Yfp) ** 2).sum()
+
+
+SHAPES = [
+    # T, K, N, group, a_bits, r_s, N_r, r_r, x dtype
+    (1, 256, 256, 64, 8, 8, 4, 4, "f32"),
+    (3, 384, 200, 64, 8, 8, 4, 4, "bf16"),
+    (16, 1024, 512, 128, 8, 32, 8, 4, "bf16"),
+    (17, 256, 136, 128, 6, 32, 8, 4, "bf16"),
+    (40, 512, 256, 128, 6, 32, 8, 4, "bf16"),
+    (129, 512, 384, 128, 6, 32, 8, 4, "bf16"),
+    (300, 256, 256, 64, 8, 0, 2, 16, "f32"),
+    (257, 1024, 640, 128, 8, 32, 8, 32, "bf16"),
+    (64, 256, 128, 128, 8, 0, 1, 0, "bf16"),
+    (520, 640, 1152, 128, 6, 32, 8, 4, "bf16"),
+]
+
+
+@pytest.mark.parametrize("T,K,N,group,a_bits,rs,nr,rr,xdt", SHAPES)
+def test_forward_shapes(T, K, N, group, a_bits, rs, nr, rr, xdt):
+    cfg = _cfg(group=group, a_bits=a_bits, rank_shared=rs, n_routed=nr, rank_routed=rr, x_dtype=xdt,
+               spec="qwen2b" if K >= 1024 else "tiny")
+    _forward_check(Case(cfg, qi.Projection("p", K, N), T))
+
+
+@pytest.mark.parametrize("T,K,N,group,bits,rs,nr,rr", [
+    (1, 256, 200, 64, 3, 8, 4, 4), (5, 384, 256, 128, 3, 32, 8, 4), (16, 256, 384, 128, 4, 32, 8, 4),
+    (33, 512, 136, 64, 3, 0, 2, 8), (4, 1024, 640, 128, 3, 32, 8, 32),
+])
+def test_forward_weight_only(T, K, N, group, bits, rs, nr, rr):
+    cfg = _cfg(group=group, w_bits=bits, a_bits=16, rank_shared=rs, n_routed=nr, rank_routed=rr, x_dtype="bf16")
+    _forward_check(Case(cfg, qi.Projection("p", K, N), T), with_acc=False)
+
+
+def test_forward_bf16_output_is_rounded_fp32_output():
+    cfg = _cfg(a_bits=6, x_dtype="bf16", group=128, rank_shared=32, n_routed=8)
+    c = Case(cfg, qi.Projection("p", 512, 384), 70)
+    y32 = c.gpu_forward(torch.float32)
+    y16 = c.gpu_forward(torch.bfloat16)
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
+def test_forward_deterministic_and_token_independent():
+    cfg = _cfg(a_bits=8, x_dtype="bf16", group=128, rank_shared=32, n_routed=8)
+    c = Case(cfg, qi.Projection("p", 512, 384), 200)
+    y1 = c.gpu_forward()
+    y2 = c.gpu_forward()
+    assert torch.equal(y1, y2)
+    p = torch.randperm(200, generator=torch.Generator().manual_seed(3))
+    Yp = c.layer.forward(c.Xd[p.cuda()].contiguous(), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(Yp, y1[p.cuda()])
+
+
+def test_forward_empty_batch_is_noop():
+    cfg = _cfg()
+    c = Case(cfg, cfg.projections[0], 4)
+    X0 = torch.empty((0, 256), dtype=torch.float32, device="cuda")
+    Y0 = c.layer.forward(X0, out_dtype=torch.float32)
+    assert Y0.shape == (0, 256)
+
+
+# ---------------------------------------------------------------- full-size layers, sampled rows
+
+def _full_size(cfg_name, proj_index, n_rows=48):
+    cfg = qi.CONFIGS[cfg_name]
+    proj = cfg.projections[proj_index]
+    c = Case(cfg, proj, cfg.T, proj_index=proj_index)
+    Y, _, expert, _, _ = c.gpu_debug(with_acc=False)
+    e = expert.cpu().numpy()
+    rows = np.random.default_rng(proj_index).choice(cfg.T, min(n_rows, cfg.T), replace=False).astype(np.int32)
+    _, e_ref = oracle.route(f32(c.inp["X"])[rows], c.inp["G"])
+    check_routing(f32(c.inp["X"])[rows], c.inp["G"], e[rows], e_ref)
+    Y_ref, _ = c.oracle_forward(rows=rows, expert_override=e[rows])
+    err = rel_err(Y.cpu().numpy()[rows], Y_ref)
+    assert err <= Y_TOL, err
+    # the whole output is finite and the integer stages are consistent
+    assert torch.isfinite(Y).all()
+    codes, scales, _, _ = c.oracle_weights()
+    got = torch.empty((proj.d_out, proj.d_in), dtype=torch.int8, device="cuda")
+    qe.unpack_weights(c.desc, c.layer.w_packed, got)
+    torch.cuda.synchronize()
+    assert (got.cpu().numpy() == codes).all()
+
+
+@pytest.mark.parametrize("proj_index", range(5))
+def test_full_size_qwen2vl2b_layer_set(proj_index):
+    _full_size("qwen2vl2b", proj_index)
+
+
+@pytest.mark.parametrize("cfg_name", ["decode72b_w4a8", "decode72b_w3a16"])
+@pytest.mark.parametrize("T", [1, 4, 16])
+@pytest.mark.parametrize("proj_index", [0, 2])
+def test_full_size_decode(cfg_name, T, proj_index):
+    cfg = qi.CONFIGS[cfg_name].with_(T=T)
+    proj = cfg.projections[proj_index]
+    c = Case(cfg, proj, T, proj_index=proj_index)
+    Y, _, expert, _, _ = c.gpu_debug(with_acc=False)
+    e = expert.cpu().numpy()
+    _, e_ref = oracle.route(c.inp["X"], c.inp["G"])
+    check_routing(c.inp["X"], c.inp["G"], e, e_ref)
+    Y_ref, _ = c.oracle_forward(expert_override=e)
+    err = rel_err(Y.cpu().numpy(), Y_ref)
+    assert err <= Y_TOL, err
