@@ -209,6 +209,21 @@ def run_reference(args, workload):
 
 # ---------------------------------------------------------------- our arm
 
+def replica_x_seed(rank: int, proj_index: int) -> int:
+    """Seed of replica `rank`'s token batch for one projection (rank 0 uses the config's own seed)."""
+    return 1000 + 7919 * rank + proj_index
+
+
+def max_over_ranks(value: float, pg, device=None) -> float:
+    """The slowest rank's time: every rank contributes its own, all receive the max."""
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
 def build_layers(cfg, T, rank, dev):
     import torch
     import quantized_gemm_moe_b200 as qe
@@ -218,7 +233,7 @@ def build_layers(cfg, T, rank, dev):
         if rank:
             # each replica gets its own token batch (same weights)
             spec = cfg.outlier_spec(proj.d_in)
-            x = qi.outlier_activations(T, proj.d_in, 1000 + 7919 * rank + pi, spec)
+            x = qi.outlier_activations(T, proj.d_in, replica_x_seed(rank, pi), spec)
             inp["X"] = qi.to_bf16(x) if cfg.x_dtype == "bf16" else x
         desc = qe.make_desc(proj.d_in, proj.d_out, cfg.group, cfg.w_bits, cfg.a_bits, cfg.rank_shared, cfg.n_routed,
                             cfg.rank_routed)
@@ -305,11 +320,7 @@ def run_ours(args, workload):
             for k in range(len(stages)):
                 stage_ms[s_i, p_i, k] = e[k].elapsed_time(e[k + 1])
     step_ms = stage_ms.sum(axis=(1, 2))
-    total_ms = float(step_ms.sum())
-    if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(step_ms.sum()), pg, dev)
     ms_per_step = total_ms / args.steps
     value = world * T * args.steps / (total_ms / 1e3)
 
@@ -377,10 +388,7 @@ def run_ours(args, workload):
             e1.synchronize()
             if it >= args.warmup:
                 e_ms += e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, pg, dev)
         e2e = {"value": world * T * args.steps / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
 

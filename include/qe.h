@@ -150,6 +150,9 @@ QE_API qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, q
  *   G   (device) bf16 [d_in][N_r]      (router: logits = X.G)
  *   out (device) qe_adapter_packed_bytes(desc) bytes
  * A_s/B_s may be NULL when r_s = 0, and A_r/B_r may be NULL when r_r = 0.
+ * The up-projections are kept as fp16 inside the packed buffer. Their magnitude
+ * must stay below 65504: a larger value is saturated and reported through
+ * qe_device_error (code 0x201).
  */
 QE_API qe_status qe_pack_adapters(const qe_layer_desc* desc, const void* A_s, const void* B_s, const void* A_r,
                            const void* B_r, const void* G, void* out, void* stream);

@@ -17,9 +17,10 @@
 //   sum (|sum| < 2^22) onto it, so the value reads as the float
 //   1.5*2^23 + sum, and one fp32 subtraction recovers the sum exactly.
 //   After the last group, the stage ring carries the adapter operands:
-//   B_catT (shared ++ routed up-projections) as A, and U_cat (the bucket-ordered,
-//   expert-masked down-projections) as B. A bf16 MMA puts them into a TMEM
-//   buffer that the epilogue adds.
+//   B_catT (shared ++ routed up-projections, fp16) as A, and U_cat (the
+//   bucket-ordered, expert-masked down-projections, fp16 with a per-token
+//   power-of-two scale su) as B. An fp16 MMA puts them into a TMEM buffer,
+//   and the epilogue adds it times su.
 //
 // k_ugemm: the adapter down-projection U = X . [A_s | A_r[0..N_r)] as a split-K
 //   bf16 tcgen05 GEMM (M = 128 tokens, N = adapter columns) with fp32 partials.
@@ -57,7 +58,7 @@ struct QCfg {
   static constexpr int kCPT = BN / 2;              // columns per epilogue thread
   static constexpr int kChunk = (kCPT >= 32) ? 32 : kCPT;
   static constexpr size_t kSmem = 1024 /*align slack*/ + size_t(kStages) * kStage + 1024 /*barriers etc*/ +
-                                  size_t(BN) * 8 /*sa + perm*/;
+                                  size_t(BN) * 12 /*sa + su + perm*/;
 };
 
 template <int N>
@@ -92,7 +93,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* done = acce + 2;        // [1] teardown
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   float* sa_s = reinterpret_cast<float*>(smem + NS * C::kStage + 512);
-  int32_t* perm_s = reinterpret_cast<int32_t*>(sa_s + BN);
+  float* su_s = sa_s + BN;
+  int32_t* perm_s = reinterpret_cast<int32_t*>(su_s + BN);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nt = blockIdx.x, o0 = nt * kTileN, p0 = blockIdx.y * BN, split = blockIdx.z;
@@ -140,6 +142,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int c = et; c < BN; c += 256) {
       const int p = p0 + c;
       sa_s[c] = (p < a.T) ? a.sa_sorted[p] : 0.0f;
+      su_s[c] = (p < a.T && a.su_sorted) ? a.su_sorted[p] : 0.0f;
       perm_s[c] = (p < a.T) ? a.perm[p] : -1;
     }
     const int q = warp & 3, h = (warp - 4) >> 2;
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(384, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
     if (lane == 0) {
       const uint32_t id_i8 = idesc_i8(128, BN);
-      const uint32_t id_bf = idesc_bf16(128, BN);
+      const uint32_t id_ad = idesc_f16(128, BN);
       int gidx = 0;
       bool ok = true;
       for (int it = 0; it < n_iters && ok; ++it) {
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           const uint32_t d = tmem + b * BN;
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16(d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), id_bf,
+            mma_f16(d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), id_ad,
                     (at > 0 || kk > 0) ? 1u : 0u);
           if (at == n_ad - 1) {
             tc_commit(&accf[b]);
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(384, 1)
           tmem_wait_ld();
           reg_fence(v);
 #pragma unroll
-          for (int i = 0; i < C::kChunk; ++i) acc[c + i] += __uint_as_float(v[i]);
+          for (int i = 0; i < C::kChunk; ++i) acc[c + i] = fmaf(su_s[h * C::kCPT + c + i], __uint_as_float(v[i]), acc[c + i]);
         }
       }
     }

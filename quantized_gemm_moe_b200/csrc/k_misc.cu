@@ -1,6 +1,7 @@
 // Weight-only (W3A16 / W4A16) product on CUDA cores, and the token-aware
 // Top-k importance statistic with its channel histogram.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 
@@ -23,7 +24,8 @@ __device__ __forceinline__ uint16_t f2bf(float v) {
 template <int TT, int BITS>
 __global__ void __launch_bounds__(128) k_wonly(const uint16_t* __restrict__ act16, const uint8_t* __restrict__ wp,
                                                const float* __restrict__ w_scale, const uint16_t* __restrict__ ucat,
-                                               const uint16_t* __restrict__ bcat, int R_pad, int has_adapters,
+                                               const float* __restrict__ su, const uint16_t* __restrict__ bcat,
+                                               int R_pad, int has_adapters,
                                                const int32_t* __restrict__ perm, int T, int N, int K, int group,
                                                int kb_per_split, void* __restrict__ Y, int y_bf16,
                                                float* __restrict__ partial) {
@@ -85,15 +87,22 @@ __global__ void __launch_bounds__(128) k_wonly(const uint16_t* __restrict__ act1
   }
   if (o >= N) return;
   if (has_adapters && split == 0) {
-    const uint16_t* brow = bcat + static_cast<size_t>(o) * R_pad;
+    const __half* brow = reinterpret_cast<const __half*>(bcat) + static_cast<size_t>(o) * R_pad;
+    const __half* uc = reinterpret_cast<const __half*>(ucat);
+    float ad[TT];
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) ad[tt] = 0.0f;
     for (int c = 0; c < R_pad; ++c) {
-      const float b = bf16_bits_to_f32(__ldg(brow + c));
+      const float b = __half2float(brow[c]);
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt) {
         const int p = p0 + tt;
-        if (p < T) acc[tt] = fmaf(bf16_bits_to_f32(__ldg(ucat + static_cast<size_t>(p) * R_pad + c)), b, acc[tt]);
+        if (p < T) ad[tt] = fmaf(__half2float(uc[static_cast<size_t>(p) * R_pad + c]), b, ad[tt]);
       }
     }
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt)
+      if (p0 + tt < T) acc[tt] = fmaf(su[p0 + tt], ad[tt], acc[tt]);
   }
 #pragma unroll
   for (int tt = 0; tt < TT; ++tt) {
@@ -111,7 +120,7 @@ __global__ void __launch_bounds__(128) k_wonly(const uint16_t* __restrict__ act1
 
 template <int TT>
 cudaError_t launch_wonly_t(const uint16_t* act16, const uint8_t* wp, const float* w_scale, int w_bits,
-                           const uint16_t* ucat, const uint16_t* bcat, int R_pad, int has_adapters,
+                           const uint16_t* ucat, const float* su, const uint16_t* bcat, int R_pad, int has_adapters,
                            const int32_t* perm, int T, int N, int K, int group, void* Y, int y_bf16,
                            float* partial, int splits, cudaStream_t st) {
   const int KB = static_cast<int>(ceil_div(K, kTileK));
@@ -120,10 +129,10 @@ cudaError_t launch_wonly_t(const uint16_t* act16, const uint8_t* wp, const float
             static_cast<unsigned>(splits));
   float* part = splits > 1 ? partial : nullptr;
   if (w_bits == 4)
-    k_wonly<TT, 4><<<grid, 128, 0, st>>>(act16, wp, w_scale, ucat, bcat, R_pad, has_adapters, perm, T, N, K, group,
+    k_wonly<TT, 4><<<grid, 128, 0, st>>>(act16, wp, w_scale, ucat, su, bcat, R_pad, has_adapters, perm, T, N, K, group,
                                          kbps, Y, y_bf16, part);
   else
-    k_wonly<TT, 3><<<grid, 128, 0, st>>>(act16, wp, w_scale, ucat, bcat, R_pad, has_adapters, perm, T, N, K, group,
+    k_wonly<TT, 3><<<grid, 128, 0, st>>>(act16, wp, w_scale, ucat, su, bcat, R_pad, has_adapters, perm, T, N, K, group,
                                          kbps, Y, y_bf16, part);
   return cudaGetLastError();
 }
@@ -308,12 +317,12 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const void* __restrict__ 
 }  // namespace
 
 cudaError_t launch_wonly(const uint16_t* act16, const uint8_t* w_packed, const float* w_scale, int w_bits,
-                         const uint16_t* ucat, const uint16_t* bcat, int R_pad, int has_adapters,
+                         const uint16_t* ucat, const float* su, const uint16_t* bcat, int R_pad, int has_adapters,
                          const int32_t* perm, int T, int N, int K, int group, void* Y, int y_bf16, float* partial,
                          int splits, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
 #define QE_WO(TT) \
-  launch_wonly_t<TT>(act16, w_packed, w_scale, w_bits, ucat, bcat, R_pad, has_adapters, perm, T, N, K, group, Y, \
+  launch_wonly_t<TT>(act16, w_packed, w_scale, w_bits, ucat, su, bcat, R_pad, has_adapters, perm, T, N, K, group, Y, \
                      y_bf16, partial, splits, st)
   if (T <= 1) return QE_WO(1);
   if (T <= 2) return QE_WO(2);

@@ -2,6 +2,7 @@
 // stable token->expert bucket sort, per-token quantization, weight
 // quantization / packing, adapter packing, adapter finalize, split-K reduce.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "qe_internal.h"
 
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(256) k_act_quant(const void* __restrict__ X, c
                                                    int T, int K, int qmax, const float* __restrict__ sa_tok,
                                                    const int32_t* __restrict__ pos, int8_t* __restrict__ codes,
                                                    float* __restrict__ sa_sorted, uint16_t* __restrict__ act16,
-                                                   uint16_t* __restrict__ xb16) {
+                                                   uint16_t* __restrict__ xb16, uint16_t* __restrict__ xlo16) {
   const int t = blockIdx.x;
   const size_t p = pos ? static_cast<size_t>(pos[t]) : static_cast<size_t>(t);
   const float sa = sa_tok ? sa_tok[t] : 0.0f;
@@ -241,12 +242,19 @@ __global__ void __launch_bounds__(256) k_act_quant(const void* __restrict__ X, c
       *reinterpret_cast<uint4*>(act16 + p * K + k0) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (xb16) {
-      uint32_t w[4];
+      // fp32 inputs feed the bf16 adapter GEMM as x = hi + lo, both bf16 (hi + lo carries 16 significant bits)
+      uint32_t w[4], wl[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        w[i] = static_cast<uint32_t>(f32_to_bf16_bits(xv[2 * i])) |
-               (static_cast<uint32_t>(f32_to_bf16_bits(xv[2 * i + 1])) << 16);
+      for (int i = 0; i < 4; ++i) {
+        const uint16_t h0 = f32_to_bf16_bits(xv[2 * i]), h1 = f32_to_bf16_bits(xv[2 * i + 1]);
+        w[i] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+        const uint16_t l0 = f32_to_bf16_bits(xv[2 * i] - bf16_bits_to_f32(h0));
+        const uint16_t l1 = f32_to_bf16_bits(xv[2 * i + 1] - bf16_bits_to_f32(h1));
+        wl[i] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+      }
       *reinterpret_cast<uint4*>(xb16 + static_cast<size_t>(t) * K + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+      if (xlo16)
+        *reinterpret_cast<uint4*>(xlo16 + static_cast<size_t>(t) * K + k0) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
     }
   }
   if (codes && sa_sorted && threadIdx.x == 0) sa_sorted[p] = sa;
@@ -383,11 +391,13 @@ __global__ void __launch_bounds__(128) k_unpack_w(const uint8_t* __restrict__ pa
 }
 
 // Adapter packing: A_catT [R_pad][K], B_catT [N][R_pad], G copy [K][n_r], all bf16.
+// The up-projections B_catT are stored as fp16 (the epilogue MMA multiplies them with the
+// fp16 U_cat). A bf16 value beyond the fp16 range is saturated and reported (DEVERR_RANGE).
 __global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a, int R_pad,
                                 const uint16_t* __restrict__ A_s, const uint16_t* __restrict__ B_s,
                                 const uint16_t* __restrict__ A_r, const uint16_t* __restrict__ B_r,
                                 const uint16_t* __restrict__ G, uint16_t* __restrict__ acat,
-                                uint16_t* __restrict__ bcat, uint16_t* __restrict__ gout) {
+                                uint16_t* __restrict__ bcat, uint16_t* __restrict__ gout, int* __restrict__ err) {
   const size_t n1 = static_cast<size_t>(R_pad) * K, n2 = static_cast<size_t>(N) * R_pad,
                n3 = static_cast<size_t>(K) * n_r;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n1 + n2 + n3;
@@ -410,7 +420,13 @@ __global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a
         const int e = (c - r_s) / r_r, j = (c - r_s) % r_r;
         v = B_r[(static_cast<size_t>(e) * r_r + j) * N + o];
       }
-      bcat[ii] = v;
+      float f = bf16_bits_to_f32(v);
+      if (fabsf(f) > 65504.0f) {
+        f = copysignf(65504.0f, f);
+        if (err) atomicCAS(err, 0, 0x201);
+      }
+      __half hv = __float2half_rn(f);
+      bcat[ii] = *reinterpret_cast<uint16_t*>(&hv);
     } else {
       const size_t ii = i - n1 - n2;
       gout[ii] = G[ii];
@@ -418,37 +434,50 @@ __global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a
   }
 }
 
-// U_cat[p][c] = bf16(sum_s P[s][t][c]) with t = perm[p]; routed columns of other experts -> 0.
-__global__ void k_ufinal(const float* __restrict__ partial, int splits, const int32_t* __restrict__ perm,
+// U_cat[p][c] = fp16((sum over partial slots of P[slot][t][c]) / su[p]) with t = perm[p].
+// Routed columns of the other experts are 0. One warp per bucket position. su[p] is a power
+// of two that puts the row's largest |U| in [2^13, 2^14), so fp16 keeps full range and
+// 11-bit precision relative to the row; the epilogue multiplies the adapter term back by su.
+__global__ void k_ufinal(const float* __restrict__ partial, int nslots, const int32_t* __restrict__ perm,
                          const int32_t* __restrict__ expert, int T, int R_pad, int r_s, int r_r, int R_a,
-                         uint16_t* __restrict__ ucat) {
-  const int chunks = R_pad / 8;
-  const size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
-  if (idx >= static_cast<size_t>(T) * chunks) return;
-  const int p = static_cast<int>(idx / chunks), c0 = static_cast<int>(idx % chunks) * 8;
+                         uint16_t* __restrict__ ucat, float* __restrict__ su_sorted) {
+  const int warp = static_cast<int>((blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const int p = warp;
   const int t = perm[p];
   const int e = expert[t];
-  float v[8];
+  constexpr int kMaxPerLane = 512 / 32;
+  float v[kMaxPerLane];
+  float mx = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-  for (int s = 0; s < splits; ++s) {
-    const float* src = partial + (static_cast<size_t>(s) * T + t) * R_pad + c0;
-    const float4 a = __ldg(reinterpret_cast<const float4*>(src));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
-    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
-  }
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int c = c0 + i;
-    bool keep = c < R_a && (c < r_s || (c - r_s) / r_r == e);
-    if (!keep) v[i] = 0.0f;
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int c = lane + 32 * i;
+    float a = 0.0f;
+    if (c < R_pad && c < R_a && (c < r_s || (c - r_s) / r_r == e)) {
+      for (int s2 = 0; s2 < nslots; ++s2) a += __ldg(partial + (static_cast<size_t>(s2) * T + t) * R_pad + c);
+    }
+    v[i] = a;
+    mx = fmaxf(mx, fabsf(a));
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    w[i] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i])) | (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i + 1])) << 16);
-  *reinterpret_cast<uint4*>(ucat + static_cast<size_t>(p) * R_pad + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float su = 1.0f;
+  if (mx > 0.0f) {
+    int ex;
+    frexpf(mx, &ex);  // mx = m * 2^ex, m in [0.5, 1)
+    su = ldexpf(1.0f, ex - 14);
+  }
+  const float inv = 1.0f / su;  // exact: su is a power of two
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int c = lane + 32 * i;
+    if (c < R_pad) {
+      __half h = __float2half_rn(v[i] * inv);
+      ucat[static_cast<size_t>(p) * R_pad + c] = *reinterpret_cast<uint16_t*>(&h);
+    }
+  }
+  if (lane == 0) su_sorted[p] = su;
 }
 
 // Y[perm[p]][o] = sum_s partial[s][p][o] (fixed order).
@@ -492,12 +521,12 @@ cudaError_t launch_bucket(const int32_t* expert, int T, int n_r, int32_t* perm, 
 
 cudaError_t launch_act_quant(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
                              const float* sa_tok, const int32_t* pos, int8_t* codes, float* sa_sorted,
-                             uint16_t* act16, uint16_t* xb16, cudaStream_t st) {
+                             uint16_t* act16, uint16_t* xb16, uint16_t* xlo16, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   if (x_bf16)
-    k_act_quant<true><<<T, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16);
+    k_act_quant<true><<<T, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16, xlo16);
   else
-    k_act_quant<false><<<T, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16);
+    k_act_quant<false><<<T, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16, xlo16);
   return cudaGetLastError();
 }
 
@@ -531,21 +560,20 @@ cudaError_t launch_unpack_weights(const uint8_t* packed, int N, int K, int w_bit
 }
 
 cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint16_t* A_s, const uint16_t* B_s,
-                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out,
+                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out, int* err,
                                  cudaStream_t st) {
   k_pack_adapters<<<592, 256, 0, st>>>(K, N, g.r_s, g.n_r, g.r_r, g.R_a, g.R_pad, A_s, B_s, A_r, B_r, G,
                                        reinterpret_cast<uint16_t*>(out + g.off_acat),
                                        reinterpret_cast<uint16_t*>(out + g.off_bcat),
-                                       reinterpret_cast<uint16_t*>(out + g.off_g));
+                                       reinterpret_cast<uint16_t*>(out + g.off_g), err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_ufinal(const float* partial, int splits, const int32_t* perm, const int32_t* expert, int T,
-                          int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, cudaStream_t st) {
-  const size_t n = static_cast<size_t>(T) * (R_pad / 8);
-  if (n == 0) return cudaSuccess;
-  k_ufinal<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, st>>>(partial, splits, perm, expert, T, R_pad, r_s,
-                                                                    r_r > 0 ? r_r : 1, R_a, ucat);
+cudaError_t launch_ufinal(const float* partial, int nslots, const int32_t* perm, const int32_t* expert, int T,
+                          int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, float* su_sorted, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  k_ufinal<<<static_cast<unsigned>(ceil_div(T, 8)), 256, 0, st>>>(partial, nslots, perm, expert, T, R_pad, r_s,
+                                                                  r_r > 0 ? r_r : 1, R_a, ucat, su_sorted);
   return cudaGetLastError();
 }
 

@@ -63,8 +63,9 @@ struct Plan {
   AdapterGeom g;
   UgemmPlan up;
   int bn, msplits, kbps;  // main product
-  size_t off_expert, off_perm, off_pos, off_offsets, off_sa_tok, off_sa_sorted, off_act, off_xb16, off_upart,
-      off_ucat, off_ypart, bytes;
+  int uslots;             // U partial slots: splits, doubled for fp32 inputs (hi and lo passes)
+  size_t off_expert, off_perm, off_pos, off_offsets, off_sa_tok, off_sa_sorted, off_su_sorted, off_act, off_xb16,
+      off_xlo16, off_upart, off_ucat, off_ypart, bytes;
 };
 
 int wonly_splits(int T, int N, int K) {
@@ -105,9 +106,12 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   p.off_offsets = take(size_t(kMaxRouted + 1) * 4);
   p.off_sa_tok = take(size_t(Tm) * 4);
   p.off_sa_sorted = take(size_t(Tm) * 4);
+  p.off_su_sorted = take(size_t(Tm) * 4);
   p.off_act = take(size_t(Tm) * p.K * (d->a_bits == 16 ? 2 : 1));
   p.off_xb16 = (!x_bf16 && p.has_ad) ? take(size_t(Tm) * p.K * 2) : 0;
-  p.off_upart = p.has_ad ? take(size_t(p.up.splits) * Tm * p.g.R_pad * 4) : 0;
+  p.off_xlo16 = (!x_bf16 && p.has_ad) ? take(size_t(Tm) * p.K * 2) : 0;
+  p.uslots = p.up.splits * (x_bf16 ? 1 : 2);
+  p.off_upart = p.has_ad ? take(size_t(p.uslots) * Tm * p.g.R_pad * 4) : 0;
   p.off_ucat = p.has_ad ? take(size_t(Tm) * p.g.R_pad * 2) : 0;
   p.off_ypart = (p.msplits > 1) ? take(size_t(p.msplits) * Tm * p.N * 4) : 0;
   p.bytes = o;
@@ -184,6 +188,7 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   int32_t* offsets = at<int32_t>(ws, p.off_offsets);
   float* sa_tok = at<float>(ws, p.off_sa_tok);
   float* sa_sorted = at<float>(ws, p.off_sa_sorted);
+  float* su_sorted = at<float>(ws, p.off_su_sorted);
   const bool wonly = d->a_bits == 16;
   const int qmax = wonly ? 1 : qmax_of(d->a_bits);
   const int K = p.K, N = p.N;
@@ -199,8 +204,10 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   int8_t* codes = wonly ? nullptr : at<int8_t>(ws, p.off_act);
   uint16_t* act16 = wonly ? at<uint16_t>(ws, p.off_act) : nullptr;
   uint16_t* xb16 = (!x_bf16 && p.has_ad) ? at<uint16_t>(ws, p.off_xb16) : nullptr;
+  uint16_t* xlo16 = (!x_bf16 && p.has_ad) ? at<uint16_t>(ws, p.off_xlo16) : nullptr;
   if (stages & QE_STAGE_QUANT)
-    QE_CUDA(launch_act_quant(X, x_bf16, w->s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16, st),
+    QE_CUDA(launch_act_quant(X, x_bf16, w->s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16, xlo16,
+                             st),
             "act_quant");
   // 4. adapter down-projection (tensor cores) -> U_cat in bucket order
   uint16_t* ucat = p.has_ad ? at<uint16_t>(ws, p.off_ucat) : nullptr;
@@ -213,8 +220,16 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
       return s;
     float* upart = at<float>(ws, p.off_upart);
     QE_CUDA(launch_ugemm(tm_x, tm_acat, p.up, T, K, p.g.R_pad, upart, err, st), "ugemm");
-    QE_CUDA(launch_ufinal(upart, p.up.splits, perm, expert, T, p.g.R_pad, d->rank_shared, d->rank_routed, p.g.R_a,
-                          ucat, st),
+    if (!x_bf16) {  // fp32 input: second pass over the low bf16 part into the next partial slots
+      CUtensorMap tm_xlo;
+      if ((s = make_tmap(&tm_xlo, xlo16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK)
+        return s;
+      QE_CUDA(launch_ugemm(tm_xlo, tm_acat, p.up, T, K, p.g.R_pad,
+                           upart + size_t(p.up.splits) * T * p.g.R_pad, err, st),
+              "ugemm_lo");
+    }
+    QE_CUDA(launch_ufinal(upart, p.uslots, perm, expert, T, p.g.R_pad, d->rank_shared, d->rank_routed, p.g.R_a, ucat,
+                          su_sorted, st),
             "ufinal");
   }
   // 5. main product
@@ -222,17 +237,17 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   float* ypart = p.msplits > 1 ? at<float>(ws, p.off_ypart) : nullptr;
   const int y_bf16 = yd == QE_BF16;
   if (wonly) {
-    QE_CUDA(launch_wonly(act16, static_cast<const uint8_t*>(w->w_packed), w->w_scale, d->w_bits, ucat, bcat,
+    QE_CUDA(launch_wonly(act16, static_cast<const uint8_t*>(w->w_packed), w->w_scale, d->w_bits, ucat, su_sorted, bcat,
                          p.g.R_pad, p.has_ad ? 1 : 0, perm, T, N, K, d->group, Y, y_bf16, ypart, p.msplits, st),
             "wonly");
   } else {
     CUtensorMap tm_xq, tm_bcat, tm_ucat;
     if ((s = make_tmap(&tm_xq, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, T, kTileK, p.bn)) != QE_OK) return s;
     if (p.has_ad) {
-      if ((s = make_tmap(&tm_bcat, bcat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.g.R_pad, N, kAdapterAtom, kTileN)) !=
+      if ((s = make_tmap(&tm_bcat, bcat, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.g.R_pad, N, kAdapterAtom, kTileN)) !=
           QE_OK)
         return s;
-      if ((s = make_tmap(&tm_ucat, ucat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.g.R_pad, T, kAdapterAtom, p.bn)) !=
+      if ((s = make_tmap(&tm_ucat, ucat, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.g.R_pad, T, kAdapterAtom, p.bn)) !=
           QE_OK)
         return s;
     } else {
@@ -243,6 +258,7 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
     a.w_packed = static_cast<const uint8_t*>(w->w_packed);
     a.w_scale = w->w_scale;
     a.sa_sorted = sa_sorted;
+    a.su_sorted = p.has_ad ? su_sorted : nullptr;
     a.perm = perm;
     a.T = T;
     a.N = N;
@@ -319,7 +335,7 @@ qe_status qe_pack_adapters(const qe_layer_desc* desc, const void* A_s, const voi
   QE_CUDA(launch_pack_adapters(g, desc->d_in, desc->d_out, static_cast<const uint16_t*>(A_s),
                                static_cast<const uint16_t*>(B_s), static_cast<const uint16_t*>(A_r),
                                static_cast<const uint16_t*>(B_r), static_cast<const uint16_t*>(G),
-                               static_cast<uint8_t*>(out), static_cast<cudaStream_t>(stream)),
+                               static_cast<uint8_t*>(out), device_error_ptr(), static_cast<cudaStream_t>(stream)),
           "pack_adapters");
   return QE_OK;
 }
@@ -365,7 +381,7 @@ int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, qe_dtype
   if (T == 0) return 0;
   const Plan p = make_plan(desc, T, x_dtype == QE_BF16);
   int n = 3;                    // route_stats, bucket, act_quant
-  if (p.has_ad) n += 2;         // ugemm, ufinal
+  if (p.has_ad) n += (x_dtype == QE_BF16) ? 2 : 3;  // ugemm (twice for fp32 inputs), ufinal
   n += 1;                       // qgemm or the weight-only product
   if (p.msplits > 1) n += 1;    // split-K reduce
   return n;
@@ -411,7 +427,7 @@ qe_status qe_act_quant(const void* X, qe_dtype x_dtype, const float* s_inv, int3
   QE_CUDA(launch_route_stats(X, x_dtype == QE_BF16, s_inv, nullptr, T, d_in, 0, qmax, nullptr, sa, nullptr, cs),
           "act_stats");
   QE_CUDA(launch_act_quant(X, x_dtype == QE_BF16, s_inv, T, d_in, qmax, sa, nullptr, codes, nullptr, nullptr,
-                           nullptr, cs),
+                           nullptr, nullptr, cs),
           "act_quant");
   return QE_OK;
 }

@@ -49,7 +49,7 @@ cudaError_t launch_colstats(const void* W, bool w_bf16, int N, int K, float* w_m
 cudaError_t launch_unpack_weights(const uint8_t* packed, int N, int K, int w_bits, int8_t* codes,
                                   cudaStream_t st);
 cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint16_t* A_s, const uint16_t* B_s,
-                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out,
+                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out, int* err,
                                  cudaStream_t st);
 
 // Router logits + argmin, and (when sa != nullptr) the per-token absmax -> scale.
@@ -61,10 +61,11 @@ cudaError_t launch_bucket(const int32_t* expert, int T, int n_r, int32_t* perm, 
 // Per-token quantization of x*s_inv with the scale sa_tok[t], written at row pos[t] (pos == nullptr: row t).
 //   codes != nullptr: int8 codes, sa_sorted[pos] = sa_tok[t]
 //   act16 != nullptr: bf16(x*s_inv) (weight-only layers)
-//   xb16  != nullptr: bf16(x) in token order (for fp32 inputs feeding the adapter GEMM)
+//   xb16  != nullptr: hi = bf16(x) in token order (fp32 inputs feeding the adapter GEMM)
+//   xlo16 != nullptr: lo = bf16(x - hi), so that hi + lo carries 16 significant bits of x
 cudaError_t launch_act_quant(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
                              const float* sa_tok, const int32_t* pos, int8_t* codes, float* sa_sorted,
-                             uint16_t* act16, uint16_t* xb16, cudaStream_t st);
+                             uint16_t* act16, uint16_t* xb16, uint16_t* xlo16, cudaStream_t st);
 
 // Adapter down-projection partials: P[split][t][c] = sum_{k in split} X[t][k] * A_catT[c][k] (tcgen05, bf16).
 struct UgemmPlan {
@@ -76,9 +77,10 @@ struct UgemmPlan {
 UgemmPlan plan_ugemm(int T, int K, int R_pad);
 cudaError_t launch_ugemm(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, const UgemmPlan& plan, int T,
                          int K, int R_pad, float* partial, int* err, cudaStream_t st);
-// U_cat[p][c] = bf16(sum_s P[s][perm[p]][c]), routed columns masked to the token's expert.
-cudaError_t launch_ufinal(const float* partial, int splits, const int32_t* perm, const int32_t* expert, int T,
-                          int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, cudaStream_t st);
+// U_cat[p][c] = fp16(sum over partial slots of P[slot][perm[p]][c] / su[p]), routed columns masked to the
+// token's expert, su[p] a per-position power of two.
+cudaError_t launch_ufinal(const float* partial, int nslots, const int32_t* perm, const int32_t* expert, int T,
+                          int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, float* su_sorted, cudaStream_t st);
 
 // Main quantized GEMM (W4 x A8/A6 codes, tcgen05 kind::i8) with per-group promotion,
 // per-token scale, adapter MMA in the epilogue and scatter to token order.
@@ -86,6 +88,7 @@ struct QgemmArgs {
   const uint8_t* w_packed;
   const float* w_scale;     // [G][N]
   const float* sa_sorted;   // [T]
+  const float* su_sorted;   // [T] adapter scale of U_cat rows
   const int32_t* perm;      // [T]
   int T, N, K, group;
   int KB;                   // ceil(K / 128)
@@ -105,7 +108,7 @@ cudaError_t launch_splitk_reduce(const float* partial, int splits, const int32_t
 
 // Weight-only (W3A16 / W4A16) product on CUDA cores, token chunks of up to 16.
 cudaError_t launch_wonly(const uint16_t* act16, const uint8_t* w_packed, const float* w_scale, int w_bits,
-                         const uint16_t* ucat, const uint16_t* bcat, int R_pad, int has_adapters,
+                         const uint16_t* ucat, const float* su_sorted, const uint16_t* bcat, int R_pad, int has_adapters,
                          const int32_t* perm, int T, int N, int K, int group, void* Y, int y_bf16, float* partial,
                          int splits, cudaStream_t st);
 
