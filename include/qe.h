@@ -228,6 +228,37 @@ QE_API qe_status qe_linear_forward_stages(const qe_layer_desc* desc, const qe_la
 /* Number of kernels one qe_linear_forward launches for this layer and T (-1 on an invalid desc). */
 QE_API int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype);
 
+/*
+ * qe_linear_forward without a caller-provided workspace. (No counterpart in
+ * the paper: this is a deployment convenience of this library.)
+ *
+ * Some host programs cannot allocate device memory for the layer. Examples:
+ * a plugin whose host framework owns all device memory and exposes no
+ * allocator to it, or a process that must not grow its device footprint
+ * after start-up. For them, this entry point uses a fixed scratch array that
+ * lives in the library's own device memory. It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * Limits and behaviour:
+ * - The scratch is QE_NOALLOC_WORKSPACE_BYTES (32 MiB) on every GPU that
+ *   loads the library, held until the process exits.
+ * - A layer, T and input dtype whose scratch need exceeds that size are
+ *   rejected with QE_ERR_WORKSPACE; qe_last_cuda_error() says how much was
+ *   needed. qe_linear_workspace_bytes is an upper bound on the need. fp32
+ *   inputs need two extra bf16 copies of X. For example, every Qwen2VL-2B
+ *   projection fits at T = 2048 with bf16 inputs.
+ * - The first call on a device looks up the array's device address for that
+ *   device (once per device). Make that first call before any stream capture.
+ * - All calls share the one array and it keeps the last call's contents.
+ *   Calls whose kernels overlap on the GPU (different streams, or
+ *   different host threads, without ordering) race on it. Order them.
+ * - Arguments, outputs and errors are as for qe_linear_forward.
+ */
+#define QE_NOALLOC_WORKSPACE_BYTES (32u << 20)
+QE_API qe_status qe_linear_forward_noalloc(const qe_layer_desc* desc, const qe_layer_weights* weights,
+                                           const void* X, qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype,
+                                           void* stream);
+
 /* ---------------------------------------------------------------- status */
 
 QE_API const char* qe_status_string(qe_status s);

@@ -23,8 +23,10 @@ EXPORTS = (
     "qe_packed_weight_bytes", "qe_adapter_packed_bytes", "qe_linear_workspace_bytes", "qe_quantize_weights",
     "qe_pack_adapters", "qe_topk_importance", "qe_route", "qe_linear_forward", "qe_status_string",
     "qe_last_cuda_error", "qe_device_error", "qe_unpack_weights", "qe_act_quant", "qe_linear_forward_debug",
-    "qe_linear_forward_stages", "qe_linear_kernel_launches",
+    "qe_linear_forward_stages", "qe_linear_kernel_launches", "qe_linear_forward_noalloc",
 )
+# fixed scratch of qe_linear_forward_noalloc (bytes), as declared in include/qe.h
+NOALLOC_WORKSPACE_BYTES = 32 << 20
 QE_STAGE_ROUTE, QE_STAGE_QUANT, QE_STAGE_ADAPTERS, QE_STAGE_PRODUCT, QE_STAGE_ALL = 1, 2, 4, 8, 15
 
 
@@ -78,6 +80,7 @@ def load() -> ctypes.CDLL:
         "qe_linear_forward_debug": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P, S, P, P, P, P, P], I),
         "qe_linear_forward_stages": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P, S, I, P], I),
         "qe_linear_kernel_launches": ([D, I, I], I),
+        "qe_linear_forward_noalloc": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P], I),
         "qe_status_string": ([I], ctypes.c_char_p),
         "qe_last_cuda_error": ([], ctypes.c_char_p),
         "qe_device_error": ([P, ctypes.POINTER(I), I], I),
@@ -190,6 +193,18 @@ def linear_forward_stages(desc, weights: LayerWeights, X, Y, workspace, stages: 
                                            _ptr(Y), _dtype(Y), _ptr(workspace),
                                            workspace.numel() * workspace.element_size(), stages, _stream(stream)),
            "qe_linear_forward_stages")
+
+
+def linear_forward_noalloc(desc, weights: LayerWeights, X, Y, stream=None):
+    """qe_linear_forward using the library's fixed device scratch instead of a workspace.
+
+    For callers that cannot allocate device memory. The scratch is shared by all
+    calls; calls that overlap on the GPU race on it.
+    """
+    _need_cuda(X, Y)
+    _check(load().qe_linear_forward_noalloc(ctypes.byref(desc), ctypes.byref(weights), _ptr(X), _dtype(X),
+                                            X.shape[0], _ptr(Y), _dtype(Y), _stream(stream)),
+           "qe_linear_forward_noalloc")
 
 
 def linear_forward_debug(desc, weights, X, Y, workspace, acc=None, expert=None, perm=None, sa=None, stream=None):

@@ -282,6 +282,35 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   return QE_OK;
 }
 
+// ------------------------------------------------------------------ no-allocation variant
+// Scratch for qe_linear_forward_noalloc: a fixed array in the library's own
+// device memory, so that caller needs to provide no workspace. It exists on
+// every GPU that loads this module and stays until the process exits. All
+// calls share it; it keeps the last call's contents (the forward overwrites
+// every byte it reads before reading it, so nothing needs clearing).
+static __device__ __align__(256) uint8_t g_static_scratch[QE_NOALLOC_WORKSPACE_BYTES];
+
+// Device address of g_static_scratch for the current device, looked up once per device.
+// Host code must not use the array's name as an address: on the host it is only a
+// stand-in symbol, not device memory.
+qe_status static_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return QE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return QE_OK;
+}
+
 }  // namespace
 }  // namespace qe
 
@@ -430,6 +459,25 @@ qe_status qe_act_quant(const void* X, qe_dtype x_dtype, const float* s_inv, int3
                            nullptr, nullptr, cs),
           "act_quant");
   return QE_OK;
+}
+
+qe_status qe_linear_forward_noalloc(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
+                                    qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* stream) {
+  qe_status s = check_desc(desc);
+  if (s != QE_OK) return s;
+  if (T < 0) return QE_ERR_INVALID_ARG;
+  if (T == 0) return QE_OK;
+  const size_t need = make_plan(desc, T, x_dtype == QE_BF16).bytes;  // the scratch this input dtype needs
+  if (need > QE_NOALLOC_WORKSPACE_BYTES) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+             "qe_linear_forward_noalloc: this layer needs %zu bytes of scratch for T=%d, above the fixed %u",
+             need, T, static_cast<unsigned>(QE_NOALLOC_WORKSPACE_BYTES));
+    return QE_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if ((s = static_scratch(&scratch)) != QE_OK) return s;
+  return forward_impl(desc, weights, X, x_dtype, T, Y, y_dtype, scratch, QE_NOALLOC_WORKSPACE_BYTES, nullptr,
+                      nullptr, nullptr, nullptr, QE_STAGE_ALL, static_cast<cudaStream_t>(stream));
 }
 
 const char* qe_status_string(qe_status s) {
