@@ -8,10 +8,15 @@
 //                 plus one bulk copy of the 8 KB packed-int4 weight block
 //     warps 2-3   unpack the int4 block into int8 in the 128B-swizzled A layout
 //     warp 1      one elected thread issues tcgen05.mma kind::i8, one TMEM
-//                 accumulator buffer per quantization group (double-buffered)
+//                 accumulator buffer per quantization group (2 buffers at BN=256,
+//                 4 below, so the MMA runs ahead of the epilogue)
 //     warps 4-11  epilogue: the per-group promotion acc += sw[o,j] * float(int32)
-//                 in registers, then * sa[t], + adapter MMA result, and a
-//                 scatter of the row to token order
+//                 in registers (f32x2, the next TMEM chunk loading meanwhile),
+//                 then * sa[t], + adapter MMA result, and a scatter of the row
+//                 to token order
+//   The kernel is persistent: one CTA per SM walks a static list of
+//   (output tile, token tile, K split) units, so barriers and TMEM are set up
+//   once and the next unit's loads and MMAs overlap the last unit's stores.
 //   Integer -> float without a convert instruction: every TMEM accumulator
 //   starts at the bit pattern of 1.5*2^23. The int32 MMA adds the exact group
 //   sum (|sum| < 2^22) onto it, so the value reads as the float
@@ -49,16 +54,25 @@ __device__ __forceinline__ uint16_t f2bf(float v) {
 
 template <int BN>
 struct QCfg {
-  static constexpr int kA = 16384;                 // 128 rows x 128 B (int8 K=128 or bf16 K=64)
+  static constexpr int kA = 16384;                 // 128 rows x 128 B (int8 K=128 or fp16 K=64)
   static constexpr int kB = BN * 128;
   static constexpr int kWP = kW4BlockBytes;         // packed int4 block
   static constexpr int kStage = kA + kB + kWP;
   static constexpr int kStages = (BN >= 256) ? 3 : (BN >= 128 ? 4 : (BN >= 64 ? 5 : 6));
-  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : 2 * BN;  // power of two for BN in {16..256}
+  static constexpr int kNBuf = (BN >= 256) ? 2 : 4;  // TMEM accumulator buffers
+  static constexpr int kTmemCols = (kNBuf * BN <= 32) ? 32 : kNBuf * BN;  // power of two for BN in {16..256}
   static constexpr int kCPT = BN / 2;              // columns per epilogue thread
-  static constexpr int kChunk = (kCPT >= 32) ? 32 : kCPT;
-  static constexpr size_t kSmem = 1024 /*align slack*/ + size_t(kStages) * kStage + 1024 /*barriers etc*/ +
+  static constexpr int kChunk = (kCPT >= 128) ? 16 : ((kCPT >= 32) ? 32 : kCPT);
+  static constexpr int kNChunk = kCPT / kChunk;
+  static constexpr int kOut = 32768;               // output staging (two 16 KB halves, one per epilogue warpgroup)
+  static constexpr size_t kSmem = 1024 /*align slack*/ + size_t(kStages) * kStage + kOut + 1024 /*barriers etc*/ +
                                   size_t(BN) * 12 /*sa + su + perm*/;
+  // setmaxnreg split of the 512 x 128 launch registers: the producer/MMA warpgroup and the
+  // unpack warpgroup drop to kRegLow, the two epilogue warpgroups rise to kRegHigh
+  // (256 * kRegLow + 256 * kRegHigh = 65536); the values were picked per tile width by spill counts.
+  static constexpr int kRegLow = (BN >= 128) ? 72 : 56;
+  static constexpr int kRegHigh = (65536 - 256 * kRegLow) / 256;
+  static_assert(256 * kRegLow + 256 * kRegHigh == 65536 && kRegLow % 8 == 0 && kRegHigh % 8 == 0, "register split");
 };
 
 template <int N>
@@ -74,56 +88,154 @@ __device__ __forceinline__ void tmem_fill(uint32_t taddr, uint32_t x) {
   else tmem_fill8(taddr, x);
 }
 
+// acc[i..i+1] += sw * (float(v[i..i+1]) - 1.5*2^23), two lanes per instruction (f32x2).
+// The subtraction is exact (both operands lie in [2^23, 2^24)); the FMA rounds once.
+__device__ __forceinline__ void promote2(float& a0, float& a1, uint32_t v0, uint32_t v1, uint64_t sw2,
+                                         uint64_t magic2) {
+  uint64_t x, acc;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(v0), "r"(v1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(acc) : "f"(a0), "f"(a1));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(x) : "l"(x), "l"(magic2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(acc) : "l"(x), "l"(sw2), "l"(acc));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+}
+
+__device__ __forceinline__ uint64_t pack2(float x) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
+  return r;
+}
+
+// One unit of work: a 128-row output tile, a BN-position token tile and a K split.
+struct Unit {
+  int nt, p0, split, kb_begin, nkb, n_ad, g_begin, n_groups;
+};
+
+__device__ __forceinline__ Unit make_unit(const QgemmArgs& a, int BN, int u) {
+  Unit w;
+  const int NT = static_cast<int>(ceil_div(a.N, kTileN));
+  const int PT = static_cast<int>(ceil_div(a.T, BN));
+  w.nt = u % NT;
+  const int rest = u / NT;
+  w.p0 = (rest % PT) * BN;
+  w.split = rest / PT;
+  w.kb_begin = w.split * a.kb_per_split;
+  const int kb_end = min(a.KB, w.kb_begin + a.kb_per_split);
+  w.nkb = max(0, kb_end - w.kb_begin);
+  w.n_ad = (w.split == 0) ? a.adapter_atoms : 0;
+  const int gpb = kTileK / a.group;
+  const int G_total = a.K / a.group;
+  w.g_begin = w.kb_begin * gpb;
+  w.n_groups = max(0, min(G_total, kb_end * gpb) - w.g_begin);
+  return w;
+}
+
+
+// Writes one epilogue warpgroup's half tile (128 output channels x CPT token columns) to Y.
+// Each pass moves PC columns: every thread puts its values for those columns into the
+// warpgroup's 16 KB staging buffer (column-major by token), then the 128 threads copy
+// whole row segments (128 channels = 256 B bf16 / 512 B fp32) to Y[token] with 16-byte
+// stores. Rows go to perm[p] (token order), or to position p of this split's partial
+// buffer. Every thread runs every pass and barrier, whatever `ok` is.
+template <int CPT, int ELEM>
+__device__ __forceinline__ void store_tile(const float (&acc)[CPT], uint8_t* stage, const int32_t* perm_cols,
+                                           const Unit& w, const QgemmArgs& a, int o0, int o_local, int wt, int h,
+                                           bool ok, bool to_partial) {
+  constexpr int kRowBytes = 128 * ELEM;
+  constexpr int kPC = (16384 / kRowBytes) < CPT ? (16384 / kRowBytes) : CPT;  // columns per pass
+  constexpr int kChunksPerRow = kRowBytes / 16;
+  constexpr int kElemsPerChunk = 16 / ELEM;
+  const bool vec_ok = ((static_cast<size_t>(a.N) * ELEM) % 16) == 0;
+#pragma unroll
+  for (int pass = 0; pass < CPT / kPC; ++pass) {
+#pragma unroll
+    for (int c = 0; c < kPC; ++c) {
+      const float v = acc[pass * kPC + c];
+      if constexpr (ELEM == 2) {
+        *reinterpret_cast<uint16_t*>(stage + c * kRowBytes + o_local * 2) = f2bf(v);
+      } else {
+        *reinterpret_cast<float*>(stage + c * kRowBytes + o_local * 4) = v;
+      }
+    }
+    asm volatile("bar.sync %0, 128;" ::"r"(2 + h) : "memory");
+    if (ok) {
+#pragma unroll
+      for (int k = 0; k < (kPC * kChunksPerRow) / 128; ++k) {
+        const int ch = wt + 128 * k;
+        const int c = ch / kChunksPerRow, part = ch % kChunksPerRow;
+        const int col = pass * kPC + c;  // column inside this warpgroup's half
+        const int p = w.p0 + h * CPT + col;
+        const int row = to_partial ? (p < a.T ? p : -1) : perm_cols[col];
+        if (row < 0) continue;
+        const int of = o0 + part * kElemsPerChunk;
+        if (of >= a.N) continue;
+        uint8_t* dst_base = to_partial
+                                ? reinterpret_cast<uint8_t*>(a.partial + (static_cast<size_t>(w.split) * a.T + row) * a.N)
+                                : static_cast<uint8_t*>(a.Y) + static_cast<size_t>(row) * a.N * ELEM;
+        const uint8_t* src = stage + c * kRowBytes + part * 16;
+        if (vec_ok && of + kElemsPerChunk <= a.N) {
+          *reinterpret_cast<uint4*>(dst_base + static_cast<size_t>(of) * ELEM) = *reinterpret_cast<const uint4*>(src);
+        } else {
+          for (int e = 0; e < kElemsPerChunk && of + e < a.N; ++e) {
+            if constexpr (ELEM == 2)
+              *reinterpret_cast<uint16_t*>(dst_base + static_cast<size_t>(of + e) * 2) =
+                  *reinterpret_cast<const uint16_t*>(src + e * 2);
+            else
+              *reinterpret_cast<float*>(dst_base + static_cast<size_t>(of + e) * 4) =
+                  *reinterpret_cast<const float*>(src + e * 4);
+          }
+        }
+      }
+    }
+    asm volatile("bar.sync %0, 128;" ::"r"(2 + h) : "memory");
+  }
+}
+
 template <int BN, bool DBG>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     k_qgemm(const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_bcat,
             const __grid_constant__ CUtensorMap tm_ucat, const QgemmArgs a) {
   using C = QCfg<BN>;
   constexpr int NS = C::kStages;
+  constexpr int NB = C::kNBuf;
   int* const a_err = a.err;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NS * C::kStage);
+  uint8_t* out_stage = smem + NS * C::kStage;  // [2][16 KB] output transpose buffers
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + C::kOut);
   uint64_t* full = bars;            // [NS] TMA bytes landed
-  uint64_t* afull = bars + NS;      // [NS] unpack done (2 warp arrivals)
+  uint64_t* afull = bars + NS;      // [NS] unpack done (4 warp arrivals)
   uint64_t* empty = bars + 2 * NS;  // [NS] MMAs done reading the stage
-  uint64_t* accf = bars + 3 * NS;   // [2] accumulator buffer ready for the epilogue
-  uint64_t* acce = accf + 2;        // [2] accumulator buffer drained (8 warp arrivals)
-  uint64_t* done = acce + 2;        // [1] teardown
+  uint64_t* accf = bars + 3 * NS;   // [NB] accumulator buffer ready for the epilogue
+  uint64_t* acce = accf + NB;       // [NB] accumulator buffer drained and re-biased (8 warp arrivals)
+  uint64_t* done = acce + NB;       // [1] teardown
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  float* sa_s = reinterpret_cast<float*>(smem + NS * C::kStage + 512);
+  float* sa_s = reinterpret_cast<float*>(out_stage + C::kOut + 512);
   float* su_s = sa_s + BN;
   int32_t* perm_s = reinterpret_cast<int32_t*>(su_s + BN);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = blockIdx.x, o0 = nt * kTileN, p0 = blockIdx.y * BN, split = blockIdx.z;
-  const int kb_begin = split * a.kb_per_split;
-  const int kb_end = min(a.KB, kb_begin + a.kb_per_split);
-  const int nkb = max(0, kb_end - kb_begin);
-  const int n_ad = (split == 0) ? a.adapter_atoms : 0;
-  const int n_iters = nkb + n_ad;
+  const int NT = static_cast<int>(ceil_div(a.N, kTileN));
+  const int PT = static_cast<int>(ceil_div(a.T, BN));
+  const int n_units = NT * PT * a.splits;
   const int gpb = kTileK / a.group;  // groups per 128-channel block
   const int G_total = a.K / a.group;
-  // groups handled by this split
-  const int g_begin = kb_begin * gpb;
-  const int g_end = min(G_total, kb_end * gpb);
-  const int n_groups = max(0, g_end - g_begin);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&afull[s], 2);
+      mbar_init(&afull[s], 4);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&accf[b], 1);
       mbar_init(&acce[b], 8);
     }
     mbar_init(done, 1);
     mbar_fence_init();
     prefetch_tmap(&tm_xq);
-    if (n_ad) {
+    if (a.adapter_atoms) {
       prefetch_tmap(&tm_bcat);
       prefetch_tmap(&tm_ucat);
     }
@@ -136,18 +248,11 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 4) {
-    // epilogue threads: stage sa/perm of the tile, put the magic bias in both buffers
-    const int et = threadIdx.x - 128;
-    for (int c = et; c < BN; c += 256) {
-      const int p = p0 + c;
-      sa_s[c] = (p < a.T) ? a.sa_sorted[p] : 0.0f;
-      su_s[c] = (p < a.T && a.su_sorted) ? a.su_sorted[p] : 0.0f;
-      perm_s[c] = (p < a.T) ? a.perm[p] : -1;
-    }
+  if (warp >= 4 && warp < 12) {
+    // epilogue threads put the magic bias into every accumulator buffer once
     const int q = warp & 3, h = (warp - 4) >> 2;
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < NB; ++b)
 #pragma unroll
       for (int c = 0; c < C::kCPT; c += C::kChunk)
         tmem_fill<C::kChunk>(tmem + (static_cast<uint32_t>(32 * q) << 16) + b * BN + h * C::kCPT + c, kMagicBits);
@@ -155,213 +260,274 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_before();
   }
   __syncthreads();
-  // Register split (launch: 384 x 168 = 64512): the producer/MMA/unpack
-  // warpgroup gives back to 56, and the two epilogue warpgroups take 224 each
-  // (128*56 + 256*224 = 64512). Each role sets its own limit at its entry.
+
+  // Roles: warp 0 TMA producer, warp 1 MMA issuer (warps 2-3 idle), warps 4-11 epilogue,
+  // warps 12-15 unpack. Register split: 256 * kRegLow + 256 * kRegHigh = 512 x 128 launch
+  // registers; each role sets its own limit at its entry.
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegLow) : "memory");
     if (lane == 0) {
-      for (int it = 0; it < n_iters; ++it) {
-        const int s = it % NS;
-        if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) break;
-        uint8_t* sa_ = stage_base + s * C::kStage;
-        uint8_t* sb_ = sa_ + C::kA;
-        uint8_t* swp = sb_ + C::kB;
-        if (it < nkb) {
-          const int kb = kb_begin + it;
-          mbar_arrive_expect_tx(&full[s], C::kB + C::kWP);
-          tma_load_2d(sb_, &tm_xq, kb * kTileK, p0, &full[s]);
-          bulk_load(swp, a.w_packed + (static_cast<size_t>(nt) * a.KB + kb) * kW4BlockBytes, C::kWP, &full[s]);
-        } else {
-          const int at = it - nkb;
-          mbar_arrive_expect_tx(&full[s], C::kA + C::kB);
-          tma_load_2d(sa_, &tm_bcat, at * kAdapterAtom, o0, &full[s]);
-          tma_load_2d(sb_, &tm_ucat, at * kAdapterAtom, p0, &full[s]);
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const Unit w = make_unit(a, BN, u);
+        for (int i = 0; i < w.nkb + w.n_ad; ++i, ++it) {
+          const int s = it % NS;
+          if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa_ = stage_base + s * C::kStage;
+          uint8_t* sb_ = sa_ + C::kA;
+          uint8_t* swp = sb_ + C::kB;
+          if (i < w.nkb) {
+            const int kb = w.kb_begin + i;
+            mbar_arrive_expect_tx(&full[s], C::kB + C::kWP);
+            tma_load_2d(sb_, &tm_xq, kb * kTileK, w.p0, &full[s]);
+            bulk_load(swp, a.w_packed + (static_cast<size_t>(w.nt) * a.KB + kb) * kW4BlockBytes, C::kWP, &full[s]);
+          } else {
+            const int at = i - w.nkb;
+            mbar_arrive_expect_tx(&full[s], C::kA + C::kB);
+            tma_load_2d(sa_, &tm_bcat, at * kAdapterAtom, w.nt * kTileN, &full[s]);
+            tma_load_2d(sb_, &tm_ucat, at * kAdapterAtom, w.p0, &full[s]);
+          }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegLow) : "memory");
     if (lane == 0) {
       const uint32_t id_i8 = idesc_i8(128, BN);
       const uint32_t id_ad = idesc_f16(128, BN);
-      int gidx = 0;
+      int it = 0, gidx = 0;
       bool ok = true;
-      for (int it = 0; it < n_iters && ok; ++it) {
-        const int s = it % NS;
-        const uint32_t ph = (it / NS) & 1;
-        if (!mbar_wait(&full[s], ph, a_err, DEVERR_WAIT_MMA) || !mbar_wait(&afull[s], ph, a_err, DEVERR_WAIT_MMA)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(stage_base + s * C::kStage);
-        const uint32_t b_addr = a_addr + C::kA;
-        if (it < nkb) {
-          const int kb = kb_begin + it;
-          for (int gi = 0; gi < gpb; ++gi) {
-            const int gglob = kb * gpb + gi;
-            if (gglob >= g_end) break;
-            const int b = gidx & 1;
-            if (!mbar_wait(&acce[b], ((gidx >> 1) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
-              ok = false;
-              break;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const Unit w = make_unit(a, BN, u);
+        for (int i = 0; i < w.nkb + w.n_ad && ok; ++i, ++it) {
+          const int s = it % NS;
+          const uint32_t ph = (it / NS) & 1;
+          if (!mbar_wait(&full[s], ph, a_err, DEVERR_WAIT_MMA) || !mbar_wait(&afull[s], ph, a_err, DEVERR_WAIT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(stage_base + s * C::kStage);
+          const uint32_t b_addr = a_addr + C::kA;
+          if (i < w.nkb) {
+            const int kb = w.kb_begin + i;
+            for (int gi = 0; gi < gpb; ++gi) {
+              if (kb * gpb + gi >= w.g_begin + w.n_groups) break;
+              const int b = gidx % NB;
+              if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t d = tmem + b * BN;
+              for (int kk = 0; kk < a.group / 32; ++kk) {
+                const uint32_t koff = gi * a.group + kk * 32;
+                mma_i8(d, smem_desc_sw128(a_addr + koff), smem_desc_sw128(b_addr + koff), id_i8, 1u);
+              }
+              tc_commit(&accf[b]);
+              ++gidx;
             }
-            tc_fence_after();
+          } else {
+            const int at = i - w.nkb;
+            const int b = gidx % NB;
+            if (at == 0) {
+              if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
             const uint32_t d = tmem + b * BN;
-            for (int kk = 0; kk < a.group / 32; ++kk) {
-              const uint32_t koff = gi * a.group + kk * 32;
-              mma_i8(d, smem_desc_sw128(a_addr + koff), smem_desc_sw128(b_addr + koff), id_i8, 1u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16(d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), id_ad,
+                      (at > 0 || kk > 0) ? 1u : 0u);
+            if (at == w.n_ad - 1) {
+              tc_commit(&accf[b]);
+              ++gidx;
             }
-            tc_commit(&accf[b]);
-            ++gidx;
           }
-        } else {
-          const int at = it - nkb;
-          const int b = gidx & 1;
-          if (at == 0) {
-            if (!mbar_wait(&acce[b], ((gidx >> 1) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          const uint32_t d = tmem + b * BN;
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16(d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), id_ad,
-                    (at > 0 || kk > 0) ? 1u : 0u);
-          if (at == n_ad - 1) {
-            tc_commit(&accf[b]);
-            ++gidx;
-          }
+          tc_commit(&empty[s]);
         }
-        tc_commit(&empty[s]);
       }
       // make sure everything issued has completed before TMEM is released
       tc_commit(done);
       mbar_wait(done, 0, a_err, DEVERR_WAIT_TEARDOWN);
     }
   } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ int4 -> int8 unpack
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
-    const int u = threadIdx.x - 64;  // 0..63
-    for (int it = 0; it < n_iters; ++it) {
-      const int s = it % NS;
-      if (!mbar_wait(&full[s], (it / NS) & 1, a_err, DEVERR_WAIT_UNPACK)) break;
-      if (it < nkb) {
-        uint8_t* sa_ = stage_base + s * C::kStage;
-        const uint8_t* swp = sa_ + C::kA + C::kB;
-#pragma unroll 2
-        for (int i = 0; i < 8; ++i) {
-          const int piece = u + 64 * i;  // 16-byte piece of the 8 KB block
-          const int r = piece >> 2, q4 = piece & 3;
-          const uint4 v = *reinterpret_cast<const uint4*>(swp + piece * 16);
-          uint4 lo, hi;
-          lo.x = sext_nibbles(v.x & 0x0F0F0F0Fu);
-          lo.y = sext_nibbles(v.y & 0x0F0F0F0Fu);
-          lo.z = sext_nibbles(v.z & 0x0F0F0F0Fu);
-          lo.w = sext_nibbles(v.w & 0x0F0F0F0Fu);
-          hi.x = sext_nibbles((v.x >> 4) & 0x0F0F0F0Fu);
-          hi.y = sext_nibbles((v.y >> 4) & 0x0F0F0F0Fu);
-          hi.z = sext_nibbles((v.z >> 4) & 0x0F0F0F0Fu);
-          hi.w = sext_nibbles((v.w >> 4) & 0x0F0F0F0Fu);
-          const int c_lo = 2 * q4, c_hi = 2 * q4 + 1;
-          *reinterpret_cast<uint4*>(sa_ + r * 128 + ((c_lo ^ (r & 7)) << 4)) = lo;
-          *reinterpret_cast<uint4*>(sa_ + r * 128 + ((c_hi ^ (r & 7)) << 4)) = hi;
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegLow) : "memory");
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ int4 -> int8 unpack (warps 12..15)
+    // Each code goes to the high nibble of its byte, so the byte reads as the int8 16*q.
+    // The factor 16 is folded into the group scale (sw/16, exact), and |16*acc| stays below 2^22.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegLow) : "memory");
+    const int uth = threadIdx.x - 384;  // 0..127
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit w = make_unit(a, BN, u);
+      for (int i = 0; i < w.nkb + w.n_ad; ++i, ++it) {
+        const int s = it % NS;
+        if (!mbar_wait(&full[s], (it / NS) & 1, a_err, DEVERR_WAIT_UNPACK)) {
+          ok = false;
+          break;
         }
-        fence_proxy_async_smem();
+        if (i < w.nkb) {
+          uint8_t* sa_ = stage_base + s * C::kStage;
+          const uint8_t* swp = sa_ + C::kA + C::kB;
+          uint4 v[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(swp + (uth + 128 * j) * 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int piece = uth + 128 * j;  // 16-byte piece of the 8 KB block
+            const int r = piece >> 2, q4 = piece & 3;
+            uint4 lo, hi;
+            lo.x = (v[j].x << 4) & 0xF0F0F0F0u;
+            lo.y = (v[j].y << 4) & 0xF0F0F0F0u;
+            lo.z = (v[j].z << 4) & 0xF0F0F0F0u;
+            lo.w = (v[j].w << 4) & 0xF0F0F0F0u;
+            hi.x = v[j].x & 0xF0F0F0F0u;
+            hi.y = v[j].y & 0xF0F0F0F0u;
+            hi.z = v[j].z & 0xF0F0F0F0u;
+            hi.w = v[j].w & 0xF0F0F0F0u;
+            const int c_lo = 2 * q4, c_hi = 2 * q4 + 1;
+            *reinterpret_cast<uint4*>(sa_ + r * 128 + ((c_lo ^ (r & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(sa_ + r * 128 + ((c_hi ^ (r & 7)) << 4)) = hi;
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[s]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[s]);
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 4..11)
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+    // Control flow here depends only on the unit schedule, never on a wait's
+    // outcome: the named barriers below must be reached by every epilogue warp.
+    // After a wait runs out, `ok` (warp-uniform) turns every later wait and TMEM access off.
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegHigh) : "memory");
     const int q = warp & 3, h = (warp - 4) >> 2;
-    const int o = o0 + 32 * q + lane;
-    const bool o_ok = o < a.N;
+    const int et = threadIdx.x - 128;      // 0..255
+    const int wt = et & 127;               // thread index inside this epilogue warpgroup
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    asm volatile("bar.sync 1, 256;" ::: "memory");  // sa_s / perm_s staged
-    float acc[C::kCPT];
-#pragma unroll
-    for (int c = 0; c < C::kCPT; ++c) acc[c] = 0.0f;
-    bool ok = true;
+    const uint64_t magic2 = pack2(kMagic);
+    uint8_t* my_out = out_stage + h * (C::kOut / 2);
     int gidx = 0;
-    float sw_next = (o_ok && n_groups > 0) ? __ldg(a.w_scale + static_cast<size_t>(g_begin) * a.N + o) : 0.0f;
-    for (int g = 0; g < n_groups; ++g) {
-      const int b = gidx & 1;
-      const float sw = sw_next;
-      if (g + 1 < n_groups && o_ok) sw_next = __ldg(a.w_scale + static_cast<size_t>(g_begin + g + 1) * a.N + o);
-      if (!mbar_wait(&accf[b], (gidx >> 1) & 1, a_err, DEVERR_WAIT_EPILOGUE)) {
-        ok = false;
-        break;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const Unit w = make_unit(a, BN, u);
+      const int o0 = w.nt * kTileN;
+      const int o = o0 + 32 * q + lane;
+      const bool o_ok = o < a.N;
+      // stage this unit's per-position scales and token ids (after everyone finished the previous unit)
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      for (int c = et; c < BN; c += 256) {
+        const int p = w.p0 + c;
+        sa_s[c] = (p < a.T) ? a.sa_sorted[p] : 0.0f;
+        su_s[c] = (p < a.T && a.su_sorted) ? a.su_sorted[p] : 0.0f;
+        perm_s[c] = (p < a.T) ? a.perm[p] : -1;
       }
-      tc_fence_after();
-      const uint32_t base = tmem + lane_base + b * BN + h * C::kCPT;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      float acc[C::kCPT];
 #pragma unroll
-      for (int c = 0; c < C::kCPT; c += C::kChunk) {
-        uint32_t v[C::kChunk];
-        tmem_ld<C::kChunk>(base + c, v);
-        tmem_wait_ld();
-        reg_fence(v);
-        tmem_fill<C::kChunk>(base + c, kMagicBits);
-        if (DBG && o_ok) {
-#pragma unroll
-          for (int i = 0; i < C::kChunk; ++i) {
-            const int t = perm_s[h * C::kCPT + c + i];
-            if (t >= 0)
-              a.dbg_acc[(static_cast<size_t>(t) * a.N + o) * G_total + g_begin + g] =
-                  static_cast<int32_t>(v[i] - kMagicBits);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < C::kChunk; ++i) acc[c + i] = fmaf(sw, __uint_as_float(v[i]) - kMagic, acc[c + i]);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[b]);
-      ++gidx;
-    }
-    // per-token scale, adapters, store
-#pragma unroll
-    for (int c = 0; c < C::kCPT; ++c) acc[c] *= sa_s[h * C::kCPT + c];
-    if (ok && n_ad > 0) {
-      const int b = gidx & 1;
-      if (mbar_wait(&accf[b], (gidx >> 1) & 1, a_err, DEVERR_WAIT_EPILOGUE)) {
+      for (int c = 0; c < C::kCPT; ++c) acc[c] = 0.0f;
+      // weight codes enter the MMA as 16*q, so the group scale is applied as sw/16 (exact)
+      float sw_next = (o_ok && w.n_groups > 0)
+                          ? __ldg(a.w_scale + static_cast<size_t>(w.g_begin) * a.N + o) * 0.0625f
+                          : 0.0f;
+      for (int g = 0; g < w.n_groups; ++g) {
+        const int b = gidx % NB;
+        ++gidx;
+        const uint64_t sw2 = pack2(sw_next);
+        if (g + 1 < w.n_groups && o_ok)
+          sw_next = __ldg(a.w_scale + static_cast<size_t>(w.g_begin + g + 1) * a.N + o) * 0.0625f;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+        if (!ok) continue;
         tc_fence_after();
         const uint32_t base = tmem + lane_base + b * BN + h * C::kCPT;
+        // chunk c+1 loads while chunk c is promoted; each drained chunk is re-biased at once
+        uint32_t va[C::kChunk], vb[C::kChunk];
+        tmem_ld<C::kChunk>(base, va);
+        tmem_wait_ld();
+        reg_fence(va);
 #pragma unroll
-        for (int c = 0; c < C::kCPT; c += C::kChunk) {
-          uint32_t v[C::kChunk];
-          tmem_ld<C::kChunk>(base + c, v);
-          tmem_wait_ld();
-          reg_fence(v);
+        for (int c = 0; c < C::kNChunk; ++c) {
+          uint32_t(&cur)[C::kChunk] = (c & 1) ? vb : va;
+          uint32_t(&nxt)[C::kChunk] = (c & 1) ? va : vb;
+          if (c + 1 < C::kNChunk) tmem_ld<C::kChunk>(base + (c + 1) * C::kChunk, nxt);
+          tmem_fill<C::kChunk>(base + c * C::kChunk, kMagicBits);
+          if (DBG && o_ok) {
 #pragma unroll
-          for (int i = 0; i < C::kChunk; ++i) acc[c + i] = fmaf(su_s[h * C::kCPT + c + i], __uint_as_float(v[i]), acc[c + i]);
-        }
-      }
-    }
-    if (o_ok) {
-      if (a.splits == 1) {
+            for (int i = 0; i < C::kChunk; ++i) {
+              const int t = perm_s[h * C::kCPT + c * C::kChunk + i];
+              if (t >= 0)
+                a.dbg_acc[(static_cast<size_t>(t) * a.N + o) * G_total + w.g_begin + g] =
+                    static_cast<int32_t>(cur[i] - kMagicBits) / 16;
+            }
+          }
 #pragma unroll
-        for (int c = 0; c < C::kCPT; ++c) {
-          const int t = perm_s[h * C::kCPT + c];
-          if (t >= 0) {
-            const size_t dst = static_cast<size_t>(t) * a.N + o;
-            if (a.y_bf16) static_cast<uint16_t*>(a.Y)[dst] = f2bf(acc[c]);
-            else static_cast<float*>(a.Y)[dst] = acc[c];
+          for (int i = 0; i < C::kChunk; i += 2)
+            promote2(acc[c * C::kChunk + i], acc[c * C::kChunk + i + 1], cur[i], cur[i + 1], sw2, magic2);
+          if (c + 1 < C::kNChunk) {
+            tmem_wait_ld();
+            reg_fence(nxt);
           }
         }
-      } else {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[b]);
+      }
+      // per-token scale
+      const float4* sa4 = reinterpret_cast<const float4*>(sa_s + h * C::kCPT);
 #pragma unroll
-        for (int c = 0; c < C::kCPT; ++c) {
-          const int p = p0 + h * C::kCPT + c;
-          if (p < a.T) a.partial[(static_cast<size_t>(split) * a.T + p) * a.N + o] = acc[c];
+      for (int c = 0; c < C::kCPT; c += 4) {
+        const float4 f = sa4[c / 4];
+        acc[c] *= f.x;
+        acc[c + 1] *= f.y;
+        acc[c + 2] *= f.z;
+        acc[c + 3] *= f.w;
+      }
+      // adapters: acc += su[t] * (U_cat . B_cat^T)
+      if (w.n_ad > 0) {
+        const int b = gidx % NB;
+        ++gidx;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+        if (ok) {
+          tc_fence_after();
+          const uint32_t base = tmem + lane_base + b * BN + h * C::kCPT;
+          const float4* su4 = reinterpret_cast<const float4*>(su_s + h * C::kCPT);
+#pragma unroll
+          for (int c = 0; c < C::kCPT; c += C::kChunk) {
+            uint32_t v[C::kChunk];
+            tmem_ld<C::kChunk>(base + c, v);
+            tmem_wait_ld();
+            reg_fence(v);
+            tmem_fill<C::kChunk>(base + c, kMagicBits);
+#pragma unroll
+            for (int i = 0; i < C::kChunk; i += 4) {
+              const float4 f = su4[(c + i) / 4];
+              acc[c + i] = fmaf(f.x, __uint_as_float(v[i]), acc[c + i]);
+              acc[c + i + 1] = fmaf(f.y, __uint_as_float(v[i + 1]), acc[c + i + 1]);
+              acc[c + i + 2] = fmaf(f.z, __uint_as_float(v[i + 2]), acc[c + i + 2]);
+              acc[c + i + 3] = fmaf(f.w, __uint_as_float(v[i + 3]), acc[c + i + 3]);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acce[b]);
         }
       }
+      // store: transpose through shared memory, then write whole row segments with 16-byte stores
+      if (a.splits == 1 && a.y_bf16) store_tile<C::kCPT, 2>(acc, my_out, perm_s + h * C::kCPT, w, a, o0, 32 * q + lane, wt, h, ok, false);
+      else store_tile<C::kCPT, 4>(acc, my_out, perm_s + h * C::kCPT, w, a, o0, 32 * q + lane, wt, h, ok, a.splits > 1);
     }
     tc_fence_before();
   }
@@ -487,10 +653,10 @@ template <int BN, bool DBG>
 cudaError_t launch_qgemm_t(const CUtensorMap& tm_xq, const CUtensorMap& tm_bcat, const CUtensorMap& tm_ucat,
                            const QgemmArgs& a, cudaStream_t st) {
   using C = QCfg<BN>;
-  // The epilogue warpgroups raise their register limit to 224 with setmaxnreg,
-  // which waits until the producer warpgroup has released its share. That only
-  // completes when the kernel was built with 168 registers per thread
-  // (384 x 168 = 128 x 56 + 256 x 224), so refuse any other build.
+  // The epilogue warpgroups raise their register limit with setmaxnreg,
+  // which waits until the other warpgroups have released their share. That only
+  // completes when the kernel was built with 128 registers per thread
+  // (512 x 128 = 256 x kRegLow + 256 x kRegHigh), so refuse any other build.
   static int regs = -1;
   if (regs < 0) {
     cudaFuncAttributes fa;
@@ -498,13 +664,21 @@ cudaError_t launch_qgemm_t(const CUtensorMap& tm_xq, const CUtensorMap& tm_bcat,
     if (ea != cudaSuccess) return ea;
     regs = fa.numRegs;
   }
-  if (regs != 168) return cudaErrorInvalidConfiguration;
+  if (regs != 128) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(k_qgemm<BN, DBG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(ceil_div(a.N, kTileN)), static_cast<unsigned>(ceil_div(a.T, BN)),
-            static_cast<unsigned>(a.splits));
-  k_qgemm<BN, DBG><<<grid, 384, C::kSmem, st>>>(tm_xq, tm_bcat, tm_ucat, a);
+  // persistent: one CTA per SM (or per unit when there are fewer units), each loops over units
+  static int n_sm = 0;
+  if (n_sm == 0) {
+    int dev = 0;
+    cudaError_t ed = cudaGetDevice(&dev);
+    if (ed == cudaSuccess) ed = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (ed != cudaSuccess) return ed;
+  }
+  const int64_t units = ceil_div(a.N, kTileN) * ceil_div(a.T, BN) * a.splits;
+  const unsigned grid = static_cast<unsigned>(units < n_sm ? units : n_sm);
+  k_qgemm<BN, DBG><<<grid, 512, C::kSmem, st>>>(tm_xq, tm_bcat, tm_ucat, a);
   return cudaGetLastError();
 }
 
