@@ -277,7 +277,7 @@ def run_ours(args, workload):
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     wonly = cfg.a_bits == 16
-    stages = (qe.QE_STAGE_ROUTE, qe.QE_STAGE_QUANT, qe.QE_STAGE_ADAPTERS, qe.QE_STAGE_PRODUCT)
+    stages = (qe.QE_STAGE_PROJECT, qe.QE_STAGE_ROUTE, qe.QE_STAGE_QUANT, qe.QE_STAGE_PRODUCT)
 
     def step(record):
         evs = []
@@ -359,7 +359,7 @@ def run_ours(args, workload):
         tot = ms.sum()
         per_proj.append({
             "proj": L["proj"].name, "K": K, "N": N, "ms": float(tot),
-            "stage_ms": {"route": float(ms[0]), "quant": float(ms[1]), "adapters": float(ms[2]), "product": float(ms[3])},
+            "stage_ms": {"project": float(ms[0]), "route": float(ms[1]), "quant": float(ms[2]), "product": float(ms[3])},
             "product_tops": (roofline.int_ops(T, K, N) / (ms[3] / 1e3) / 1e12) if not wonly else None,
             "product_gbs": roofline.layer_bytes(T, K, N, cfg.group, cfg.w_bits, cfg.rank_shared, cfg.n_routed,
                                                 cfg.rank_routed, 1 if not wonly else 2, 2) / (ms[3] / 1e3) / 1e9,

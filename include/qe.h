@@ -198,11 +198,13 @@ QE_API qe_status qe_route(const void* X, qe_dtype x_dtype, const void* G, int32_
  *   workspace (device) scratch of at least qe_linear_workspace_bytes(desc, T)
  *             bytes. Contents on entry are ignored. Calls that share a
  *             workspace must not overlap on the GPU.
- * Steps (all on the GPU): router + per-token absmax -> stable bucket sort ->
- * per-token quantization in bucket order -> adapter down-projection
- * (tensor cores) -> int8 tcgen05 GEMM with per-group scale promotion and the
- * adapter up-projection in its epilogue -> scatter to token order. With
- * a_bits = 16 the main product is the weight-only bf16 path.
+ * Steps (all on the GPU): one tensor-core GEMM for the adapter
+ * down-projections and the router logits (with the per-token absmax) ->
+ * argmin routing and the stable bucket sort -> per-token quantization and the
+ * expert-masked adapter rows, in bucket order -> int8 tcgen05 GEMM with
+ * per-group scale promotion and the adapter up-projection in its epilogue ->
+ * scatter to token order. With a_bits = 16 the main product is the
+ * weight-only path.
  * T = 0 is a no-op.
  */
 QE_API qe_status qe_linear_forward(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
@@ -216,10 +218,10 @@ QE_API qe_status qe_linear_forward(const qe_layer_desc* desc, const qe_layer_wei
  * what qe_linear_forward computes. A stage reads what earlier stages left in
  * the workspace. Unknown bits -> QE_ERR_INVALID_ARG.
  */
-#define QE_STAGE_ROUTE 1    /* router + per-token absmax, stable bucket sort          */
-#define QE_STAGE_QUANT 2    /* per-token quantization in bucket order                 */
-#define QE_STAGE_ADAPTERS 4 /* adapter down-projection (tensor cores), expert masking  */
-#define QE_STAGE_PRODUCT 8  /* main product with the adapter epilogue, scatter to Y   */
+#define QE_STAGE_PROJECT 1 /* tensor-core GEMM: adapter down-projections + router logits, per-token absmax */
+#define QE_STAGE_ROUTE 2   /* argmin routing, per-token scale, stable bucket sort                        */
+#define QE_STAGE_QUANT 4   /* per-token quantization and the expert-masked adapter rows, bucket order   */
+#define QE_STAGE_PRODUCT 8 /* main product with the adapter epilogue, scatter to Y                      */
 #define QE_STAGE_ALL 15
 QE_API qe_status qe_linear_forward_stages(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
                                           qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,
@@ -248,7 +250,9 @@ QE_API int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, q
  *   inputs need two extra bf16 copies of X. For example, every Qwen2VL-2B
  *   projection fits at T = 2048 with bf16 inputs.
  * - The first call on a device looks up the array's device address for that
- *   device (once per device). Make that first call before any stream capture.
+ *   device, then synchronizes the device once, because loading the array
+ *   initializes it asynchronously. Make that first call before any stream
+ *   capture.
  * - All calls share the one array and it keeps the last call's contents.
  *   Calls whose kernels overlap on the GPU (different streams, or
  *   different host threads, without ordering) race on it. Order them.

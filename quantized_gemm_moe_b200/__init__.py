@@ -27,7 +27,7 @@ EXPORTS = (
 )
 # fixed scratch of qe_linear_forward_noalloc (bytes), as declared in include/qe.h
 NOALLOC_WORKSPACE_BYTES = 32 << 20
-QE_STAGE_ROUTE, QE_STAGE_QUANT, QE_STAGE_ADAPTERS, QE_STAGE_PRODUCT, QE_STAGE_ALL = 1, 2, 4, 8, 15
+QE_STAGE_PROJECT, QE_STAGE_ROUTE, QE_STAGE_QUANT, QE_STAGE_PRODUCT, QE_STAGE_ALL = 1, 2, 4, 8, 15
 
 
 class QEError(RuntimeError):

@@ -539,12 +539,14 @@ __global__ void __launch_bounds__(512, 1)
 }
 
 // ---------------------------------------------------------------------- U GEMM
-// P[split][t][c] = sum over this split's K range of X[t][k] * A_catT[c][k].
+// P[slot][t][c] = sum over this split's K range of X[t][k] * A_catT[c][k] for c in this CTA's
+// column tile: the adapter down-projections and the router logits in one bf16 tcgen05 GEMM
+// (M = 128 tokens, N = adapter + router columns, K split across CTAs, fp32 partial slots).
 // 192 threads: warp 0 TMA, warp 1 MMA (+ TMEM owner), warps 2-5 epilogue.
 template <int NU>
 struct UCfg {
   static constexpr int kA = 16384;     // 128 tokens x 64 bf16
-  static constexpr int kB = NU * 128;  // NU adapter columns x 64 bf16
+  static constexpr int kB = NU * 128;  // NU columns x 64 bf16
   static constexpr int kStage = kA + kB;
   static constexpr int kStages = 4;
   static constexpr int kTmemCols = NU <= 32 ? 32 : (NU <= 64 ? 64 : (NU <= 128 ? 128 : 256));
@@ -554,7 +556,7 @@ struct UCfg {
 template <int NU>
 __global__ void __launch_bounds__(192, 1)
     k_ugemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_acat, int T, int K,
-            int R_pad, int kchunks_per_split, float* __restrict__ partial, int* a_err) {
+            int R_tot, int kchunks_per_split, float* __restrict__ partial, int* a_err) {
   using C = UCfg<NU>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -594,8 +596,8 @@ __global__ void __launch_bounds__(192, 1)
         const int s = it % NS;
         if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) break;
         uint8_t* sa_ = smem + s * C::kStage;
-        mbar_arrive_expect_tx(&full[s], C::kStage);
         const int kx = (kc_begin + it) * kAdapterAtom;
+        mbar_arrive_expect_tx(&full[s], C::kA + C::kB);
         tma_load_2d(sa_, &tm_x, kx, m0, &full[s]);
         tma_load_2d(sa_ + C::kA, &tm_acat, kx, c0, &full[s]);
       }
@@ -617,11 +619,12 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     const int q = warp & 3;
-    const int row = m0 + 32 * q + lane;
-    const bool ok = mbar_wait(accf, 0, a_err, DEVERR_WAIT_EPILOGUE);
+    const int r = 32 * q + lane;  // tile row == TMEM lane of this thread
+    const int row = m0 + r;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, a_err, DEVERR_WAIT_EPILOGUE));
     tc_fence_after();
     if (ok) {
-      float* dst = partial + (static_cast<size_t>(split) * T + row) * R_pad + c0;
+      float* dst = partial + (static_cast<size_t>(split) * T + row) * R_tot + c0;
 #pragma unroll 1
       for (int c = 0; c < NU; c += 16) {
         uint32_t v[16];
@@ -691,14 +694,18 @@ cudaError_t launch_qgemm_bn(const CUtensorMap& tm_xq, const CUtensorMap& tm_bcat
 
 template <int NU>
 cudaError_t launch_ugemm_t(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, const UgemmPlan& p, int T, int K,
-                           int R_pad, float* partial, int* err, cudaStream_t st) {
+                           int R_tot, float* partial, int* err, cudaStream_t st) {
   using C = UCfg<NU>;
-  cudaError_t e = cudaFuncSetAttribute(k_ugemm<NU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(C::kSmem));
-  if (e != cudaSuccess) return e;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_ugemm<NU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::kSmem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   dim3 grid(static_cast<unsigned>(ceil_div(T, 128)), static_cast<unsigned>(p.ntiles),
             static_cast<unsigned>(p.splits));
-  k_ugemm<NU><<<grid, 192, C::kSmem, st>>>(tm_x, tm_acat, T, K, R_pad, p.kchunks_per_split, partial, err);
+  k_ugemm<NU><<<grid, 192, C::kSmem, st>>>(tm_x, tm_acat, T, K, R_tot, p.kchunks_per_split, partial, err);
   return cudaGetLastError();
 }
 
@@ -742,30 +749,31 @@ cudaError_t launch_qgemm(int BN, const CUtensorMap& tm_xq, const CUtensorMap& tm
   }
 }
 
-UgemmPlan plan_ugemm(int T, int K, int R_pad) {
+UgemmPlan plan_ugemm(int T, int K, int R_tot) {
   UgemmPlan p;
-  if (R_pad <= 256) p.nu = R_pad;
-  else if (R_pad % 256 == 0) p.nu = 256;
-  else if (R_pad % 192 == 0) p.nu = 192;
-  else if (R_pad % 128 == 0) p.nu = 128;
+  if (R_tot <= 256) p.nu = R_tot;
+  else if (R_tot % 256 == 0) p.nu = 256;
+  else if (R_tot % 192 == 0) p.nu = 192;
+  else if (R_tot % 128 == 0) p.nu = 128;
   else p.nu = 64;
-  p.ntiles = static_cast<int>(ceil_div(R_pad, p.nu));
+  p.ntiles = static_cast<int>(ceil_div(R_tot, p.nu));
   const int mtiles = static_cast<int>(ceil_div(T, 128));
   const int nk = static_cast<int>(ceil_div(K, kAdapterAtom));
+  // about two waves of CTAs, each with at least 4 K chunks
   int splits = static_cast<int>(ceil_div(2 * 148, int64_t(mtiles) * p.ntiles));
-  splits = std::max(1, std::min(splits, std::max(1, nk / 2)));
+  splits = std::max(1, std::min(splits, std::max(1, nk / 4)));
   p.kchunks_per_split = static_cast<int>(ceil_div(nk, splits));
   p.splits = static_cast<int>(ceil_div(nk, p.kchunks_per_split));
   return p;
 }
 
 cudaError_t launch_ugemm(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, const UgemmPlan& plan, int T, int K,
-                         int R_pad, float* partial, int* err, cudaStream_t st) {
+                         int R_tot, float* partial, int* err, cudaStream_t st) {
   switch (plan.nu) {
-    case 64: return launch_ugemm_t<64>(tm_x, tm_acat, plan, T, K, R_pad, partial, err, st);
-    case 128: return launch_ugemm_t<128>(tm_x, tm_acat, plan, T, K, R_pad, partial, err, st);
-    case 192: return launch_ugemm_t<192>(tm_x, tm_acat, plan, T, K, R_pad, partial, err, st);
-    case 256: return launch_ugemm_t<256>(tm_x, tm_acat, plan, T, K, R_pad, partial, err, st);
+#define QE_NU(n) \
+  case n: return launch_ugemm_t<n>(tm_x, tm_acat, plan, T, K, R_tot, partial, err, st);
+    QE_NU(16) QE_NU(80) QE_NU(144) QE_NU(208) QE_NU(64) QE_NU(128) QE_NU(192) QE_NU(256)
+#undef QE_NU
     default: return cudaErrorInvalidValue;
   }
 }

@@ -391,16 +391,17 @@ __global__ void __launch_bounds__(128) k_unpack_w(const uint8_t* __restrict__ pa
 }
 
 // Adapter packing: A_catT [R_pad][K], B_catT [N][R_pad], G copy [K][n_r], all bf16.
-// The up-projections B_catT are stored as fp16 (the epilogue MMA multiplies them with the
-// fp16 U_cat). A bf16 value beyond the fp16 range is saturated and reported (DEVERR_RANGE).
-__global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a, int R_pad,
+// A_catT [R_tot][K] bf16 (down-projections, then the router G in rows R_pad..R_pad+N_r) and
+// B_catT [N][R_pad] fp16 (up-projections). The up-projections are fp16 because the epilogue
+// MMA multiplies them with the fp16 U_cat; a bf16 value beyond the fp16 range is saturated
+// and reported (device error 0x201).
+__global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a, int R_pad, int R_tot,
                                 const uint16_t* __restrict__ A_s, const uint16_t* __restrict__ B_s,
                                 const uint16_t* __restrict__ A_r, const uint16_t* __restrict__ B_r,
                                 const uint16_t* __restrict__ G, uint16_t* __restrict__ acat,
-                                uint16_t* __restrict__ bcat, uint16_t* __restrict__ gout, int* __restrict__ err) {
-  const size_t n1 = static_cast<size_t>(R_pad) * K, n2 = static_cast<size_t>(N) * R_pad,
-               n3 = static_cast<size_t>(K) * n_r;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n1 + n2 + n3;
+                                uint16_t* __restrict__ bcat, int* __restrict__ err) {
+  const size_t n1 = static_cast<size_t>(R_tot) * K, n2 = static_cast<size_t>(N) * R_pad;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n1 + n2;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     if (i < n1) {
       const int c = static_cast<int>(i / K), k = static_cast<int>(i % K);
@@ -409,9 +410,11 @@ __global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a
       else if (c < R_a) {
         const int e = (c - r_s) / r_r, j = (c - r_s) % r_r;
         v = A_r[(static_cast<size_t>(e) * K + k) * r_r + j];
+      } else if (c >= R_pad && c < R_pad + n_r) {
+        v = G[static_cast<size_t>(k) * n_r + (c - R_pad)];
       }
       acat[i] = v;
-    } else if (i < n1 + n2) {
+    } else {
       const size_t ii = i - n1;
       const int o = static_cast<int>(ii / R_pad), c = static_cast<int>(ii % R_pad);
       uint16_t v = 0;
@@ -427,57 +430,164 @@ __global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a
       }
       __half hv = __float2half_rn(f);
       bcat[ii] = *reinterpret_cast<uint16_t*>(&hv);
-    } else {
-      const size_t ii = i - n1 - n2;
-      gout[ii] = G[ii];
     }
   }
 }
 
-// U_cat[p][c] = fp16((sum over partial slots of P[slot][t][c]) / su[p]) with t = perm[p].
-// Routed columns of the other experts are 0. One warp per bucket position. su[p] is a power
-// of two that puts the row's largest |U| in [2^13, 2^14), so fp16 keeps full range and
-// 11-bit precision relative to the row; the epilogue multiplies the adapter term back by su.
-__global__ void k_ufinal(const float* __restrict__ partial, int nslots, const int32_t* __restrict__ perm,
-                         const int32_t* __restrict__ expert, int T, int R_pad, int r_s, int r_r, int R_a,
-                         uint16_t* __restrict__ ucat, float* __restrict__ su_sorted) {
-  const int warp = static_cast<int>((blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x) >> 5);
+// fp32 inputs: hi = bf16(x), lo = bf16(x - hi) in token order, and amax[t] = max_k |fl32(x*s_inv)|.
+// One warp per token.
+__global__ void k_split_f32(const float* __restrict__ X, const float* __restrict__ s_inv, int T, int K,
+                            uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo, float* __restrict__ amax) {
+  const int t = static_cast<int>((blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  const int p = warp;
-  const int t = perm[p];
-  const int e = expert[t];
-  constexpr int kMaxPerLane = 512 / 32;
-  float v[kMaxPerLane];
+  if (t >= T) return;
   float mx = 0.0f;
+  for (int k0 = lane * 8; k0 < K; k0 += 256) {
+    float xv[8], si[8];
+    load8<false>(X, t, K, k0, xv);
+    load8f(s_inv + k0, si);
+    uint32_t wh[4], wl[4];
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
-    const int c = lane + 32 * i;
-    float a = 0.0f;
-    if (c < R_pad && c < R_a && (c < r_s || (c - r_s) / r_r == e)) {
-      for (int s2 = 0; s2 < nslots; ++s2) a += __ldg(partial + (static_cast<size_t>(s2) * T + t) * R_pad + c);
+    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(__fmul_rn(xv[i], si[i])));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint16_t h0 = f32_to_bf16_bits(xv[2 * i]), h1 = f32_to_bf16_bits(xv[2 * i + 1]);
+      wh[i] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+      const uint16_t l0 = f32_to_bf16_bits(xv[2 * i] - bf16_bits_to_f32(h0));
+      const uint16_t l1 = f32_to_bf16_bits(xv[2 * i + 1] - bf16_bits_to_f32(h1));
+      wl[i] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
     }
-    v[i] = a;
-    mx = fmaxf(mx, fabsf(a));
+    *reinterpret_cast<uint4*>(xhi + static_cast<size_t>(t) * K + k0) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4*>(xlo + static_cast<size_t>(t) * K + k0) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  float su = 1.0f;
-  if (mx > 0.0f) {
-    int ex;
-    frexpf(mx, &ex);  // mx = m * 2^ex, m in [0.5, 1)
-    su = ldexpf(1.0f, ex - 14);
-  }
-  const float inv = 1.0f / su;  // exact: su is a power of two
+  if (lane == 0) amax[t] = mx;
+}
+
+// Per token (one warp): router logits from the GEMM partials, argmin with the lowest index on
+// exact ties, and sa = fl32(max_k |fl32(x*s_inv)| / qmax). The absmax is read from X for bf16
+// inputs, or taken from amax[t] (fp32 inputs, computed by k_split_f32).
+template <bool BF16>
+__global__ void k_tokfinal(const float* __restrict__ partial, int nslots, int R_tot, int R_pad, int n_r,
+                           const void* __restrict__ X, const float* __restrict__ s_inv, int K,
+                           const float* __restrict__ amax, int qmax, int T, int32_t* __restrict__ expert,
+                           float* __restrict__ sa_tok, float* __restrict__ logits) {
+  const int t = static_cast<int>((blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  float L = 0.0f;
+  if (lane < n_r)
+    for (int s2 = 0; s2 < nslots; ++s2) L += __ldg(partial + (static_cast<size_t>(s2) * T + t) * R_tot + R_pad + lane);
+  float best = (lane < n_r) ? L : INFINITY;
+  int bi = (lane < n_r) ? lane : 0x7fffffff;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
-    const int c = lane + 32 * i;
-    if (c < R_pad) {
-      __half h = __float2half_rn(v[i] * inv);
-      ucat[static_cast<size_t>(p) * R_pad + c] = *reinterpret_cast<uint16_t*>(&h);
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+    if (ov < best || (ov == best && oi < bi)) {
+      best = ov;
+      bi = oi;
     }
   }
-  if (lane == 0) su_sorted[p] = su;
+  float mx = 0.0f;
+  if (sa_tok) {
+    if (BF16) {
+      for (int k0 = lane * 8; k0 < K; k0 += 256) {
+        float xv[8], si[8];
+        load8<true>(X, t, K, k0, xv);
+        load8f(s_inv + k0, si);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(__fmul_rn(xv[i], si[i])));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    } else {
+      mx = amax[t];
+    }
+  }
+  if (logits && lane < n_r) logits[static_cast<size_t>(t) * n_r + lane] = L;
+  if (lane == 0) {
+    expert[t] = bi;
+    if (sa_tok) sa_tok[t] = __fdiv_rn(mx, static_cast<float>(qmax));
+  }
+}
+
+// Per token (one warp), in bucket order p = pos[t]: the activation codes (or the bf16
+// activations of weight-only layers), sa_sorted[p], and the adapter row U_cat[p]: the sum of
+// the GEMM partial slots, with the routed columns of every other expert zeroed, in fp16 after
+// division by su[p], a power of two that puts the row's largest |U| in [2^13, 2^14).
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_quant_u(const void* __restrict__ X, const float* __restrict__ s_inv, int T,
+                                                 int K, int qmax, const float* __restrict__ sa_tok,
+                                                 const int32_t* __restrict__ pos, const int32_t* __restrict__ expert,
+                                                 int8_t* __restrict__ codes, uint16_t* __restrict__ act16,
+                                                 float* __restrict__ sa_sorted, const float* __restrict__ partial,
+                                                 int nslots, int R_tot, int R_pad, int r_s, int r_r, int R_a,
+                                                 uint16_t* __restrict__ ucat, float* __restrict__ su_sorted) {
+  const int t = static_cast<int>((blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const size_t p = static_cast<size_t>(pos[t]);
+  const float sa = sa_tok ? sa_tok[t] : 0.0f;
+  for (int k0 = lane * 8; k0 < K; k0 += 256) {
+    float xv[8], si[8], v[8];
+    load8<BF16>(X, t, K, k0, xv);
+    load8f(s_inv + k0, si);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(xv[i], si[i]);
+    if (codes) {
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        w0 |= (static_cast<uint32_t>(rtn_code(v[i], sa, qmax)) & 0xFFu) << (8 * i);
+        w1 |= (static_cast<uint32_t>(rtn_code(v[4 + i], sa, qmax)) & 0xFFu) << (8 * i);
+      }
+      *reinterpret_cast<uint2*>(codes + p * K + k0) = make_uint2(w0, w1);
+    } else {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w[i] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i])) |
+               (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i + 1])) << 16);
+      *reinterpret_cast<uint4*>(act16 + p * K + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  if (codes && lane == 0) sa_sorted[p] = sa;
+  if (R_pad > 0) {
+    const int e = expert[t];
+    constexpr int kMaxPerLane = 512 / 32;
+    float u[kMaxPerLane];
+    float mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int c = lane + 32 * i;
+      float a2 = 0.0f;
+      if (c < R_a && (c < r_s || (c - r_s) / r_r == e)) {
+        for (int s2 = 0; s2 < nslots; ++s2) a2 += __ldg(partial + (static_cast<size_t>(s2) * T + t) * R_tot + c);
+      }
+      u[i] = a2;
+      mx = fmaxf(mx, fabsf(a2));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float su = 1.0f;
+    if (mx > 0.0f) {
+      int ex;
+      frexpf(mx, &ex);  // mx = m * 2^ex, m in [0.5, 1)
+      su = ldexpf(1.0f, ex - 14);
+    }
+    const float inv = 1.0f / su;  // exact: su is a power of two
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int c = lane + 32 * i;
+      if (c < R_pad) {
+        __half h = __float2half_rn(u[i] * inv);
+        ucat[p * R_pad + c] = *reinterpret_cast<uint16_t*>(&h);
+      }
+    }
+    if (lane == 0) su_sorted[p] = su;
+  }
 }
 
 // Y[perm[p]][o] = sum_s partial[s][p][o] (fixed order).
@@ -562,18 +672,46 @@ cudaError_t launch_unpack_weights(const uint8_t* packed, int N, int K, int w_bit
 cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint16_t* A_s, const uint16_t* B_s,
                                  const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out, int* err,
                                  cudaStream_t st) {
-  k_pack_adapters<<<592, 256, 0, st>>>(K, N, g.r_s, g.n_r, g.r_r, g.R_a, g.R_pad, A_s, B_s, A_r, B_r, G,
-                                       reinterpret_cast<uint16_t*>(out + g.off_acat),
-                                       reinterpret_cast<uint16_t*>(out + g.off_bcat),
-                                       reinterpret_cast<uint16_t*>(out + g.off_g), err);
+  k_pack_adapters<<<592, 256, 0, st>>>(K, N, g.r_s, g.n_r, g.r_r > 0 ? g.r_r : 1, g.R_a, g.R_pad, g.R_tot, A_s, B_s,
+                                       A_r, B_r, G, reinterpret_cast<uint16_t*>(out + g.off_acat),
+                                       reinterpret_cast<uint16_t*>(out + g.off_bcat), err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_ufinal(const float* partial, int nslots, const int32_t* perm, const int32_t* expert, int T,
-                          int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, float* su_sorted, cudaStream_t st) {
+cudaError_t launch_split_f32(const float* X, const float* s_inv, int T, int K, uint16_t* xhi, uint16_t* xlo,
+                             float* amax, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  k_ufinal<<<static_cast<unsigned>(ceil_div(T, 8)), 256, 0, st>>>(partial, nslots, perm, expert, T, R_pad, r_s,
-                                                                  r_r > 0 ? r_r : 1, R_a, ucat, su_sorted);
+  k_split_f32<<<static_cast<unsigned>(ceil_div(T, 8)), 256, 0, st>>>(X, s_inv, T, K, xhi, xlo, amax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tokfinal(const float* partial, int nslots, int R_tot, int R_pad, int n_r, const void* X,
+                            bool x_bf16, const float* s_inv, int K, const float* amax, int qmax, int T,
+                            int32_t* expert, float* sa_tok, float* logits, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>(ceil_div(T, 8));
+  if (x_bf16)
+    k_tokfinal<true><<<grid, 256, 0, st>>>(partial, nslots, R_tot, R_pad, n_r, X, s_inv, K, amax, qmax, T, expert,
+                                           sa_tok, logits);
+  else
+    k_tokfinal<false><<<grid, 256, 0, st>>>(partial, nslots, R_tot, R_pad, n_r, X, s_inv, K, amax, qmax, T, expert,
+                                            sa_tok, logits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_u(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
+                           const float* sa_tok, const int32_t* pos, const int32_t* expert, int8_t* codes,
+                           uint16_t* act16, float* sa_sorted, const float* partial, int nslots, int R_tot,
+                           int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, float* su_sorted, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>(ceil_div(T, 8));
+  if (x_bf16)
+    k_quant_u<true><<<grid, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, expert, codes, act16, sa_sorted, partial,
+                                          nslots, R_tot, R_pad, r_s, r_r > 0 ? r_r : 1, R_a, ucat, su_sorted);
+  else
+    k_quant_u<false><<<grid, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, expert, codes, act16, sa_sorted,
+                                           partial, nslots, R_tot, R_pad, r_s, r_r > 0 ? r_r : 1, R_a, ucat,
+                                           su_sorted);
   return cudaGetLastError();
 }
 

@@ -63,9 +63,9 @@ struct Plan {
   AdapterGeom g;
   UgemmPlan up;
   int bn, msplits, kbps;  // main product
-  int uslots;             // U partial slots: splits, doubled for fp32 inputs (hi and lo passes)
-  size_t off_expert, off_perm, off_pos, off_offsets, off_sa_tok, off_sa_sorted, off_su_sorted, off_act, off_xb16,
-      off_xlo16, off_upart, off_ucat, off_ypart, bytes;
+  int uslots;             // GEMM partial slots: splits, doubled for fp32 inputs (hi and lo passes)
+  size_t off_expert, off_perm, off_pos, off_offsets, off_sa_tok, off_sa_sorted, off_su_sorted, off_act, off_xhi,
+      off_xlo, off_amax, off_upart, off_ucat, off_ypart, bytes;
 };
 
 int wonly_splits(int T, int N, int K) {
@@ -86,7 +86,7 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   p.g = geom_of(d);
   p.has_ad = p.g.R_a > 0;
   const int Tm = std::max(T, 1);
-  p.up = plan_ugemm(Tm, p.K, p.g.R_pad);
+  p.up = plan_ugemm(Tm, p.K, p.g.R_tot);
   if (d->a_bits == 16) {
     p.bn = 0;
     p.msplits = wonly_splits(Tm, p.N, p.K);
@@ -94,6 +94,7 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   } else {
     p.bn = pick_qgemm_bn(Tm, p.N, p.K, &p.msplits, &p.kbps);
   }
+  p.uslots = p.up.splits * (x_bf16 ? 1 : 2);
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -108,10 +109,10 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   p.off_sa_sorted = take(size_t(Tm) * 4);
   p.off_su_sorted = take(size_t(Tm) * 4);
   p.off_act = take(size_t(Tm) * p.K * (d->a_bits == 16 ? 2 : 1));
-  p.off_xb16 = (!x_bf16 && p.has_ad) ? take(size_t(Tm) * p.K * 2) : 0;
-  p.off_xlo16 = (!x_bf16 && p.has_ad) ? take(size_t(Tm) * p.K * 2) : 0;
-  p.uslots = p.up.splits * (x_bf16 ? 1 : 2);
-  p.off_upart = p.has_ad ? take(size_t(p.uslots) * Tm * p.g.R_pad * 4) : 0;
+  p.off_xhi = x_bf16 ? 0 : take(size_t(Tm) * p.K * 2);
+  p.off_xlo = x_bf16 ? 0 : take(size_t(Tm) * p.K * 2);
+  p.off_amax = x_bf16 ? 0 : take(size_t(Tm) * 4);
+  p.off_upart = take(size_t(p.uslots) * Tm * p.g.R_tot * 4);
   p.off_ucat = p.has_ad ? take(size_t(Tm) * p.g.R_pad * 2) : 0;
   p.off_ypart = (p.msplits > 1) ? take(size_t(p.msplits) * Tm * p.N * 4) : 0;
   p.bytes = o;
@@ -181,7 +182,6 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   const uint8_t* ad = static_cast<const uint8_t*>(w->adapters);
   const uint16_t* acat = reinterpret_cast<const uint16_t*>(ad + p.g.off_acat);
   const uint16_t* bcat = reinterpret_cast<const uint16_t*>(ad + p.g.off_bcat);
-  const uint16_t* G = reinterpret_cast<const uint16_t*>(ad + p.g.off_g);
   int32_t* expert = at<int32_t>(ws, p.off_expert);
   int32_t* perm = at<int32_t>(ws, p.off_perm);
   int32_t* pos = at<int32_t>(ws, p.off_pos);
@@ -189,49 +189,52 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   float* sa_tok = at<float>(ws, p.off_sa_tok);
   float* sa_sorted = at<float>(ws, p.off_sa_sorted);
   float* su_sorted = at<float>(ws, p.off_su_sorted);
+  float* amax = x_bf16 ? nullptr : at<float>(ws, p.off_amax);
+  float* upart = at<float>(ws, p.off_upart);
   const bool wonly = d->a_bits == 16;
   const int qmax = wonly ? 1 : qmax_of(d->a_bits);
   const int K = p.K, N = p.N;
 
-  // 1. router + per-token absmax, then the stable bucket sort
-  if (stages & QE_STAGE_ROUTE) {
-    QE_CUDA(launch_route_stats(X, x_bf16, w->s_inv, G, T, K, d->n_routed, qmax, expert, wonly ? nullptr : sa_tok,
-                               nullptr, st),
-            "route_stats");
-    QE_CUDA(launch_bucket(expert, T, d->n_routed, perm, pos, offsets, st), "bucket");
-  }
-  // 3. quantize in bucket order
-  int8_t* codes = wonly ? nullptr : at<int8_t>(ws, p.off_act);
-  uint16_t* act16 = wonly ? at<uint16_t>(ws, p.off_act) : nullptr;
-  uint16_t* xb16 = (!x_bf16 && p.has_ad) ? at<uint16_t>(ws, p.off_xb16) : nullptr;
-  uint16_t* xlo16 = (!x_bf16 && p.has_ad) ? at<uint16_t>(ws, p.off_xlo16) : nullptr;
-  if (stages & QE_STAGE_QUANT)
-    QE_CUDA(launch_act_quant(X, x_bf16, w->s_inv, T, K, qmax, sa_tok, pos, codes, sa_sorted, act16, xb16, xlo16,
-                             st),
-            "act_quant");
-  // 4. adapter down-projection (tensor cores) -> U_cat in bucket order
-  uint16_t* ucat = p.has_ad ? at<uint16_t>(ws, p.off_ucat) : nullptr;
-  if (p.has_ad && (stages & QE_STAGE_ADAPTERS)) {
-    CUtensorMap tm_x, tm_acat;
-    const void* xsrc = x_bf16 ? X : static_cast<const void*>(xb16);
-    if ((s = make_tmap(&tm_x, xsrc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK) return s;
-    if ((s = make_tmap(&tm_acat, acat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, p.g.R_pad, kAdapterAtom,
-                       p.up.nu)) != QE_OK)
+  // 1. one tensor-core GEMM: adapter down-projections + router logits
+  if (stages & QE_STAGE_PROJECT) {
+    CUtensorMap tm_acat;
+    if ((s = make_tmap(&tm_acat, acat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, p.g.R_tot, kAdapterAtom, p.up.nu)) !=
+        QE_OK)
       return s;
-    float* upart = at<float>(ws, p.off_upart);
-    QE_CUDA(launch_ugemm(tm_x, tm_acat, p.up, T, K, p.g.R_pad, upart, err, st), "ugemm");
-    if (!x_bf16) {  // fp32 input: second pass over the low bf16 part into the next partial slots
-      CUtensorMap tm_xlo;
-      if ((s = make_tmap(&tm_xlo, xlo16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK)
-        return s;
-      QE_CUDA(launch_ugemm(tm_xlo, tm_acat, p.up, T, K, p.g.R_pad,
-                           upart + size_t(p.up.splits) * T * p.g.R_pad, err, st),
+    if (x_bf16) {
+      CUtensorMap tm_x;
+      if ((s = make_tmap(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK) return s;
+      QE_CUDA(launch_ugemm(tm_x, tm_acat, p.up, T, K, p.g.R_tot, upart, err, st), "ugemm");
+    } else {
+      // fp32 input: x = hi + lo in bf16, two passes into consecutive partial slots
+      uint16_t* xhi = at<uint16_t>(ws, p.off_xhi);
+      uint16_t* xlo = at<uint16_t>(ws, p.off_xlo);
+      QE_CUDA(launch_split_f32(static_cast<const float*>(X), w->s_inv, T, K, xhi, xlo, amax, st), "split_f32");
+      CUtensorMap tm_hi, tm_lo;
+      if ((s = make_tmap(&tm_hi, xhi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK) return s;
+      if ((s = make_tmap(&tm_lo, xlo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK) return s;
+      QE_CUDA(launch_ugemm(tm_hi, tm_acat, p.up, T, K, p.g.R_tot, upart, err, st), "ugemm_hi");
+      QE_CUDA(launch_ugemm(tm_lo, tm_acat, p.up, T, K, p.g.R_tot, upart + size_t(p.up.splits) * T * p.g.R_tot,
+                           err, st),
               "ugemm_lo");
     }
-    QE_CUDA(launch_ufinal(upart, p.uslots, perm, expert, T, p.g.R_pad, d->rank_shared, d->rank_routed, p.g.R_a, ucat,
-                          su_sorted, st),
-            "ufinal");
   }
+  // 2. argmin routing, per-token absmax and scale, stable bucket sort
+  if (stages & QE_STAGE_ROUTE) {
+    QE_CUDA(launch_tokfinal(upart, p.uslots, p.g.R_tot, p.g.R_pad, d->n_routed, X, x_bf16, w->s_inv, K, amax, qmax,
+                            T, expert, wonly ? nullptr : sa_tok, nullptr, st),
+            "tokfinal");
+    QE_CUDA(launch_bucket(expert, T, d->n_routed, perm, pos, offsets, st), "bucket");
+  }
+  // 3. quantize in bucket order, and the expert-masked adapter rows U_cat
+  int8_t* codes = wonly ? nullptr : at<int8_t>(ws, p.off_act);
+  uint16_t* act16 = wonly ? at<uint16_t>(ws, p.off_act) : nullptr;
+  uint16_t* ucat = p.has_ad ? at<uint16_t>(ws, p.off_ucat) : nullptr;
+  if (stages & QE_STAGE_QUANT)
+    QE_CUDA(launch_quant_u(X, x_bf16, w->s_inv, T, K, qmax, wonly ? nullptr : sa_tok, pos, expert, codes, act16,
+                           sa_sorted, upart, p.uslots, p.g.R_tot, p.g.R_pad, d->rank_shared, d->rank_routed, p.g.R_a,
+                           ucat, su_sorted, st),
+            "quant_u");
   // 5. main product
   if (!(stages & QE_STAGE_PRODUCT)) return QE_OK;
   float* ypart = p.msplits > 1 ? at<float>(ws, p.off_ypart) : nullptr;
@@ -305,6 +308,10 @@ qe_status static_scratch(void** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    // The lookup can load this module onto the device, and the loader initializes the
+    // array asynchronously. Wait for that once, so it cannot overwrite the first call's data.
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize(static scratch set-up)");
     addr[dev] = p;
   }
   *out = addr[dev];
@@ -409,10 +416,10 @@ int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, qe_dtype
   if (check_desc(desc) != QE_OK || T < 0) return -1;
   if (T == 0) return 0;
   const Plan p = make_plan(desc, T, x_dtype == QE_BF16);
-  int n = 3;                    // route_stats, bucket, act_quant
-  if (p.has_ad) n += (x_dtype == QE_BF16) ? 2 : 3;  // ugemm (twice for fp32 inputs), ufinal
-  n += 1;                       // qgemm or the weight-only product
-  if (p.msplits > 1) n += 1;    // split-K reduce
+  int n = (x_dtype == QE_BF16) ? 1 : 3;  // down-projection GEMM (fp32 inputs: split + hi and lo passes)
+  n += 3;                                // tokfinal, bucket, quant_u
+  n += 1;                                // main product (int8 GEMM or weight-only)
+  if (p.msplits > 1) n += 1;             // split-K reduce
   return n;
 }
 

@@ -19,11 +19,16 @@ __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Packed adapter buffer geometry.
+//   A_catT [R_tot][K] bf16: rows [0, R_a) are the shared and routed down-projections
+//     (A_s columns, then A_r[e] columns expert by expert), rows [R_pad, R_pad + N_r) are the
+//     router G (transposed), all other rows zero. One GEMM gives U and the router logits.
+//   B_catT [N][R_pad] fp16: the matching up-projections (absent when R_pad = 0).
 struct AdapterGeom {
   int r_s, n_r, r_r;
   int R_a;    // r_s + n_r * r_r
-  int R_pad;  // round_up(R_a, 64), >= 64
-  size_t off_acat, off_bcat, off_g, bytes;
+  int R_pad;  // round_up(R_a, 64), or 0 when the layer has no adapters
+  int R_tot;  // R_pad + 16 when that fits one 256-column MMA, else R_pad + 64
+  size_t off_acat, off_bcat, bytes;
 };
 inline AdapterGeom adapter_geom(int K, int N, int r_s, int n_r, int r_r) {
   AdapterGeom g;
@@ -31,11 +36,11 @@ inline AdapterGeom adapter_geom(int K, int N, int r_s, int n_r, int r_r) {
   g.n_r = n_r;
   g.r_r = r_r;
   g.R_a = r_s + n_r * r_r;
-  g.R_pad = static_cast<int>(round_up(g.R_a > 0 ? g.R_a : 1, kAdapterAtom));
+  g.R_pad = g.R_a > 0 ? static_cast<int>(round_up(g.R_a, kAdapterAtom)) : 0;
+  g.R_tot = (g.R_pad + 16 <= 256) ? g.R_pad + 16 : g.R_pad + 64;
   g.off_acat = 0;
-  g.off_bcat = align256(g.off_acat + size_t(g.R_pad) * K * 2);
-  g.off_g = align256(g.off_bcat + size_t(N) * g.R_pad * 2);
-  g.bytes = align256(g.off_g + size_t(K) * n_r * 2);
+  g.off_bcat = align256(g.off_acat + size_t(g.R_tot) * K * 2);
+  g.bytes = align256(g.off_bcat + size_t(N) * g.R_pad * 2);
   return g;
 }
 
@@ -52,7 +57,8 @@ cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint1
                                  const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out, int* err,
                                  cudaStream_t st);
 
-// Router logits + argmin, and (when sa != nullptr) the per-token absmax -> scale.
+// Router logits + argmin, and (when sa != nullptr) the per-token absmax -> scale, on CUDA cores
+// (the standalone router entry point and the activation-quantization diagnostic).
 cudaError_t launch_route_stats(const void* X, bool x_bf16, const float* s_inv, const uint16_t* G, int T, int K,
                                int n_r, int qmax, int32_t* expert, float* sa, float* logits, cudaStream_t st);
 // Stable bucket sort of tokens by expert: perm (sorted pos -> token), pos (token -> sorted pos), offsets.
@@ -61,26 +67,39 @@ cudaError_t launch_bucket(const int32_t* expert, int T, int n_r, int32_t* perm, 
 // Per-token quantization of x*s_inv with the scale sa_tok[t], written at row pos[t] (pos == nullptr: row t).
 //   codes != nullptr: int8 codes, sa_sorted[pos] = sa_tok[t]
 //   act16 != nullptr: bf16(x*s_inv) (weight-only layers)
-//   xb16  != nullptr: hi = bf16(x) in token order (fp32 inputs feeding the adapter GEMM)
-//   xlo16 != nullptr: lo = bf16(x - hi), so that hi + lo carries 16 significant bits of x
+// (used by the activation-quantization diagnostic entry point)
 cudaError_t launch_act_quant(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
                              const float* sa_tok, const int32_t* pos, int8_t* codes, float* sa_sorted,
                              uint16_t* act16, uint16_t* xb16, uint16_t* xlo16, cudaStream_t st);
 
-// Adapter down-projection partials: P[split][t][c] = sum_{k in split} X[t][k] * A_catT[c][k] (tcgen05, bf16).
+// fp32 inputs: x = hi + lo (both bf16, token order) for the bf16 tensor-core GEMM, and the
+// per-token absmax of fl32(x*s_inv) (one slot).
+cudaError_t launch_split_f32(const float* X, const float* s_inv, int T, int K, uint16_t* xhi, uint16_t* xlo,
+                             float* amax, cudaStream_t st);
+
+// P[slot][t][c] = sum over this split's K range of X[t][k] * A_catT[c][k], c < R_tot (tcgen05, bf16):
+// the adapter down-projections and, in columns [R_pad, R_pad + N_r), the router logits.
 struct UgemmPlan {
   int splits;
   int kchunks_per_split;  // 64-wide K chunks per split
   int nu;                 // N tile (columns of A_catT per CTA), <= 256
   int ntiles;
 };
-UgemmPlan plan_ugemm(int T, int K, int R_pad);
+UgemmPlan plan_ugemm(int T, int K, int R_tot);
 cudaError_t launch_ugemm(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, const UgemmPlan& plan, int T,
-                         int K, int R_pad, float* partial, int* err, cudaStream_t st);
-// U_cat[p][c] = fp16(sum over partial slots of P[slot][perm[p]][c] / su[p]), routed columns masked to the
-// token's expert, su[p] a per-position power of two.
-cudaError_t launch_ufinal(const float* partial, int nslots, const int32_t* perm, const int32_t* expert, int T,
-                          int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, float* su_sorted, cudaStream_t st);
+                         int K, int R_tot, float* partial, int* err, cudaStream_t st);
+// Per token: logits = sum over slots, expert = argmin (lowest index on ties); sa = absmax / qmax, with
+// the absmax max_k |fl32(x*s_inv)| taken from X (bf16 inputs) or from amax[t] (fp32 inputs, from
+// launch_split_f32). sa_tok == nullptr skips the scale.
+cudaError_t launch_tokfinal(const float* partial, int nslots, int R_tot, int R_pad, int n_r, const void* X,
+                            bool x_bf16, const float* s_inv, int K, const float* amax, int qmax, int T,
+                            int32_t* expert, float* sa_tok, float* logits, cudaStream_t st);
+// Per token, in bucket order p = pos[t]: activation codes (or bf16 activations), sa_sorted, and
+// U_cat[p] = fp16((sum of U slots, routed columns of other experts zeroed) / su[p]).
+cudaError_t launch_quant_u(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
+                           const float* sa_tok, const int32_t* pos, const int32_t* expert, int8_t* codes,
+                           uint16_t* act16, float* sa_sorted, const float* partial, int nslots, int R_tot,
+                           int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, float* su_sorted, cudaStream_t st);
 
 // Main quantized GEMM (W4 x A8/A6 codes, tcgen05 kind::i8) with per-group promotion,
 // per-token scale, adapter MMA in the epilogue and scatter to token order.

@@ -41,12 +41,16 @@ def test_sizes_follow_documented_layout(lib):
     # ragged d_out pads to whole 128-row blocks
     dr = qe.make_desc(256, 200, 64, 4, 8, 8, 4, 4)
     assert qe.packed_weight_bytes(dr) == 2 * 2 * 8192
-    # adapters: A_catT [R_pad][K] + B_catT [N][R_pad] + G [K][N_r], bf16, 256-byte aligned pieces
-    R_pad = 64
+    # adapters: A_catT [R_pad + 16][K] bf16 (down-projections + router rows) + B_catT [N][R_pad] fp16,
+    # 256-byte aligned pieces; R_pad = round_up(r_s + N_r*r_r, 64) = 64 here
+    R_pad, R_tot = 64, 80
     expect = 0
-    for nbytes in (R_pad * 1536 * 2, 8960 * R_pad * 2, 1536 * 8 * 2):
+    for nbytes in (R_tot * 1536 * 2, 8960 * R_pad * 2):
         expect = ((expect + nbytes + 255) // 256) * 256
     assert qe.adapter_packed_bytes(d) == expect
+    # a layer without adapters keeps only the router rows
+    d0 = qe.make_desc(1536, 8960, 128, 4, 6, 0, 8, 0)
+    assert qe.adapter_packed_bytes(d0) == ((16 * 1536 * 2 + 255) // 256) * 256
     assert qe.linear_workspace_bytes(d, 2048) > 2048 * 1536  # at least the int8 codes
     assert qe.linear_workspace_bytes(d, 0) > 0
 

@@ -314,3 +314,33 @@ def test_full_size_decode(cfg_name, T, proj_index):
     Y_ref, _ = c.oracle_forward(expert_override=e)
     err = rel_err(Y.cpu().numpy(), Y_ref)
     assert err <= Y_TOL, err
+
+
+@pytest.mark.parametrize("cfg_name,proj_index,T", [("tiny", 0, 64), ("qwen2vl2b", 4, 300), ("qwen2vl2b", 0, 129)])
+def test_forward_ignores_workspace_contents(cfg_name, proj_index, T):
+    # The header promises that the workspace's contents on entry do not matter:
+    # garbage in the scratch must give bit-identical results.
+    cfg = qi.CONFIGS[cfg_name]
+    c = Case(cfg, cfg.projections[proj_index], T, proj_index=proj_index)
+    ws = c.layer.workspace(T)
+    outs = []
+    for fill in (0x00, 0xFF, 0x7F):
+        ws.fill_(fill)
+        Y = torch.empty((T, c.proj.d_out), dtype=torch.float32, device="cuda")
+        qe.linear_forward(c.desc, c.layer.weights, c.Xd, Y, ws)
+        torch.cuda.synchronize()
+        assert qe.device_error() == 0
+        outs.append(Y)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+@pytest.mark.parametrize("proj_index", [2, 4])
+def test_forward_full_size_is_deterministic(proj_index):
+    # Every output element comes from one fixed sequence of operations: repeated runs of a
+    # full-size layer must be bit-identical (a race shows up as a few differing rows).
+    cfg = qi.CONFIGS["qwen2vl2b"]
+    c = Case(cfg, cfg.projections[proj_index], cfg.T, proj_index=proj_index)
+    ys = [c.gpu_forward() for _ in range(8)]
+    for y in ys[1:]:
+        bad = (~(y == ys[0]).all(dim=1)).nonzero().flatten().tolist()
+        assert not bad, f"rows differing between runs: {bad[:10]}"
