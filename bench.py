@@ -4,14 +4,18 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 A step is one pass of the hot path over one batch: every projection of the
-workload's layer set goes through qe_linear_forward. Each forward is router
-+ bucket sort, per-token quantization, adapter down-projection, and the int8
-tcgen05 product with its adapter epilogue. Inputs are synthetic and seeded,
-with the shapes of the named model (qe_inputs), and resident in HBM when the
-timed region starts. L2 is flushed between steps, outside the per-step event
-pairs. The step time is the sum of the per-step event pairs. Under torchrun
-each rank runs an independent replica on its own token batch (weak
-scaling, no data-path collective), and the time is the max over ranks.
+workload's layer set goes through the QE forward, in four stages: the
+tensor-core down-projection with the router logits, routing and the bucket
+sort, quantization with the expert-masked adapter rows, and the int8
+tcgen05 product with its adapter epilogue. The step is captured once as a
+CUDA graph with timing events between the stages, and replayed. Inputs are
+synthetic and seeded, with the shapes of the named model (qe_inputs), and
+resident in HBM when the timed region starts. L2 is flushed between steps,
+outside the timed intervals. The step time is the sum of the stage
+intervals. Under torchrun each rank runs an independent replica on its own
+token batch (weak scaling, no data-path collective), and the time is the
+max over ranks. e2e times the plain public call with pinned host buffers
+and the copies inside the timed region.
 
 `--impl reference` times the CPU oracle (a deliberately slow, plain program)
 on a bounded token sample of the same workload, on the host's cores.
@@ -279,46 +283,52 @@ def run_ours(args, workload):
     wonly = cfg.a_bits == 16
     stages = (qe.QE_STAGE_PROJECT, qe.QE_STAGE_ROUTE, qe.QE_STAGE_QUANT, qe.QE_STAGE_PRODUCT)
 
-    def step(record):
-        evs = []
+    def step_plain():
         for L in layers:
-            if record:
-                e = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
-                e[0].record(stream)
-                for i, sm in enumerate(stages):
-                    qe.linear_forward_stages(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"], sm)
-                    e[i + 1].record(stream)
-                evs.append(e)
-            else:
-                qe.linear_forward(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"])
-        return evs
+            qe.linear_forward(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"])
 
     for _ in range(max(args.warmup, 0)):
         flush.zero_()
-        step(False)
+        step_plain()
     torch.cuda.synchronize()
     assert qe.device_error() == 0, "a device wait ran out during warm-up"
 
-    all_evs = []
+    # One step = every projection through its four stages, captured once into a CUDA graph
+    # with timing events between the stages. The hot path is a chain of short kernels, so the
+    # graph removes host launch gaps from the device timeline. Each replay is timed by its
+    # own events; they are read back after the replay, outside the timed intervals.
+    cap = torch.cuda.Stream()
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)] for _ in layers]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap):
+        for L, e in zip(layers, evs):
+            e[0].record()
+            for i, sm in enumerate(stages):
+                qe.linear_forward_stages(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"], sm)
+                e[i + 1].record()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    n_proj = len(layers)
+    stage_ms = np.zeros((args.steps, n_proj, len(stages)))
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        for _ in range(args.steps):
+        for s_i in range(args.steps):
             flush.zero_()
-            all_evs.append(step(True))
-        torch.cuda.synchronize()
+            graph.replay()
+            torch.cuda.synchronize()
+            for p_i, e in enumerate(evs):
+                for k in range(len(stages)):
+                    stage_ms[s_i, p_i, k] = e[k].elapsed_time(e[k + 1])
     if pg:
         pg.barrier()
     err = qe.device_error()
     assert err == 0, f"device wait ran out (code {err:#x})"
+    del graph
 
-    n_proj = len(layers)
-    stage_ms = np.zeros((args.steps, n_proj, len(stages)))
-    for s_i, evs in enumerate(all_evs):
-        for p_i, e in enumerate(evs):
-            for k in range(len(stages)):
-                stage_ms[s_i, p_i, k] = e[k].elapsed_time(e[k + 1])
     step_ms = stage_ms.sum(axis=(1, 2))
     total_ms = max_over_ranks(float(step_ms.sum()), pg, dev)
     ms_per_step = total_ms / args.steps
