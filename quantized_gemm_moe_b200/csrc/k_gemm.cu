@@ -6,10 +6,11 @@
 //   operand). Each pipeline stage covers 128 input channels:
 //     warp 0      TMA producer: activation codes (tensor map, 128B swizzle),
 //                 plus one bulk copy of the 8 KB packed-int4 weight block
-//     warps 2-3   unpack the int4 block into int8 in the 128B-swizzled A layout
-//     warp 1      one elected thread issues tcgen05.mma kind::i8, one TMEM
-//                 accumulator buffer per quantization group (2 buffers at BN=256,
-//                 4 below, so the MMA runs ahead of the epilogue)
+//     warps 12-15 unpack the int4 block into int8 in the 128B-swizzled A layout
+//     warps 1-2   one thread each issues tcgen05.mma kind::i8 for alternate
+//                 stages, one TMEM accumulator buffer per quantization group
+//                 (2 buffers at BN=256, 4 below, so the MMA runs ahead of the
+//                 epilogue)
 //     warps 4-11  epilogue: the per-group promotion acc += sw[o,j] * float(int32)
 //                 in registers (f32x2, the next TMEM chunk loading meanwhile),
 //                 then * sa[t], + adapter MMA result, and a scatter of the row
@@ -232,7 +233,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&accf[b], 1);
       mbar_init(&acce[b], 8);
     }
-    mbar_init(done, 1);
+    mbar_init(done, 2);
     mbar_fence_init();
     prefetch_tmap(&tm_xq);
     if (a.adapter_atoms) {
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(512, 1)
   }
   __syncthreads();
 
-  // Roles: warp 0 TMA producer, warp 1 MMA issuer (warps 2-3 idle), warps 4-11 epilogue,
+  // Roles: warp 0 TMA producer, warps 1-2 MMA issuers (warp 3 idle), warps 4-11 epilogue,
   // warps 12-15 unpack. Register split: 256 * kRegLow + 256 * kRegHigh = 512 x 128 launch
   // registers; each role sets its own limit at its entry.
   if (warp == 0) {
@@ -295,30 +296,42 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // One thread issuing every tcgen05.mma cannot keep the tensor pipe busy: each issue,
+    // barrier wait and commit costs it tens of cycles. Two issuers split the stages by
+    // parity of the running stage index. A unit's adapter atoms accumulate into one TMEM
+    // buffer, so one issuer takes all of them and their fp32 sums keep a fixed order.
+    // The unpack warps wait for the TMA bytes before they arrive on afull, so afull alone
+    // tells an issuer that both operands of the stage are in shared memory.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegLow) : "memory");
+    const int qi = warp - 1;
     if (lane == 0) {
       const uint32_t id_i8 = idesc_i8(128, BN);
       const uint32_t id_ad = idesc_f16(128, BN);
+      const int ksteps = a.group / 32;
       int it = 0, gidx = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const Unit w = make_unit(a, BN, u);
+        const int ad_owner = (it + w.nkb) & 1;
         for (int i = 0; i < w.nkb + w.n_ad && ok; ++i, ++it) {
           const int s = it % NS;
           const uint32_t ph = (it / NS) & 1;
-          if (!mbar_wait(&full[s], ph, a_err, DEVERR_WAIT_MMA) || !mbar_wait(&afull[s], ph, a_err, DEVERR_WAIT_MMA)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
           const uint32_t a_addr = smem_u32(stage_base + s * C::kStage);
           const uint32_t b_addr = a_addr + C::kA;
           if (i < w.nkb) {
             const int kb = w.kb_begin + i;
-            for (int gi = 0; gi < gpb; ++gi) {
-              if (kb * gpb + gi >= w.g_begin + w.n_groups) break;
+            const int ng = max(0, min(gpb, w.g_begin + w.n_groups - kb * gpb));
+            if ((it & 1) != qi) {
+              gidx += ng;
+              continue;
+            }
+            if (!mbar_wait(&afull[s], ph, a_err, DEVERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
+            for (int gi = 0; gi < ng; ++gi) {
               const int b = gidx % NB;
               if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
                 ok = false;
@@ -326,7 +339,7 @@ __global__ void __launch_bounds__(512, 1)
               }
               tc_fence_after();
               const uint32_t d = tmem + b * BN;
-              for (int kk = 0; kk < a.group / 32; ++kk) {
+              for (int kk = 0; kk < ksteps; ++kk) {
                 const uint32_t koff = gi * a.group + kk * 32;
                 mma_i8(d, smem_desc_sw128(a_addr + koff), smem_desc_sw128(b_addr + koff), id_i8, 1u);
               }
@@ -336,13 +349,21 @@ __global__ void __launch_bounds__(512, 1)
           } else {
             const int at = i - w.nkb;
             const int b = gidx % NB;
+            if (ad_owner != qi) {
+              if (at == w.n_ad - 1) ++gidx;
+              continue;
+            }
+            if (!mbar_wait(&afull[s], ph, a_err, DEVERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
             if (at == 0) {
               if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
                 ok = false;
                 break;
               }
-              tc_fence_after();
             }
+            tc_fence_after();
             const uint32_t d = tmem + b * BN;
             for (int kk = 0; kk < 4; ++kk)
               mma_f16(d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), id_ad,
@@ -355,11 +376,11 @@ __global__ void __launch_bounds__(512, 1)
           tc_commit(&empty[s]);
         }
       }
-      // make sure everything issued has completed before TMEM is released
+      // make sure everything this thread issued has completed before TMEM is released
       tc_commit(done);
       mbar_wait(done, 0, a_err, DEVERR_WAIT_TEARDOWN);
     }
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp == 3) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegLow) : "memory");
   } else if (warp >= 12) {
     // ------------------------------------------------------------ int4 -> int8 unpack (warps 12..15)
