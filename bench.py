@@ -4,15 +4,17 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 A step is one pass of the hot path over one batch: every projection of the
-workload's layer set goes through the QE forward, in four stages: the
-tensor-core down-projection with the router logits, routing and the bucket
-sort, quantization with the expert-masked adapter rows, and the int8
-tcgen05 product with its adapter epilogue. The step is captured once as a
-CUDA graph with timing events between the stages, and replayed. Inputs are
-synthetic and seeded, with the shapes of the named model (qe_inputs), and
-resident in HBM when the timed region starts. L2 is flushed between steps,
-outside the timed intervals. The step time is the sum of the stage
-intervals. Under torchrun each rank runs an independent replica on its own
+workload's layer set goes through the QE forward, in three stages: the
+tensor-core down-projection with the router logits; routing, the bucket
+sort and quantization with the expert-masked adapter rows (one cooperative
+launch); and the int8 tcgen05 product with its adapter epilogue. The step is captured once as a
+CUDA graph of the public forward calls with a timing event at each end, and
+replayed. Inputs are synthetic and seeded, with the shapes of the named
+model (qe_inputs), and resident in HBM when the timed region starts. L2 is
+flushed between steps, outside the timed intervals. A second graph with
+events between the stages, replayed after the timed region, gives the
+per-stage breakdown (per_projection) and the product kernels' time for the
+roofline. Under torchrun each rank runs an independent replica on its own
 token batch (weak scaling, no data-path collective), and the time is the
 max over ranks. e2e times the plain public call with pinned host buffers
 and the copies inside the timed region.
@@ -281,7 +283,7 @@ def run_ours(args, workload):
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     wonly = cfg.a_bits == 16
-    stages = (qe.QE_STAGE_PROJECT, qe.QE_STAGE_ROUTE, qe.QE_STAGE_QUANT, qe.QE_STAGE_PRODUCT)
+    stages = (qe.QE_STAGE_PROJECT, qe.QE_STAGE_ROUTE | qe.QE_STAGE_QUANT, qe.QE_STAGE_PRODUCT)
 
     def step_plain():
         for L in layers:
@@ -293,14 +295,23 @@ def run_ours(args, workload):
     torch.cuda.synchronize()
     assert qe.device_error() == 0, "a device wait ran out during warm-up"
 
-    # One step = every projection through its four stages, captured once into a CUDA graph
-    # with timing events between the stages. The hot path is a chain of short kernels, so the
-    # graph removes host launch gaps from the device timeline. Each replay is timed by its
-    # own events; they are read back after the replay, outside the timed intervals.
+    # One step = every projection through the public forward call, captured once into a CUDA
+    # graph with one timing event at each end. The hot path is a chain of short kernels, so the
+    # graph removes host launch gaps from the device timeline. Each replay is timed by its own
+    # events, read back after the replay, outside the timed interval.
     cap = torch.cuda.Stream()
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)] for _ in layers]
+    ev0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev1 = torch.cuda.Event(enable_timing=True, external=True)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=cap):
+        ev0.record()
+        step_plain()
+        ev1.record()
+    # A second graph splits each forward into its three stages with events between them; its
+    # replays (after the timed region) give the per-stage breakdown and the product kernels' time.
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)] for _ in layers]
+    sgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(sgraph, stream=cap):
         for L, e in zip(layers, evs):
             e[0].record()
             for i, sm in enumerate(stages):
@@ -308,10 +319,11 @@ def run_ours(args, workload):
                 e[i + 1].record()
     for _ in range(2):
         graph.replay()
+        sgraph.replay()
     torch.cuda.synchronize()
 
     n_proj = len(layers)
-    stage_ms = np.zeros((args.steps, n_proj, len(stages)))
+    step_ms = np.zeros(args.steps)
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
@@ -320,16 +332,22 @@ def run_ours(args, workload):
             flush.zero_()
             graph.replay()
             torch.cuda.synchronize()
-            for p_i, e in enumerate(evs):
-                for k in range(len(stages)):
-                    stage_ms[s_i, p_i, k] = e[k].elapsed_time(e[k + 1])
+            step_ms[s_i] = ev0.elapsed_time(ev1)
     if pg:
         pg.barrier()
+    n_diag = max(3, min(args.steps, 10))
+    stage_ms = np.zeros((n_diag, n_proj, len(stages)))
+    for s_i in range(n_diag):
+        flush.zero_()
+        sgraph.replay()
+        torch.cuda.synchronize()
+        for p_i, e in enumerate(evs):
+            for k in range(len(stages)):
+                stage_ms[s_i, p_i, k] = e[k].elapsed_time(e[k + 1])
     err = qe.device_error()
     assert err == 0, f"device wait ran out (code {err:#x})"
-    del graph
+    del graph, sgraph
 
-    step_ms = stage_ms.sum(axis=(1, 2))
     total_ms = max_over_ranks(float(step_ms.sum()), pg, dev)
     ms_per_step = total_ms / args.steps
     value = world * T * args.steps / (total_ms / 1e3)
@@ -344,7 +362,7 @@ def run_ours(args, workload):
     nbytes = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
                                       cfg.n_routed, cfg.rank_routed, xb, 2) for L in layers)
     peaks = load_peaks()
-    prod_ms = stage_ms[:, :, 3].sum(axis=1).mean()  # the product kernels of one step
+    prod_ms = stage_ms[:, :, 2].sum(axis=1).mean()  # the product kernels of one step
     int8_peak = 2.0 * peaks["bf16_tflops"]           # int8 dense = 2x bf16 dense (nominal ratio)
     decode = T <= 16
     kernel_file = "quantized_gemm_moe_b200/csrc/k_misc.cu" if wonly else "quantized_gemm_moe_b200/csrc/k_gemm.cu"
@@ -369,10 +387,10 @@ def run_ours(args, workload):
         tot = ms.sum()
         per_proj.append({
             "proj": L["proj"].name, "K": K, "N": N, "ms": float(tot),
-            "stage_ms": {"project": float(ms[0]), "route": float(ms[1]), "quant": float(ms[2]), "product": float(ms[3])},
-            "product_tops": (roofline.int_ops(T, K, N) / (ms[3] / 1e3) / 1e12) if not wonly else None,
+            "stage_ms": {"project": float(ms[0]), "route_quant": float(ms[1]), "product": float(ms[2])},
+            "product_tops": (roofline.int_ops(T, K, N) / (ms[2] / 1e3) / 1e12) if not wonly else None,
             "product_gbs": roofline.layer_bytes(T, K, N, cfg.group, cfg.w_bits, cfg.rank_shared, cfg.n_routed,
-                                                cfg.rank_routed, 1 if not wonly else 2, 2) / (ms[3] / 1e3) / 1e9,
+                                                cfg.rank_routed, 1 if not wonly else 2, 2) / (ms[2] / 1e3) / 1e9,
             "layer_tokens_per_s": T / (tot / 1e3),
         })
 

@@ -199,12 +199,12 @@ QE_API qe_status qe_route(const void* X, qe_dtype x_dtype, const void* G, int32_
  *             bytes. Contents on entry are ignored. Calls that share a
  *             workspace must not overlap on the GPU.
  * Steps (all on the GPU): one tensor-core GEMM for the adapter
- * down-projections and the router logits (with the per-token absmax) ->
- * argmin routing and the stable bucket sort -> per-token quantization and the
- * expert-masked adapter rows, in bucket order -> int8 tcgen05 GEMM with
- * per-group scale promotion and the adapter up-projection in its epilogue ->
- * scatter to token order. With a_bits = 16 the main product is the
- * weight-only path.
+ * down-projections and the router logits -> one cooperative launch for the
+ * argmin routing, the per-token absmax and scale, the stable bucket sort,
+ * and the per-token quantization and expert-masked adapter rows in bucket
+ * order -> int8 tcgen05 GEMM with per-group scale promotion and the adapter
+ * up-projection in its epilogue -> scatter to token order. With a_bits = 16
+ * the main product is the weight-only path.
  * T = 0 is a no-op.
  */
 QE_API qe_status qe_linear_forward(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
@@ -216,11 +216,12 @@ QE_API qe_status qe_linear_forward(const qe_layer_desc* desc, const qe_layer_wei
  * bitmask of QE_STAGE_* run in the documented order. Running every stage in
  * separate calls on one stream, with the same workspace, computes exactly
  * what qe_linear_forward computes. A stage reads what earlier stages left in
- * the workspace. Unknown bits -> QE_ERR_INVALID_ARG.
+ * the workspace. ROUTE and QUANT requested together run as one launch.
+ * Unknown bits -> QE_ERR_INVALID_ARG.
  */
-#define QE_STAGE_PROJECT 1 /* tensor-core GEMM: adapter down-projections + router logits, per-token absmax */
-#define QE_STAGE_ROUTE 2   /* argmin routing, per-token scale, stable bucket sort                        */
-#define QE_STAGE_QUANT 4   /* per-token quantization and the expert-masked adapter rows, bucket order   */
+#define QE_STAGE_PROJECT 1 /* tensor-core GEMM: adapter down-projections + router logits                */
+#define QE_STAGE_ROUTE 2   /* argmin routing, per-token absmax and scale, stable bucket sort          */
+#define QE_STAGE_QUANT 4   /* per-token quantization and the expert-masked adapter rows, bucket order */
 #define QE_STAGE_PRODUCT 8 /* main product with the adapter epilogue, scatter to Y                      */
 #define QE_STAGE_ALL 15
 QE_API qe_status qe_linear_forward_stages(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,

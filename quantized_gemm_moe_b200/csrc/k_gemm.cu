@@ -577,7 +577,7 @@ struct UCfg {
 template <int NU>
 __global__ void __launch_bounds__(192, 1)
     k_ugemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_acat, int T, int K,
-            int R_tot, int kchunks_per_split, float* __restrict__ partial, int* a_err) {
+            int R_tot, int kchunks_per_split, float* __restrict__ partial, unsigned* zero_ctr, int* a_err) {
   using C = UCfg<NU>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -594,6 +594,7 @@ __global__ void __launch_bounds__(192, 1)
   const int nk = max(0, min(nk_total, kc_begin + kchunks_per_split) - kc_begin);
 
   if (threadIdx.x == 0) {
+    if (zero_ctr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) *zero_ctr = 0u;
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -715,7 +716,7 @@ cudaError_t launch_qgemm_bn(const CUtensorMap& tm_xq, const CUtensorMap& tm_bcat
 
 template <int NU>
 cudaError_t launch_ugemm_t(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, const UgemmPlan& p, int T, int K,
-                           int R_tot, float* partial, int* err, cudaStream_t st) {
+                           int R_tot, float* partial, unsigned* zero_ctr, int* err, cudaStream_t st) {
   using C = UCfg<NU>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -726,7 +727,8 @@ cudaError_t launch_ugemm_t(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, 
   }
   dim3 grid(static_cast<unsigned>(ceil_div(T, 128)), static_cast<unsigned>(p.ntiles),
             static_cast<unsigned>(p.splits));
-  k_ugemm<NU><<<grid, 192, C::kSmem, st>>>(tm_x, tm_acat, T, K, R_tot, p.kchunks_per_split, partial, err);
+  k_ugemm<NU><<<grid, 192, C::kSmem, st>>>(tm_x, tm_acat, T, K, R_tot, p.kchunks_per_split, partial, zero_ctr,
+                                             err);
   return cudaGetLastError();
 }
 
@@ -789,10 +791,10 @@ UgemmPlan plan_ugemm(int T, int K, int R_tot) {
 }
 
 cudaError_t launch_ugemm(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, const UgemmPlan& plan, int T, int K,
-                         int R_tot, float* partial, int* err, cudaStream_t st) {
+                         int R_tot, float* partial, unsigned* zero_ctr, int* err, cudaStream_t st) {
   switch (plan.nu) {
 #define QE_NU(n) \
-  case n: return launch_ugemm_t<n>(tm_x, tm_acat, plan, T, K, R_tot, partial, err, st);
+  case n: return launch_ugemm_t<n>(tm_x, tm_acat, plan, T, K, R_tot, partial, zero_ctr, err, st);
     QE_NU(16) QE_NU(80) QE_NU(144) QE_NU(208) QE_NU(64) QE_NU(128) QE_NU(192) QE_NU(256)
 #undef QE_NU
     default: return cudaErrorInvalidValue;

@@ -5,6 +5,7 @@
 #include <cuda_fp16.h>
 
 #include "qe_internal.h"
+#include "qe_ptx.cuh"
 
 namespace qe {
 
@@ -75,6 +76,46 @@ __device__ __forceinline__ int rtn_code(float v, float scale, int qmax) {
   float r = rintf(__fdiv_rn(v, scale));
   r = fminf(fmaxf(r, -static_cast<float>(qmax)), static_cast<float>(qmax));
   return static_cast<int>(r);
+}
+
+// Eight codes rtn_code(v[i], scale, qmax), packed little-endian into two words, without a division
+// in the common case. inv = fl32(1/scale), the correctly rounded reciprocal. g = fl32(v*inv) differs
+// from the correctly rounded quotient fl32(v/scale) by at most 3 units of 2^-24 |g|, so rint(g)
+// equals rint(fl32(v/scale)) unless g lies within that distance of a half-integer; the test below
+// asks for a margin of 2^-20 |g| and sends the rest through rtn_code. The fast path also needs a
+// normal scale, and |g| < qmax + 0.5 so that the clamp does not bind (|v| <= absmax keeps
+// |g| <= qmax (1 + 2^-22) when the scale came from this row's absmax).
+// rint uses the 1.5*2^23 trick: fl32(g + 1.5*2^23) holds rint(g) (half to even) in its low bits.
+__device__ __forceinline__ void rtn_code8(const float (&v)[8], float scale, float inv, bool fast, int qmax,
+                                          uint32_t& w0, uint32_t& w1) {
+  constexpr float kM = 12582912.0f;
+  const float qmax_f = static_cast<float>(qmax) + 0.5f;
+  uint32_t b[8];
+  bool ok = fast;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float g = __fmul_rn(v[i], inv);
+    const float t = __fadd_rn(g, kM);
+    const float d = fabsf(__fsub_rn(g, __fsub_rn(t, kM)));
+    ok = ok && (__fmaf_rn(fabsf(g), 9.5367431640625e-07f, d) < 0.5f) && (fabsf(g) < qmax_f);
+    b[i] = __float_as_uint(t);
+  }
+  if (ok) {
+    w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+    return;
+  }
+  w0 = 0;
+  w1 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    w0 |= (static_cast<uint32_t>(rtn_code(v[i], scale, qmax)) & 0xFFu) << (8 * i);
+    w1 |= (static_cast<uint32_t>(rtn_code(v[4 + i], scale, qmax)) & 0xFFu) << (8 * i);
+  }
+}
+// Whether rtn_code8's fast path may be used for this scale (and its reciprocal).
+__device__ __forceinline__ bool rtn_fast_ok(float scale, float inv) {
+  return scale >= 1.17549435e-38f && inv < 3.0e38f;
 }
 
 // ------------------------------------------------------------------ router + absmax
@@ -217,6 +258,8 @@ __global__ void __launch_bounds__(256) k_act_quant(const void* __restrict__ X, c
   const int t = blockIdx.x;
   const size_t p = pos ? static_cast<size_t>(pos[t]) : static_cast<size_t>(t);
   const float sa = sa_tok ? sa_tok[t] : 0.0f;
+  const float inv = (sa > 0.0f) ? __frcp_rn(sa) : 0.0f;
+  const bool fast = rtn_fast_ok(sa, inv);
   for (int k0 = threadIdx.x * 8; k0 < K; k0 += blockDim.x * 8) {
     float xv[8], si[8];
     load8<BF16>(X, t, K, k0, xv);
@@ -225,12 +268,8 @@ __global__ void __launch_bounds__(256) k_act_quant(const void* __restrict__ X, c
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(xv[i], si[i]);
     if (codes) {
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        w0 |= (static_cast<uint32_t>(rtn_code(v[i], sa, qmax)) & 0xFFu) << (8 * i);
-        w1 |= (static_cast<uint32_t>(rtn_code(v[4 + i], sa, qmax)) & 0xFFu) << (8 * i);
-      }
+      uint32_t w0, w1;
+      rtn_code8(v, sa, inv, fast, qmax, w0, w1);
       *reinterpret_cast<uint2*>(codes + p * K + k0) = make_uint2(w0, w1);
     }
     if (act16) {
@@ -465,128 +504,343 @@ __global__ void k_split_f32(const float* __restrict__ X, const float* __restrict
   if (lane == 0) amax[t] = mx;
 }
 
-// Per token (one warp): router logits from the GEMM partials, argmin with the lowest index on
-// exact ties, and sa = fl32(max_k |fl32(x*s_inv)| / qmax). The absmax is read from X for bf16
-// inputs, or taken from amax[t] (fp32 inputs, computed by k_split_f32).
-template <bool BF16>
-__global__ void k_tokfinal(const float* __restrict__ partial, int nslots, int R_tot, int R_pad, int n_r,
-                           const void* __restrict__ X, const float* __restrict__ s_inv, int K,
-                           const float* __restrict__ amax, int qmax, int T, int32_t* __restrict__ expert,
-                           float* __restrict__ sa_tok, float* __restrict__ logits) {
-  const int t = static_cast<int>((blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  float L = 0.0f;
-  if (lane < n_r)
-    for (int s2 = 0; s2 < nslots; ++s2) L += __ldg(partial + (static_cast<size_t>(s2) * T + t) * R_tot + R_pad + lane);
-  float best = (lane < n_r) ? L : INFINITY;
-  int bi = (lane < n_r) ? lane : 0x7fffffff;
+// Sum over the GEMM's partial slots of one value, p[s * slot_stride] for s < nslots, in slot
+// order, with eight loads in flight. The padding terms are +0.0f and leave the sum unchanged.
+__device__ __forceinline__ float slot_sum(const float* __restrict__ p, size_t slot_stride, int nslots) {
+  float acc = 0.0f;
+  for (int s = 0; s < nslots; s += 8) {
+    float v[8];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, best, off);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-    if (ov < best || (ov == best && oi < bi)) {
-      best = ov;
-      bi = oi;
+    for (int i = 0; i < 8; ++i) v[i] = (s + i < nslots) ? __ldg(p + static_cast<size_t>(s + i) * slot_stride) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc += v[i];
+  }
+  return acc;
+}
+
+// Grid-wide barrier for a cooperative launch: every CTA is resident, so each waits until all
+// have arrived. *ctr must be 0 when the kernel starts. The wait gives up after about two
+// seconds of clock cycles, records an error and returns false.
+__device__ bool grid_barrier(unsigned* ctr, int* err) {
+  __shared__ int ok_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    int ok = 1;
+    const long long t0 = clock64();
+    while (true) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+      if (v >= gridDim.x) break;
+      if (clock64() - t0 > 4000000000ll) {
+        record_error(err, DEVERR_GRID_BARRIER);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+// Routing, stable bucket sort and activation quantization of one layer call, in one cooperative
+// launch. CTA c owns the contiguous token range [c*chunk, (c+1)*chunk), one warp per token.
+//  route:  logits = sum of the U GEMM partial slots in columns [R_pad, R_pad+N_r); expert[t] =
+//          argmin (lowest index on exact ties); sa_tok[t] = fl32(max_k |fl32(x*s_inv)| / qmax), the
+//          absmax read from X (bf16 inputs) or amax[t] (fp32 inputs); per-CTA expert counts.
+//  (grid barrier)
+//  sort:   each CTA adds the counts of all experts before e and of all earlier CTAs for e, then
+//          ranks its own tokens in token order (warp ballots), so the sort is stable:
+//          perm[p] = t, pos[t] = p, offsets[e].
+//  quant:  at row p = pos[t]: the activation codes (or bf16(x*s_inv) for weight-only layers),
+//          sa_sorted[p], and U_cat[p] = fp16((sum of U slots, routed columns of the other experts
+//          zeroed) / su[p]), su[p] a power of two that puts the row's largest |U| in [2^13, 2^14).
+struct RouteQuantArgs {
+  const float* partial;
+  int nslots, R_tot, R_pad, n_r, r_s, r_r, R_a;
+  const void* X;
+  const float* s_inv;
+  const float* amax;
+  int T, K, qmax, chunk;
+  int do_route, do_quant;
+  int32_t* expert;
+  float* sa_tok;
+  int32_t* perm;
+  int32_t* pos;
+  int32_t* offsets;
+  int32_t* counts;  // [gridDim.x][kMaxRouted]
+  unsigned* barrier;
+  int8_t* codes;
+  uint16_t* act16;
+  float* sa_sorted;
+  uint16_t* ucat;
+  float* su_sorted;
+  int* err;
+};
+
+constexpr int kRQThreads = 512;
+// Row loads in flight per lane: 8 x 16 B of a bf16 row, 4 x 32 B of an fp32 row.
+template <bool BF16>
+struct RowBatch {
+  static constexpr int kIters = BF16 ? 8 : 4;
+};
+
+// Raw bytes of x[t][k0 .. k0+8) for the batch's iterations (k0 = lane*8 + 256*j), loaded first so
+// that every load of the batch is in flight before any is used.
+template <bool BF16>
+struct RowRaw {
+  uint4 v[RowBatch<BF16>::kIters][BF16 ? 1 : 2];
+};
+template <bool BF16>
+__device__ __forceinline__ void row_load(const void* X, size_t t, int K, int k0, RowRaw<BF16>& r) {
+#pragma unroll
+  for (int j = 0; j < RowBatch<BF16>::kIters; ++j) {
+    const int k = k0 + 256 * j;
+    if (k < K) {
+      if constexpr (BF16) {
+        r.v[j][0] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(X) + t * K + k));
+      } else {
+        const uint4* q = reinterpret_cast<const uint4*>(static_cast<const float*>(X) + t * K + k);
+        r.v[j][0] = __ldg(q);
+        r.v[j][1] = __ldg(q + 1);
+      }
     }
   }
-  float mx = 0.0f;
-  if (sa_tok) {
-    if (BF16) {
-      for (int k0 = lane * 8; k0 < K; k0 += 256) {
-        float xv[8], si[8];
-        load8<true>(X, t, K, k0, xv);
-        load8f(s_inv + k0, si);
+}
+// v[i] = fl32(x[k+i] * s_inv[k+i]) for iteration j of the batch (s_inv from shared memory).
+template <bool BF16>
+__device__ __forceinline__ void row_scaled(const RowRaw<BF16>& r, int j, const float* s_inv_s, int k, float (&v)[8]) {
+  float xv[8];
+  if constexpr (BF16) {
+    const uint32_t w[4] = {r.v[j][0].x, r.v[j][0].y, r.v[j][0].z, r.v[j][0].w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(__fmul_rn(xv[i], si[i])));
+    for (int i = 0; i < 4; ++i) {
+      xv[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+      xv[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+    }
+  } else {
+    const uint4 a0 = r.v[j][0], a1 = r.v[j][1];
+    xv[0] = __uint_as_float(a0.x); xv[1] = __uint_as_float(a0.y); xv[2] = __uint_as_float(a0.z); xv[3] = __uint_as_float(a0.w);
+    xv[4] = __uint_as_float(a1.x); xv[5] = __uint_as_float(a1.y); xv[6] = __uint_as_float(a1.z); xv[7] = __uint_as_float(a1.w);
+  }
+  const float4 s0 = *reinterpret_cast<const float4*>(s_inv_s + k);
+  const float4 s1 = *reinterpret_cast<const float4*>(s_inv_s + k + 4);
+  const float si[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(xv[i], si[i]);
+}
+
+// Dynamic shared memory of k_route_quant: s_inv (K floats), then the range's expert ids and bucket
+// positions (chunk ints each).
+size_t route_quant_smem(int K, int chunk) { return size_t(K) * 4 + size_t(chunk) * 8; }
+
+template <bool BF16>
+__global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs a) {
+  constexpr int kWarps = kRQThreads / 32;
+  constexpr int kB = RowBatch<BF16>::kIters;
+  __shared__ int wcnt[kWarps][kMaxRouted], wbase[kWarps][kMaxRouted];
+  __shared__ int tot_s[kMaxRouted], before_s[kMaxRouted], run_s[kMaxRouted];
+  extern __shared__ float4 rq_dyn[];
+  float* s_inv_s = reinterpret_cast<float*>(rq_dyn);
+  int* e_s = reinterpret_cast<int*>(s_inv_s + a.K);
+  int* pos_s = e_s + a.chunk;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = min(a.T, static_cast<int>(blockIdx.x) * a.chunk), t1 = min(a.T, t0 + a.chunk);
+  const int n_r = a.n_r;
+  for (int i = threadIdx.x; i < a.K / 4; i += kRQThreads)
+    reinterpret_cast<float4*>(s_inv_s)[i] = __ldg(reinterpret_cast<const float4*>(a.s_inv) + i);
+  __syncthreads();
+
+  if (a.do_route) {
+    // ---- per token: logits, argmin, absmax
+    const size_t slot_stride = static_cast<size_t>(a.T) * a.R_tot;
+    for (int t = t0 + warp; t < t1; t += kWarps) {
+      const float L = (lane < n_r)
+                          ? slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_pad + lane, slot_stride, a.nslots)
+                          : 0.0f;
+      float best = (lane < n_r) ? L : INFINITY;
+      int bi = (lane < n_r) ? lane : 0x7fffffff;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (ov < best || (ov == best && oi < bi)) {
+          best = ov;
+          bi = oi;
+        }
+      }
+      if (a.sa_tok) {
+        float mx = 0.0f;
+        if (BF16) {
+          for (int k0 = lane * 8; k0 < a.K; k0 += 256 * kB) {
+            RowRaw<true> r;
+            row_load<true>(a.X, t, a.K, k0, r);
+#pragma unroll
+            for (int j = 0; j < kB; ++j) {
+              const int k = k0 + 256 * j;
+              if (k < a.K) {
+                float v[8];
+                row_scaled<true>(r, j, s_inv_s, k, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
+              }
+            }
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        } else {
+          mx = a.amax[t];
+        }
+        if (lane == 0) a.sa_tok[t] = __fdiv_rn(mx, static_cast<float>(a.qmax));
+      }
+      if (lane == 0) {
+        a.expert[t] = bi;
+        e_s[t - t0] = bi;
+      }
+    }
+    __syncthreads();
+    // ---- this CTA's count per expert
+    if (warp < n_r) {
+      int c = 0;
+      for (int i = lane; i < t1 - t0; i += 32) c += (e_s[i] == warp) ? 1 : 0;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+      if (lane == 0) a.counts[blockIdx.x * kMaxRouted + warp] = c;
+    }
+    if (!grid_barrier(a.barrier, a.err)) return;
+    // ---- bucket offsets: experts before e, plus earlier CTAs' tokens of e
+    if (warp < n_r) {
+      int tot = 0, before = 0;
+#pragma unroll 8
+      for (int c = lane; c < static_cast<int>(gridDim.x); c += 32) {
+        const int v = __ldcg(a.counts + c * kMaxRouted + warp);
+        tot += v;
+        before += (c < static_cast<int>(blockIdx.x)) ? v : 0;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        tot += __shfl_xor_sync(0xffffffffu, tot, off);
+        before += __shfl_xor_sync(0xffffffffu, before, off);
+      }
+      if (lane == 0) {
+        tot_s[warp] = tot;
+        before_s[warp] = before;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < n_r) {
+      int start = 0;
+      for (int e = 0; e < static_cast<int>(threadIdx.x); ++e) start += tot_s[e];
+      run_s[threadIdx.x] = start + before_s[threadIdx.x];
+      if (blockIdx.x == 0) {
+        a.offsets[threadIdx.x] = start;
+        if (threadIdx.x == n_r - 1) a.offsets[n_r] = start + tot_s[threadIdx.x];
+      }
+    }
+    __syncthreads();
+    // ---- stable ranks inside this CTA's range, kRQThreads tokens at a time
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int c0 = t0; c0 < t1; c0 += kRQThreads) {
+      const int t = c0 + static_cast<int>(threadIdx.x);
+      const int e = (t < t1) ? e_s[t - t0] : -1;
+      int rank = 0;
+      for (int ee = 0; ee < n_r; ++ee) {
+        const uint32_t m = __ballot_sync(0xffffffffu, e == ee);
+        if (lane == 0) wcnt[warp][ee] = __popc(m);
+        if (e == ee) rank = __popc(m & lt_mask);
+      }
+      __syncthreads();
+      if (threadIdx.x < n_r) {
+        int run = run_s[threadIdx.x];
+        for (int w = 0; w < kWarps; ++w) {
+          wbase[w][threadIdx.x] = run;
+          run += wcnt[w][threadIdx.x];
+        }
+        run_s[threadIdx.x] = run;
+      }
+      __syncthreads();
+      if (t < t1) {
+        const int p = wbase[warp][e] + rank;
+        a.perm[p] = t;
+        a.pos[t] = p;
+        pos_s[t - t0] = p;
+      }
+      __syncthreads();
+    }
+  } else if (a.do_quant) {
+    for (int i = threadIdx.x; i < t1 - t0; i += kRQThreads) {
+      pos_s[i] = a.pos[t0 + i];
+      e_s[i] = a.expert[t0 + i];
+    }
+    __syncthreads();
+  }
+  if (!a.do_quant) return;
+  // ---- per token, in bucket order
+  for (int t = t0 + warp; t < t1; t += kWarps) {
+    const size_t p = static_cast<size_t>(pos_s[t - t0]);
+    const float sa = a.codes ? a.sa_tok[t] : 0.0f;
+    const float inv = (sa > 0.0f) ? __frcp_rn(sa) : 0.0f;
+    const bool fast = rtn_fast_ok(sa, inv);
+    for (int k0 = lane * 8; k0 < a.K; k0 += 256 * kB) {
+      RowRaw<BF16> r;
+      row_load<BF16>(a.X, t, a.K, k0, r);
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        const int k = k0 + 256 * j;
+        if (k >= a.K) break;
+        float v[8];
+        row_scaled<BF16>(r, j, s_inv_s, k, v);
+        if (a.codes) {
+          uint32_t w0, w1;
+          rtn_code8(v, sa, inv, fast, a.qmax, w0, w1);
+          *reinterpret_cast<uint2*>(a.codes + p * a.K + k) = make_uint2(w0, w1);
+        } else {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            w[i] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i])) |
+                   (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i + 1])) << 16);
+          *reinterpret_cast<uint4*>(a.act16 + p * a.K + k) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    if (a.codes && lane == 0) a.sa_sorted[p] = sa;
+    if (a.R_pad > 0) {
+      const int e = e_s[t - t0];
+      constexpr int kMaxPerLane = 512 / 32;
+      float u[kMaxPerLane];
+      float mx = 0.0f;
+#pragma unroll
+      for (int i = 0; i < kMaxPerLane; ++i) {
+        const int c = lane + 32 * i;
+        float a2 = 0.0f;
+        if (c < a.R_a && (c < a.r_s || (c - a.r_s) / a.r_r == e))
+          a2 = slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + c, static_cast<size_t>(a.T) * a.R_tot, a.nslots);
+        u[i] = a2;
+        mx = fmaxf(mx, fabsf(a2));
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    } else {
-      mx = amax[t];
-    }
-  }
-  if (logits && lane < n_r) logits[static_cast<size_t>(t) * n_r + lane] = L;
-  if (lane == 0) {
-    expert[t] = bi;
-    if (sa_tok) sa_tok[t] = __fdiv_rn(mx, static_cast<float>(qmax));
-  }
-}
-
-// Per token (one warp), in bucket order p = pos[t]: the activation codes (or the bf16
-// activations of weight-only layers), sa_sorted[p], and the adapter row U_cat[p]: the sum of
-// the GEMM partial slots, with the routed columns of every other expert zeroed, in fp16 after
-// division by su[p], a power of two that puts the row's largest |U| in [2^13, 2^14).
-template <bool BF16>
-__global__ void __launch_bounds__(256) k_quant_u(const void* __restrict__ X, const float* __restrict__ s_inv, int T,
-                                                 int K, int qmax, const float* __restrict__ sa_tok,
-                                                 const int32_t* __restrict__ pos, const int32_t* __restrict__ expert,
-                                                 int8_t* __restrict__ codes, uint16_t* __restrict__ act16,
-                                                 float* __restrict__ sa_sorted, const float* __restrict__ partial,
-                                                 int nslots, int R_tot, int R_pad, int r_s, int r_r, int R_a,
-                                                 uint16_t* __restrict__ ucat, float* __restrict__ su_sorted) {
-  const int t = static_cast<int>((blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  const size_t p = static_cast<size_t>(pos[t]);
-  const float sa = sa_tok ? sa_tok[t] : 0.0f;
-  for (int k0 = lane * 8; k0 < K; k0 += 256) {
-    float xv[8], si[8], v[8];
-    load8<BF16>(X, t, K, k0, xv);
-    load8f(s_inv + k0, si);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(xv[i], si[i]);
-    if (codes) {
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        w0 |= (static_cast<uint32_t>(rtn_code(v[i], sa, qmax)) & 0xFFu) << (8 * i);
-        w1 |= (static_cast<uint32_t>(rtn_code(v[4 + i], sa, qmax)) & 0xFFu) << (8 * i);
+      float su = 1.0f;
+      if (mx > 0.0f) {
+        int ex;
+        frexpf(mx, &ex);  // mx = m * 2^ex, m in [0.5, 1)
+        su = ldexpf(1.0f, ex - 14);
       }
-      *reinterpret_cast<uint2*>(codes + p * K + k0) = make_uint2(w0, w1);
-    } else {
-      uint32_t w[4];
+      const float inv_su = 1.0f / su;  // exact: su is a power of two
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        w[i] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i])) |
-               (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i + 1])) << 16);
-      *reinterpret_cast<uint4*>(act16 + p * K + k0) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
-  if (codes && lane == 0) sa_sorted[p] = sa;
-  if (R_pad > 0) {
-    const int e = expert[t];
-    constexpr int kMaxPerLane = 512 / 32;
-    float u[kMaxPerLane];
-    float mx = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
-      const int c = lane + 32 * i;
-      float a2 = 0.0f;
-      if (c < R_a && (c < r_s || (c - r_s) / r_r == e)) {
-        for (int s2 = 0; s2 < nslots; ++s2) a2 += __ldg(partial + (static_cast<size_t>(s2) * T + t) * R_tot + c);
+      for (int i = 0; i < kMaxPerLane; ++i) {
+        const int c = lane + 32 * i;
+        if (c < a.R_pad) {
+          __half h = __float2half_rn(u[i] * inv_su);
+          a.ucat[p * a.R_pad + c] = *reinterpret_cast<uint16_t*>(&h);
+        }
       }
-      u[i] = a2;
-      mx = fmaxf(mx, fabsf(a2));
+      if (lane == 0) a.su_sorted[p] = su;
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float su = 1.0f;
-    if (mx > 0.0f) {
-      int ex;
-      frexpf(mx, &ex);  // mx = m * 2^ex, m in [0.5, 1)
-      su = ldexpf(1.0f, ex - 14);
-    }
-    const float inv = 1.0f / su;  // exact: su is a power of two
-#pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
-      const int c = lane + 32 * i;
-      if (c < R_pad) {
-        __half h = __float2half_rn(u[i] * inv);
-        ucat[p * R_pad + c] = *reinterpret_cast<uint16_t*>(&h);
-      }
-    }
-    if (lane == 0) su_sorted[p] = su;
   }
 }
 
@@ -685,34 +939,77 @@ cudaError_t launch_split_f32(const float* X, const float* s_inv, int T, int K, u
   return cudaGetLastError();
 }
 
-cudaError_t launch_tokfinal(const float* partial, int nslots, int R_tot, int R_pad, int n_r, const void* X,
-                            bool x_bf16, const float* s_inv, int K, const float* amax, int qmax, int T,
-                            int32_t* expert, float* sa_tok, float* logits, cudaStream_t st) {
-  if (T == 0) return cudaSuccess;
-  const unsigned grid = static_cast<unsigned>(ceil_div(T, 8));
-  if (x_bf16)
-    k_tokfinal<true><<<grid, 256, 0, st>>>(partial, nslots, R_tot, R_pad, n_r, X, s_inv, K, amax, qmax, T, expert,
-                                           sa_tok, logits);
-  else
-    k_tokfinal<false><<<grid, 256, 0, st>>>(partial, nslots, R_tot, R_pad, n_r, X, s_inv, K, amax, qmax, T, expert,
-                                            sa_tok, logits);
-  return cudaGetLastError();
+constexpr int kRQMaxSmem = 200 * 1024;
+
+int route_quant_grid() {
+  static int grid = 0;
+  if (grid == 0) {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 0;
+    if (cudaFuncSetAttribute(k_route_quant<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRQMaxSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(k_route_quant<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRQMaxSmem) !=
+            cudaSuccess)
+      return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_route_quant<true>, kRQThreads, kRQMaxSmem) !=
+            cudaSuccess ||
+        per_sm < 1)
+      return 0;
+    grid = std::min(sms, kRouteQuantMaxGrid);
+  }
+  return grid;
 }
 
-cudaError_t launch_quant_u(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
-                           const float* sa_tok, const int32_t* pos, const int32_t* expert, int8_t* codes,
-                           uint16_t* act16, float* sa_sorted, const float* partial, int nslots, int R_tot,
-                           int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, float* su_sorted, cudaStream_t st) {
-  if (T == 0) return cudaSuccess;
-  const unsigned grid = static_cast<unsigned>(ceil_div(T, 8));
-  if (x_bf16)
-    k_quant_u<true><<<grid, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, expert, codes, act16, sa_sorted, partial,
-                                          nslots, R_tot, R_pad, r_s, r_r > 0 ? r_r : 1, R_a, ucat, su_sorted);
-  else
-    k_quant_u<false><<<grid, 256, 0, st>>>(X, s_inv, T, K, qmax, sa_tok, pos, expert, codes, act16, sa_sorted,
-                                           partial, nslots, R_tot, R_pad, r_s, r_r > 0 ? r_r : 1, R_a, ucat,
-                                           su_sorted);
-  return cudaGetLastError();
+cudaError_t launch_route_quant(const RouteQuantParams& q, cudaStream_t st) {
+  if (q.T == 0) return cudaSuccess;
+  const int grid = route_quant_grid();
+  if (grid == 0) return cudaErrorInvalidConfiguration;
+  RouteQuantArgs a{};
+  a.partial = q.partial;
+  a.nslots = q.nslots;
+  a.R_tot = q.R_tot;
+  a.R_pad = q.R_pad;
+  a.n_r = q.n_r;
+  a.r_s = q.r_s;
+  a.r_r = q.r_r > 0 ? q.r_r : 1;
+  a.R_a = q.R_a;
+  a.X = q.X;
+  a.s_inv = q.s_inv;
+  a.amax = q.amax;
+  a.T = q.T;
+  a.K = q.K;
+  a.qmax = q.qmax;
+  a.chunk = static_cast<int>(ceil_div(q.T, grid));
+  const size_t smem = route_quant_smem(q.K, a.chunk);
+  if (smem > static_cast<size_t>(kRQMaxSmem)) return cudaErrorInvalidValue;
+  a.do_route = q.do_route;
+  a.do_quant = q.do_quant;
+  a.expert = q.expert;
+  a.sa_tok = q.sa_tok;
+  a.perm = q.perm;
+  a.pos = q.pos;
+  a.offsets = q.offsets;
+  a.counts = q.counts;
+  a.barrier = q.barrier;
+  a.codes = q.codes;
+  a.act16 = q.act16;
+  a.sa_sorted = q.sa_sorted;
+  a.ucat = q.ucat;
+  a.su_sorted = q.su_sorted;
+  a.err = q.err;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kRQThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (q.x_bf16) return cudaLaunchKernelEx(&cfg, k_route_quant<true>, a);
+  return cudaLaunchKernelEx(&cfg, k_route_quant<false>, a);
 }
 
 cudaError_t launch_splitk_reduce(const float* partial, int splits, const int32_t* perm, int T, int N, void* Y,

@@ -65,7 +65,7 @@ struct Plan {
   int bn, msplits, kbps;  // main product
   int uslots;             // GEMM partial slots: splits, doubled for fp32 inputs (hi and lo passes)
   size_t off_expert, off_perm, off_pos, off_offsets, off_sa_tok, off_sa_sorted, off_su_sorted, off_act, off_xhi,
-      off_xlo, off_amax, off_upart, off_ucat, off_ypart, bytes;
+      off_xlo, off_amax, off_upart, off_ucat, off_ypart, off_counts, off_barrier, bytes;
 };
 
 int wonly_splits(int T, int N, int K) {
@@ -115,6 +115,8 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   p.off_upart = take(size_t(p.uslots) * Tm * p.g.R_tot * 4);
   p.off_ucat = p.has_ad ? take(size_t(Tm) * p.g.R_pad * 2) : 0;
   p.off_ypart = (p.msplits > 1) ? take(size_t(p.msplits) * Tm * p.N * 4) : 0;
+  p.off_counts = take(size_t(kRouteQuantMaxGrid) * kMaxRouted * 4);
+  p.off_barrier = take(4);
   p.bytes = o;
   return p;
 }
@@ -195,8 +197,16 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   const int qmax = wonly ? 1 : qmax_of(d->a_bits);
   const int K = p.K, N = p.N;
 
+  unsigned* barrier = at<unsigned>(ws, p.off_barrier);
+  int8_t* codes = wonly ? nullptr : at<int8_t>(ws, p.off_act);
+  uint16_t* act16 = wonly ? at<uint16_t>(ws, p.off_act) : nullptr;
+  uint16_t* ucat = p.has_ad ? at<uint16_t>(ws, p.off_ucat) : nullptr;
+
   // 1. one tensor-core GEMM: adapter down-projections + router logits
-  if (stages & QE_STAGE_PROJECT) {
+  //    (its first CTA also clears the grid barrier of step 2)
+  const bool project = (stages & QE_STAGE_PROJECT) != 0;
+  const bool route = (stages & QE_STAGE_ROUTE) != 0, quant = (stages & QE_STAGE_QUANT) != 0;
+  if (project) {
     CUtensorMap tm_acat;
     if ((s = make_tmap(&tm_acat, acat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, p.g.R_tot, kAdapterAtom, p.up.nu)) !=
         QE_OK)
@@ -204,7 +214,7 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
     if (x_bf16) {
       CUtensorMap tm_x;
       if ((s = make_tmap(&tm_x, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK) return s;
-      QE_CUDA(launch_ugemm(tm_x, tm_acat, p.up, T, K, p.g.R_tot, upart, err, st), "ugemm");
+      QE_CUDA(launch_ugemm(tm_x, tm_acat, p.up, T, K, p.g.R_tot, upart, barrier, err, st), "ugemm");
     } else {
       // fp32 input: x = hi + lo in bf16, two passes into consecutive partial slots
       uint16_t* xhi = at<uint16_t>(ws, p.off_xhi);
@@ -213,28 +223,49 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
       CUtensorMap tm_hi, tm_lo;
       if ((s = make_tmap(&tm_hi, xhi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK) return s;
       if ((s = make_tmap(&tm_lo, xlo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, kAdapterAtom, 128)) != QE_OK) return s;
-      QE_CUDA(launch_ugemm(tm_hi, tm_acat, p.up, T, K, p.g.R_tot, upart, err, st), "ugemm_hi");
+      QE_CUDA(launch_ugemm(tm_hi, tm_acat, p.up, T, K, p.g.R_tot, upart, barrier, err, st), "ugemm_hi");
       QE_CUDA(launch_ugemm(tm_lo, tm_acat, p.up, T, K, p.g.R_tot, upart + size_t(p.up.splits) * T * p.g.R_tot,
-                           err, st),
+                           nullptr, err, st),
               "ugemm_lo");
     }
   }
-  // 2. argmin routing, per-token absmax and scale, stable bucket sort
-  if (stages & QE_STAGE_ROUTE) {
-    QE_CUDA(launch_tokfinal(upart, p.uslots, p.g.R_tot, p.g.R_pad, d->n_routed, X, x_bf16, w->s_inv, K, amax, qmax,
-                            T, expert, wonly ? nullptr : sa_tok, nullptr, st),
-            "tokfinal");
-    QE_CUDA(launch_bucket(expert, T, d->n_routed, perm, pos, offsets, st), "bucket");
+  // 2. argmin routing, per-token absmax and scale, stable bucket sort, then quantization in bucket
+  //    order and the expert-masked adapter rows U_cat: one cooperative launch
+  if (route || quant) {
+    if (route && !project) QE_CUDA(cudaMemsetAsync(barrier, 0, 4, st), "memset");
+    RouteQuantParams q{};
+    q.partial = upart;
+    q.nslots = p.uslots;
+    q.R_tot = p.g.R_tot;
+    q.R_pad = p.g.R_pad;
+    q.n_r = d->n_routed;
+    q.r_s = d->rank_shared;
+    q.r_r = d->rank_routed;
+    q.R_a = p.g.R_a;
+    q.X = X;
+    q.x_bf16 = x_bf16;
+    q.s_inv = w->s_inv;
+    q.amax = amax;
+    q.T = T;
+    q.K = K;
+    q.qmax = qmax;
+    q.do_route = route;
+    q.do_quant = quant;
+    q.expert = expert;
+    q.sa_tok = wonly ? nullptr : sa_tok;
+    q.perm = perm;
+    q.pos = pos;
+    q.offsets = offsets;
+    q.counts = at<int32_t>(ws, p.off_counts);
+    q.barrier = barrier;
+    q.codes = codes;
+    q.act16 = act16;
+    q.sa_sorted = sa_sorted;
+    q.ucat = ucat;
+    q.su_sorted = su_sorted;
+    q.err = err;
+    QE_CUDA(launch_route_quant(q, st), "route_quant");
   }
-  // 3. quantize in bucket order, and the expert-masked adapter rows U_cat
-  int8_t* codes = wonly ? nullptr : at<int8_t>(ws, p.off_act);
-  uint16_t* act16 = wonly ? at<uint16_t>(ws, p.off_act) : nullptr;
-  uint16_t* ucat = p.has_ad ? at<uint16_t>(ws, p.off_ucat) : nullptr;
-  if (stages & QE_STAGE_QUANT)
-    QE_CUDA(launch_quant_u(X, x_bf16, w->s_inv, T, K, qmax, wonly ? nullptr : sa_tok, pos, expert, codes, act16,
-                           sa_sorted, upart, p.uslots, p.g.R_tot, p.g.R_pad, d->rank_shared, d->rank_routed, p.g.R_a,
-                           ucat, su_sorted, st),
-            "quant_u");
   // 5. main product
   if (!(stages & QE_STAGE_PRODUCT)) return QE_OK;
   float* ypart = p.msplits > 1 ? at<float>(ws, p.off_ypart) : nullptr;
@@ -417,7 +448,7 @@ int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, qe_dtype
   if (T == 0) return 0;
   const Plan p = make_plan(desc, T, x_dtype == QE_BF16);
   int n = (x_dtype == QE_BF16) ? 1 : 3;  // down-projection GEMM (fp32 inputs: split + hi and lo passes)
-  n += 3;                                // tokfinal, bucket, quant_u
+  n += 1;                                // routing + bucket sort + quantization (cooperative)
   n += 1;                                // main product (int8 GEMM or weight-only)
   if (p.msplits > 1) n += 1;             // split-K reduce
   return n;

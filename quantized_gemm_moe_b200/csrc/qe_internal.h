@@ -86,20 +86,40 @@ struct UgemmPlan {
   int ntiles;
 };
 UgemmPlan plan_ugemm(int T, int K, int R_tot);
+// zero_ctr != nullptr: the first CTA also sets *zero_ctr = 0 (the route/quant launch's barrier).
 cudaError_t launch_ugemm(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, const UgemmPlan& plan, int T,
-                         int K, int R_tot, float* partial, int* err, cudaStream_t st);
-// Per token: logits = sum over slots, expert = argmin (lowest index on ties); sa = absmax / qmax, with
-// the absmax max_k |fl32(x*s_inv)| taken from X (bf16 inputs) or from amax[t] (fp32 inputs, from
-// launch_split_f32). sa_tok == nullptr skips the scale.
-cudaError_t launch_tokfinal(const float* partial, int nslots, int R_tot, int R_pad, int n_r, const void* X,
-                            bool x_bf16, const float* s_inv, int K, const float* amax, int qmax, int T,
-                            int32_t* expert, float* sa_tok, float* logits, cudaStream_t st);
-// Per token, in bucket order p = pos[t]: activation codes (or bf16 activations), sa_sorted, and
-// U_cat[p] = fp16((sum of U slots, routed columns of other experts zeroed) / su[p]).
-cudaError_t launch_quant_u(const void* X, bool x_bf16, const float* s_inv, int T, int K, int qmax,
-                           const float* sa_tok, const int32_t* pos, const int32_t* expert, int8_t* codes,
-                           uint16_t* act16, float* sa_sorted, const float* partial, int nslots, int R_tot,
-                           int R_pad, int r_s, int r_r, int R_a, uint16_t* ucat, float* su_sorted, cudaStream_t st);
+                         int K, int R_tot, float* partial, unsigned* zero_ctr, int* err, cudaStream_t st);
+// Routing, stable bucket sort and activation quantization in one cooperative launch (grid barrier
+// between the per-token routing and the sort). route: expert = argmin of the router logits (sum of
+// the U partial slots, columns [R_pad, R_pad+N_r)), sa_tok = absmax/qmax (absmax from X for bf16
+// inputs, amax[t] for fp32 inputs; sa_tok == nullptr for weight-only layers), perm/pos/offsets.
+// quant: codes (or bf16 act16) at row pos[t], sa_sorted, and U_cat / su_sorted.
+// *barrier must be 0 when the launch starts.
+constexpr int kRouteQuantMaxGrid = 1024;
+struct RouteQuantParams {
+  const float* partial;
+  int nslots, R_tot, R_pad, n_r, r_s, r_r, R_a;
+  const void* X;
+  bool x_bf16;
+  const float* s_inv;
+  const float* amax;
+  int T, K, qmax;
+  int do_route, do_quant;
+  int32_t* expert;
+  float* sa_tok;
+  int32_t* perm;
+  int32_t* pos;
+  int32_t* offsets;
+  int32_t* counts;  // [kRouteQuantMaxGrid][kMaxRouted]
+  unsigned* barrier;
+  int8_t* codes;
+  uint16_t* act16;
+  float* sa_sorted;
+  uint16_t* ucat;
+  float* su_sorted;
+  int* err;
+};
+cudaError_t launch_route_quant(const RouteQuantParams& q, cudaStream_t st);
 
 // Main quantized GEMM (W4 x A8/A6 codes, tcgen05 kind::i8) with per-group promotion,
 // per-token scale, adapter MMA in the epilogue and scatter to token order.

@@ -19,6 +19,7 @@ enum : int {
   DEVERR_WAIT_MMA = 0x103,
   DEVERR_WAIT_EPILOGUE = 0x104,
   DEVERR_WAIT_TEARDOWN = 0x105,
+  DEVERR_GRID_BARRIER = 0x106,
 };
 __device__ __forceinline__ void record_error(int* flag, int code) {
   if (flag) atomicCAS(flag, 0, code);

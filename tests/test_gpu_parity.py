@@ -77,6 +77,39 @@ def test_activation_quantization_bit_exact(T, K, bits, xdt):
     assert (codes.cpu().numpy() == q_ref).all()
 
 
+@pytest.mark.parametrize("bits", [8, 6])
+def test_activation_quantization_at_half_integers(bits):
+    """Quotients x/sa on and next to half-integers: the kernel's division-free rounding must defer
+    to the exact quotient there and give the oracle's codes (round half to even)."""
+    qmax = 2 ** (bits - 1) - 1
+    T, K = 6, 256
+    rng = np.random.default_rng(77)
+    X = np.zeros((T, K), np.float32)
+    for t in range(T):
+        S = np.float32(rng.uniform(0.003, 0.07))
+        X[t, 0] = np.float32(qmax) * S                      # the row's absmax
+        sa = np.float32(X[t, 0] / np.float32(qmax))         # what the oracle's scale will be
+        n = rng.integers(-qmax, qmax, size=K - 1).astype(np.float32)
+        x = (n + np.float32(0.5)) * sa                        # about half-integer quotients
+        steps = rng.integers(-3, 4, size=K - 1)               # nudge by up to 3 ulps either way
+        for i, st in enumerate(steps):
+            for _ in range(abs(int(st))):
+                x[i] = np.nextafter(x[i], np.float32(np.inf) if st > 0 else np.float32(-np.inf))
+        X[t, 1:] = np.clip(x, -X[t, 0], X[t, 0])
+    s_inv = np.ones(K, np.float32)
+    q_ref, sa_ref = oracle.act_quant(X, s_inv, bits)
+    codes = torch.empty((T, K), dtype=torch.int8, device="cuda")
+    sa = torch.empty(T, dtype=torch.float32, device="cuda")
+    qe.act_quant(cuda(X), cuda(s_inv), bits, codes, sa)
+    torch.cuda.synchronize()
+    assert (sa.cpu().numpy() == sa_ref).all()
+    assert (codes.cpu().numpy() == q_ref).all()
+    # the set really contains ties broken to even and quotients that miss the half-integer
+    quot = X.astype(np.float64) / sa_ref.astype(np.float64)[:, None]
+    frac = np.abs(quot - np.floor(quot) - 0.5)
+    assert (frac == 0).sum() >= 1 and ((frac > 0) & (frac < 1e-6)).sum() >= 100
+
+
 @pytest.mark.parametrize("T,K,Nr,xdt", [(1, 256, 4, "f32"), (64, 256, 4, "f32"), (300, 1536, 8, "bf16"),
                                         (2048, 1536, 8, "bf16"), (77, 512, 16, "bf16"), (40, 256, 3, "f32"),
                                         (33, 256, 1, "bf16")])
