@@ -205,7 +205,9 @@ QE_API qe_status qe_route(const void* X, qe_dtype x_dtype, const void* G, int32_
  * order -> int8 tcgen05 GEMM with per-group scale promotion and the adapter
  * up-projection in its epilogue -> scatter to token order. With a_bits = 16
  * the main product is the weight-only path.
- * T = 0 is a no-op.
+ * T = 0 is a no-op. T <= 1<<20 (else QE_ERR_INVALID_ARG); d_in <= 32768
+ * (else QE_ERR_UNSUPPORTED: the cooperative launch keeps s_inv in shared
+ * memory).
  */
 QE_API qe_status qe_linear_forward(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
                             qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,

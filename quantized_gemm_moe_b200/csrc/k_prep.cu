@@ -78,6 +78,20 @@ __device__ __forceinline__ int rtn_code(float v, float scale, int qmax) {
   return static_cast<int>(r);
 }
 
+// Eight codes through rtn_code, packed little-endian into two words. Kept out of line: callers
+// unroll their loops, and this rare path would otherwise be copied into every unrolled step.
+__device__ __noinline__ uint2 rtn_code8_exact(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                                              float v7, float scale, int qmax) {
+  const float v[8] = {v0, v1, v2, v3, v4, v5, v6, v7};
+  uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    w0 |= (static_cast<uint32_t>(rtn_code(v[i], scale, qmax)) & 0xFFu) << (8 * i);
+    w1 |= (static_cast<uint32_t>(rtn_code(v[4 + i], scale, qmax)) & 0xFFu) << (8 * i);
+  }
+  return make_uint2(w0, w1);
+}
+
 // Eight codes rtn_code(v[i], scale, qmax), packed little-endian into two words, without a division
 // in the common case. inv = fl32(1/scale), the correctly rounded reciprocal. g = fl32(v*inv) differs
 // from the correctly rounded quotient fl32(v/scale) by at most 3 units of 2^-24 |g|, so rint(g)
@@ -105,13 +119,9 @@ __device__ __forceinline__ void rtn_code8(const float (&v)[8], float scale, floa
     w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
     return;
   }
-  w0 = 0;
-  w1 = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    w0 |= (static_cast<uint32_t>(rtn_code(v[i], scale, qmax)) & 0xFFu) << (8 * i);
-    w1 |= (static_cast<uint32_t>(rtn_code(v[4 + i], scale, qmax)) & 0xFFu) << (8 * i);
-  }
+  const uint2 w = rtn_code8_exact(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7], scale, qmax);
+  w0 = w.x;
+  w1 = w.y;
 }
 // Whether rtn_code8's fast path may be used for this scale (and its reciprocal).
 __device__ __forceinline__ bool rtn_fast_ok(float scale, float inv) {
@@ -633,9 +643,11 @@ __device__ __forceinline__ void row_scaled(const RowRaw<BF16>& r, int j, const f
   for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(xv[i], si[i]);
 }
 
-// Dynamic shared memory of k_route_quant: s_inv (K floats), then the range's expert ids and bucket
-// positions (chunk ints each).
-size_t route_quant_smem(int K, int chunk) { return size_t(K) * 4 + size_t(chunk) * 8; }
+// Dynamic shared memory of k_route_quant: s_inv (K floats), one adapter row per warp (R_pad floats
+// each), then the range's expert ids and bucket positions (chunk ints each).
+size_t route_quant_smem(int K, int chunk, int R_pad) {
+  return size_t(K) * 4 + size_t(kRQThreads / 32) * R_pad * 4 + size_t(chunk) * 8;
+}
 
 template <bool BF16>
 __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs a) {
@@ -645,8 +657,10 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
   __shared__ int tot_s[kMaxRouted], before_s[kMaxRouted], run_s[kMaxRouted];
   extern __shared__ float4 rq_dyn[];
   float* s_inv_s = reinterpret_cast<float*>(rq_dyn);
-  int* e_s = reinterpret_cast<int*>(s_inv_s + a.K);
+  float* u_w = s_inv_s + a.K;
+  int* e_s = reinterpret_cast<int*>(u_w + kWarps * a.R_pad);
   int* pos_s = e_s + a.chunk;
+  const size_t slot_stride = static_cast<size_t>(a.T) * a.R_tot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = min(a.T, static_cast<int>(blockIdx.x) * a.chunk), t1 = min(a.T, t0 + a.chunk);
   const int n_r = a.n_r;
@@ -656,7 +670,6 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
 
   if (a.do_route) {
     // ---- per token: logits, argmin, absmax
-    const size_t slot_stride = static_cast<size_t>(a.T) * a.R_tot;
     for (int t = t0 + warp; t < t1; t += kWarps) {
       const float L = (lane < n_r)
                           ? slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_pad + lane, slot_stride, a.nslots)
@@ -809,18 +822,17 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
     }
     if (a.codes && lane == 0) a.sa_sorted[p] = sa;
     if (a.R_pad > 0) {
+      // the token's adapter row: shared columns and its own expert's routed columns are the
+      // sums of the U slots; the others stay zero
       const int e = e_s[t - t0];
-      constexpr int kMaxPerLane = 512 / 32;
-      float u[kMaxPerLane];
+      float* uw = u_w + warp * a.R_pad;
+      const float* prow = a.partial + static_cast<size_t>(t) * a.R_tot;
       float mx = 0.0f;
-#pragma unroll
-      for (int i = 0; i < kMaxPerLane; ++i) {
-        const int c = lane + 32 * i;
-        float a2 = 0.0f;
-        if (c < a.R_a && (c < a.r_s || (c - a.r_s) / a.r_r == e))
-          a2 = slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + c, static_cast<size_t>(a.T) * a.R_tot, a.nslots);
-        u[i] = a2;
-        mx = fmaxf(mx, fabsf(a2));
+      for (int c = lane; c < a.R_pad; c += 32) {
+        float v = 0.0f;
+        if (c < a.R_a && (c < a.r_s || (c - a.r_s) / a.r_r == e)) v = slot_sum(prow + c, slot_stride, a.nslots);
+        uw[c] = v;
+        mx = fmaxf(mx, fabsf(v));
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -831,13 +843,9 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
         su = ldexpf(1.0f, ex - 14);
       }
       const float inv_su = 1.0f / su;  // exact: su is a power of two
-#pragma unroll
-      for (int i = 0; i < kMaxPerLane; ++i) {
-        const int c = lane + 32 * i;
-        if (c < a.R_pad) {
-          __half h = __float2half_rn(u[i] * inv_su);
-          a.ucat[p * a.R_pad + c] = *reinterpret_cast<uint16_t*>(&h);
-        }
+      for (int c = lane; c < a.R_pad; c += 32) {
+        __half h = __float2half_rn(uw[c] * inv_su);
+        a.ucat[p * a.R_pad + c] = *reinterpret_cast<uint16_t*>(&h);
       }
       if (lane == 0) a.su_sorted[p] = su;
     }
@@ -939,7 +947,7 @@ cudaError_t launch_split_f32(const float* X, const float* s_inv, int T, int K, u
   return cudaGetLastError();
 }
 
-constexpr int kRQMaxSmem = 200 * 1024;
+constexpr int kRQMaxSmem = 220 * 1024;  // covers d_in <= 32768, R_pad <= 512, T <= 2^20
 
 int route_quant_grid() {
   static int grid = 0;
@@ -981,7 +989,7 @@ cudaError_t launch_route_quant(const RouteQuantParams& q, cudaStream_t st) {
   a.K = q.K;
   a.qmax = q.qmax;
   a.chunk = static_cast<int>(ceil_div(q.T, grid));
-  const size_t smem = route_quant_smem(q.K, a.chunk);
+  const size_t smem = route_quant_smem(q.K, a.chunk, q.R_pad);
   if (smem > static_cast<size_t>(kRQMaxSmem)) return cudaErrorInvalidValue;
   a.do_route = q.do_route;
   a.do_quant = q.do_quant;

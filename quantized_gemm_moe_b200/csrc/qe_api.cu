@@ -169,6 +169,7 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   if (s != QE_OK) return s;
   if (!w || !w->w_packed || !w->w_scale || !w->s_inv || !w->adapters) return QE_ERR_INVALID_ARG;
   if (T < 0 || T > (1 << 20)) return QE_ERR_INVALID_ARG;
+  if (d->d_in > kMaxForwardDin) return QE_ERR_UNSUPPORTED;
   if (xd != QE_F32 && xd != QE_BF16) return QE_ERR_INVALID_ARG;
   if (yd != QE_F32 && yd != QE_BF16) return QE_ERR_INVALID_ARG;
   if (T == 0) return QE_OK;

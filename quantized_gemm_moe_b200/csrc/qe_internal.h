@@ -96,6 +96,7 @@ cudaError_t launch_ugemm(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, co
 // quant: codes (or bf16 act16) at row pos[t], sa_sorted, and U_cat / su_sorted.
 // *barrier must be 0 when the launch starts.
 constexpr int kRouteQuantMaxGrid = 1024;
+constexpr int kMaxForwardDin = 32768;  // the route/quant launch keeps s_inv in shared memory
 struct RouteQuantParams {
   const float* partial;
   int nslots, R_tot, R_pad, n_r, r_s, r_r, R_a;
