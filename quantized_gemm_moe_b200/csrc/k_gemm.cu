@@ -309,7 +309,9 @@ __global__ void __launch_bounds__(512, 1)
     if (lane == 0) {
       const uint32_t id_i8 = idesc_i8(128, BN);
       const uint32_t id_ad = idesc_f16(128, BN);
-      const int ksteps = a.group / 32;
+      // Descriptors are built once; a stage or a 32-byte K step only moves the start address
+      // field (16-byte units in the low bits, no carry below 256 KB of shared memory).
+      const uint64_t desc0 = smem_desc_sw128(smem_u32(stage_base));
       int it = 0, gidx = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -318,8 +320,8 @@ __global__ void __launch_bounds__(512, 1)
         for (int i = 0; i < w.nkb + w.n_ad && ok; ++i, ++it) {
           const int s = it % NS;
           const uint32_t ph = (it / NS) & 1;
-          const uint32_t a_addr = smem_u32(stage_base + s * C::kStage);
-          const uint32_t b_addr = a_addr + C::kA;
+          const uint64_t da = desc0 + static_cast<uint64_t>((s * C::kStage) >> 4);
+          const uint64_t db = da + (C::kA >> 4);
           if (i < w.nkb) {
             const int kb = w.kb_begin + i;
             const int ng = max(0, min(gpb, w.g_begin + w.n_groups - kb * gpb));
@@ -331,7 +333,10 @@ __global__ void __launch_bounds__(512, 1)
               ok = false;
               break;
             }
-            for (int gi = 0; gi < ng; ++gi) {
+            // four K steps of 32 per stage: one group (g = 128) or two (g = 64)
+#pragma unroll
+            for (int gi = 0; gi < 2; ++gi) {
+              if (gi >= ng) break;
               const int b = gidx % NB;
               if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
                 ok = false;
@@ -339,9 +344,12 @@ __global__ void __launch_bounds__(512, 1)
               }
               tc_fence_after();
               const uint32_t d = tmem + b * BN;
-              for (int kk = 0; kk < ksteps; ++kk) {
-                const uint32_t koff = gi * a.group + kk * 32;
-                mma_i8(d, smem_desc_sw128(a_addr + koff), smem_desc_sw128(b_addr + koff), id_i8, 1u);
+              if (gpb == 1) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) mma_i8(d, da + 2 * kk, db + 2 * kk, id_i8, 1u);
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) mma_i8(d, da + 4 * gi + 2 * kk, db + 4 * gi + 2 * kk, id_i8, 1u);
               }
               tc_commit(&accf[b]);
               ++gidx;
@@ -365,9 +373,8 @@ __global__ void __launch_bounds__(512, 1)
             }
             tc_fence_after();
             const uint32_t d = tmem + b * BN;
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16(d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), id_ad,
-                      (at > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) mma_f16(d, da + 2 * kk, db + 2 * kk, id_ad, (at > 0 || kk > 0) ? 1u : 0u);
             if (at == w.n_ad - 1) {
               tc_commit(&accf[b]);
               ++gidx;
@@ -458,16 +465,21 @@ __global__ void __launch_bounds__(512, 1)
       float acc[C::kCPT];
 #pragma unroll
       for (int c = 0; c < C::kCPT; ++c) acc[c] = 0.0f;
-      // weight codes enter the MMA as 16*q, so the group scale is applied as sw/16 (exact)
-      float sw_next = (o_ok && w.n_groups > 0)
-                          ? __ldg(a.w_scale + static_cast<size_t>(w.g_begin) * a.N + o) * 0.0625f
-                          : 0.0f;
+      // weight codes enter the MMA as 16*q, so the group scale is applied as sw/16 (exact).
+      // The scales are loaded kSwAhead groups ahead (a load can outlast a group's drain).
+      constexpr int kSwAhead = 2;
+      const float* swp = a.w_scale + static_cast<size_t>(w.g_begin) * a.N + o;
+      float swq[kSwAhead];
+#pragma unroll
+      for (int j = 0; j < kSwAhead; ++j)
+        swq[j] = (o_ok && j < w.n_groups) ? __ldg(swp + static_cast<size_t>(j) * a.N) : 0.0f;
       for (int g = 0; g < w.n_groups; ++g) {
         const int b = gidx % NB;
         ++gidx;
-        const uint64_t sw2 = pack2(sw_next);
-        if (g + 1 < w.n_groups && o_ok)
-          sw_next = __ldg(a.w_scale + static_cast<size_t>(w.g_begin + g + 1) * a.N + o) * 0.0625f;
+        const uint64_t sw2 = pack2(swq[0] * 0.0625f);
+#pragma unroll
+        for (int j = 0; j + 1 < kSwAhead; ++j) swq[j] = swq[j + 1];
+        swq[kSwAhead - 1] = (o_ok && g + kSwAhead < w.n_groups) ? __ldg(swp + static_cast<size_t>(g + kSwAhead) * a.N) : 0.0f;
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (!ok) continue;
         tc_fence_after();
