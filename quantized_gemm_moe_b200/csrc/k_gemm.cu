@@ -9,7 +9,7 @@
 //     warps 12-15 unpack the int4 block into int8 in the 128B-swizzled A layout
 //     warps 1-2   one thread each issues tcgen05.mma kind::i8 for alternate
 //                 stages, one TMEM accumulator buffer per quantization group
-//                 (2 buffers at BN=256, 4 below, so the MMA runs ahead of the
+//                 (2 buffers at BN >= 192, 4 below, so the MMA runs ahead of the
 //                 epilogue)
 //     warps 4-11  epilogue: the per-group promotion acc += sw[o,j] * float(int32)
 //                 in registers (f32x2, the next TMEM chunk loading meanwhile),
@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "qe_internal.h"
 #include "qe_ptx.cuh"
@@ -59,11 +60,12 @@ struct QCfg {
   static constexpr int kB = BN * 128;
   static constexpr int kWP = kW4BlockBytes;         // packed int4 block
   static constexpr int kStage = kA + kB + kWP;
-  static constexpr int kStages = (BN >= 256) ? 3 : (BN >= 128 ? 4 : (BN >= 64 ? 5 : 6));
-  static constexpr int kNBuf = (BN >= 256) ? 2 : 4;  // TMEM accumulator buffers
-  static constexpr int kTmemCols = (kNBuf * BN <= 32) ? 32 : kNBuf * BN;  // power of two for BN in {16..256}
+  static constexpr int kStages = (BN >= 192) ? 3 : (BN >= 128 ? 4 : (BN >= 64 ? 5 : 6));
+  static constexpr int kNBuf = (BN >= 192) ? 2 : 4;  // TMEM accumulator buffers
+  // TMEM is allocated in powers of two (>= 32 columns)
+  static constexpr int kTmemCols = (kNBuf * BN <= 32) ? 32 : (kNBuf * BN <= 128 ? 128 : (kNBuf * BN <= 256 ? 256 : 512));
   static constexpr int kCPT = BN / 2;              // columns per epilogue thread
-  static constexpr int kChunk = (kCPT >= 128) ? 16 : ((kCPT >= 32) ? 32 : kCPT);
+  static constexpr int kChunk = (kCPT >= 96) ? 16 : ((kCPT >= 32) ? 32 : kCPT);
   static constexpr int kNChunk = kCPT / kChunk;
   static constexpr int kOut = 32768;               // output staging (two 16 KB halves, one per epilogue warpgroup)
   static constexpr size_t kSmem = 1024 /*align slack*/ + size_t(kStages) * kStage + kOut + 1024 /*barriers etc*/ +
@@ -132,6 +134,13 @@ __device__ __forceinline__ Unit make_unit(const QgemmArgs& a, int BN, int u) {
 }
 
 
+// Largest divisor of cpt that is at most cap (the columns one staging pass can hold).
+__host__ __device__ constexpr int pass_columns(int cpt, int cap) {
+  int d = cap < cpt ? cap : cpt;
+  while (cpt % d != 0) --d;
+  return d;
+}
+
 // Writes one epilogue warpgroup's half tile (128 output channels x CPT token columns) to Y.
 // Each pass moves PC columns: every thread puts its values for those columns into the
 // warpgroup's 16 KB staging buffer (column-major by token), then the 128 threads copy
@@ -143,7 +152,7 @@ __device__ __forceinline__ void store_tile(const float (&acc)[CPT], uint8_t* sta
                                            const Unit& w, const QgemmArgs& a, int o0, int o_local, int wt, int h,
                                            bool ok, bool to_partial) {
   constexpr int kRowBytes = 128 * ELEM;
-  constexpr int kPC = (16384 / kRowBytes) < CPT ? (16384 / kRowBytes) : CPT;  // columns per pass
+  constexpr int kPC = pass_columns(CPT, 16384 / kRowBytes);  // columns per pass (divides CPT)
   constexpr int kChunksPerRow = kRowBytes / 16;
   constexpr int kElemsPerChunk = 16 / ELEM;
   const bool vec_ok = ((static_cast<size_t>(a.N) * ELEM) % 16) == 0;
@@ -261,6 +270,9 @@ __global__ void __launch_bounds__(512, 1)
     tc_fence_before();
   }
   __syncthreads();
+  // everything above touched only this CTA's shared memory and TMEM
+  grid_dep_wait();
+  grid_dep_launch();
 
   // Roles: warp 0 TMA producer, warps 1-2 MMA issuers (warp 3 idle), warps 4-11 epilogue,
   // warps 12-15 unpack. Register split: 256 * kRegLow + 256 * kRegHigh = 512 x 128 launch
@@ -606,7 +618,6 @@ __global__ void __launch_bounds__(192, 1)
   const int nk = max(0, min(nk_total, kc_begin + kchunks_per_split) - kc_begin);
 
   if (threadIdx.x == 0) {
-    if (zero_ctr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) *zero_ctr = 0u;
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -623,6 +634,9 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();
+  grid_dep_launch();
+  if (zero_ctr && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) *zero_ctr = 0u;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -686,6 +700,24 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled while the previous
+// kernel on the stream drains, and waits for it (grid_dep_wait) after its own set-up.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int BN, bool DBG>
 cudaError_t launch_qgemm_t(const CUtensorMap& tm_xq, const CUtensorMap& tm_bcat, const CUtensorMap& tm_ucat,
                            const QgemmArgs& a, cudaStream_t st) {
@@ -715,8 +747,7 @@ cudaError_t launch_qgemm_t(const CUtensorMap& tm_xq, const CUtensorMap& tm_bcat,
   }
   const int64_t units = ceil_div(a.N, kTileN) * ceil_div(a.T, BN) * a.splits;
   const unsigned grid = static_cast<unsigned>(units < n_sm ? units : n_sm);
-  k_qgemm<BN, DBG><<<grid, 512, C::kSmem, st>>>(tm_xq, tm_bcat, tm_ucat, a);
-  return cudaGetLastError();
+  return launch_pdl(k_qgemm<BN, DBG>, dim3(grid), dim3(512), C::kSmem, st, tm_xq, tm_bcat, tm_ucat, a);
 }
 
 template <int BN>
@@ -739,13 +770,17 @@ cudaError_t launch_ugemm_t(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, 
   }
   dim3 grid(static_cast<unsigned>(ceil_div(T, 128)), static_cast<unsigned>(p.ntiles),
             static_cast<unsigned>(p.splits));
-  k_ugemm<NU><<<grid, 192, C::kSmem, st>>>(tm_x, tm_acat, T, K, R_tot, p.kchunks_per_split, partial, zero_ctr,
-                                             err);
-  return cudaGetLastError();
+  return launch_pdl(k_ugemm<NU>, grid, dim3(192), C::kSmem, st, tm_x, tm_acat, T, K, R_tot, p.kchunks_per_split,
+                    partial, zero_ctr, err);
 }
 
 }  // namespace
 
+// Token-tile width and K split of the int8 GEMM. Small T takes the smallest tile that covers it.
+// Otherwise each candidate width is priced by a model of the persistent kernel: rounds of units
+// over the SMs, each unit costing its groups at the width's measured per-group time plus a fixed
+// unit cost (epilogue scaling, adapter and store). Wider tiles run the tensor core closer to its
+// peak, narrower ones fill the SMs better.
 int pick_qgemm_bn(int T, int N, int K, int* splits_out, int* kbps_out) {
   const int ntiles = static_cast<int>(ceil_div(N, kTileN));
   const int KB = static_cast<int>(ceil_div(K, kTileK));
@@ -755,9 +790,20 @@ int pick_qgemm_bn(int T, int N, int K, int* splits_out, int* kbps_out) {
   else if (T <= 64) bn = 64;
   else if (T <= 128) bn = 128;
   else {
-    // fill the 148 SMs: prefer 256-token tiles when they already give >= 1 full wave
-    const int64_t tiles256 = int64_t(ntiles) * ceil_div(T, 256);
-    bn = (tiles256 >= 148) ? 256 : 128;
+    constexpr int kCand[3] = {128, 192, 256};
+    constexpr double kGroupUs[3] = {0.37, 0.46, 0.56};  // per 128-deep K block
+    constexpr double kUnitUs = 4.0;
+    double best = 1e30;
+    bn = 128;
+    for (int i = 0; i < 3; ++i) {
+      const int64_t units = int64_t(ntiles) * ceil_div(T, kCand[i]);
+      const int64_t rounds = ceil_div(units, 148);
+      const double cost = double(rounds) * (KB * kGroupUs[i] + kUnitUs);
+      if (cost < best - 1e-9) {
+        best = cost;
+        bn = kCand[i];
+      }
+    }
   }
   const int64_t tiles = int64_t(ntiles) * ceil_div(T, bn);
   int splits = 1;
@@ -779,6 +825,7 @@ cudaError_t launch_qgemm(int BN, const CUtensorMap& tm_xq, const CUtensorMap& tm
     case 32: return launch_qgemm_bn<32>(tm_xq, tm_bcat, tm_ucat, a, st);
     case 64: return launch_qgemm_bn<64>(tm_xq, tm_bcat, tm_ucat, a, st);
     case 128: return launch_qgemm_bn<128>(tm_xq, tm_bcat, tm_ucat, a, st);
+    case 192: return launch_qgemm_bn<192>(tm_xq, tm_bcat, tm_ucat, a, st);
     case 256: return launch_qgemm_bn<256>(tm_xq, tm_bcat, tm_ucat, a, st);
     default: return cudaErrorInvalidValue;
   }
