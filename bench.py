@@ -365,15 +365,15 @@ def run_ours(args, workload):
     prod_ms = stage_ms[:, :, 2].sum(axis=1).mean()  # the product kernels of one step
     int8_peak = 2.0 * peaks["bf16_tflops"]           # int8 dense = 2x bf16 dense (nominal ratio)
     decode = T <= 16
-    kernel_file = "quantized_gemm_moe_b200/csrc/k_misc.cu" if wonly else "quantized_gemm_moe_b200/csrc/k_gemm.cu"
+    kernel_file = "quantized_gemm_moe_b200/csrc/k_wgemm.cu" if wonly else "quantized_gemm_moe_b200/csrc/k_gemm.cu"
     prod_bytes = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
                                           cfg.n_routed, cfg.rank_routed, 1 if not wonly else 2, 2) for L in layers)
-    traffic = read_traffic(kernel_file, ("wonly_" if wonly else "qgemm_") + workload)
+    traffic = read_traffic(kernel_file, ("wgemm_" if wonly else "qgemm_") + workload)
     if decode:
         ach = prod_bytes / (prod_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "wonly" if wonly else "qgemm", "peak_source": peaks["source"] + " hbm copy"}
+                "kernel": "wgemm" if wonly else "qgemm", "peak_source": peaks["source"] + " hbm copy"}
     else:
         ach = ints / (prod_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": int8_peak, "unit": "TOP/s",

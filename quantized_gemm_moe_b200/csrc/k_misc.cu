@@ -1,5 +1,4 @@
-// Weight-only (W3A16 / W4A16) product on CUDA cores, and the token-aware
-// Top-k importance statistic with its channel histogram.
+// The token-aware Top-k importance statistic with its channel histogram.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -14,127 +13,6 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as
 __device__ __forceinline__ uint16_t f2bf(float v) {
   __nv_bfloat16 h = __float2bfloat16_rn(v);
   return *reinterpret_cast<uint16_t*>(&h);
-}
-
-// ------------------------------------------------------------------ weight-only
-// CTA = 128 output rows x TT token positions x one K range; thread = row.
-// Per 128-channel block the TT activations (bf16(x*s_inv), bucket order) are
-// staged as fp32 in shared memory. Each thread decodes its row's codes, keeps
-// the exact sum_k x*q per group, and folds in the group scale at the group's end.
-template <int TT, int BITS>
-__global__ void __launch_bounds__(128) k_wonly(const uint16_t* __restrict__ act16, const uint8_t* __restrict__ wp,
-                                               const float* __restrict__ w_scale, const uint16_t* __restrict__ ucat,
-                                               const float* __restrict__ su, const uint16_t* __restrict__ bcat,
-                                               int R_pad, int has_adapters,
-                                               const int32_t* __restrict__ perm, int T, int N, int K, int group,
-                                               int kb_per_split, void* __restrict__ Y, int y_bf16,
-                                               float* __restrict__ partial) {
-  __shared__ __align__(16) float act[kTileK][TT];
-  const int r = threadIdx.x, nt = blockIdx.x, p0 = blockIdx.y * TT, split = blockIdx.z;
-  const int o = nt * kTileN + r;
-  const int KB = static_cast<int>(ceil_div(K, kTileK));
-  const int kb0 = split * kb_per_split, kb1 = min(KB, kb0 + kb_per_split);
-  constexpr int kBlockBytes = (BITS == 4) ? kW4BlockBytes : kW3BlockBytes;
-  constexpr int kRowBytes = kBlockBytes / kTileN;
-  float acc[TT], part[TT];
-#pragma unroll
-  for (int i = 0; i < TT; ++i) acc[i] = part[i] = 0.0f;
-  for (int kb = kb0; kb < kb1; ++kb) {
-    __syncthreads();
-    for (int i = r; i < kTileK * TT; i += blockDim.x) {
-      const int kl = i / TT, tt = i % TT, k = kb * kTileK + kl, p = p0 + tt;
-      act[kl][tt] = (k < K && p < T) ? bf16_bits_to_f32(act16[static_cast<size_t>(p) * K + k]) : 0.0f;
-    }
-    __syncthreads();
-    const uint8_t* row = wp + (static_cast<size_t>(nt) * KB + kb) * kBlockBytes + r * kRowBytes;
-    uint32_t wv[kRowBytes / 4];
-#pragma unroll
-    for (int i = 0; i < kRowBytes / 16; ++i) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(row) + i);
-      wv[4 * i] = u.x; wv[4 * i + 1] = u.y; wv[4 * i + 2] = u.z; wv[4 * i + 3] = u.w;
-    }
-    const int gpb = kTileK / group;
-#pragma unroll 1
-    for (int gi = 0; gi < gpb; ++gi) {
-      const int j = kb * gpb + gi;
-      if (j * group >= K) break;
-#pragma unroll 4
-      for (int kk = 0; kk < group; ++kk) {
-        const int kl = gi * group + kk;
-        int qv;
-        if constexpr (BITS == 4) {
-          const int h = kl >> 5, i = kl & 31, hi = i >> 4, w = (i & 15) >> 2, b = i & 3;
-          const uint32_t nib = (wv[4 * h + w] >> (8 * b + 4 * hi)) & 0xFu;
-          qv = static_cast<int>(nib) - static_cast<int>((nib & 8u) << 1);
-        } else {
-          const int m = kl >> 4, pp = (kl & 15) >> 1, odd = kl & 1;
-          const int hw = kl >> 5, hp = (kl & 31) >> 1;
-          const uint32_t lo2 = (wv[m] >> (odd ? 16 + 2 * pp : 2 * pp)) & 3u;
-          const uint32_t b2 = (wv[8 + hw] >> (odd ? 16 + hp : hp)) & 1u;
-          qv = static_cast<int>(lo2 | (b2 << 2)) - 4;
-        }
-        const float qf = static_cast<float>(qv);
-#pragma unroll
-        for (int tt = 0; tt < TT; ++tt) part[tt] = fmaf(qf, act[kl][tt], part[tt]);
-      }
-      const float sw = (o < N) ? __ldg(w_scale + static_cast<size_t>(j) * N + o) : 0.0f;
-#pragma unroll
-      for (int tt = 0; tt < TT; ++tt) {
-        acc[tt] = fmaf(sw, part[tt], acc[tt]);
-        part[tt] = 0.0f;
-      }
-    }
-  }
-  if (o >= N) return;
-  if (has_adapters && split == 0) {
-    const __half* brow = reinterpret_cast<const __half*>(bcat) + static_cast<size_t>(o) * R_pad;
-    const __half* uc = reinterpret_cast<const __half*>(ucat);
-    float ad[TT];
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt) ad[tt] = 0.0f;
-    for (int c = 0; c < R_pad; ++c) {
-      const float b = __half2float(brow[c]);
-#pragma unroll
-      for (int tt = 0; tt < TT; ++tt) {
-        const int p = p0 + tt;
-        if (p < T) ad[tt] = fmaf(__half2float(uc[static_cast<size_t>(p) * R_pad + c]), b, ad[tt]);
-      }
-    }
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-      if (p0 + tt < T) acc[tt] = fmaf(su[p0 + tt], ad[tt], acc[tt]);
-  }
-#pragma unroll
-  for (int tt = 0; tt < TT; ++tt) {
-    const int p = p0 + tt;
-    if (p >= T) break;
-    if (partial) {
-      partial[(static_cast<size_t>(split) * T + p) * N + o] = acc[tt];
-    } else {
-      const size_t dst = static_cast<size_t>(perm[p]) * N + o;
-      if (y_bf16) static_cast<uint16_t*>(Y)[dst] = f2bf(acc[tt]);
-      else static_cast<float*>(Y)[dst] = acc[tt];
-    }
-  }
-}
-
-template <int TT>
-cudaError_t launch_wonly_t(const uint16_t* act16, const uint8_t* wp, const float* w_scale, int w_bits,
-                           const uint16_t* ucat, const float* su, const uint16_t* bcat, int R_pad, int has_adapters,
-                           const int32_t* perm, int T, int N, int K, int group, void* Y, int y_bf16,
-                           float* partial, int splits, cudaStream_t st) {
-  const int KB = static_cast<int>(ceil_div(K, kTileK));
-  const int kbps = static_cast<int>(ceil_div(KB, splits));
-  dim3 grid(static_cast<unsigned>(ceil_div(N, kTileN)), static_cast<unsigned>(ceil_div(T, TT)),
-            static_cast<unsigned>(splits));
-  float* part = splits > 1 ? partial : nullptr;
-  if (w_bits == 4)
-    k_wonly<TT, 4><<<grid, 128, 0, st>>>(act16, wp, w_scale, ucat, su, bcat, R_pad, has_adapters, perm, T, N, K, group,
-                                         kbps, Y, y_bf16, part);
-  else
-    k_wonly<TT, 3><<<grid, 128, 0, st>>>(act16, wp, w_scale, ucat, su, bcat, R_pad, has_adapters, perm, T, N, K, group,
-                                         kbps, Y, y_bf16, part);
-  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ Top-k importance
@@ -316,21 +194,6 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const void* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_wonly(const uint16_t* act16, const uint8_t* w_packed, const float* w_scale, int w_bits,
-                         const uint16_t* ucat, const float* su, const uint16_t* bcat, int R_pad, int has_adapters,
-                         const int32_t* perm, int T, int N, int K, int group, void* Y, int y_bf16, float* partial,
-                         int splits, cudaStream_t st) {
-  if (T == 0) return cudaSuccess;
-#define QE_WO(TT) \
-  launch_wonly_t<TT>(act16, w_packed, w_scale, w_bits, ucat, su, bcat, R_pad, has_adapters, perm, T, N, K, group, Y, \
-                     y_bf16, partial, splits, st)
-  if (T <= 1) return QE_WO(1);
-  if (T <= 2) return QE_WO(2);
-  if (T <= 4) return QE_WO(4);
-  if (T <= 8) return QE_WO(8);
-  return QE_WO(16);
-#undef QE_WO
-}
 
 cudaError_t launch_topk(const void* X, bool x_bf16, const float* w_mean, int T, int K, int k, int32_t* idx,
                         int32_t* hist, cudaStream_t st) {

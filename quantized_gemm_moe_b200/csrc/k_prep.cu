@@ -971,7 +971,8 @@ int route_quant_grid() {
 
 cudaError_t launch_route_quant(const RouteQuantParams& q, cudaStream_t st) {
   if (q.T == 0) return cudaSuccess;
-  const int grid = route_quant_grid();
+  // one CTA per SM, or one per token when there are fewer tokens (decode)
+  const int grid = std::min(route_quant_grid(), q.T);
   if (grid == 0) return cudaErrorInvalidConfiguration;
   RouteQuantArgs a{};
   a.partial = q.partial;

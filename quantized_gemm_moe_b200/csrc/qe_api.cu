@@ -68,16 +68,6 @@ struct Plan {
       off_xlo, off_amax, off_upart, off_ucat, off_ypart, off_counts, off_barrier, bytes;
 };
 
-int wonly_splits(int T, int N, int K) {
-  const int64_t ntiles = ceil_div(N, kTileN);
-  const int64_t ttiles = ceil_div(T, 16);
-  const int KB = static_cast<int>(ceil_div(K, kTileK));
-  int splits = static_cast<int>(ceil_div(2 * 148, ntiles * ttiles));
-  splits = std::max(1, std::min(splits, std::max(1, KB / 4)));
-  const int kbps = static_cast<int>(ceil_div(KB, splits));
-  return static_cast<int>(ceil_div(KB, kbps));
-}
-
 Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   Plan p{};
   p.T = T;
@@ -88,9 +78,7 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   const int Tm = std::max(T, 1);
   p.up = plan_ugemm(Tm, p.K, p.g.R_tot);
   if (d->a_bits == 16) {
-    p.bn = 0;
-    p.msplits = wonly_splits(Tm, p.N, p.K);
-    p.kbps = 0;
+    p.bn = pick_wgemm_bn(Tm, p.N, p.K, &p.msplits, &p.kbps);
   } else {
     p.bn = pick_qgemm_bn(Tm, p.N, p.K, &p.msplits, &p.kbps);
   }
@@ -271,13 +259,13 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   if (!(stages & QE_STAGE_PRODUCT)) return QE_OK;
   float* ypart = p.msplits > 1 ? at<float>(ws, p.off_ypart) : nullptr;
   const int y_bf16 = yd == QE_BF16;
-  if (wonly) {
-    QE_CUDA(launch_wonly(act16, static_cast<const uint8_t*>(w->w_packed), w->w_scale, d->w_bits, ucat, su_sorted, bcat,
-                         p.g.R_pad, p.has_ad ? 1 : 0, perm, T, N, K, d->group, Y, y_bf16, ypart, p.msplits, st),
-            "wonly");
-  } else {
-    CUtensorMap tm_xq, tm_bcat, tm_ucat;
-    if ((s = make_tmap(&tm_xq, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, T, kTileK, p.bn)) != QE_OK) return s;
+  {
+    CUtensorMap tm_act, tm_bcat, tm_ucat;
+    if (wonly) {
+      if ((s = make_tmap(&tm_act, act16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, T, 64, p.bn)) != QE_OK) return s;
+    } else {
+      if ((s = make_tmap(&tm_act, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, T, kTileK, p.bn)) != QE_OK) return s;
+    }
     if (p.has_ad) {
       if ((s = make_tmap(&tm_bcat, bcat, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.g.R_pad, N, kAdapterAtom, kTileN)) !=
           QE_OK)
@@ -286,8 +274,8 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
           QE_OK)
         return s;
     } else {
-      tm_bcat = tm_xq;
-      tm_ucat = tm_xq;
+      tm_bcat = tm_act;
+      tm_ucat = tm_act;
     }
     QgemmArgs a{};
     a.w_packed = static_cast<const uint8_t*>(w->w_packed);
@@ -306,9 +294,12 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
     a.Y = Y;
     a.y_bf16 = y_bf16;
     a.partial = ypart;
-    a.dbg_acc = dbg_acc;
+    a.dbg_acc = wonly ? nullptr : dbg_acc;
     a.err = err;
-    QE_CUDA(launch_qgemm(p.bn, tm_xq, tm_bcat, tm_ucat, a, st), "qgemm");
+    if (wonly)
+      QE_CUDA(launch_wgemm(d->w_bits, p.bn, tm_act, tm_bcat, tm_ucat, a, st), "wgemm");
+    else
+      QE_CUDA(launch_qgemm(p.bn, tm_act, tm_bcat, tm_ucat, a, st), "qgemm");
   }
   if (p.msplits > 1) QE_CUDA(launch_splitk_reduce(ypart, p.msplits, perm, T, N, Y, y_bf16, st), "splitk_reduce");
   if (dbg_expert) QE_CUDA(cudaMemcpyAsync(dbg_expert, expert, size_t(T) * 4, cudaMemcpyDeviceToDevice, st), "copy");

@@ -146,11 +146,11 @@ cudaError_t launch_qgemm(int BN, const CUtensorMap& tm_xq, const CUtensorMap& tm
 cudaError_t launch_splitk_reduce(const float* partial, int splits, const int32_t* perm, int T, int N, void* Y,
                                  int y_bf16, cudaStream_t st);
 
-// Weight-only (W3A16 / W4A16) product on CUDA cores, token chunks of up to 16.
-cudaError_t launch_wonly(const uint16_t* act16, const uint8_t* w_packed, const float* w_scale, int w_bits,
-                         const uint16_t* ucat, const float* su_sorted, const uint16_t* bcat, int R_pad, int has_adapters,
-                         const int32_t* perm, int T, int N, int K, int group, void* Y, int y_bf16, float* partial,
-                         int splits, cudaStream_t st);
+// Weight-only (W3A16 / W4A16) product on the tensor cores: codes unpacked to bf16, bf16
+// activations (act16, bucket order), per-group fp32 sums scaled by sw, adapter epilogue.
+int pick_wgemm_bn(int T, int N, int K, int* splits_out, int* kbps_out);
+cudaError_t launch_wgemm(int bits, int BN, const CUtensorMap& tm_act, const CUtensorMap& tm_bcat,
+                         const CUtensorMap& tm_ucat, const QgemmArgs& a, cudaStream_t st);
 
 // Device error word (one per device, in the library's own device memory).
 int* device_error_ptr();  // nullptr when the symbol lookup fails
