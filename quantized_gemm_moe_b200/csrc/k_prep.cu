@@ -644,9 +644,9 @@ __device__ __forceinline__ void row_scaled(const RowRaw<BF16>& r, int j, const f
 }
 
 // Dynamic shared memory of k_route_quant: s_inv (K floats), one adapter row per warp (R_pad floats
-// each), then the range's expert ids and bucket positions (chunk ints each).
+// each), then the range's expert ids, bucket positions and absmax bits (chunk ints each).
 size_t route_quant_smem(int K, int chunk, int R_pad) {
-  return size_t(K) * 4 + size_t(kRQThreads / 32) * R_pad * 4 + size_t(chunk) * 8;
+  return size_t(K) * 4 + size_t(kRQThreads / 32) * R_pad * 4 + size_t(chunk) * 12;
 }
 
 template <bool BF16>
@@ -660,61 +660,77 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
   float* u_w = s_inv_s + a.K;
   int* e_s = reinterpret_cast<int*>(u_w + kWarps * a.R_pad);
   int* pos_s = e_s + a.chunk;
+  int* mx_s = pos_s + a.chunk;  // per-token absmax as int bits (non-negative floats order as ints)
   const size_t slot_stride = static_cast<size_t>(a.T) * a.R_tot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = min(a.T, static_cast<int>(blockIdx.x) * a.chunk), t1 = min(a.T, t0 + a.chunk);
   const int n_r = a.n_r;
+  // With fewer tokens than warps, wpt warps share a token's row (wpt a power of two).
+  int wpt = 1;
+  while (wpt * 2 * a.chunk <= kWarps) wpt *= 2;
+  const int sub = warp % wpt, slot = warp / wpt, nslot_w = kWarps / wpt;
   for (int i = threadIdx.x; i < a.K / 4; i += kRQThreads)
     reinterpret_cast<float4*>(s_inv_s)[i] = __ldg(reinterpret_cast<const float4*>(a.s_inv) + i);
+  for (int i = threadIdx.x; i < t1 - t0; i += kRQThreads) mx_s[i] = 0;
   __syncthreads();
 
   if (a.do_route) {
-    // ---- per token: logits, argmin, absmax
-    for (int t = t0 + warp; t < t1; t += kWarps) {
-      const float L = (lane < n_r)
-                          ? slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_pad + lane, slot_stride, a.nslots)
-                          : 0.0f;
-      float best = (lane < n_r) ? L : INFINITY;
-      int bi = (lane < n_r) ? lane : 0x7fffffff;
+    // ---- per token: logits, argmin (the token's first warp), absmax (all of its warps)
+    for (int t = t0 + slot; t < t1; t += nslot_w) {
+      if (sub == 0) {
+        const float L = (lane < n_r) ? slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_pad + lane,
+                                                slot_stride, a.nslots)
+                                     : 0.0f;
+        float best = (lane < n_r) ? L : INFINITY;
+        int bi = (lane < n_r) ? lane : 0x7fffffff;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, best, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (ov < best || (ov == best && oi < bi)) {
-          best = ov;
-          bi = oi;
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (ov < best || (ov == best && oi < bi)) {
+            best = ov;
+            bi = oi;
+          }
+        }
+        if (lane == 0) {
+          a.expert[t] = bi;
+          e_s[t - t0] = bi;
         }
       }
-      if (a.sa_tok) {
+      if (a.sa_tok && BF16) {
         float mx = 0.0f;
-        if (BF16) {
-          for (int k0 = lane * 8; k0 < a.K; k0 += 256 * kB) {
-            RowRaw<true> r;
-            row_load<true>(a.X, t, a.K, k0, r);
+        for (int k0 = (sub * 32 + lane) * 8; k0 < a.K; k0 += 256 * wpt * kB) {
+          RowRaw<true> r;
 #pragma unroll
-            for (int j = 0; j < kB; ++j) {
-              const int k = k0 + 256 * j;
-              if (k < a.K) {
-                float v[8];
-                row_scaled<true>(r, j, s_inv_s, k, v);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
-              }
-            }
+          for (int j = 0; j < kB; ++j) {
+            const int k = k0 + 256 * wpt * j;
+            if (k < a.K)
+              r.v[j][0] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.X) +
+                                                                static_cast<size_t>(t) * a.K + k));
           }
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        } else {
-          mx = a.amax[t];
+          for (int j = 0; j < kB; ++j) {
+            const int k = k0 + 256 * wpt * j;
+            if (k < a.K) {
+              float v[8];
+              row_scaled<true>(r, j, s_inv_s, k, v);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
+            }
+          }
         }
-        if (lane == 0) a.sa_tok[t] = __fdiv_rn(mx, static_cast<float>(a.qmax));
-      }
-      if (lane == 0) {
-        a.expert[t] = bi;
-        e_s[t - t0] = bi;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) atomicMax(&mx_s[t - t0], __float_as_int(mx));
       }
     }
     __syncthreads();
+    if (a.sa_tok) {
+      for (int i = threadIdx.x; i < t1 - t0; i += kRQThreads) {
+        const float mx = BF16 ? __int_as_float(mx_s[i]) : a.amax[t0 + i];
+        a.sa_tok[t0 + i] = __fdiv_rn(mx, static_cast<float>(a.qmax));
+      }
+    }
     // ---- this CTA's count per expert
     if (warp < n_r) {
       int c = 0;
@@ -791,18 +807,31 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
     __syncthreads();
   }
   if (!a.do_quant) return;
-  // ---- per token, in bucket order
-  for (int t = t0 + warp; t < t1; t += kWarps) {
+  // ---- per token, in bucket order (the token's warps share the row; its first warp writes the rest)
+  for (int t = t0 + slot; t < t1; t += nslot_w) {
     const size_t p = static_cast<size_t>(pos_s[t - t0]);
     const float sa = a.codes ? a.sa_tok[t] : 0.0f;
     const float inv = (sa > 0.0f) ? __frcp_rn(sa) : 0.0f;
     const bool fast = rtn_fast_ok(sa, inv);
-    for (int k0 = lane * 8; k0 < a.K; k0 += 256 * kB) {
+    for (int k0 = (sub * 32 + lane) * 8; k0 < a.K; k0 += 256 * wpt * kB) {
       RowRaw<BF16> r;
-      row_load<BF16>(a.X, t, a.K, k0, r);
 #pragma unroll
       for (int j = 0; j < kB; ++j) {
-        const int k = k0 + 256 * j;
+        const int k = k0 + 256 * wpt * j;
+        if (k < a.K) {
+          if constexpr (BF16) {
+            r.v[j][0] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.X) +
+                                                              static_cast<size_t>(t) * a.K + k));
+          } else {
+            const uint4* q = reinterpret_cast<const uint4*>(static_cast<const float*>(a.X) + static_cast<size_t>(t) * a.K + k);
+            r.v[j][0] = __ldg(q);
+            r.v[j][1] = __ldg(q + 1);
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        const int k = k0 + 256 * wpt * j;
         if (k >= a.K) break;
         float v[8];
         row_scaled<BF16>(r, j, s_inv_s, k, v);
@@ -820,6 +849,7 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
         }
       }
     }
+    if (sub != 0) continue;
     if (a.codes && lane == 0) a.sa_sorted[p] = sa;
     if (a.R_pad > 0) {
       // the token's adapter row: shared columns and its own expert's routed columns are the

@@ -13,8 +13,8 @@
 //   warp 3      TMA loads of the activation tile (two 64-wide K atoms) into the operand slot,
 //               and of the adapter operands after the last block of a unit
 //   warps 8-15  unpack 3- or 4-bit codes into bf16 in the 128B-swizzled A layout of the slot
-//   warp 1      one thread issues tcgen05.mma kind::f16 (bf16), 8 K steps per 128-deep block;
-//               the first step of each group starts a fresh accumulator
+//   warps 1-2   one thread each issues tcgen05.mma kind::f16 (bf16) for alternate blocks, 8 K
+//               steps per 128-deep block; the first step of a group starts a fresh accumulator
 //   warps 4-7   epilogue: per group acc += sw * tmem; at the end of a unit + su * adapter,
 //               then a scatter of the rows to token order through shared memory
 // Unpacking writes bf16(128 + u) with a byte permute (u = the code's offset-binary value) and
@@ -37,12 +37,14 @@ struct WCfg {
   static constexpr int kAtomB = BN * 128;
   static constexpr int kB = 2 * kAtomB;
   static constexpr int kSlot = kA + kB;
-  static constexpr int kNA = 3;                 // operand slots (A + B)
-  static constexpr int kNW = (BN >= 64) ? 6 : 8;  // packed weight ring
+  // Operand slots: each holds a 32 KB bf16 weight tile, so they bound the blocks in flight
+  // between unpacking and the MMA; narrow tiles leave room for one more.
+  static constexpr int kNA = (BN <= 32) ? 4 : 3;
+  static constexpr int kNW = 6;                 // packed weight ring
   static constexpr int kWP = 8192;
   static constexpr int kNB = 8;                 // TMEM accumulator buffers (fp32, BN columns each)
   static constexpr int kTmemCols = (kNB * BN <= 128) ? 128 : (kNB * BN <= 256 ? 256 : 512);
-  static constexpr int kOut = 16384;            // output staging
+  static constexpr int kOut = (BN <= 32) ? 8192 : 16384;  // output staging
   static constexpr int kChunk = (BN >= 16) ? 16 : BN;
   static constexpr size_t kSmem =
       1024 + size_t(kNA) * kSlot + size_t(kNW) * kWP + kOut + 1024 + size_t(BN) * 8;
@@ -89,12 +91,18 @@ __device__ __forceinline__ uint2 w4_to_bf16(uint32_t v, int shift) {
 }
 
 // Two 3-bit offset-binary codes u = q + 4: low two bits at bits [lo_shift, +2) and [16 + lo_shift, +2)
-// of lw, bit 2 at bits hi_shift and 16 + hi_shift of hw -> bf16 pair (q_even, q_odd).
+// of lw, bit 2 at bits hi_shift and 16 + hi_shift of hw -> bf16 pair (q_even, q_odd). Two
+// three-input logic ops build bf16(128 + u) in both halves; one bf16x2 subtraction leaves q.
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));  // (a & b) | c
+  return d;
+}
 __device__ __forceinline__ uint32_t w3_pair_to_bf16(uint32_t lw, uint32_t hw, int lo_shift, int hi_shift) {
-  const uint32_t l = (lw >> lo_shift) & 0x00030003u;
-  const uint32_t h = ((hw >> hi_shift) & 0x00010001u) << 2;
-  const uint32_t bf = l | h | 0x43004300u;  // bf16(128 + u) in each half
-  return bf16x2_sub(bf, 0x43044304u);       // - bf16(132)
+  const uint32_t l = lop3_and_or(lw >> lo_shift, 0x00030003u, 0x43004300u);  // bf16(128 + low bits)
+  const uint32_t hs = (hi_shift >= 2) ? (hw >> (hi_shift - 2)) : (hw << (2 - hi_shift));
+  const uint32_t bf = lop3_and_or(hs, 0x00040004u, l);                        // + 4 * bit 2
+  return bf16x2_sub(bf, 0x43044304u);                                         // - bf16(132)
 }
 
 template <int BITS, int BN>
@@ -141,7 +149,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&accf[b], 1);
       mbar_init(&acce[b], 4);
     }
-    mbar_init(done, 1);
+    mbar_init(done, 2);
     mbar_fence_init();
     prefetch_tmap(&tm_act);
     if (a.adapter_atoms) {
@@ -208,8 +216,12 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads issue alternate blocks: one thread's issue rate, not the tensor pipe, limits
+    // these narrow (BN <= 64) MMAs. A unit's adapter atoms accumulate into one TMEM buffer, so
+    // one issuer takes all of them.
+    const int qi = warp - 1;
     if (lane == 0) {
       const uint32_t id_bf = idesc_bf16(128, BN);
       const uint32_t id_ad = idesc_f16(128, BN);
@@ -218,17 +230,22 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const WUnit w = make_wunit(a, BN, u);
+        const int ad_owner = (it + w.nkb) & 1;
         for (int i = 0; i < w.nkb + w.n_ad && ok; ++i, ++it) {
           const int s = it % NA;
-          if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
-            ok = false;
-            break;
-          }
           const uint64_t da = desc_a0 + static_cast<uint64_t>((s * C::kSlot) >> 4);
           const uint64_t db = da + (C::kA >> 4);
           if (i < w.nkb) {
             const int kb = w.kb_begin + i;
             const int ng = max(0, min(gpb, w.g_begin + w.n_groups - kb * gpb));
+            if ((it & 1) != qi) {
+              gidx += ng;
+              continue;
+            }
+            if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
             // 8 K steps of 16 per block (4 per 64-wide atom): one group (g = 128) or two (g = 64)
 #pragma unroll
             for (int gi = 0; gi < 2; ++gi) {
@@ -255,6 +272,14 @@ __global__ void __launch_bounds__(512, 1)
           } else {
             const int at = i - w.nkb;
             const int b = gidx % NB;
+            if (ad_owner != qi) {
+              if (at == w.n_ad - 1) ++gidx;
+              continue;
+            }
+            if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
             if (at == 0) {
               if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
                 ok = false;
