@@ -278,6 +278,15 @@ QE_API const char* qe_last_cuda_error(void);
  */
 QE_API qe_status qe_device_error(void* stream, int32_t* code, int32_t clear);
 
+/*
+ * Self-test of the bounded device waits (a library convenience; the paper has no counterpart).
+ * Launches one thread that waits on a barrier nothing arrives on, for at most limit_us
+ * microseconds (1 .. 1000000). The wait runs out, records code 0x107 in the device error word,
+ * and the kernel returns normally, so the context stays usable and qe_device_error() then reports
+ * QE_ERR_TIMEOUT. limit_us outside that range -> QE_ERR_INVALID_ARG.
+ */
+QE_API qe_status qe_selftest_wait_timeout(int32_t limit_us, void* stream);
+
 /* ---------------------------------------------------------------- diagnostics (tests) */
 
 /* Unpacks w_packed to int8 codes [d_out, d_in] (device), one code per byte. */

@@ -24,6 +24,7 @@ EXPORTS = (
     "qe_pack_adapters", "qe_topk_importance", "qe_route", "qe_linear_forward", "qe_status_string",
     "qe_last_cuda_error", "qe_device_error", "qe_unpack_weights", "qe_act_quant", "qe_linear_forward_debug",
     "qe_linear_forward_stages", "qe_linear_kernel_launches", "qe_linear_forward_noalloc",
+    "qe_selftest_wait_timeout",
 )
 # fixed scratch of qe_linear_forward_noalloc (bytes), as declared in include/qe.h
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -86,6 +87,7 @@ def load() -> ctypes.CDLL:
         "qe_device_error": ([P, ctypes.POINTER(I), I], I),
         "qe_unpack_weights": ([D, P, P, P], I),
         "qe_act_quant": ([P, I, P, I, I, I, P, P, P], I),
+        "qe_selftest_wait_timeout": ([I, P], I),
     }
     for name, (args, res) in sigs.items():
         f = getattr(L, name)
@@ -235,6 +237,11 @@ def device_error(clear: bool = True, stream=None) -> int:
     if rc not in (QE_OK, QE_ERR_TIMEOUT):
         _check(rc, "qe_device_error")
     return int(code.value)
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Launches one device wait that runs out after limit_us (it records code 0x107)."""
+    _check(load().qe_selftest_wait_timeout(int(limit_us), _stream(stream)), "qe_selftest_wait_timeout")
 
 
 # ---------------------------------------------------------------- a layer object (device buffers via torch)

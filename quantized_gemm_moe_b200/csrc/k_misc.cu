@@ -5,6 +5,7 @@
 #include <algorithm>
 
 #include "qe_internal.h"
+#include "qe_ptx.cuh"
 
 namespace qe {
 namespace {
@@ -192,6 +193,18 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const void* __restrict__ 
   }
 }
 
+// Self-test of the bounded waits: one thread waits on a barrier that nothing arrives on. The
+// wait runs out after limit_ns, records DEVERR_SELFTEST and the kernel returns.
+__global__ void k_wait_selftest(int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_for(&bar, 0, err, DEVERR_SELFTEST, limit_ns);
+}
+
 }  // namespace
 
 
@@ -212,4 +225,11 @@ cudaError_t launch_topk(const void* X, bool x_bf16, const float* w_mean, int T, 
   return cudaGetLastError();
 }
 
+}  // namespace qe
+
+namespace qe {
+cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st) {
+  k_wait_selftest<<<1, 32, 0, st>>>(err, limit_ns);
+  return cudaGetLastError();
+}
 }  // namespace qe

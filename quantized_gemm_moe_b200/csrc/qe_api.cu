@@ -532,4 +532,13 @@ qe_status qe_device_error(void* stream, int32_t* code, int32_t clear) {
   return v ? QE_ERR_TIMEOUT : QE_OK;
 }
 
+qe_status qe_selftest_wait_timeout(int32_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return QE_ERR_INVALID_ARG;
+  int* err = device_error_ptr();
+  if (!err) return cuda_fail(cudaErrorInvalidSymbol, "device error word");
+  QE_CUDA(launch_wait_selftest(err, static_cast<uint64_t>(limit_us) * 1000ull, static_cast<cudaStream_t>(stream)),
+          "wait_selftest");
+  return QE_OK;
+}
+
 }  // extern "C"

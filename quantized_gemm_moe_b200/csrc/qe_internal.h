@@ -152,6 +152,9 @@ int pick_wgemm_bn(int T, int N, int K, int* splits_out, int* kbps_out);
 cudaError_t launch_wgemm(int bits, int BN, const CUtensorMap& tm_act, const CUtensorMap& tm_bcat,
                          const CUtensorMap& tm_ucat, const QgemmArgs& a, cudaStream_t st);
 
+// One CTA whose single wait runs out after limit_ns (the bounded-wait self-test).
+cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
+
 // Device error word (one per device, in the library's own device memory).
 int* device_error_ptr();  // nullptr when the symbol lookup fails
 cudaError_t read_device_error(int* value, bool clear, cudaStream_t st);

@@ -20,6 +20,7 @@ enum : int {
   DEVERR_WAIT_EPILOGUE = 0x104,
   DEVERR_WAIT_TEARDOWN = 0x105,
   DEVERR_GRID_BARRIER = 0x106,
+  DEVERR_SELFTEST = 0x107,
 };
 __device__ __forceinline__ void record_error(int* flag, int code) {
   if (flag) atomicCAS(flag, 0, code);
@@ -64,18 +65,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete. Returns false (and
-// records err) when the wait ran out; callers then stop issuing work.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* flag, int err) {
+// records err) when the wait ran out after limit_ns; callers then stop issuing work.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int* flag, int err,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if ((++spins & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((++spins & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
       record_error(flag, err);
       return false;
     }
   }
   return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* flag, int err) {
+  return mbar_wait_for(bar, parity, flag, err, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ async copies
