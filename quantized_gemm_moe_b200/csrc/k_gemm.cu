@@ -465,15 +465,27 @@ __global__ void __launch_bounds__(512, 1)
       const int o0 = w.nt * kTileN;
       const int o = o0 + 32 * q + lane;
       const bool o_ok = o < a.N;
-      // stage this unit's per-position scales and token ids (after everyone finished the previous unit)
+      // this unit's per-position scales and token ids: copied asynchronously into shared memory
+      // (after everyone finished the previous unit's store), waited for when the epilogue needs them
       asm volatile("bar.sync 1, 256;" ::: "memory");
       for (int c = et; c < BN; c += 256) {
         const int p = w.p0 + c;
-        sa_s[c] = (p < a.T) ? a.sa_sorted[p] : 0.0f;
-        su_s[c] = (p < a.T && a.su_sorted) ? a.su_sorted[p] : 0.0f;
-        perm_s[c] = (p < a.T) ? a.perm[p] : -1;
+        if (p < a.T) {
+          cp_async4(&sa_s[c], a.sa_sorted + p);
+          if (a.su_sorted) cp_async4(&su_s[c], a.su_sorted + p);
+          else su_s[c] = 0.0f;
+          cp_async4(&perm_s[c], a.perm + p);
+        } else {
+          sa_s[c] = 0.0f;
+          su_s[c] = 0.0f;
+          perm_s[c] = -1;
+        }
       }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      cp_async_commit();
+      if (DBG) {
+        cp_async_wait_all();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+      }
       float acc[C::kCPT];
 #pragma unroll
       for (int c = 0; c < C::kCPT; ++c) acc[c] = 0.0f;
@@ -529,6 +541,8 @@ __global__ void __launch_bounds__(512, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce[b]);
       }
+      cp_async_wait_all();
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       // per-token scale
       const float4* sa4 = reinterpret_cast<const float4*>(sa_s + h * C::kCPT);
 #pragma unroll
