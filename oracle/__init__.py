@@ -17,6 +17,8 @@ Parity status per function (pins live in tests/test_oracle_pins.py):
   qe_forward                   pinned: zero adapters = literal dequant matmul,
                                token independence, identical experts, SVD fixture
   topk                         pinned: brute force, sum(hist) = T*k, order
+  cooccurrence, npmi           pinned: a hand-counted example, symmetry, diagonal = channel counts,
+                               closed-form NPMI cases (independent 0, always together 1, never -1)
 """
 from __future__ import annotations
 
@@ -187,3 +189,49 @@ def router_near_tie_bound(X, G) -> np.ndarray:
     G = _f32(G).astype(np.float64)
     K = X.shape[1]
     return 2.0 * K * 2.0 ** -24 * (np.abs(X) @ np.abs(G).max(axis=1))
+
+
+def cooccurrence(idx, channel_pos, C: int) -> np.ndarray:
+    """Co-occurrence counts of the token-dependent channels ([DR] \u00a7Method, routed experts).
+
+    idx [T][k]: each token's Top-k channel indices (qe_topk_importance). channel_pos [d_in]: the
+    position in [0, C) of each token-dependent channel, -1 for every other channel. O[i][j] is the
+    number of tokens whose important set holds both channels i and j; O[i][i] is how many tokens
+    hold channel i. Built as the 0/1 token x channel indicator M, then O = M^T M in int64.
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    pos = np.asarray(channel_pos, dtype=np.int64)
+    T = idx.shape[0]
+    M = np.zeros((T, C), dtype=np.int64)
+    rows = np.repeat(np.arange(T), idx.shape[1])
+    cols = pos[idx.ravel()]
+    keep = cols >= 0
+    M[rows[keep], cols[keep]] = 1
+    return M.T @ M
+
+
+def npmi(O, T: int, threshold: float = -1.0) -> np.ndarray:
+    """Normalized pointwise mutual information of channel pairs ([DR] \u00a7Method), in fp64.
+
+    p(i) = O[i][i] / T, p(i,j) = O[i][j] / T and S[i][j] = ln(p(i,j) / (p(i) p(j))) / (-ln p(i,j)).
+    Readings where the formula is undefined: S = -1 when p(i,j) = 0 (the pair never co-occurs) and
+    S = 1 when p(i,j) = 1 (both channels are in every token's set). Entries below `threshold` are
+    set to 0 (the pages suggest 0.2); threshold <= -1 keeps every entry.
+    """
+    O = np.asarray(O, dtype=np.float64)
+    p = O / float(T)
+    pi = np.diag(p).copy()
+    S = np.full(p.shape, -1.0)
+    C = p.shape[0]
+    for i in range(C):
+        for j in range(C):
+            pij = p[i, j]
+            if pij <= 0.0:
+                continue
+            if pij >= 1.0:
+                S[i, j] = 1.0
+                continue
+            S[i, j] = np.log(pij / (pi[i] * pi[j])) / (-np.log(pij))
+    if threshold > -1.0:
+        S = np.where(S >= threshold, S, 0.0)
+    return S

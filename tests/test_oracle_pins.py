@@ -334,3 +334,57 @@ def test_topk_all_zero_row_takes_first_k_channels():
     X = np.zeros((1, 20), np.float32)
     idx, hist = oracle.topk(X, np.ones(20, np.float32), 5)
     assert idx[0].tolist() == [0, 1, 2, 3, 4]
+
+
+# ---------------------------------------------------------------- co-occurrence and NPMI
+
+def test_cooccurrence_hand_counted_example():
+    # three tokens, channels 5, 7, 9 token-dependent (positions 0, 1, 2), channel 3 not:
+    # token sets {5,7,3}, {7,9}, {5,7,9} -> pairs counted by hand
+    idx = np.array([[5, 7, 3], [7, 9, 3], [5, 7, 9]])
+    pos = np.full(12, -1)
+    pos[5], pos[7], pos[9] = 0, 1, 2
+    O = oracle.cooccurrence(idx, pos, 3)
+    expect = np.array([[2, 2, 1],
+                       [2, 3, 2],
+                       [1, 2, 2]])
+    assert (O == expect).all()
+
+
+def test_cooccurrence_properties_on_topk_output():
+    rng = np.random.default_rng(3)
+    T, K, k, C = 200, 96, 8, 24
+    X = rng.standard_normal((T, K)).astype(np.float32)
+    w = np.abs(rng.standard_normal(K)).astype(np.float32)
+    idx, hist = oracle.topk(X, w, k)
+    dep = rng.permutation(K)[:C]           # some channels are token-dependent
+    pos = np.full(K, -1)
+    pos[dep] = np.arange(C)
+    O = oracle.cooccurrence(idx, pos, C)
+    assert (O == O.T).all()
+    assert (np.diag(O) == hist[dep]).all()  # diagonal = how often the channel was picked
+    # each token contributes |S_t ∩ dep|^2 pairs in total
+    n_dep = (pos[idx] >= 0).sum(axis=1)
+    assert O.sum() == (n_dep ** 2).sum()
+    assert (O <= np.minimum.outer(np.diag(O), np.diag(O))).all()
+
+
+def test_npmi_closed_forms():
+    T = 8
+    # channel 0 and 1 independent (p = 1/2 each, together 1/4), 0 and 2 always together,
+    # 0 and 3 never together, channel 4 in every token
+    O = np.array([[4, 2, 4, 0, 4],
+                  [2, 4, 2, 2, 4],
+                  [4, 2, 4, 0, 4],
+                  [0, 2, 0, 4, 4],
+                  [4, 4, 4, 4, 8]])
+    S = oracle.npmi(O, T)
+    assert S[0, 1] == pytest.approx(0.0, abs=1e-15)
+    assert S[0, 2] == pytest.approx(1.0)
+    assert S[0, 3] == -1.0
+    assert S[4, 4] == 1.0                    # p = 1
+    assert np.allclose(np.diag(S)[:4], 1.0)  # a channel with itself
+    assert (S >= -1 - 1e-12).all() and (S <= 1 + 1e-12).all()
+    assert (S == S.T).all()
+    St = oracle.npmi(O, T, threshold=0.2)
+    assert St[0, 1] == 0.0 and St[0, 3] == 0.0 and St[0, 2] == pytest.approx(1.0)
