@@ -17,6 +17,7 @@ Parity status per function (pins live in tests/test_oracle_pins.py):
   qe_forward                   pinned: zero adapters = literal dequant matmul,
                                token independence, identical experts, SVD fixture
   topk                         pinned: brute force, sum(hist) = T*k, order
+  split_channels               pinned: a hand-ranked example with ties, d_in < k + C, count order
   cooccurrence, npmi           pinned: a hand-counted example, symmetry, diagonal = channel counts,
                                closed-form NPMI cases (independent 0, always together 1, never -1)
 """
@@ -189,6 +190,23 @@ def router_near_tie_bound(X, G) -> np.ndarray:
     G = _f32(G).astype(np.float64)
     K = X.shape[1]
     return 2.0 * K * 2.0 ** -24 * (np.abs(X) @ np.abs(G).max(axis=1))
+
+
+def split_channels(hist, k: int, C: int) -> np.ndarray:
+    """Token-dependent channel positions from the calibration histogram ([DR] \u00a7Method).
+
+    Channels are ranked by how often they were in a token's Top-k set (higher count first, equal
+    counts by lower channel index). The first k of that ranking are the token-independent channels
+    the shared expert covers; the next C (= N_r * k) are the token-dependent ones. Returns int32
+    [d_in]: rank - k for those C channels, -1 for every other channel.
+    """
+    h = np.asarray(hist, dtype=np.int64)
+    d = h.shape[0]
+    order = np.lexsort((np.arange(d), -h))   # primary key: count desc; then index asc
+    pos = np.full(d, -1, dtype=np.int32)
+    for r in range(k, min(k + C, d)):
+        pos[order[r]] = r - k
+    return pos
 
 
 def cooccurrence(idx, channel_pos, C: int) -> np.ndarray:

@@ -388,3 +388,35 @@ def test_npmi_closed_forms():
     assert (S == S.T).all()
     St = oracle.npmi(O, T, threshold=0.2)
     assert St[0, 1] == 0.0 and St[0, 3] == 0.0 and St[0, 2] == pytest.approx(1.0)
+
+
+def test_split_channels_hand_ranked_example():
+    # counts:   ch0 3, ch1 9, ch2 3, ch3 0, ch4 9, ch5 5, ch6 3
+    # ranking:  ch1, ch4 (9; lower index first), ch5 (5), ch0, ch2, ch6 (3), ch3 (0)
+    hist = [3, 9, 3, 0, 9, 5, 3]
+    # k = 2 token-independent (ch1, ch4); C = 3 dependent: ch5 -> 0, ch0 -> 1, ch2 -> 2
+    assert oracle.split_channels(hist, 2, 3).tolist() == [1, -1, 2, -1, -1, 0, -1]
+    # C larger than what is left: every remaining channel gets a position
+    assert oracle.split_channels(hist, 2, 10).tolist() == [1, -1, 2, 4, -1, 0, 3]
+    # k = 0: the dependent set starts at the top of the ranking
+    assert oracle.split_channels(hist, 0, 2).tolist() == [-1, 0, -1, -1, 1, -1, -1]
+
+
+def test_split_channels_order_property():
+    rng = np.random.default_rng(3)
+    hist = rng.integers(0, 6, size=500)     # many ties
+    k, C = 16, 128
+    pos = oracle.split_channels(hist, k, C)
+    sel = np.flatnonzero(pos >= 0)
+    assert sorted(pos[sel].tolist()) == list(range(C))
+    by_pos = sel[np.argsort(pos[sel])]
+    # along the positions, counts never increase and equal counts go by index
+    for a, b in zip(by_pos[:-1], by_pos[1:]):
+        assert hist[a] > hist[b] or (hist[a] == hist[b] and a < b)
+    rest = np.flatnonzero(pos < 0)
+    # exactly k channels outrank every selected one; every unselected one is outranked by them
+    outrank = [c for c in rest if hist[c] > hist[by_pos[0]] or (hist[c] == hist[by_pos[0]] and c < by_pos[0])]
+    assert len(outrank) == k
+    below = [c for c in rest if c not in outrank]
+    last = by_pos[-1]
+    assert all(hist[c] < hist[last] or (hist[c] == hist[last] and c > last) for c in below)
