@@ -54,6 +54,16 @@ WORKLOADS = {
 }
 METRIC = "QE linear tokens/s and effective TOPS; % of int8-TC / HBM roofline, 1 B200"
 
+# The calibration statistics: per-token Top-k importance with its histogram, the channel split,
+# the co-occurrence counts of the token-dependent channels and their NPMI.
+CALIB_WORKLOADS = {
+    # name: (T, d, k, N_r, description)
+    "calib72b": (8192, 29568, 32, 8, "Qwen2VL-72B-shaped calibration statistic: T=8192 tokens of the 29568-wide down "
+                                     "projection input, Top-k k=32, N_r=8 (C=256 token-dependent channels), NPMI "
+                                     "threshold 0.2"),
+}
+CALIB_METRIC = "QE calibration statistic tokens/s (Top-k, split, co-occurrence, NPMI); % of HBM roofline, 1 B200"
+
 
 def parse_args():
     ap = argparse.ArgumentParser()
@@ -61,7 +71,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2vl2b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CALIB_WORKLOADS), default="qwen2vl2b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
@@ -457,9 +467,175 @@ def run_ours(args, workload):
         pg.destroy_process_group()
     return 0
 
+# ---------------------------------------------------------------- calibration statistic
+
+def calib_inputs(T, d, seed=0):
+    """Activations with the 72B outlier structure and the weight column means w_mean."""
+    cfg = qi.CONFIGS["qwen2vl72b"]
+    X = qi.to_bf16(qi.outlier_activations(T, d, 4242 + seed, cfg.outlier_spec(d)))
+    w_mean = np.abs(qi.gaussian(d, 0.02, 4243)).astype(np.float32)
+    return X, w_mean
+
+
+def calib_oracle_run(X, w_mean, k, C):
+    """The oracle's calibration chain on a token sample. Returns seconds."""
+    import oracle
+    t0 = time.perf_counter()
+    idx, hist = oracle.topk(X, w_mean, k)
+    pos = oracle.split_channels(hist, k, C)
+    O = oracle.cooccurrence(idx, pos, C)
+    oracle.npmi(O, X.shape[0], 0.2)
+    return time.perf_counter() - t0
+
+
+def run_calib(args, workload):
+    T, d, k, n_routed, desc_txt = CALIB_WORKLOADS[workload]
+    C = n_routed * k
+    rank, local_rank, world = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cores = 1   # the oracle's Top-k, counts and NPMI run on one thread
+        sample = max(1, min(args.cpu_sample_tokens, T))
+        X, w_mean = calib_inputs(sample, d)
+        for _ in range(args.warmup):
+            calib_oracle_run(X[:4], w_mean, k, C)
+        tot = sum(calib_oracle_run(X, w_mean, k, C) for _ in range(args.steps))
+        value = sample * args.steps / tot
+        print(json.dumps({
+            "impl": "reference", "metric": CALIB_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/int64/f64",
+            "data": "synthetic", "config": {"workload": workload, "description": desc_txt, "T": T,
+                                            "sample_tokens_per_step": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{sample} tokens through Top-k, split, co-occurrence and NPMI per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }), flush=True)
+        return 0
+
+    import torch
+    import quantized_gemm_moe_b200 as qe
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    qe.load()
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    X_h, w_mean_h = calib_inputs(T, d, seed=rank)
+    X = X_h.to(dev)
+    w_mean = torch.from_numpy(w_mean_h).to(dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    hist = torch.empty(d, dtype=torch.int32, device=dev)
+    pos = torch.empty(d, dtype=torch.int32, device=dev)
+    O = torch.empty((C, C), dtype=torch.int32, device=dev)
+    S = torch.empty((C, C), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def step(record=False):
+        if record:
+            ev[0].record(stream)
+        qe.topk_importance(X, w_mean, k, idx, hist)
+        if record:
+            ev[1].record(stream)
+        qe.split_channels(hist, k, C, pos)
+        if record:
+            ev[2].record(stream)
+        qe.cooccurrence_npmi(idx, pos, C, O, S, 0.2)
+        if record:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    step_ms = np.zeros(args.steps)
+    part_ms = np.zeros((args.steps, 3))
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for s_i in range(args.steps):
+            flush.zero_()
+            step(record=True)
+            torch.cuda.synchronize()
+            step_ms[s_i] = ev[0].elapsed_time(ev[3])
+            part_ms[s_i] = [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
+    if pg:
+        pg.barrier()
+    total_ms = max_over_ranks(float(step_ms.sum()), pg, dev)
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+    parts = part_ms.mean(axis=0)
+
+    peaks = load_peaks()
+    # Top-k reads X (bf16) and w_mean once and writes idx and hist
+    topk_bytes = T * d * 2 + d * 4 + T * k * 4 + d * 4
+    ach = topk_bytes / (parts[0] / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+            "traffic": read_traffic("quantized_gemm_moe_b200/csrc/k_misc.cu", "topk_" + workload), "kernel": "topk",
+            "peak_source": peaks["source"] + " hbm copy"}
+
+    e2e = None
+    if not args.no_e2e:
+        xh = X_h.contiguous().pin_memory()
+        Oh = torch.empty((C, C), dtype=torch.int32).pin_memory()
+        Sh = torch.empty((C, C), dtype=torch.float32).pin_memory()
+        e_ms = 0.0
+        for it in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            X.copy_(xh, non_blocking=True)
+            step()
+            Oh.copy_(O, non_blocking=True)
+            Sh.copy_(S, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= args.warmup:
+                e_ms += e0.elapsed_time(e1)
+        e_ms = max_over_ranks(e_ms, pg, dev)
+        e2e = {"value": world * T * args.steps / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": xh.numel() * xh.element_size(), "d2h_bytes_per_step": 2 * C * C * 4}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = max(1, min(args.cpu_sample_tokens, T))
+        secs = calib_oracle_run(X_h[:sample], w_mean_h, k, C)
+        cpu = {"value": sample / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{sample} tokens through Top-k, split, co-occurrence and NPMI"}
+    line = {
+        "metric": CALIB_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32/int32", "data": "synthetic",
+        "config": {"workload": workload, "description": desc_txt, "T_per_gpu": T, "d": d, "k": k, "C": C,
+                   "l2": "inputs larger than L2 (X is 484 MB) and a 256 MB flush between steps",
+                   "parallelism": f"replicas x{world}"},
+        "stage_ms": {"topk": float(parts[0]), "split": float(parts[1]), "cooc_npmi": float(parts[2])},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "gpu_launches": 4 * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
 
 def main():
     args = parse_args()
+    if args.workload in CALIB_WORKLOADS:
+        return run_calib(args, args.workload)
     if args.impl == "reference":
         return run_reference(args, args.workload)
     return run_ours(args, args.workload)

@@ -279,6 +279,42 @@ QE_API const char* qe_last_cuda_error(void);
 QE_API qe_status qe_device_error(void* stream, int32_t* code, int32_t clear);
 
 /*
+ * Split of the channels by calibration frequency ([DR]: Quant Experts, MCISLAB DeepRead summary,
+ * Method: the k channels most often in a token's Top-k set are token-independent and go to the
+ * shared expert; the next N_r * k are token-dependent and are clustered into routed experts).
+ *   hist        (device) int32 [d_in]: per-channel Top-k counts (qe_topk_importance's histogram)
+ *   k           number of token-independent channels (0 <= k <= 128)
+ *   C           number of token-dependent channels (N_r * k; 1 <= C <= 4096)
+ *   channel_pos (device) out int32 [d_in]: for the channel of rank r (higher count first, equal
+ *               counts by lower channel index) r - k when k <= r < k + C, else -1.
+ * One CTA, exact (integer compares only). Limits: 1 <= d_in <= 1<<24, else QE_ERR_INVALID_ARG.
+ */
+QE_API qe_status qe_split_channels(const int32_t* hist, int32_t d_in, int32_t k, int32_t C, int32_t* channel_pos,
+                                   void* stream);
+
+/*
+ * Co-occurrence of the token-dependent channels and their NPMI similarity ([DR]: Quant Experts,
+ * MCISLAB DeepRead summary, Method, routed experts: channels that are often important in the
+ * same token are counted together, and NPMI measures how strongly a pair co-occurs).
+ *   idx         (device) int32 [T][k]: each token's Top-k channels (as qe_topk_importance writes)
+ *   channel_pos (device) int32 [d_in]: the position in [0, C) of each token-dependent channel,
+ *               -1 for every other channel. Distinct channels need distinct positions.
+ *   O           (device) out int32 [C][C]: O[i][j] = number of tokens whose set holds both
+ *               channels i and j; O[i][i] = number of tokens holding channel i. Zeroed first.
+ *   S           (device) out fp32 [C][C], may be NULL: NPMI with p(i) = O[i][i]/T and
+ *               p(i,j) = O[i][j]/T, S = ln(p(i,j)/(p(i)p(j))) / (-ln p(i,j)), computed in fp64
+ *               and rounded once; -1 where p(i,j) = 0 and 1 where p(i,j) = 1. With
+ *               threshold > -1, entries below it become 0 (the pages suggest 0.2).
+ * Each idx row must name distinct channels (a Top-k set does). Counts use integer atomics, so
+ * the result is exact and does not depend on the schedule. Index values outside [0, d_in) and
+ * positions outside [0, C) are ignored.
+ * Limits: 1 <= k <= 128, 1 <= C <= 4096, 0 <= T <= 1<<20 (else QE_ERR_INVALID_ARG).
+ */
+QE_API qe_status qe_cooccurrence_npmi(const int32_t* idx, int32_t T, int32_t k, const int32_t* channel_pos,
+                                      int32_t d_in, int32_t C, int32_t* O, float* S, float threshold,
+                                      void* stream);
+
+/*
  * Self-test of the bounded device waits (a library convenience; the paper has no counterpart).
  * Launches one thread that waits on a barrier nothing arrives on, for at most limit_us
  * microseconds (1 .. 1000000). The wait runs out, records code 0x107 in the device error word,

@@ -28,7 +28,7 @@ import torch
 
 __all__ = [
     "LayerConfig", "Projection", "CONFIGS", "config_by_name",
-    "outlier_activations", "gaussian", "layer_inputs", "to_bf16",
+    "outlier_activations", "gaussian", "layer_inputs", "to_bf16", "topk_like_sets",
 ]
 
 
@@ -94,6 +94,37 @@ def outlier_activations(T: int, d: int, seed: int, spec: OutlierSpec) -> np.ndar
             if spec.draw_hi > spec.draw_lo else np.full(k, spec.draw_lo, np.float32)
         x[t, ch] *= mult
     return x
+
+
+def topk_like_sets(T: int, d: int, k: int, seed: int) -> np.ndarray:
+    """Seeded int32 [T, k] rows of k distinct channels in [0, d), shaped like Top-k sets.
+
+    A quarter of each row is a fixed always-important set; half comes from the token's modality
+    pool (image tokens first, then text tokens; pools of 8k channels, weights falling as
+    1/(rank+1), so a few channels co-occur often); the rest is uniform over the other channels.
+    """
+    g = _rng(seed)
+    n_always, n_pool = k // 4, k // 2
+    n_rest = k - n_always - n_pool
+    perm = g.permutation(d)
+    always = perm[:n_always]
+    psz = min(8 * k, max(n_pool, (d - n_always) // 2))
+    pools = [perm[n_always:n_always + psz], perm[n_always + psz:n_always + 2 * psz]]
+    w = 1.0 / np.arange(1, psz + 1)
+    w /= w.sum()
+    out = np.empty((T, k), dtype=np.int32)
+    for t in range(T):
+        pool = pools[0] if t < T // 2 else pools[1]
+        ch = np.concatenate([always, g.choice(pool, size=n_pool, replace=False, p=w)])
+        taken = set(ch.tolist())
+        rest = []
+        while len(rest) < n_rest:          # uniform draws, skipping channels already in the row
+            c = int(g.integers(0, d))
+            if c not in taken:
+                taken.add(c)
+                rest.append(c)
+        out[t] = g.permutation(np.concatenate([ch, np.asarray(rest, dtype=ch.dtype)]))
+    return out
 
 
 def gaussian(shape, std: float, seed: int) -> np.ndarray:

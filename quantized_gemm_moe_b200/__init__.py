@@ -24,7 +24,7 @@ EXPORTS = (
     "qe_pack_adapters", "qe_topk_importance", "qe_route", "qe_linear_forward", "qe_status_string",
     "qe_last_cuda_error", "qe_device_error", "qe_unpack_weights", "qe_act_quant", "qe_linear_forward_debug",
     "qe_linear_forward_stages", "qe_linear_kernel_launches", "qe_linear_forward_noalloc",
-    "qe_selftest_wait_timeout",
+    "qe_selftest_wait_timeout", "qe_split_channels", "qe_cooccurrence_npmi",
 )
 # fixed scratch of qe_linear_forward_noalloc (bytes), as declared in include/qe.h
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -88,6 +88,8 @@ def load() -> ctypes.CDLL:
         "qe_unpack_weights": ([D, P, P, P], I),
         "qe_act_quant": ([P, I, P, I, I, I, P, P, P], I),
         "qe_selftest_wait_timeout": ([I, P], I),
+        "qe_split_channels": ([P, I, I, I, P, P], I),
+        "qe_cooccurrence_npmi": ([P, I, I, P, I, I, P, P, ctypes.c_float, P], I),
     }
     for name, (args, res) in sigs.items():
         f = getattr(L, name)
@@ -169,6 +171,21 @@ def topk_importance(X, w_mean, k, idx, hist=None, accumulate=False, stream=None)
     T, K = X.shape
     _check(load().qe_topk_importance(_ptr(X), _dtype(X), _ptr(w_mean), T, K, k, _ptr(idx), _ptr(hist),
                                      1 if accumulate else 0, _stream(stream)), "qe_topk_importance")
+
+
+def split_channels(hist, k, C, channel_pos, stream=None):
+    """channel_pos[c] = rank(c) - k for the C channels after the k most frequent ones, else -1."""
+    _need_cuda(hist, channel_pos)
+    _check(load().qe_split_channels(_ptr(hist), hist.numel(), k, C, _ptr(channel_pos), _stream(stream)),
+           "qe_split_channels")
+
+
+def cooccurrence_npmi(idx, channel_pos, C, O, S=None, threshold=-1.0, stream=None):
+    """Counts O[i][j] (int32 [C][C]) and, when S is given, writes their NPMI into S (fp32 [C][C])."""
+    _need_cuda(idx, channel_pos, O, S)
+    T, k = idx.shape
+    _check(load().qe_cooccurrence_npmi(_ptr(idx), T, k, _ptr(channel_pos), channel_pos.numel(), C, _ptr(O), _ptr(S),
+                                       float(threshold), _stream(stream)), "qe_cooccurrence_npmi")
 
 
 def route(X, G, expert, perm, offsets, logits=None, stream=None):

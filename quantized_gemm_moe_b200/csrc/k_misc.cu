@@ -31,10 +31,12 @@ __device__ __forceinline__ uint32_t order_key(float v) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// marked_only: the CTAs stride over the tokens and take only those whose first index slot holds
+// the mark -1 (left by k_topk_stream for rows it does not resolve).
 template <bool BF16>
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const void* __restrict__ X, const float* __restrict__ w,
                                                        int T, int K, int k, int32_t* __restrict__ idx_out,
-                                                       int32_t* __restrict__ hist) {
+                                                       int32_t* __restrict__ hist, int marked_only) {
   extern __shared__ uint32_t keys[];  // [K]
   __shared__ int whist[kTopkWarps][256];
   __shared__ int digits[256];
@@ -42,7 +44,24 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const void* __restrict__ 
   __shared__ int s_remaining;
   __shared__ int sgt[kTopkThreads], seq[kTopkThreads];
   __shared__ unsigned long long sel[128];
-  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ int mlist[kTopkThreads];
+  __shared__ int s_nm;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int tb = blockIdx.x; tb < T; tb += gridDim.x * kTopkThreads) {
+  int nm = 1;
+  if (marked_only) {
+    // this CTA's next kTopkThreads tokens, one per thread: list the marked ones
+    __syncthreads();
+    if (tid == 0) s_nm = 0;
+    __syncthreads();
+    const int tc = tb + tid * static_cast<int>(gridDim.x);
+    if (tc < T && idx_out[static_cast<size_t>(tc) * k] < 0) mlist[atomicAdd(&s_nm, 1)] = tc;
+    __syncthreads();
+    nm = s_nm;
+  }
+  for (int q = 0; q < nm; ++q) {
+  const int t = marked_only ? mlist[q] : tb;
+  __syncthreads();  // shared memory of the previous token is free
   const size_t rowoff = static_cast<size_t>(t) * K;
   for (int k0 = tid * 8; k0 < K; k0 += kTopkThreads * 8) {
     float xv[8];
@@ -191,6 +210,550 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const void* __restrict__ 
     idx_out[static_cast<size_t>(t) * k + i] = c;
     if (hist) atomicAdd(hist + c, 1);
   }
+  }
+  }
+}
+
+// ------------------------------------------------------------------ Top-k importance, streaming form
+// bf16 rows with 7936 <= K <= 31744. Persistent CTAs (one per SM, 1024 threads) stride over the
+// tokens; each token's row is staged in shared memory by an untiled bulk copy, two rows in
+// flight. Warps 0-30 score: their weight column means live in registers (4 chunks of 8 channels
+// per thread); warp 31 selects. Per token:
+//  1. scores s = fl32(|x| * w); each scoring thread keeps the maximum of each of its chunks.
+//     Every scoring warp takes the j-th largest of its 32 lane maxima (j = ceil(k/31)): a score
+//     that j distinct channels of the warp reach. tau = the minimum over the 31 warps is reached
+//     by at least 31 j >= k channels, so every channel of the Top-k set has s >= tau;
+//  2. the chunks whose maximum reaches tau are listed (with their 8 weights) by their owners,
+//     at offsets from per-warp counts; one thread per listed chunk then scores it again and
+//     appends its channels with s >= tau (the candidates) as 64-bit keys (score desc, channel
+//     asc);
+//  3. warp 31 selects from the candidates while the others score the next token. With the
+//     score keys in registers, a bit-serial search (two bits per step, warp sums) raises a
+//     threshold v while at least k candidates reach it, and stops once at most kTSSel do; the
+//     candidates with key >= v are ranked among themselves by counting, and ranks below k are
+//     the output slots.
+// A row with more than kTSCap candidates, or more than kTSSel at or above the final threshold
+// (rows of mostly equal scores), is marked -1 in its first slot and resolved by k_topk
+// (marked_only).
+constexpr int kTSThreads = 1024;
+constexpr int kTSWarps = kTSThreads / 32;
+constexpr int kTSScorers = kTSThreads - 32;  // warps 0-30
+constexpr int kTSChunks = 4;  // channels (tid + 992 j) * 8 .. +7, j < 4: K <= 31744
+constexpr int kTSCap = 1024;
+constexpr int kTSChunkCap = 512;
+constexpr int kTSRegKeys = 12;  // score keys per lane held in registers by the selecting warp
+constexpr int kTSSel = 64;
+constexpr int kTSMinK = kTSScorers * 8;
+constexpr int kTSMaxK = kTSScorers * 8 * kTSChunks;
+
+__device__ __forceinline__ unsigned long long topk_comp(float s, int c) {
+  return (static_cast<unsigned long long>(order_key(s)) << 32) |
+         static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(c));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// the 8 scores of one chunk (8 bf16 x values, 8 weights)
+__device__ __forceinline__ void chunk_scores(const uint4 u, const float (&w8)[8], float (&sc)[8]) {
+  const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    sc[2 * i] = __fmul_rn(fabsf(__uint_as_float(uu[i] << 16)), w8[2 * i]);
+    sc[2 * i + 1] = __fmul_rn(fabsf(__uint_as_float(uu[i] & 0xFFFF0000u)), w8[2 * i + 1]);
+  }
+}
+
+// Step 3 for one token, by one warp: candidates ck[0..nc) -> idx_out row t (+ hist).
+__device__ __forceinline__ void topk_select(int t, const unsigned long long* ck, int nc, int k,
+                                            int32_t* __restrict__ idx_out, int32_t* __restrict__ hist,
+                                            unsigned long long* skey, int lane) {
+  if (nc < k || nc > 32 * kTSRegKeys) {
+    if (lane == 0) idx_out[static_cast<size_t>(t) * k] = -1;
+    return;
+  }
+  uint32_t key[kTSRegKeys];
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int r = 0; r < kTSRegKeys; ++r) {
+    const int i = lane + 32 * r;
+    key[r] = i < nc ? static_cast<uint32_t>(ck[i] >> 32) : 0u;  // 0 is below every score key
+    if (i < nc) {
+      kmin = min(kmin, key[r]);
+      kmax = max(kmax, key[r]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  // Every key lies in [kmin, kmax], so the bits above the highest differing bit are kmax's.
+  // Invariant: count(key >= v) >= k. Stop early once count <= kTSSel.
+  uint32_t v = kmax;
+  if (kmin != kmax) {
+    int b = 31 - __clz(kmin ^ kmax);
+    v = b == 31 ? 0u : (kmax & ~((2u << b) - 1u));
+    int cv = nc;
+    for (; b >= 1 && cv > kTSSel; b -= 2) {
+      const uint32_t p1 = v | (1u << (b - 1)), p2 = v | (2u << (b - 1)), p3 = v | (3u << (b - 1));
+      int c1 = 0, c2 = 0, c3 = 0;
+#pragma unroll
+      for (int r = 0; r < kTSRegKeys; ++r) {
+        c1 += key[r] >= p1 ? 1 : 0;
+        c2 += key[r] >= p2 ? 1 : 0;
+        c3 += key[r] >= p3 ? 1 : 0;
+      }
+      c1 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c1)));
+      c2 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c2)));
+      c3 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c3)));
+      if (c3 >= k) {
+        v = p3;
+        cv = c3;
+      } else if (c2 >= k) {
+        v = p2;
+        cv = c2;
+      } else if (c1 >= k) {
+        v = p1;
+        cv = c1;
+      }
+    }
+    if (b == 0 && cv > kTSSel) {
+      int c1 = 0;
+#pragma unroll
+      for (int r = 0; r < kTSRegKeys; ++r) c1 += key[r] >= (v | 1u) ? 1 : 0;
+      if (static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c1))) >= k) v |= 1u;
+    }
+  }
+  // the set S = {score key >= v} (k of them at least): compact, rank by counting within S
+  int ns = 0;
+#pragma unroll
+  for (int r = 0; r < kTSRegKeys; ++r) {
+    const int i = lane + 32 * r;
+    const bool in = i < nc && key[r] >= v;
+    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+    const int at = ns + __popc(bal & ((1u << lane) - 1u));
+    if (in && at < kTSSel) skey[at] = ck[i];
+    ns += __popc(bal);
+  }
+  if (ns > kTSSel) {
+    if (lane == 0) idx_out[static_cast<size_t>(t) * k] = -1;
+    return;
+  }
+  for (int x = ns + lane; x < ((ns + 7) & ~7); x += 32) skey[x] = 0ull;  // pad to a multiple of 8
+  __syncwarp();
+  for (int q = lane; q < ns; q += 32) {
+    const unsigned long long me = skey[q];
+    int r = 0;
+    for (int x = 0; x < ns; x += 8) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r += skey[x + u] > me ? 1 : 0;
+    }
+    if (r < k) {
+      const int c = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(me & 0xFFFFFFFFull));
+      idx_out[static_cast<size_t>(t) * k + r] = c;
+      if (hist) atomicAdd(hist + c, 1);
+    }
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* __restrict__ X,
+                                                               const float* __restrict__ w, int T, int K, int k,
+                                                               int32_t* __restrict__ idx_out,
+                                                               int32_t* __restrict__ hist, int* err) {
+  extern __shared__ __align__(128) uint16_t rows[];  // [2][K]
+  __shared__ unsigned long long ckey[2][kTSCap];
+  __shared__ unsigned long long skey[kTSSel + 8];
+  __shared__ __align__(16) float cw[kTSChunkCap][8];
+  __shared__ int clist[kTSChunkCap];
+  __shared__ int wcnt[kTSWarps];
+  __shared__ float wthr[kTSWarps];
+  __shared__ int s_nc[2];
+  __shared__ __align__(8) uint64_t full[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool scorer = warp < kTSWarps - 1;
+  const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
+  float wr[kTSChunks][8];
+#pragma unroll
+  for (int j = 0; j < kTSChunks; ++j) {
+    const int c0 = (tid + kTSScorers * j) * 8;
+    if (scorer && c0 < K) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(w + c0));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(w + c0) + 1);
+      wr[j][0] = a.x; wr[j][1] = a.y; wr[j][2] = a.z; wr[j][3] = a.w;
+      wr[j][4] = b.x; wr[j][5] = b.y; wr[j][6] = b.z; wr[j][7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wr[j][i] = 0.0f;
+    }
+  }
+  if (tid == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      const int t = blockIdx.x + b * static_cast<int>(gridDim.x);
+      if (t < T) {
+        mbar_arrive_expect_tx(&full[b], row_bytes);
+        bulk_load(rows + b * K, X + static_cast<size_t>(t) * K, row_bytes, &full[b]);
+      }
+    }
+  }
+  if (!scorer) {
+    // The selecting warp: it takes part in the same four barriers per token as the scoring
+    // warps and finishes each token while the next row is scored.
+    if (lane == 0) wcnt[warp] = 0;
+    int it = 0, prev_t = -1;
+    for (int t = blockIdx.x; t < T; t += gridDim.x, ++it) {
+      if (prev_t >= 0) topk_select(prev_t, ckey[(it - 1) & 1], s_nc[(it - 1) & 1], k, idx_out, hist, skey, lane);
+      if (__syncthreads_or(0)) return;  // a row copy never landed (the scoring warps stop too)
+      __syncthreads();
+      __syncthreads();
+      __syncthreads();
+      prev_t = t;
+    }
+    if (prev_t >= 0) topk_select(prev_t, ckey[(it - 1) & 1], s_nc[(it - 1) & 1], k, idx_out, hist, skey, lane);
+    return;
+  }
+  const int jj = (k + kTSWarps - 2) / (kTSWarps - 1);
+  int it = 0;
+  for (int t = blockIdx.x; t < T; t += gridDim.x, ++it) {
+    const int b = it & 1;
+    const uint16_t* row = rows + b * K;
+    const bool ok = mbar_wait(&full[b], static_cast<uint32_t>((it >> 1) & 1), err, DEVERR_WAIT_PRODUCER);
+    // 1. chunk maxima; the warp's j-th largest lane maximum
+    float cmax[kTSChunks];
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kTSChunks; ++j) {
+      const int c0 = (tid + kTSScorers * j) * 8;
+      cmax[j] = -INFINITY;
+      if (c0 < K) {
+        float sc[8];
+        chunk_scores(*reinterpret_cast<const uint4*>(row + c0), wr[j], sc);
+        cmax[j] = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])),
+                        fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
+        m = fmaxf(m, cmax[j]);
+      }
+    }
+    float tw = warp_max(m);
+    for (int r = 1; r < jj; ++r) {
+      // drop one lane holding the current maximum, take the maximum of the rest
+      const uint32_t holder = __ballot_sync(0xffffffffu, m == tw);
+      if (lane == __ffs(holder) - 1) m = -INFINITY;
+      tw = warp_max(m);
+    }
+    if (lane == 0) wthr[warp] = tw;
+    if (tid == 0) s_nc[b] = 0;
+    if (__syncthreads_or(!ok)) {
+      // a row copy never landed: let the other buffer's copy (if one was issued) finish, then stop
+      if (tid == 0 && t + static_cast<int>(gridDim.x) < T)
+        mbar_wait_for(&full[b ^ 1], static_cast<uint32_t>(((it + 1) >> 1) & 1), nullptr, 0, 10000000ull);
+      return;
+    }
+    const float tau = warp_min(lane < kTSWarps - 1 ? wthr[lane] : INFINITY);
+    // 2a. list the chunks that reach tau, with their weights: per-warp counts, then every warp
+    //     finds its offset from the counts of the warps before it
+    uint32_t bal[kTSChunks];
+    int wc = 0;
+#pragma unroll
+    for (int j = 0; j < kTSChunks; ++j) {
+      bal[j] = __ballot_sync(0xffffffffu, cmax[j] >= tau);
+      wc += __popc(bal[j]);
+    }
+    if (lane == 0) wcnt[warp] = wc;
+    __syncthreads();
+    int incl = wcnt[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int nch = __shfl_sync(0xffffffffu, incl, 31);
+    int slot = __shfl_sync(0xffffffffu, incl, warp) - wc;
+#pragma unroll
+    for (int j = 0; j < kTSChunks; ++j) {
+      if ((bal[j] >> lane) & 1u) {
+        const int at = slot + __popc(bal[j] & ((1u << lane) - 1u));
+        if (at < kTSChunkCap) {
+          clist[at] = (tid + kTSScorers * j) * 8;
+          *reinterpret_cast<float4*>(&cw[at][0]) = make_float4(wr[j][0], wr[j][1], wr[j][2], wr[j][3]);
+          *reinterpret_cast<float4*>(&cw[at][4]) = make_float4(wr[j][4], wr[j][5], wr[j][6], wr[j][7]);
+        }
+      }
+      slot += __popc(bal[j]);
+    }
+    __syncthreads();
+    // 2b. one thread per listed chunk: its channels with s >= tau become candidates
+    if (nch > kTSChunkCap) {
+      if (tid == 0) s_nc[b] = kTSCap + 1;  // too many: the row goes to the radix-select kernel
+    } else if (warp * 32 < nch) {
+      uint32_t m8 = 0u;
+      float sc[8];
+      int c0 = 0;
+      if (tid < nch) {
+        c0 = clist[tid];
+        float w8[8];
+        const float4 wa = *reinterpret_cast<const float4*>(&cw[tid][0]);
+        const float4 wb = *reinterpret_cast<const float4*>(&cw[tid][4]);
+        w8[0] = wa.x; w8[1] = wa.y; w8[2] = wa.z; w8[3] = wa.w;
+        w8[4] = wb.x; w8[5] = wb.y; w8[6] = wb.z; w8[7] = wb.w;
+        chunk_scores(*reinterpret_cast<const uint4*>(row + c0), w8, sc);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8 |= (sc[i] >= tau ? 1u : 0u) << i;
+      }
+      const int cnt = __popc(m8);
+      int ic = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, ic, o);
+        if (lane >= o) ic += y;
+      }
+      int base = 0;
+      if (lane == 31 && ic > 0) base = atomicAdd(&s_nc[b], ic);
+      base = __shfl_sync(0xffffffffu, base, 31);
+      int p = base + ic - cnt;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if ((m8 >> i) & 1u) {
+          if (p < kTSCap) ckey[b][p] = topk_comp(sc[i], c0 + i);
+          ++p;
+        }
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      // every thread is done with this row: stage the token two steps ahead into the buffer
+      const int t2 = t + 2 * static_cast<int>(gridDim.x);
+      if (t2 < T) {
+        mbar_arrive_expect_tx(&full[b], row_bytes);
+        bulk_load(rows + b * K, X + static_cast<size_t>(t2) * K, row_bytes, &full[b]);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ channel split by frequency
+// Ranks channels by calibration count (higher first, equal counts by lower index). Rank r in
+// [k, k + C) gets position r - k; every other channel gets -1. One CTA, the counts staged in
+// shared memory as order-preserving keys when they fit: a radix select (4 passes
+// of 8 bits over order-preserving keys) finds the count v* of the n-th ranked channel,
+// n = min(k + C, d); one pass in index order then compacts the channels above v* and numbers
+// the ties at v* by block scans; the channels above v* (fewer than n) are ranked among
+// themselves by counting.
+constexpr int kSplitThreads = 1024;
+constexpr int kSplitMaxSel = 4096 + 128;
+constexpr int kSplitStageMax = 45056;  // counts staged in shared memory up to this many channels (176 KB)
+
+__device__ __forceinline__ uint32_t split_key(int32_t v) { return static_cast<uint32_t>(v) ^ 0x80000000u; }
+
+// exclusive scan of v over the block (kSplitThreads threads); *total gets the block sum
+__device__ __forceinline__ int split_block_scan(int v, int* wt, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wt[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int t = wt[lane];
+    int sc = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, sc, o);
+      if (lane >= o) sc += y;
+    }
+    wt[lane] = sc - t;
+    if (lane == 31) wt[32] = sc;
+  }
+  __syncthreads();
+  const int ex = wt[warp] + x - v;
+  *total = wt[32];
+  __syncthreads();
+  return ex;
+}
+
+// keys of the counts: staged in shared memory when they fit (staged != 0), else read from hist
+__device__ __forceinline__ uint32_t split_key_at(const int32_t* __restrict__ hist, const uint32_t* sk, bool staged,
+                                                 int c) {
+  return staged ? sk[c] : split_key(hist[c]);
+}
+
+__global__ void __launch_bounds__(kSplitThreads) k_split_channels(const int32_t* __restrict__ hist, int d, int k,
+                                                                   int C, int32_t* __restrict__ pos, int staged) {
+  extern __shared__ uint32_t sk[];  // [d] when staged
+  __shared__ int bins[256];
+  __shared__ int wt[33];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_rem;
+  __shared__ int a_idx[kSplitMaxSel];
+  __shared__ uint32_t a_key[kSplitMaxSel];
+  const int tid = threadIdx.x;
+  const int n = min(k + C, d);
+  if (staged)
+    for (int c = tid; c < d; c += kSplitThreads) sk[c] = split_key(hist[c]);
+  // radix select of the n-th largest key
+  uint32_t prefix = 0, mask = 0;
+  int rem = n;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kSplitThreads) bins[i] = 0;
+    __syncthreads();
+    for (int base = 0; base < d; base += kSplitThreads) {
+      const int c = base + tid;
+      const uint32_t u = c < d ? split_key_at(hist, sk, staged, c) : 0u;
+      const bool match = c < d && (u & mask) == prefix;
+      const uint32_t active = __ballot_sync(0xffffffffu, match);
+      if (match) {
+        // one add per distinct digit in the warp: counts mostly share their high bits
+        const int dg = static_cast<int>((u >> shift) & 255u);
+        const uint32_t peers = __match_any_sync(active, dg);
+        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&bins[dg], __popc(peers));
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int cum = 0, dg = 255;
+      for (; dg > 0; --dg) {
+        if (cum + bins[dg] >= rem) break;
+        cum += bins[dg];
+      }
+      s_prefix = prefix | (static_cast<uint32_t>(dg) << shift);
+      s_rem = rem - cum;
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    rem = s_rem;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  // prefix = key of v*; n - rem channels lie above it, the first rem ties (by index) are taken
+  const int nA = n - rem;
+  int runA = 0, runB = 0;
+  for (int base = 0; base < d; base += kSplitThreads) {
+    const int c = base + tid;
+    const uint32_t u = c < d ? split_key_at(hist, sk, staged, c) : 0u;
+    const bool fa = c < d && u > prefix, fb = c < d && u == prefix;
+    int tot;
+    const int ex = split_block_scan((fa ? 1 : 0) | (fb ? 0x10000 : 0), wt, &tot);
+    if (fa) {
+      const int slot = runA + (ex & 0xffff);
+      a_idx[slot] = c;
+      a_key[slot] = u;
+    }
+    int p = -1;
+    if (fb) {
+      const int e = runB + (ex >> 16);
+      if (e < rem && nA + e >= k) p = nA + e - k;
+    }
+    if (c < d && !fa) pos[c] = p;
+    runA += tot & 0xffff;
+    runB += tot >> 16;
+  }
+  __syncthreads();
+  for (int i = tid; i < nA; i += kSplitThreads) {
+    const uint32_t u = a_key[i];
+    const int c = a_idx[i];
+    int r = 0;
+    for (int j = 0; j < nA; ++j) {
+      const uint32_t uj = a_key[j];
+      r += (uj > u || (uj == u && a_idx[j] < c)) ? 1 : 0;
+    }
+    pos[c] = r >= k ? r - k : -1;
+  }
+}
+
+// ------------------------------------------------------------------ co-occurrence and NPMI
+// O[i][j] = number of tokens whose Top-k set holds both token-dependent channels i and j.
+// CTA (row block of RB rows, token chunk): the block's RB x C counters live in shared memory.
+// The chunk's index rows are staged in batches, mapped through channel_pos to positions (int16,
+// -1 for other channels) by all threads at once. A warp then takes a token with its positions in
+// lane registers; for every position inside the row block (a ballot) it adds 1 to that counter
+// row at each of the token's positions (shared-memory atomics). The block finally adds its counts
+// to O with integer atomics, so the result does not depend on the schedule.
+constexpr int kCoocThreads = 512;
+constexpr int kCoocWarps = kCoocThreads / 32;
+constexpr int kCoocCounters = 16384;  // 64 KB of counters per CTA
+constexpr int kCoocStage = 16384;     // staged positions per batch (32 KB)
+
+__global__ void __launch_bounds__(kCoocThreads) k_cooc(const int32_t* __restrict__ idx, int T, int k,
+                                                        const int32_t* __restrict__ pos, int d_in, int C, int RB,
+                                                        int tokens_per_cta, int32_t* __restrict__ O) {
+  extern __shared__ __align__(16) int cnt[];  // [RB][C], then int16 positions [batch][k]
+  int16_t* qs = reinterpret_cast<int16_t*>(cnt + RB * C);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = blockIdx.x * RB;
+  const int rows = min(RB, C - r0);
+  const int t0 = blockIdx.y * tokens_per_cta, t1 = min(T, t0 + tokens_per_cta);
+  const int batch = kCoocStage / k;
+  for (int i = threadIdx.x; i < RB * C; i += kCoocThreads) cnt[i] = 0;
+  for (int tb = t0; tb < t1; tb += batch) {
+    const int nb = min(batch, t1 - tb);
+    __syncthreads();  // counters zeroed / previous batch consumed
+    const int32_t* src = idx + static_cast<size_t>(tb) * k;
+    for (int e = threadIdx.x; e < nb * k; e += kCoocThreads) {
+      const int c = src[e];
+      int m = -1;
+      if (c >= 0 && c < d_in) m = pos[c];
+      qs[e] = static_cast<int16_t>((m >= 0 && m < C) ? m : -1);
+    }
+    __syncthreads();
+    for (int tt = warp; tt < nb; tt += kCoocWarps) {
+      const int16_t* q = qs + tt * k;
+      int v[4];
+#pragma unroll
+      for (int s4 = 0; s4 < 4; ++s4) v[s4] = (lane + 32 * s4 < k) ? q[lane + 32 * s4] : -1;
+#pragma unroll
+      for (int s4 = 0; s4 < 4; ++s4) {
+        if (32 * s4 >= k) break;
+        uint32_t hb = __ballot_sync(0xffffffffu, v[s4] >= r0 && v[s4] < r0 + rows);
+        while (hb) {
+          const int la = __ffs(hb) - 1;
+          hb &= hb - 1;
+          int* crow = cnt + (__shfl_sync(0xffffffffu, v[s4], la) - r0) * C;
+#pragma unroll
+          for (int s2 = 0; s2 < 4; ++s2)
+            if (v[s2] >= 0) atomicAdd(crow + v[s2], 1);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < rows * C; i += kCoocThreads)
+    if (cnt[i]) atomicAdd(&O[static_cast<size_t>(r0) * C + i], cnt[i]);
+}
+
+// S[i][j] = NPMI of channels i and j, in fp64 before the final rounding: p(i) = O[i][i] / T,
+// p(i,j) = O[i][j] / T, S = ln(p(i,j) / (p(i) p(j))) / (-ln p(i,j)); -1 where the pair never
+// co-occurs, 1 where it is in every token; entries below threshold -> 0 when threshold > -1.
+__global__ void k_npmi(const int32_t* __restrict__ O, int C, int T, float threshold, float* __restrict__ S) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= C * C) return;
+  const int i = e / C, j = e % C;
+  const double inv_t = 1.0 / static_cast<double>(T);
+  const double pij = O[e] * inv_t;
+  double v;
+  if (pij <= 0.0) {
+    v = -1.0;
+  } else if (pij >= 1.0) {
+    v = 1.0;
+  } else {
+    const double pi = O[static_cast<size_t>(i) * C + i] * inv_t, pj = O[static_cast<size_t>(j) * C + j] * inv_t;
+    v = log(pij / (pi * pj)) / (-log(pij));
+  }
+  if (threshold > -1.0f && v < static_cast<double>(threshold)) v = 0.0;
+  S[e] = static_cast<float>(v);
 }
 
 // Self-test of the bounded waits: one thread waits on a barrier that nothing arrives on. The
@@ -209,18 +772,38 @@ __global__ void k_wait_selftest(int* err, uint64_t limit_ns) {
 
 
 cudaError_t launch_topk(const void* X, bool x_bf16, const float* w_mean, int T, int K, int k, int32_t* idx,
-                        int32_t* hist, cudaStream_t st) {
+                        int32_t* hist, int* err, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const size_t smem = static_cast<size_t>(K) * 4;
   cudaError_t e;
-  if (x_bf16) {
+  if (x_bf16 && K >= kTSMinK && K <= kTSMaxK) {
+    static int n_sm = 0;
+    if (n_sm == 0) {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        n_sm = 148;
+    }
+    const int grid = std::min(T, n_sm);
+    const size_t smem_s = static_cast<size_t>(K) * 2 * 2;
+    e = cudaFuncSetAttribute(k_topk_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_s));
+    if (e != cudaSuccess) return e;
+    k_topk_stream<<<grid, kTSThreads, smem_s, st>>>(static_cast<const uint16_t*>(X), w_mean, T, K, k, idx, hist,
+                                                    err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // rows the streaming pass left unresolved (marked -1)
     e = cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k_topk<true><<<T, kTopkThreads, smem, st>>>(X, w_mean, T, K, k, idx, hist);
+    k_topk<true><<<grid, kTopkThreads, smem, st>>>(X, w_mean, T, K, k, idx, hist, 1);
+  } else if (x_bf16) {
+    e = cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    k_topk<true><<<T, kTopkThreads, smem, st>>>(X, w_mean, T, K, k, idx, hist, 0);
   } else {
     e = cudaFuncSetAttribute(k_topk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k_topk<false><<<T, kTopkThreads, smem, st>>>(X, w_mean, T, K, k, idx, hist);
+    k_topk<false><<<T, kTopkThreads, smem, st>>>(X, w_mean, T, K, k, idx, hist, 0);
   }
   return cudaGetLastError();
 }
@@ -231,5 +814,47 @@ namespace qe {
 cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st) {
   k_wait_selftest<<<1, 32, 0, st>>>(err, limit_ns);
   return cudaGetLastError();
+}
+}  // namespace qe
+
+namespace qe {
+cudaError_t launch_split_channels(const int32_t* hist, int d, int k, int C, int32_t* pos, cudaStream_t st) {
+  const int staged = d <= kSplitStageMax ? 1 : 0;
+  const size_t smem = staged ? static_cast<size_t>(d) * 4 : 0;
+  if (staged) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k_split_channels, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  k_split_channels<<<1, kSplitThreads, smem, st>>>(hist, d, k, C, pos, staged);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cooc_npmi(const int32_t* idx, int T, int k, const int32_t* pos, int d_in, int C, int32_t* O,
+                             float* S, float threshold, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(O, 0, static_cast<size_t>(C) * C * sizeof(int32_t), st);
+  if (e != cudaSuccess) return e;
+  if (T > 0) {
+    // about 16 row blocks: each CTA re-reads its chunk's index rows (cheap), and every token chunk
+    // costs one global add per counter, so about one CTA per SM with long chunks
+    const int RB = std::max(1, std::min(static_cast<int>(ceil_div(C, 16)), kCoocCounters / C));
+    const int nrb = static_cast<int>(ceil_div(C, RB));
+    int chunks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(148, nrb), ceil_div(T, 64))));
+    const int tpc = static_cast<int>(ceil_div(T, chunks));
+    chunks = static_cast<int>(ceil_div(T, tpc));
+    const size_t smem = static_cast<size_t>(RB) * C * sizeof(int) + kCoocStage * sizeof(int16_t);
+    e = cudaFuncSetAttribute(k_cooc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    k_cooc<<<dim3(static_cast<unsigned>(nrb), static_cast<unsigned>(chunks)), kCoocThreads, smem, st>>>(
+        idx, T, k, pos, d_in, C, RB, tpc, O);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (S && T > 0) {
+    const int n = C * C;
+    k_npmi<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, st>>>(O, C, T, threshold, S);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 }  // namespace qe

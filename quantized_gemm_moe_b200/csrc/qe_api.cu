@@ -408,7 +408,7 @@ qe_status qe_topk_importance(const void* X, qe_dtype x_dtype, const float* w_mea
   if ((X && !aligned16(X)) || !aligned16(w_mean)) return QE_ERR_ALIGNMENT;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (hist && !accumulate_hist) QE_CUDA(cudaMemsetAsync(hist, 0, size_t(d_in) * 4, cs), "memset hist");
-  QE_CUDA(launch_topk(X, x_dtype == QE_BF16, w_mean, T, d_in, k, idx, hist, cs), "topk");
+  QE_CUDA(launch_topk(X, x_dtype == QE_BF16, w_mean, T, d_in, k, idx, hist, device_error_ptr(), cs), "topk");
   return QE_OK;
 }
 
@@ -530,6 +530,24 @@ qe_status qe_device_error(void* stream, int32_t* code, int32_t clear) {
   QE_CUDA(read_device_error(&v, clear != 0, static_cast<cudaStream_t>(stream)), "device_error");
   if (code) *code = v;
   return v ? QE_ERR_TIMEOUT : QE_OK;
+}
+
+qe_status qe_split_channels(const int32_t* hist, int32_t d_in, int32_t k, int32_t C, int32_t* channel_pos,
+                            void* stream) {
+  if (d_in < 1 || d_in > (1 << 24) || k < 0 || k > 128 || C < 1 || C > 4096) return QE_ERR_INVALID_ARG;
+  if (!hist || !channel_pos) return QE_ERR_INVALID_ARG;
+  QE_CUDA(launch_split_channels(hist, d_in, k, C, channel_pos, static_cast<cudaStream_t>(stream)), "split_channels");
+  return QE_OK;
+}
+
+qe_status qe_cooccurrence_npmi(const int32_t* idx, int32_t T, int32_t k, const int32_t* channel_pos, int32_t d_in,
+                               int32_t C, int32_t* O, float* S, float threshold, void* stream) {
+  if (T < 0 || T > (1 << 20) || k < 1 || k > 128 || C < 1 || C > 4096 || d_in < 1) return QE_ERR_INVALID_ARG;
+  if (!O || !channel_pos || (T > 0 && !idx)) return QE_ERR_INVALID_ARG;
+  if (!aligned16(O) || (S && !aligned16(S))) return QE_ERR_ALIGNMENT;
+  QE_CUDA(launch_cooc_npmi(idx, T, k, channel_pos, d_in, C, O, S, threshold, static_cast<cudaStream_t>(stream)),
+          "cooc_npmi");
+  return QE_OK;
 }
 
 qe_status qe_selftest_wait_timeout(int32_t limit_us, void* stream) {

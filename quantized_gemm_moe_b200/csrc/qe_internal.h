@@ -152,6 +152,14 @@ int pick_wgemm_bn(int T, int N, int K, int* splits_out, int* kbps_out);
 cudaError_t launch_wgemm(int bits, int BN, const CUtensorMap& tm_act, const CUtensorMap& tm_bcat,
                          const CUtensorMap& tm_ucat, const QgemmArgs& a, cudaStream_t st);
 
+// Positions of the token-dependent channels (histogram rank k .. k+C-1), -1 elsewhere.
+cudaError_t launch_split_channels(const int32_t* hist, int d, int k, int C, int32_t* pos, cudaStream_t st);
+
+// Co-occurrence counts O [C][C] of the token-dependent channels in each token's Top-k set, and
+// their NPMI S (optional). O is zeroed here.
+cudaError_t launch_cooc_npmi(const int32_t* idx, int T, int k, const int32_t* pos, int d_in, int C, int32_t* O,
+                             float* S, float threshold, cudaStream_t st);
+
 // One CTA whose single wait runs out after limit_ns (the bounded-wait self-test).
 cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
 
@@ -159,8 +167,9 @@ cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
 int* device_error_ptr();  // nullptr when the symbol lookup fails
 cudaError_t read_device_error(int* value, bool clear, cudaStream_t st);
 
-// Top-k importance.
+// Top-k importance. bf16 rows with 7936 <= K <= 31744 take the streaming kernel (one CTA per
+// SM, rows staged by bulk copies); others, and rows it leaves unresolved, the radix-select kernel.
 cudaError_t launch_topk(const void* X, bool x_bf16, const float* w_mean, int T, int K, int k, int32_t* idx,
-                        int32_t* hist, cudaStream_t st);
+                        int32_t* hist, int* err, cudaStream_t st);
 
 }  // namespace qe

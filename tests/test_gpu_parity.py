@@ -175,6 +175,29 @@ def test_topk_bit_exact(T, K, k, xdt):
     assert (hist.cpu().numpy() == 2 * hist_ref).all()
 
 
+def test_topk_streaming_rows_with_degenerate_rows_mixed_in():
+    # More tokens than SMs (the streaming kernel strides), with all-zero and constant rows that
+    # it leaves to the radix-select kernel, spread over several CTAs and both row buffers.
+    T, K, k = 400, 8192, 32
+    cfg = _cfg(x_dtype="bf16", spec="qwen2b")
+    X = qi.outlier_activations(T, K, 91, cfg.outlier_spec(K))
+    for r in (0, 150, 151, 299, 399):
+        X[r] = 0.0
+    X[5] = 3.0
+    X[6, ::2] = 0.0
+    Xs = qi.to_bf16(X)
+    w_mean = np.abs(qi.gaussian(K, 0.02, 92)).astype(np.float32)
+    w_mean[100:140] = w_mean[99]
+    idx_ref, hist_ref = oracle.topk(Xs, w_mean, k)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    hist = torch.empty(K, dtype=torch.int32, device="cuda")
+    qe.topk_importance(cuda(Xs), cuda(w_mean), k, idx, hist)
+    torch.cuda.synchronize()
+    assert (idx.cpu().numpy() == idx_ref).all()
+    assert (hist.cpu().numpy() == hist_ref).all()
+    assert qe.device_error() == 0
+
+
 def test_topk_full_size_sampled_rows():
     # 72B-shaped statistic: all 8192 tokens at d = 29568 on the GPU; the oracle checks a
     # seeded sample of rows, and sum(hist) = T*k, hist == bincount(idx) hold for the whole run.
