@@ -215,33 +215,40 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const void* __restrict__ 
 }
 
 // ------------------------------------------------------------------ Top-k importance, streaming form
-// bf16 rows with 7936 <= K <= 31744. Persistent CTAs (one per SM, 1024 threads) stride over the
-// tokens; each token's row is staged in shared memory by an untiled bulk copy, two rows in
-// flight. Warps 0-30 score: their weight column means live in registers (4 chunks of 8 channels
-// per thread); warp 31 selects. Per token:
-//  1. scores s = fl32(|x| * w); each scoring thread keeps the maximum of each of its chunks.
-//     Every scoring warp takes the j-th largest of its 32 lane maxima (j = ceil(k/31)): a score
-//     that j distinct channels of the warp reach. tau = the minimum over the 31 warps is reached
-//     by at least 31 j >= k channels, so every channel of the Top-k set has s >= tau;
-//  2. the chunks whose maximum reaches tau are listed (with their 8 weights) by their owners,
-//     at offsets from per-warp counts; one thread per listed chunk then scores it again and
-//     appends its channels with s >= tau (the candidates) as 64-bit keys (score desc, channel
-//     asc);
-//  3. warp 31 selects from the candidates while the others score the next token. With the
-//     score keys in registers, a bit-serial search (two bits per step, warp sums) raises a
-//     threshold v while at least k candidates reach it, and stops once at most kTSSel do; the
-//     candidates with key >= v are ranked among themselves by counting, and ranks below k are
-//     the output slots.
-// A row with more than kTSCap candidates, or more than kTSSel at or above the final threshold
-// (rows of mostly equal scores), is marked -1 in its first slot and resolved by k_topk
-// (marked_only).
+// bf16 rows with 7680 <= K <= 30720. Persistent CTAs (one per SM, 1024 threads) stride over the
+// tokens, three row buffers in flight (untiled bulk copies). Warp roles, linked by mbarriers:
+//  - scoring warps 0-29 hold the weight column means in registers (4 chunks of 8 channels per
+//    thread). Per token: scores s = fl32(|x| * w); each thread keeps the maximum of each of its
+//    chunks, and every warp publishes the j-th largest of its 32 lane maxima (j = ceil(k/30)),
+//    a score that j distinct channels of the warp reach. After a barrier among the scoring
+//    warps, tau = the minimum of the 30 published values is reached by at least 30 j >= k
+//    channels, so every channel of the Top-k set has s >= tau. The owners of the chunks whose
+//    maximum reaches tau list them (channel base, 8 x values, 8 weights) for the token, at
+//    offsets from per-warp counts exchanged through a second barrier;
+//  - selecting warps 30-31 take the tokens in turn: once a token's list is complete the warp
+//    stages the token three steps ahead into the freed row buffer and raises the threshold to
+//    tau' = the m-th largest of the 30 published values (m = ceil(k/j): m warps with j channels
+//    each reach it). It scores the listed chunks whose maximum reaches tau' again and keeps the
+//    channels with s >= tau' as 64-bit keys (score desc, channel asc). With
+//    the score keys in registers, a bit-serial search (two bits per step, warp sums) raises a
+//    threshold v while at least k candidates reach it and stops once at most kTSSel do; the
+//    candidates with key >= v are ranked among themselves by counting, and ranks below k are
+//    the output slots.
+// The first kTSChunkCap listed chunks carry their x values and weights; later ones are read from
+// the row (whose refill then waits) and from memory. A row with more than kTSListCap listed
+// chunks, more than kTSChunkCap of them reaching tau', more than kTSCap candidates or more than
+// kTSSel at or above the final threshold (rows of mostly equal scores) is marked -1 in its first
+// slot and resolved by k_topk (marked_only).
 constexpr int kTSThreads = 1024;
-constexpr int kTSWarps = kTSThreads / 32;
-constexpr int kTSScorers = kTSThreads - 32;  // warps 0-30
-constexpr int kTSChunks = 4;  // channels (tid + 992 j) * 8 .. +7, j < 4: K <= 31744
-constexpr int kTSCap = 1024;
-constexpr int kTSChunkCap = 512;
-constexpr int kTSRegKeys = 12;  // score keys per lane held in registers by the selecting warp
+constexpr int kTSSelectors = 2;  // = list buffers
+constexpr int kTSRowStages = 3;
+constexpr int kTSScorerWarps = kTSThreads / 32 - kTSSelectors;
+constexpr int kTSScorers = kTSScorerWarps * 32;
+constexpr int kTSChunks = 4;  // channels (tid + 960 j) * 8 .. +7, j < 4
+constexpr int kTSRegKeys = 12;  // score keys per lane held in registers by a selecting warp
+constexpr int kTSCap = 32 * kTSRegKeys;
+constexpr int kTSChunkCap = 320;   // listed chunks whose x and weights are staged
+constexpr int kTSListCap = 1024;   // listed chunks (index and maximum)
 constexpr int kTSSel = 64;
 constexpr int kTSMinK = kTSScorers * 8;
 constexpr int kTSMaxK = kTSScorers * 8 * kTSChunks;
@@ -363,182 +370,287 @@ __device__ __forceinline__ void topk_select(int t, const unsigned long long* ck,
   __syncwarp();
 }
 
+// A bounded wait that also gives up once another thread of the CTA has given up.
+__device__ __forceinline__ bool ts_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    // back off: a waiting warp leaves its issue slots to the warps it waits for
+    __nanosleep(spins < 4 ? 32 : 128);
+    if ((++spins & 15u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_error(err, DEVERR_WAIT_PRODUCER);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
+// Barrier 1 over the scoring warps; returns whether any of them passed pred = true.
+__device__ __forceinline__ bool scorers_sync_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "n"(kTSScorers)
+      : "memory");
+  return r != 0;
+}
+
+struct TSList {
+  uint4 x[kTSChunkCap];      // the chunk's 8 bf16 x values (first kTSChunkCap listed chunks)
+  float4 w[kTSChunkCap][2];  // its 8 weights
+  float cm[kTSListCap];      // its maximum score
+  int16_t ci[kTSListCap];    // chunk index (channel base / 8)
+};
+
 __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* __restrict__ X,
                                                                const float* __restrict__ w, int T, int K, int k,
                                                                int32_t* __restrict__ idx_out,
                                                                int32_t* __restrict__ hist, int* err) {
-  extern __shared__ __align__(128) uint16_t rows[];  // [2][K]
-  __shared__ unsigned long long ckey[2][kTSCap];
-  __shared__ unsigned long long skey[kTSSel + 8];
-  __shared__ __align__(16) float cw[kTSChunkCap][8];
-  __shared__ int clist[kTSChunkCap];
-  __shared__ int wcnt[kTSWarps];
-  __shared__ float wthr[kTSWarps];
-  __shared__ int s_nc[2];
-  __shared__ __align__(8) uint64_t full[2];
+  extern __shared__ __align__(128) uint8_t tsm[];
+  uint16_t* rows = reinterpret_cast<uint16_t*>(tsm);  // [3][K]
+  TSList* lists = reinterpret_cast<TSList*>(tsm + kTSRowStages * K * 2);  // [2]
+  __shared__ unsigned long long ckey[kTSSelectors][kTSCap];
+  __shared__ unsigned long long skey[kTSSelectors][kTSSel + 8];
+  __shared__ int16_t sq[kTSSelectors][kTSChunkCap];  // listed chunks that reach tau'
+  __shared__ float wthr[kTSSelectors][32];
+  __shared__ int wcnt[kTSSelectors][32];
+  __shared__ int lcount[kTSSelectors];
+  __shared__ __align__(8) uint64_t row_full[kTSRowStages], list_full[kTSSelectors], list_empty[kTSSelectors];
+  __shared__ int issued[kTSRowStages], consumed[kTSRowStages];
+  __shared__ int s_abort;
+  volatile int* abort_flag = &s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool scorer = warp < kTSWarps - 1;
   const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
-  float wr[kTSChunks][8];
-#pragma unroll
-  for (int j = 0; j < kTSChunks; ++j) {
-    const int c0 = (tid + kTSScorers * j) * 8;
-    if (scorer && c0 < K) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(w + c0));
-      const float4 b = __ldg(reinterpret_cast<const float4*>(w + c0) + 1);
-      wr[j][0] = a.x; wr[j][1] = a.y; wr[j][2] = a.z; wr[j][3] = a.w;
-      wr[j][4] = b.x; wr[j][5] = b.y; wr[j][6] = b.z; wr[j][7] = b.w;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) wr[j][i] = 0.0f;
-    }
-  }
+  const int G = static_cast<int>(gridDim.x);
+  const int KC = K / 8;
   if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
+    for (int r = 0; r < kTSRowStages; ++r) {
+      mbar_init(&row_full[r], 1);
+      issued[r] = 0;
+      consumed[r] = 0;
+    }
+    for (int l = 0; l < kTSSelectors; ++l) {
+      mbar_init(&list_full[l], kTSScorerWarps);
+      mbar_init(&list_empty[l], 1);
+      lcount[l] = 0;
+    }
+    s_abort = 0;
     mbar_fence_init();
   }
   __syncthreads();
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
-      const int t = blockIdx.x + b * static_cast<int>(gridDim.x);
+    for (int r = 0; r < kTSRowStages; ++r) {
+      const int t = blockIdx.x + r * G;
       if (t < T) {
-        mbar_arrive_expect_tx(&full[b], row_bytes);
-        bulk_load(rows + b * K, X + static_cast<size_t>(t) * K, row_bytes, &full[b]);
+        issued[r] = 1;
+        mbar_arrive_expect_tx(&row_full[r], row_bytes);
+        bulk_load(rows + r * K, X + static_cast<size_t>(t) * K, row_bytes, &row_full[r]);
       }
     }
   }
-  if (!scorer) {
-    // The selecting warp: it takes part in the same four barriers per token as the scoring
-    // warps and finishes each token while the next row is scored.
-    if (lane == 0) wcnt[warp] = 0;
-    int it = 0, prev_t = -1;
-    for (int t = blockIdx.x; t < T; t += gridDim.x, ++it) {
-      if (prev_t >= 0) topk_select(prev_t, ckey[(it - 1) & 1], s_nc[(it - 1) & 1], k, idx_out, hist, skey, lane);
-      if (__syncthreads_or(0)) return;  // a row copy never landed (the scoring warps stop too)
-      __syncthreads();
-      __syncthreads();
-      __syncthreads();
-      prev_t = t;
-    }
-    if (prev_t >= 0) topk_select(prev_t, ckey[(it - 1) & 1], s_nc[(it - 1) & 1], k, idx_out, hist, skey, lane);
-    return;
-  }
-  const int jj = (k + kTSWarps - 2) / (kTSWarps - 1);
-  int it = 0;
-  for (int t = blockIdx.x; t < T; t += gridDim.x, ++it) {
-    const int b = it & 1;
-    const uint16_t* row = rows + b * K;
-    const bool ok = mbar_wait(&full[b], static_cast<uint32_t>((it >> 1) & 1), err, DEVERR_WAIT_PRODUCER);
-    // 1. chunk maxima; the warp's j-th largest lane maximum
-    float cmax[kTSChunks];
-    float m = -INFINITY;
+  if (warp < kTSScorerWarps) {
+    // ---------------- scoring warps
+    float wr[kTSChunks][8];
 #pragma unroll
     for (int j = 0; j < kTSChunks; ++j) {
       const int c0 = (tid + kTSScorers * j) * 8;
-      cmax[j] = -INFINITY;
       if (c0 < K) {
-        float sc[8];
-        chunk_scores(*reinterpret_cast<const uint4*>(row + c0), wr[j], sc);
-        cmax[j] = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])),
-                        fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
-        m = fmaxf(m, cmax[j]);
+        const float4 a = __ldg(reinterpret_cast<const float4*>(w + c0));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(w + c0) + 1);
+        wr[j][0] = a.x; wr[j][1] = a.y; wr[j][2] = a.z; wr[j][3] = a.w;
+        wr[j][4] = b.x; wr[j][5] = b.y; wr[j][6] = b.z; wr[j][7] = b.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wr[j][i] = 0.0f;
       }
     }
-    float tw = warp_max(m);
-    for (int r = 1; r < jj; ++r) {
-      // drop one lane holding the current maximum, take the maximum of the rest
-      const uint32_t holder = __ballot_sync(0xffffffffu, m == tw);
-      if (lane == __ffs(holder) - 1) m = -INFINITY;
-      tw = warp_max(m);
-    }
-    if (lane == 0) wthr[warp] = tw;
-    if (tid == 0) s_nc[b] = 0;
-    if (__syncthreads_or(!ok)) {
-      // a row copy never landed: let the other buffer's copy (if one was issued) finish, then stop
-      if (tid == 0 && t + static_cast<int>(gridDim.x) < T)
-        mbar_wait_for(&full[b ^ 1], static_cast<uint32_t>(((it + 1) >> 1) & 1), nullptr, 0, 10000000ull);
-      return;
-    }
-    const float tau = warp_min(lane < kTSWarps - 1 ? wthr[lane] : INFINITY);
-    // 2a. list the chunks that reach tau, with their weights: per-warp counts, then every warp
-    //     finds its offset from the counts of the warps before it
-    uint32_t bal[kTSChunks];
-    int wc = 0;
+    const int jj = (k + kTSScorerWarps - 1) / kTSScorerWarps;
+    int it = 0;
+    for (int t = blockIdx.x; t < T; t += G, ++it) {
+      const int r = it % kTSRowStages, l = it & 1;
+      bool ok = ts_wait(&row_full[r], static_cast<uint32_t>((it / kTSRowStages) & 1), abort_flag, err);
+      if (ok && tid == 0) consumed[r] += 1;
+      if (ok && it >= kTSSelectors) ok = ts_wait(&list_empty[l], static_cast<uint32_t>(((it >> 1) - 1) & 1), abort_flag, err);
+      const uint16_t* row = rows + r * K;
+      float cmax[kTSChunks];
+      float m = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kTSChunks; ++j) {
-      bal[j] = __ballot_sync(0xffffffffu, cmax[j] >= tau);
-      wc += __popc(bal[j]);
-    }
-    if (lane == 0) wcnt[warp] = wc;
-    __syncthreads();
-    int incl = wcnt[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int nch = __shfl_sync(0xffffffffu, incl, 31);
-    int slot = __shfl_sync(0xffffffffu, incl, warp) - wc;
-#pragma unroll
-    for (int j = 0; j < kTSChunks; ++j) {
-      if ((bal[j] >> lane) & 1u) {
-        const int at = slot + __popc(bal[j] & ((1u << lane) - 1u));
-        if (at < kTSChunkCap) {
-          clist[at] = (tid + kTSScorers * j) * 8;
-          *reinterpret_cast<float4*>(&cw[at][0]) = make_float4(wr[j][0], wr[j][1], wr[j][2], wr[j][3]);
-          *reinterpret_cast<float4*>(&cw[at][4]) = make_float4(wr[j][4], wr[j][5], wr[j][6], wr[j][7]);
+      for (int j = 0; j < kTSChunks; ++j) {
+        const int ci = tid + kTSScorers * j;
+        cmax[j] = -INFINITY;
+        if (ci < KC) {
+          float sc[8];
+          chunk_scores(*reinterpret_cast<const uint4*>(row + ci * 8), wr[j], sc);
+          cmax[j] = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])),
+                          fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
+          m = fmaxf(m, cmax[j]);
         }
       }
-      slot += __popc(bal[j]);
-    }
-    __syncthreads();
-    // 2b. one thread per listed chunk: its channels with s >= tau become candidates
-    if (nch > kTSChunkCap) {
-      if (tid == 0) s_nc[b] = kTSCap + 1;  // too many: the row goes to the radix-select kernel
-    } else if (warp * 32 < nch) {
-      uint32_t m8 = 0u;
-      float sc[8];
-      int c0 = 0;
-      if (tid < nch) {
-        c0 = clist[tid];
-        float w8[8];
-        const float4 wa = *reinterpret_cast<const float4*>(&cw[tid][0]);
-        const float4 wb = *reinterpret_cast<const float4*>(&cw[tid][4]);
-        w8[0] = wa.x; w8[1] = wa.y; w8[2] = wa.z; w8[3] = wa.w;
-        w8[4] = wb.x; w8[5] = wb.y; w8[6] = wb.z; w8[7] = wb.w;
-        chunk_scores(*reinterpret_cast<const uint4*>(row + c0), w8, sc);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8 |= (sc[i] >= tau ? 1u : 0u) << i;
+      float tw = warp_max(m);
+      for (int q = 1; q < jj; ++q) {
+        // drop one lane holding the current maximum, take the maximum of the rest
+        const uint32_t holder = __ballot_sync(0xffffffffu, m == tw);
+        if (lane == __ffs(holder) - 1) m = -INFINITY;
+        tw = warp_max(m);
       }
-      const int cnt = __popc(m8);
-      int ic = cnt;
+      if (lane == 0) wthr[l][warp] = tw;
+      if (scorers_sync_or(!ok)) break;  // every warp's value is published (or a wait gave up)
+      const float tau = warp_min(lane < kTSScorerWarps ? wthr[l][lane] : INFINITY);
+      // list the chunks that reach tau, at offsets from the per-warp counts
+      uint32_t bal[kTSChunks];
+      int wc = 0;
+#pragma unroll
+      for (int j = 0; j < kTSChunks; ++j) {
+        bal[j] = __ballot_sync(0xffffffffu, cmax[j] >= tau);
+        wc += __popc(bal[j]);
+      }
+      if (lane == 0) wcnt[l][warp] = wc;
+      scorers_sync_or(false);
+      int incl = lane < kTSScorerWarps ? wcnt[l][lane] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, ic, o);
-        if (lane >= o) ic += y;
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      int base = 0;
-      if (lane == 31 && ic > 0) base = atomicAdd(&s_nc[b], ic);
-      base = __shfl_sync(0xffffffffu, base, 31);
-      int p = base + ic - cnt;
+      int base = __shfl_sync(0xffffffffu, incl, warp) - wc;
+      if (warp == 0 && lane == 31) lcount[l] = incl;
+      TSList& L = lists[l];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if ((m8 >> i) & 1u) {
-          if (p < kTSCap) ckey[b][p] = topk_comp(sc[i], c0 + i);
-          ++p;
+      for (int j = 0; j < kTSChunks; ++j) {
+        if ((bal[j] >> lane) & 1u) {
+          const int at = base + __popc(bal[j] & ((1u << lane) - 1u));
+          if (at < kTSListCap) {
+            const int ci = tid + kTSScorers * j;
+            L.ci[at] = static_cast<int16_t>(ci);
+            L.cm[at] = cmax[j];
+            if (at < kTSChunkCap) {
+              L.x[at] = *reinterpret_cast<const uint4*>(row + ci * 8);
+              L.w[at][0] = make_float4(wr[j][0], wr[j][1], wr[j][2], wr[j][3]);
+              L.w[at][1] = make_float4(wr[j][4], wr[j][5], wr[j][6], wr[j][7]);
+            }
+          }
+        }
+        base += __popc(bal[j]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&list_full[l]);
+    }
+  } else {
+    // ---------------- selecting warps: warp 30 + l takes the tokens with it % 2 == l
+    const int l = warp - kTSScorerWarps;
+    for (int it = l, t = blockIdx.x + l * G; t < T; it += kTSSelectors, t += kTSSelectors * G) {
+      if (!ts_wait(&list_full[l], static_cast<uint32_t>((it >> 1) & 1), abort_flag, err)) break;
+      const int r = it % kTSRowStages;
+      const int nch = lcount[l];
+      // Every scoring warp is done with this row: stage the token three steps ahead into it,
+      // unless listed chunks beyond the staged ones still have to be read from it.
+      auto refill = [&]() {
+        const int t3 = t + kTSRowStages * G;
+        if (lane == 0 && t3 < T) {
+          atomicAdd(&issued[r], 1);  // both selecting warps fill this buffer over time
+          mbar_arrive_expect_tx(&row_full[r], row_bytes);
+          bulk_load(rows + r * K, X + static_cast<size_t>(t3) * K, row_bytes, &row_full[r]);
+        }
+      };
+      if (nch <= kTSChunkCap) refill();
+      // the tighter threshold: the m-th largest of the 30 published values (m = ceil(k/j)), which
+      // m warps x j channels each reach; m <= 30 since j = ceil(k/30)
+      float v = lane < kTSScorerWarps ? wthr[l][lane] : -INFINITY;
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const float o = __shfl_xor_sync(0xffffffffu, v, stride);
+          const bool desc = (lane & size) == 0 || size == 32;
+          v = (((lane & stride) == 0) == desc) ? fmaxf(v, o) : fminf(v, o);
         }
       }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      // every thread is done with this row: stage the token two steps ahead into the buffer
-      const int t2 = t + 2 * static_cast<int>(gridDim.x);
-      if (t2 < T) {
-        mbar_arrive_expect_tx(&full[b], row_bytes);
-        bulk_load(rows + b * K, X + static_cast<size_t>(t2) * K, row_bytes, &full[b]);
+      const int jj = (k + kTSScorerWarps - 1) / kTSScorerWarps;
+      const float tau = __shfl_sync(0xffffffffu, v, (k + jj - 1) / jj - 1);
+      const TSList& L = lists[l];
+      int nc = 0;
+      if (nch > kTSListCap) {
+        nc = kTSCap + 1;
+      } else {
+        // keep the listed chunks whose maximum reaches tau
+        int nq = 0;
+        for (int q0 = 0; q0 < nch; q0 += 32) {
+          const int q = q0 + lane;
+          const bool keep = q < nch && L.cm[q] >= tau;
+          const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+          const int at = nq + __popc(bal & ((1u << lane) - 1u));
+          if (keep && at < kTSChunkCap) sq[l][at] = static_cast<int16_t>(q);
+          nq += __popc(bal);
+        }
+        if (nq > kTSChunkCap) {
+          nq = 0;
+          nc = kTSCap + 1;
+        }
+        __syncwarp();
+        for (int q0 = 0; q0 < nq; q0 += 32) {
+          const int qq = q0 + lane;
+          uint32_t m8 = 0u;
+          float sc[8];
+          int c0 = 0;
+          if (qq < nq) {
+            const int q = sq[l][qq];
+            c0 = static_cast<int>(L.ci[q]) * 8;
+            float4 wa, wb;
+            uint4 xv;
+            if (q < kTSChunkCap) {
+              wa = L.w[q][0];
+              wb = L.w[q][1];
+              xv = L.x[q];
+            } else {
+              // listed beyond the staged ones: x from the row (not yet refilled), w from memory
+              wa = __ldg(reinterpret_cast<const float4*>(w + c0));
+              wb = __ldg(reinterpret_cast<const float4*>(w + c0) + 1);
+              xv = *reinterpret_cast<const uint4*>(rows + r * K + c0);
+            }
+            const float w8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            chunk_scores(xv, w8, sc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m8 |= (sc[i] >= tau ? 1u : 0u) << i;
+          }
+          const int c = __popc(m8);
+          int ic = c;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, ic, o);
+            if (lane >= o) ic += y;
+          }
+          int p = nc + ic - c;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if ((m8 >> i) & 1u) {
+              if (p < kTSCap) ckey[l][p] = topk_comp(sc[i], c0 + i);
+              ++p;
+            }
+          }
+          nc += __shfl_sync(0xffffffffu, ic, 31);
+        }
       }
+      __syncwarp();
+      if (nch > kTSChunkCap) refill();
+      if (lane == 0) mbar_arrive(&list_empty[l]);  // the list buffer is free for token it + 2
+      topk_select(t, ckey[l], nc, k, idx_out, hist, skey[l], lane);
     }
+  }
+  __syncthreads();
+  if (tid == 0 && s_abort) {
+    // a wait gave up: let every copy still in flight land before the CTA exits
+    for (int r = 0; r < kTSRowStages; ++r)
+      if (issued[r] > consumed[r])
+        mbar_wait_for(&row_full[r], static_cast<uint32_t>(consumed[r] & 1), nullptr, 0, 10000000ull);
   }
 }
 
@@ -785,7 +897,7 @@ cudaError_t launch_topk(const void* X, bool x_bf16, const float* w_mean, int T, 
         n_sm = 148;
     }
     const int grid = std::min(T, n_sm);
-    const size_t smem_s = static_cast<size_t>(K) * 2 * 2;
+    const size_t smem_s = static_cast<size_t>(K) * 2 * kTSRowStages + sizeof(TSList) * kTSSelectors;
     e = cudaFuncSetAttribute(k_topk_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_s));
     if (e != cudaSuccess) return e;
     k_topk_stream<<<grid, kTSThreads, smem_s, st>>>(static_cast<const uint16_t*>(X), w_mean, T, K, k, idx, hist,

@@ -167,7 +167,7 @@ cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
 int* device_error_ptr();  // nullptr when the symbol lookup fails
 cudaError_t read_device_error(int* value, bool clear, cudaStream_t st);
 
-// Top-k importance. bf16 rows with 7936 <= K <= 31744 take the streaming kernel (one CTA per
+// Top-k importance. bf16 rows with 7680 <= K <= 30720 take the streaming kernel (one CTA per
 // SM, rows staged by bulk copies); others, and rows it leaves unresolved, the radix-select kernel.
 cudaError_t launch_topk(const void* X, bool x_bf16, const float* w_mean, int T, int K, int k, int32_t* idx,
                         int32_t* hist, int* err, cudaStream_t st);
