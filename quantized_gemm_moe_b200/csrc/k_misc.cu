@@ -664,7 +664,7 @@ __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* _
 // themselves by counting.
 constexpr int kSplitThreads = 1024;
 constexpr int kSplitMaxSel = 4096 + 128;
-constexpr int kSplitStageMax = 45056;  // counts staged in shared memory up to this many channels (176 KB)
+constexpr int kSplitStageMax = 36864;  // counts staged in shared memory up to this many channels (144 KB)
 
 __device__ __forceinline__ uint32_t split_key(int32_t v) { return static_cast<uint32_t>(v) ^ 0x80000000u; }
 
@@ -705,22 +705,47 @@ __device__ __forceinline__ uint32_t split_key_at(const int32_t* __restrict__ his
 
 __global__ void __launch_bounds__(kSplitThreads) k_split_channels(const int32_t* __restrict__ hist, int d, int k,
                                                                    int C, int32_t* __restrict__ pos, int staged) {
-  extern __shared__ uint32_t sk[];  // [d] when staged
+  extern __shared__ uint32_t split_dyn[];  // per-warp digit counts [32][256], then the keys [d] when staged
+  int (*wbins)[256] = reinterpret_cast<int (*)[256]>(split_dyn);
+  uint32_t* sk = split_dyn + (kSplitThreads / 32) * 256;
   __shared__ int bins[256];
   __shared__ int wt[33];
-  __shared__ uint32_t s_prefix;
+  __shared__ uint32_t s_prefix, s_kmin, s_kmax;
   __shared__ int s_rem;
   __shared__ int a_idx[kSplitMaxSel];
   __shared__ uint32_t a_key[kSplitMaxSel];
-  const int tid = threadIdx.x;
+  int* a_rank = &wbins[0][0];  // reused once the radix passes are done (8192 >= kSplitMaxSel)
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = min(k + C, d);
-  if (staged)
-    for (int c = tid; c < d; c += kSplitThreads) sk[c] = split_key(hist[c]);
-  // radix select of the n-th largest key
-  uint32_t prefix = 0, mask = 0;
+  if (tid == 0) {
+    s_kmin = 0xFFFFFFFFu;
+    s_kmax = 0u;
+  }
+  __syncthreads();
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll 8
+  for (int c = tid; c < d; c += kSplitThreads) {
+    const uint32_t u = split_key(__ldg(hist + c));
+    if (staged) sk[c] = u;
+    lo = min(lo, u);
+    hi = max(hi, u);
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) {
+    atomicMin(&s_kmin, lo);
+    atomicMax(&s_kmax, hi);
+  }
+  __syncthreads();
+  // radix select of the n-th largest key, from the highest byte in which the keys differ
+  const uint32_t kdiff = s_kmin ^ s_kmax;
+  int shift = kdiff == 0u ? 0 : ((31 - __clz(kdiff)) / 8) * 8;
+  uint32_t mask = shift == 24 ? 0u : ~((1u << (shift + 8)) - 1u);
+  uint32_t prefix = s_kmax & mask;
   int rem = n;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += kSplitThreads) bins[i] = 0;
+    for (int i = lane; i < 256; i += 32) wbins[warp][i] = 0;
     __syncthreads();
     for (int base = 0; base < d; base += kSplitThreads) {
       const int c = base + tid;
@@ -728,21 +753,56 @@ __global__ void __launch_bounds__(kSplitThreads) k_split_channels(const int32_t*
       const bool match = c < d && (u & mask) == prefix;
       const uint32_t active = __ballot_sync(0xffffffffu, match);
       if (match) {
-        // one add per distinct digit in the warp: counts mostly share their high bits
         const int dg = static_cast<int>((u >> shift) & 255u);
-        const uint32_t peers = __match_any_sync(active, dg);
-        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&bins[dg], __popc(peers));
+        const int lead = __ffs(active) - 1;
+        const int d0 = __shfl_sync(active, dg, lead);
+        // counts mostly share their high bits: one add when the whole warp has one digit
+        if (__all_sync(active, dg == d0)) {
+          if (lane == lead) atomicAdd(&bins[dg], __popc(active));
+        } else {
+          atomicAdd(&wbins[warp][dg], 1);
+        }
       }
     }
     __syncthreads();
-    if (tid == 0) {
-      int cum = 0, dg = 255;
-      for (; dg > 0; --dg) {
-        if (cum + bins[dg] >= rem) break;
-        cum += bins[dg];
+    if (tid < 256) {
+      int sum = bins[tid];
+#pragma unroll 8
+      for (int w2 = 0; w2 < kSplitThreads / 32; ++w2) sum += wbins[w2][tid];
+      bins[tid] = sum;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns digits 255-8l .. 248-8l (descending); find where the count from the top
+      // reaches rem
+      int cnt[8];
+      int lsum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = bins[255 - 8 * lane - j];
+        lsum += cnt[j];
       }
-      s_prefix = prefix | (static_cast<uint32_t>(dg) << shift);
-      s_rem = rem - cum;
+      int incl = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - lsum;
+      const uint32_t hm = __ballot_sync(0xffffffffu, excl < rem && incl >= rem);
+      if (lane == __ffs(hm) - 1) {
+        int run = excl, dg = 255 - 8 * lane - 7;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (run + cnt[j] >= rem) {
+            dg = 255 - 8 * lane - j;
+            break;
+          }
+          run += cnt[j];
+        }
+        s_prefix = prefix | (static_cast<uint32_t>(dg) << shift);
+        s_rem = rem - run;
+      }
     }
     __syncthreads();
     prefix = s_prefix;
@@ -750,39 +810,63 @@ __global__ void __launch_bounds__(kSplitThreads) k_split_channels(const int32_t*
     mask |= 255u << shift;
     __syncthreads();
   }
-  // prefix = key of v*; n - rem channels lie above it, the first rem ties (by index) are taken
+  // prefix = key of v*; n - rem channels lie above it, the first rem ties (by index) are taken.
+  // Each thread takes a contiguous range of channels, so one block scan orders them by index.
   const int nA = n - rem;
-  int runA = 0, runB = 0;
-  for (int base = 0; base < d; base += kSplitThreads) {
-    const int c = base + tid;
-    const uint32_t u = c < d ? split_key_at(hist, sk, staged, c) : 0u;
-    const bool fa = c < d && u > prefix, fb = c < d && u == prefix;
-    int tot;
-    const int ex = split_block_scan((fa ? 1 : 0) | (fb ? 0x10000 : 0), wt, &tot);
-    if (fa) {
-      const int slot = runA + (ex & 0xffff);
-      a_idx[slot] = c;
-      a_key[slot] = u;
-    }
+  const int per = (d + kSplitThreads - 1) / kSplitThreads;
+  const int c_lo = min(d, tid * per), c_hi = min(d, c_lo + per);
+  int na = 0, nb = 0;
+  for (int c = c_lo; c < c_hi; ++c) {
+    const uint32_t u = split_key_at(hist, sk, staged, c);
+    na += u > prefix ? 1 : 0;
+    nb += u == prefix ? 1 : 0;
+  }
+  int tot;
+  int ia = split_block_scan(na, wt, &tot);
+  int ib = split_block_scan(nb, wt, &tot);
+  for (int c = c_lo; c < c_hi; ++c) {
+    const uint32_t u = split_key_at(hist, sk, staged, c);
     int p = -1;
-    if (fb) {
-      const int e = runB + (ex >> 16);
-      if (e < rem && nA + e >= k) p = nA + e - k;
+    if (u > prefix) {
+      a_idx[ia] = c;
+      a_key[ia] = u;
+      ++ia;
+      continue;
     }
-    if (c < d && !fa) pos[c] = p;
-    runA += tot & 0xffff;
-    runB += tot >> 16;
+    if (u == prefix) {
+      if (ib < rem && nA + ib >= k) p = nA + ib - k;
+      ++ib;
+    }
+    pos[c] = p;
+  }
+  // ranks of the channels above v* by counting: candidate i = tid % nap against slice tid / nap
+  // of the list (partial counts added in shared memory)
+  for (int i = tid; i < nA; i += kSplitThreads) a_rank[i] = 0;
+  __syncthreads();
+  const int nap = (nA + 31) & ~31;
+  if (nap > 0) {
+    const int P = nap <= kSplitThreads ? kSplitThreads / nap : 1;
+    for (int i0 = 0; i0 < nA; i0 += kSplitThreads) {
+      const int i = i0 + (P > 1 ? tid % nap : tid), part = P > 1 ? tid / nap : 0;
+      if (i < nA && part < P) {
+        const uint32_t u = a_key[i];
+        const int c = a_idx[i];
+        const int j0 = part * nA / P, j1 = (part + 1) * nA / P;
+        int r = 0;
+#pragma unroll 4
+        for (int j = j0; j < j1; ++j) {
+          const uint32_t uj = a_key[j];
+          r += (uj > u || (uj == u && a_idx[j] < c)) ? 1 : 0;
+        }
+        atomicAdd(&a_rank[i], r);
+      }
+      if (P > 1) break;
+    }
   }
   __syncthreads();
   for (int i = tid; i < nA; i += kSplitThreads) {
-    const uint32_t u = a_key[i];
-    const int c = a_idx[i];
-    int r = 0;
-    for (int j = 0; j < nA; ++j) {
-      const uint32_t uj = a_key[j];
-      r += (uj > u || (uj == u && a_idx[j] < c)) ? 1 : 0;
-    }
-    pos[c] = r >= k ? r - k : -1;
+    const int r = a_rank[i];
+    pos[a_idx[i]] = r >= k ? r - k : -1;
   }
 }
 
@@ -932,12 +1016,10 @@ cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st) {
 namespace qe {
 cudaError_t launch_split_channels(const int32_t* hist, int d, int k, int C, int32_t* pos, cudaStream_t st) {
   const int staged = d <= kSplitStageMax ? 1 : 0;
-  const size_t smem = staged ? static_cast<size_t>(d) * 4 : 0;
-  if (staged) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(k_split_channels, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
+  const size_t smem = static_cast<size_t>(kSplitThreads / 32) * 256 * 4 + (staged ? static_cast<size_t>(d) * 4 : 0);
+  const cudaError_t e0 =
+      cudaFuncSetAttribute(k_split_channels, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e0 != cudaSuccess) return e0;
   k_split_channels<<<1, kSplitThreads, smem, st>>>(hist, d, k, C, pos, staged);
   return cudaGetLastError();
 }

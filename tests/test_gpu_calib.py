@@ -32,6 +32,7 @@ def _split(hist, k, C):
 @pytest.mark.parametrize("d,k,C,hi,seed", [
     (7, 2, 3, 10, 0), (500, 16, 128, 6, 1), (1536, 32, 256, 4, 2), (29568, 32, 256, 8192, 3),
     (100, 0, 50, 3, 4), (40, 16, 128, 5, 5), (5000, 128, 4096, 2, 6), (3000, 8, 64, 1, 7),
+    (1000, 8, 64, 0, 10), (40000, 32, 256, 3000, 11), (70000, 16, 1024, 1 << 20, 12),
 ])
 def test_split_channels_bit_exact(d, k, C, hi, seed):
     hist = np.random.default_rng(seed).integers(0, hi + 1, size=d)
