@@ -108,7 +108,10 @@ def read_traffic(kernel_file: str, name: str):
     for line in open(p):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
+            v = v.strip()
+            if v.startswith("`") and "`" in v[1:]:
+                v = v[1:v.index("`", 1)]  # the value is the first backticked word
+            vals[k.strip()] = v
     try:
         if vals.get("source_hash") != git_src_hash([kernel_file]):
             return None
