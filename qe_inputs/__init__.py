@@ -183,6 +183,17 @@ CONFIGS = {
          Projection("o", 8192, 8192), Projection("gate", 8192, 29568), Projection("up", 8192, 29568),
          Projection("down", 29568, 8192)),
         4, 6, 128, 32, 8, 4, 32, "bf16", "scaled", 4),
+    # weight-only prefill variants of the 2B layer set (W4A16 and W3A16 tables)
+    "qwen2vl2b_w4a16": LayerConfig(
+        "qwen2vl2b_w4a16", 2048,
+        (Projection("q", 1536, 1536), Projection("o", 1536, 1536), Projection("gate", 1536, 8960),
+         Projection("up", 1536, 8960), Projection("down", 8960, 1536)),
+        4, 16, 128, 32, 8, 4, 32, "bf16", "qwen2b", 7),
+    "qwen2vl2b_w3a16": LayerConfig(
+        "qwen2vl2b_w3a16", 2048,
+        (Projection("q", 1536, 1536), Projection("o", 1536, 1536), Projection("gate", 1536, 8960),
+         Projection("up", 1536, 8960), Projection("down", 8960, 1536)),
+        3, 16, 128, 32, 8, 4, 32, "bf16", "qwen2b", 8),
     "decode72b_w4a8": LayerConfig(
         "decode72b_w4a8", 16,
         (Projection("gate", 8192, 29568), Projection("up", 8192, 29568), Projection("down", 29568, 8192)),

@@ -39,10 +39,19 @@ struct WCfg {
   static constexpr int kSlot = kA + kB;
   // Operand slots: each holds a 32 KB bf16 weight tile, so they bound the blocks in flight
   // between unpacking and the MMA; narrow tiles leave room for one more.
-  static constexpr int kNA = (BN <= 32) ? 4 : 3;
+  static constexpr int kNA = (BN <= 32) ? 4 : (BN <= 64 ? 3 : 2);
   static constexpr int kNW = 6;                 // packed weight ring
   static constexpr int kWP = 8192;
-  static constexpr int kNB = 8;                 // TMEM accumulator buffers (fp32, BN columns each)
+  static constexpr int kNB = (BN <= 64) ? 8 : 4;  // TMEM accumulator buffers (fp32, BN columns each)
+  // Roles (512 threads): warp 0 weight blocks, warps 1-2 MMA issuers, warp 3 activation tiles,
+  // then the epilogue warps, then the unpack warps. 128-token tiles take a second team of 4
+  // epilogue warps from the unpack warps: each team keeps half of the tile's columns in
+  // registers, and 4 unpack warps convert a row each.
+  static constexpr int kThreads = 512;
+  static constexpr int kEpiWarps = (BN <= 64) ? 4 : 8;
+  static constexpr int kUnpackW0 = 4 + kEpiWarps;
+  static constexpr int kUnpackWarps = 16 - kUnpackW0;
+  static constexpr int kEC = BN * 4 / kEpiWarps;  // columns per epilogue thread
   static constexpr int kTmemCols = (kNB * BN <= 128) ? 128 : (kNB * BN <= 256 ? 256 : 512);
   static constexpr int kOut = (BN <= 32) ? 8192 : 16384;  // output staging
   static constexpr int kChunk = (BN >= 16) ? 16 : BN;
@@ -120,11 +129,11 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* out_stage = wring + NW * C::kWP;        // [16 KB]
   uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + C::kOut);
   uint64_t* wfull = bars;             // [NW] packed block landed
-  uint64_t* wempty = wfull + NW;      // [NW] unpack warps read it (8 arrivals)
-  uint64_t* afull = wempty + NW;      // [NA] A unpacked (8 arrivals) + B landed (1 arrival + bytes)
+  uint64_t* wempty = wfull + NW;      // [NW] unpack warps read it (one arrival per unpack warp)
+  uint64_t* afull = wempty + NW;      // [NA] A unpacked (one per unpack warp) + B landed (1 + bytes)
   uint64_t* aempty = afull + NA;      // [NA] MMAs done with the slot
   uint64_t* accf = aempty + NA;       // [NB] group sum ready
-  uint64_t* acce = accf + NB;         // [NB] group sum read (4 epilogue warps)
+  uint64_t* acce = accf + NB;         // [NB] group sum read (every epilogue warp)
   uint64_t* done = acce + NB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   float* su_s = reinterpret_cast<float*>(bars + 64);
@@ -139,15 +148,15 @@ __global__ void __launch_bounds__(512, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NW; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 8);
+      mbar_init(&wempty[s], C::kUnpackWarps);
     }
     for (int s = 0; s < NA; ++s) {
-      mbar_init(&afull[s], 9);
+      mbar_init(&afull[s], C::kUnpackWarps + 1);
       mbar_init(&aempty[s], 1);
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], 4);
+      mbar_init(&acce[b], C::kEpiWarps);
     }
     mbar_init(done, 2);
     mbar_fence_init();
@@ -301,11 +310,13 @@ __global__ void __launch_bounds__(512, 1)
       tc_commit(done);
       mbar_wait(done, 0, a_err, DEVERR_WAIT_TEARDOWN);
     }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ unpack (warps 8..15)
-    // Thread t takes row r = t/2 of the block and the 64-wide K atom t%2 of it.
-    const int ut = threadIdx.x - 256;  // 0..255
-    const int r = ut >> 1, atom = ut & 1;
+  } else if (warp >= C::kUnpackW0) {
+    // ------------------------------------------------------------ unpack
+    // 8 warps: thread t takes row r = t/2 of the block and the 64-wide K atom t%2 of it.
+    // 4 warps: thread t takes row t, both atoms.
+    constexpr int kAtomsPerThread = C::kUnpackWarps == 8 ? 1 : 2;
+    const int ut = threadIdx.x - 32 * C::kUnpackW0;
+    const int r = kAtomsPerThread == 1 ? ut >> 1 : ut;
     int it = 0, jw = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -320,13 +331,18 @@ __global__ void __launch_bounds__(512, 1)
             break;
           }
           const uint8_t* src = wring + ws * C::kWP;
+#pragma unroll
+          for (int ai = 0; ai < kAtomsPerThread; ++ai) {
+          const int atom = kAtomsPerThread == 1 ? (ut & 1) : ai;
           uint8_t* dst = slots + s * C::kSlot + atom * C::kAtomA + r * 128;
           if constexpr (BITS == 4) {
             // row r: 64 bytes, four 16-byte pieces; this atom is pieces 2*atom and 2*atom+1
             const uint4 p0 = *reinterpret_cast<const uint4*>(src + r * 64 + atom * 32);
             const uint4 p1 = *reinterpret_cast<const uint4*>(src + r * 64 + atom * 32 + 16);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&wempty[ws]);
+            if (ai == kAtomsPerThread - 1) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&wempty[ws]);
+            }
             const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
             for (int pc = 0; pc < 2; ++pc) {
@@ -347,8 +363,10 @@ __global__ void __launch_bounds__(512, 1)
             // row r: 48 bytes; low two bits in words m = 4*atom + 0..3, bit 2 in words h = 2*atom + 0..1
             const uint4 lq = *reinterpret_cast<const uint4*>(src + r * 48 + atom * 16);
             const uint2 hq = *reinterpret_cast<const uint2*>(src + r * 48 + 32 + atom * 8);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&wempty[ws]);
+            if (ai == kAtomsPerThread - 1) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&wempty[ws]);
+            }
             const uint32_t lw[4] = {lq.x, lq.y, lq.z, lq.w};
             const uint32_t hw[2] = {hq.x, hq.y};
 #pragma unroll
@@ -364,6 +382,7 @@ __global__ void __launch_bounds__(512, 1)
               *reinterpret_cast<uint4*>(dst + ((ch ^ (r & 7)) << 4)) = make_uint4(e[0], e[1], e[2], e[3]);
             }
           }
+          }
           fence_proxy_async_smem();
           ++jw;
         } else {
@@ -377,11 +396,14 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ epilogue (warps 4..7)
+    // ------------------------------------------------------------ epilogue (warps 4..4+kEpiWarps)
     // Control flow depends only on the unit schedule; after a wait runs out, `ok` turns every
     // later wait and TMEM access off (the named barrier below is still reached by all).
+    constexpr int EC = C::kEC, NE = 32 * C::kEpiWarps;
     const int q = warp & 3;
-    const int et = threadIdx.x - 128;  // 0..127
+    const int team = C::kEpiWarps == 8 ? (warp - 4) >> 2 : 0;
+    const int ch0 = team * EC;          // this team's first column
+    const int et = threadIdx.x - 128;   // 0..NE-1
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     int gidx = 0;
     bool ok = true;
@@ -390,16 +412,16 @@ __global__ void __launch_bounds__(512, 1)
       const int o0 = w.nt * kTileN;
       const int o = o0 + 32 * q + lane;
       const bool o_ok = o < a.N;
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      for (int c = et; c < BN; c += 128) {
+      asm volatile("bar.sync 2, %0;" ::"n"(NE) : "memory");
+      for (int c = et; c < BN; c += NE) {
         const int p = w.p0 + c;
         su_s[c] = (p < a.T && a.su_sorted) ? a.su_sorted[p] : 0.0f;
         perm_s[c] = (p < a.T) ? a.perm[p] : -1;
       }
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      float acc[BN];
+      asm volatile("bar.sync 2, %0;" ::"n"(NE) : "memory");
+      float acc[EC];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) acc[c] = 0.0f;
+      for (int c = 0; c < EC; ++c) acc[c] = 0.0f;
       const float* swp = a.w_scale + static_cast<size_t>(w.g_begin) * a.N + o;
       float sw_next = (o_ok && w.n_groups > 0) ? __ldg(swp) : 0.0f;
       for (int g = 0; g < w.n_groups; ++g) {
@@ -410,9 +432,9 @@ __global__ void __launch_bounds__(512, 1)
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (!ok) continue;
         tc_fence_after();
-        const uint32_t base = tmem + lane_base + b * BN;
+        const uint32_t base = tmem + lane_base + b * BN + ch0;
 #pragma unroll
-        for (int c = 0; c < BN; c += C::kChunk) {
+        for (int c = 0; c < EC; c += C::kChunk) {
           uint32_t v[C::kChunk];
           if constexpr (C::kChunk == 16) tmem_ld16(base + c, v);
           else tmem_ld8(base + c, v);
@@ -431,16 +453,17 @@ __global__ void __launch_bounds__(512, 1)
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (ok) {
           tc_fence_after();
-          const uint32_t base = tmem + lane_base + b * BN;
+          const uint32_t base = tmem + lane_base + b * BN + ch0;
 #pragma unroll
-          for (int c = 0; c < BN; c += C::kChunk) {
+          for (int c = 0; c < EC; c += C::kChunk) {
             uint32_t v[C::kChunk];
             if constexpr (C::kChunk == 16) tmem_ld16(base + c, v);
             else tmem_ld8(base + c, v);
             tmem_wait_ld();
             reg_fence(v);
 #pragma unroll
-            for (int i = 0; i < C::kChunk; ++i) acc[c + i] = fmaf(su_s[c + i], __uint_as_float(v[i]), acc[c + i]);
+            for (int i = 0; i < C::kChunk; ++i)
+              acc[c + i] = fmaf(su_s[ch0 + c + i], __uint_as_float(v[i]), acc[c + i]);
           }
           tc_fence_before();
           __syncwarp();
@@ -457,20 +480,21 @@ __global__ void __launch_bounds__(512, 1)
       const bool vec_ok = ((static_cast<size_t>(a.N) * elem) % 16) == 0;
       for (int pass = 0; pass < BN / PC; ++pass) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
+        for (int cc = 0; cc < EC; ++cc) {
+          const int c = ch0 + cc;
           if (c < pass * PC || c >= (pass + 1) * PC) continue;
           const int cl = c - pass * PC;
           if (bf) {
-            __nv_bfloat16 h = __float2bfloat16_rn(acc[c]);
+            __nv_bfloat16 h = __float2bfloat16_rn(acc[cc]);
             *reinterpret_cast<__nv_bfloat16*>(out_stage + cl * row_bytes + (32 * q + lane) * 2) = h;
           } else {
-            *reinterpret_cast<float*>(out_stage + cl * row_bytes + (32 * q + lane) * 4) = acc[c];
+            *reinterpret_cast<float*>(out_stage + cl * row_bytes + (32 * q + lane) * 4) = acc[cc];
           }
         }
-        asm volatile("bar.sync 2, 128;" ::: "memory");
+        asm volatile("bar.sync 2, %0;" ::"n"(NE) : "memory");
         if (ok) {
           const int chunks_per_row = row_bytes / 16, elems = 16 / elem;
-          for (int ch = et; ch < PC * chunks_per_row; ch += 128) {
+          for (int ch = et; ch < PC * chunks_per_row; ch += NE) {
             const int cl = ch / chunks_per_row, part = ch % chunks_per_row;
             const int col = pass * PC + cl;
             const int p = w.p0 + col;
@@ -496,7 +520,7 @@ __global__ void __launch_bounds__(512, 1)
             }
           }
         }
-        asm volatile("bar.sync 2, 128;" ::: "memory");
+        asm volatile("bar.sync 2, %0;" ::"n"(NE) : "memory");
       }
     }
     tc_fence_before();
@@ -526,7 +550,7 @@ cudaError_t launch_wgemm_t(const CUtensorMap& tm_act, const CUtensorMap& tm_bcat
   const unsigned grid = static_cast<unsigned>(units < n_sm ? units : n_sm);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(512);
+  cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -541,7 +565,9 @@ cudaError_t launch_wgemm_t(const CUtensorMap& tm_act, const CUtensorMap& tm_bcat
 }  // namespace
 
 int pick_wgemm_bn(int T, int N, int K, int* splits_out, int* kbps_out) {
-  const int bn = (T <= 16) ? 16 : (T <= 32 ? 32 : 64);
+  // a weight block is unpacked once per token tile: wide tiles once there are enough tiles
+  const int64_t nt = ceil_div(N, kTileN);
+  const int bn = (T <= 16) ? 16 : (T <= 32 ? 32 : ((T <= 64 || nt * ceil_div(T, 128) < 148) ? 64 : 128));
   const int ntiles = static_cast<int>(ceil_div(N, kTileN));
   const int KB = static_cast<int>(ceil_div(K, kTileK));
   const int64_t tiles = int64_t(ntiles) * ceil_div(T, bn);
@@ -561,10 +587,12 @@ cudaError_t launch_wgemm(int bits, int BN, const CUtensorMap& tm_act, const CUte
     if (BN == 16) return launch_wgemm_t<4, 16>(tm_act, tm_bcat, tm_ucat, a, st);
     if (BN == 32) return launch_wgemm_t<4, 32>(tm_act, tm_bcat, tm_ucat, a, st);
     if (BN == 64) return launch_wgemm_t<4, 64>(tm_act, tm_bcat, tm_ucat, a, st);
+    if (BN == 128) return launch_wgemm_t<4, 128>(tm_act, tm_bcat, tm_ucat, a, st);
   } else if (bits == 3) {
     if (BN == 16) return launch_wgemm_t<3, 16>(tm_act, tm_bcat, tm_ucat, a, st);
     if (BN == 32) return launch_wgemm_t<3, 32>(tm_act, tm_bcat, tm_ucat, a, st);
     if (BN == 64) return launch_wgemm_t<3, 64>(tm_act, tm_bcat, tm_ucat, a, st);
+    if (BN == 128) return launch_wgemm_t<3, 128>(tm_act, tm_bcat, tm_ucat, a, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -294,6 +294,8 @@ def test_forward_shapes(T, K, N, group, a_bits, rs, nr, rr, xdt):
 @pytest.mark.parametrize("T,K,N,group,bits,rs,nr,rr", [
     (1, 256, 200, 64, 3, 8, 4, 4), (5, 384, 256, 128, 3, 32, 8, 4), (16, 256, 384, 128, 4, 32, 8, 4),
     (33, 512, 136, 64, 3, 0, 2, 8), (4, 1024, 640, 128, 3, 32, 8, 32),
+    # enough output tiles for 128-token tiles (two epilogue teams), with ragged token tails
+    (300, 256, 8960, 128, 3, 32, 8, 4), (129, 384, 17920, 64, 4, 32, 8, 4),
 ])
 def test_forward_weight_only(T, K, N, group, bits, rs, nr, rr):
     cfg = _cfg(group=group, w_bits=bits, a_bits=16, rank_shared=rs, n_routed=nr, rank_routed=rr, x_dtype="bf16")
@@ -354,6 +356,13 @@ def _full_size(cfg_name, proj_index, n_rows=48):
 @pytest.mark.parametrize("proj_index", range(5))
 def test_full_size_qwen2vl2b_layer_set(proj_index):
     _full_size("qwen2vl2b", proj_index)
+
+
+@pytest.mark.parametrize("cfg_name", ["qwen2vl2b_w4a16", "qwen2vl2b_w3a16"])
+@pytest.mark.parametrize("proj_index", range(5))
+def test_full_size_weight_only_prefill(cfg_name, proj_index):
+    # W4A16 / W3A16 prefill of the 2B layer set (T = 2048): 128-token tiles
+    _full_size(cfg_name, proj_index)
 
 
 @pytest.mark.parametrize("cfg_name", ["decode72b_w4a8", "decode72b_w3a16"])
