@@ -79,6 +79,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="token count per GPU instead of the workload's own (smaller cases for ncu captures)")
     return ap.parse_args()
 
 
@@ -208,7 +210,7 @@ def run_reference(args, workload):
         return 0
     cfg_name, t_over, desc = WORKLOADS[workload]
     cfg = qi.CONFIGS[cfg_name]
-    T = t_over or cfg.T
+    T = args.tokens or t_over or cfg.T
     cores = os.cpu_count() or 1
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
     sample = max(1, min(args.cpu_sample_tokens, T))
@@ -295,7 +297,7 @@ def run_ours(args, workload):
         pg = dist
     cfg_name, t_over, desc_txt = WORKLOADS[workload]
     cfg = qi.CONFIGS[cfg_name]
-    T = t_over or cfg.T
+    T = args.tokens or t_over or cfg.T
     layers = build_layers(cfg, T, rank, dev)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
@@ -385,7 +387,7 @@ def run_ours(args, workload):
     kernel_file = "quantized_gemm_moe_b200/csrc/k_wgemm.cu" if wonly else "quantized_gemm_moe_b200/csrc/k_gemm.cu"
     prod_bytes = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
                                           cfg.n_routed, cfg.rank_routed, 1 if not wonly else 2, 2) for L in layers)
-    traffic = read_traffic(kernel_file, ("wgemm_" if wonly else "qgemm_") + workload)
+    traffic = read_traffic(kernel_file, ("wgemm_" if wonly else "qgemm_") + workload) if not args.tokens else None
     if decode:
         ach = prod_bytes / (prod_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -504,6 +506,7 @@ def calib_oracle_run(X, w_mean, k, C):
 
 def run_calib(args, workload):
     T, d, k, n_routed, desc_txt = CALIB_WORKLOADS[workload]
+    T = args.tokens or T
     C = n_routed * k
     rank, local_rank, world = dist_env()
     if args.impl == "reference":
@@ -590,11 +593,15 @@ def run_calib(args, workload):
     parts = part_ms.mean(axis=0)
 
     peaks = load_peaks()
+    # the committed capture is per full-size launch; DRAM traffic grows with the tokens
+    scaled_traffic = read_traffic("quantized_gemm_moe_b200/csrc/k_misc.cu", "topk_" + workload)
+    if scaled_traffic is not None:
+        scaled_traffic *= T / CALIB_WORKLOADS[workload][0]
     # Top-k reads X (bf16) and w_mean once and writes idx and hist
     topk_bytes = T * d * 2 + d * 4 + T * k * 4 + d * 4
     ach = topk_bytes / (parts[0] / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
-            "traffic": read_traffic("quantized_gemm_moe_b200/csrc/k_misc.cu", "topk_" + workload), "kernel": "topk",
+            "traffic": scaled_traffic, "kernel": "topk",
             "peak_source": peaks["source"] + " hbm copy"}
 
     e2e = None
