@@ -221,24 +221,19 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const void* __restrict__ 
 //    thread). Per token: scores s = fl32(|x| * w); each thread keeps the maximum of each of its
 //    chunks, and every warp publishes the j-th largest of its 32 lane maxima (j = ceil(k/30)),
 //    a score that j distinct channels of the warp reach. After a barrier among the scoring
-//    warps, tau = the minimum of the 30 published values is reached by at least 30 j >= k
-//    channels, so every channel of the Top-k set has s >= tau. The owners of the chunks whose
-//    maximum reaches tau list them (channel base, 8 x values, 8 weights) for the token, at
-//    offsets from per-warp counts exchanged through a second barrier;
+//    warps, each takes tau = the m-th largest of the 30 published values (m = ceil(k/j)): m
+//    warps with j distinct channels each reach it, so at least k channels do, and every channel
+//    of the Top-k set has s >= tau. The owners of the chunks whose maximum reaches tau list them
+//    (channel base, 8 x values, 8 weights) in their warp's region of the token's list;
 //  - selecting warps 30-31 take the tokens in turn: once a token's list is complete the warp
-//    stages the token three steps ahead into the freed row buffer and raises the threshold to
-//    tau' = the m-th largest of the 30 published values (m = ceil(k/j): m warps with j channels
-//    each reach it). It scores the listed chunks whose maximum reaches tau' again and keeps the
-//    channels with s >= tau' as 64-bit keys (score desc, channel asc). With
-//    the score keys in registers, a bit-serial search (two bits per step, warp sums) raises a
-//    threshold v while at least k candidates reach it and stops once at most kTSSel do; the
-//    candidates with key >= v are ranked among themselves by counting, and ranks below k are
-//    the output slots.
-// The first kTSChunkCap listed chunks carry their x values and weights; later ones are read from
-// the row (whose refill then waits) and from memory. A row with more than kTSListCap listed
-// chunks, more than kTSChunkCap of them reaching tau', more than kTSCap candidates or more than
-// kTSSel at or above the final threshold (rows of mostly equal scores) is marked -1 in its first
-// slot and resolved by k_topk (marked_only).
+//    stages the token three steps ahead into the freed row buffer, scores the listed chunks again
+//    and keeps the channels with s >= tau as 64-bit keys (score desc, channel asc). At most
+//    kTSSel candidates are ranked among themselves by counting; more go through a bit-serial
+//    threshold search (two bits per step, warp sums) on the score keys held in registers until
+//    at most kTSSel remain. Ranks below k are the output slots.
+// A row with more than kTSWarpCap listed chunks in one warp's region, more than kTSCap candidates
+// or more than kTSSel at or above the final threshold (rows of mostly equal scores) is marked -1
+// in its first slot and resolved by k_topk (marked_only).
 constexpr int kTSThreads = 1024;
 constexpr int kTSSelectors = 2;  // = list buffers
 constexpr int kTSRowStages = 3;
@@ -247,8 +242,8 @@ constexpr int kTSScorers = kTSScorerWarps * 32;
 constexpr int kTSChunks = 4;  // channels (tid + 960 j) * 8 .. +7, j < 4
 constexpr int kTSRegKeys = 12;  // score keys per lane held in registers by a selecting warp
 constexpr int kTSCap = 32 * kTSRegKeys;
-constexpr int kTSChunkCap = 320;   // listed chunks whose x and weights are staged
-constexpr int kTSListCap = 1024;   // listed chunks (index and maximum)
+constexpr int kTSWarpCap = 12;  // listed chunks per scoring warp and token
+constexpr int kTSListSlots = kTSScorerWarps * kTSWarpCap;
 constexpr int kTSSel = 64;
 constexpr int kTSMinK = kTSScorers * 8;
 constexpr int kTSMaxK = kTSScorers * 8 * kTSChunks;
@@ -285,6 +280,24 @@ __device__ __forceinline__ void topk_select(int t, const unsigned long long* ck,
                                             unsigned long long* skey, int lane) {
   if (nc < k || nc > 32 * kTSRegKeys) {
     if (lane == 0) idx_out[static_cast<size_t>(t) * k] = -1;
+    return;
+  }
+  if (nc <= kTSSel) {
+    // few candidates: rank them all directly (ck is padded with zero keys to a multiple of 8)
+    for (int q = lane; q < nc; q += 32) {
+      const unsigned long long me = ck[q];
+      int r = 0;
+      for (int x = 0; x < nc; x += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r += ck[x + u] > me ? 1 : 0;
+      }
+      if (r < k) {
+        const int c = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(me & 0xFFFFFFFFull));
+        idx_out[static_cast<size_t>(t) * k + r] = c;
+        if (hist) atomicAdd(hist + c, 1);
+      }
+    }
+    __syncwarp();
     return;
   }
   uint32_t key[kTSRegKeys];
@@ -405,10 +418,10 @@ __device__ __forceinline__ bool scorers_sync_or(bool pred) {
 }
 
 struct TSList {
-  uint4 x[kTSChunkCap];      // the chunk's 8 bf16 x values (first kTSChunkCap listed chunks)
-  float4 w[kTSChunkCap][2];  // its 8 weights
-  float cm[kTSListCap];      // its maximum score
-  int16_t ci[kTSListCap];    // chunk index (channel base / 8)
+  uint4 x[kTSListSlots];      // the chunk's 8 bf16 x values
+  float4 w[kTSListSlots][2];  // its 8 weights
+  int16_t ci[kTSListSlots];   // chunk index (channel base / 8)
+  int count[32];              // listed chunks per scoring warp (kTSWarpCap + 1: overflow)
 };
 
 __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* __restrict__ X,
@@ -418,12 +431,10 @@ __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* _
   extern __shared__ __align__(128) uint8_t tsm[];
   uint16_t* rows = reinterpret_cast<uint16_t*>(tsm);  // [3][K]
   TSList* lists = reinterpret_cast<TSList*>(tsm + kTSRowStages * K * 2);  // [2]
-  __shared__ unsigned long long ckey[kTSSelectors][kTSCap];
+  __shared__ unsigned long long ckey[kTSSelectors][kTSCap + 8];
   __shared__ unsigned long long skey[kTSSelectors][kTSSel + 8];
-  __shared__ int16_t sq[kTSSelectors][kTSChunkCap];  // listed chunks that reach tau'
+  __shared__ int16_t sq[kTSSelectors][kTSListSlots];
   __shared__ float wthr[kTSSelectors][32];
-  __shared__ int wcnt[kTSSelectors][32];
-  __shared__ int lcount[kTSSelectors];
   __shared__ __align__(8) uint64_t row_full[kTSRowStages], list_full[kTSSelectors], list_empty[kTSSelectors];
   __shared__ int issued[kTSRowStages], consumed[kTSRowStages];
   __shared__ int s_abort;
@@ -432,6 +443,8 @@ __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* _
   const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
   const int G = static_cast<int>(gridDim.x);
   const int KC = K / 8;
+  const int jj = (k + kTSScorerWarps - 1) / kTSScorerWarps;  // order statistic per warp
+  const int mm = (k + jj - 1) / jj;                           // warps combined, <= 30
   if (tid == 0) {
     for (int r = 0; r < kTSRowStages; ++r) {
       mbar_init(&row_full[r], 1);
@@ -441,7 +454,6 @@ __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* _
     for (int l = 0; l < kTSSelectors; ++l) {
       mbar_init(&list_full[l], kTSScorerWarps);
       mbar_init(&list_empty[l], 1);
-      lcount[l] = 0;
     }
     s_abort = 0;
     mbar_fence_init();
@@ -473,7 +485,6 @@ __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* _
         for (int i = 0; i < 8; ++i) wr[j][i] = 0.0f;
       }
     }
-    const int jj = (k + kTSScorerWarps - 1) / kTSScorerWarps;
     int it = 0;
     for (int t = blockIdx.x; t < T; t += G, ++it) {
       const int r = it % kTSRowStages, l = it & 1;
@@ -504,66 +515,7 @@ __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* _
       }
       if (lane == 0) wthr[l][warp] = tw;
       if (scorers_sync_or(!ok)) break;  // every warp's value is published (or a wait gave up)
-      const float tau = warp_min(lane < kTSScorerWarps ? wthr[l][lane] : INFINITY);
-      // list the chunks that reach tau, at offsets from the per-warp counts
-      uint32_t bal[kTSChunks];
-      int wc = 0;
-#pragma unroll
-      for (int j = 0; j < kTSChunks; ++j) {
-        bal[j] = __ballot_sync(0xffffffffu, cmax[j] >= tau);
-        wc += __popc(bal[j]);
-      }
-      if (lane == 0) wcnt[l][warp] = wc;
-      scorers_sync_or(false);
-      int incl = lane < kTSScorerWarps ? wcnt[l][lane] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int base = __shfl_sync(0xffffffffu, incl, warp) - wc;
-      if (warp == 0 && lane == 31) lcount[l] = incl;
-      TSList& L = lists[l];
-#pragma unroll
-      for (int j = 0; j < kTSChunks; ++j) {
-        if ((bal[j] >> lane) & 1u) {
-          const int at = base + __popc(bal[j] & ((1u << lane) - 1u));
-          if (at < kTSListCap) {
-            const int ci = tid + kTSScorers * j;
-            L.ci[at] = static_cast<int16_t>(ci);
-            L.cm[at] = cmax[j];
-            if (at < kTSChunkCap) {
-              L.x[at] = *reinterpret_cast<const uint4*>(row + ci * 8);
-              L.w[at][0] = make_float4(wr[j][0], wr[j][1], wr[j][2], wr[j][3]);
-              L.w[at][1] = make_float4(wr[j][4], wr[j][5], wr[j][6], wr[j][7]);
-            }
-          }
-        }
-        base += __popc(bal[j]);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&list_full[l]);
-    }
-  } else {
-    // ---------------- selecting warps: warp 30 + l takes the tokens with it % 2 == l
-    const int l = warp - kTSScorerWarps;
-    for (int it = l, t = blockIdx.x + l * G; t < T; it += kTSSelectors, t += kTSSelectors * G) {
-      if (!ts_wait(&list_full[l], static_cast<uint32_t>((it >> 1) & 1), abort_flag, err)) break;
-      const int r = it % kTSRowStages;
-      const int nch = lcount[l];
-      // Every scoring warp is done with this row: stage the token three steps ahead into it,
-      // unless listed chunks beyond the staged ones still have to be read from it.
-      auto refill = [&]() {
-        const int t3 = t + kTSRowStages * G;
-        if (lane == 0 && t3 < T) {
-          atomicAdd(&issued[r], 1);  // both selecting warps fill this buffer over time
-          mbar_arrive_expect_tx(&row_full[r], row_bytes);
-          bulk_load(rows + r * K, X + static_cast<size_t>(t3) * K, row_bytes, &row_full[r]);
-        }
-      };
-      if (nch <= kTSChunkCap) refill();
-      // the tighter threshold: the m-th largest of the 30 published values (m = ceil(k/j)), which
-      // m warps x j channels each reach; m <= 30 since j = ceil(k/30)
+      // tau = the mm-th largest of the 30 published values (a sort across the lanes)
       float v = lane < kTSScorerWarps ? wthr[l][lane] : -INFINITY;
 #pragma unroll
       for (int size = 2; size <= 32; size <<= 1) {
@@ -574,73 +526,107 @@ __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* _
           v = (((lane & stride) == 0) == desc) ? fmaxf(v, o) : fminf(v, o);
         }
       }
-      const int jj = (k + kTSScorerWarps - 1) / kTSScorerWarps;
-      const float tau = __shfl_sync(0xffffffffu, v, (k + jj - 1) / jj - 1);
-      const TSList& L = lists[l];
-      int nc = 0;
-      if (nch > kTSListCap) {
-        nc = kTSCap + 1;
-      } else {
-        // keep the listed chunks whose maximum reaches tau
-        int nq = 0;
-        for (int q0 = 0; q0 < nch; q0 += 32) {
-          const int q = q0 + lane;
-          const bool keep = q < nch && L.cm[q] >= tau;
-          const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-          const int at = nq + __popc(bal & ((1u << lane) - 1u));
-          if (keep && at < kTSChunkCap) sq[l][at] = static_cast<int16_t>(q);
-          nq += __popc(bal);
+      const float tau = __shfl_sync(0xffffffffu, v, mm - 1);
+      // list the chunks that reach tau in this warp's region
+      TSList& L = lists[l];
+      int wc = 0;
+#pragma unroll
+      for (int j = 0; j < kTSChunks; ++j) {
+        const bool cand = cmax[j] >= tau;
+        const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+        if (cand) {
+          const int at = wc + __popc(bal & ((1u << lane) - 1u));
+          if (at < kTSWarpCap) {
+            const int slot = warp * kTSWarpCap + at;
+            const int ci = tid + kTSScorers * j;
+            L.ci[slot] = static_cast<int16_t>(ci);
+            L.x[slot] = *reinterpret_cast<const uint4*>(row + ci * 8);
+            L.w[slot][0] = make_float4(wr[j][0], wr[j][1], wr[j][2], wr[j][3]);
+            L.w[slot][1] = make_float4(wr[j][4], wr[j][5], wr[j][6], wr[j][7]);
+          }
         }
-        if (nq > kTSChunkCap) {
-          nq = 0;
-          nc = kTSCap + 1;
-        }
-        __syncwarp();
-        for (int q0 = 0; q0 < nq; q0 += 32) {
-          const int qq = q0 + lane;
-          uint32_t m8 = 0u;
-          float sc[8];
-          int c0 = 0;
-          if (qq < nq) {
-            const int q = sq[l][qq];
-            c0 = static_cast<int>(L.ci[q]) * 8;
-            float4 wa, wb;
-            uint4 xv;
-            if (q < kTSChunkCap) {
-              wa = L.w[q][0];
-              wb = L.w[q][1];
-              xv = L.x[q];
-            } else {
-              // listed beyond the staged ones: x from the row (not yet refilled), w from memory
-              wa = __ldg(reinterpret_cast<const float4*>(w + c0));
-              wb = __ldg(reinterpret_cast<const float4*>(w + c0) + 1);
-              xv = *reinterpret_cast<const uint4*>(rows + r * K + c0);
-            }
-            const float w8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-            chunk_scores(xv, w8, sc);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) m8 |= (sc[i] >= tau ? 1u : 0u) << i;
-          }
-          const int c = __popc(m8);
-          int ic = c;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, ic, o);
-            if (lane >= o) ic += y;
-          }
-          int p = nc + ic - c;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if ((m8 >> i) & 1u) {
-              if (p < kTSCap) ckey[l][p] = topk_comp(sc[i], c0 + i);
-              ++p;
-            }
-          }
-          nc += __shfl_sync(0xffffffffu, ic, 31);
+        wc += __popc(bal);
+      }
+      if (lane == 0) L.count[warp] = wc > kTSWarpCap ? kTSWarpCap + 1 : wc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&list_full[l]);
+    }
+  } else {
+    // ---------------- selecting warps: warp 30 + l takes the tokens with it % 2 == l
+    const int l = warp - kTSScorerWarps;
+    for (int it = l, t = blockIdx.x + l * G; t < T; it += kTSSelectors, t += kTSSelectors * G) {
+      if (!ts_wait(&list_full[l], static_cast<uint32_t>((it >> 1) & 1), abort_flag, err)) break;
+      if (lane == 0) {
+        // every scoring warp is done with this row: stage the token three steps ahead into it
+        const int r = it % kTSRowStages;
+        const int t3 = t + kTSRowStages * G;
+        if (t3 < T) {
+          atomicAdd(&issued[r], 1);  // both selecting warps fill this buffer over time
+          mbar_arrive_expect_tx(&row_full[r], row_bytes);
+          bulk_load(rows + r * K, X + static_cast<size_t>(t3) * K, row_bytes, &row_full[r]);
         }
       }
+      const TSList& L = lists[l];
+      // the same tau as the scoring warps
+      float v = lane < kTSScorerWarps ? wthr[l][lane] : -INFINITY;
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const float o = __shfl_xor_sync(0xffffffffu, v, stride);
+          const bool desc = (lane & size) == 0 || size == 32;
+          v = (((lane & stride) == 0) == desc) ? fmaxf(v, o) : fminf(v, o);
+        }
+      }
+      const float tau = __shfl_sync(0xffffffffu, v, mm - 1);
+      // gather the listed chunks: warp region counts -> one index list
+      const int cnt = lane < kTSScorerWarps ? L.count[lane] : 0;
+      const bool overflow = __any_sync(0xffffffffu, cnt > kTSWarpCap);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int nch = overflow ? 0 : __shfl_sync(0xffffffffu, incl, 31);
+      if (!overflow)
+        for (int e = 0; e < cnt; ++e) sq[l][incl - cnt + e] = static_cast<int16_t>(lane * kTSWarpCap + e);
       __syncwarp();
-      if (nch > kTSChunkCap) refill();
+      int nc = overflow ? kTSCap + 1 : 0;
+      for (int q0 = 0; q0 < nch; q0 += 32) {
+        const int qq = q0 + lane;
+        uint32_t m8 = 0u;
+        float sc[8];
+        int c0 = 0;
+        if (qq < nch) {
+          const int q = sq[l][qq];
+          c0 = static_cast<int>(L.ci[q]) * 8;
+          const float4 wa = L.w[q][0], wb = L.w[q][1];
+          const float w8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+          chunk_scores(L.x[q], w8, sc);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8 |= (sc[i] >= tau ? 1u : 0u) << i;
+        }
+        const int c = __popc(m8);
+        int ic = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, ic, o);
+          if (lane >= o) ic += y;
+        }
+        int p = nc + ic - c;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if ((m8 >> i) & 1u) {
+            if (p < kTSCap) ckey[l][p] = topk_comp(sc[i], c0 + i);
+            ++p;
+          }
+        }
+        nc += __shfl_sync(0xffffffffu, ic, 31);
+      }
+      // zero keys up to a multiple of 8 for the unrolled ranking
+      if (nc <= kTSCap && lane < ((nc + 7) & ~7) - nc) ckey[l][nc + lane] = 0ull;
+      __syncwarp();
       if (lane == 0) mbar_arrive(&list_empty[l]);  // the list buffer is free for token it + 2
       topk_select(t, ckey[l], nc, k, idx_out, hist, skey[l], lane);
     }
