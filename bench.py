@@ -47,6 +47,8 @@ WORKLOADS = {
                                      "T=2048, W4A6 g128, r_s=32, N_r=8, r_r=4"),
     "internvl2_8b": ("internvl2_8b", None, "InternVL2-8B-shaped layer set, T=4096, W4A8 g128"),
     "qwen2vl72b": ("qwen2vl72b", None, "Qwen2VL-72B-shaped layer set, T=8192, W4A6 g128"),
+    "qwen2vl2b_sparse": ("qwen2vl2b", None, "Qwen2VL-2B-shaped layer set, T=2048, W4A6 g128, r_s=32, N_r=8, "
+                                            "r_r=4, cluster-sparse routed experts on 32 channels each", 32),
     "qwen2vl2b_w4a16": ("qwen2vl2b_w4a16", None, "Qwen2VL-2B-shaped layer set, T=2048, W4A16 g128 (weight-only "
                                                  "prefill), r_s=32, N_r=8, r_r=4"),
     "qwen2vl2b_w3a16": ("qwen2vl2b_w3a16", None, "Qwen2VL-2B-shaped layer set, T=2048, W3A16 g128 (weight-only "
@@ -208,7 +210,7 @@ def run_reference(args, workload):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
-    cfg_name, t_over, desc = WORKLOADS[workload]
+    cfg_name, t_over, desc = WORKLOADS[workload][:3]
     cfg = qi.CONFIGS[cfg_name]
     T = args.tokens or t_over or cfg.T
     cores = os.cpu_count() or 1
@@ -249,7 +251,7 @@ def max_over_ranks(value: float, pg, device=None) -> float:
     return float(t.item())
 
 
-def build_layers(cfg, T, rank, dev):
+def build_layers(cfg, T, rank, dev, routed_channels=0):
     import torch
     import quantized_gemm_moe_b200 as qe
     layers = []
@@ -261,14 +263,20 @@ def build_layers(cfg, T, rank, dev):
             x = qi.outlier_activations(T, proj.d_in, replica_x_seed(rank, pi), spec)
             inp["X"] = qi.to_bf16(x) if cfg.x_dtype == "bf16" else x
         desc = qe.make_desc(proj.d_in, proj.d_out, cfg.group, cfg.w_bits, cfg.a_bits, cfg.rank_shared, cfg.n_routed,
-                            cfg.rank_routed)
+                            cfg.rank_routed, routed_channels)
 
         def c(a):
             t = torch.from_numpy(np.ascontiguousarray(a)) if isinstance(a, np.ndarray) else a
             return t.contiguous().to(dev)
 
+        channels = None
+        if routed_channels:
+            # cluster-sparse routed experts: seeded disjoint channel clusters with their own A_r
+            channels, inp["A_r"] = qi.sparse_routed(proj.d_in, cfg.n_routed, routed_channels, cfg.rank_routed,
+                                                    6000 + pi)
+            channels = c(channels)
         layer = qe.QELayer.from_float(desc, c(inp["W"]), c(inp["s"]), c(inp["A_s"]), c(inp["B_s"]), c(inp["A_r"]),
-                                      c(inp["B_r"]), c(inp["G"]), s_inv=c(inp["s_inv"]))
+                                      c(inp["B_r"]), c(inp["G"]), s_inv=c(inp["s_inv"]), channels=channels)
         X = c(inp["X"])
         Y = torch.empty((T, proj.d_out), dtype=torch.bfloat16, device=dev)
         ws = layer.workspace(T)
@@ -295,10 +303,11 @@ def run_ours(args, workload):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         pg = dist
-    cfg_name, t_over, desc_txt = WORKLOADS[workload]
+    cfg_name, t_over, desc_txt = WORKLOADS[workload][:3]
+    routed_channels = WORKLOADS[workload][3] if len(WORKLOADS[workload]) > 3 else 0
     cfg = qi.CONFIGS[cfg_name]
     T = args.tokens or t_over or cfg.T
-    layers = build_layers(cfg, T, rank, dev)
+    layers = build_layers(cfg, T, rank, dev, routed_channels)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     wonly = cfg.a_bits == 16

@@ -75,6 +75,12 @@ typedef struct {
   int32_t rank_shared;  /* r_s >= 0                                                */
   int32_t n_routed;     /* N_r in [1, 16]                                          */
   int32_t rank_routed;  /* r_r >= 0; r_s + N_r*r_r <= 512                          */
+  int32_t routed_channels; /* k_c: 0 = dense routed experts (A_r[e] spans d_in).     */
+                           /* k_c > 0 = cluster-sparse routed experts (Method,      */
+                           /* "Routed Experts": each expert serves a cluster of     */
+                           /* token-dependent channels): A_r[e] is nonzero only on  */
+                           /* k_c channels, given to qe_pack_adapters_sparse.       */
+                           /* Needs r_r > 0 and r_s <= 240; k_c <= d_in.           */
 } qe_layer_desc;
 
 /*
@@ -156,6 +162,23 @@ QE_API qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, q
  */
 QE_API qe_status qe_pack_adapters(const qe_layer_desc* desc, const void* A_s, const void* B_s, const void* A_r,
                            const void* B_r, const void* G, void* out, void* stream);
+
+/*
+ * The same packing for cluster-sparse routed experts (desc->routed_channels = k_c > 0; the
+ * cluster reading of Method, "Routed Experts": an expert's down-projection touches only the
+ * token-dependent channels of its cluster):
+ *   channels (device) int32 [N_r][k_c]: expert e's channels, distinct, in [0, d_in)
+ *   A_r      (device) bf16 [N_r][k_c][r_r]: its down-projection over those channels, so that
+ *            U_r[t] = sum_i x[t][channels[e][i]] * A_r[e][i][:] (equal to a dense A_r that is zero
+ *            outside the channels)
+ * A_s, B_s, B_r and G are as for qe_pack_adapters. The forward then leaves the routed columns
+ * out of its adapter/router GEMM and gathers them per token. A channel outside [0, d_in) is
+ * replaced by channel 0 with zero weights and reported through qe_device_error (code 0x202).
+ * qe_pack_adapters accepts only routed_channels = 0 (QE_ERR_INVALID_ARG otherwise).
+ */
+QE_API qe_status qe_pack_adapters_sparse(const qe_layer_desc* desc, const void* A_s, const void* B_s,
+                                  const int32_t* channels, const void* A_r, const void* B_r, const void* G,
+                                  void* out, void* stream);
 
 /* ---------------------------------------------------------------- the hot path */
 

@@ -28,7 +28,7 @@ import torch
 
 __all__ = [
     "LayerConfig", "Projection", "CONFIGS", "config_by_name",
-    "outlier_activations", "gaussian", "layer_inputs", "to_bf16", "topk_like_sets",
+    "outlier_activations", "gaussian", "layer_inputs", "to_bf16", "topk_like_sets", "sparse_routed",
 ]
 
 
@@ -125,6 +125,23 @@ def topk_like_sets(T: int, d: int, k: int, seed: int) -> np.ndarray:
                 rest.append(c)
         out[t] = g.permutation(np.concatenate([ch, np.asarray(rest, dtype=ch.dtype)]))
     return out
+
+
+def sparse_routed(d: int, n_routed: int, kc: int, r_r: int, seed: int):
+    """Cluster-sparse routed experts: disjoint seeded channel clusters and their down-projections.
+
+    Returns channels int32 [n_routed][kc] (expert e's cluster, distinct channels, disjoint across
+    experts while d allows) and A_r bf16 [n_routed][kc][r_r] ~ N(0, 0.02).
+    """
+    g = _rng(seed)
+    perm = g.permutation(d)
+    if n_routed * kc > d:
+        perm = np.concatenate([perm] + [g.permutation(d) for _ in range((n_routed * kc) // d)])
+    ch = np.empty((n_routed, kc), dtype=np.int32)
+    for e in range(n_routed):
+        ch[e] = np.sort(perm[e * kc:(e + 1) * kc])
+    A = (g.standard_normal((n_routed, kc, r_r), dtype=np.float32) * np.float32(0.02)).astype(np.float32)
+    return ch, to_bf16(A)
 
 
 def gaussian(shape, std: float, seed: int) -> np.ndarray:

@@ -24,7 +24,7 @@ EXPORTS = (
     "qe_pack_adapters", "qe_topk_importance", "qe_route", "qe_linear_forward", "qe_status_string",
     "qe_last_cuda_error", "qe_device_error", "qe_unpack_weights", "qe_act_quant", "qe_linear_forward_debug",
     "qe_linear_forward_stages", "qe_linear_kernel_launches", "qe_linear_forward_noalloc",
-    "qe_selftest_wait_timeout", "qe_split_channels", "qe_cooccurrence_npmi",
+    "qe_selftest_wait_timeout", "qe_split_channels", "qe_cooccurrence_npmi", "qe_pack_adapters_sparse",
 )
 # fixed scratch of qe_linear_forward_noalloc (bytes), as declared in include/qe.h
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -45,7 +45,7 @@ class QEError(RuntimeError):
 class LayerDesc(ctypes.Structure):
     _fields_ = [("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("w_bits", ctypes.c_int32), ("a_bits", ctypes.c_int32), ("rank_shared", ctypes.c_int32),
-                ("n_routed", ctypes.c_int32), ("rank_routed", ctypes.c_int32)]
+                ("n_routed", ctypes.c_int32), ("rank_routed", ctypes.c_int32), ("routed_channels", ctypes.c_int32)]
 
     def __repr__(self):
         return "LayerDesc(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -75,6 +75,7 @@ def load() -> ctypes.CDLL:
         "qe_linear_workspace_bytes": ([D, I], S),
         "qe_quantize_weights": ([D, P, I, P, P, P, P, P, P], I),
         "qe_pack_adapters": ([D, P, P, P, P, P, P, P], I),
+        "qe_pack_adapters_sparse": ([D, P, P, P, P, P, P, P, P], I),
         "qe_topk_importance": ([P, I, P, I, I, I, P, P, I, P], I),
         "qe_route": ([P, I, P, I, I, I, P, P, P, P, P], I),
         "qe_linear_forward": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P, S, P], I),
@@ -135,8 +136,10 @@ def _need_cuda(*ts):
             raise QEError(QE_ERR_INVALID_ARG, "layout", "tensors passed to the QE library must be contiguous")
 
 
-def make_desc(d_in, d_out, group=128, w_bits=4, a_bits=8, rank_shared=32, n_routed=8, rank_routed=4) -> LayerDesc:
-    return LayerDesc(d_in, d_out, group, w_bits, a_bits, rank_shared, n_routed, rank_routed)
+def make_desc(d_in, d_out, group=128, w_bits=4, a_bits=8, rank_shared=32, n_routed=8, rank_routed=4,
+              routed_channels=0) -> LayerDesc:
+    """routed_channels > 0: cluster-sparse routed experts over that many channels each."""
+    return LayerDesc(d_in, d_out, group, w_bits, a_bits, rank_shared, n_routed, rank_routed, routed_channels)
 
 
 # ---------------------------------------------------------------- the C ABI, one wrapper per entry point
@@ -164,6 +167,13 @@ def pack_adapters(desc, A_s, B_s, A_r, B_r, G, out, stream=None):
     _need_cuda(A_s, B_s, A_r, B_r, G, out)
     _check(load().qe_pack_adapters(ctypes.byref(desc), _ptr(A_s), _ptr(B_s), _ptr(A_r), _ptr(B_r), _ptr(G),
                                    _ptr(out), _stream(stream)), "qe_pack_adapters")
+
+
+def pack_adapters_sparse(desc, A_s, B_s, channels, A_r, B_r, G, out, stream=None):
+    """Cluster-sparse routed experts: channels int32 [N_r][k_c], A_r bf16 [N_r][k_c][r_r]."""
+    _need_cuda(A_s, B_s, channels, A_r, B_r, G, out)
+    _check(load().qe_pack_adapters_sparse(ctypes.byref(desc), _ptr(A_s), _ptr(B_s), _ptr(channels), _ptr(A_r),
+                                          _ptr(B_r), _ptr(G), _ptr(out), _stream(stream)), "qe_pack_adapters_sparse")
 
 
 def topk_importance(X, w_mean, k, idx, hist=None, accumulate=False, stream=None):
@@ -278,11 +288,13 @@ class QELayer:
         self._ws = None
 
     @classmethod
-    def from_float(cls, desc: LayerDesc, W, s, A_s, B_s, A_r, B_r, G, s_inv=None, stream=None) -> "QELayer":
+    def from_float(cls, desc: LayerDesc, W, s, A_s, B_s, A_r, B_r, G, s_inv=None, stream=None,
+                   channels=None) -> "QELayer":
         """W [d_out, d_in] (fp32/bf16), s [d_in] fp32, adapters/G bf16 in their natural layouts (CUDA tensors).
 
         s_inv (fp32 [d_in]) is the stored reciprocal smoothing factor the activations are
-        multiplied by. When omitted, it is fl32(1/s).
+        multiplied by. When omitted, it is fl32(1/s). With desc.routed_channels > 0, A_r is
+        bf16 [N_r][k_c][r_r] over `channels` (int32 [N_r][k_c]).
         """
         import torch
         dev = W.device
@@ -293,7 +305,10 @@ class QELayer:
         w_colmax = torch.empty(K, dtype=torch.float32, device=dev)
         quantize_weights(desc, W, s, w_packed, w_scale, w_mean, w_colmax, stream)
         adapters = torch.empty(adapter_packed_bytes(desc), dtype=torch.uint8, device=dev)
-        pack_adapters(desc, A_s, B_s, A_r, B_r, G, adapters, stream)
+        if desc.routed_channels > 0:
+            pack_adapters_sparse(desc, A_s, B_s, channels, A_r, B_r, G, adapters, stream)
+        else:
+            pack_adapters(desc, A_s, B_s, A_r, B_r, G, adapters, stream)
         if s_inv is None:
             s_inv = (torch.ones_like(s) / s).contiguous()
         return cls(desc, w_packed, w_scale, s_inv.contiguous(), adapters, w_mean, w_colmax)

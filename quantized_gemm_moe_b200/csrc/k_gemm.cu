@@ -868,7 +868,7 @@ cudaError_t launch_ugemm(const CUtensorMap& tm_x, const CUtensorMap& tm_acat, co
   switch (plan.nu) {
 #define QE_NU(n) \
   case n: return launch_ugemm_t<n>(tm_x, tm_acat, plan, T, K, R_tot, partial, zero_ctr, err, st);
-    QE_NU(16) QE_NU(80) QE_NU(144) QE_NU(208) QE_NU(64) QE_NU(128) QE_NU(192) QE_NU(256)
+    QE_NU(16) QE_NU(32) QE_NU(48) QE_NU(80) QE_NU(144) QE_NU(208) QE_NU(64) QE_NU(128) QE_NU(192) QE_NU(256)
 #undef QE_NU
     default: return cudaErrorInvalidValue;
   }

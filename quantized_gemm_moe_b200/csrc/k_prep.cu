@@ -444,23 +444,42 @@ __global__ void __launch_bounds__(128) k_unpack_w(const uint8_t* __restrict__ pa
 // B_catT [N][R_pad] fp16 (up-projections). The up-projections are fp16 because the epilogue
 // MMA multiplies them with the fp16 U_cat; a bf16 value beyond the fp16 range is saturated
 // and reported (device error 0x201).
-__global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a, int R_pad, int R_tot,
-                                const uint16_t* __restrict__ A_s, const uint16_t* __restrict__ B_s,
+// Cluster-sparse routed experts (kc > 0): A_r is [n_r][kc][r_r] over the channels ch[n_r][kc];
+// they are copied to rch/rar (a channel outside [0, K) becomes channel 0 with zero weights and is
+// reported as device error 0x202), and A_catT holds no routed rows.
+__global__ void k_pack_adapters(int K, int N, int r_s, int n_r, int r_r, int R_a, int R_pad, int R_tot, int R_rt,
+                                int kc, const uint16_t* __restrict__ A_s, const uint16_t* __restrict__ B_s,
                                 const uint16_t* __restrict__ A_r, const uint16_t* __restrict__ B_r,
-                                const uint16_t* __restrict__ G, uint16_t* __restrict__ acat,
-                                uint16_t* __restrict__ bcat, int* __restrict__ err) {
+                                const uint16_t* __restrict__ G, const int32_t* __restrict__ ch,
+                                uint16_t* __restrict__ acat, uint16_t* __restrict__ bcat,
+                                int32_t* __restrict__ rch, uint16_t* __restrict__ rar, int* __restrict__ err) {
   const size_t n1 = static_cast<size_t>(R_tot) * K, n2 = static_cast<size_t>(N) * R_pad;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n1 + n2;
+  const size_t n3 = static_cast<size_t>(n_r) * kc, n4 = n3 * (kc ? r_r : 0);
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n1 + n2 + n3 + n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    if (i >= n1 + n2) {
+      const size_t ii = i - n1 - n2;
+      if (ii < n3) {
+        const int c = ch[ii];
+        const bool ok = c >= 0 && c < K;
+        if (!ok && err) atomicCAS(err, 0, 0x202);
+        rch[ii] = ok ? c : 0;
+      } else {
+        const size_t jj = ii - n3;  // (e * kc + i) * r_r + j
+        const int c = ch[jj / r_r];
+        rar[jj] = (c >= 0 && c < K) ? A_r[jj] : 0;
+      }
+      continue;
+    }
     if (i < n1) {
       const int c = static_cast<int>(i / K), k = static_cast<int>(i % K);
       uint16_t v = 0;
       if (c < r_s) v = A_s[static_cast<size_t>(k) * r_s + c];
-      else if (c < R_a) {
+      else if (kc == 0 && c < R_a) {
         const int e = (c - r_s) / r_r, j = (c - r_s) % r_r;
         v = A_r[(static_cast<size_t>(e) * K + k) * r_r + j];
-      } else if (c >= R_pad && c < R_pad + n_r) {
-        v = G[static_cast<size_t>(k) * n_r + (c - R_pad)];
+      } else if (c >= R_rt && c < R_rt + n_r) {
+        v = G[static_cast<size_t>(k) * n_r + (c - R_rt)];
       }
       acat[i] = v;
     } else {
@@ -570,7 +589,10 @@ __device__ bool grid_barrier(unsigned* ctr, int* err) {
 //          zeroed) / su[p]), su[p] a power of two that puts the row's largest |U| in [2^13, 2^14).
 struct RouteQuantArgs {
   const float* partial;
-  int nslots, R_tot, R_pad, n_r, r_s, r_r, R_a;
+  int nslots, R_tot, R_pad, R_rt, n_r, r_s, r_r, R_a;
+  int kc;               // cluster-sparse routed experts: channels per expert (0: dense)
+  const int32_t* rch;   // [n_r][kc]
+  const uint16_t* rar;  // bf16 [n_r][kc][r_r]
   const void* X;
   const float* s_inv;
   const float* amax;
@@ -678,7 +700,7 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
     // ---- per token: logits, argmin (the token's first warp), absmax (all of its warps)
     for (int t = t0 + slot; t < t1; t += nslot_w) {
       if (sub == 0) {
-        const float L = (lane < n_r) ? slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_pad + lane,
+        const float L = (lane < n_r) ? slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_rt + lane,
                                                 slot_stride, a.nslots)
                                      : 0.0f;
         float best = (lane < n_r) ? L : INFINITY;
@@ -860,9 +882,43 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
       float mx = 0.0f;
       for (int c = lane; c < a.R_pad; c += 32) {
         float v = 0.0f;
-        if (c < a.R_a && (c < a.r_s || (c - a.r_s) / a.r_r == e)) v = slot_sum(prow + c, slot_stride, a.nslots);
+        if (c < a.R_a && (c < a.r_s || (a.kc == 0 && (c - a.r_s) / a.r_r == e)))
+          v = slot_sum(prow + c, slot_stride, a.nslots);
         uw[c] = v;
         mx = fmaxf(mx, fabsf(v));
+      }
+      if (a.kc > 0) {
+        // cluster-sparse expert: its routed columns gather the expert's channels of the raw row
+        __syncwarp();
+        const int32_t* chs = a.rch + static_cast<size_t>(e) * a.kc;
+        const uint16_t* ar = a.rar + static_cast<size_t>(e) * a.kc * a.r_r;
+        for (int j0 = 0; j0 < a.r_r; j0 += 8) {
+          float acc[8];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.0f;
+          for (int i = lane; i < a.kc; i += 32) {
+            const int c = chs[i];
+            const float x = BF16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.X)[static_cast<size_t>(t) * a.K + c])
+                                 : static_cast<const float*>(a.X)[static_cast<size_t>(t) * a.K + c];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+              if (j0 + jj < a.r_r) acc[jj] = fmaf(x, bf16_bits_to_f32(ar[static_cast<size_t>(i) * a.r_r + j0 + jj]), acc[jj]);
+          }
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc[jj] += __shfl_xor_sync(0xffffffffu, acc[jj], off);
+          }
+          if (lane < 8 && j0 + lane < a.r_r) {
+            float v = acc[0];
+#pragma unroll
+            for (int jj = 1; jj < 8; ++jj)
+              if (lane == jj) v = acc[jj];
+            uw[a.r_s + e * a.r_r + j0 + lane] = v;
+            mx = fmaxf(mx, fabsf(v));
+          }
+        }
+        __syncwarp();
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -962,11 +1018,14 @@ cudaError_t launch_unpack_weights(const uint8_t* packed, int N, int K, int w_bit
 }
 
 cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint16_t* A_s, const uint16_t* B_s,
-                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out, int* err,
-                                 cudaStream_t st) {
-  k_pack_adapters<<<592, 256, 0, st>>>(K, N, g.r_s, g.n_r, g.r_r > 0 ? g.r_r : 1, g.R_a, g.R_pad, g.R_tot, A_s, B_s,
-                                       A_r, B_r, G, reinterpret_cast<uint16_t*>(out + g.off_acat),
-                                       reinterpret_cast<uint16_t*>(out + g.off_bcat), err);
+                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, const int32_t* channels,
+                                 uint8_t* out, int* err, cudaStream_t st) {
+  k_pack_adapters<<<592, 256, 0, st>>>(K, N, g.r_s, g.n_r, g.r_r > 0 ? g.r_r : 1, g.R_a, g.R_pad, g.R_tot, g.R_rt,
+                                       g.kc, A_s, B_s, A_r, B_r, G, channels,
+                                       reinterpret_cast<uint16_t*>(out + g.off_acat),
+                                       reinterpret_cast<uint16_t*>(out + g.off_bcat),
+                                       reinterpret_cast<int32_t*>(out + g.off_rch),
+                                       reinterpret_cast<uint16_t*>(out + g.off_rar), err);
   return cudaGetLastError();
 }
 
@@ -1009,6 +1068,10 @@ cudaError_t launch_route_quant(const RouteQuantParams& q, cudaStream_t st) {
   a.nslots = q.nslots;
   a.R_tot = q.R_tot;
   a.R_pad = q.R_pad;
+  a.R_rt = q.R_rt;
+  a.kc = q.kc;
+  a.rch = q.rch;
+  a.rar = q.rar;
   a.n_r = q.n_r;
   a.r_s = q.r_s;
   a.r_r = q.r_r > 0 ? q.r_r : 1;

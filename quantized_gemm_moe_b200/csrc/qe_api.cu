@@ -42,6 +42,9 @@ qe_status check_desc(const qe_layer_desc* d) {
   if (d->rank_shared < 0 || d->rank_routed < 0) return QE_ERR_INVALID_ARG;
   if (d->rank_shared + int64_t(d->n_routed) * d->rank_routed > 512) return QE_ERR_UNSUPPORTED;
   if (d->d_in > (1 << 24) || d->d_out > (1 << 24)) return QE_ERR_UNSUPPORTED;
+  if (d->routed_channels < 0 || d->routed_channels > d->d_in) return QE_ERR_INVALID_ARG;
+  if (d->routed_channels > 0 && (d->rank_routed == 0 || sparse_gemm_width(d->rank_shared) == 0))
+    return QE_ERR_UNSUPPORTED;
   return QE_OK;
 }
 
@@ -53,7 +56,7 @@ size_t packed_bytes(const qe_layer_desc* d) {
 }
 
 AdapterGeom geom_of(const qe_layer_desc* d) {
-  return adapter_geom(d->d_in, d->d_out, d->rank_shared, d->n_routed, d->rank_routed);
+  return adapter_geom(d->d_in, d->d_out, d->rank_shared, d->n_routed, d->rank_routed, d->routed_channels);
 }
 
 // ------------------------------------------------------------------ workspace plan
@@ -227,6 +230,10 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
     q.nslots = p.uslots;
     q.R_tot = p.g.R_tot;
     q.R_pad = p.g.R_pad;
+    q.R_rt = p.g.R_rt;
+    q.kc = p.g.kc;
+    q.rch = reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(w->adapters) + p.g.off_rch);
+    q.rar = reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(w->adapters) + p.g.off_rar);
     q.n_r = d->n_routed;
     q.r_s = d->rank_shared;
     q.r_r = d->rank_routed;
@@ -384,16 +391,24 @@ qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, qe_dtype
 
 qe_status qe_pack_adapters(const qe_layer_desc* desc, const void* A_s, const void* B_s, const void* A_r,
                            const void* B_r, const void* G, void* out, void* stream) {
+  if (desc && desc->routed_channels != 0) return QE_ERR_INVALID_ARG;  // cluster-sparse: qe_pack_adapters_sparse
+  return qe_pack_adapters_sparse(desc, A_s, B_s, nullptr, A_r, B_r, G, out, stream);
+}
+
+qe_status qe_pack_adapters_sparse(const qe_layer_desc* desc, const void* A_s, const void* B_s,
+                                  const int32_t* channels, const void* A_r, const void* B_r, const void* G, void* out,
+                                  void* stream) {
   qe_status st = check_desc(desc);
   if (st != QE_OK) return st;
   if (!G || !out) return QE_ERR_INVALID_ARG;
+  if (desc->routed_channels > 0 && !channels) return QE_ERR_INVALID_ARG;
   if (desc->rank_shared > 0 && (!A_s || !B_s)) return QE_ERR_INVALID_ARG;
   if (desc->rank_routed > 0 && (!A_r || !B_r)) return QE_ERR_INVALID_ARG;
   if (!aligned16(out)) return QE_ERR_ALIGNMENT;
   const AdapterGeom g = geom_of(desc);
   QE_CUDA(launch_pack_adapters(g, desc->d_in, desc->d_out, static_cast<const uint16_t*>(A_s),
                                static_cast<const uint16_t*>(B_s), static_cast<const uint16_t*>(A_r),
-                               static_cast<const uint16_t*>(B_r), static_cast<const uint16_t*>(G),
+                               static_cast<const uint16_t*>(B_r), static_cast<const uint16_t*>(G), channels,
                                static_cast<uint8_t*>(out), device_error_ptr(), static_cast<cudaStream_t>(stream)),
           "pack_adapters");
   return QE_OK;

@@ -19,28 +19,52 @@ __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Packed adapter buffer geometry.
-//   A_catT [R_tot][K] bf16: rows [0, R_a) are the shared and routed down-projections
-//     (A_s columns, then A_r[e] columns expert by expert), rows [R_pad, R_pad + N_r) are the
-//     router G (transposed), all other rows zero. One GEMM gives U and the router logits.
-//   B_catT [N][R_pad] fp16: the matching up-projections (absent when R_pad = 0).
+//   A_catT [R_tot][K] bf16: the rows of the adapter/router GEMM. Rows [0, r_s) are the shared
+//     down-projection. Dense routed experts add rows [r_s, R_a) (A_r[e] columns expert by
+//     expert) and the router G (transposed) sits at rows [R_rt, R_rt + N_r) with R_rt = R_pad.
+//     Cluster-sparse routed experts (kc > 0) have no GEMM rows: the router follows the shared
+//     rows (R_rt = the smallest supported GEMM width >= round_up(r_s, 16) + 16, minus 16).
+//     All other rows are zero. One GEMM gives U and the router logits.
+//   B_catT [N][R_pad] fp16: the up-projections of the shared and all routed columns.
+//   kc > 0: the channels of each expert, int32 [N_r][kc], and its down-projection over them,
+//     bf16 [N_r][kc][r_r].
 struct AdapterGeom {
   int r_s, n_r, r_r;
   int R_a;    // r_s + n_r * r_r
   int R_pad;  // round_up(R_a, 64), or 0 when the layer has no adapters
-  int R_tot;  // R_pad + 16 when that fits one 256-column MMA, else R_pad + 64
-  size_t off_acat, off_bcat, bytes;
+  int R_tot;  // rows of A_catT = columns of the adapter/router GEMM
+  int R_rt;   // first router row
+  int kc;     // channels per routed expert (0: dense routed experts)
+  size_t off_acat, off_bcat, off_rch, off_rar, bytes;
 };
-inline AdapterGeom adapter_geom(int K, int N, int r_s, int n_r, int r_r) {
+inline int sparse_gemm_width(int r_s) {
+  // adapter/router GEMM widths the library instantiates (see launch_ugemm)
+  const int need = static_cast<int>(round_up(r_s, 16)) + 16;
+  const int widths[] = {16, 32, 48, 64, 80, 128, 144, 192, 208, 256};
+  for (int w : widths)
+    if (w >= need) return w;
+  return 0;
+}
+inline AdapterGeom adapter_geom(int K, int N, int r_s, int n_r, int r_r, int kc) {
   AdapterGeom g;
   g.r_s = r_s;
   g.n_r = n_r;
   g.r_r = r_r;
+  g.kc = (r_r > 0) ? kc : 0;
   g.R_a = r_s + n_r * r_r;
   g.R_pad = g.R_a > 0 ? static_cast<int>(round_up(g.R_a, kAdapterAtom)) : 0;
-  g.R_tot = (g.R_pad + 16 <= 256) ? g.R_pad + 16 : g.R_pad + 64;
+  if (g.kc == 0) {
+    g.R_tot = (g.R_pad + 16 <= 256) ? g.R_pad + 16 : g.R_pad + 64;
+    g.R_rt = g.R_pad;
+  } else {
+    g.R_tot = sparse_gemm_width(r_s);
+    g.R_rt = g.R_tot - 16;
+  }
   g.off_acat = 0;
   g.off_bcat = align256(g.off_acat + size_t(g.R_tot) * K * 2);
-  g.bytes = align256(g.off_bcat + size_t(N) * g.R_pad * 2);
+  g.off_rch = align256(g.off_bcat + size_t(N) * g.R_pad * 2);
+  g.off_rar = align256(g.off_rch + size_t(n_r) * g.kc * 4);
+  g.bytes = align256(g.off_rar + size_t(n_r) * g.kc * (g.kc ? r_r : 0) * 2);
   return g;
 }
 
@@ -54,8 +78,8 @@ cudaError_t launch_colstats(const void* W, bool w_bf16, int N, int K, float* w_m
 cudaError_t launch_unpack_weights(const uint8_t* packed, int N, int K, int w_bits, int8_t* codes,
                                   cudaStream_t st);
 cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint16_t* A_s, const uint16_t* B_s,
-                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, uint8_t* out, int* err,
-                                 cudaStream_t st);
+                                 const uint16_t* A_r, const uint16_t* B_r, const uint16_t* G, const int32_t* channels,
+                                 uint8_t* out, int* err, cudaStream_t st);
 
 // Router logits + argmin, and (when sa != nullptr) the per-token absmax -> scale, on CUDA cores
 // (the standalone router entry point and the activation-quantization diagnostic).
@@ -99,7 +123,12 @@ constexpr int kRouteQuantMaxGrid = 1024;
 constexpr int kMaxForwardDin = 32768;  // the route/quant launch keeps s_inv in shared memory
 struct RouteQuantParams {
   const float* partial;
-  int nslots, R_tot, R_pad, n_r, r_s, r_r, R_a;
+  int nslots, R_tot, R_pad, R_rt, n_r, r_s, r_r, R_a;
+  // cluster-sparse routed experts (kc > 0): expert e's routed U columns are
+  // sum_i x[t][rch[e][i]] * rar[e][i][j] (raw x), not GEMM columns
+  int kc;
+  const int32_t* rch;
+  const uint16_t* rar;
   const void* X;
   bool x_bf16;
   const float* s_inv;

@@ -42,17 +42,30 @@ def f32(a) -> np.ndarray:
 class Case:
     """One layer with its inputs on both sides (CPU oracle and GPU library)."""
 
-    def __init__(self, cfg: qi.LayerConfig, proj: qi.Projection, T: int, proj_index: int = 0, inp=None):
+    def __init__(self, cfg: qi.LayerConfig, proj: qi.Projection, T: int, proj_index: int = 0, inp=None,
+                 routed_channels: int = 0, sparse_seed: int = 77):
+        """routed_channels > 0: cluster-sparse routed experts (qe_inputs.sparse_routed). The oracle
+        then gets the equivalent dense A_r: zero outside each expert's channels."""
         self.cfg = cfg
         self.proj = proj
         self.T = T
         self.inp = inp if inp is not None else qi.layer_inputs(cfg, proj, T=T, proj_index=proj_index)
         self.desc = qe.make_desc(proj.d_in, proj.d_out, cfg.group, cfg.w_bits, cfg.a_bits, cfg.rank_shared,
-                                 cfg.n_routed, cfg.rank_routed)
+                                 cfg.n_routed, cfg.rank_routed, routed_channels)
         i = self.inp
         self.Xd = cuda(i["X"])
-        self.layer = qe.QELayer.from_float(self.desc, cuda(i["W"]), cuda(i["s"]), cuda(i["A_s"]), cuda(i["B_s"]),
-                                           cuda(i["A_r"]), cuda(i["B_r"]), cuda(i["G"]), s_inv=cuda(i["s_inv"]))
+        if routed_channels:
+            ch, A_rs = qi.sparse_routed(proj.d_in, cfg.n_routed, routed_channels, cfg.rank_routed, sparse_seed)
+            dense = torch.zeros((cfg.n_routed, proj.d_in, cfg.rank_routed), dtype=torch.bfloat16)
+            for e in range(cfg.n_routed):
+                dense[e, torch.from_numpy(ch[e]).long()] += A_rs[e]
+            i["A_r"] = dense
+            self.layer = qe.QELayer.from_float(self.desc, cuda(i["W"]), cuda(i["s"]), cuda(i["A_s"]), cuda(i["B_s"]),
+                                               cuda(A_rs), cuda(i["B_r"]), cuda(i["G"]), s_inv=cuda(i["s_inv"]),
+                                               channels=cuda(ch))
+        else:
+            self.layer = qe.QELayer.from_float(self.desc, cuda(i["W"]), cuda(i["s"]), cuda(i["A_s"]), cuda(i["B_s"]),
+                                               cuda(i["A_r"]), cuda(i["B_r"]), cuda(i["G"]), s_inv=cuda(i["s_inv"]))
         self._ref = None
 
     def oracle_weights(self):

@@ -302,6 +302,21 @@ def test_forward_weight_only(T, K, N, group, bits, rs, nr, rr):
     _forward_check(Case(cfg, qi.Projection("p", K, N), T), with_acc=False)
 
 
+@pytest.mark.parametrize("T,K,N,group,a_bits,w_bits,rs,nr,rr,kc,xdt", [
+    (64, 256, 256, 64, 8, 4, 8, 4, 4, 16, "f32"),         # adapter/router GEMM 32 wide
+    (300, 1536, 1536, 128, 6, 4, 32, 8, 4, 32, "bf16"),   # 48 wide
+    (129, 512, 384, 128, 8, 4, 32, 8, 32, 16, "bf16"),    # r_r = 32: U_cat 320 wide, GEMM 48 wide
+    (16, 1024, 640, 128, 16, 3, 32, 8, 4, 32, "bf16"),    # weight-only
+    (40, 512, 256, 128, 6, 4, 0, 4, 8, 24, "bf16"),       # no shared expert: GEMM 16 wide
+])
+def test_forward_cluster_sparse_routed(T, K, N, group, a_bits, w_bits, rs, nr, rr, kc, xdt):
+    # Routed experts that touch only their cluster's channels: the forward gathers them per token;
+    # the oracle runs the dense formula with A_r zero outside the clusters.
+    cfg = _cfg(group=group, a_bits=a_bits, w_bits=w_bits, rank_shared=rs, n_routed=nr, rank_routed=rr,
+               x_dtype=xdt, spec="qwen2b" if K >= 1024 else "tiny")
+    _forward_check(Case(cfg, qi.Projection("p", K, N), T, routed_channels=kc), with_acc=(a_bits != 16))
+
+
 def test_forward_bf16_output_is_rounded_fp32_output():
     cfg = _cfg(a_bits=6, x_dtype="bf16", group=128, rank_shared=32, n_routed=8)
     c = Case(cfg, qi.Projection("p", 512, 384), 70)
@@ -332,10 +347,10 @@ def test_forward_empty_batch_is_noop():
 
 # ---------------------------------------------------------------- full-size layers, sampled rows
 
-def _full_size(cfg_name, proj_index, n_rows=48):
+def _full_size(cfg_name, proj_index, n_rows=48, routed_channels=0):
     cfg = qi.CONFIGS[cfg_name]
     proj = cfg.projections[proj_index]
-    c = Case(cfg, proj, cfg.T, proj_index=proj_index)
+    c = Case(cfg, proj, cfg.T, proj_index=proj_index, routed_channels=routed_channels)
     Y, _, expert, _, _ = c.gpu_debug(with_acc=False)
     e = expert.cpu().numpy()
     rows = np.random.default_rng(proj_index).choice(cfg.T, min(n_rows, cfg.T), replace=False).astype(np.int32)
@@ -356,6 +371,12 @@ def _full_size(cfg_name, proj_index, n_rows=48):
 @pytest.mark.parametrize("proj_index", range(5))
 def test_full_size_qwen2vl2b_layer_set(proj_index):
     _full_size("qwen2vl2b", proj_index)
+
+
+@pytest.mark.parametrize("proj_index", [0, 4])
+def test_full_size_cluster_sparse_routed(proj_index):
+    # the 2B layer set at T = 2048 with each routed expert on 32 channels
+    _full_size("qwen2vl2b", proj_index, routed_channels=32)
 
 
 @pytest.mark.parametrize("cfg_name", ["qwen2vl2b_w4a16", "qwen2vl2b_w3a16"])
