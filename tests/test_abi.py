@@ -63,6 +63,8 @@ def test_sizes_follow_documented_layout(lib):
     ("n_routed", 17, qe.QE_ERR_UNSUPPORTED),
     ("rank_shared", -1, qe.QE_ERR_INVALID_ARG),
     ("rank_routed", 200, qe.QE_ERR_UNSUPPORTED),  # 8 + 4*200 > 512
+    ("routed_channels", -1, qe.QE_ERR_INVALID_ARG),
+    ("routed_channels", 257, qe.QE_ERR_INVALID_ARG),   # more channels than d_in
 ])
 def test_invalid_desc_rejected_before_launch(lib, field, value, status):
     d = qe.make_desc(256, 256, 64, 4, 8, 8, 4, 4)
@@ -101,6 +103,25 @@ def test_other_entry_points_validate(lib):
     assert lib.qe_pack_adapters(ctypes.byref(d), 16, 16, 16, 16, None, 16, None) == qe.QE_ERR_INVALID_ARG
     for s in range(7):
         assert lib.qe_status_string(s)
+
+
+def test_cluster_sparse_sizes_and_checks(lib):
+    # A_catT keeps the shared rows and the router (48 rows at r_s = 32), B_catT is unchanged, and the
+    # packed buffer adds the channel lists (int32 [N_r][k_c]) and their weights (bf16 [N_r][k_c][r_r])
+    d = qe.make_desc(1536, 8960, 128, 4, 6, 32, 8, 4, 32)
+    expect = 0
+    for nbytes in (48 * 1536 * 2, 8960 * 64 * 2, 8 * 32 * 4, 8 * 32 * 4 * 2):
+        expect = ((expect + nbytes + 255) // 256) * 256
+    assert qe.adapter_packed_bytes(d) == expect
+    # no shared expert: the router alone is 16 rows; r_s = 8: 32 rows
+    assert qe.adapter_packed_bytes(qe.make_desc(1536, 8960, 128, 4, 6, 0, 8, 4, 32)) > 0
+    # the dense packing call refuses a sparse descriptor, and sparse routing needs routed ranks
+    assert lib.qe_pack_adapters(ctypes.byref(d), 16, 16, 16, 16, 16, 16, None) == qe.QE_ERR_INVALID_ARG
+    assert lib.qe_pack_adapters_sparse(ctypes.byref(d), 16, 16, None, 16, 16, 16, 16, None) == qe.QE_ERR_INVALID_ARG
+    d_nr = qe.make_desc(1536, 8960, 128, 4, 6, 32, 8, 0, 32)
+    assert qe.packed_weight_bytes(d_nr) == 0  # rejected: k_c > 0 without routed ranks
+    d_wide = qe.make_desc(1536, 8960, 128, 4, 6, 248, 8, 4, 32)
+    assert qe.packed_weight_bytes(d_wide) == 0  # r_s beyond the sparse GEMM widths
 
 
 def test_binding_refuses_cpu_tensors(lib):
