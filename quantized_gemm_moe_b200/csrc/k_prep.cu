@@ -761,6 +761,33 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
       for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
       if (lane == 0) a.counts[blockIdx.x * kMaxRouted + warp] = c;
     }
+    // ---- stable ranks inside this CTA's range (they need no other CTA), kRQThreads tokens at a
+    //      time: pos_s holds each token's rank among this CTA's tokens of its expert
+    if (threadIdx.x < n_r) run_s[threadIdx.x] = 0;
+    __syncthreads();
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int c0 = t0; c0 < t1; c0 += kRQThreads) {
+      const int t = c0 + static_cast<int>(threadIdx.x);
+      const int e = (t < t1) ? e_s[t - t0] : -1;
+      int rank = 0;
+      for (int ee = 0; ee < n_r; ++ee) {
+        const uint32_t m = __ballot_sync(0xffffffffu, e == ee);
+        if (lane == 0) wcnt[warp][ee] = __popc(m);
+        if (e == ee) rank = __popc(m & lt_mask);
+      }
+      __syncthreads();
+      if (threadIdx.x < n_r) {
+        int run = run_s[threadIdx.x];
+        for (int w = 0; w < kWarps; ++w) {
+          wbase[w][threadIdx.x] = run;
+          run += wcnt[w][threadIdx.x];
+        }
+        run_s[threadIdx.x] = run;
+      }
+      __syncthreads();
+      if (t < t1) pos_s[t - t0] = wbase[warp][e] + rank;
+      __syncthreads();
+    }
     if (!grid_barrier(a.barrier, a.err)) return;
     // ---- bucket offsets: experts before e, plus earlier CTAs' tokens of e
     if (warp < n_r) {
@@ -792,35 +819,13 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
       }
     }
     __syncthreads();
-    // ---- stable ranks inside this CTA's range, kRQThreads tokens at a time
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int c0 = t0; c0 < t1; c0 += kRQThreads) {
-      const int t = c0 + static_cast<int>(threadIdx.x);
-      const int e = (t < t1) ? e_s[t - t0] : -1;
-      int rank = 0;
-      for (int ee = 0; ee < n_r; ++ee) {
-        const uint32_t m = __ballot_sync(0xffffffffu, e == ee);
-        if (lane == 0) wcnt[warp][ee] = __popc(m);
-        if (e == ee) rank = __popc(m & lt_mask);
-      }
-      __syncthreads();
-      if (threadIdx.x < n_r) {
-        int run = run_s[threadIdx.x];
-        for (int w = 0; w < kWarps; ++w) {
-          wbase[w][threadIdx.x] = run;
-          run += wcnt[w][threadIdx.x];
-        }
-        run_s[threadIdx.x] = run;
-      }
-      __syncthreads();
-      if (t < t1) {
-        const int p = wbase[warp][e] + rank;
-        a.perm[p] = t;
-        a.pos[t] = p;
-        pos_s[t - t0] = p;
-      }
-      __syncthreads();
+    for (int i = threadIdx.x; i < t1 - t0; i += kRQThreads) {
+      const int p = run_s[e_s[i]] + pos_s[i];
+      a.perm[p] = t0 + i;
+      a.pos[t0 + i] = p;
+      pos_s[i] = p;
     }
+    __syncthreads();
   } else if (a.do_quant) {
     for (int i = threadIdx.x; i < t1 - t0; i += kRQThreads) {
       pos_s[i] = a.pos[t0 + i];
