@@ -750,7 +750,9 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
     if (a.sa_tok) {
       for (int i = threadIdx.x; i < t1 - t0; i += kRQThreads) {
         const float mx = BF16 ? __int_as_float(mx_s[i]) : a.amax[t0 + i];
-        a.sa_tok[t0 + i] = __fdiv_rn(mx, static_cast<float>(a.qmax));
+        const float sa = __fdiv_rn(mx, static_cast<float>(a.qmax));
+        a.sa_tok[t0 + i] = sa;
+        mx_s[i] = __float_as_int(sa);  // the quantization below reads it from here
       }
     }
     // ---- this CTA's count per expert
@@ -837,7 +839,7 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
   // ---- per token, in bucket order (the token's warps share the row; its first warp writes the rest)
   for (int t = t0 + slot; t < t1; t += nslot_w) {
     const size_t p = static_cast<size_t>(pos_s[t - t0]);
-    const float sa = a.codes ? a.sa_tok[t] : 0.0f;
+    const float sa = a.codes ? (a.do_route ? __int_as_float(mx_s[t - t0]) : a.sa_tok[t]) : 0.0f;
     const float inv = (sa > 0.0f) ? __frcp_rn(sa) : 0.0f;
     const bool fast = rtn_fast_ok(sa, inv);
     for (int k0 = (sub * 32 + lane) * 8; k0 < a.K; k0 += 256 * wpt * kB) {
