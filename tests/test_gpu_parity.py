@@ -325,6 +325,23 @@ def test_forward_bf16_output_is_rounded_fp32_output():
     assert torch.equal(y16, y32.to(torch.bfloat16))
 
 
+@pytest.mark.parametrize("cfg_name,proj_index,T,N", [
+    ("qwen2vl2b", 0, 2048, None), ("qwen2vl2b", 2, 2048, None), ("qwen2vl2b", 4, 2048, None),
+    ("qwen2vl2b", 0, 300, 1001), ("qwen2vl2b", 4, 1000, 1000), ("tiny", 0, 64, None),
+])
+def test_forward_bf16_output_full_size(cfg_name, proj_index, T, N):
+    # bf16 output (the staged-tile store for tiles up to 192 tokens, the pass-wise store above)
+    # equals the fp32 output (checked against the oracle elsewhere) rounded to bf16, element by element
+    cfg = qi.CONFIGS[cfg_name]
+    proj = cfg.projections[proj_index]
+    if N is not None:
+        proj = qi.Projection(proj.name, proj.d_in, N)
+    c = Case(cfg, proj, T, proj_index=proj_index)
+    y32 = c.gpu_forward(torch.float32)
+    y16 = c.gpu_forward(torch.bfloat16)
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
 def test_forward_deterministic_and_token_independent():
     cfg = _cfg(a_bits=8, x_dtype="bf16", group=128, rank_shared=32, n_routed=8)
     c = Case(cfg, qi.Projection("p", 512, 384), 200)
