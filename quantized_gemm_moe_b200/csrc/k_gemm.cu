@@ -10,7 +10,7 @@
 //     warps 1-2   one thread each issues tcgen05.mma kind::i8 for alternate
 //                 stages, one TMEM accumulator buffer per quantization group
 //                 (2 buffers at BN >= 192, 4 below, so the MMA runs ahead of the
-//                 epilogue)
+//                 epilogue; each issuer owns half of them)
 //     warps 4-11  epilogue: the per-group promotion acc += sw[o,j] * float(int32)
 //                 in registers (f32x2, the next TMEM chunk loading meanwhile),
 //                 then * sa[t], + adapter MMA result, and a scatter of the row
@@ -62,6 +62,7 @@ struct QCfg {
   static constexpr int kStage = kA + kB + kWP;
   static constexpr int kStages = (BN >= 192) ? 3 : (BN >= 128 ? 4 : (BN >= 64 ? 5 : 6));
   static constexpr int kNBuf = (BN >= 192) ? 2 : 4;  // TMEM accumulator buffers
+  static_assert(kNBuf % 2 == 0, "each MMA issuer owns half of the buffers");
   // TMEM is allocated in powers of two (>= 32 columns)
   static constexpr int kTmemCols = (kNBuf * BN <= 32) ? 32 : (kNBuf * BN <= 128 ? 128 : (kNBuf * BN <= 256 ? 256 : 512));
   static constexpr int kCPT = BN / 2;              // columns per epilogue thread
@@ -107,6 +108,21 @@ __device__ __forceinline__ uint64_t pack2(float x) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
   return r;
+}
+
+// Which TMEM buffer the epilogue drains next. The two MMA issuers take alternate stages, and
+// issuer q cycles through its own buffers q, q+2, ..., q+2(kOwn-1). The epilogue tracks the
+// issuers' progress in one word: bit 0 = parity of the current unit's first stage, bits 1..3 /
+// 4..6 = groups issued so far by issuer 0 / 1, mod 8 (enough for kOwn <= 4). Returns the
+// buffer and sets `use_parity` to the parity of that buffer's use.
+template <int kOwn>
+__device__ __forceinline__ int epi_next_buffer(uint32_t& st, int iq, uint32_t& use_parity) {
+  static_assert(kOwn >= 1 && kOwn <= 4, "buffer state holds counts mod 8");
+  const int sh = 1 + 3 * iq;
+  const uint32_t oc = (st >> sh) & 7u;
+  st = (st & ~(7u << sh)) | (((oc + 1u) & 7u) << sh);
+  use_parity = (oc / kOwn) & 1u;
+  return iq + 2 * static_cast<int>(oc % kOwn);
 }
 
 // One unit of work: a 128-row output tile, a BN-position token tile and a K split.
@@ -220,7 +236,9 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* accf = bars + 3 * NS;   // [NB] accumulator buffer ready for the epilogue
   uint64_t* acce = accf + NB;       // [NB] accumulator buffer drained and re-biased (8 warp arrivals)
   uint64_t* done = acce + NB;       // [1] teardown
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* adone = done + 1;       // [1] adapter block: its issuer waited for all of its stages
+  uint64_t* aack = adone + 1;       // [1] adapter block: the other issuer saw adone
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aack + 1);
   float* sa_s = reinterpret_cast<float*>(out_stage + C::kOut + 512);
   float* su_s = sa_s + BN;
   int32_t* perm_s = reinterpret_cast<int32_t*>(su_s + BN);
@@ -243,6 +261,9 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&acce[b], 8);
     }
     mbar_init(done, 2);
+    mbar_init(adone, 1);
+    mbar_init(aack, 1);
+    mbar_arrive(aack);  // phase 0: nothing to acknowledge before the first adapter block
     mbar_fence_init();
     prefetch_tmap(&tm_xq);
     if (a.adapter_atoms) {
@@ -316,6 +337,14 @@ __global__ void __launch_bounds__(512, 1)
     // buffer, so one issuer takes all of them and their fp32 sums keep a fixed order.
     // The unpack warps wait for the TMA bytes before they arrive on afull, so afull alone
     // tells an issuer that both operands of the stage are in shared memory.
+    // A parity wait is only sound when the waiter is at most one phase ahead of the barrier.
+    // An issuer skips the other's stages, so two rules keep it within one phase:
+    //  - TMEM buffers are owned: issuer q uses buffers q, q+2, ... in turn, so its waits on
+    //    a buffer's acce are for consecutive drains of that buffer;
+    //  - after skipping another issuer's adapter block (possibly longer than the stage ring),
+    //    an issuer waits on adone, which the owner arrives on once it has waited for every
+    //    stage of the block; the owner of the next block first waits on aack, so adone is
+    //    never two blocks ahead of its waiter.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegLow) : "memory");
     const int qi = warp - 1;
     if (lane == 0) {
@@ -324,7 +353,9 @@ __global__ void __launch_bounds__(512, 1)
       // Descriptors are built once; a stage or a 32-byte K step only moves the start address
       // field (16-byte units in the low bits, no carry below 256 KB of shared memory).
       const uint64_t desc0 = smem_desc_sw128(smem_u32(stage_base));
-      int it = 0, gidx = 0;
+      constexpr int kOwn = NB / 2;  // TMEM buffers per issuer
+      int it = 0;
+      uint32_t own = 0, ablk = 0;  // groups this issuer took (mod 8), adapter blocks seen (mod 2)
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const Unit w = make_unit(a, BN, u);
@@ -335,12 +366,9 @@ __global__ void __launch_bounds__(512, 1)
           const uint64_t da = desc0 + static_cast<uint64_t>((s * C::kStage) >> 4);
           const uint64_t db = da + (C::kA >> 4);
           if (i < w.nkb) {
+            if ((it & 1) != qi) continue;
             const int kb = w.kb_begin + i;
             const int ng = max(0, min(gpb, w.g_begin + w.n_groups - kb * gpb));
-            if ((it & 1) != qi) {
-              gidx += ng;
-              continue;
-            }
             if (!mbar_wait(&afull[s], ph, a_err, DEVERR_WAIT_MMA)) {
               ok = false;
               break;
@@ -349,8 +377,10 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int gi = 0; gi < 2; ++gi) {
               if (gi >= ng) break;
-              const int b = gidx % NB;
-              if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
+              const int b = qi + 2 * static_cast<int>(own % kOwn);
+              const uint32_t use = own / kOwn;
+              own = (own + 1) & 7u;
+              if (!mbar_wait(&acce[b], (use & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
                 ok = false;
                 break;
               }
@@ -364,21 +394,27 @@ __global__ void __launch_bounds__(512, 1)
                 for (int kk = 0; kk < 2; ++kk) mma_i8(d, da + 4 * gi + 2 * kk, db + 4 * gi + 2 * kk, id_i8, 1u);
               }
               tc_commit(&accf[b]);
-              ++gidx;
             }
           } else {
             const int at = i - w.nkb;
-            const int b = gidx % NB;
             if (ad_owner != qi) {
-              if (at == w.n_ad - 1) ++gidx;
+              if (at == w.n_ad - 1) {
+                if (!mbar_wait(adone, ablk, a_err, DEVERR_WAIT_MMA)) {
+                  ok = false;
+                  break;
+                }
+                mbar_arrive(aack);
+                ablk ^= 1u;
+              }
               continue;
             }
+            const int b = qi + 2 * static_cast<int>(own % kOwn);
             if (!mbar_wait(&afull[s], ph, a_err, DEVERR_WAIT_MMA)) {
               ok = false;
               break;
             }
             if (at == 0) {
-              if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
+              if (!mbar_wait(&acce[b], ((own / kOwn) & 1u) ^ 1u, a_err, DEVERR_WAIT_MMA)) {
                 ok = false;
                 break;
               }
@@ -389,10 +425,19 @@ __global__ void __launch_bounds__(512, 1)
             for (int kk = 0; kk < 4; ++kk) mma_f16(d, da + 2 * kk, db + 2 * kk, id_ad, (at > 0 || kk > 0) ? 1u : 0u);
             if (at == w.n_ad - 1) {
               tc_commit(&accf[b]);
-              ++gidx;
+              own = (own + 1) & 7u;
             }
           }
           tc_commit(&empty[s]);
+          if (i >= w.nkb && i - w.nkb == w.n_ad - 1) {
+            // this issuer owned the adapter block and has waited for all of its stages
+            if (!mbar_wait(aack, ablk, a_err, DEVERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive(adone);
+            ablk ^= 1u;
+          }
         }
       }
       // make sure everything this thread issued has completed before TMEM is released
@@ -458,7 +503,10 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     const uint64_t magic2 = pack2(kMagic);
     uint8_t* my_out = out_stage + h * (C::kOut / 2);
-    int gidx = 0;
+    // group -> TMEM buffer as the issuers assign it: K block i of a unit is issued by the
+    // issuer of the stage's parity, which takes its buffers q, q+2, ... in turn
+    constexpr int kOwn = NB / 2;
+    uint32_t bstate = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const Unit w = make_unit(a, BN, u);
@@ -498,13 +546,15 @@ __global__ void __launch_bounds__(512, 1)
       for (int j = 0; j < kSwAhead; ++j)
         swq[j] = (o_ok && j < w.n_groups) ? __ldg(swp + static_cast<size_t>(j) * a.N) : 0.0f;
       for (int g = 0; g < w.n_groups; ++g) {
-        const int b = gidx % NB;
-        ++gidx;
+        uint32_t use;
+        const int b = epi_next_buffer<kOwn>(bstate, static_cast<int>(bstate & 1u), use);
+        // bit 0 follows the stage parity: flip it after the last group of each K block
+        if (a.group == kTileK || (g & 1) || g + 1 == w.n_groups) bstate ^= 1u;
         const uint64_t sw2 = pack2(swq[0] * 0.0625f);
 #pragma unroll
         for (int j = 0; j + 1 < kSwAhead; ++j) swq[j] = swq[j + 1];
         swq[kSwAhead - 1] = (o_ok && g + kSwAhead < w.n_groups) ? __ldg(swp + static_cast<size_t>(g + kSwAhead) * a.N) : 0.0f;
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], use & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (!ok) continue;
         tc_fence_after();
         const uint32_t base = tmem + lane_base + b * BN + h * C::kCPT;
@@ -555,9 +605,9 @@ __global__ void __launch_bounds__(512, 1)
       }
       // adapters: acc += su[t] * (U_cat . B_cat^T)
       if (w.n_ad > 0) {
-        const int b = gidx % NB;
-        ++gidx;
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+        uint32_t use;
+        const int b = epi_next_buffer<kOwn>(bstate, static_cast<int>(bstate & 1u), use);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], use & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (ok) {
           tc_fence_after();
           const uint32_t base = tmem + lane_base + b * BN + h * C::kCPT;
@@ -587,6 +637,7 @@ __global__ void __launch_bounds__(512, 1)
       // store: transpose through shared memory, then write whole row segments with 16-byte stores
       if (a.splits == 1 && a.y_bf16) store_tile<C::kCPT, 2>(acc, my_out, perm_s + h * C::kCPT, w, a, o0, 32 * q + lane, wt, h, ok, false);
       else store_tile<C::kCPT, 4>(acc, my_out, perm_s + h * C::kCPT, w, a, o0, 32 * q + lane, wt, h, ok, a.splits > 1);
+      bstate ^= static_cast<uint32_t>(w.n_ad) & 1u;
     }
     tc_fence_before();
   }

@@ -43,6 +43,7 @@ struct WCfg {
   static constexpr int kNW = 6;                 // packed weight ring
   static constexpr int kWP = 8192;
   static constexpr int kNB = (BN <= 64) ? 8 : 4;  // TMEM accumulator buffers (fp32, BN columns each)
+  static_assert(kNB % 2 == 0, "each MMA issuer owns half of the buffers");
   // Roles (512 threads): warp 0 weight blocks, warps 1-2 MMA issuers, warp 3 activation tiles,
   // then the epilogue warps, then the unpack warps. 128-token tiles take a second team of 4
   // epilogue warps from the unpack warps: each team keeps half of the tile's columns in
@@ -59,6 +60,21 @@ struct WCfg {
       1024 + size_t(kNA) * kSlot + size_t(kNW) * kWP + kOut + 1024 + size_t(BN) * 8;
   static_assert(kSmem <= 232448, "shared memory");
 };
+
+// Which TMEM buffer the epilogue drains next. The two MMA issuers take alternate stages, and
+// issuer q cycles through its own buffers q, q+2, ..., q+2(kOwn-1). The epilogue tracks the
+// issuers' progress in one word: bit 0 = parity of the current unit's first stage, bits 1..3 /
+// 4..6 = groups issued so far by issuer 0 / 1, mod 8 (enough for kOwn <= 4). Returns the
+// buffer and sets `use_parity` to the parity of that buffer's use.
+template <int kOwn>
+__device__ __forceinline__ int epi_next_buffer(uint32_t& st, int iq, uint32_t& use_parity) {
+  static_assert(kOwn >= 1 && kOwn <= 4, "buffer state holds counts mod 8");
+  const int sh = 1 + 3 * iq;
+  const uint32_t oc = (st >> sh) & 7u;
+  st = (st & ~(7u << sh)) | (((oc + 1u) & 7u) << sh);
+  use_parity = (oc / kOwn) & 1u;
+  return iq + 2 * static_cast<int>(oc % kOwn);
+}
 
 struct WUnit {
   int nt, p0, split, kb_begin, nkb, n_ad, g_begin, n_groups;
@@ -135,7 +151,9 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* accf = aempty + NA;       // [NB] group sum ready
   uint64_t* acce = accf + NB;         // [NB] group sum read (every epilogue warp)
   uint64_t* done = acce + NB;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* adone = done + 1;         // adapter block: its issuer waited for all of its slots
+  uint64_t* aack = adone + 1;         // adapter block: the other issuer saw adone
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aack + 1);
   float* su_s = reinterpret_cast<float*>(bars + 64);
   int32_t* perm_s = reinterpret_cast<int32_t*>(su_s + BN);
 
@@ -159,6 +177,9 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&acce[b], C::kEpiWarps);
     }
     mbar_init(done, 2);
+    mbar_init(adone, 1);
+    mbar_init(aack, 1);
+    mbar_arrive(aack);  // phase 0: nothing to acknowledge before the first adapter block
     mbar_fence_init();
     prefetch_tmap(&tm_act);
     if (a.adapter_atoms) {
@@ -229,13 +250,18 @@ __global__ void __launch_bounds__(512, 1)
     // ------------------------------------------------------------ MMA issuers
     // Two threads issue alternate blocks: one thread's issue rate, not the tensor pipe, limits
     // these narrow (BN <= 64) MMAs. A unit's adapter atoms accumulate into one TMEM buffer, so
-    // one issuer takes all of them.
+    // one issuer takes all of them. Parity waits stay within one phase of their barrier as in
+    // the int8 kernel: issuer q owns TMEM buffers q, q+2, ..., and an issuer that skipped an
+    // adapter block waits on adone (the owner waited for every slot of the block) before its
+    // next slot; the owner of the next block first waits on aack.
     const int qi = warp - 1;
     if (lane == 0) {
       const uint32_t id_bf = idesc_bf16(128, BN);
       const uint32_t id_ad = idesc_f16(128, BN);
       const uint64_t desc_a0 = smem_desc_sw128(smem_u32(slots));
-      int it = 0, gidx = 0;
+      constexpr int kOwn = NB / 2;  // TMEM buffers per issuer
+      int it = 0;
+      uint32_t own = 0, ablk = 0;  // groups this issuer took (mod 8), adapter blocks seen (mod 2)
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const WUnit w = make_wunit(a, BN, u);
@@ -247,10 +273,7 @@ __global__ void __launch_bounds__(512, 1)
           if (i < w.nkb) {
             const int kb = w.kb_begin + i;
             const int ng = max(0, min(gpb, w.g_begin + w.n_groups - kb * gpb));
-            if ((it & 1) != qi) {
-              gidx += ng;
-              continue;
-            }
+            if ((it & 1) != qi) continue;
             if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
               ok = false;
               break;
@@ -259,8 +282,10 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int gi = 0; gi < 2; ++gi) {
               if (gi >= ng) break;
-              const int b = gidx % NB;
-              if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
+              const int b = qi + 2 * static_cast<int>(own % kOwn);
+              const uint32_t use = own / kOwn;
+              own = (own + 1) & 7u;
+              if (!mbar_wait(&acce[b], (use & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
                 ok = false;
                 break;
               }
@@ -276,21 +301,27 @@ __global__ void __launch_bounds__(512, 1)
                 mma_f16(d, da + off, db + offb, id_bf, kk > 0 ? 1u : 0u);
               }
               tc_commit(&accf[b]);
-              ++gidx;
             }
           } else {
             const int at = i - w.nkb;
-            const int b = gidx % NB;
             if (ad_owner != qi) {
-              if (at == w.n_ad - 1) ++gidx;
+              if (at == w.n_ad - 1) {
+                if (!mbar_wait(adone, ablk, a_err, DEVERR_WAIT_MMA)) {
+                  ok = false;
+                  break;
+                }
+                mbar_arrive(aack);
+                ablk ^= 1u;
+              }
               continue;
             }
+            const int b = qi + 2 * static_cast<int>(own % kOwn);
             if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
               ok = false;
               break;
             }
             if (at == 0) {
-              if (!mbar_wait(&acce[b], ((gidx / NB) & 1) ^ 1, a_err, DEVERR_WAIT_MMA)) {
+              if (!mbar_wait(&acce[b], ((own / kOwn) & 1u) ^ 1u, a_err, DEVERR_WAIT_MMA)) {
                 ok = false;
                 break;
               }
@@ -301,10 +332,19 @@ __global__ void __launch_bounds__(512, 1)
             for (int kk = 0; kk < 4; ++kk) mma_f16(d, da + 2 * kk, db + 2 * kk, id_ad, (at > 0 || kk > 0) ? 1u : 0u);
             if (at == w.n_ad - 1) {
               tc_commit(&accf[b]);
-              ++gidx;
+              own = (own + 1) & 7u;
             }
           }
           tc_commit(&aempty[s]);
+          if (i >= w.nkb && i - w.nkb == w.n_ad - 1) {
+            // this issuer owned the adapter block and has waited for all of its slots
+            if (!mbar_wait(aack, ablk, a_err, DEVERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive(adone);
+            ablk ^= 1u;
+          }
         }
       }
       tc_commit(done);
@@ -405,7 +445,9 @@ __global__ void __launch_bounds__(512, 1)
     const int ch0 = team * EC;          // this team's first column
     const int et = threadIdx.x - 128;   // 0..NE-1
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    int gidx = 0;
+    // group -> TMEM buffer as the issuers assign it (issuer of the block's parity, its buffers in turn)
+    constexpr int kOwn = NB / 2;
+    uint32_t bstate = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const WUnit w = make_wunit(a, BN, u);
@@ -425,11 +467,13 @@ __global__ void __launch_bounds__(512, 1)
       const float* swp = a.w_scale + static_cast<size_t>(w.g_begin) * a.N + o;
       float sw_next = (o_ok && w.n_groups > 0) ? __ldg(swp) : 0.0f;
       for (int g = 0; g < w.n_groups; ++g) {
-        const int b = gidx % NB;
-        ++gidx;
+        uint32_t use;
+        const int b = epi_next_buffer<kOwn>(bstate, static_cast<int>(bstate & 1u), use);
+        // bit 0 follows the stage parity: flip it after the last group of each K block
+        if (a.group == kTileK || (g & 1) || g + 1 == w.n_groups) bstate ^= 1u;
         const float sw = sw_next;
         if (o_ok && g + 1 < w.n_groups) sw_next = __ldg(swp + static_cast<size_t>(g + 1) * a.N);
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], use & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (!ok) continue;
         tc_fence_after();
         const uint32_t base = tmem + lane_base + b * BN + ch0;
@@ -448,9 +492,9 @@ __global__ void __launch_bounds__(512, 1)
         if (lane == 0) mbar_arrive(&acce[b]);
       }
       if (w.n_ad > 0) {
-        const int b = gidx % NB;
-        ++gidx;
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], ((gidx - 1) / NB) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+        uint32_t use;
+        const int b = epi_next_buffer<kOwn>(bstate, static_cast<int>(bstate & 1u), use);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], use & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (ok) {
           tc_fence_after();
           const uint32_t base = tmem + lane_base + b * BN + ch0;
@@ -522,6 +566,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         asm volatile("bar.sync 2, %0;" ::"n"(NE) : "memory");
       }
+      bstate ^= static_cast<uint32_t>(w.n_ad) & 1u;
     }
     tc_fence_before();
   }

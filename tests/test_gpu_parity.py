@@ -368,9 +368,16 @@ def _full_size(cfg_name, proj_index, n_rows=48, routed_channels=0):
     cfg = qi.CONFIGS[cfg_name]
     proj = cfg.projections[proj_index]
     c = Case(cfg, proj, cfg.T, proj_index=proj_index, routed_channels=routed_channels)
+    _sampled_check(c, n_rows, proj_index)
+
+
+def _sampled_check(c, n_rows, seed):
+    # sampled output rows against the oracle (routing checked on the same rows), the whole
+    # output finite, and the weight codes bit-exact
+    cfg, proj = c.cfg, c.proj
     Y, _, expert, _, _ = c.gpu_debug(with_acc=False)
     e = expert.cpu().numpy()
-    rows = np.random.default_rng(proj_index).choice(cfg.T, min(n_rows, cfg.T), replace=False).astype(np.int32)
+    rows = np.random.default_rng(seed).choice(c.T, min(n_rows, c.T), replace=False).astype(np.int32)
     _, e_ref = oracle.route(f32(c.inp["X"])[rows], c.inp["G"])
     check_routing(f32(c.inp["X"])[rows], c.inp["G"], e[rows], e_ref)
     Y_ref, _ = c.oracle_forward(rows=rows, expert_override=e[rows])
@@ -383,6 +390,32 @@ def _full_size(cfg_name, proj_index, n_rows=48, routed_channels=0):
     qe.unpack_weights(c.desc, c.layer.w_packed, got)
     torch.cuda.synchronize()
     assert (got.cpu().numpy() == codes).all()
+    return Y
+
+
+@pytest.mark.parametrize("T,K,N,group,a_bits,w_bits,rr", [
+    (2048, 512, 2048, 128, 8, 4, 32),    # 256-token tiles (3 stages, 2 TMEM buffers), 5 adapter atoms
+    (2048, 512, 2048, 64, 6, 4, 4),      # 256-token tiles, g = 64: two groups per stage on 2 buffers
+    (2048, 512, 2048, 64, 8, 4, 32),     # both
+    (2048, 1536, 1536, 64, 6, 4, 32),    # 192-token tiles
+    (1000, 512, 1024, 128, 8, 4, 16),    # 128-token tiles (4 stages), 3 adapter atoms
+    (1200, 512, 2048, 128, 16, 3, 32),   # weight-only 128-token tiles (2 operand slots), 5 atoms
+    (1200, 512, 2048, 64, 16, 4, 32),
+    (48, 512, 1024, 64, 16, 4, 32),      # weight-only 64-token tile (3 slots)
+    (200, 512, 1024, 128, 16, 3, 16),
+])
+def test_forward_long_adapter_blocks_and_two_group_stages(T, K, N, group, a_bits, w_bits, rr):
+    # Shapes where one MMA issuer skips more of the other's stages than the ring holds (an
+    # adapter block of R_pad/64 atoms), or where a stage carries two groups on two TMEM
+    # buffers: each issuer must still wait on the right barrier phase. Sampled rows against
+    # the oracle, and a repeat must be bit-identical (a missed wait shows up as a race).
+    cfg = _cfg(group=group, a_bits=a_bits, w_bits=w_bits, rank_shared=32, n_routed=8, rank_routed=rr,
+               x_dtype="bf16", spec="qwen2b" if K >= 1024 else "tiny")
+    c = Case(cfg, qi.Projection("p", K, N), T)
+    Y = _sampled_check(c, 48, T + rr)
+    for _ in range(3):
+        assert torch.equal(c.gpu_forward(), Y)
+    assert qe.device_error() == 0
 
 
 @pytest.mark.parametrize("proj_index", range(5))
