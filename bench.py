@@ -57,6 +57,13 @@ WORKLOADS = {
     "decode72b_w4a8_t1": ("decode72b_w4a8", 1, "72B decode gate/up/down, T=1, W4A8 g128"),
     "decode72b_w3a16": ("decode72b_w3a16", 16, "72B decode gate/up/down, T=16, W3A16 g128"),
     "decode72b_w3a16_t1": ("decode72b_w3a16", 1, "72B decode gate/up/down, T=1, W3A16 g128"),
+    "decode72b_w4a8_t4": ("decode72b_w4a8", 4, "72B decode gate/up/down, T=4, W4A8 g128"),
+    "decode72b_w3a16_t4": ("decode72b_w3a16", 4, "72B decode gate/up/down, T=4, W3A16 g128"),
+    "qwen2vl72b_rr32": ("qwen2vl72b_rr32", None, "Qwen2VL-72B-shaped layer set, T=8192, W4A6 g128, routed rank 32 "
+                                                 "(ablation)"),
+    "qwen2vl72b_rr32_sparse": ("qwen2vl72b_rr32", None, "Qwen2VL-72B-shaped layer set, T=8192, W4A6 g128, routed rank "
+                                                        "32 (ablation), cluster-sparse routed experts on 32 channels",
+                               32),
 }
 METRIC = "QE linear tokens/s and effective TOPS; % of int8-TC / HBM roofline, 1 B200"
 

@@ -211,6 +211,12 @@ CONFIGS = {
         (Projection("q", 1536, 1536), Projection("o", 1536, 1536), Projection("gate", 1536, 8960),
          Projection("up", 1536, 8960), Projection("down", 8960, 1536)),
         3, 16, 128, 32, 8, 4, 32, "bf16", "qwen2b", 8),
+    "qwen2vl72b_rr32": LayerConfig(
+        "qwen2vl72b_rr32", 8192,
+        (Projection("q", 8192, 8192), Projection("k", 8192, 1024), Projection("v", 8192, 1024),
+         Projection("o", 8192, 8192), Projection("gate", 8192, 29568), Projection("up", 8192, 29568),
+         Projection("down", 29568, 8192)),
+        4, 6, 128, 32, 8, 32, 32, "bf16", "scaled", 9),
     "decode72b_w4a8": LayerConfig(
         "decode72b_w4a8", 16,
         (Projection("gate", 8192, 29568), Projection("up", 8192, 29568), Projection("down", 29568, 8192)),
