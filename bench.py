@@ -87,7 +87,9 @@ def parse_args():
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CALIB_WORKLOADS), default="qwen2vl2b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=64)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="oracle time the cpu_baseline sample is sized for (the reference arm: per step, "
+                         "capped so that all steps take about two minutes)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="token count per GPU instead of the workload's own (smaller cases for ncu captures)")
     return ap.parse_args()
@@ -198,19 +200,50 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- reference arm (CPU oracle)
 
-def oracle_sample_run(cfg, T_total, sample_tokens, seed_shift=0):
-    """Times the oracle's forward over `sample_tokens` tokens of every projection. Returns seconds."""
+ORACLE_PREP_TOKENS = 2048  # token rows prepared for the oracle's timed sample
+
+
+def oracle_layer_set(cfg, n_tokens, seed_shift=0):
+    """The oracle's inputs for every projection (weights quantized once, outside any timing) and a
+    function that times its forward over the first n of `n_tokens` tokens. Returns (run, n_tokens)."""
     import oracle
     prep = []
     for pi, proj in enumerate(cfg.projections):
-        inp = qi.layer_inputs(cfg, proj, T=sample_tokens, proj_index=pi + seed_shift)
+        inp = qi.layer_inputs(cfg, proj, T=n_tokens, proj_index=pi + seed_shift)
         codes, scales, _, _ = oracle.quantize_weights(inp["W"], inp["s"], cfg.group, cfg.w_bits)
+        del inp["W"]
         prep.append((inp, codes, scales))
-    t0 = time.perf_counter()
-    for inp, codes, scales in prep:
-        oracle.qe_forward(inp["X"], codes, scales, inp["s_inv"], inp["A_s"], inp["B_s"], inp["A_r"], inp["B_r"],
-                          inp["G"], cfg.group, cfg.a_bits)
-    return time.perf_counter() - t0
+
+    def run(n):
+        t0 = time.perf_counter()
+        for inp, codes, scales in prep:
+            oracle.qe_forward(inp["X"][:n], codes, scales, inp["s_inv"], inp["A_s"], inp["B_s"], inp["A_r"],
+                              inp["B_r"], inp["G"], cfg.group, cfg.a_bits)
+        return time.perf_counter() - t0
+    return run, n_tokens
+
+
+def sized_oracle_sample(run, n_avail, target_s, probe=16, max_passes=10):
+    """Times `run(n)` (the oracle over the first n tokens, in seconds) on a sample sized for about
+    target_s seconds: a probe of a few tokens gives the rate, then n = min(n_avail, rate * target_s)
+    tokens, passed again over the same tokens while the total is short of the target (tokens are
+    independent, so a pass costs the same each time). Returns (tokens processed, seconds, n)."""
+    p = max(1, min(probe, n_avail))
+    sp = run(p)
+    n = int(min(n_avail, max(p, p * target_s / max(sp, 1e-9))))
+    tok, secs = 0, 0.0
+    for _ in range(max_passes):
+        secs += run(n)
+        tok += n
+        if secs >= 0.8 * target_s:
+            break
+    return tok, secs, n
+
+
+def reference_step_seconds(args):
+    """Oracle time per reference-arm step: the cpu_baseline target, capped so that all steps take
+    about two minutes."""
+    return max(0.5, min(args.cpu_seconds, 120.0 / max(1, args.steps)))
 
 
 def run_reference(args, workload):
@@ -222,19 +255,25 @@ def run_reference(args, workload):
     T = args.tokens or t_over or cfg.T
     cores = os.cpu_count() or 1
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
-    sample = max(1, min(args.cpu_sample_tokens, T))
+    run, n_avail = oracle_layer_set(cfg, min(T, ORACLE_PREP_TOKENS))
     for _ in range(args.warmup):
-        oracle_sample_run(cfg, T, min(sample, 4))
-    secs = [oracle_sample_run(cfg, T, sample) for _ in range(args.steps)]
-    tot = sum(secs)
-    value = sample * args.steps / tot
+        run(min(n_avail, 4))
+    target = reference_step_seconds(args)
+    tok, tot, sample = 0, 0.0, 0
+    for _ in range(args.steps):
+        t_, s_, sample = sized_oracle_sample(run, n_avail, target)
+        tok += t_
+        tot += s_
+    value = tok / tot
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64", "data": "synthetic",
-        "config": {"workload": workload, "description": desc, "T": T, "sample_tokens_per_step": sample},
+        "config": {"workload": workload, "description": desc, "T": T, "sample_tokens_per_step": tok // args.steps},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{sample} tokens of every projection per step (tokens are independent)"},
+                         "sample": f"{tok // args.steps} token passes of every projection per step, about "
+                                   f"{target:.0f} s each (passes over the first {sample} tokens; tokens are "
+                                   f"independent)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -466,10 +505,11 @@ def run_ours(args, workload):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
         os.environ.setdefault("OMP_NUM_THREADS", str(cores))
-        sample = max(1, min(args.cpu_sample_tokens, T))
-        secs = oracle_sample_run(cfg, T, sample)
-        cpu = {"value": sample / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{sample} tokens through every projection of the layer set (tokens are independent)"}
+        run, n_avail = oracle_layer_set(cfg, min(T, ORACLE_PREP_TOKENS))
+        tok, secs, sample = sized_oracle_sample(run, n_avail, args.cpu_seconds)
+        cpu = {"value": tok / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{tok} token passes through every projection of the layer set in {secs:.1f} s "
+                         f"(the first {sample} tokens of the workload; tokens are independent)"}
 
     launches = sum(qe.linear_kernel_launches(L["desc"], T, qe.QE_BF16 if cfg.x_dtype == "bf16" else qe.QE_F32)
                    for L in layers) * args.steps
@@ -529,20 +569,25 @@ def run_calib(args, workload):
         if rank != 0:
             return 0
         cores = 1   # the oracle's Top-k, counts and NPMI run on one thread
-        sample = max(1, min(args.cpu_sample_tokens, T))
-        X, w_mean = calib_inputs(sample, d)
+        X, w_mean = calib_inputs(min(T, ORACLE_PREP_TOKENS), d)
         for _ in range(args.warmup):
             calib_oracle_run(X[:4], w_mean, k, C)
-        tot = sum(calib_oracle_run(X, w_mean, k, C) for _ in range(args.steps))
-        value = sample * args.steps / tot
+        target = reference_step_seconds(args)
+        tok, tot, sample = 0, 0.0, 0
+        for _ in range(args.steps):
+            t_, s_, sample = sized_oracle_sample(lambda n: calib_oracle_run(X[:n], w_mean, k, C), len(X), target)
+            tok += t_
+            tot += s_
+        value = tok / tot
         print(json.dumps({
             "impl": "reference", "metric": CALIB_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/int64/f64",
             "data": "synthetic", "config": {"workload": workload, "description": desc_txt, "T": T,
-                                            "sample_tokens_per_step": sample},
+                                            "sample_tokens_per_step": tok // args.steps},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{sample} tokens through Top-k, split, co-occurrence and NPMI per step"},
+                             "sample": f"{tok // args.steps} tokens through Top-k, split, co-occurrence and NPMI "
+                                       f"per step, about {target:.0f} s each (samples of the first {sample} tokens)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }), flush=True)
         return 0
@@ -643,10 +688,12 @@ def run_calib(args, workload):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sample = max(1, min(args.cpu_sample_tokens, T))
-        secs = calib_oracle_run(X_h[:sample], w_mean_h, k, C)
-        cpu = {"value": sample / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"{sample} tokens through Top-k, split, co-occurrence and NPMI"}
+        n_avail = min(T, ORACLE_PREP_TOKENS)
+        tok, secs, sample = sized_oracle_sample(lambda n: calib_oracle_run(X_h[:n], w_mean_h, k, C), n_avail,
+                                                args.cpu_seconds)
+        cpu = {"value": tok / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{tok} tokens through Top-k, split, co-occurrence and NPMI in {secs:.1f} s "
+                         f"(samples of the first {sample} tokens)"}
     line = {
         "metric": CALIB_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
