@@ -257,6 +257,23 @@ QE_API qe_status qe_linear_forward_stages(const qe_layer_desc* desc, const qe_la
 QE_API int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype);
 
 /*
+ * How qe_linear_forward runs this layer for T tokens (host only; no GPU call).
+ *   product_tile_tokens  token positions per tile of the main product (16 .. 256)
+ *   product_k_splits     K splits of the main product (> 1 adds a reduce launch)
+ *   adapter_atoms        64-wide adapter atoms per unit (R_pad / 64; 0 without adapters)
+ *   adapter_gemm_width   columns of the adapter/router GEMM (R_tot)
+ *   adapter_gemm_tile    its columns per CTA
+ *   adapter_gemm_splits  its K splits (partial slots; doubled for fp32 inputs)
+ *   weight_only          1 for a_bits = 16 (the weight-only product)
+ * Returns QE_ERR_INVALID_ARG for a null pointer or T < 1, and check errors of desc.
+ */
+typedef struct {
+  int32_t product_tile_tokens, product_k_splits, adapter_atoms, adapter_gemm_width, adapter_gemm_tile,
+      adapter_gemm_splits, weight_only;
+} qe_linear_plan_info;
+QE_API qe_status qe_linear_plan(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype, qe_linear_plan_info* out);
+
+/*
  * qe_linear_forward without a caller-provided workspace. (No counterpart in
  * the paper: this is a deployment convenience of this library.)
  *

@@ -25,6 +25,7 @@ EXPORTS = (
     "qe_last_cuda_error", "qe_device_error", "qe_unpack_weights", "qe_act_quant", "qe_linear_forward_debug",
     "qe_linear_forward_stages", "qe_linear_kernel_launches", "qe_linear_forward_noalloc",
     "qe_selftest_wait_timeout", "qe_split_channels", "qe_cooccurrence_npmi", "qe_pack_adapters_sparse",
+    "qe_linear_plan",
 )
 # fixed scratch of qe_linear_forward_noalloc (bytes), as declared in include/qe.h
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -49,6 +50,12 @@ class LayerDesc(ctypes.Structure):
 
     def __repr__(self):
         return "LayerDesc(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class LinearPlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("product_tile_tokens", "product_k_splits", "adapter_atoms",
+                                              "adapter_gemm_width", "adapter_gemm_tile", "adapter_gemm_splits",
+                                              "weight_only")]
 
 
 class LayerWeights(ctypes.Structure):
@@ -82,6 +89,7 @@ def load() -> ctypes.CDLL:
         "qe_linear_forward_debug": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P, S, P, P, P, P, P], I),
         "qe_linear_forward_stages": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P, S, I, P], I),
         "qe_linear_kernel_launches": ([D, I, I], I),
+        "qe_linear_plan": ([D, I, I, ctypes.POINTER(LinearPlan)], I),
         "qe_linear_forward_noalloc": ([D, ctypes.POINTER(LayerWeights), P, I, I, P, I, P], I),
         "qe_status_string": ([I], ctypes.c_char_p),
         "qe_last_cuda_error": ([], ctypes.c_char_p),
@@ -214,6 +222,13 @@ def linear_forward(desc, weights: LayerWeights, X, Y, workspace, stream=None):
 
 def linear_kernel_launches(desc: LayerDesc, T: int, x_dtype: int = QE_BF16) -> int:
     return int(load().qe_linear_kernel_launches(ctypes.byref(desc), T, x_dtype))
+
+
+def linear_plan(desc: LayerDesc, T: int, x_dtype: int = QE_BF16) -> dict:
+    """How the forward runs this layer for T tokens (tile width, splits, adapter atoms); host only."""
+    out = LinearPlan()
+    _check(load().qe_linear_plan(ctypes.byref(desc), T, x_dtype, ctypes.byref(out)), "qe_linear_plan")
+    return {n: getattr(out, n) for n, _ in LinearPlan._fields_}
 
 
 def linear_forward_stages(desc, weights: LayerWeights, X, Y, workspace, stages: int, stream=None):

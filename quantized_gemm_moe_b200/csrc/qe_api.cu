@@ -461,6 +461,22 @@ int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, qe_dtype
   return n;
 }
 
+qe_status qe_linear_plan(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype, qe_linear_plan_info* out) {
+  const qe_status st = check_desc(desc);
+  if (st != QE_OK) return st;
+  if (!out || T < 1) return QE_ERR_INVALID_ARG;
+  if (x_dtype != QE_F32 && x_dtype != QE_BF16) return QE_ERR_INVALID_ARG;
+  const Plan p = make_plan(desc, T, x_dtype == QE_BF16);
+  out->product_tile_tokens = p.bn;
+  out->product_k_splits = p.msplits;
+  out->adapter_atoms = p.has_ad ? p.g.R_pad / kAdapterAtom : 0;
+  out->adapter_gemm_width = p.g.R_tot;
+  out->adapter_gemm_tile = p.up.nu;
+  out->adapter_gemm_splits = p.uslots;
+  out->weight_only = desc->a_bits == 16 ? 1 : 0;
+  return QE_OK;
+}
+
 qe_status qe_linear_forward_stages(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
                                    qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* workspace,
                                    size_t workspace_bytes, int32_t stages, void* stream) {

@@ -130,3 +130,41 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises(qe.QEError):
         qe.quantize_weights(d, torch.zeros(256, 256), torch.ones(256), torch.zeros(10, dtype=torch.uint8),
                             torch.zeros(4, 256))
+
+
+# (T, K, N, group, a_bits, w_bits, r_r) -> (tile tokens, adapter atoms): the GPU parity shapes
+# that exercise the issuers' barrier rules must reach the tiles and atom counts they name
+@pytest.mark.parametrize("T,K,N,group,a_bits,w_bits,rr,tile,atoms", [
+    (2048, 512, 2048, 128, 8, 4, 32, 256, 5),
+    (2048, 512, 2048, 64, 6, 4, 4, 256, 1),
+    (2048, 512, 2048, 64, 8, 4, 32, 256, 5),
+    (2048, 1536, 1536, 64, 6, 4, 32, 192, 5),
+    (1000, 512, 1024, 128, 8, 4, 16, 128, 3),
+    (1200, 512, 2048, 128, 16, 3, 32, 128, 5),
+    (1200, 512, 2048, 64, 16, 4, 32, 128, 5),
+    (48, 512, 1024, 64, 16, 4, 32, 64, 5),
+    (200, 512, 1024, 128, 16, 3, 16, 64, 3),
+])
+def test_linear_plan_of_issuer_protocol_shapes(T, K, N, group, a_bits, w_bits, rr, tile, atoms):
+    d = qe.make_desc(K, N, group, w_bits, a_bits, 32, 8, rr)
+    p = qe.linear_plan(d, T)
+    assert (p["product_tile_tokens"], p["adapter_atoms"]) == (tile, atoms)
+    assert p["weight_only"] == (1 if a_bits == 16 else 0)
+
+
+def test_linear_plan_of_the_2b_layer_set_and_72b_rank32():
+    # the 2B layer set at T = 2048: q/o and down on 192-token tiles, gate/up on 256
+    for K, N, tile in [(1536, 1536, 192), (1536, 8960, 256), (8960, 1536, 192)]:
+        p = qe.linear_plan(qe.make_desc(K, N, 128, 4, 6, 32, 8, 4), 2048)
+        assert (p["product_tile_tokens"], p["product_k_splits"], p["adapter_atoms"]) == (tile, 1, 1)
+        assert (p["adapter_gemm_width"], p["adapter_gemm_tile"]) == (80, 80)
+    # routed rank 32 at the 72B size: R_pad = 320 (five atoms), the router GEMM 384 wide in two tiles
+    p = qe.linear_plan(qe.make_desc(8192, 29568, 128, 4, 6, 32, 8, 32), 8192)
+    assert (p["product_tile_tokens"], p["adapter_atoms"], p["adapter_gemm_width"], p["adapter_gemm_tile"]) == \
+        (256, 5, 384, 192)
+    # fp32 inputs run the adapter GEMM twice (hi and lo), so the partial slots double
+    pb = qe.linear_plan(qe.make_desc(1536, 1536, 128, 4, 8, 32, 8, 4), 300, qe.QE_BF16)
+    pf = qe.linear_plan(qe.make_desc(1536, 1536, 128, 4, 8, 32, 8, 4), 300, qe.QE_F32)
+    assert pf["adapter_gemm_splits"] == 2 * pb["adapter_gemm_splits"]
+    with pytest.raises(qe.QEError):
+        qe.linear_plan(qe.make_desc(1536, 1536, 128, 4, 8, 32, 8, 4), 0)
