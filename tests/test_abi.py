@@ -168,3 +168,42 @@ def test_linear_plan_of_the_2b_layer_set_and_72b_rank32():
     assert pf["adapter_gemm_splits"] == 2 * pb["adapter_gemm_splits"]
     with pytest.raises(qe.QEError):
         qe.linear_plan(qe.make_desc(1536, 1536, 128, 4, 8, 32, 8, 4), 0)
+
+
+C_CLIENT = r"""
+#include "qe.h"
+#include <stdio.h>
+int main(void) {
+  qe_layer_desc d = {1536, 1536, 128, 4, 6, 32, 8, 4, 0};
+  qe_linear_plan_info p;
+  qe_status s = qe_linear_plan(&d, 2048, QE_BF16, &p);
+  printf("%d %s %d %d %zu %d\n", (int)s, qe_status_string(s), p.product_tile_tokens, p.adapter_atoms,
+         qe_linear_workspace_bytes(&d, 2048), (int)qe_linear_kernel_launches(&d, 2048, QE_BF16));
+  return s == QE_OK ? 0 : 1;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    # the boundary is a C ABI: a strict C99 client compiles against include/qe.h without
+    # warnings, links libqe.so and gets the same answers as the binding (host-only calls)
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src, exe = tmp_path / "client.c", tmp_path / "client"
+    src.write_text(C_CLIENT)
+    libdir = os.path.join(ROOT, "quantized_gemm_moe_b200")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-L", libdir, "-lqe", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    st, text, tile, atoms, ws, launches = out.stdout.split()
+    d = qe.make_desc(1536, 1536, 128, 4, 6, 32, 8, 4)
+    assert (int(st), text) == (0, "ok")
+    assert (int(tile), int(atoms)) == (192, 1)
+    assert int(ws) == qe.linear_workspace_bytes(d, 2048)
+    assert int(launches) == qe.linear_kernel_launches(d, 2048)
