@@ -9,7 +9,9 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "table7_complexity.tx
 
 
 def _rows():
-    for line in open(GOLDEN):
+    with open(GOLDEN) as f:
+        lines = f.read().splitlines()
+    for line in lines:
         line = line.strip()
         if line and not line.startswith("#"):
             yield [int(v) for v in line.split()]
