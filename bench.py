@@ -115,7 +115,8 @@ def load_peaks():
 def git_src_hash(paths):
     h = hashlib.sha256()
     for p in paths:
-        h.update(open(os.path.join(ROOT, p), "rb").read())
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -126,7 +127,9 @@ def read_traffic(kernel_file: str, name: str):
     if not os.path.exists(p):
         return None
     vals = {}
-    for line in open(p):
+    with open(p) as f:
+        lines = f.read().splitlines()
+    for line in lines:
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             v = v.strip()
