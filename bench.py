@@ -7,17 +7,22 @@ A step is one pass of the hot path over one batch: every projection of the
 workload's layer set goes through the QE forward, in three stages: the
 tensor-core down-projection with the router logits; routing, the bucket
 sort and quantization with the expert-masked adapter rows (one cooperative
-launch); and the int8 tcgen05 product with its adapter epilogue. The step is captured once as a
-CUDA graph of the public forward calls with a timing event at each end, and
-replayed. Inputs are synthetic and seeded, with the shapes of the named
-model (qe_inputs), and resident in HBM when the timed region starts. L2 is
-flushed between steps, outside the timed intervals. A second graph with
-events between the stages, replayed after the timed region, gives the
-per-stage breakdown (per_projection) and the product kernels' time for the
-roofline. Under torchrun each rank runs an independent replica on its own
-token batch (weak scaling, no data-path collective), and the time is the
-max over ranks. e2e times the plain public call with pinned host buffers
-and the copies inside the timed region.
+launch); and the int8 tcgen05 product with its adapter epilogue. The default
+workload is the largest layer set that fits one GPU: the Qwen2VL-72B-shaped
+projections at T = 8192. The step is captured once as a CUDA graph of the
+public forward calls with a timing event at each end, and replayed. Inputs
+are synthetic and seeded, with the shapes of the named model (qe_inputs),
+and resident in HBM when the timed region starts. L2 is flushed between
+steps, outside the timed intervals. A second graph with events between the
+stages, replayed after the timed region, gives the per-stage breakdown
+(per_projection) and the product kernels' time for the roofline. With the
+default workload, the line also carries `decode`: the 72B decode-shaped
+gate/up/down layers (W4A8 and W3A16, T = 16 and T = 1), each timed the same
+way against the HBM roofline. Under torchrun each rank runs an independent
+replica on its own token batch (weak scaling, no data-path collective), and
+the time is the max over ranks; `--gpus N` without torchrun launches the N
+ranks itself. e2e times the plain public call with pinned host buffers and
+the copies inside the timed region.
 
 `--impl reference` times the CPU oracle (a deliberately slow, plain program)
 on a bounded token sample of the same workload, on the host's cores.
@@ -66,6 +71,8 @@ WORKLOADS = {
                                32),
 }
 METRIC = "QE linear tokens/s and effective TOPS; % of int8-TC / HBM roofline, 1 B200"
+# The largest layer set that fits one GPU: the Qwen2VL-72B-shaped projections at T = 8192.
+DEFAULT_WORKLOAD = "qwen2vl72b"
 
 # The calibration statistics: per-token Top-k importance with its histogram, the channel split,
 # the co-occurrence counts of the token-dependent channels and their NPMI.
@@ -78,13 +85,15 @@ CALIB_WORKLOADS = {
 CALIB_METRIC = "QE calibration statistic tokens/s (Top-k, split, co-occurrence, NPMI); % of HBM roofline, 1 B200"
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CALIB_WORKLOADS), default="qwen2vl2b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CALIB_WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-decode", action="store_true",
+                    help="leave out the decode-shaped 72B layers measured beside the default workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-mode", choices=["serial", "overlap"], default="serial",
@@ -96,7 +105,7 @@ def parse_args():
                          "capped so that all steps take about two minutes)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="token count per GPU instead of the workload's own (smaller cases for ncu captures)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def dist_env():
@@ -224,7 +233,7 @@ def oracle_layer_set(cfg, n_tokens, seed_shift=0):
     def run(n):
         t0 = time.perf_counter()
         for inp, codes, scales in prep:
-            oracle.qe_forward(inp["X"][:n], codes, scales, inp["s_inv"], inp["A_s"], inp["B_s"], inp["A_r"],
+            oracle.qe_forward(inp["X"][:n], codes, scales, oracle.smoothing_inverse(inp["s"]), inp["A_s"], inp["B_s"], inp["A_r"],
                               inp["B_r"], inp["G"], cfg.group, cfg.a_bits)
         return time.perf_counter() - t0
     return run, n_tokens
@@ -329,7 +338,7 @@ def build_layers(cfg, T, rank, dev, routed_channels=0):
                                                     6000 + pi)
             channels = c(channels)
         layer = qe.QELayer.from_float(desc, c(inp["W"]), c(inp["s"]), c(inp["A_s"]), c(inp["B_s"]), c(inp["A_r"]),
-                                      c(inp["B_r"]), c(inp["G"]), s_inv=c(inp["s_inv"]), channels=channels)
+                                      c(inp["B_r"]), c(inp["G"]), channels=channels)
         X = c(inp["X"])
         Y = torch.empty((T, proj.d_out), dtype=torch.bfloat16, device=dev)
         ws = layer.workspace(T)
@@ -370,6 +379,162 @@ def e2e_overlapped_step(qe, layers, xh, yh, stream, s_in, s_out):
     stream.wait_event(out_done)
 
 
+def time_layer_set(qe, layers, T, args, flush, pg, stages, clocks=True):
+    """Times one step (every projection through the public forward call, T tokens each) as a CUDA
+    graph replay with an event at each end, L2 flushed before each replay. A second graph splits
+    each forward into its stages with events between them; its replays after the timed region give
+    the per-stage breakdown. Returns (step_ms [steps], stage_ms [n_diag, proj, stage], clocks)."""
+    import torch
+    ins = [(L["desc"], L["layer"].weights, L["X"][:T], L["Y"][:T], L["layer"].workspace(T)) for L in layers]
+
+    def step_plain():
+        for d, w, X, Y, ws in ins:
+            qe.linear_forward(d, w, X, Y, ws)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step_plain()
+    torch.cuda.synchronize()
+    assert qe.device_error() == 0, "a device wait ran out during warm-up"
+    cap = torch.cuda.Stream()
+    ev0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev1 = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap):
+        ev0.record()
+        step_plain()
+        ev1.record()
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)] for _ in ins]
+    sgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(sgraph, stream=cap):
+        for (d, w, X, Y, ws), e in zip(ins, evs):
+            e[0].record()
+            for i, sm in enumerate(stages):
+                qe.linear_forward_stages(d, w, X, Y, ws, sm)
+                e[i + 1].record()
+    for _ in range(2):
+        graph.replay()
+        sgraph.replay()
+    torch.cuda.synchronize()
+    step_ms = np.zeros(args.steps)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if clk:
+        clk.__enter__()
+    try:
+        for s_i in range(args.steps):
+            flush.zero_()
+            graph.replay()
+            torch.cuda.synchronize()
+            step_ms[s_i] = ev0.elapsed_time(ev1)
+    finally:
+        if clk:
+            clk.__exit__(None, None, None)
+    if pg:
+        pg.barrier()
+    n_diag = max(3, min(args.steps, 10))
+    stage_ms = np.zeros((n_diag, len(ins), len(stages)))
+    for s_i in range(n_diag):
+        flush.zero_()
+        sgraph.replay()
+        torch.cuda.synchronize()
+        for p_i, e in enumerate(evs):
+            for k in range(len(stages)):
+                stage_ms[s_i, p_i, k] = e[k].elapsed_time(e[k + 1])
+    err = qe.device_error()
+    assert err == 0, f"device wait ran out (code {err:#x})"
+    del graph, sgraph
+    return step_ms, stage_ms, (clk.summary() if clk else None)
+
+
+def measure_int8_peak(dev):
+    """Dense int8 tensor-core throughput of the library GEMM on this GPU: torch._int_mm (cuBLASLt)
+    of 8192^3, best of 10 CUDA-event timings after warm-up. None if the call is unavailable."""
+    import torch
+    n = 8192
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev).t()
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._int_mm(a, b)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        torch.cuda.empty_cache()
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:  # pragma: no cover - reported as unavailable
+        return None
+
+
+def product_roofline(cfg, layers, T, prod_ms, peaks, int8, traffic):
+    """Roofline of the dominant kernel (the main product) for one timed layer set."""
+    from quantized_gemm_moe_b200 import roofline
+    wonly = cfg.a_bits == 16
+    kernel = "wgemm" if wonly else "qgemm"
+    if T <= 16:
+        # decode: HBM bound; the product streams the packed codes, the scales and the adapters
+        by = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
+                                      cfg.n_routed, cfg.rank_routed, 1 if not wonly else 2, 2) for L in layers)
+        ach = by / (prod_ms / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "kernel": kernel,
+                "peak_source": peaks["source"] + " hbm copy (of measured)"}
+    if wonly:
+        wfl = sum(2 * T * L["proj"].d_in * L["proj"].d_out for L in layers)
+        ach = wfl / (prod_ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "traffic": traffic, "kernel": kernel,
+                "peak_source": f"{peaks['source']} bf16 burst (of measured)"}
+    ints = sum(roofline.int_ops(T, L["proj"].d_in, L["proj"].d_out) for L in layers)
+    ach = ints / (prod_ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": int8["peak"], "unit": "TOP/s", "frac": ach / int8["peak"],
+            "traffic": traffic, "kernel": kernel, "peak_source": int8["source"]}
+
+
+def per_projection(cfg, layers, T, stage_ms):
+    from quantized_gemm_moe_b200 import roofline
+    wonly = cfg.a_bits == 16
+    out = []
+    for p_i, L in enumerate(layers):
+        ms = stage_ms[:, p_i, :].mean(axis=0)
+        K, N = L["proj"].d_in, L["proj"].d_out
+        tot = ms.sum()
+        out.append({
+            "proj": L["proj"].name, "K": K, "N": N, "ms": float(tot),
+            "stage_ms": {"project": float(ms[0]), "route_quant": float(ms[1]), "product": float(ms[2])},
+            "product_tops": (roofline.int_ops(T, K, N) / (ms[2] / 1e3) / 1e12) if not wonly else None,
+            "product_gbs": roofline.layer_bytes(T, K, N, cfg.group, cfg.w_bits, cfg.rank_shared, cfg.n_routed,
+                                                cfg.rank_routed, 1 if not wonly else 2, 2) / (ms[2] / 1e3) / 1e9,
+            "layer_tokens_per_s": T / (tot / 1e3),
+        })
+    return out
+
+
+def oracle_baseline(cfg, T, seconds):
+    """The oracle timed on the host cores on a bounded token sample of the workload."""
+    cores = os.cpu_count() or 1
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    run, n_avail = oracle_layer_set(cfg, min(T, ORACLE_PREP_TOKENS))
+    tok, secs, sample = sized_oracle_sample(run, n_avail, seconds)
+    return {"value": tok / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{tok} token passes through every projection of the layer set in {secs:.1f} s "
+                      f"(the first {sample} tokens of the workload; tokens are independent)"}
+
+
+# Decode-shaped 72B layers (gate/up/down at T <= 16), measured beside the headline workload:
+# each variant's layers are built once and timed at every T of the list.
+DECODE_SETS = (("decode72b_w4a8", (16, 1)), ("decode72b_w3a16", (16, 1)))
+
+
 def run_ours(args, workload):
     import torch
     import quantized_gemm_moe_b200 as qe
@@ -391,75 +556,26 @@ def run_ours(args, workload):
     routed_channels = WORKLOADS[workload][3] if len(WORKLOADS[workload]) > 3 else 0
     cfg = qi.CONFIGS[cfg_name]
     T = args.tokens or t_over or cfg.T
-    layers = build_layers(cfg, T, rank, dev, routed_channels)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     wonly = cfg.a_bits == 16
     stages = (qe.QE_STAGE_PROJECT, qe.QE_STAGE_ROUTE | qe.QE_STAGE_QUANT, qe.QE_STAGE_PRODUCT)
+    peaks = load_peaks()
 
-    def step_plain():
-        for L in layers:
-            qe.linear_forward(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"])
+    # int8 denominator: the library GEMM measured here, or 2x the bf16 burst (the nominal
+    # int8:bf16 ratio), whichever is larger (the smaller fraction)
+    int8_meas = measure_int8_peak(dev) if not wonly else None
+    twice_bf16 = 2.0 * peaks["bf16_tflops"]
+    if int8_meas is not None and int8_meas >= twice_bf16:
+        int8 = {"peak": int8_meas, "source": f"measured torch._int_mm 8192^3 on this GPU: {int8_meas:.0f} TOP/s "
+                                             f"(2x the bf16 burst: {twice_bf16:.0f})"}
+    else:
+        meas = "unavailable" if int8_meas is None else f"{int8_meas:.0f} TOP/s"
+        int8 = {"peak": twice_bf16, "source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TF/s x 2 "
+                                              f"(int8:bf16 nominal ratio); torch._int_mm 8192^3 measured {meas}"}
 
-    for _ in range(max(args.warmup, 0)):
-        flush.zero_()
-        step_plain()
-    torch.cuda.synchronize()
-    assert qe.device_error() == 0, "a device wait ran out during warm-up"
-
-    # One step = every projection through the public forward call, captured once into a CUDA
-    # graph with one timing event at each end. The hot path is a chain of short kernels, so the
-    # graph removes host launch gaps from the device timeline. Each replay is timed by its own
-    # events, read back after the replay, outside the timed interval.
-    cap = torch.cuda.Stream()
-    ev0 = torch.cuda.Event(enable_timing=True, external=True)
-    ev1 = torch.cuda.Event(enable_timing=True, external=True)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=cap):
-        ev0.record()
-        step_plain()
-        ev1.record()
-    # A second graph splits each forward into its three stages with events between them; its
-    # replays (after the timed region) give the per-stage breakdown and the product kernels' time.
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)] for _ in layers]
-    sgraph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(sgraph, stream=cap):
-        for L, e in zip(layers, evs):
-            e[0].record()
-            for i, sm in enumerate(stages):
-                qe.linear_forward_stages(L["desc"], L["layer"].weights, L["X"], L["Y"], L["ws"], sm)
-                e[i + 1].record()
-    for _ in range(2):
-        graph.replay()
-        sgraph.replay()
-    torch.cuda.synchronize()
-
-    n_proj = len(layers)
-    step_ms = np.zeros(args.steps)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for s_i in range(args.steps):
-            flush.zero_()
-            graph.replay()
-            torch.cuda.synchronize()
-            step_ms[s_i] = ev0.elapsed_time(ev1)
-    if pg:
-        pg.barrier()
-    n_diag = max(3, min(args.steps, 10))
-    stage_ms = np.zeros((n_diag, n_proj, len(stages)))
-    for s_i in range(n_diag):
-        flush.zero_()
-        sgraph.replay()
-        torch.cuda.synchronize()
-        for p_i, e in enumerate(evs):
-            for k in range(len(stages)):
-                stage_ms[s_i, p_i, k] = e[k].elapsed_time(e[k + 1])
-    err = qe.device_error()
-    assert err == 0, f"device wait ran out (code {err:#x})"
-    del graph, sgraph
-
+    layers = build_layers(cfg, T, rank, dev, routed_channels)
+    step_ms, stage_ms, clocks = time_layer_set(qe, layers, T, args, flush, pg, stages)
     total_ms = max_over_ranks(float(step_ms.sum()), pg, dev)
     ms_per_step = total_ms / args.steps
     value = world * T * args.steps / (total_ms / 1e3)
@@ -473,45 +589,11 @@ def run_ours(args, workload):
     xb = 2 if cfg.x_dtype == "bf16" else 4
     nbytes = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
                                       cfg.n_routed, cfg.rank_routed, xb, 2) for L in layers)
-    peaks = load_peaks()
     prod_ms = stage_ms[:, :, 2].sum(axis=1).mean()  # the product kernels of one step
-    int8_peak = 2.0 * peaks["bf16_tflops"]           # int8 dense = 2x bf16 dense (nominal ratio)
-    decode = T <= 16
     kernel_file = "quantized_gemm_moe_b200/csrc/k_wgemm.cu" if wonly else "quantized_gemm_moe_b200/csrc/k_gemm.cu"
-    prod_bytes = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
-                                          cfg.n_routed, cfg.rank_routed, 1 if not wonly else 2, 2) for L in layers)
     traffic = read_traffic(kernel_file, ("wgemm_" if wonly else "qgemm_") + workload) if not args.tokens else None
-    if decode:
-        ach = prod_bytes / (prod_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "wgemm" if wonly else "qgemm", "peak_source": peaks["source"] + " hbm copy"}
-    elif wonly:
-        # weight-only prefill: the product is a bf16 tensor-core GEMM (2 T K N flops per projection)
-        wfl = sum(2 * T * L["proj"].d_in * L["proj"].d_out for L in layers)
-        ach = wfl / (prod_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"], "traffic": traffic, "kernel": "wgemm",
-                "peak_source": f"{peaks['source']} bf16 burst"}
-    else:
-        ach = ints / (prod_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": int8_peak, "unit": "TOP/s",
-                "frac": ach / int8_peak, "traffic": traffic, "kernel": "qgemm",
-                "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TF/s x 2 (int8:bf16 nominal ratio)"}
-
-    per_proj = []
-    for p_i, L in enumerate(layers):
-        ms = stage_ms[:, p_i, :].mean(axis=0)
-        K, N = L["proj"].d_in, L["proj"].d_out
-        tot = ms.sum()
-        per_proj.append({
-            "proj": L["proj"].name, "K": K, "N": N, "ms": float(tot),
-            "stage_ms": {"project": float(ms[0]), "route_quant": float(ms[1]), "product": float(ms[2])},
-            "product_tops": (roofline.int_ops(T, K, N) / (ms[2] / 1e3) / 1e12) if not wonly else None,
-            "product_gbs": roofline.layer_bytes(T, K, N, cfg.group, cfg.w_bits, cfg.rank_shared, cfg.n_routed,
-                                                cfg.rank_routed, 1 if not wonly else 2, 2) / (ms[2] / 1e3) / 1e9,
-            "layer_tokens_per_s": T / (tot / 1e3),
-        })
+    roof = product_roofline(cfg, layers, T, prod_ms, peaks, int8, traffic)
+    per_proj = per_projection(cfg, layers, T, stage_ms)
 
     # end to end through the public call with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -542,40 +624,70 @@ def run_ours(args, workload):
         e_ms = max_over_ranks(e_ms, pg, dev)
         e2e = {"value": world * T * args.steps / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "mode": args.e2e_mode}
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cores = os.cpu_count() or 1
-        os.environ.setdefault("OMP_NUM_THREADS", str(cores))
-        run, n_avail = oracle_layer_set(cfg, min(T, ORACLE_PREP_TOKENS))
-        tok, secs, sample = sized_oracle_sample(run, n_avail, args.cpu_seconds)
-        cpu = {"value": tok / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{tok} token passes through every projection of the layer set in {secs:.1f} s "
-                         f"(the first {sample} tokens of the workload; tokens are independent)"}
+        del xh, yh
 
     launches = sum(qe.linear_kernel_launches(L["desc"], T, qe.QE_BF16 if cfg.x_dtype == "bf16" else qe.QE_F32)
                    for L in layers) * args.steps
+    for L in layers:
+        L.clear()
+    del layers
+    torch.cuda.empty_cache()
+
+    # decode-shaped layers (HBM bound), each at its own roofline
+    decode = None
+    if not args.no_decode and args.tokens == 0 and workload == DEFAULT_WORKLOAD:
+        decode = []
+        for dname, Ts in DECODE_SETS:
+            dcfg = qi.CONFIGS[dname]
+            dl = build_layers(dcfg, max(Ts), rank, dev)
+            dcpu = None
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                dcpu = oracle_baseline(dcfg, max(Ts), args.cpu_seconds / 2)
+            for dT in Ts:
+                s_ms, st_ms, dclk = time_layer_set(qe, dl, dT, args, flush, pg, stages)
+                tot = max_over_ranks(float(s_ms.sum()), pg, dev)
+                pm = st_ms[:, :, 2].sum(axis=1).mean()
+                dfile = "quantized_gemm_moe_b200/csrc/" + ("k_wgemm.cu" if dcfg.a_bits == 16 else "k_gemm.cu")
+                dtraffic = read_traffic(dfile, ("wgemm_" if dcfg.a_bits == 16 else "qgemm_") + f"{dname}_t{dT}")
+                decode.append({
+                    "workload": dname, "T": dT, "description": f"72B decode gate/up/down, T={dT}, "
+                                                               f"{'W3A16' if dcfg.w_bits == 3 else 'W4A8'} g128",
+                    "value": world * dT * args.steps / (tot / 1e3), "unit": "tokens/s",
+                    "ms_per_step": tot / args.steps,
+                    "roofline": product_roofline(dcfg, dl, dT, pm, peaks, int8, dtraffic),
+                    "per_projection": per_projection(dcfg, dl, dT, st_ms),
+                    "cpu_baseline": dcpu, "clocks": dclk,
+                })
+            for L in dl:
+                L.clear()
+            del dl
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(cfg, T, args.cpu_seconds)
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if wonly else "int8", "data": "synthetic",
         "config": {"workload": workload, "description": desc_txt, "T_per_gpu": T,
-                   "projections": [[L["proj"].name, L["proj"].d_in, L["proj"].d_out] for L in layers],
+                   "projections": [[p.name, p.d_in, p.d_out] for p in cfg.projections],
                    "l2": "flushed between steps (256 MB write outside the per-step events)",
                    "parallelism": f"replicas x{world}"},
         "effective_tops": (ints + fl) / (ms_per_step / 1e3) / 1e12 * world,
         "hbm_gbs_algorithmic": nbytes / (ms_per_step / 1e3) / 1e9,
         "roofline": roof,
+        "int8_peak": {"torch_int_mm_tops": int8_meas, "twice_bf16_burst_tops": twice_bf16, "used": int8["peak"]},
         "per_projection": per_proj,
+        "decode": decode,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "gpu_launches": launches,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for L in layers:
-        L.clear()
     if pg:
         pg.barrier()
         pg.destroy_process_group()
@@ -758,8 +870,30 @@ def run_calib(args, workload):
     return 0
 
 
-def main():
-    args = parse_args()
+def free_port() -> int:
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def spawn_ranks(args, argv) -> int:
+    """--gpus N > 1 outside torchrun: run this script again under torch.distributed.run with N
+    ranks on this node (rendezvous on 127.0.0.1). Returns the launcher's exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = parse_args(argv)
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return spawn_ranks(args, argv)
+    if "WORLD_SIZE" in os.environ and int(os.environ["WORLD_SIZE"]) != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {os.environ['WORLD_SIZE']} ranks")
     if args.workload in CALIB_WORKLOADS:
         return run_calib(args, args.workload)
     if args.impl == "reference":

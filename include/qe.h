@@ -22,9 +22,11 @@
  *
  * Conventions for every entry point
  * - Pointers marked (device) are CUDA device pointers. The caller allocates
- *   and owns all of them. The library allocates no device memory and keeps
- *   no device state except one error word (qe_device_error). It never frees
- *   anything it did not allocate.
+ *   and owns all of them. The library allocates no device memory at run
+ *   time and never frees anything it did not allocate. Its own device state
+ *   is static, on every device that loads the library: one error word
+ *   (qe_device_error) and the fixed scratch array of
+ *   qe_linear_forward_noalloc (QE_NOALLOC_WORKSPACE_BYTES).
  * - Matrices are row-major. W is [d_out, d_in] (the nn.Linear convention),
  *   X is [T, d_in] and Y is [T, d_out].
  * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
@@ -140,13 +142,17 @@ QE_API size_t qe_linear_workspace_bytes(const qe_layer_desc* desc, int32_t T);
  *   w_scale  (device) out, fp32 [d_in/group][d_out]
  *   w_mean   (device) out, fp32 [d_in], may be NULL
  *   w_colmax (device) out, fp32 [d_in] = max_o |W[o][k]|, may be NULL
+ *   s_inv    (device) out, fp32 [d_in] = fl32(1/s[k]) (one IEEE division per
+ *            channel): the stored factor qe_layer_weights.s_inv that the
+ *            activations are multiplied by. May be NULL.
  * For each (o, group j): scale = fl32(max_k |fl32(W[o][k]*s[k])| / qmax) and
  * code = clamp(rint(fl32(fl32(W*s)/scale)), -qmax, qmax), with ties to
  * even. A zero scale gives zero codes. qmax = 7 (W4) or 3 (W3). w_mean
  * is summed in fp64 and rounded once.
  */
 QE_API qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, qe_dtype w_dtype, const float* s,
-                              void* w_packed, float* w_scale, float* w_mean, float* w_colmax, void* stream);
+                              void* w_packed, float* w_scale, float* w_mean, float* w_colmax, float* s_inv,
+                              void* stream);
 
 /*
  * Packs the shared expert, the routed experts and the router into the
@@ -265,11 +271,14 @@ QE_API int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, q
  *   adapter_gemm_tile    its columns per CTA
  *   adapter_gemm_splits  its K splits (partial slots; doubled for fp32 inputs)
  *   weight_only          1 for a_bits = 16 (the weight-only product)
+ *   workspace_bytes      the scratch this call needs for this x_dtype (qe_linear_workspace_bytes
+ *                        is the larger of the fp32 and bf16 needs)
  * Returns QE_ERR_INVALID_ARG for a null pointer or T < 1, and check errors of desc.
  */
 typedef struct {
   int32_t product_tile_tokens, product_k_splits, adapter_atoms, adapter_gemm_width, adapter_gemm_tile,
       adapter_gemm_splits, weight_only;
+  int64_t workspace_bytes;
 } qe_linear_plan_info;
 QE_API qe_status qe_linear_plan(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype, qe_linear_plan_info* out);
 
@@ -295,7 +304,8 @@ QE_API qe_status qe_linear_plan(const qe_layer_desc* desc, int32_t T, qe_dtype x
  * - The first call on a device looks up the array's device address for that
  *   device, then synchronizes the device once, because loading the array
  *   initializes it asynchronously. Make that first call before any stream
- *   capture.
+ *   capture. The lookup is repeated (with its synchronization) when the
+ *   device's context has changed since, e.g. after cudaDeviceReset.
  * - All calls share the one array and it keeps the last call's contents.
  *   Calls whose kernels overlap on the GPU (different streams, or
  *   different host threads, without ordering) race on it. Order them.

@@ -12,6 +12,7 @@ invariant checks.
 
 Parity status per function (pins live in tests/test_oracle_pins.py):
   quantize_weights, act_quant  pinned: grid round-trip, per-row RTN at g=K, hand cases
+  smoothing_inverse            pinned: nearest fp32 to 1/s (neighbour check in fp64), powers of two exact
   route, bucket                pinned: brute-force argmin / stable sort, permutation
   group_acc                    pinned: bound |acc| <= g*qmax_a*qmax_w, numpy int64
   qe_forward                   pinned: zero adapters = literal dequant matmul,
@@ -83,6 +84,14 @@ def quantize_weights(W, s, group: int, bits: int):
     _check(lib().oracle_quantize_weights(_p(W), _p(s), N, K, group, bits, _p(codes), _p(scales),
                                          _p(w_mean), _p(w_colmax)), "quantize_weights")
     return codes, scales, w_mean, w_colmax
+
+
+def smoothing_inverse(s) -> np.ndarray:
+    """The stored smoothing factor of the activations ([DR] \u00a7Method, Shared Expert: activations are
+    divided by s): s_inv[k] = fl32(1/s[k]), one IEEE fp32 division per channel (numpy float32
+    division is correctly rounded)."""
+    s = _f32(s)
+    return (np.float32(1.0) / s).astype(np.float32)
 
 
 def act_quant(X, s_inv, bits: int):

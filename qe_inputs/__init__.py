@@ -267,12 +267,11 @@ def layer_inputs(cfg: LayerConfig, proj: Projection, T: int | None = None, proj_
     s = np.ones(K, np.float64)
     s[ok] = np.sqrt(amax_x[ok] / amax_w[ok])
     s = s.astype(np.float32)
-    s_inv = (np.float32(1.0) / s).astype(np.float32)
     rs, nr, rr = cfg.rank_shared, cfg.n_routed, cfg.rank_routed
     A_s = to_bf16(gaussian((K, rs), adapter_std, 3000 + sb))
     B_s = to_bf16(gaussian((rs, N), adapter_std, 3100 + sb))
     A_r = to_bf16(gaussian((nr, K, rr), adapter_std, 3200 + sb))
     B_r = to_bf16(gaussian((nr, rr, N), adapter_std, 3300 + sb))
     G = to_bf16(gaussian((K, nr), 0.02, 4000 + sb))
-    return dict(X=x_store, W=w_store, s=s, s_inv=s_inv, A_s=A_s, B_s=B_s, A_r=A_r, B_r=B_r, G=G,
+    return dict(X=x_store, W=w_store, s=s, A_s=A_s, B_s=B_s, A_r=A_r, B_r=B_r, G=G,
                 T=T, K=K, N=N)

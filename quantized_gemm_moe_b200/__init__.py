@@ -55,7 +55,7 @@ class LayerDesc(ctypes.Structure):
 class LinearPlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("product_tile_tokens", "product_k_splits", "adapter_atoms",
                                               "adapter_gemm_width", "adapter_gemm_tile", "adapter_gemm_splits",
-                                              "weight_only")]
+                                              "weight_only")] + [("workspace_bytes", ctypes.c_int64)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -80,7 +80,7 @@ def load() -> ctypes.CDLL:
         "qe_packed_weight_bytes": ([D], S),
         "qe_adapter_packed_bytes": ([D], S),
         "qe_linear_workspace_bytes": ([D, I], S),
-        "qe_quantize_weights": ([D, P, I, P, P, P, P, P, P], I),
+        "qe_quantize_weights": ([D, P, I, P, P, P, P, P, P, P], I),
         "qe_pack_adapters": ([D, P, P, P, P, P, P, P], I),
         "qe_pack_adapters_sparse": ([D, P, P, P, P, P, P, P, P], I),
         "qe_topk_importance": ([P, I, P, I, I, I, P, P, I, P], I),
@@ -164,10 +164,10 @@ def linear_workspace_bytes(desc: LayerDesc, T: int) -> int:
     return int(load().qe_linear_workspace_bytes(ctypes.byref(desc), T))
 
 
-def quantize_weights(desc, W, s, w_packed, w_scale, w_mean=None, w_colmax=None, stream=None):
-    _need_cuda(W, s, w_packed, w_scale, w_mean, w_colmax)
+def quantize_weights(desc, W, s, w_packed, w_scale, w_mean=None, w_colmax=None, s_inv=None, stream=None):
+    _need_cuda(W, s, w_packed, w_scale, w_mean, w_colmax, s_inv)
     _check(load().qe_quantize_weights(ctypes.byref(desc), _ptr(W), _dtype(W), _ptr(s), _ptr(w_packed),
-                                      _ptr(w_scale), _ptr(w_mean), _ptr(w_colmax), _stream(stream)),
+                                      _ptr(w_scale), _ptr(w_mean), _ptr(w_colmax), _ptr(s_inv), _stream(stream)),
            "qe_quantize_weights")
 
 
@@ -308,8 +308,9 @@ class QELayer:
         """W [d_out, d_in] (fp32/bf16), s [d_in] fp32, adapters/G bf16 in their natural layouts (CUDA tensors).
 
         s_inv (fp32 [d_in]) is the stored reciprocal smoothing factor the activations are
-        multiplied by. When omitted, it is fl32(1/s). With desc.routed_channels > 0, A_r is
-        bf16 [N_r][k_c][r_r] over `channels` (int32 [N_r][k_c]).
+        multiplied by. When omitted, the library computes it (qe_quantize_weights writes
+        fl32(1/s)). With desc.routed_channels > 0, A_r is bf16 [N_r][k_c][r_r] over `channels`
+        (int32 [N_r][k_c]).
         """
         import torch
         dev = W.device
@@ -318,14 +319,15 @@ class QELayer:
         w_scale = torch.empty((K // desc.group, N), dtype=torch.float32, device=dev)
         w_mean = torch.empty(K, dtype=torch.float32, device=dev)
         w_colmax = torch.empty(K, dtype=torch.float32, device=dev)
-        quantize_weights(desc, W, s, w_packed, w_scale, w_mean, w_colmax, stream)
+        s_inv_out = torch.empty(K, dtype=torch.float32, device=dev) if s_inv is None else None
+        quantize_weights(desc, W, s, w_packed, w_scale, w_mean, w_colmax, s_inv_out, stream)
         adapters = torch.empty(adapter_packed_bytes(desc), dtype=torch.uint8, device=dev)
         if desc.routed_channels > 0:
             pack_adapters_sparse(desc, A_s, B_s, channels, A_r, B_r, G, adapters, stream)
         else:
             pack_adapters(desc, A_s, B_s, A_r, B_r, G, adapters, stream)
         if s_inv is None:
-            s_inv = (torch.ones_like(s) / s).contiguous()
+            s_inv = s_inv_out
         return cls(desc, w_packed, w_scale, s_inv.contiguous(), adapters, w_mean, w_colmax)
 
     def workspace(self, T: int):

@@ -110,21 +110,6 @@ __device__ __forceinline__ uint64_t pack2(float x) {
   return r;
 }
 
-// Which TMEM buffer the epilogue drains next. The two MMA issuers take alternate stages, and
-// issuer q cycles through its own buffers q, q+2, ..., q+2(kOwn-1). The epilogue tracks the
-// issuers' progress in one word: bit 0 = parity of the current unit's first stage, bits 1..3 /
-// 4..6 = groups issued so far by issuer 0 / 1, mod 8 (enough for kOwn <= 4). Returns the
-// buffer and sets `use_parity` to the parity of that buffer's use.
-template <int kOwn>
-__device__ __forceinline__ int epi_next_buffer(uint32_t& st, int iq, uint32_t& use_parity) {
-  static_assert(kOwn >= 1 && kOwn <= 4, "buffer state holds counts mod 8");
-  const int sh = 1 + 3 * iq;
-  const uint32_t oc = (st >> sh) & 7u;
-  st = (st & ~(7u << sh)) | (((oc + 1u) & 7u) << sh);
-  use_parity = (oc / kOwn) & 1u;
-  return iq + 2 * static_cast<int>(oc % kOwn);
-}
-
 // One unit of work: a 128-row output tile, a BN-position token tile and a K split.
 struct Unit {
   int nt, p0, split, kb_begin, nkb, n_ad, g_begin, n_groups;
@@ -328,6 +313,7 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
       }
+      drain_ring(full, NS, it);
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
@@ -705,7 +691,8 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int it = 0; it < nk; ++it) {
+      int it = 0;
+      for (; it < nk; ++it) {
         const int s = it % NS;
         if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) break;
         uint8_t* sa_ = smem + s * C::kStage;
@@ -714,6 +701,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_2d(sa_, &tm_x, kx, m0, &full[s]);
         tma_load_2d(sa_ + C::kA, &tm_acat, kx, c0, &full[s]);
       }
+      drain_ring(full, NS, it);
     }
   } else if (warp == 1) {
     if (lane == 0) {

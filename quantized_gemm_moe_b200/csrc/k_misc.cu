@@ -636,7 +636,7 @@ __global__ void __launch_bounds__(kTSThreads, 1) k_topk_stream(const uint16_t* _
     // a wait gave up: let every copy still in flight land before the CTA exits
     for (int r = 0; r < kTSRowStages; ++r)
       if (issued[r] > consumed[r])
-        mbar_wait_for(&row_full[r], static_cast<uint32_t>(consumed[r] & 1), nullptr, 0, 10000000ull);
+        mbar_wait_for(&row_full[r], static_cast<uint32_t>(consumed[r] & 1), nullptr, 0, kDrainLimitNs);
   }
 }
 

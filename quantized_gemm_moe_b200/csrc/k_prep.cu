@@ -4,22 +4,48 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "qe_internal.h"
 #include "qe_ptx.cuh"
 
 namespace qe {
 
-// The library's only device state: the error word that bounded waits write.
+// Library-owned device state, on every device that loads this module: the error word that
+// bounded waits write (here), and the fixed scratch array of qe_linear_forward_noalloc
+// (QE_NOALLOC_WORKSPACE_BYTES, in qe_api.cu).
 __device__ int g_device_error = 0;
 
+void* current_context() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  static GetCurrent fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<GetCurrent>(nullptr);
+    return reinterpret_cast<GetCurrent>(f);
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// The error word's device address, looked up once per device and context (a replaced context,
+// e.g. after cudaDeviceReset, loads the module again at a new address).
 int* device_error_ptr() {
+  static std::mutex mu;
   static int* cached[64] = {nullptr};
+  static void* ctx_of[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cached[dev]) {
+  std::lock_guard<std::mutex> lock(mu);
+  void* ctx = current_context();
+  if (!cached[dev] || ctx != ctx_of[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
     cached[dev] = static_cast<int*>(p);
+    ctx_of[dev] = current_context();
   }
   return cached[dev];
 }
@@ -404,6 +430,13 @@ __global__ void __launch_bounds__(64) k_colstats(const void* __restrict__ W, int
   }
   if (w_mean) w_mean[k] = static_cast<float>(sum / static_cast<double>(N));
   if (w_colmax) w_colmax[k] = mx;
+}
+
+// The stored smoothing factor of the activations: s_inv[k] = fl32(1/s[k]), one correctly rounded
+// IEEE division per channel (the activations are divided by s, Method, "Shared Expert").
+__global__ void k_recip(const float* __restrict__ s, int K, float* __restrict__ s_inv) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k < K) s_inv[k] = __fdiv_rn(1.0f, s[k]);
 }
 
 // Inverse of the packing above (diagnostics).
@@ -1013,6 +1046,11 @@ cudaError_t launch_colstats(const void* W, bool w_bf16, int N, int K, float* w_m
   const unsigned grid = static_cast<unsigned>(ceil_div(K, 64));
   if (w_bf16) k_colstats<true><<<grid, 64, 0, st>>>(W, N, K, w_mean, w_colmax);
   else k_colstats<false><<<grid, 64, 0, st>>>(W, N, K, w_mean, w_colmax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_recip(const float* s, int K, float* s_inv, cudaStream_t st) {
+  k_recip<<<static_cast<unsigned>(ceil_div(K, 256)), 256, 0, st>>>(s, K, s_inv);
   return cudaGetLastError();
 }
 

@@ -61,21 +61,6 @@ struct WCfg {
   static_assert(kSmem <= 232448, "shared memory");
 };
 
-// Which TMEM buffer the epilogue drains next. The two MMA issuers take alternate stages, and
-// issuer q cycles through its own buffers q, q+2, ..., q+2(kOwn-1). The epilogue tracks the
-// issuers' progress in one word: bit 0 = parity of the current unit's first stage, bits 1..3 /
-// 4..6 = groups issued so far by issuer 0 / 1, mod 8 (enough for kOwn <= 4). Returns the
-// buffer and sets `use_parity` to the parity of that buffer's use.
-template <int kOwn>
-__device__ __forceinline__ int epi_next_buffer(uint32_t& st, int iq, uint32_t& use_parity) {
-  static_assert(kOwn >= 1 && kOwn <= 4, "buffer state holds counts mod 8");
-  const int sh = 1 + 3 * iq;
-  const uint32_t oc = (st >> sh) & 7u;
-  st = (st & ~(7u << sh)) | (((oc + 1u) & 7u) << sh);
-  use_parity = (oc / kOwn) & 1u;
-  return iq + 2 * static_cast<int>(oc % kOwn);
-}
-
 struct WUnit {
   int nt, p0, split, kb_begin, nkb, n_ad, g_begin, n_groups;
 };
@@ -146,14 +131,15 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + C::kOut);
   uint64_t* wfull = bars;             // [NW] packed block landed
   uint64_t* wempty = wfull + NW;      // [NW] unpack warps read it (one arrival per unpack warp)
-  uint64_t* afull = wempty + NW;      // [NA] A unpacked (one per unpack warp) + B landed (1 + bytes)
+  uint64_t* afull = wempty + NW;      // [NA] A unpacked (one arrival per unpack warp)
   uint64_t* aempty = afull + NA;      // [NA] MMAs done with the slot
   uint64_t* accf = aempty + NA;       // [NB] group sum ready
   uint64_t* acce = accf + NB;         // [NB] group sum read (every epilogue warp)
   uint64_t* done = acce + NB;
   uint64_t* adone = done + 1;         // adapter block: its issuer waited for all of its slots
   uint64_t* aack = adone + 1;         // adapter block: the other issuer saw adone
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aack + 1);
+  uint64_t* bfull = aack + 1;         // [NA] the slot's TMA tiles landed (1 + bytes)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bfull + NA);
   float* su_s = reinterpret_cast<float*>(bars + 64);
   int32_t* perm_s = reinterpret_cast<int32_t*>(su_s + BN);
 
@@ -169,7 +155,8 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&wempty[s], C::kUnpackWarps);
     }
     for (int s = 0; s < NA; ++s) {
-      mbar_init(&afull[s], C::kUnpackWarps + 1);
+      mbar_init(&afull[s], C::kUnpackWarps);
+      mbar_init(&bfull[s], 1);
       mbar_init(&aempty[s], 1);
     }
     for (int b = 0; b < NB; ++b) {
@@ -216,6 +203,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (!ok) break;
       }
+      drain_ring(wfull, NW, jw);
     }
   } else if (warp == 3) {
     // ------------------------------------------------------------ activation / adapter tiles
@@ -234,17 +222,18 @@ __global__ void __launch_bounds__(512, 1)
           uint8_t* sb_ = sa_ + C::kA;
           if (i < w.nkb) {
             const int k0 = (w.kb_begin + i) * kTileK;
-            mbar_arrive_expect_tx(&afull[s], C::kB);
-            tma_load_2d(sb_, &tm_act, k0, w.p0, &afull[s]);
-            tma_load_2d(sb_ + C::kAtomB, &tm_act, k0 + 64, w.p0, &afull[s]);
+            mbar_arrive_expect_tx(&bfull[s], C::kB);
+            tma_load_2d(sb_, &tm_act, k0, w.p0, &bfull[s]);
+            tma_load_2d(sb_ + C::kAtomB, &tm_act, k0 + 64, w.p0, &bfull[s]);
           } else {
             const int at = i - w.nkb;
-            mbar_arrive_expect_tx(&afull[s], C::kAtomA + C::kAtomB);
-            tma_load_2d(sa_, &tm_bcat, at * kAdapterAtom, w.nt * kTileN, &afull[s]);
-            tma_load_2d(sb_, &tm_ucat, at * kAdapterAtom, w.p0, &afull[s]);
+            mbar_arrive_expect_tx(&bfull[s], C::kAtomA + C::kAtomB);
+            tma_load_2d(sa_, &tm_bcat, at * kAdapterAtom, w.nt * kTileN, &bfull[s]);
+            tma_load_2d(sb_, &tm_ucat, at * kAdapterAtom, w.p0, &bfull[s]);
           }
         }
       }
+      drain_ring(bfull, NA, it);
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
@@ -274,7 +263,8 @@ __global__ void __launch_bounds__(512, 1)
             const int kb = w.kb_begin + i;
             const int ng = max(0, min(gpb, w.g_begin + w.n_groups - kb * gpb));
             if ((it & 1) != qi) continue;
-            if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
+            if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA) ||
+                !mbar_wait(&bfull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
               ok = false;
               break;
             }
@@ -316,7 +306,8 @@ __global__ void __launch_bounds__(512, 1)
               continue;
             }
             const int b = qi + 2 * static_cast<int>(own % kOwn);
-            if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
+            if (!mbar_wait(&afull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA) ||
+                !mbar_wait(&bfull[s], (it / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
               ok = false;
               break;
             }

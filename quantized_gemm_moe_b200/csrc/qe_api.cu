@@ -153,9 +153,11 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const void* X, qe_dtype xd, int32_t T,
-                       void* Y, qe_dtype yd, void* ws, size_t ws_bytes, int32_t* dbg_acc, int32_t* dbg_expert,
-                       int32_t* dbg_perm, float* dbg_sa, int32_t stages, cudaStream_t st) {
+// Every check of a forward call that does not depend on the workspace, in the order the
+// header documents them. Both forward entry points run it before they size any scratch.
+// T == 0 passes (the caller returns QE_OK without launching anything).
+qe_status check_forward_args(const qe_layer_desc* d, const qe_layer_weights* w, const void* X, qe_dtype xd,
+                             int32_t T, const void* Y, qe_dtype yd) {
   qe_status s = check_desc(d);
   if (s != QE_OK) return s;
   if (!w || !w->w_packed || !w->w_scale || !w->s_inv || !w->adapters) return QE_ERR_INVALID_ARG;
@@ -168,6 +170,14 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
   if (!aligned16(X) || !aligned16(Y) || !aligned16(w->w_packed) || !aligned16(w->w_scale) ||
       !aligned16(w->s_inv) || !aligned16(w->adapters))
     return QE_ERR_ALIGNMENT;
+  return QE_OK;
+}
+
+qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const void* X, qe_dtype xd, int32_t T,
+                       void* Y, qe_dtype yd, void* ws, size_t ws_bytes, int32_t* dbg_acc, int32_t* dbg_expert,
+                       int32_t* dbg_perm, float* dbg_sa, int32_t stages, cudaStream_t st) {
+  qe_status s = check_forward_args(d, w, X, xd, T, Y, yd);
+  if (s != QE_OK || T == 0) return s;
   const bool x_bf16 = xd == QE_BF16;
   const Plan p = make_plan(d, T, x_bf16);
   if (!ws || ws_bytes < p.bytes) return QE_ERR_WORKSPACE;
@@ -323,18 +333,21 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
 // every byte it reads before reading it, so nothing needs clearing).
 static __device__ __align__(256) uint8_t g_static_scratch[QE_NOALLOC_WORKSPACE_BYTES];
 
-// Device address of g_static_scratch for the current device, looked up once per device.
-// Host code must not use the array's name as an address: on the host it is only a
-// stand-in symbol, not device memory.
+// Device address of g_static_scratch for the current device. Host code must not use the
+// array's name as an address: on the host it is only a stand-in symbol, not device memory.
+// The address is looked up once per device and context: if the device's context is replaced
+// (after cudaDeviceReset, the module is loaded again), the next call looks it up again.
 qe_status static_scratch(void** out) {
   static std::mutex mu;
   static void* addr[64] = {nullptr};
+  static void* ctx_of[64] = {nullptr};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return QE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  void* ctx = current_context();
+  if (!addr[dev] || ctx != ctx_of[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
@@ -343,6 +356,7 @@ qe_status static_scratch(void** out) {
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize(static scratch set-up)");
     addr[dev] = p;
+    ctx_of[dev] = current_context();
   }
   *out = addr[dev];
   return QE_OK;
@@ -372,13 +386,14 @@ size_t qe_linear_workspace_bytes(const qe_layer_desc* desc, int32_t T) {
 }
 
 qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, qe_dtype w_dtype, const float* s,
-                              void* w_packed, float* w_scale, float* w_mean, float* w_colmax, void* stream) {
+                              void* w_packed, float* w_scale, float* w_mean, float* w_colmax, float* s_inv,
+                              void* stream) {
   qe_status st = check_desc(desc);
   if (st != QE_OK) return st;
   if (!W || !s || !w_packed || !w_scale) return QE_ERR_INVALID_ARG;
   if (w_dtype != QE_F32 && w_dtype != QE_BF16) return QE_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(s) || !aligned16(w_packed) || !aligned16(w_scale) ||
-      (w_mean && !aligned16(w_mean)) || (w_colmax && !aligned16(w_colmax)))
+      (w_mean && !aligned16(w_mean)) || (w_colmax && !aligned16(w_colmax)) || (s_inv && !aligned16(s_inv)))
     return QE_ERR_ALIGNMENT;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   QE_CUDA(launch_quantize_weights(W, w_dtype == QE_BF16, s, desc->d_out, desc->d_in, desc->group, desc->w_bits,
@@ -386,6 +401,7 @@ qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, qe_dtype
           "quantize_weights");
   if (w_mean || w_colmax)
     QE_CUDA(launch_colstats(W, w_dtype == QE_BF16, desc->d_out, desc->d_in, w_mean, w_colmax, cs), "colstats");
+  if (s_inv) QE_CUDA(launch_recip(s, desc->d_in, s_inv, cs), "recip");
   return QE_OK;
 }
 
@@ -474,6 +490,7 @@ qe_status qe_linear_plan(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype,
   out->adapter_gemm_tile = p.up.nu;
   out->adapter_gemm_splits = p.uslots;
   out->weight_only = desc->a_bits == 16 ? 1 : 0;
+  out->workspace_bytes = static_cast<int64_t>(p.bytes);
   return QE_OK;
 }
 
@@ -524,10 +541,9 @@ qe_status qe_act_quant(const void* X, qe_dtype x_dtype, const float* s_inv, int3
 
 qe_status qe_linear_forward_noalloc(const qe_layer_desc* desc, const qe_layer_weights* weights, const void* X,
                                     qe_dtype x_dtype, int32_t T, void* Y, qe_dtype y_dtype, void* stream) {
-  qe_status s = check_desc(desc);
-  if (s != QE_OK) return s;
-  if (T < 0) return QE_ERR_INVALID_ARG;
-  if (T == 0) return QE_OK;
+  // the same argument checks as qe_linear_forward, before the scratch is sized
+  qe_status s = check_forward_args(desc, weights, X, x_dtype, T, Y, y_dtype);
+  if (s != QE_OK || T == 0) return s;
   const size_t need = make_plan(desc, T, x_dtype == QE_BF16).bytes;  // the scratch this input dtype needs
   if (need > QE_NOALLOC_WORKSPACE_BYTES) {
     snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),

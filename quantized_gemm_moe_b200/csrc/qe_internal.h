@@ -75,6 +75,8 @@ cudaError_t launch_quantize_weights(const void* W, bool w_bf16, const float* s, 
                                     int w_bits, uint8_t* packed, float* w_scale, cudaStream_t st);
 cudaError_t launch_colstats(const void* W, bool w_bf16, int N, int K, float* w_mean, float* w_colmax,
                             cudaStream_t st);
+// s_inv[k] = fl32(1/s[k]) (IEEE division).
+cudaError_t launch_recip(const float* s, int K, float* s_inv, cudaStream_t st);
 cudaError_t launch_unpack_weights(const uint8_t* packed, int N, int K, int w_bits, int8_t* codes,
                                   cudaStream_t st);
 cudaError_t launch_pack_adapters(const AdapterGeom& g, int K, int N, const uint16_t* A_s, const uint16_t* B_s,
@@ -194,6 +196,9 @@ cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
 
 // Device error word (one per device, in the library's own device memory).
 int* device_error_ptr();  // nullptr when the symbol lookup fails
+// The calling thread's current CUDA context (CUcontext), or nullptr; keys the per-device
+// caches of device symbol addresses.
+void* current_context();
 cudaError_t read_device_error(int* value, bool clear, cudaStream_t st);
 
 // Top-k importance. bf16 rows with 7680 <= K <= 30720 take the streaming kernel (one CTA per

@@ -34,6 +34,7 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // A wait gives up after this long. Healthy waits here last microseconds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kDrainLimitNs = 10000000ull;    // 10 ms: copies in flight at teardown
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -81,6 +82,29 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, in
 }
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* flag, int err) {
   return mbar_wait_for(bar, parity, flag, err, kWaitLimitNs);
+}
+// Which TMEM buffer the epilogue drains next. The two MMA issuers take alternate stages, and
+// issuer q cycles through its own buffers q, q+2, ..., q+2(kOwn-1). The epilogue tracks the
+// issuers' progress in one word: bit 0 = parity of the current unit's first stage, bits 1..3 /
+// 4..6 = groups issued so far by issuer 0 / 1, mod 8 (enough for kOwn <= 4). Returns the
+// buffer and sets `use_parity` to the parity of that buffer's use.
+template <int kOwn>
+__device__ __forceinline__ int epi_next_buffer(uint32_t& st, int iq, uint32_t& use_parity) {
+  static_assert(kOwn >= 1 && kOwn <= 4, "buffer state holds counts mod 8");
+  const int sh = 1 + 3 * iq;
+  const uint32_t oc = (st >> sh) & 7u;
+  st = (st & ~(7u << sh)) | (((oc + 1u) & 7u) << sh);
+  use_parity = (oc / kOwn) & 1u;
+  return iq + 2 * static_cast<int>(oc % kOwn);
+}
+
+// Before a CTA exits, the thread that issued a ring's loads waits (bounded) for the last `depth`
+// of its `issued` loads to land: after a wait ran out, their consumer may have stopped, and a
+// copy must not land in the shared memory of a CTA that has exited. On a normal run these
+// phases are already complete, or complete while the consumers finish.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int depth, int issued) {
+  for (int j = issued > depth ? issued - depth : 0; j < issued; ++j)
+    mbar_wait_for(&full[j % depth], static_cast<uint32_t>((j / depth) & 1), nullptr, 0, kDrainLimitNs);
 }
 
 // ------------------------------------------------------------------ async copies

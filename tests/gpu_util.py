@@ -61,11 +61,11 @@ class Case:
                 dense[e, torch.from_numpy(ch[e]).long()] += A_rs[e]
             i["A_r"] = dense
             self.layer = qe.QELayer.from_float(self.desc, cuda(i["W"]), cuda(i["s"]), cuda(i["A_s"]), cuda(i["B_s"]),
-                                               cuda(A_rs), cuda(i["B_r"]), cuda(i["G"]), s_inv=cuda(i["s_inv"]),
+                                               cuda(A_rs), cuda(i["B_r"]), cuda(i["G"]),
                                                channels=cuda(ch))
         else:
             self.layer = qe.QELayer.from_float(self.desc, cuda(i["W"]), cuda(i["s"]), cuda(i["A_s"]), cuda(i["B_s"]),
-                                               cuda(i["A_r"]), cuda(i["B_r"]), cuda(i["G"]), s_inv=cuda(i["s_inv"]))
+                                               cuda(i["A_r"]), cuda(i["B_r"]), cuda(i["G"]))
         self._ref = None
 
     def oracle_weights(self):
@@ -76,7 +76,7 @@ class Case:
     def oracle_forward(self, rows=None, expert_override=None):
         codes, scales, _, _ = self.oracle_weights()
         i = self.inp
-        return oracle.qe_forward(i["X"], codes, scales, i["s_inv"], i["A_s"], i["B_s"], i["A_r"], i["B_r"], i["G"],
+        return oracle.qe_forward(i["X"], codes, scales, oracle.smoothing_inverse(i["s"]), i["A_s"], i["B_s"], i["A_r"], i["B_r"], i["G"],
                                  self.cfg.group, self.cfg.a_bits, rows=rows, expert_override=expert_override)
 
     def gpu_forward(self, out_dtype=torch.float32):

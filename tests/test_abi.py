@@ -99,8 +99,11 @@ def test_other_entry_points_validate(lib):
     assert lib.qe_route(16, 1, 16, 4, 256, 17, 16, 16, 16, None, None) == qe.QE_ERR_INVALID_ARG
     assert lib.qe_act_quant(16, 1, 16, 4, 256, 5, 16, 16, None) == qe.QE_ERR_INVALID_ARG  # a_bits 5
     d = qe.make_desc(256, 256, 64, 4, 8, 8, 4, 4)
-    assert lib.qe_quantize_weights(ctypes.byref(d), None, 0, 16, 16, 16, None, None, None) == qe.QE_ERR_INVALID_ARG
-    assert lib.qe_quantize_weights(ctypes.byref(d), 8, 0, 16, 16, 16, None, None, None) == qe.QE_ERR_ALIGNMENT
+    assert lib.qe_quantize_weights(ctypes.byref(d), None, 0, 16, 16, 16, None, None, None, None) == \
+        qe.QE_ERR_INVALID_ARG
+    assert lib.qe_quantize_weights(ctypes.byref(d), 8, 0, 16, 16, 16, None, None, None, None) == qe.QE_ERR_ALIGNMENT
+    # the s_inv output must be 16-byte aligned too
+    assert lib.qe_quantize_weights(ctypes.byref(d), 16, 0, 16, 16, 16, None, None, 8, None) == qe.QE_ERR_ALIGNMENT
     assert lib.qe_pack_adapters(ctypes.byref(d), 16, 16, 16, 16, None, 16, None) == qe.QE_ERR_INVALID_ARG
     for s in range(7):
         assert lib.qe_status_string(s)

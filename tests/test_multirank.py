@@ -52,3 +52,31 @@ def test_two_rank_replicas_take_max_time_and_distinct_batches():
 def test_single_process_needs_no_group():
     import bench
     assert bench.max_over_ranks(3.5, None) == 3.5
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    # `bench.py --gpus 2` outside torchrun starts two ranks itself (torch.distributed.run on
+    # 127.0.0.1). The reference arm runs on CPU: rank 0 times the oracle and prints the line,
+    # rank 1 exits without work, and n_gpus reports the launched world size.
+    import json
+    import subprocess
+    env = dict(os.environ)
+    for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    env["OMP_NUM_THREADS"] = "2"
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0", "--cpu-seconds", "0.3", "--workload", "qwen2vl2b"],
+                       capture_output=True, text=True, timeout=600, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+
+
+def test_gpus_flag_must_match_the_launcher():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode != 0 and "launcher started 3 ranks" in r.stderr

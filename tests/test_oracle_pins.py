@@ -47,6 +47,21 @@ def test_zero_group_gives_zero_scale_and_codes():
     assert codes[1, 4:].tolist() == [2, -3, 5, -7]
 
 
+def test_smoothing_inverse_is_the_nearest_fp32_reciprocal():
+    # s_inv = fl32(1/s): no fp32 neighbour of the stored value is closer to the exact 1/s
+    # (checked in fp64, where 1/s and the distances are exact enough), and powers of two invert exactly
+    g = np.random.default_rng(5)
+    s = np.concatenate([g.uniform(0.01, 100.0, 4000), 2.0 ** g.integers(-20, 20, 64)]).astype(np.float32)
+    si = oracle.smoothing_inverse(s)
+    assert si.dtype == np.float32
+    exact = 1.0 / s.astype(np.float64)
+    d0 = np.abs(si.astype(np.float64) - exact)
+    for nb in (np.nextafter(si, np.float32(np.inf)), np.nextafter(si, np.float32(0))):
+        assert (d0 <= np.abs(nb.astype(np.float64) - exact)).all()
+    p2 = s[-64:]
+    assert (si[-64:].astype(np.float64) * p2.astype(np.float64) == 1.0).all()
+
+
 def test_channel_scale_multiplies_weights_and_divides_activations():
     # Scaling moves magnitude between X and W (Shared Expert paragraph): with s
     # a power of two the scaled weight W*s is exact, so the weight codes of
@@ -113,7 +128,7 @@ def test_activation_invariants():
     X[5] = 0.0  # an all-zero token
     for bits in (6, 8):
         qm = oracle.qmax(bits)
-        q, sa = oracle.act_quant(X, inp["s_inv"], bits)
+        q, sa = oracle.act_quant(X, oracle.smoothing_inverse(inp["s"]), bits)
         assert np.abs(q).max() <= qm
         nz = sa > 0
         assert (np.abs(q[nz]).max(axis=1) == qm).all()
@@ -170,9 +185,9 @@ def test_zero_adapters_equal_literal_dequant_matmul():
     # the accuracy tables). The oracle's per-group int64 form must match the
     # literal (sa*q_x) . (sw*q_w)^T computed as one fp64 matmul.
     cfg, inp, codes, scales, ad = _tiny_layer(zero_adapters=True)
-    Y, _ = oracle.qe_forward(inp["X"], codes, scales, inp["s_inv"], ad["A_s"], ad["B_s"], ad["A_r"],
+    Y, _ = oracle.qe_forward(inp["X"], codes, scales, oracle.smoothing_inverse(inp["s"]), ad["A_s"], ad["B_s"], ad["A_r"],
                              ad["B_r"], inp["G"], cfg.group, 8)
-    xq, sa = oracle.act_quant(inp["X"], inp["s_inv"], 8)
+    xq, sa = oracle.act_quant(inp["X"], oracle.smoothing_inverse(inp["s"]), 8)
     deq_x = xq.astype(np.float64) * sa.astype(np.float64)[:, None]
     deq_w = codes.astype(np.float64) * np.repeat(scales.astype(np.float64), cfg.group, axis=1)
     Ylit = deq_x @ deq_w.T
@@ -182,10 +197,10 @@ def test_zero_adapters_equal_literal_dequant_matmul():
 def test_adapter_terms_match_formula():
     # Y - Y(adapters=0) = (X A_s) B_s + (X A_r[e]) B_r[e] for the routed e.
     cfg, inp, codes, scales, ad = _tiny_layer()
-    Y, e = oracle.qe_forward(inp["X"], codes, scales, inp["s_inv"], ad["A_s"], ad["B_s"], ad["A_r"],
+    Y, e = oracle.qe_forward(inp["X"], codes, scales, oracle.smoothing_inverse(inp["s"]), ad["A_s"], ad["B_s"], ad["A_r"],
                              ad["B_r"], inp["G"], cfg.group, 8)
     z = {k: torch.zeros_like(v) for k, v in ad.items()}
-    Y0, e0 = oracle.qe_forward(inp["X"], codes, scales, inp["s_inv"], z["A_s"], z["B_s"], z["A_r"],
+    Y0, e0 = oracle.qe_forward(inp["X"], codes, scales, oracle.smoothing_inverse(inp["s"]), z["A_s"], z["B_s"], z["A_r"],
                                z["B_r"], inp["G"], cfg.group, 8)
     assert (e == e0).all()
     X = np.asarray(inp["X"], np.float64)
@@ -202,7 +217,7 @@ def test_token_independence_rows_permute():
     cfg, inp, codes, scales, ad = _tiny_layer()
     X = np.asarray(inp["X"])
     p = np.random.default_rng(8).permutation(X.shape[0])
-    args = (codes, scales, inp["s_inv"], ad["A_s"], ad["B_s"], ad["A_r"], ad["B_r"], inp["G"], cfg.group, 8)
+    args = (codes, scales, oracle.smoothing_inverse(inp["s"]), ad["A_s"], ad["B_s"], ad["A_r"], ad["B_r"], inp["G"], cfg.group, 8)
     Y, e = oracle.qe_forward(X, *args)
     Yp, ep = oracle.qe_forward(X[p], *args)
     assert (Yp == Y[p]).all() and (ep == e[p]).all()
@@ -217,7 +232,7 @@ def test_identical_experts_make_routing_irrelevant():
     B_r = ad["B_r"].clone()
     A_r[:] = A_r[0]
     B_r[:] = B_r[0]
-    args = (codes, scales, inp["s_inv"], ad["A_s"], ad["B_s"], A_r, B_r, inp["G"], cfg.group, 8)
+    args = (codes, scales, oracle.smoothing_inverse(inp["s"]), ad["A_s"], ad["B_s"], A_r, B_r, inp["G"], cfg.group, 8)
     Y, _ = oracle.qe_forward(inp["X"], *args)
     T = Y.shape[0]
     for ov in (np.zeros(T), np.full(T, 3), np.arange(T) % 4):
@@ -259,9 +274,9 @@ def test_svd_adapters_reduce_layer_output_error_through_oracle():
     X = np.asarray(inp["X"])
     Yfp = X.astype(np.float64) @ np.asarray(inp["W"], np.float64).T
     z = np.zeros_like
-    Yq, _ = oracle.qe_forward(X, codes, scales, inp["s_inv"], z(A_s), z(B_s), z(A_r), z(B_r), inp["G"],
+    Yq, _ = oracle.qe_forward(X, codes, scales, oracle.smoothing_inverse(inp["s"]), z(A_s), z(B_s), z(A_r), z(B_r), inp["G"],
                               cfg.group, 16)
-    Yqe, _ = oracle.qe_forward(X, codes, scales, inp["s_inv"], A_s, B_s, A_r, B_r, inp["G"], cfg.group, 16)
+    Yqe, _ = oracle.qe_forward(X, codes, scales, oracle.smoothing_inverse(inp["s"]), A_s, B_s, A_r, B_r, inp["G"], cfg.group, 16)
     err_q = ((Yq - Yfp) ** 2).sum()
     err_qe = ((Yqe - Yfp) ** 2).sum()
     # a_bits=16 leaves only the bf16 activation rounding besides the weight error
@@ -270,7 +285,7 @@ def test_svd_adapters_reduce_layer_output_error_through_oracle():
 
 def test_group_accumulator_bound_and_numpy():
     cfg, inp, codes, scales, ad = _tiny_layer()
-    xq, _ = oracle.act_quant(inp["X"], inp["s_inv"], 8)
+    xq, _ = oracle.act_quant(inp["X"], oracle.smoothing_inverse(inp["s"]), 8)
     acc = oracle.group_acc(xq, codes, cfg.group)
     ref = np.einsum("tjg,ojg->toj", xq.reshape(64, 4, 64).astype(np.int64),
                     codes.reshape(256, 4, 64).astype(np.int64))
