@@ -1,0 +1,657 @@
+// Product of a decode-sized batch (T <= 16 tokens) of the QE linear layer on the tensor cores.
+//
+// At T <= 16 the layer streams the packed weights once and does little arithmetic per byte, so
+// HBM bandwidth bounds it (the 72B decode layers move ~120 MB of codes for 16 tokens). The
+// prefill kernels tile by output block and split K only when tiles are scarce; here the whole
+// (output tile, K block) sequence is split evenly over the SMs instead ("stream-K"): CTA c takes
+// blocks [c*NB/G, (c+1)*NB/G) of the tile-major order, so every SM streams the same number of
+// bytes whatever the shape. A CTA's range crosses at most a few tile boundaries; each piece of a
+// tile (a segment) leaves an fp32 partial, and the CTA that finishes a tile's last segment adds the
+// tile's partials in segment order (deterministic), applies the token scale and the adapter term,
+// and writes Y.
+//
+// Per 128 x 128 weight block:
+//   warp 0      bulk copy of the packed block and TMA of the activation tile (16 tokens x 128
+//               channels) into a 10-deep ring: up to 80 KB of weights in flight per SM
+//   warps 4-11  unpack the block straight into tensor memory with tcgen05.st: the MMA takes its
+//               A operand (the weights, M = 128 output rows = TMEM lanes, K along the columns)
+//               from TMEM, so the unpacked weights never pass through shared memory (whose
+//               bandwidth the unpack would otherwise exceed at the HBM rate). Two warps per TMEM
+//               lane quarter, each one half of the block's columns.
+//   warps 1-2   one thread each issues the MMAs of alternate blocks: kind::i8 (codes x16 against
+//               int8 activation codes, 4 K steps) or kind::f16 (bf16 weights against bf16
+//               activations, 8 K steps). Every quantization group gets a fresh 16-column
+//               accumulator (the first K step does not accumulate), issuer q owning slots
+//               q, q+2, ...
+//   warps 12-15 epilogue, one output row per thread: per group acc += sw * group sum (the int8
+//               sums converted exactly), with the scales loaded six blocks ahead; the adapter term
+//               of a tile on CUDA cores (fp16 inputs, fp32 sums) in the CTA that holds its first
+//               block; the segment partials and the per-tile fix-up.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
+#include "qe_internal.h"
+#include "qe_ptx.cuh"
+
+namespace qe {
+namespace {
+
+constexpr int kDN = 16;          // token columns: the whole batch, padded (MMA N)
+constexpr int kDThreads = 512;   // 16 warps
+constexpr int kDStages = 10;     // packed block + activation tile ring
+constexpr int kDASlots = 4;      // unpacked A blocks in TMEM
+constexpr int kDTmemCols = 512;
+constexpr int kDSwAhead = 6;     // blocks of group scales in flight per epilogue thread
+
+template <bool I8, int BITS>
+struct DCfg {
+  static constexpr int kWBlock = (BITS == 4) ? kW4BlockBytes : kW3BlockBytes;
+  static constexpr int kXAtom = kDN * 128;                // 16 rows x 128 bytes (one swizzle atom pair)
+  static constexpr int kXTile = I8 ? kXAtom : 2 * kXAtom;  // 128 input channels: int8 codes or bf16
+  static constexpr int kACols = I8 ? 32 : 64;             // TMEM columns of one unpacked block
+  static constexpr int kKSteps = I8 ? 4 : 8;              // MMA K steps per block (32 int8 / 16 bf16)
+  static constexpr int kAccSlots = (kDTmemCols - kDASlots * kACols) / kDN;  // 24 (int8) / 16 (bf16)
+  static constexpr int kOwn = kAccSlots / 2;              // accumulator slots per issuer
+  static constexpr int kUcatBytes = kDN * 512 * 2;        // U_cat staging, R_pad <= 512
+  static constexpr size_t kSmem = 1024 + size_t(kDStages) * kXTile + size_t(kDStages) * kWBlock + kUcatBytes + 1024;
+  static_assert(kAccSlots % 2 == 0, "each issuer owns half of the accumulator slots");
+  static_assert(kSmem <= 232448, "shared memory");
+};
+
+struct DecArgs {
+  const uint8_t* w_packed;
+  const float* w_scale;     // [G][N]
+  const float* sa_sorted;   // [T]
+  const float* su_sorted;   // [T] or nullptr (no adapters)
+  const int32_t* perm;      // [T]
+  const uint16_t* ucat;     // fp16 [T][R_pad], bucket order
+  const uint16_t* bcat;     // fp16 [N][R_pad]
+  int R_pad;
+  int T, N, K, group, KB, NT, G_total;
+  int64_t NB;               // NT * KB
+  int maxseg;
+  void* Y;
+  int y_bf16;
+  float* part;              // [NT][maxseg][128][16]
+  float* ad;                // [NT][128][16]
+  unsigned* cnt;            // [NT], zero at launch
+  int32_t* dbg_acc;         // [T][N][G] token order, or nullptr
+  int* err;
+};
+
+// CTA c of G owns blocks [range_begin(c), range_begin(c+1)) of the NB blocks in tile-major order;
+// block f belongs to CTA cta_of(f).
+__host__ __device__ __forceinline__ int64_t range_begin(int c, int64_t NB, int G) {
+  return static_cast<int64_t>(c) * NB / G;
+}
+__host__ __device__ __forceinline__ int cta_of(int64_t f, int64_t NB, int G) {
+  return static_cast<int>(((f + 1) * G - 1) / NB);
+}
+
+__device__ __forceinline__ void mma_i8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t x, uint32_t y) {
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&x);
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&y);
+  __nv_bfloat162 r = __hsub2(a, b);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+// Four 4-bit two's-complement codes (one nibble per byte, at `shift`) -> bf16 pairs (q0,q1), (q2,q3):
+// bf16(128 + q + 8) built by a byte permute, then bf16(136) subtracted (exact for these integers).
+__device__ __forceinline__ uint2 w4_to_bf16(uint32_t v, int shift) {
+  const uint32_t u = ((v >> shift) & 0x0F0F0F0Fu) ^ 0x08080808u;
+  const uint32_t lo = __byte_perm(u, 0x00004300u, 0x5150);
+  const uint32_t hi = __byte_perm(u, 0x00004300u, 0x5352);
+  return make_uint2(bf16x2_sub(lo, 0x43084308u), bf16x2_sub(hi, 0x43084308u));
+}
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));  // (a & b) | c
+  return d;
+}
+// Two 3-bit offset-binary codes u = q + 4 (low two bits at lo_shift and 16 + lo_shift of lw, bit 2
+// at hi_shift and 16 + hi_shift of hw) -> the bf16 pair (q_even, q_odd).
+__device__ __forceinline__ uint32_t w3_pair_to_bf16(uint32_t lw, uint32_t hw, int lo_shift, int hi_shift) {
+  const uint32_t l = lop3_and_or(lw >> lo_shift, 0x00030003u, 0x43004300u);
+  const uint32_t hs = (hi_shift >= 2) ? (hw >> (hi_shift - 2)) : (hw << (2 - hi_shift));
+  return bf16x2_sub(lop3_and_or(hs, 0x00040004u, l), 0x43044304u);
+}
+
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// One thread's half row (64 input channels) of block rows r, unpacked into TMEM columns
+// [col, col + kACols/2) of its lane: the A operand layout (row = lane, K along the columns, four
+// int8 or two bf16 per 32-bit column, lowest channel in the low bits).
+template <bool I8, int BITS>
+__device__ __forceinline__ void unpack_half_row(const uint8_t* blk, int r, int half, uint32_t taddr) {
+  if constexpr (BITS == 4) {
+    // row r: four 16-byte pieces; piece i holds channels 32i..32i+15 in the low nibbles of its words
+    // (word w: channels 32i+4w..+3) and 32i+16..32i+31 in the high nibbles
+    const uint4 p0 = *reinterpret_cast<const uint4*>(blk + r * 64 + half * 32);
+    const uint4 p1 = *reinterpret_cast<const uint4*>(blk + r * 64 + half * 32 + 16);
+    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    if constexpr (I8) {
+      // the code goes to the high nibble of its byte: the byte is the int8 16*q (the x16 is folded
+      // into the group scale)
+      uint32_t v[16];
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[8 * pc + j] = (w[4 * pc + j] << 4) & 0xF0F0F0F0u;
+          v[8 * pc + 4 + j] = w[4 * pc + j] & 0xF0F0F0F0u;
+        }
+      tmem_st_x16(taddr, v);
+    } else {
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc) {
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint2 lo = w4_to_bf16(w[4 * pc + j], 0), hi = w4_to_bf16(w[4 * pc + j], 4);
+          v[2 * j] = lo.x;
+          v[2 * j + 1] = lo.y;
+          v[8 + 2 * j] = hi.x;
+          v[8 + 2 * j + 1] = hi.y;
+        }
+        tmem_st_x16(taddr + 16 * pc, v);
+      }
+    }
+  } else {
+    // row r: 48 bytes; column c (channels 2c, 2c+1) of this half: low word 4*half + (c%32)/8 at
+    // pair c%8, high word 2*half + (c%32)/16 at pair c%16
+    const uint4 lq = *reinterpret_cast<const uint4*>(blk + r * 48 + half * 16);
+    const uint2 hq = *reinterpret_cast<const uint2*>(blk + r * 48 + 32 + half * 8);
+    const uint32_t lw[4] = {lq.x, lq.y, lq.z, lq.w};
+    const uint32_t hw[2] = {hq.x, hq.y};
+#pragma unroll
+    for (int pc = 0; pc < 2; ++pc) {
+      uint32_t v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int c = 16 * pc + j;
+        v[j] = w3_pair_to_bf16(lw[c >> 3], hw[c >> 4], 2 * (c & 7), c & 15);
+      }
+      tmem_st_x16(taddr + 16 * pc, v);
+    }
+  }
+}
+
+template <bool I8, int BITS>
+__global__ void __launch_bounds__(kDThreads, 1)
+    k_qdec(const __grid_constant__ CUtensorMap tm_x, const DecArgs a) {
+  using C = DCfg<I8, BITS>;
+  constexpr int NS = kDStages, NA = kDASlots;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xring = smem;                              // [NS][kXTile], 1024-aligned (128B swizzle)
+  uint8_t* wring = xring + NS * C::kXTile;            // [NS][kWBlock]
+  __half* ucat_s = reinterpret_cast<__half*>(wring + NS * C::kWBlock);  // [16][R_pad]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ucat_s) + C::kUcatBytes);
+  uint64_t* wfull = bars;                  // [NS] block + tile landed (1 + bytes)
+  uint64_t* wempty = wfull + NS;           // [NS] the MMAs of the block are done (ring slot free)
+  uint64_t* afull = wempty + NS;           // [NA] A unpacked into TMEM (8 unpack warps)
+  uint64_t* aempty = afull + NA;           // [NA] the MMAs of the block are done (A slot free)
+  uint64_t* accf = aempty + NA;            // [kAccSlots] group sum ready
+  uint64_t* acce = accf + C::kAccSlots;    // [kAccSlots] group sum read (4 epilogue warps)
+  uint64_t* done = acce + C::kAccSlots;    // teardown
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  int* flag_s = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int64_t b0 = range_begin(c, a.NB, G), b1 = range_begin(c + 1, a.NB, G);
+  const int nblk = static_cast<int>(b1 - b0);
+  const int gpb = kTileK / a.group;
+  int* const a_err = a.err;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 1);
+    }
+    for (int s = 0; s < NA; ++s) {
+      mbar_init(&afull[s], 8);
+      mbar_init(&aempty[s], 1);
+    }
+    for (int b = 0; b < C::kAccSlots; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 4);
+    }
+    mbar_init(done, 2);
+    mbar_fence_init();
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kDTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t colA = 0, colAcc = kDASlots * C::kACols;
+  grid_dep_wait();
+  grid_dep_launch();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int i = 0;
+      for (; i < nblk; ++i) {
+        const int s = i % NS;
+        if (!mbar_wait(&wempty[s], ((i / NS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) break;
+        const int64_t f = b0 + i;
+        const int kb = static_cast<int>(f % a.KB);
+        mbar_arrive_expect_tx(&wfull[s], C::kWBlock + C::kXTile);
+        bulk_load(wring + s * C::kWBlock, a.w_packed + f * C::kWBlock, C::kWBlock, &wfull[s]);
+        tma_load_2d(xring + s * C::kXTile, &tm_x, kb * kTileK, 0, &wfull[s]);
+        if constexpr (!I8) tma_load_2d(xring + s * C::kXTile + C::kXAtom, &tm_x, kb * kTileK + 64, 0, &wfull[s]);
+      }
+      drain_ring(wfull, NS, i);
+    }
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers (alternate blocks)
+    const int qi = warp - 1;
+    if (lane == 0) {
+      const uint32_t idesc = I8 ? idesc_i8(128, kDN) : idesc_bf16(128, kDN);
+      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xring));
+      int own = 0;
+      bool ok = true;
+      for (int i = qi; i < nblk && ok; i += 2) {
+        const int s = i % NS, as = i % NA;
+        const int64_t f = b0 + i;
+        const int kb = static_cast<int>(f % a.KB);
+        const int ng = min(gpb, a.G_total - kb * gpb);
+        if (!mbar_wait(&afull[as], (i / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t xdesc = xdesc0 + static_cast<uint64_t>((s * C::kXTile) >> 4);
+        const uint32_t a_col = tmem + colA + as * C::kACols;
+        for (int gi = 0; gi < ng; ++gi) {
+          const int slot = qi + 2 * (own % C::kOwn);
+          const uint32_t use = static_cast<uint32_t>(own / C::kOwn);
+          ++own;
+          if (!mbar_wait(&acce[slot], (use & 1u) ^ 1u, a_err, DEVERR_WAIT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + colAcc + slot * kDN;
+          const int k0 = (gpb == 1) ? 0 : gi * (C::kKSteps / 2);
+          const int nk = (gpb == 1) ? C::kKSteps : C::kKSteps / 2;
+          for (int kk = 0; kk < nk; ++kk) {
+            const int ks = k0 + kk;
+            if constexpr (I8) {
+              // K step of 32 int8: 8 TMEM columns of A, 32 bytes along the tile's swizzled rows
+              mma_i8_ta(d, a_col + ks * 8, xdesc + static_cast<uint64_t>(2 * ks), idesc, kk > 0 ? 1u : 0u);
+            } else {
+              // K step of 16 bf16: 8 TMEM columns of A; the tile is two 64-channel atoms
+              const uint64_t offb = static_cast<uint64_t>((ks >> 2) * (C::kXAtom >> 4) + (ks & 3) * 2);
+              mma_f16_ta(d, a_col + ks * 8, xdesc + offb, idesc, kk > 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(&accf[slot]);
+        }
+        tc_commit(&aempty[as]);
+        tc_commit(&wempty[s]);
+      }
+      tc_commit(done);
+      mbar_wait(done, 0, a_err, DEVERR_WAIT_TEARDOWN);
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ unpack into TMEM
+    const int q4 = warp & 3, half = (warp - 4) >> 2;
+    const int r = 32 * q4 + lane;  // block row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
+    for (int i = 0; i < nblk; ++i) {
+      const int s = i % NS, as = i % NA;
+      if (!mbar_wait(&wfull[s], (i / NS) & 1, a_err, DEVERR_WAIT_UNPACK) ||
+          !mbar_wait(&aempty[as], ((i / NA) & 1) ^ 1, a_err, DEVERR_WAIT_UNPACK))
+        break;
+      tc_fence_after();
+      unpack_half_row<I8, BITS>(wring + s * C::kWBlock, r, half,
+                                tmem + lane_base + colA + as * C::kACols + half * (C::kACols / 2));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[as]);
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ epilogue, one output row per thread
+    // Control flow follows the block schedule only; after a wait ran out, `ok` turns off every
+    // later wait and TMEM access, and the named barriers are still reached by all four warps.
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;
+    const int et = threadIdx.x - 384;  // 0..127
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
+    const int T = a.T;
+    bool ok = true;
+    int cnt0 = 0, cnt1 = 0;           // groups drained from issuer 0 / 1
+    // group scales of the next kDSwAhead blocks (two groups per block at g = 64)
+    float sw0[kDSwAhead], sw1[kDSwAhead];
+    auto load_sw = [&](int i, float& s0, float& s1) {
+      s0 = 0.0f;
+      s1 = 0.0f;
+      if (i >= nblk) return;
+      const int64_t f = b0 + i;
+      const int nt = static_cast<int>(f / a.KB), kb = static_cast<int>(f % a.KB);
+      const int o = nt * kTileN + r;
+      if (o >= a.N) return;
+      const int j = kb * gpb;
+      s0 = __ldg(a.w_scale + static_cast<size_t>(j) * a.N + o);
+      if (gpb == 2 && j + 1 < a.G_total) s1 = __ldg(a.w_scale + static_cast<size_t>(j + 1) * a.N + o);
+    };
+#pragma unroll
+    for (int k = 0; k < kDSwAhead; ++k) load_sw(k, sw0[k], sw1[k]);
+    float acc[kDN], adr[kDN];
+#pragma unroll
+    for (int p = 0; p < kDN; ++p) {
+      acc[p] = 0.0f;
+      adr[p] = 0.0f;
+    }
+    int cur_nt = -1;
+    bool have_ad = false;  // adr holds this CTA's adapter term of tile cur_nt
+
+    // The tile's adapter term su-less: ad[p] = sum_r B_catT[o][r] * U_cat[p][r] (fp32 sums of fp16 inputs).
+    auto adapter_term = [&](int nt) {
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int rp = a.R_pad;
+      for (int e = et; e < kDN * rp / 8; e += 128) {
+        const int p = e / (rp / 8), c8 = e % (rp / 8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (p < T) v = __ldg(reinterpret_cast<const uint4*>(a.ucat + static_cast<size_t>(p) * rp) + c8);
+        *reinterpret_cast<uint4*>(ucat_s + static_cast<size_t>(p) * rp + c8 * 8) = v;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int o = nt * kTileN + r;
+#pragma unroll
+      for (int p = 0; p < kDN; ++p) adr[p] = 0.0f;
+      if (o < a.N) {
+        const uint4* brow = reinterpret_cast<const uint4*>(a.bcat + static_cast<size_t>(o) * rp);
+        for (int c8 = 0; c8 < rp / 8; ++c8) {
+          const uint4 bv = __ldg(brow + c8);
+          const __half2* bh = reinterpret_cast<const __half2*>(&bv);
+          float2 bf[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) bf[k] = __half22float2(bh[k]);
+#pragma unroll
+          for (int p = 0; p < kDN; ++p) {
+            const uint4 uv = *reinterpret_cast<const uint4*>(ucat_s + static_cast<size_t>(p) * rp + c8 * 8);
+            const __half2* uh = reinterpret_cast<const __half2*>(&uv);
+            float s = adr[p];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 uf = __half22float2(uh[k]);
+              s = fmaf(bf[k].x, uf.x, s);
+              s = fmaf(bf[k].y, uf.y, s);
+            }
+            adr[p] = s;
+          }
+        }
+      }
+    };
+
+    // End of a segment of tile nt: a tile held by this CTA alone is written at once; otherwise the
+    // partial goes to its slot and the last CTA to finish the tile adds the partials in segment order.
+    auto finish_segment = [&](int nt) {
+      const int64_t f0 = static_cast<int64_t>(nt) * a.KB;
+      const int c_first = cta_of(f0, a.NB, G);
+      const int nseg = cta_of(f0 + a.KB - 1, a.NB, G) - c_first + 1;
+      const int seg = c - c_first;
+      const int o = nt * kTileN + r;
+      const size_t tile_row = (static_cast<size_t>(nt) * kTileN + r) * kDN;
+      bool last = true;
+      if (nseg > 1) {
+        float4* dst = reinterpret_cast<float4*>(a.part + (static_cast<size_t>(nt) * a.maxseg + seg) * kTileN * kDN +
+                                                static_cast<size_t>(r) * kDN);
+#pragma unroll
+        for (int k = 0; k < kDN / 4; ++k) dst[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
+        if (have_ad) {
+          float4* ad = reinterpret_cast<float4*>(a.ad + tile_row);
+#pragma unroll
+          for (int k = 0; k < kDN / 4; ++k) ad[k] = make_float4(adr[4 * k], adr[4 * k + 1], adr[4 * k + 2], adr[4 * k + 3]);
+        }
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (et == 0) {
+          const unsigned old = atomicAdd(a.cnt + nt, 1u);
+          *flag_s = (old == static_cast<unsigned>(nseg - 1)) ? 1 : 0;
+          __threadfence();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        last = *flag_s != 0;
+        if (last) {
+#pragma unroll
+          for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
+          for (int sgi = 0; sgi < nseg; ++sgi) {
+            const float4* src = reinterpret_cast<const float4*>(
+                a.part + (static_cast<size_t>(nt) * a.maxseg + sgi) * kTileN * kDN + static_cast<size_t>(r) * kDN);
+#pragma unroll
+            for (int k = 0; k < kDN / 4; ++k) {
+              const float4 v = __ldcg(src + k);
+              acc[4 * k] += v.x;
+              acc[4 * k + 1] += v.y;
+              acc[4 * k + 2] += v.z;
+              acc[4 * k + 3] += v.w;
+            }
+          }
+          if (!have_ad && a.su_sorted) {
+            const float4* ad = reinterpret_cast<const float4*>(a.ad + tile_row);
+#pragma unroll
+            for (int k = 0; k < kDN / 4; ++k) {
+              const float4 v = __ldcg(ad + k);
+              adr[4 * k] = v.x;
+              adr[4 * k + 1] = v.y;
+              adr[4 * k + 2] = v.z;
+              adr[4 * k + 3] = v.w;
+            }
+          }
+        }
+      }
+      if (last) {
+        if (o < a.N) {
+#pragma unroll
+          for (int p = 0; p < kDN; ++p) {
+            if (p >= T) break;
+            float y = acc[p] * __ldg(a.sa_sorted + p);
+            if (a.su_sorted) y = fmaf(__ldg(a.su_sorted + p), adr[p], y);
+            const size_t at = static_cast<size_t>(__ldg(a.perm + p)) * a.N + o;
+            if (a.y_bf16) {
+              const __nv_bfloat16 h = __float2bfloat16_rn(y);
+              static_cast<__nv_bfloat16*>(a.Y)[at] = h;
+            } else {
+              static_cast<float*>(a.Y)[at] = y;
+            }
+          }
+        }
+        if (nseg > 1 && et == 0) a.cnt[nt] = 0u;  // leave the counter at zero for the next launch
+      }
+      have_ad = false;
+    };
+
+    for (int i = 0; i < nblk; ++i) {
+      const int64_t f = b0 + i;
+      const int nt = static_cast<int>(f / a.KB), kb = static_cast<int>(f % a.KB);
+      if (nt != cur_nt) {
+        if (cur_nt >= 0) finish_segment(cur_nt);
+        cur_nt = nt;
+#pragma unroll
+        for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
+        if (kb == 0 && a.su_sorted) {
+          adapter_term(nt);
+          have_ad = true;
+        }
+      }
+      const float s0 = sw0[0], s1 = sw1[0];
+#pragma unroll
+      for (int k = 0; k + 1 < kDSwAhead; ++k) {
+        sw0[k] = sw0[k + 1];
+        sw1[k] = sw1[k + 1];
+      }
+      load_sw(i + kDSwAhead, sw0[kDSwAhead - 1], sw1[kDSwAhead - 1]);
+      const int q = i & 1;
+      const int ng = min(gpb, a.G_total - kb * gpb);
+      for (int gi = 0; gi < ng; ++gi) {
+        const int n_q = q ? cnt1 : cnt0;
+        const int slot = q + 2 * (n_q % C::kOwn);
+        const uint32_t use = static_cast<uint32_t>(n_q / C::kOwn);
+        if (q) ++cnt1;
+        else ++cnt0;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[slot], use & 1u, a_err, DEVERR_WAIT_EPILOGUE));
+        if (!ok) continue;
+        tc_fence_after();
+        uint32_t v[kDN];
+        tmem_ld16(tmem + lane_base + colAcc + slot * kDN, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[slot]);
+        const float sw = gi ? s1 : s0;
+        if constexpr (I8) {
+          const float swq = sw * 0.0625f;  // codes entered the MMA as 16*q
+#pragma unroll
+          for (int p = 0; p < kDN; ++p) acc[p] = fmaf(static_cast<float>(static_cast<int32_t>(v[p])), swq, acc[p]);
+          if (a.dbg_acc) {
+            const int o = nt * kTileN + r;
+            if (o < a.N) {
+#pragma unroll
+              for (int p = 0; p < kDN; ++p) {
+                if (p >= T) break;
+                a.dbg_acc[(static_cast<size_t>(__ldg(a.perm + p)) * a.N + o) * a.G_total + kb * gpb + gi] =
+                    static_cast<int32_t>(v[p]) / 16;
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < kDN; ++p) acc[p] = fmaf(__uint_as_float(v[p]), sw, acc[p]);
+        }
+      }
+    }
+    if (cur_nt >= 0) finish_segment(cur_nt);
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kDTmemCols);
+  }
+}
+
+template <bool I8, int BITS>
+cudaError_t launch_qdec_t(const CUtensorMap& tm_x, const DecArgs& a, int grid, cudaStream_t st) {
+  using C = DCfg<I8, BITS>;
+  cudaError_t e = cudaFuncSetAttribute(k_qdec<I8, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kDThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_qdec<I8, BITS>, tm_x, a);
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess)
+      n = 0;
+  }
+  return n;
+}
+
+}  // namespace
+
+DecodePlan plan_decode(int N, int K, int n_sm) {
+  DecodePlan p;
+  p.NT = static_cast<int>(ceil_div(N, kTileN));
+  p.KB = static_cast<int>(ceil_div(K, kTileK));
+  p.NB = int64_t(p.NT) * p.KB;
+  p.grid = static_cast<int>(std::min<int64_t>(p.NB, n_sm > 0 ? n_sm : 148));
+  // a tile of KB consecutive blocks meets at most (KB - 1) / Lmin + 2 of the ranges (Lmin >= 1 blocks each)
+  const int64_t lmin = p.NB / p.grid;
+  p.maxseg = static_cast<int>((p.KB - 1) / lmin + 2);
+  p.part_bytes = size_t(p.NT) * p.maxseg * kTileN * kDN * 4;
+  p.ad_bytes = size_t(p.NT) * kTileN * kDN * 4;
+  p.cnt_words = p.NT;
+  return p;
+}
+
+int decode_grid_sms() { return sm_count(); }
+
+cudaError_t launch_qdec(int w_bits, bool int8, const CUtensorMap& tm_x, const DecodePlan& plan,
+                        const QgemmArgs& q, const uint16_t* ucat, const uint16_t* bcat, int R_pad, float* part,
+                        float* ad, unsigned* cnt, cudaStream_t st) {
+  DecArgs a{};
+  a.w_packed = q.w_packed;
+  a.w_scale = q.w_scale;
+  a.sa_sorted = q.sa_sorted;
+  a.su_sorted = q.su_sorted;
+  a.perm = q.perm;
+  a.ucat = ucat;
+  a.bcat = bcat;
+  a.R_pad = R_pad;
+  a.T = q.T;
+  a.N = q.N;
+  a.K = q.K;
+  a.group = q.group;
+  a.KB = plan.KB;
+  a.NT = plan.NT;
+  a.G_total = q.K / q.group;
+  a.NB = plan.NB;
+  a.maxseg = plan.maxseg;
+  a.Y = q.Y;
+  a.y_bf16 = q.y_bf16;
+  a.part = part;
+  a.ad = ad;
+  a.cnt = cnt;
+  a.dbg_acc = q.dbg_acc;
+  a.err = q.err;
+  if (q.T > kDN || q.T < 1 || R_pad > 512) return cudaErrorInvalidValue;
+  if (int8) {
+    if (w_bits != 4) return cudaErrorInvalidValue;
+    return launch_qdec_t<true, 4>(tm_x, a, plan.grid, st);
+  }
+  if (w_bits == 4) return launch_qdec_t<false, 4>(tm_x, a, plan.grid, st);
+  if (w_bits == 3) return launch_qdec_t<false, 3>(tm_x, a, plan.grid, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace qe

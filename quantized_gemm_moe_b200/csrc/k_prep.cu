@@ -643,6 +643,8 @@ struct RouteQuantArgs {
   float* sa_sorted;
   uint16_t* ucat;
   float* su_sorted;
+  unsigned* zero_words;
+  int n_zero_words;
   int* err;
 };
 
@@ -727,6 +729,9 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
   for (int i = threadIdx.x; i < a.K / 4; i += kRQThreads)
     reinterpret_cast<float4*>(s_inv_s)[i] = __ldg(reinterpret_cast<const float4*>(a.s_inv) + i);
   for (int i = threadIdx.x; i < t1 - t0; i += kRQThreads) mx_s[i] = 0;
+  // the decode product's tile counters start at zero (the product runs after this launch)
+  for (int i = blockIdx.x * kRQThreads + threadIdx.x; i < a.n_zero_words; i += gridDim.x * kRQThreads)
+    a.zero_words[i] = 0u;
   __syncthreads();
 
   if (a.do_route) {
@@ -1144,6 +1149,8 @@ cudaError_t launch_route_quant(const RouteQuantParams& q, cudaStream_t st) {
   a.sa_sorted = q.sa_sorted;
   a.ucat = q.ucat;
   a.su_sorted = q.su_sorted;
+  a.zero_words = q.zero_words;
+  a.n_zero_words = q.zero_words ? q.n_zero_words : 0;
   a.err = q.err;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));

@@ -67,8 +67,11 @@ struct Plan {
   UgemmPlan up;
   int bn, msplits, kbps;  // main product
   int uslots;             // GEMM partial slots: splits, doubled for fp32 inputs (hi and lo passes)
+  bool dec;               // T <= 16: the decode product (stream-K over the SMs, in-kernel fix-up)
+  DecodePlan dp;
   size_t off_expert, off_perm, off_pos, off_offsets, off_sa_tok, off_sa_sorted, off_su_sorted, off_act, off_xhi,
-      off_xlo, off_amax, off_upart, off_ucat, off_ypart, off_counts, off_barrier, bytes;
+      off_xlo, off_amax, off_upart, off_ucat, off_ypart, off_counts, off_barrier, off_dpart, off_dad, off_dcnt,
+      bytes;
 };
 
 Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
@@ -80,7 +83,13 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   p.has_ad = p.g.R_a > 0;
   const int Tm = std::max(T, 1);
   p.up = plan_ugemm(Tm, p.K, p.g.R_tot);
-  if (d->a_bits == 16) {
+  p.dec = Tm <= kDecodeMaxT;
+  if (p.dec) {
+    p.dp = plan_decode(p.N, p.K, decode_grid_sms());
+    p.bn = 16;
+    p.msplits = 1;
+    p.kbps = static_cast<int>(ceil_div(p.K, kTileK));
+  } else if (d->a_bits == 16) {
     p.bn = pick_wgemm_bn(Tm, p.N, p.K, &p.msplits, &p.kbps);
   } else {
     p.bn = pick_qgemm_bn(Tm, p.N, p.K, &p.msplits, &p.kbps);
@@ -108,6 +117,11 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   p.off_ypart = (p.msplits > 1) ? take(size_t(p.msplits) * Tm * p.N * 4) : 0;
   p.off_counts = take(size_t(kRouteQuantMaxGrid) * kMaxRouted * 4);
   p.off_barrier = take(4);
+  if (p.dec) {
+    p.off_dpart = take(p.dp.part_bytes);
+    p.off_dad = take(p.dp.ad_bytes);
+    p.off_dcnt = take(size_t(p.dp.cnt_words) * 4);
+  }
   p.bytes = o;
   return p;
 }
@@ -269,6 +283,8 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
     q.sa_sorted = sa_sorted;
     q.ucat = ucat;
     q.su_sorted = su_sorted;
+    q.zero_words = p.dec ? at<unsigned>(ws, p.off_dcnt) : nullptr;
+    q.n_zero_words = p.dec ? p.dp.cnt_words : 0;
     q.err = err;
     QE_CUDA(launch_route_quant(q, st), "route_quant");
   }
@@ -313,7 +329,11 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
     a.partial = ypart;
     a.dbg_acc = wonly ? nullptr : dbg_acc;
     a.err = err;
-    if (wonly)
+    if (p.dec)
+      QE_CUDA(launch_qdec(d->w_bits, !wonly, tm_act, p.dp, a, ucat, bcat, p.g.R_pad, at<float>(ws, p.off_dpart),
+                          at<float>(ws, p.off_dad), at<unsigned>(ws, p.off_dcnt), st),
+              "qdec");
+    else if (wonly)
       QE_CUDA(launch_wgemm(d->w_bits, p.bn, tm_act, tm_bcat, tm_ucat, a, st), "wgemm");
     else
       QE_CUDA(launch_qgemm(p.bn, tm_act, tm_bcat, tm_ucat, a, st), "qgemm");

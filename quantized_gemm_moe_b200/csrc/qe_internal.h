@@ -149,6 +149,8 @@ struct RouteQuantParams {
   float* sa_sorted;
   uint16_t* ucat;
   float* su_sorted;
+  unsigned* zero_words;  // cleared by the launch (the decode product's tile counters), may be null
+  int n_zero_words;
   int* err;
 };
 cudaError_t launch_route_quant(const RouteQuantParams& q, cudaStream_t st);
@@ -176,6 +178,24 @@ cudaError_t launch_qgemm(int BN, const CUtensorMap& tm_xq, const CUtensorMap& tm
                          const QgemmArgs& a, cudaStream_t st);
 cudaError_t launch_splitk_reduce(const float* partial, int splits, const int32_t* perm, int T, int N, void* Y,
                                  int y_bf16, cudaStream_t st);
+
+// Product of a decode-sized batch (T <= 16): every (output tile, K block) split evenly over the
+// SMs, weights unpacked into TMEM as the MMA's A operand, per-tile fix-up of the segment partials
+// in a fixed order. int8 = W4 x A8/A6 codes (kind::i8); otherwise bf16 activations against W4/W3
+// weights (kind::f16). part/ad/cnt live in the workspace; cnt must be zero at launch (the
+// route/quantize launch clears it, and each launch leaves it zero).
+struct DecodePlan {
+  int NT, KB, grid, maxseg;
+  int64_t NB;
+  size_t part_bytes, ad_bytes;
+  int cnt_words;
+};
+DecodePlan plan_decode(int N, int K, int n_sm);
+int decode_grid_sms();  // SMs of the current device (0 when there is none)
+cudaError_t launch_qdec(int w_bits, bool int8, const CUtensorMap& tm_x, const DecodePlan& plan, const QgemmArgs& q,
+                        const uint16_t* ucat, const uint16_t* bcat, int R_pad, float* part, float* ad,
+                        unsigned* cnt, cudaStream_t st);
+constexpr int kDecodeMaxT = 16;
 
 // Weight-only (W3A16 / W4A16) product on the tensor cores: codes unpacked to bf16, bf16
 // activations (act16, bucket order), per-group fp32 sums scaled by sw, adapter epilogue.

@@ -294,6 +294,39 @@ def test_forward_shapes(T, K, N, group, a_bits, rs, nr, rr, xdt):
     _forward_check(Case(cfg, qi.Projection("p", K, N), T))
 
 
+# Decode-sized batches (T <= 16) take the stream-K decode product: blocks split evenly over the
+# SMs, the weights unpacked into TMEM, a per-tile fix-up of the segment partials. These shapes
+# reach its corners: a K tail of one group (K % 128 = 64 at g = 64), ragged N, one output tile
+# split over 64 CTAs (64 segments), many segments per tile at K = 29568, fewer blocks than SMs,
+# no adapters, five adapter atoms, a single routed expert, A6 and A8 codes, W3 and W4 weight-only.
+DECODE_SHAPES = [
+    # T, K, N, group, a_bits, w_bits, r_s, N_r, r_r, x dtype
+    (1, 320, 200, 64, 8, 4, 8, 4, 4, "f32"),
+    (2, 320, 200, 64, 16, 3, 8, 4, 4, "bf16"),
+    (7, 8192, 128, 128, 8, 4, 32, 8, 4, "bf16"),
+    (16, 8192, 128, 128, 16, 4, 32, 8, 4, "bf16"),
+    (16, 29568, 256, 128, 6, 4, 32, 8, 4, "bf16"),
+    (5, 29568, 256, 128, 16, 3, 32, 8, 4, "bf16"),
+    (16, 1024, 1000, 128, 8, 4, 0, 1, 0, "bf16"),
+    (13, 1024, 640, 128, 6, 4, 32, 8, 32, "bf16"),
+    (16, 1536, 8960, 128, 16, 3, 32, 8, 32, "bf16"),
+    (3, 2048, 4096, 64, 8, 4, 32, 2, 8, "bf16"),
+]
+
+
+@pytest.mark.parametrize("T,K,N,group,a_bits,w_bits,rs,nr,rr,xdt", DECODE_SHAPES)
+def test_forward_decode_batches(T, K, N, group, a_bits, w_bits, rs, nr, rr, xdt):
+    cfg = _cfg(group=group, a_bits=a_bits, w_bits=w_bits, rank_shared=rs, n_routed=nr, rank_routed=rr,
+               x_dtype=xdt, spec="qwen2b" if K >= 1024 else "tiny")
+    c = Case(cfg, qi.Projection("p", K, N), T)
+    assert qe.linear_plan(c.desc, T)["product_k_splits"] == 1
+    Y, _ = _forward_check(c, with_acc=(a_bits != 16))
+    # the fix-up adds the segment partials in a fixed order: repeats are bit-identical
+    for _ in range(2):
+        assert torch.equal(c.gpu_forward(), Y)
+    assert torch.equal(c.gpu_forward(torch.bfloat16), c.gpu_forward().to(torch.bfloat16))
+
+
 @pytest.mark.parametrize("T,K,N,group,bits,rs,nr,rr", [
     (1, 256, 200, 64, 3, 8, 4, 4), (5, 384, 256, 128, 3, 32, 8, 4), (16, 256, 384, 128, 4, 32, 8, 4),
     (33, 512, 136, 64, 3, 0, 2, 8), (4, 1024, 640, 128, 3, 32, 8, 32),
