@@ -11,7 +11,8 @@ pages' construction (whitened SVD of the quantization error) for the
 invariant checks.
 
 Parity status per function (pins live in tests/test_oracle_pins.py):
-  quantize_weights, act_quant  pinned: grid round-trip, per-row RTN at g=K, hand cases
+  quantize_weights, act_quant  pinned: grid round-trip, per-row RTN at g=K, hand cases; fp16 scales:
+                               numpy's binary16 rounding, an on-grid round trip, a hand case
   smoothing_inverse            pinned: nearest fp32 to 1/s (neighbour check in fp64), powers of two exact
   route, bucket                pinned: brute-force argmin / stable sort, permutation
   group_acc                    pinned: bound |acc| <= g*qmax_a*qmax_w, numpy int64
@@ -41,7 +42,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i = ctypes.c_int
-        L.oracle_quantize_weights.argtypes = [P, P, i, i, i, i, P, P, P, P]
+        L.oracle_quantize_weights.argtypes = [P, P, i, i, i, i, i, P, P, P, P]
         L.oracle_act_quant.argtypes = [P, P, i, i, i, P, P]
         L.oracle_route.argtypes = [P, P, i, i, i, P, P]
         L.oracle_bucket.argtypes = [P, i, i, P, P]
@@ -50,6 +51,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_topk.argtypes = [P, P, i, i, i, P, P]
         L.oracle_round_bf16.argtypes = [ctypes.c_float]
         L.oracle_round_bf16.restype = ctypes.c_float
+        L.oracle_round_fp16.argtypes = [ctypes.c_float]
+        L.oracle_round_fp16.restype = ctypes.c_float
         for name in ("oracle_quantize_weights", "oracle_act_quant", "oracle_route", "oracle_bucket",
                      "oracle_group_acc", "oracle_qe_forward", "oracle_topk"):
             getattr(L, name).restype = ctypes.c_int
@@ -72,8 +75,12 @@ def _check(rc: int, what: str):
         raise ValueError(f"oracle {what} rejected its arguments (rc={rc})")
 
 
-def quantize_weights(W, s, group: int, bits: int):
-    """codes [N,K] int8, scales [N,K/group] fp32, w_mean [K], w_colmax [K]."""
+def quantize_weights(W, s, group: int, bits: int, scale_fp16: bool = False):
+    """codes [N,K] int8, scales [N,K/group] fp32, w_mean [K], w_colmax [K].
+
+    scale_fp16: the group scales are stored as fp16 (the fp32 scale rounded to nearest even,
+    saturating at 65504) and the codes are computed from the stored scale; `scales` then holds
+    those fp16 values widened to fp32."""
     W = _f32(W)
     s = _f32(s)
     N, K = W.shape
@@ -81,8 +88,8 @@ def quantize_weights(W, s, group: int, bits: int):
     scales = np.zeros((N, K // group), np.float32)
     w_mean = np.zeros(K, np.float32)
     w_colmax = np.zeros(K, np.float32)
-    _check(lib().oracle_quantize_weights(_p(W), _p(s), N, K, group, bits, _p(codes), _p(scales),
-                                         _p(w_mean), _p(w_colmax)), "quantize_weights")
+    _check(lib().oracle_quantize_weights(_p(W), _p(s), N, K, group, bits, 1 if scale_fp16 else 0, _p(codes),
+                                         _p(scales), _p(w_mean), _p(w_colmax)), "quantize_weights")
     return codes, scales, w_mean, w_colmax
 
 
@@ -185,6 +192,10 @@ def topk(X, w_mean, k: int):
 
 def round_bf16(v: float) -> float:
     return float(lib().oracle_round_bf16(ctypes.c_float(v)))
+
+
+def round_fp16(v: float) -> float:
+    return float(lib().oracle_round_fp16(ctypes.c_float(v)))
 
 
 def qmax(bits: int) -> int:

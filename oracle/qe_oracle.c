@@ -63,6 +63,27 @@ static float round_bf16(float v) {
     return r;
 }
 
+/*
+ * fp32 -> fp16 (IEEE binary16) with round-to-nearest-even, returned widened to fp32: the value is
+ * rounded to a multiple of its binary16 quantum, 2^(e-10) in the normal range (e >= -14, where
+ * 2^e <= |v| < 2^(e+1)) and 2^-24 below it (subnormals). A magnitude that rounds beyond the
+ * largest finite binary16 (65504) saturates to it: the stored scale stays finite (a reading of
+ * the library's; the pages give no fp16 format). Not used on NaN/Inf.
+ */
+static float round_fp16(float v) {
+    if (v == 0.0f) return v;
+    int e;
+    frexpf(v, &e);          /* |v| = m * 2^e, m in [0.5, 1): 2^(e-1) <= |v| < 2^e */
+    e -= 1;
+    if (e < -14) e = -14;   /* subnormal range: quantum 2^-24 */
+    const float quantum = ldexpf(1.0f, e - 10);
+    volatile float q = v / quantum;   /* exact: division by a power of two */
+    float r = rintf(q) * quantum;     /* ties to even */
+    if (r > 65504.0f) r = 65504.0f;
+    if (r < -65504.0f) r = -65504.0f;
+    return r;
+}
+
 /* One symmetric RTN code: clamp(rint(fl32(v / scale)), -qmax, qmax); zero scale -> 0. */
 static int rtn_code(float v, float scale, int qmax) {
     if (scale == 0.0f) return 0;
@@ -75,13 +96,16 @@ static int rtn_code(float v, float scale, int qmax) {
 
 /*
  * Weight quantization with channel scaling (Shared Expert paragraph, DeepRead
- * summary: weights are multiplied by the per-channel factor s).
+ * summary: weights are multiplied by the per-channel factor s). scale_fp16 != 0
+ * stores every group scale as fp16 (an optional byte saving the pages do not
+ * fix: the fp32 scale is rounded to fp16 and the codes are computed from the
+ * stored value).
  *   W [N][K] fp32 values (bf16-stored weights widened exactly), s [K].
  *   codes [N][K] int8, scales [N][K/group] (natural row-major layout),
  *   w_mean [K] = Meanrow(|W|) (mean over the N output rows, fp64 sum, one
  *   rounding), w_colmax [K] = max_o |W[o][k]|.
  */
-int oracle_quantize_weights(const float* W, const float* s, int N, int K, int group, int bits,
+int oracle_quantize_weights(const float* W, const float* s, int N, int K, int group, int bits, int scale_fp16,
                             int8_t* codes, float* scales, float* w_mean, float* w_colmax) {
     if (N <= 0 || K <= 0 || group <= 0 || K % group != 0 || bits < 2 || bits > 8) return ORACLE_BAD_ARG;
     const int qmax = qmax_of(bits);
@@ -95,6 +119,8 @@ int oracle_quantize_weights(const float* W, const float* s, int N, int K, int gr
                 if (a > amax) amax = a;
             }
             volatile float sc = amax / (float)qmax;
+            /* fp16 scales: the stored scale is fp16(sc), and the codes are recomputed from it */
+            if (scale_fp16) sc = round_fp16(sc);
             scales[(size_t)o * G + j] = sc;
             for (int k = j * group; k < (j + 1) * group; ++k) {
                 volatile float ws = W[(size_t)o * K + k] * s[k];
@@ -329,3 +355,5 @@ int oracle_topk(const float* X, const float* w_mean, int T, int K, int k, int32_
 
 /* The bf16 rounding used above, exported so that tests can pin it against torch. */
 float oracle_round_bf16(float v) { return round_bf16(v); }
+/* The fp16 rounding of the weight scales, exported so that tests can pin it against numpy. */
+float oracle_round_fp16(float v) { return round_fp16(v); }

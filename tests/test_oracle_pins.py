@@ -47,6 +47,60 @@ def test_zero_group_gives_zero_scale_and_codes():
     assert codes[1, 4:].tolist() == [2, -3, 5, -7]
 
 
+# ---------------------------------------------------------------- fp16 group scales
+
+def test_fp16_rounding_matches_ieee_binary16():
+    # round to nearest even on the binary16 grid, normal and subnormal, ties included; numpy's
+    # float32 -> float16 cast is IEEE round-to-nearest-even
+    g = np.random.default_rng(11)
+    vals = np.concatenate([
+        g.uniform(-2.0, 2.0, 3000), g.uniform(-60000, 60000, 500), g.uniform(-1e-4, 1e-4, 500),
+        g.uniform(-1e-7, 1e-7, 200),
+        # exact halfway points between neighbouring fp16 values (ties) in the normal and subnormal range
+        (np.arange(1, 200, dtype=np.float32) + np.float32(0.5)) * np.float32(2.0 ** -24),
+        (np.float32(1024) + np.arange(0, 64, dtype=np.float32) + np.float32(0.5)) * np.float32(2.0 ** -10),
+    ]).astype(np.float32)
+    ref = vals.astype(np.float16).astype(np.float32)
+    got = np.array([oracle.round_fp16(float(v)) for v in vals], np.float32)
+    assert (got == ref).all()
+    # beyond the largest finite fp16 the stored scale saturates (it stays finite)
+    assert oracle.round_fp16(70000.0) == 65504.0 and oracle.round_fp16(-1e9) == -65504.0
+
+
+def test_fp16_scales_on_grid_weights_round_trip():
+    # W' = 2^m * q with max |q| = qmax per group: the scale 2^m is exact in fp16 as in fp32,
+    # so the codes come back exactly and the stored scales are the powers of two
+    g = np.random.default_rng(12)
+    for bits in (4, 3):
+        qmax = 2 ** (bits - 1) - 1
+        N, K, grp = 6, 256, 64
+        q = g.integers(-qmax, qmax + 1, size=(N, K))
+        q[:, ::grp] = qmax
+        m = g.integers(-12, 4, size=(N, K // grp))
+        W = (q * 2.0 ** np.repeat(m, grp, axis=1)).astype(np.float32)
+        codes, scales, _, _ = oracle.quantize_weights(W, np.ones(K, np.float32), grp, bits, scale_fp16=True)
+        assert (codes == q).all()
+        assert (scales == (2.0 ** m).astype(np.float32)).all()
+
+
+def test_fp16_scale_recomputes_the_codes():
+    # absmax 1, W4: the fp32 scale fl32(1/7) = 0.142857149 becomes fp16 0.142822265625
+    # (1/7 = 1.142857 * 2^-3; the 10-bit mantissa of 0.142857 * 1024 = 146.29 rounds to 146).
+    # 0.5 / 0.142822265625 = 3.5009 -> 4, where the fp32 scale gives 3.4999998 -> 3; the other
+    # codes are unchanged: 1 -> 7.0017 -> 7, 0.25 -> 1.7504 -> 2.
+    W = np.array([[0.5, -1.0, 0.25, 0.0]], np.float32)
+    c32, s32, _, _ = oracle.quantize_weights(W, np.ones(4, np.float32), 4, 4)
+    c16, s16, _, _ = oracle.quantize_weights(W, np.ones(4, np.float32), 4, 4, scale_fp16=True)
+    assert s16[0, 0] == np.float32(0.142822265625) and s32[0, 0] == np.float32(1.0) / np.float32(7.0)
+    assert c32.tolist() == [[3, -7, 2, 0]] and c16.tolist() == [[4, -7, 2, 0]]
+    # codes stay in range and every scale is an fp16 value
+    g = np.random.default_rng(13)
+    W = g.standard_normal((20, 384)).astype(np.float32) * 0.02
+    codes, scales, _, _ = oracle.quantize_weights(W, np.ones(384, np.float32), 128, 4, scale_fp16=True)
+    assert np.abs(codes).max() <= 7
+    assert (scales.astype(np.float16).astype(np.float32) == scales).all()
+
+
 def test_smoothing_inverse_is_the_nearest_fp32_reciprocal():
     # s_inv = fl32(1/s): no fp32 neighbour of the stored value is closer to the exact 1/s
     # (checked in fp64, where 1/s and the distances are exact enough), and powers of two invert exactly
