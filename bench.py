@@ -64,6 +64,9 @@ WORKLOADS = {
     "decode72b_w3a16_t1": ("decode72b_w3a16", 1, "72B decode gate/up/down, T=1, W3A16 g128"),
     "decode72b_w4a8_t4": ("decode72b_w4a8", 4, "72B decode gate/up/down, T=4, W4A8 g128"),
     "decode72b_w3a16_t4": ("decode72b_w3a16", 4, "72B decode gate/up/down, T=4, W3A16 g128"),
+    "qwen2vl2b_w4a8_s16": ("qwen2vl2b_w4a8_s16", None, "Qwen2VL-2B-shaped layer set, T=2048, W4A8 g128 with fp16 "
+                                                       "group scales, r_s=32, N_r=8, r_r=4"),
+    "decode72b_w4a8_s16": ("decode72b_w4a8_s16", 16, "72B decode gate/up/down, T=16, W4A8 g128, fp16 group scales"),
     "qwen2vl72b_rr32": ("qwen2vl72b_rr32", None, "Qwen2VL-72B-shaped layer set, T=8192, W4A6 g128, routed rank 32 "
                                                  "(ablation)"),
     "qwen2vl72b_rr32_sparse": ("qwen2vl72b_rr32", None, "Qwen2VL-72B-shaped layer set, T=8192, W4A6 g128, routed rank "
@@ -226,7 +229,8 @@ def oracle_layer_set(cfg, n_tokens, seed_shift=0):
     prep = []
     for pi, proj in enumerate(cfg.projections):
         inp = qi.layer_inputs(cfg, proj, T=n_tokens, proj_index=pi + seed_shift)
-        codes, scales, _, _ = oracle.quantize_weights(inp["W"], inp["s"], cfg.group, cfg.w_bits)
+        codes, scales, _, _ = oracle.quantize_weights(inp["W"], inp["s"], cfg.group, cfg.w_bits,
+                                                      scale_fp16=cfg.scale_fp16)
         del inp["W"]
         prep.append((inp, codes, scales))
 
@@ -325,7 +329,7 @@ def build_layers(cfg, T, rank, dev, routed_channels=0):
             x = qi.outlier_activations(T, proj.d_in, replica_x_seed(rank, pi), spec)
             inp["X"] = qi.to_bf16(x) if cfg.x_dtype == "bf16" else x
         desc = qe.make_desc(proj.d_in, proj.d_out, cfg.group, cfg.w_bits, cfg.a_bits, cfg.rank_shared, cfg.n_routed,
-                            cfg.rank_routed, routed_channels)
+                            cfg.rank_routed, routed_channels, cfg.scale_fp16)
 
         def c(a):
             t = torch.from_numpy(np.ascontiguousarray(a)) if isinstance(a, np.ndarray) else a
@@ -483,7 +487,8 @@ def product_roofline(cfg, layers, T, prod_ms, peaks, int8, traffic):
     if T <= 16:
         # decode: HBM bound; the product streams the packed codes, the scales and the adapters
         by = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
-                                      cfg.n_routed, cfg.rank_routed, 1 if not wonly else 2, 2) for L in layers)
+                                      cfg.n_routed, cfg.rank_routed, 1 if not wonly else 2, 2,
+                                      2 if cfg.scale_fp16 else 4) for L in layers)
         ach = by / (prod_ms / 1e3) / 1e9
         return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "kernel": kernel,
@@ -513,7 +518,8 @@ def per_projection(cfg, layers, T, stage_ms):
             "stage_ms": {"project": float(ms[0]), "route_quant": float(ms[1]), "product": float(ms[2])},
             "product_tops": (roofline.int_ops(T, K, N) / (ms[2] / 1e3) / 1e12) if not wonly else None,
             "product_gbs": roofline.layer_bytes(T, K, N, cfg.group, cfg.w_bits, cfg.rank_shared, cfg.n_routed,
-                                                cfg.rank_routed, 1 if not wonly else 2, 2) / (ms[2] / 1e3) / 1e9,
+                                                cfg.rank_routed, 1 if not wonly else 2, 2,
+                                                2 if cfg.scale_fp16 else 4) / (ms[2] / 1e3) / 1e9,
             "layer_tokens_per_s": T / (tot / 1e3),
         })
     return out
@@ -532,7 +538,7 @@ def oracle_baseline(cfg, T, seconds):
 
 # Decode-shaped 72B layers (gate/up/down at T <= 16), measured beside the headline workload:
 # each variant's layers are built once and timed at every T of the list.
-DECODE_SETS = (("decode72b_w4a8", (16, 1)), ("decode72b_w3a16", (16, 1)))
+DECODE_SETS = (("decode72b_w4a8", (16, 1)), ("decode72b_w3a16", (16, 1)), ("decode72b_w4a8_s16", (16, 1)))
 
 
 def run_ours(args, workload):
@@ -588,7 +594,8 @@ def run_ours(args, workload):
         fl += sum(2 * T * L["proj"].d_in * L["proj"].d_out for L in layers)
     xb = 2 if cfg.x_dtype == "bf16" else 4
     nbytes = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
-                                      cfg.n_routed, cfg.rank_routed, xb, 2) for L in layers)
+                                      cfg.n_routed, cfg.rank_routed, xb, 2, 2 if cfg.scale_fp16 else 4)
+                 for L in layers)
     prod_ms = stage_ms[:, :, 2].sum(axis=1).mean()  # the product kernels of one step
     kernel_file = "quantized_gemm_moe_b200/csrc/k_wgemm.cu" if wonly else "quantized_gemm_moe_b200/csrc/k_gemm.cu"
     traffic = read_traffic(kernel_file, ("wgemm_" if wonly else "qgemm_") + workload) if not args.tokens else None
@@ -650,8 +657,9 @@ def run_ours(args, workload):
                 dfile = "quantized_gemm_moe_b200/csrc/" + ("k_wgemm.cu" if dcfg.a_bits == 16 else "k_gemm.cu")
                 dtraffic = read_traffic(dfile, ("wgemm_" if dcfg.a_bits == 16 else "qgemm_") + f"{dname}_t{dT}")
                 decode.append({
-                    "workload": dname, "T": dT, "description": f"72B decode gate/up/down, T={dT}, "
-                                                               f"{'W3A16' if dcfg.w_bits == 3 else 'W4A8'} g128",
+                    "workload": dname, "T": dT,
+                    "description": f"72B decode gate/up/down, T={dT}, {'W3A16' if dcfg.w_bits == 3 else 'W4A8'} g128"
+                                   + (", fp16 group scales" if dcfg.scale_fp16 else ""),
                     "value": world * dT * args.steps / (tot / 1e3), "unit": "tokens/s",
                     "ms_per_step": tot / args.steps,
                     "roofline": product_roofline(dcfg, dl, dT, pm, peaks, int8, dtraffic),

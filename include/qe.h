@@ -83,6 +83,9 @@ typedef struct {
                            /* token-dependent channels): A_r[e] is nonzero only on  */
                            /* k_c channels, given to qe_pack_adapters_sparse.       */
                            /* Needs r_r > 0 and r_s <= 240; k_c <= d_in.           */
+  int32_t w_scale_fp16;    /* 0: fp32 weight group scales; 1: fp16 scales (half the */
+                           /* scale bytes; the codes are computed from the stored  */
+                           /* fp16 scale)                                          */
 } qe_layer_desc;
 
 /*
@@ -105,8 +108,9 @@ typedef struct {
  *     [16+2p, 18+2p), p = 0..7. Bytes 32..47 are four 32-bit words of
  *     high bits: word h holds bit 2 of u for code 32h + 2p at bit p, and for
  *     code 32h + 2p + 1 at bit 16 + p, p = 0..15.
- * w_scale (device, fp32 [d_in/group][d_out], group-major): the weight scale of
- *   (output row o, group j) is w_scale[j*d_out + o].
+ * w_scale (device, [d_in/group][d_out], group-major, fp32; fp16 when
+ *   desc->w_scale_fp16 = 1): the weight scale of (output row o, group j) is
+ *   w_scale[j*d_out + o].
  * s_inv (device, fp32 [d_in]): 1/s, the reciprocal channel smoothing factor.
  * adapters (device, qe_adapter_packed_bytes bytes): produced by
  *   qe_pack_adapters from the natural-layout adapters and router.
@@ -139,7 +143,7 @@ QE_API size_t qe_linear_workspace_bytes(const qe_layer_desc* desc, int32_t T);
  *   W        (device) [d_out, d_in], fp32 or bf16 (w_dtype)
  *   s        (device) fp32 [d_in] smoothing factor (the weights are multiplied by it)
  *   w_packed (device) out, qe_packed_weight_bytes(desc) bytes
- *   w_scale  (device) out, fp32 [d_in/group][d_out]
+ *   w_scale  (device) out, [d_in/group][d_out], fp32 (fp16 with desc->w_scale_fp16)
  *   w_mean   (device) out, fp32 [d_in], may be NULL
  *   w_colmax (device) out, fp32 [d_in] = max_o |W[o][k]|, may be NULL
  *   s_inv    (device) out, fp32 [d_in] = fl32(1/s[k]) (one IEEE division per
@@ -148,7 +152,10 @@ QE_API size_t qe_linear_workspace_bytes(const qe_layer_desc* desc, int32_t T);
  * For each (o, group j): scale = fl32(max_k |fl32(W[o][k]*s[k])| / qmax) and
  * code = clamp(rint(fl32(fl32(W*s)/scale)), -qmax, qmax), with ties to
  * even. A zero scale gives zero codes. qmax = 7 (W4) or 3 (W3). w_mean
- * is summed in fp64 and rounded once.
+ * is summed in fp64 and rounded once. With fp16 scales, the scale is rounded
+ * to fp16 (nearest even) before the codes are computed from it; a scale
+ * above 65504 is stored as 65504 and reported through qe_device_error
+ * (code 0x203).
  */
 QE_API qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, qe_dtype w_dtype, const float* s,
                               void* w_packed, float* w_scale, float* w_mean, float* w_colmax, float* s_inv,

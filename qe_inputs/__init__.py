@@ -170,6 +170,7 @@ class LayerConfig:
     x_dtype: str           # "f32" or "bf16"
     spec: str              # outlier recipe: "tiny" | "qwen2b" | "scaled"
     seed_base: int
+    scale_fp16: bool = False   # weight group scales stored as fp16
 
     def outlier_spec(self, d: int) -> OutlierSpec:
         if self.spec == "tiny":
@@ -221,6 +222,16 @@ CONFIGS = {
         "decode72b_w4a8", 16,
         (Projection("gate", 8192, 29568), Projection("up", 8192, 29568), Projection("down", 29568, 8192)),
         4, 8, 128, 32, 8, 4, 32, "bf16", "scaled", 5),
+    # W4A8 with fp16 group scales (the W4A8 rows of the pages' tables, half the scale bytes)
+    "qwen2vl2b_w4a8_s16": LayerConfig(
+        "qwen2vl2b_w4a8_s16", 2048,
+        (Projection("q", 1536, 1536), Projection("o", 1536, 1536), Projection("gate", 1536, 8960),
+         Projection("up", 1536, 8960), Projection("down", 8960, 1536)),
+        4, 8, 128, 32, 8, 4, 32, "bf16", "qwen2b", 10, True),
+    "decode72b_w4a8_s16": LayerConfig(
+        "decode72b_w4a8_s16", 16,
+        (Projection("gate", 8192, 29568), Projection("up", 8192, 29568), Projection("down", 29568, 8192)),
+        4, 8, 128, 32, 8, 4, 32, "bf16", "scaled", 11, True),
     "decode72b_w3a16": LayerConfig(
         "decode72b_w3a16", 16,
         (Projection("gate", 8192, 29568), Projection("up", 8192, 29568), Projection("down", 29568, 8192)),

@@ -46,7 +46,8 @@ class QEError(RuntimeError):
 class LayerDesc(ctypes.Structure):
     _fields_ = [("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("w_bits", ctypes.c_int32), ("a_bits", ctypes.c_int32), ("rank_shared", ctypes.c_int32),
-                ("n_routed", ctypes.c_int32), ("rank_routed", ctypes.c_int32), ("routed_channels", ctypes.c_int32)]
+                ("n_routed", ctypes.c_int32), ("rank_routed", ctypes.c_int32), ("routed_channels", ctypes.c_int32),
+                ("w_scale_fp16", ctypes.c_int32)]
 
     def __repr__(self):
         return "LayerDesc(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -145,9 +146,11 @@ def _need_cuda(*ts):
 
 
 def make_desc(d_in, d_out, group=128, w_bits=4, a_bits=8, rank_shared=32, n_routed=8, rank_routed=4,
-              routed_channels=0) -> LayerDesc:
-    """routed_channels > 0: cluster-sparse routed experts over that many channels each."""
-    return LayerDesc(d_in, d_out, group, w_bits, a_bits, rank_shared, n_routed, rank_routed, routed_channels)
+              routed_channels=0, w_scale_fp16=0) -> LayerDesc:
+    """routed_channels > 0: cluster-sparse routed experts over that many channels each.
+    w_scale_fp16 = 1: the weight group scales are stored as fp16."""
+    return LayerDesc(d_in, d_out, group, w_bits, a_bits, rank_shared, n_routed, rank_routed, routed_channels,
+                     1 if w_scale_fp16 else 0)
 
 
 # ---------------------------------------------------------------- the C ABI, one wrapper per entry point
@@ -316,7 +319,8 @@ class QELayer:
         dev = W.device
         K, N = desc.d_in, desc.d_out
         w_packed = torch.empty(packed_weight_bytes(desc), dtype=torch.uint8, device=dev)
-        w_scale = torch.empty((K // desc.group, N), dtype=torch.float32, device=dev)
+        w_scale = torch.empty((K // desc.group, N), dtype=torch.float16 if desc.w_scale_fp16 else torch.float32,
+                              device=dev)
         w_mean = torch.empty(K, dtype=torch.float32, device=dev)
         w_colmax = torch.empty(K, dtype=torch.float32, device=dev)
         s_inv_out = torch.empty(K, dtype=torch.float32, device=dev) if s_inv is None else None

@@ -62,7 +62,8 @@ struct DCfg {
 
 struct DecArgs {
   const uint8_t* w_packed;
-  const float* w_scale;     // [G][N]
+  const float* w_scale;     // [G][N] fp32, or fp16 when sw_f16
+  int sw_f16;
   const float* sa_sorted;   // [T]
   const float* su_sorted;   // [T] or nullptr (no adapters)
   const int32_t* perm;      // [T]
@@ -366,8 +367,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const int o = nt * kTileN + r;
       if (o >= a.N) return;
       const int j = kb * gpb;
-      s0 = __ldg(a.w_scale + static_cast<size_t>(j) * a.N + o);
-      if (gpb == 2 && j + 1 < a.G_total) s1 = __ldg(a.w_scale + static_cast<size_t>(j + 1) * a.N + o);
+      s0 = load_scale(a.w_scale, static_cast<size_t>(j) * a.N + o, a.sw_f16);
+      if (gpb == 2 && j + 1 < a.G_total) s1 = load_scale(a.w_scale, static_cast<size_t>(j + 1) * a.N + o, a.sw_f16);
     };
 #pragma unroll
     for (int k = 0; k < kDSwAhead; ++k) load_sw(k, sw0[k], sw1[k]);
@@ -622,6 +623,7 @@ cudaError_t launch_qdec(int w_bits, bool int8, const CUtensorMap& tm_x, const De
   DecArgs a{};
   a.w_packed = q.w_packed;
   a.w_scale = q.w_scale;
+  a.sw_f16 = q.sw_f16;
   a.sa_sorted = q.sa_sorted;
   a.su_sorted = q.su_sorted;
   a.perm = q.perm;

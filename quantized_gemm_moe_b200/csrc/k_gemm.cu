@@ -526,11 +526,11 @@ __global__ void __launch_bounds__(512, 1)
       // weight codes enter the MMA as 16*q, so the group scale is applied as sw/16 (exact).
       // The scales are loaded kSwAhead groups ahead (a load can outlast a group's drain).
       constexpr int kSwAhead = 2;
-      const float* swp = a.w_scale + static_cast<size_t>(w.g_begin) * a.N + o;
+      const size_t sw0 = static_cast<size_t>(w.g_begin) * a.N + o;  // scale of (o, first group)
       float swq[kSwAhead];
 #pragma unroll
       for (int j = 0; j < kSwAhead; ++j)
-        swq[j] = (o_ok && j < w.n_groups) ? __ldg(swp + static_cast<size_t>(j) * a.N) : 0.0f;
+        swq[j] = (o_ok && j < w.n_groups) ? load_scale(a.w_scale, sw0 + static_cast<size_t>(j) * a.N, a.sw_f16) : 0.0f;
       for (int g = 0; g < w.n_groups; ++g) {
         uint32_t use;
         const int b = epi_next_buffer<kOwn>(bstate, static_cast<int>(bstate & 1u), use);
@@ -539,7 +539,9 @@ __global__ void __launch_bounds__(512, 1)
         const uint64_t sw2 = pack2(swq[0] * 0.0625f);
 #pragma unroll
         for (int j = 0; j + 1 < kSwAhead; ++j) swq[j] = swq[j + 1];
-        swq[kSwAhead - 1] = (o_ok && g + kSwAhead < w.n_groups) ? __ldg(swp + static_cast<size_t>(g + kSwAhead) * a.N) : 0.0f;
+        swq[kSwAhead - 1] = (o_ok && g + kSwAhead < w.n_groups)
+                                ? load_scale(a.w_scale, sw0 + static_cast<size_t>(g + kSwAhead) * a.N, a.sw_f16)
+                                : 0.0f;
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], use & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (!ok) continue;
         tc_fence_after();

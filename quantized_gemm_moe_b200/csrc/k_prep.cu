@@ -338,10 +338,13 @@ __global__ void __launch_bounds__(256) k_act_quant(const void* __restrict__ X, c
 // ------------------------------------------------------------------ weight quantization + packing
 // One CTA per (128-row tile, 128-channel block), thread = row. Two passes over
 // the block: group absmax -> scale, then codes, packed 32 codes at a time.
+// With fp16 scales (s16), each group scale is rounded to fp16 (nearest even) and the codes are
+// computed from the stored value; a scale beyond the fp16 range is saturated to 65504 and
+// reported (device error 0x203).
 template <bool BF16, int BITS>
 __global__ void __launch_bounds__(128) k_quant_w(const void* __restrict__ W, const float* __restrict__ s, int N,
                                                  int K, int group, uint8_t* __restrict__ packed,
-                                                 float* __restrict__ w_scale) {
+                                                 void* __restrict__ w_scale, int s16, int* err) {
   constexpr int qmax = (1 << (BITS - 1)) - 1;
   const int nt = blockIdx.x, kb = blockIdx.y, r = threadIdx.x;
   const int o = nt * kTileN + r;
@@ -362,7 +365,18 @@ __global__ void __launch_bounds__(128) k_quant_w(const void* __restrict__ W, con
     float amax = 0.0f;
     for (int k = k0; k < k0 + group; ++k) amax = fmaxf(amax, fabsf(wval(k)));
     sc[gi] = __fdiv_rn(amax, static_cast<float>(qmax));
-    if (row_ok) w_scale[static_cast<size_t>(k0 / group) * N + o] = sc[gi];
+    const size_t at = static_cast<size_t>(k0 / group) * N + o;
+    if (s16) {
+      __half h = __float2half_rn(sc[gi]);
+      if (__hisinf(h)) {
+        h = __ushort_as_half(static_cast<unsigned short>(0x7BFFu));  // 65504
+        if (row_ok) record_error(err, 0x203);
+      }
+      sc[gi] = __half2float(h);
+      if (row_ok) static_cast<__half*>(w_scale)[at] = h;
+    } else if (row_ok) {
+      static_cast<float*>(w_scale)[at] = sc[gi];
+    }
   }
   const size_t block = static_cast<size_t>(nt) * KB + kb;
   for (int h = 0; h < 4; ++h) {  // 32 codes at a time
@@ -1034,14 +1048,15 @@ cudaError_t launch_act_quant(const void* X, bool x_bf16, const float* s_inv, int
 }
 
 cudaError_t launch_quantize_weights(const void* W, bool w_bf16, const float* s, int N, int K, int group,
-                                    int w_bits, uint8_t* packed, float* w_scale, cudaStream_t st) {
+                                    int w_bits, uint8_t* packed, void* w_scale, int s16, int* err,
+                                    cudaStream_t st) {
   dim3 grid(static_cast<unsigned>(ceil_div(N, kTileN)), static_cast<unsigned>(ceil_div(K, kTileK)));
   if (w_bits == 4) {
-    if (w_bf16) k_quant_w<true, 4><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale);
-    else k_quant_w<false, 4><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale);
+    if (w_bf16) k_quant_w<true, 4><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale, s16, err);
+    else k_quant_w<false, 4><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale, s16, err);
   } else {
-    if (w_bf16) k_quant_w<true, 3><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale);
-    else k_quant_w<false, 3><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale);
+    if (w_bf16) k_quant_w<true, 3><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale, s16, err);
+    else k_quant_w<false, 3><<<grid, 128, 0, st>>>(W, s, N, K, group, packed, w_scale, s16, err);
   }
   return cudaGetLastError();
 }

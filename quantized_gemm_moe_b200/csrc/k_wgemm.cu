@@ -455,15 +455,15 @@ __global__ void __launch_bounds__(512, 1)
       float acc[EC];
 #pragma unroll
       for (int c = 0; c < EC; ++c) acc[c] = 0.0f;
-      const float* swp = a.w_scale + static_cast<size_t>(w.g_begin) * a.N + o;
-      float sw_next = (o_ok && w.n_groups > 0) ? __ldg(swp) : 0.0f;
+      const size_t sw0 = static_cast<size_t>(w.g_begin) * a.N + o;  // scale of (o, first group)
+      float sw_next = (o_ok && w.n_groups > 0) ? load_scale(a.w_scale, sw0, a.sw_f16) : 0.0f;
       for (int g = 0; g < w.n_groups; ++g) {
         uint32_t use;
         const int b = epi_next_buffer<kOwn>(bstate, static_cast<int>(bstate & 1u), use);
         // bit 0 follows the stage parity: flip it after the last group of each K block
         if (a.group == kTileK || (g & 1) || g + 1 == w.n_groups) bstate ^= 1u;
         const float sw = sw_next;
-        if (o_ok && g + 1 < w.n_groups) sw_next = __ldg(swp + static_cast<size_t>(g + 1) * a.N);
+        if (o_ok && g + 1 < w.n_groups) sw_next = load_scale(a.w_scale, sw0 + static_cast<size_t>(g + 1) * a.N, a.sw_f16);
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[b], use & 1, a_err, DEVERR_WAIT_EPILOGUE));
         if (!ok) continue;
         tc_fence_after();

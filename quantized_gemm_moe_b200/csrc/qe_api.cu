@@ -45,6 +45,7 @@ qe_status check_desc(const qe_layer_desc* d) {
   if (d->routed_channels < 0 || d->routed_channels > d->d_in) return QE_ERR_INVALID_ARG;
   if (d->routed_channels > 0 && (d->rank_routed == 0 || sparse_gemm_width(d->rank_shared) == 0))
     return QE_ERR_UNSUPPORTED;
+  if (d->w_scale_fp16 != 0 && d->w_scale_fp16 != 1) return QE_ERR_INVALID_ARG;
   return QE_OK;
 }
 
@@ -313,6 +314,7 @@ qe_status forward_impl(const qe_layer_desc* d, const qe_layer_weights* w, const 
     QgemmArgs a{};
     a.w_packed = static_cast<const uint8_t*>(w->w_packed);
     a.w_scale = w->w_scale;
+    a.sw_f16 = d->w_scale_fp16;
     a.sa_sorted = sa_sorted;
     a.su_sorted = p.has_ad ? su_sorted : nullptr;
     a.perm = perm;
@@ -417,7 +419,8 @@ qe_status qe_quantize_weights(const qe_layer_desc* desc, const void* W, qe_dtype
     return QE_ERR_ALIGNMENT;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   QE_CUDA(launch_quantize_weights(W, w_dtype == QE_BF16, s, desc->d_out, desc->d_in, desc->group, desc->w_bits,
-                                  static_cast<uint8_t*>(w_packed), w_scale, cs),
+                                  static_cast<uint8_t*>(w_packed), w_scale, desc->w_scale_fp16,
+                                  device_error_ptr(), cs),
           "quantize_weights");
   if (w_mean || w_colmax)
     QE_CUDA(launch_colstats(W, w_dtype == QE_BF16, desc->d_out, desc->d_in, w_mean, w_colmax, cs), "colstats");

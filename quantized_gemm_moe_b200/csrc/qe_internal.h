@@ -71,8 +71,10 @@ inline AdapterGeom adapter_geom(int K, int N, int r_s, int n_r, int r_r, int kc)
 // ------------------------------------------------------------------ kernel launchers
 // Each returns the launch's cudaError_t. The host API validates before calling.
 
+// w_scale: fp32 [G][N], or fp16 when s16 != 0 (a scale beyond fp16 is saturated, device error 0x203).
 cudaError_t launch_quantize_weights(const void* W, bool w_bf16, const float* s, int N, int K, int group,
-                                    int w_bits, uint8_t* packed, float* w_scale, cudaStream_t st);
+                                    int w_bits, uint8_t* packed, void* w_scale, int s16, int* err,
+                                    cudaStream_t st);
 cudaError_t launch_colstats(const void* W, bool w_bf16, int N, int K, float* w_mean, float* w_colmax,
                             cudaStream_t st);
 // s_inv[k] = fl32(1/s[k]) (IEEE division).
@@ -159,7 +161,8 @@ cudaError_t launch_route_quant(const RouteQuantParams& q, cudaStream_t st);
 // per-token scale, adapter MMA in the epilogue and scatter to token order.
 struct QgemmArgs {
   const uint8_t* w_packed;
-  const float* w_scale;     // [G][N]
+  const float* w_scale;     // [G][N] fp32, or fp16 when sw_f16
+  int sw_f16;
   const float* sa_sorted;   // [T]
   const float* su_sorted;   // [T] adapter scale of U_cat rows
   const int32_t* perm;      // [T]

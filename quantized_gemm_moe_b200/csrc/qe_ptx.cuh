@@ -98,6 +98,17 @@ __device__ __forceinline__ int epi_next_buffer(uint32_t& st, int iq, uint32_t& u
   return iq + 2 * static_cast<int>(oc % kOwn);
 }
 
+// Group scale idx of a [G][N] table stored as fp32, or as fp16 when f16 != 0 (read-only path).
+__device__ __forceinline__ float load_scale(const float* base, size_t idx, int f16) {
+  if (f16) {
+    const unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(base) + idx);
+    float f;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
+    return f;
+  }
+  return __ldg(base + idx);
+}
+
 // Before a CTA exits, the thread that issued a ring's loads waits (bounded) for the last `depth`
 // of its `issued` loads to land: after a wait ran out, their consumer may have stopped, and a
 // copy must not land in the shared memory of a CTA that has exited. On a normal run these

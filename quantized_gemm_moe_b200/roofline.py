@@ -7,7 +7,7 @@ Counts are of what the method must do, not of what a kernel happens to move:
   2*T*(K+N)*r_s, the routed expert 2*T*(K+N)*r_r (one expert per token), and
   the router 2*T*K*N_r.
 * bytes: X once (2 B per element for bf16), the packed codes (b_w/8 B per weight),
-  fp32 group scales, the shared adapters, the routed adapters that are touched
+  the group scales (fp32, or fp16), the shared adapters, the routed adapters that are touched
   (at most min(T, N_r) experts), the router, and Y once.
 With d_in = d_out = d and r_s = r_r = r/2, (int ops + bf16 flops)/2 equals the
 QE row of the complexity table on the thelatestinai listing (Table 7):
@@ -25,8 +25,9 @@ def adapter_flops(T: int, K: int, N: int, r_s: int, n_r: int, r_r: int) -> int:
 
 
 def layer_bytes(T: int, K: int, N: int, group: int, w_bits: int, r_s: int, n_r: int, r_r: int,
-                x_bytes: int = 2, y_bytes: int = 2) -> int:
-    return (x_bytes * T * K + (K * N * w_bits) // 8 + 4 * N * (K // group) + 2 * (K + N) * r_s
+                x_bytes: int = 2, y_bytes: int = 2, scale_bytes: int = 4) -> int:
+    """scale_bytes: 4 for fp32 group scales, 2 for fp16."""
+    return (x_bytes * T * K + (K * N * w_bits) // 8 + scale_bytes * N * (K // group) + 2 * (K + N) * r_s
             + min(T, n_r) * 2 * (K + N) * r_r + 2 * K * n_r + y_bytes * T * N)
 
 

@@ -51,7 +51,7 @@ class Case:
         self.T = T
         self.inp = inp if inp is not None else qi.layer_inputs(cfg, proj, T=T, proj_index=proj_index)
         self.desc = qe.make_desc(proj.d_in, proj.d_out, cfg.group, cfg.w_bits, cfg.a_bits, cfg.rank_shared,
-                                 cfg.n_routed, cfg.rank_routed, routed_channels)
+                                 cfg.n_routed, cfg.rank_routed, routed_channels, cfg.scale_fp16)
         i = self.inp
         self.Xd = cuda(i["X"])
         if routed_channels:
@@ -70,7 +70,8 @@ class Case:
 
     def oracle_weights(self):
         if self._ref is None:
-            self._ref = oracle.quantize_weights(self.inp["W"], self.inp["s"], self.cfg.group, self.cfg.w_bits)
+            self._ref = oracle.quantize_weights(self.inp["W"], self.inp["s"], self.cfg.group, self.cfg.w_bits,
+                                                scale_fp16=self.cfg.scale_fp16)
         return self._ref
 
     def oracle_forward(self, rows=None, expert_override=None):

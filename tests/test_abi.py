@@ -178,7 +178,7 @@ C_CLIENT = r"""
 #include "qe.h"
 #include <stdio.h>
 int main(void) {
-  qe_layer_desc d = {1536, 1536, 128, 4, 6, 32, 8, 4, 0};
+  qe_layer_desc d = {1536, 1536, 128, 4, 6, 32, 8, 4, 0, 0};
   qe_linear_plan_info p;
   qe_status s = qe_linear_plan(&d, 2048, QE_BF16, &p);
   printf("%d %s %d %d %zu %d\n", (int)s, qe_status_string(s), p.product_tile_tokens, p.adapter_atoms,

@@ -23,18 +23,20 @@ def _cfg(base="tiny", **kw):
 
 # ---------------------------------------------------------------- weight quantization
 
-@pytest.mark.parametrize("N,K,group,bits,wdt", [
-    (256, 256, 64, 4, "f32"), (200, 384, 64, 4, "bf16"), (1536, 1536, 128, 4, "bf16"),
-    (300, 256, 128, 3, "bf16"), (256, 320, 64, 3, "f32"), (8960, 1536, 128, 4, "bf16"),
+@pytest.mark.parametrize("N,K,group,bits,wdt,s16", [
+    (256, 256, 64, 4, "f32", 0), (200, 384, 64, 4, "bf16", 0), (1536, 1536, 128, 4, "bf16", 0),
+    (300, 256, 128, 3, "bf16", 0), (256, 320, 64, 3, "f32", 0), (8960, 1536, 128, 4, "bf16", 0),
+    # fp16 group scales: the codes come from the stored fp16 scale
+    (8960, 1536, 128, 4, "bf16", 1), (200, 384, 64, 4, "f32", 1), (300, 256, 128, 3, "bf16", 1),
 ])
-def test_weight_quantization_bit_exact(N, K, group, bits, wdt):
+def test_weight_quantization_bit_exact(N, K, group, bits, wdt, s16):
     cfg = _cfg(group=group, w_bits=bits, a_bits=8 if bits == 4 else 16, x_dtype=wdt)
     inp = qi.layer_inputs(cfg, qi.Projection("w", K, N), T=4)
-    codes, scales, w_mean, colmax = oracle.quantize_weights(inp["W"], inp["s"], group, bits)
-    desc = qe.make_desc(K, N, group, bits, cfg.a_bits, 8, 4, 4)
+    codes, scales, w_mean, colmax = oracle.quantize_weights(inp["W"], inp["s"], group, bits, scale_fp16=bool(s16))
+    desc = qe.make_desc(K, N, group, bits, cfg.a_bits, 8, 4, 4, w_scale_fp16=s16)
     Wd = cuda(inp["W"])
     wp = torch.empty(qe.packed_weight_bytes(desc), dtype=torch.uint8, device="cuda")
-    ws = torch.empty((K // group, N), dtype=torch.float32, device="cuda")
+    ws = torch.empty((K // group, N), dtype=torch.float16 if s16 else torch.float32, device="cuda")
     wm = torch.empty(K, dtype=torch.float32, device="cuda")
     wc = torch.empty(K, dtype=torch.float32, device="cuda")
     si = torch.empty(K, dtype=torch.float32, device="cuda")
@@ -43,7 +45,7 @@ def test_weight_quantization_bit_exact(N, K, group, bits, wdt):
     qe.unpack_weights(desc, wp, got)
     torch.cuda.synchronize()
     assert (got.cpu().numpy() == codes).all()
-    assert (ws.cpu().numpy().T == scales).all()
+    assert (ws.float().cpu().numpy().T == scales).all()
     assert (wc.cpu().numpy() == colmax).all()
     # the stored smoothing factor is the correctly rounded fp32 reciprocal of s
     assert (si.cpu().numpy() == (np.float32(1.0) / inp["s"]).astype(np.float32)).all()
@@ -500,6 +502,28 @@ def test_full_size_qwen2vl72b_routed_rank32(proj_index, routed_channels):
     for _ in range(3):
         assert torch.equal(c.gpu_forward(), Y)
     assert qe.device_error() == 0
+
+
+@pytest.mark.parametrize("proj_index", range(5))
+def test_full_size_qwen2vl2b_w4a8_fp16_scales(proj_index):
+    # W4A8 with fp16 group scales, the 2B layer set at T = 2048
+    _full_size("qwen2vl2b_w4a8_s16", proj_index)
+
+
+@pytest.mark.parametrize("T", [1, 16])
+@pytest.mark.parametrize("proj_index", [0, 2])
+def test_full_size_decode_w4a8_fp16_scales(T, proj_index):
+    cfg = qi.CONFIGS["decode72b_w4a8_s16"].with_(T=T)
+    c = Case(cfg, cfg.projections[proj_index], T, proj_index=proj_index)
+    _forward_check(c, with_acc=False)
+
+
+@pytest.mark.parametrize("T,K,N,group,a_bits", [(16, 1024, 640, 64, 8), (300, 512, 2048, 128, 6), (3, 384, 200, 64, 6)])
+def test_forward_fp16_scales_small(T, K, N, group, a_bits):
+    # every accumulator bit-exact with codes computed from fp16 scales (prefill and decode kernels)
+    cfg = _cfg(group=group, a_bits=a_bits, rank_shared=32, n_routed=8, rank_routed=4, x_dtype="bf16",
+               spec="qwen2b" if K >= 1024 else "tiny", scale_fp16=True)
+    _forward_check(Case(cfg, qi.Projection("p", K, N), T))
 
 
 @pytest.mark.parametrize("cfg_name", ["qwen2vl2b_w4a16", "qwen2vl2b_w3a16"])
