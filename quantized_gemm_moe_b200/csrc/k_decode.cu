@@ -11,22 +11,24 @@
 // and writes Y.
 //
 // Per 128 x 128 weight block:
-//   warp 0      bulk copy of the packed block and TMA of the activation tile (16 tokens x 128
-//               channels) into a 10-deep ring: up to 80 KB of weights in flight per SM
+//   warp 0      bulk copies of the packed block and of its group-scale slabs, and TMA of the
+//               activation tile (16 tokens x 128 channels), into a 14-16 deep ring: up to 128 KB
+//               of weights in flight per SM. The epilogue frees a slot once it has read the scales.
 //   warps 4-11  unpack the block straight into tensor memory with tcgen05.st: the MMA takes its
 //               A operand (the weights, M = 128 output rows = TMEM lanes, K along the columns)
 //               from TMEM, so the unpacked weights never pass through shared memory (whose
-//               bandwidth the unpack would otherwise exceed at the HBM rate). Two warps per TMEM
-//               lane quarter, each one half of the block's columns.
+//               bandwidth the unpack would otherwise exceed at the HBM rate). Two teams of four
+//               warps (one per TMEM lane quarter) take alternate blocks, a full row per thread.
 //   warps 1-2   one thread each issues the MMAs of alternate blocks: kind::i8 (codes x16 against
 //               int8 activation codes, 4 K steps) or kind::f16 (bf16 weights against bf16
 //               activations, 8 K steps). Every quantization group gets a fresh 16-column
 //               accumulator (the first K step does not accumulate), issuer q owning slots
 //               q, q+2, ...
+//   warp 3      the adapter term U_cat . B_catT of every tile whose first block this CTA streams,
+//               on CUDA cores (fp16 inputs, fp32 sums), written to the workspace off the epilogue's path
 //   warps 12-15 epilogue, one output row per thread: per group acc += sw * group sum (the int8
-//               sums converted exactly), with the scales loaded six blocks ahead; the adapter term
-//               of a tile on CUDA cores (fp16 inputs, fp32 sums) in the CTA that holds its first
-//               block; the segment partials and the per-tile fix-up.
+//               sums converted exactly, the scale read from the ring slot); the segment partials
+//               and the per-tile fix-up.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -40,10 +42,8 @@ namespace {
 
 constexpr int kDN = 16;          // token columns: the whole batch, padded (MMA N)
 constexpr int kDThreads = 512;   // 16 warps
-constexpr int kDStages = 10;     // packed block + activation tile ring
 constexpr int kDASlots = 4;      // unpacked A blocks in TMEM
 constexpr int kDTmemCols = 512;
-constexpr int kDSwAhead = 6;     // blocks of group scales in flight per epilogue thread
 
 template <bool I8, int BITS>
 struct DCfg {
@@ -55,7 +55,14 @@ struct DCfg {
   static constexpr int kAccSlots = (kDTmemCols - kDASlots * kACols) / kDN;  // 24 (int8) / 16 (bf16)
   static constexpr int kOwn = kAccSlots / 2;              // accumulator slots per issuer
   static constexpr int kUcatBytes = kDN * 512 * 2;        // U_cat staging, R_pad <= 512
-  static constexpr size_t kSmem = 1024 + size_t(kDStages) * kXTile + size_t(kDStages) * kWBlock + kUcatBytes + 1024;
+  static constexpr int kSBlock = 2 * 128 * 4;             // group scale slabs of a block (2 groups x 128 rows)
+  // Ring of blocks in flight (packed block + activation tile + scale slabs), even so that each
+  // unpack team keeps its own slots. A slot is freed once the epilogue has read its scales, so
+  // the ring spans the whole pipeline from the load to the drained group.
+  static constexpr int kStages = (I8 || BITS == 3) ? 16 : 14;
+  static constexpr size_t kSmem =
+      1024 + size_t(kStages) * (kXTile + kWBlock + kSBlock) + kUcatBytes + 1024;
+  static_assert(kStages % 2 == 0, "each unpack team keeps its own ring slots");
   static_assert(kAccSlots % 2 == 0, "each issuer owns half of the accumulator slots");
   static_assert(kSmem <= 232448, "shared memory");
 };
@@ -63,7 +70,8 @@ struct DCfg {
 struct DecArgs {
   const uint8_t* w_packed;
   const float* w_scale;     // [G][N] fp32, or fp16 when sw_f16
-  int sw_f16;
+  int sw_f16, sw_elem;      // scale bytes: 4 or 2
+  int sw_vec;               // N * sw_elem is a multiple of 16: slabs travel with the blocks
   const float* sa_sorted;   // [T]
   const float* su_sorted;   // [T] or nullptr (no adapters)
   const int32_t* perm;      // [T]
@@ -90,6 +98,18 @@ __host__ __device__ __forceinline__ int64_t range_begin(int c, int64_t NB, int G
 __host__ __device__ __forceinline__ int cta_of(int64_t f, int64_t NB, int G) {
   return static_cast<int>(((f + 1) * G - 1) / NB);
 }
+
+// (output tile, K block) of consecutive blocks, advanced without divisions (a 64-bit division per
+// block costs hundreds of cycles on a role's critical path).
+struct BlockPos {
+  int nt, kb;
+  __device__ __forceinline__ void next(int KB) {
+    if (++kb == KB) {
+      kb = 0;
+      ++nt;
+    }
+  }
+};
 
 __device__ __forceinline__ void mma_i8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -208,21 +228,23 @@ template <bool I8, int BITS>
 __global__ void __launch_bounds__(kDThreads, 1)
     k_qdec(const __grid_constant__ CUtensorMap tm_x, const DecArgs a) {
   using C = DCfg<I8, BITS>;
-  constexpr int NS = kDStages, NA = kDASlots;
+  constexpr int NS = C::kStages, NA = kDASlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xring = smem;                              // [NS][kXTile], 1024-aligned (128B swizzle)
   uint8_t* wring = xring + NS * C::kXTile;            // [NS][kWBlock]
-  __half* ucat_s = reinterpret_cast<__half*>(wring + NS * C::kWBlock);  // [16][R_pad]
+  uint8_t* sring = wring + NS * C::kWBlock;           // [NS][2 groups][128 rows] group scales
+  __half* ucat_s = reinterpret_cast<__half*>(sring + NS * C::kSBlock);  // [16][R_pad]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ucat_s) + C::kUcatBytes);
-  uint64_t* wfull = bars;                  // [NS] block + tile landed (1 + bytes)
-  uint64_t* wempty = wfull + NS;           // [NS] the MMAs of the block are done (ring slot free)
-  uint64_t* afull = wempty + NS;           // [NA] A unpacked into TMEM (8 unpack warps)
+  uint64_t* wfull = bars;                  // [NS] block, tile and scales landed (1 + bytes)
+  uint64_t* wempty = wfull + NS;           // [NS] the epilogue read the block's scales (its MMAs are done)
+  uint64_t* afull = wempty + NS;           // [NA] A unpacked into TMEM (the 4 warps of a team)
   uint64_t* aempty = afull + NA;           // [NA] the MMAs of the block are done (A slot free)
   uint64_t* accf = aempty + NA;            // [kAccSlots] group sum ready
   uint64_t* acce = accf + C::kAccSlots;    // [kAccSlots] group sum read (4 epilogue warps)
   uint64_t* done = acce + C::kAccSlots;    // teardown
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* adready = done + 1;            // the adapter terms of this CTA's tiles are in memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(adready + 1);
   int* flag_s = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -230,15 +252,19 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const int64_t b0 = range_begin(c, a.NB, G), b1 = range_begin(c + 1, a.NB, G);
   const int nblk = static_cast<int>(b1 - b0);
   const int gpb = kTileK / a.group;
+  const BlockPos pos0{static_cast<int>(b0 / a.KB), static_cast<int>(b0 % a.KB)};
   int* const a_err = a.err;
+  // tiles whose first block lies in this CTA's range: their adapter terms are computed here
+  const int nt_ad0 = static_cast<int>((b0 + a.KB - 1) / a.KB), nt_ad1 = static_cast<int>((b1 - 1) / a.KB);
+  const bool any_ad = a.su_sorted != nullptr && nt_ad0 <= nt_ad1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 1);
+      mbar_init(&wempty[s], 4);
     }
     for (int s = 0; s < NA; ++s) {
-      mbar_init(&afull[s], 8);
+      mbar_init(&afull[s], 4);
       mbar_init(&aempty[s], 1);
     }
     for (int b = 0; b < C::kAccSlots; ++b) {
@@ -246,6 +272,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
       mbar_init(&acce[b], 4);
     }
     mbar_init(done, 2);
+    mbar_init(adready, 1);
     mbar_fence_init();
     prefetch_tmap(&tm_x);
   }
@@ -264,15 +291,26 @@ __global__ void __launch_bounds__(kDThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int i = 0;
-      for (; i < nblk; ++i) {
+      BlockPos bp = pos0;
+      for (; i < nblk; ++i, bp.next(a.KB)) {
         const int s = i % NS;
         if (!mbar_wait(&wempty[s], ((i / NS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) break;
-        const int64_t f = b0 + i;
-        const int kb = static_cast<int>(f % a.KB);
-        mbar_arrive_expect_tx(&wfull[s], C::kWBlock + C::kXTile);
-        bulk_load(wring + s * C::kWBlock, a.w_packed + f * C::kWBlock, C::kWBlock, &wfull[s]);
+        const int kb = bp.kb;
+        // the 128-row scale slab of each of the block's groups (contiguous: group-major [G][N])
+        const int ng = min(gpb, a.G_total - kb * gpb);
+        const uint32_t sbytes = a.sw_vec ? static_cast<uint32_t>(128 * a.sw_elem) : 0u;
+        const int o0 = bp.nt * kTileN;
+        const uint32_t svalid = min(128, a.N - o0) * a.sw_elem;  // the last tile's slab stops at d_out
+        const uint32_t scopy = sbytes ? ((svalid + 15u) & ~15u) : 0u;
+        mbar_arrive_expect_tx(&wfull[s], C::kWBlock + C::kXTile + ng * scopy);
+        bulk_load(wring + s * C::kWBlock, a.w_packed + (b0 + i) * C::kWBlock, C::kWBlock, &wfull[s]);
         tma_load_2d(xring + s * C::kXTile, &tm_x, kb * kTileK, 0, &wfull[s]);
         if constexpr (!I8) tma_load_2d(xring + s * C::kXTile + C::kXAtom, &tm_x, kb * kTileK + 64, 0, &wfull[s]);
+        for (int gi = 0; gi < (scopy ? ng : 0); ++gi)
+          bulk_load(sring + s * C::kSBlock + gi * 512,
+                    reinterpret_cast<const uint8_t*>(a.w_scale) +
+                        (static_cast<size_t>(kb * gpb + gi) * a.N + o0) * a.sw_elem,
+                    scopy, &wfull[s]);
       }
       drain_ring(wfull, NS, i);
     }
@@ -284,10 +322,11 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xring));
       int own = 0;
       bool ok = true;
-      for (int i = qi; i < nblk && ok; i += 2) {
+      BlockPos bp = pos0;
+      if (qi) bp.next(a.KB);
+      for (int i = qi; i < nblk && ok; i += 2, bp.next(a.KB), bp.next(a.KB)) {
         const int s = i % NS, as = i % NA;
-        const int64_t f = b0 + i;
-        const int kb = static_cast<int>(f % a.KB);
+        const int kb = bp.kb;
         const int ng = min(gpb, a.G_total - kb * gpb);
         if (!mbar_wait(&afull[as], (i / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
           ok = false;
@@ -322,24 +361,86 @@ __global__ void __launch_bounds__(kDThreads, 1)
           tc_commit(&accf[slot]);
         }
         tc_commit(&aempty[as]);
-        tc_commit(&wempty[s]);
       }
       tc_commit(done);
       mbar_wait(done, 0, a_err, DEVERR_WAIT_TEARDOWN);
     }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ adapter terms (CUDA cores)
+    // ad[nt][r][p] = sum_j B_catT[o][j] * U_cat[p][j] (fp16 inputs, fp32 sums) for every tile whose
+    // first block this CTA streams; lane l takes rows l, l+32, l+64, l+96. Off the epilogue's path:
+    // the segment holding the tile's first block waits on adready only when it finishes.
+    if (any_ad) {
+      const int rp = a.R_pad, T = a.T;
+      for (int e = lane; e < kDN * rp / 8; e += 32) {
+        const int p = e / (rp / 8), c8 = e % (rp / 8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (p < T) v = __ldg(reinterpret_cast<const uint4*>(a.ucat + static_cast<size_t>(p) * rp) + c8);
+        *reinterpret_cast<uint4*>(ucat_s + static_cast<size_t>(p) * rp + c8 * 8) = v;
+      }
+      __syncwarp();
+      for (int nt = nt_ad0; nt <= nt_ad1; ++nt) {
+        for (int rr = 0; rr < 4; ++rr) {
+          const int r = lane + 32 * rr;
+          const int o = nt * kTileN + r;
+          float adr[kDN];
+#pragma unroll
+          for (int p = 0; p < kDN; ++p) adr[p] = 0.0f;
+          if (o < a.N) {
+            const uint4* brow = reinterpret_cast<const uint4*>(a.bcat + static_cast<size_t>(o) * rp);
+            for (int c0 = 0; c0 < rp / 8; c0 += 8) {
+              uint4 bv[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) bv[k] = (c0 + k < rp / 8) ? __ldg(brow + c0 + k) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                if (c0 + k >= rp / 8) break;
+                const __half2* bh = reinterpret_cast<const __half2*>(&bv[k]);
+                float2 bf[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) bf[q] = __half22float2(bh[q]);
+#pragma unroll
+                for (int p = 0; p < kDN; ++p) {
+                  if (p >= T) break;
+                  const uint4 uv = *reinterpret_cast<const uint4*>(ucat_s + static_cast<size_t>(p) * rp + (c0 + k) * 8);
+                  const __half2* uh = reinterpret_cast<const __half2*>(&uv);
+                  float sacc = adr[p];
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) {
+                    const float2 uf = __half22float2(uh[q]);
+                    sacc = fmaf(bf[q].x, uf.x, sacc);
+                    sacc = fmaf(bf[q].y, uf.y, sacc);
+                  }
+                  adr[p] = sacc;
+                }
+              }
+            }
+          }
+          float4* dst = reinterpret_cast<float4*>(a.ad + (static_cast<size_t>(nt) * kTileN + r) * kDN);
+#pragma unroll
+          for (int k = 0; k < kDN / 4; ++k) dst[k] = make_float4(adr[4 * k], adr[4 * k + 1], adr[4 * k + 2], adr[4 * k + 3]);
+        }
+      }
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(adready);
+    }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ unpack into TMEM
-    const int q4 = warp & 3, half = (warp - 4) >> 2;
+    // Two teams of four warps (one per TMEM lane quarter) take alternate blocks, so two blocks are
+    // in flight; each thread unpacks one full row of the block.
+    const int q4 = warp & 3, team = (warp - 4) >> 2;
     const int r = 32 * q4 + lane;  // block row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
-    for (int i = 0; i < nblk; ++i) {
+    for (int i = team; i < nblk; i += 2) {
       const int s = i % NS, as = i % NA;
       if (!mbar_wait(&wfull[s], (i / NS) & 1, a_err, DEVERR_WAIT_UNPACK) ||
           !mbar_wait(&aempty[as], ((i / NA) & 1) ^ 1, a_err, DEVERR_WAIT_UNPACK))
         break;
       tc_fence_after();
-      unpack_half_row<I8, BITS>(wring + s * C::kWBlock, r, half,
-                                tmem + lane_base + colA + as * C::kACols + half * (C::kACols / 2));
+      const uint32_t ta = tmem + lane_base + colA + as * C::kACols;
+      unpack_half_row<I8, BITS>(wring + s * C::kWBlock, r, 0, ta);
+      unpack_half_row<I8, BITS>(wring + s * C::kWBlock, r, 1, ta + C::kACols / 2);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -354,92 +455,43 @@ __global__ void __launch_bounds__(kDThreads, 1)
     const int et = threadIdx.x - 384;  // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
     const int T = a.T;
-    bool ok = true;
-    int cnt0 = 0, cnt1 = 0;           // groups drained from issuer 0 / 1
-    // group scales of the next kDSwAhead blocks (two groups per block at g = 64)
-    float sw0[kDSwAhead], sw1[kDSwAhead];
-    auto load_sw = [&](int i, float& s0, float& s1) {
-      s0 = 0.0f;
-      s1 = 0.0f;
-      if (i >= nblk) return;
-      const int64_t f = b0 + i;
-      const int nt = static_cast<int>(f / a.KB), kb = static_cast<int>(f % a.KB);
+    // the group scales of block i: the 128-row slab(s) the producer copied into ring slot i % NS
+    // (or, when a row of scales is not a multiple of 16 bytes, this thread's own scale from memory)
+    auto scale_at = [&](int s, int gi, int nt, int j) -> float {
+      if (a.sw_vec) {
+        const uint8_t* slab = sring + s * C::kSBlock + gi * 512;
+        if (a.sw_f16) return __half2float(*reinterpret_cast<const __half*>(slab + r * 2));
+        return *reinterpret_cast<const float*>(slab + r * 4);
+      }
       const int o = nt * kTileN + r;
-      if (o >= a.N) return;
-      const int j = kb * gpb;
-      s0 = load_scale(a.w_scale, static_cast<size_t>(j) * a.N + o, a.sw_f16);
-      if (gpb == 2 && j + 1 < a.G_total) s1 = load_scale(a.w_scale, static_cast<size_t>(j + 1) * a.N + o, a.sw_f16);
+      return (o < a.N) ? load_scale(a.w_scale, static_cast<size_t>(j) * a.N + o, a.sw_f16) : 0.0f;
     };
-#pragma unroll
-    for (int k = 0; k < kDSwAhead; ++k) load_sw(k, sw0[k], sw1[k]);
-    float acc[kDN], adr[kDN];
-#pragma unroll
-    for (int p = 0; p < kDN; ++p) {
-      acc[p] = 0.0f;
-      adr[p] = 0.0f;
-    }
-    int cur_nt = -1;
-    bool have_ad = false;  // adr holds this CTA's adapter term of tile cur_nt
 
-    // The tile's adapter term su-less: ad[p] = sum_r B_catT[o][r] * U_cat[p][r] (fp32 sums of fp16 inputs).
-    auto adapter_term = [&](int nt) {
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      const int rp = a.R_pad;
-      for (int e = et; e < kDN * rp / 8; e += 128) {
-        const int p = e / (rp / 8), c8 = e % (rp / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (p < T) v = __ldg(reinterpret_cast<const uint4*>(a.ucat + static_cast<size_t>(p) * rp) + c8);
-        *reinterpret_cast<uint4*>(ucat_s + static_cast<size_t>(p) * rp + c8 * 8) = v;
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      const int o = nt * kTileN + r;
+    bool ok = true;
+    int cnt0 = 0, cnt1 = 0;  // groups drained from issuer 0 / 1
+    float acc[kDN];
 #pragma unroll
-      for (int p = 0; p < kDN; ++p) adr[p] = 0.0f;
-      if (o < a.N) {
-        const uint4* brow = reinterpret_cast<const uint4*>(a.bcat + static_cast<size_t>(o) * rp);
-        for (int c8 = 0; c8 < rp / 8; ++c8) {
-          const uint4 bv = __ldg(brow + c8);
-          const __half2* bh = reinterpret_cast<const __half2*>(&bv);
-          float2 bf[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) bf[k] = __half22float2(bh[k]);
-#pragma unroll
-          for (int p = 0; p < kDN; ++p) {
-            const uint4 uv = *reinterpret_cast<const uint4*>(ucat_s + static_cast<size_t>(p) * rp + c8 * 8);
-            const __half2* uh = reinterpret_cast<const __half2*>(&uv);
-            float s = adr[p];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 uf = __half22float2(uh[k]);
-              s = fmaf(bf[k].x, uf.x, s);
-              s = fmaf(bf[k].y, uf.y, s);
-            }
-            adr[p] = s;
-          }
-        }
-      }
-    };
+    for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
+    int cur_nt = -1;
+    bool cur_ad = false;     // this segment holds its tile's first block
 
     // End of a segment of tile nt: a tile held by this CTA alone is written at once; otherwise the
     // partial goes to its slot and the last CTA to finish the tile adds the partials in segment order.
-    auto finish_segment = [&](int nt) {
+    auto finish_segment = [&](int nt, bool has_first) {
       const int64_t f0 = static_cast<int64_t>(nt) * a.KB;
       const int c_first = cta_of(f0, a.NB, G);
       const int nseg = cta_of(f0 + a.KB - 1, a.NB, G) - c_first + 1;
       const int seg = c - c_first;
       const int o = nt * kTileN + r;
       const size_t tile_row = (static_cast<size_t>(nt) * kTileN + r) * kDN;
+      // the adapter term of this tile was computed by warp 3 of this CTA
+      if (has_first && a.su_sorted && ok) ok = __all_sync(0xffffffffu, mbar_wait(adready, 0, a_err, DEVERR_WAIT_EPILOGUE));
       bool last = true;
       if (nseg > 1) {
         float4* dst = reinterpret_cast<float4*>(a.part + (static_cast<size_t>(nt) * a.maxseg + seg) * kTileN * kDN +
                                                 static_cast<size_t>(r) * kDN);
 #pragma unroll
         for (int k = 0; k < kDN / 4; ++k) dst[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
-        if (have_ad) {
-          float4* ad = reinterpret_cast<float4*>(a.ad + tile_row);
-#pragma unroll
-          for (int k = 0; k < kDN / 4; ++k) ad[k] = make_float4(adr[4 * k], adr[4 * k + 1], adr[4 * k + 2], adr[4 * k + 3]);
-        }
         __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (et == 0) {
@@ -464,30 +516,33 @@ __global__ void __launch_bounds__(kDThreads, 1)
               acc[4 * k + 3] += v.w;
             }
           }
-          if (!have_ad && a.su_sorted) {
-            const float4* ad = reinterpret_cast<const float4*>(a.ad + tile_row);
-#pragma unroll
-            for (int k = 0; k < kDN / 4; ++k) {
-              const float4 v = __ldcg(ad + k);
-              adr[4 * k] = v.x;
-              adr[4 * k + 1] = v.y;
-              adr[4 * k + 2] = v.z;
-              adr[4 * k + 3] = v.w;
-            }
-          }
         }
       }
       if (last) {
+        float adr[kDN];
+#pragma unroll
+        for (int p = 0; p < kDN; ++p) adr[p] = 0.0f;
+        if (a.su_sorted) {
+          const float4* ad = reinterpret_cast<const float4*>(a.ad + tile_row);
+#pragma unroll
+          for (int k = 0; k < kDN / 4; ++k) {
+            const float4 v = __ldcg(ad + k);
+            adr[4 * k] = v.x;
+            adr[4 * k + 1] = v.y;
+            adr[4 * k + 2] = v.z;
+            adr[4 * k + 3] = v.w;
+          }
+        }
         if (o < a.N) {
 #pragma unroll
           for (int p = 0; p < kDN; ++p) {
             if (p >= T) break;
-            float y = acc[p] * __ldg(a.sa_sorted + p);
+            // int8 codes carry the token scale; weight-only layers computed with the bf16 activation itself
+            float y = I8 ? acc[p] * __ldg(a.sa_sorted + p) : acc[p];
             if (a.su_sorted) y = fmaf(__ldg(a.su_sorted + p), adr[p], y);
             const size_t at = static_cast<size_t>(__ldg(a.perm + p)) * a.N + o;
             if (a.y_bf16) {
-              const __nv_bfloat16 h = __float2bfloat16_rn(y);
-              static_cast<__nv_bfloat16*>(a.Y)[at] = h;
+              static_cast<__nv_bfloat16*>(a.Y)[at] = __float2bfloat16_rn(y);
             } else {
               static_cast<float*>(a.Y)[at] = y;
             }
@@ -495,29 +550,24 @@ __global__ void __launch_bounds__(kDThreads, 1)
         }
         if (nseg > 1 && et == 0) a.cnt[nt] = 0u;  // leave the counter at zero for the next launch
       }
-      have_ad = false;
     };
 
-    for (int i = 0; i < nblk; ++i) {
-      const int64_t f = b0 + i;
-      const int nt = static_cast<int>(f / a.KB), kb = static_cast<int>(f % a.KB);
+    BlockPos bp = pos0;
+    for (int i = 0; i < nblk; ++i, bp.next(a.KB)) {
+      const int nt = bp.nt, kb = bp.kb;
       if (nt != cur_nt) {
-        if (cur_nt >= 0) finish_segment(cur_nt);
+        if (cur_nt >= 0) finish_segment(cur_nt, cur_ad);
         cur_nt = nt;
+        cur_ad = kb == 0;
 #pragma unroll
         for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
-        if (kb == 0 && a.su_sorted) {
-          adapter_term(nt);
-          have_ad = true;
-        }
       }
-      const float s0 = sw0[0], s1 = sw1[0];
-#pragma unroll
-      for (int k = 0; k + 1 < kDSwAhead; ++k) {
-        sw0[k] = sw0[k + 1];
-        sw1[k] = sw1[k + 1];
-      }
-      load_sw(i + kDSwAhead, sw0[kDSwAhead - 1], sw1[kDSwAhead - 1]);
+      // this block's scales arrived with it in ring slot s (the phase cannot move on before this
+      // epilogue frees the slot, so the parity wait is exact)
+      const int s = i % NS;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&wfull[s], (i / NS) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+      const float s0 = scale_at(s, 0, nt, kb * gpb);
+      const float s1 = (gpb == 2) ? scale_at(s, 1, nt, kb * gpb + 1) : 0.0f;
       const int q = i & 1;
       const int ng = min(gpb, a.G_total - kb * gpb);
       for (int gi = 0; gi < ng; ++gi) {
@@ -557,8 +607,11 @@ __global__ void __launch_bounds__(kDThreads, 1)
           for (int p = 0; p < kDN; ++p) acc[p] = fmaf(__uint_as_float(v[p]), sw, acc[p]);
         }
       }
+      // the block's MMAs are done and its scales read: the ring slot can take a new block
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wempty[s]);
     }
-    if (cur_nt >= 0) finish_segment(cur_nt);
+    if (cur_nt >= 0) finish_segment(cur_nt, cur_ad);
     tc_fence_before();
   }
   __syncthreads();
@@ -624,6 +677,8 @@ cudaError_t launch_qdec(int w_bits, bool int8, const CUtensorMap& tm_x, const De
   a.w_packed = q.w_packed;
   a.w_scale = q.w_scale;
   a.sw_f16 = q.sw_f16;
+  a.sw_elem = q.sw_f16 ? 2 : 4;
+  a.sw_vec = ((static_cast<int64_t>(q.N) * a.sw_elem) % 16) == 0 ? 1 : 0;
   a.sa_sorted = q.sa_sorted;
   a.su_sorted = q.su_sorted;
   a.perm = q.perm;

@@ -370,10 +370,6 @@ __global__ void __launch_bounds__(512, 1)
             // row r: 64 bytes, four 16-byte pieces; this atom is pieces 2*atom and 2*atom+1
             const uint4 p0 = *reinterpret_cast<const uint4*>(src + r * 64 + atom * 32);
             const uint4 p1 = *reinterpret_cast<const uint4*>(src + r * 64 + atom * 32 + 16);
-            if (ai == kAtomsPerThread - 1) {
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&wempty[ws]);
-            }
             const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
             for (int pc = 0; pc < 2; ++pc) {
@@ -394,10 +390,6 @@ __global__ void __launch_bounds__(512, 1)
             // row r: 48 bytes; low two bits in words m = 4*atom + 0..3, bit 2 in words h = 2*atom + 0..1
             const uint4 lq = *reinterpret_cast<const uint4*>(src + r * 48 + atom * 16);
             const uint2 hq = *reinterpret_cast<const uint2*>(src + r * 48 + 32 + atom * 8);
-            if (ai == kAtomsPerThread - 1) {
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&wempty[ws]);
-            }
             const uint32_t lw[4] = {lq.x, lq.y, lq.z, lq.w};
             const uint32_t hw[2] = {hq.x, hq.y};
 #pragma unroll
@@ -414,6 +406,10 @@ __global__ void __launch_bounds__(512, 1)
             }
           }
           }
+          // free the packed block only now: its values have been used, so every load from it has
+          // completed before the next bulk copy can land in the slot
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&wempty[ws]);
           fence_proxy_async_smem();
           ++jw;
         } else {

@@ -65,15 +65,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with a suspend-time hint: while the phase is open the thread is suspended in
+// hardware (for at most hint_ns) instead of spinning, so waiting warps leave the issue slots
+// to the warps that work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+constexpr uint32_t kWaitHintNs = 20000;  // one suspension; the overall bound is checked between them
+
 // Wait for the phase with the given parity to complete. Returns false (and
 // records err) when the wait ran out after limit_ns; callers then stop issuing work.
 __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int* flag, int err,
                                               uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if ((++spins & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
+  while (!mbar_try_wait_sleep(bar, parity, kWaitHintNs)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       record_error(flag, err);
       return false;
     }

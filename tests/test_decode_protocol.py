@@ -6,9 +6,10 @@
    segments than the workspace holds (the partial slot index stays in bounds), and that the
    per-tile fix-up (the last of the tile's segments to arrive adds them in segment order) runs
    exactly once per tile, whatever order the CTAs finish in.
-2. The mbarrier protocol: a producer fills the packed-block ring in order, eight unpack warps
-   put each block into one of four TMEM A slots, two issuers take alternate blocks (issuer q owns
-   accumulator slots q, q+2, ...), four epilogue warps drain the groups in block order. Random
+2. The mbarrier protocol: a producer fills the packed-block ring in order, two teams of four
+   unpack warps take alternate blocks and put each into one of four TMEM A slots, two issuers take
+   alternate blocks (issuer q owns accumulator slots q, q+2, ...), four epilogue warps drain the
+   groups in block order, reading each block's scale slabs from its ring slot and then freeing it. Random
    interleavings; every parity wait must be sound (the barrier has completed n or n+1 phases
    when a wait for phase n passes) and everything must finish.
 """
@@ -109,8 +110,8 @@ def test_fixup_runs_once_per_tile_in_segment_order(N, K):
 def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
     """nblk blocks; gpb_of(i) = groups of block i (1, or 2 at g = 64)."""
     wfull = [Barrier(f"wfull{i}", 1) for i in range(NS)]
-    wempty = [Barrier(f"wempty{i}", 1) for i in range(NS)]
-    afull = [Barrier(f"afull{i}", n_unpack) for i in range(NA)]
+    wempty = [Barrier(f"wempty{i}", n_epi) for i in range(NS)]
+    afull = [Barrier(f"afull{i}", n_unpack // 2) for i in range(NA)]
     aempty = [Barrier(f"aempty{i}", 1) for i in range(NA)]
     accf = [Barrier(f"accf{i}", 1) for i in range(n_slots)]
     acce = [Barrier(f"acce{i}", n_epi) for i in range(n_slots)]
@@ -126,7 +127,8 @@ def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
             yield
 
     def unpack(k):
-        for i in range(nblk):
+        team = k // 4          # two teams of four warps take alternate blocks
+        for i in range(team, nblk, 2):
             s, a = i % NS, i % NA
             yield from _wait(wfull[s], i // NS, f"unpack{k}")
             if i // NA > 0:
@@ -148,12 +150,12 @@ def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
                 yield
                 pending.append([rng.randint(1, 5), accf[slot].arrive])
             pending.append([rng.randint(1, 5), aempty[a].arrive])
-            pending.append([rng.randint(1, 5), wempty[s].arrive])
 
     def epilogue(k):
         n = [0, 0]
         for i in range(nblk):
-            q = i & 1
+            q, s = i & 1, i % NS
+            yield from _wait(wfull[s], i // NS, f"epilogue{k}")   # the block's scale slabs
             for _ in range(gpb_of(i)):
                 slot, use = q + 2 * (n[q] % own_n), n[q] // own_n
                 n[q] += 1
@@ -161,6 +163,7 @@ def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
                 for _ in range(rng.randint(0, 6)):
                     yield
                 acce[slot].arrive()
+            wempty[s].arrive()     # scales read, MMAs done: the ring slot is free
 
     roles = [producer(), issuer(0), issuer(1)] + [unpack(k) for k in range(n_unpack)]
     roles += [epilogue(k) for k in range(n_epi)]
@@ -181,10 +184,10 @@ def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
     raise Unsound("no progress (deadlock)")
 
 
-# (accumulator slots) of the two instances: int8 24, bf16 16; ring 10, A slots 4
-@pytest.mark.parametrize("n_slots", [24, 16])
+# accumulator slots: int8 24, bf16 16; ring 16 (int8, W3) or 14 (W4 bf16); A slots 4
+@pytest.mark.parametrize("n_slots,NS", [(24, 16), (16, 16), (16, 14)])
 @pytest.mark.parametrize("kind", ["g128", "g64", "ragged_g64", "one", "two"])
-def test_decode_barrier_protocol_is_sound(n_slots, kind):
+def test_decode_barrier_protocol_is_sound(n_slots, NS, kind):
     shapes = {
         "g128": (100, lambda i: 1),
         "g64": (60, lambda i: 2),
@@ -194,4 +197,4 @@ def test_decode_barrier_protocol_is_sound(n_slots, kind):
     }
     nblk, gpb_of = shapes[kind]
     for seed in range(3):
-        run_decode_model(nblk, gpb_of, 10, 4, n_slots, random.Random(seed))
+        run_decode_model(nblk, gpb_of, NS, 4, n_slots, random.Random(seed))
