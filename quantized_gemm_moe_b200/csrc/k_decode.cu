@@ -42,7 +42,6 @@ namespace {
 
 constexpr int kDN = 16;          // token columns: the whole batch, padded (MMA N)
 constexpr int kDThreads = 512;   // 16 warps
-constexpr int kDASlots = 4;      // unpacked A blocks in TMEM
 constexpr int kDTmemCols = 512;
 
 template <bool I8, int BITS>
@@ -52,18 +51,25 @@ struct DCfg {
   static constexpr int kXTile = I8 ? kXAtom : 2 * kXAtom;  // 128 input channels: int8 codes or bf16
   static constexpr int kACols = I8 ? 32 : 64;             // TMEM columns of one unpacked block
   static constexpr int kKSteps = I8 ? 4 : 8;              // MMA K steps per block (32 int8 / 16 bf16)
-  static constexpr int kAccSlots = (kDTmemCols - kDASlots * kACols) / kDN;  // 24 (int8) / 16 (bf16)
+  // unpacked A blocks in TMEM: the loop unpack -> MMA -> slot free spans this many blocks
+  static constexpr int kASlots = I8 ? 8 : 6;
+  static constexpr int kAccSlots = (kDTmemCols - kASlots * kACols) / kDN;  // 16 (int8) / 8 (bf16)
   static constexpr int kOwn = kAccSlots / 2;              // accumulator slots per issuer
   static constexpr int kUcatBytes = kDN * 512 * 2;        // U_cat staging, R_pad <= 512
   static constexpr int kSBlock = 2 * 128 * 4;             // group scale slabs of a block (2 groups x 128 rows)
-  // Ring of blocks in flight (packed block + activation tile + scale slabs), even so that each
-  // unpack team keeps its own slots. A slot is freed once the epilogue has read its scales, so
-  // the ring spans the whole pipeline from the load to the drained group.
-  static constexpr int kStages = (I8 || BITS == 3) ? 16 : 14;
-  static constexpr size_t kSmem =
-      1024 + size_t(kStages) * (kXTile + kWBlock + kSBlock) + kUcatBytes + 1024;
-  static_assert(kStages % 2 == 0, "each unpack team keeps its own ring slots");
+  // Three rings, all even so that each unpack team / issuer keeps its own slots:
+  //  packed blocks: freed by the unpack team as soon as it has used them, so the HBM stream only
+  //    waits on one hand-off (load -> unpack);
+  //  activation tiles: freed by the MMA commit;  scale slabs: freed by the epilogue.
+  // The last two recycle later in the pipeline, so they are deeper (and small).
+  static constexpr int kWStages = (I8 || BITS == 3) ? 16 : 12;
+  static constexpr int kXStages = I8 ? 24 : 16;
+  static constexpr int kSStages = I8 ? 24 : 16;
+  static constexpr size_t kSmem = 1024 + size_t(kXStages) * kXTile + size_t(kWStages) * kWBlock +
+                                  size_t(kSStages) * kSBlock + kUcatBytes + 1024;
+  static_assert(kWStages % 2 == 0 && kXStages % 2 == 0 && kSStages % 2 == 0, "team / issuer owned ring slots");
   static_assert(kAccSlots % 2 == 0, "each issuer owns half of the accumulator slots");
+  static_assert(kASlots % 2 == 0, "each unpack team and issuer keeps its own A slots");
   static_assert(kSmem <= 232448, "shared memory");
 };
 
@@ -228,24 +234,28 @@ template <bool I8, int BITS>
 __global__ void __launch_bounds__(kDThreads, 1)
     k_qdec(const __grid_constant__ CUtensorMap tm_x, const DecArgs a) {
   using C = DCfg<I8, BITS>;
-  constexpr int NS = C::kStages, NA = kDASlots;
+  constexpr int NW = C::kWStages, NX = C::kXStages, NSS = C::kSStages, NA = C::kASlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* xring = smem;                              // [NS][kXTile], 1024-aligned (128B swizzle)
-  uint8_t* wring = xring + NS * C::kXTile;            // [NS][kWBlock]
-  uint8_t* sring = wring + NS * C::kWBlock;           // [NS][2 groups][128 rows] group scales
-  __half* ucat_s = reinterpret_cast<__half*>(sring + NS * C::kSBlock);  // [16][R_pad]
+  uint8_t* xring = smem;                              // [NX][kXTile], 1024-aligned (128B swizzle)
+  uint8_t* wring = xring + NX * C::kXTile;            // [NW][kWBlock]
+  uint8_t* sring = wring + NW * C::kWBlock;           // [NSS][2 groups][128 rows] group scales
+  __half* ucat_s = reinterpret_cast<__half*>(sring + NSS * C::kSBlock);  // [16][R_pad]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ucat_s) + C::kUcatBytes);
-  uint64_t* wfull = bars;                  // [NS] block, tile and scales landed (1 + bytes)
-  uint64_t* wempty = wfull + NS;           // [NS] the epilogue read the block's scales (its MMAs are done)
-  uint64_t* afull = wempty + NS;           // [NA] A unpacked into TMEM (the 4 warps of a team)
+  uint64_t* wfull = bars;                  // [NW] packed block landed (1 + bytes)
+  uint64_t* wempty = wfull + NW;           // [NW] the unpack team has used it (4 warps)
+  uint64_t* xfull = wempty + NW;           // [NX] activation tile landed (1 + bytes)
+  uint64_t* xempty = xfull + NX;           // [NX] the block's MMAs are done
+  uint64_t* sfull = xempty + NX;           // [NSS] scale slabs landed (1 + bytes)
+  uint64_t* sempty = sfull + NSS;          // [NSS] the epilogue read them (4 warps)
+  uint64_t* afull = sempty + NSS;          // [NA] A unpacked into TMEM (the 4 warps of a team)
   uint64_t* aempty = afull + NA;           // [NA] the MMAs of the block are done (A slot free)
   uint64_t* accf = aempty + NA;            // [kAccSlots] group sum ready
   uint64_t* acce = accf + C::kAccSlots;    // [kAccSlots] group sum read (4 epilogue warps)
   uint64_t* done = acce + C::kAccSlots;    // teardown
-  uint64_t* adready = done + 1;            // the adapter terms of this CTA's tiles are in memory
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(adready + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   int* flag_s = reinterpret_cast<int*>(tmem_slot + 1);
+  volatile int* ad_done = reinterpret_cast<volatile int*>(tmem_slot + 2);  // adapter tiles written so far
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
@@ -259,10 +269,19 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const bool any_ad = a.su_sorted != nullptr && nt_ad0 <= nt_ad1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NW; ++s) {
       mbar_init(&wfull[s], 1);
       mbar_init(&wempty[s], 4);
     }
+    for (int s = 0; s < NX; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);
+    }
+    for (int s = 0; s < NSS; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 4);
+    }
+    *ad_done = 0;
     for (int s = 0; s < NA; ++s) {
       mbar_init(&afull[s], 4);
       mbar_init(&aempty[s], 1);
@@ -272,7 +291,6 @@ __global__ void __launch_bounds__(kDThreads, 1)
       mbar_init(&acce[b], 4);
     }
     mbar_init(done, 2);
-    mbar_init(adready, 1);
     mbar_fence_init();
     prefetch_tmap(&tm_x);
   }
@@ -283,36 +301,55 @@ __global__ void __launch_bounds__(kDThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t colA = 0, colAcc = kDASlots * C::kACols;
+  const uint32_t colA = 0, colAcc = NA * C::kACols;
   grid_dep_wait();
   grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // per block: the packed block, its activation tile and its scale slabs, each into its own ring
     if (lane == 0) {
       int i = 0;
       BlockPos bp = pos0;
+      bool ok = true;
       for (; i < nblk; ++i, bp.next(a.KB)) {
-        const int s = i % NS;
-        if (!mbar_wait(&wempty[s], ((i / NS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) break;
         const int kb = bp.kb;
-        // the 128-row scale slab of each of the block's groups (contiguous: group-major [G][N])
+        const int sw = i % NW, sx = i % NX, ss = i % NSS;
+        if (!mbar_wait(&wempty[sw], ((i / NW) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&wfull[sw], C::kWBlock);
+        bulk_load(wring + sw * C::kWBlock, a.w_packed + (b0 + i) * C::kWBlock, C::kWBlock, &wfull[sw]);
+        if (!mbar_wait(&xempty[sx], ((i / NX) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) {
+          ok = false;
+          ++i;
+          break;
+        }
+        mbar_arrive_expect_tx(&xfull[sx], C::kXTile);
+        tma_load_2d(xring + sx * C::kXTile, &tm_x, kb * kTileK, 0, &xfull[sx]);
+        if constexpr (!I8) tma_load_2d(xring + sx * C::kXTile + C::kXAtom, &tm_x, kb * kTileK + 64, 0, &xfull[sx]);
+        if (!mbar_wait(&sempty[ss], ((i / NSS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) {
+          ok = false;
+          ++i;
+          break;
+        }
+        // the 128-row scale slab of each of the block's groups (contiguous: group-major [G][N]);
+        // with a row pitch that is not a multiple of 16 bytes the epilogue reads its scales itself
         const int ng = min(gpb, a.G_total - kb * gpb);
-        const uint32_t sbytes = a.sw_vec ? static_cast<uint32_t>(128 * a.sw_elem) : 0u;
         const int o0 = bp.nt * kTileN;
-        const uint32_t svalid = min(128, a.N - o0) * a.sw_elem;  // the last tile's slab stops at d_out
-        const uint32_t scopy = sbytes ? ((svalid + 15u) & ~15u) : 0u;
-        mbar_arrive_expect_tx(&wfull[s], C::kWBlock + C::kXTile + ng * scopy);
-        bulk_load(wring + s * C::kWBlock, a.w_packed + (b0 + i) * C::kWBlock, C::kWBlock, &wfull[s]);
-        tma_load_2d(xring + s * C::kXTile, &tm_x, kb * kTileK, 0, &wfull[s]);
-        if constexpr (!I8) tma_load_2d(xring + s * C::kXTile + C::kXAtom, &tm_x, kb * kTileK + 64, 0, &wfull[s]);
+        const uint32_t scopy = a.sw_vec ? static_cast<uint32_t>(min(128, a.N - o0) * a.sw_elem) : 0u;
+        mbar_arrive_expect_tx(&sfull[ss], ng * scopy);
         for (int gi = 0; gi < (scopy ? ng : 0); ++gi)
-          bulk_load(sring + s * C::kSBlock + gi * 512,
+          bulk_load(sring + ss * C::kSBlock + gi * 512,
                     reinterpret_cast<const uint8_t*>(a.w_scale) +
                         (static_cast<size_t>(kb * gpb + gi) * a.N + o0) * a.sw_elem,
-                    scopy, &wfull[s]);
+                    scopy, &sfull[ss]);
       }
-      drain_ring(wfull, NS, i);
+      (void)ok;
+      drain_ring(wfull, NW, i);
+      drain_ring(xfull, NX, i);
+      drain_ring(sfull, NSS, i);
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers (alternate blocks)
@@ -325,15 +362,16 @@ __global__ void __launch_bounds__(kDThreads, 1)
       BlockPos bp = pos0;
       if (qi) bp.next(a.KB);
       for (int i = qi; i < nblk && ok; i += 2, bp.next(a.KB), bp.next(a.KB)) {
-        const int s = i % NS, as = i % NA;
+        const int sx = i % NX, as = i % NA;
         const int kb = bp.kb;
         const int ng = min(gpb, a.G_total - kb * gpb);
-        if (!mbar_wait(&afull[as], (i / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
+        if (!mbar_wait(&afull[as], (i / NA) & 1, a_err, DEVERR_WAIT_MMA) ||
+            !mbar_wait(&xfull[sx], (i / NX) & 1, a_err, DEVERR_WAIT_MMA)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t xdesc = xdesc0 + static_cast<uint64_t>((s * C::kXTile) >> 4);
+        const uint64_t xdesc = xdesc0 + static_cast<uint64_t>((sx * C::kXTile) >> 4);
         const uint32_t a_col = tmem + colA + as * C::kACols;
         for (int gi = 0; gi < ng; ++gi) {
           const int slot = qi + 2 * (own % C::kOwn);
@@ -361,6 +399,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
           tc_commit(&accf[slot]);
         }
         tc_commit(&aempty[as]);
+        tc_commit(&xempty[sx]);
       }
       tc_commit(done);
       mbar_wait(done, 0, a_err, DEVERR_WAIT_TEARDOWN);
@@ -369,7 +408,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
     // ------------------------------------------------------------ adapter terms (CUDA cores)
     // ad[nt][r][p] = sum_j B_catT[o][j] * U_cat[p][j] (fp16 inputs, fp32 sums) for every tile whose
     // first block this CTA streams; lane l takes rows l, l+32, l+64, l+96. Off the epilogue's path:
-    // the segment holding the tile's first block waits on adready only when it finishes.
+    // the segment holding a tile's first block waits for that tile's term (the count ad_done)
+    // only when it finishes.
     if (any_ad) {
       const int rp = a.R_pad, T = a.T;
       for (int e = lane; e < kDN * rp / 8; e += 32) {
@@ -420,10 +460,11 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
           for (int k = 0; k < kDN / 4; ++k) dst[k] = make_float4(adr[4 * k], adr[4 * k + 1], adr[4 * k + 2], adr[4 * k + 3]);
         }
+        // this tile's term is in memory: the epilogue can finish the tile's first segment
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) *ad_done = nt - nt_ad0 + 1;
       }
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(adready);
     }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ unpack into TMEM
@@ -433,14 +474,18 @@ __global__ void __launch_bounds__(kDThreads, 1)
     const int r = 32 * q4 + lane;  // block row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
     for (int i = team; i < nblk; i += 2) {
-      const int s = i % NS, as = i % NA;
-      if (!mbar_wait(&wfull[s], (i / NS) & 1, a_err, DEVERR_WAIT_UNPACK) ||
+      const int sw = i % NW, as = i % NA;
+      if (!mbar_wait(&wfull[sw], (i / NW) & 1, a_err, DEVERR_WAIT_UNPACK) ||
           !mbar_wait(&aempty[as], ((i / NA) & 1) ^ 1, a_err, DEVERR_WAIT_UNPACK))
         break;
       tc_fence_after();
       const uint32_t ta = tmem + lane_base + colA + as * C::kACols;
-      unpack_half_row<I8, BITS>(wring + s * C::kWBlock, r, 0, ta);
-      unpack_half_row<I8, BITS>(wring + s * C::kWBlock, r, 1, ta + C::kACols / 2);
+      unpack_half_row<I8, BITS>(wring + sw * C::kWBlock, r, 0, ta);
+      unpack_half_row<I8, BITS>(wring + sw * C::kWBlock, r, 1, ta + C::kACols / 2);
+      // the packed block's values have been used (the stores below hold them): free its slot now,
+      // so the next load can land while this block goes through the MMA
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wempty[sw]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -485,7 +530,18 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const int o = nt * kTileN + r;
       const size_t tile_row = (static_cast<size_t>(nt) * kTileN + r) * kDN;
       // the adapter term of this tile was computed by warp 3 of this CTA
-      if (has_first && a.su_sorted && ok) ok = __all_sync(0xffffffffu, mbar_wait(adready, 0, a_err, DEVERR_WAIT_EPILOGUE));
+      if (has_first && a.su_sorted && ok) {
+        // warp 3 writes the terms in tile order; this is tile nt - nt_ad0 of that list
+        const int need = nt - nt_ad0 + 1;
+        bool got = *ad_done >= need;
+        if (!got) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!(got = (*ad_done >= need)) && globaltimer_ns() - t0 < kWaitLimitNs) __nanosleep(256);
+        }
+        if (!got) record_error(a_err, DEVERR_WAIT_EPILOGUE);
+        __threadfence_block();
+        ok = __all_sync(0xffffffffu, got);
+      }
       bool last = true;
       if (nseg > 1) {
         float4* dst = reinterpret_cast<float4*>(a.part + (static_cast<size_t>(nt) * a.maxseg + seg) * kTileN * kDN +
@@ -562,12 +618,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
         for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
       }
-      // this block's scales arrived with it in ring slot s (the phase cannot move on before this
-      // epilogue frees the slot, so the parity wait is exact)
-      const int s = i % NS;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&wfull[s], (i / NS) & 1, a_err, DEVERR_WAIT_EPILOGUE));
-      const float s0 = scale_at(s, 0, nt, kb * gpb);
-      const float s1 = (gpb == 2) ? scale_at(s, 1, nt, kb * gpb + 1) : 0.0f;
+      // this block's scale slabs (the phase cannot move on before this epilogue frees the slot,
+      // so the parity wait is exact)
+      const int ss = i % NSS;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sfull[ss], (i / NSS) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+      const float s0 = scale_at(ss, 0, nt, kb * gpb);
+      const float s1 = (gpb == 2) ? scale_at(ss, 1, nt, kb * gpb + 1) : 0.0f;
       const int q = i & 1;
       const int ng = min(gpb, a.G_total - kb * gpb);
       for (int gi = 0; gi < ng; ++gi) {
@@ -607,9 +663,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
           for (int p = 0; p < kDN; ++p) acc[p] = fmaf(__uint_as_float(v[p]), sw, acc[p]);
         }
       }
-      // the block's MMAs are done and its scales read: the ring slot can take a new block
+      // the block's scales have been read: the slot can take a later block's
       __syncwarp();
-      if (lane == 0) mbar_arrive(&wempty[s]);
+      if (lane == 0) mbar_arrive(&sempty[ss]);
     }
     if (cur_nt >= 0) finish_segment(cur_nt, cur_ad);
     tc_fence_before();

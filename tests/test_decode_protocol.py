@@ -9,7 +9,8 @@
 2. The mbarrier protocol: a producer fills the packed-block ring in order, two teams of four
    unpack warps take alternate blocks and put each into one of four TMEM A slots, two issuers take
    alternate blocks (issuer q owns accumulator slots q, q+2, ...), four epilogue warps drain the
-   groups in block order, reading each block's scale slabs from its ring slot and then freeing it. Random
+   groups in block order. Three rings: packed blocks (freed by the unpack team once used),
+   activation tiles (freed by the MMA commit) and scale slabs (freed by the epilogue). Random
    interleavings; every parity wait must be sound (the barrier has completed n or n+1 phases
    when a wait for phase n passes) and everything must finish.
 """
@@ -107,10 +108,14 @@ def test_fixup_runs_once_per_tile_in_segment_order(N, K):
         assert all(v == 0 for v in cnt)                             # counters left at zero
 
 
-def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
+def run_decode_model(nblk, gpb_of, NW, NX, NSS, NA, n_slots, rng, n_unpack=8, n_epi=4):
     """nblk blocks; gpb_of(i) = groups of block i (1, or 2 at g = 64)."""
-    wfull = [Barrier(f"wfull{i}", 1) for i in range(NS)]
-    wempty = [Barrier(f"wempty{i}", n_epi) for i in range(NS)]
+    wfull = [Barrier(f"wfull{i}", 1) for i in range(NW)]
+    wempty = [Barrier(f"wempty{i}", n_unpack // 2) for i in range(NW)]
+    xfull = [Barrier(f"xfull{i}", 1) for i in range(NX)]
+    xempty = [Barrier(f"xempty{i}", 1) for i in range(NX)]
+    sfull = [Barrier(f"sfull{i}", 1) for i in range(NSS)]
+    sempty = [Barrier(f"sempty{i}", n_epi) for i in range(NSS)]
     afull = [Barrier(f"afull{i}", n_unpack // 2) for i in range(NA)]
     aempty = [Barrier(f"aempty{i}", 1) for i in range(NA)]
     accf = [Barrier(f"accf{i}", 1) for i in range(n_slots)]
@@ -120,28 +125,31 @@ def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
 
     def producer():
         for i in range(nblk):
-            s, n = i % NS, i // NS
-            if n > 0:
-                yield from _wait(wempty[s], n - 1, "producer")
-            pending.append([rng.randint(1, 8), wfull[s].arrive])
-            yield
+            for full, empty, depth in ((wfull, wempty, NW), (xfull, xempty, NX), (sfull, sempty, NSS)):
+                s, n = i % depth, i // depth
+                if n > 0:
+                    yield from _wait(empty[s], n - 1, "producer")
+                pending.append([rng.randint(1, 8), full[s].arrive])
+                yield
 
     def unpack(k):
         team = k // 4          # two teams of four warps take alternate blocks
         for i in range(team, nblk, 2):
-            s, a = i % NS, i % NA
-            yield from _wait(wfull[s], i // NS, f"unpack{k}")
+            s, a = i % NW, i % NA
+            yield from _wait(wfull[s], i // NW, f"unpack{k}")
             if i // NA > 0:
                 yield from _wait(aempty[a], i // NA - 1, f"unpack{k}")
             for _ in range(rng.randint(0, 3)):
                 yield
+            wempty[s].arrive()     # the packed block has been used
             afull[a].arrive()
 
     def issuer(q):
         own = 0
         for i in range(q, nblk, 2):
-            s, a = i % NS, i % NA
+            a, sx = i % NA, i % NX
             yield from _wait(afull[a], i // NA, f"issuer{q}")
+            yield from _wait(xfull[sx], i // NX, f"issuer{q}")
             for _ in range(gpb_of(i)):
                 slot, use = q + 2 * (own % own_n), own // own_n
                 own += 1
@@ -150,12 +158,13 @@ def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
                 yield
                 pending.append([rng.randint(1, 5), accf[slot].arrive])
             pending.append([rng.randint(1, 5), aempty[a].arrive])
+            pending.append([rng.randint(1, 5), xempty[sx].arrive])
 
     def epilogue(k):
         n = [0, 0]
         for i in range(nblk):
-            q, s = i & 1, i % NS
-            yield from _wait(wfull[s], i // NS, f"epilogue{k}")   # the block's scale slabs
+            q, ss = i & 1, i % NSS
+            yield from _wait(sfull[ss], i // NSS, f"epilogue{k}")   # the block's scale slabs
             for _ in range(gpb_of(i)):
                 slot, use = q + 2 * (n[q] % own_n), n[q] // own_n
                 n[q] += 1
@@ -163,7 +172,7 @@ def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
                 for _ in range(rng.randint(0, 6)):
                     yield
                 acce[slot].arrive()
-            wempty[s].arrive()     # scales read, MMAs done: the ring slot is free
+            sempty[ss].arrive()    # scales read: the slot is free
 
     roles = [producer(), issuer(0), issuer(1)] + [unpack(k) for k in range(n_unpack)]
     roles += [epilogue(k) for k in range(n_epi)]
@@ -184,10 +193,11 @@ def run_decode_model(nblk, gpb_of, NS, NA, n_slots, rng, n_unpack=8, n_epi=4):
     raise Unsound("no progress (deadlock)")
 
 
-# accumulator slots: int8 24, bf16 16; ring 16 (int8, W3) or 14 (W4 bf16); A slots 4
-@pytest.mark.parametrize("n_slots,NS", [(24, 16), (16, 16), (16, 14)])
+# rings (packed, tile, scales), A slots, accumulator slots of the three instances:
+# int8 (16, 24, 24, 8, 16); W4 bf16 (12, 16, 16, 6, 8); W3 bf16 (16, 16, 16, 6, 8)
+@pytest.mark.parametrize("NW,NX,NSS,NA,n_slots", [(16, 24, 24, 8, 16), (12, 16, 16, 6, 8), (16, 16, 16, 6, 8)])
 @pytest.mark.parametrize("kind", ["g128", "g64", "ragged_g64", "one", "two"])
-def test_decode_barrier_protocol_is_sound(n_slots, NS, kind):
+def test_decode_barrier_protocol_is_sound(NW, NX, NSS, NA, n_slots, kind):
     shapes = {
         "g128": (100, lambda i: 1),
         "g64": (60, lambda i: 2),
@@ -197,4 +207,4 @@ def test_decode_barrier_protocol_is_sound(n_slots, NS, kind):
     }
     nblk, gpb_of = shapes[kind]
     for seed in range(3):
-        run_decode_model(nblk, gpb_of, NS, 4, n_slots, random.Random(seed))
+        run_decode_model(nblk, gpb_of, NW, NX, NSS, NA, n_slots, random.Random(seed))
