@@ -10,25 +10,28 @@
 // tile's partials in segment order (deterministic), applies the token scale and the adapter term,
 // and writes Y.
 //
-// Per 128 x 128 weight block:
-//   warp 0      bulk copies of the packed block and of its group-scale slabs, and TMA of the
-//               activation tile (16 tokens x 128 channels), into a 14-16 deep ring: up to 128 KB
-//               of weights in flight per SM. The epilogue frees a slot once it has read the scales.
+// At 16 tokens a 128 x 128 block carries little work for any role, so the fixed cost of each
+// hand-off decides the speed: an MMA or a commit keeps its issuing thread ~140 cycles whatever N
+// is (several issuing threads overlap), and every dependent barrier step of a role costs a few
+// hundred cycles. The roles are laid out to keep those steps few per byte:
+//   warp 0      bulk copy of each packed block into a 20-24 deep ring (~150 KB in flight per SM),
+//               freed by the unpack team as soon as it has read the block; and TMA of each
+//               block's activation tile (16 tokens x 128 channels) into the slot of the block's
+//               unpacked weights, free again once the block's MMAs are done. One thread polls both.
 //   warps 4-11  unpack the block straight into tensor memory with tcgen05.st: the MMA takes its
 //               A operand (the weights, M = 128 output rows = TMEM lanes, K along the columns)
-//               from TMEM, so the unpacked weights never pass through shared memory (whose
-//               bandwidth the unpack would otherwise exceed at the HBM rate). Two teams of four
-//               warps (one per TMEM lane quarter) take alternate blocks, a full row per thread.
-//   warps 1-2   one thread each issues the MMAs of alternate blocks: kind::i8 (codes x16 against
+//               from TMEM, so the unpacked weights never pass through shared memory. Two teams of
+//               four warps (one per TMEM lane quarter) take alternate blocks, a row per thread.
+//   warps 1-3   one thread each issues the MMAs of every third block: kind::i8 (codes x16 against
 //               int8 activation codes, 4 K steps) or kind::f16 (bf16 weights against bf16
-//               activations, 8 K steps). Every quantization group gets a fresh 16-column
-//               accumulator (the first K step does not accumulate), issuer q owning slots
-//               q, q+2, ...
-//   warp 3      the adapter term U_cat . B_catT of every tile whose first block this CTA streams,
-//               on CUDA cores (fp16 inputs, fp32 sums), written to the workspace off the epilogue's path
-//   warps 12-15 epilogue, one output row per thread: per group acc += sw * group sum (the int8
-//               sums converted exactly, the scale read from the ring slot); the segment partials
-//               and the per-tile fix-up.
+//               activations, 8 K steps), one commit per block (frees the A slot and the tile).
+//               Every quantization group gets a fresh 16-column accumulator; eight (bf16: four)
+//               consecutive groups share one batch buffer (two buffers), committed once per batch.
+//   warps 12-15 epilogue, one output row per thread, a batch of groups at a time: the group
+//               sums (int8 sums converted exactly) times the group scales (loaded by the thread a
+//               batch ahead), the segment partials and the per-tile fix-up, which adds su times
+//               the adapter term U_cat . B_catT of the tile. The adapter terms of the tiles whose
+//               first block this CTA streams are computed by these threads while the pipeline fills.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -43,6 +46,8 @@ namespace {
 constexpr int kDN = 16;          // token columns: the whole batch, padded (MMA N)
 constexpr int kDThreads = 512;   // 16 warps
 constexpr int kDTmemCols = 512;
+constexpr int kMaxRpad = kDecodeMaxRpad;  // adapter rank (padded) the decode product takes
+constexpr int kIssuers = 3;      // MMA issuing threads (warps 1-3): an MMA keeps its thread ~140 cycles
 
 template <bool I8, int BITS>
 struct DCfg {
@@ -51,33 +56,26 @@ struct DCfg {
   static constexpr int kXTile = I8 ? kXAtom : 2 * kXAtom;  // 128 input channels: int8 codes or bf16
   static constexpr int kACols = I8 ? 32 : 64;             // TMEM columns of one unpacked block
   static constexpr int kKSteps = I8 ? 4 : 8;              // MMA K steps per block (32 int8 / 16 bf16)
-  // unpacked A blocks in TMEM: the loop unpack -> MMA -> slot free spans this many blocks
-  static constexpr int kASlots = I8 ? 8 : 6;
-  static constexpr int kAccSlots = (kDTmemCols - kASlots * kACols) / kDN;  // 16 (int8) / 8 (bf16)
-  static constexpr int kOwn = kAccSlots / 2;              // accumulator slots per issuer
-  static constexpr int kUcatBytes = kDN * 512 * 2;        // U_cat staging, R_pad <= 512
-  static constexpr int kSBlock = 2 * 128 * 4;             // group scale slabs of a block (2 groups x 128 rows)
-  // Three rings, all even so that each unpack team / issuer keeps its own slots:
-  //  packed blocks: freed by the unpack team as soon as it has used them, so the HBM stream only
-  //    waits on one hand-off (load -> unpack);
-  //  activation tiles: freed by the MMA commit;  scale slabs: freed by the epilogue.
-  // The last two recycle later in the pipeline, so they are deeper (and small).
-  static constexpr int kWStages = (I8 || BITS == 3) ? 16 : 12;
-  static constexpr int kXStages = I8 ? 24 : 16;
-  static constexpr int kSStages = I8 ? 24 : 16;
-  static constexpr size_t kSmem = 1024 + size_t(kXStages) * kXTile + size_t(kWStages) * kWBlock +
-                                  size_t(kSStages) * kSBlock + kUcatBytes + 1024;
-  static_assert(kWStages % 2 == 0 && kXStages % 2 == 0 && kSStages % 2 == 0, "team / issuer owned ring slots");
-  static_assert(kAccSlots % 2 == 0, "each issuer owns half of the accumulator slots");
-  static_assert(kASlots % 2 == 0, "each unpack team and issuer keeps its own A slots");
+  // unpacked blocks in TMEM (the activation tile of a block sits in the shared-memory slot of the
+  // same index): unpack -> MMA -> slot free spans this many blocks. A multiple of 6, so that each
+  // of the two unpack teams and each of the three issuers keeps its own slots.
+  static constexpr int kASlots = 6;
+  static constexpr int kBatch = I8 ? 8 : 4;               // groups per epilogue batch (16 columns each)
+  static constexpr int kBufs = 2;                         // batch buffers
+  static constexpr int kXSlots = 2 * kASlots;             // activation tiles: block i's tile in slot i % 12
+  static constexpr int kWStages = (I8 || BITS == 3) ? 20 : 16;  // packed-block ring
+  static constexpr int kScaleBatches = 4;                 // scale ring: batches in flight + the one in use
+  static constexpr size_t kSmem = 1024 + size_t(kXSlots) * kXTile + size_t(kWStages) * kWBlock +
+                                  size_t(kDN) * kMaxRpad * 4 + size_t(kScaleBatches) * kBatch * kTileN * 4 + 1024;
+  static_assert(kASlots * kACols + kBufs * kBatch * kDN <= kDTmemCols, "tensor memory");
+  static_assert(kWStages % 2 == 0 && kASlots % 6 == 0, "each unpack team / issuer keeps its own slots");
   static_assert(kSmem <= 232448, "shared memory");
 };
 
 struct DecArgs {
   const uint8_t* w_packed;
   const float* w_scale;     // [G][N] fp32, or fp16 when sw_f16
-  int sw_f16, sw_elem;      // scale bytes: 4 or 2
-  int sw_vec;               // N * sw_elem is a multiple of 16: slabs travel with the blocks
+  int sw_f16;
   const float* sa_sorted;   // [T]
   const float* su_sorted;   // [T] or nullptr (no adapters)
   const int32_t* perm;      // [T]
@@ -230,32 +228,93 @@ __device__ __forceinline__ void unpack_half_row(const uint8_t* blk, int r, int h
   }
 }
 
+// Walks the quantization groups of consecutive blocks: block position, group within the block and
+// groups of the block (the last K block of a ragged K holds fewer).
+struct GroupPos {
+  BlockPos bp;
+  int gi, ng;
+  __device__ __forceinline__ void init(BlockPos p, int gpb, int G_total) {
+    bp = p;
+    gi = 0;
+    ng = min(gpb, G_total - p.kb * gpb);
+  }
+  __device__ __forceinline__ void next(int KB, int gpb, int G_total) {
+    if (++gi == ng) {
+      gi = 0;
+      bp.next(KB);
+      ng = min(gpb, G_total - bp.kb * gpb);
+    }
+  }
+};
+
+// ad[nt][r][p] = sum_j B_catT[nt*128 + r][j] * U_cat[p][j] for p < T (zero for p >= T and rows past
+// d_out): the adapter term of row r of tile nt, fp16 inputs (U_cat staged as fp32 in u_s) and fp32
+// sums. Two passes of eight tokens keep the register footprint small (the row's second read hits L1).
+__device__ __forceinline__ void adapter_row(const DecArgs& a, const float* u_s, int nt, int r) {
+  const int o = nt * kTileN + r;
+  float4* dst = reinterpret_cast<float4*>(a.ad + (static_cast<size_t>(nt) * kTileN + r) * kDN);
+  const uint4* brow = reinterpret_cast<const uint4*>(a.bcat + static_cast<size_t>(o) * a.R_pad);
+  const int n8 = (o < a.N) ? a.R_pad / 8 : 0;
+#pragma unroll 1
+  for (int ph = 0; ph < 2; ++ph) {
+    float acc[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) acc[p] = 0.0f;
+#pragma unroll 2
+    for (int c = 0; c < n8; ++c) {
+      const uint4 bv = __ldg(brow + c);
+      const __half2* bh = reinterpret_cast<const __half2*>(&bv);
+      float bf[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(bh[q]);
+        bf[2 * q] = f.x;
+        bf[2 * q + 1] = f.y;
+      }
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const float* u = u_s + (8 * ph + p) * a.R_pad + c * 8;
+        const float4 u0 = *reinterpret_cast<const float4*>(u);
+        const float4 u1 = *reinterpret_cast<const float4*>(u + 4);
+        float t = acc[p];
+        t = fmaf(bf[0], u0.x, t);
+        t = fmaf(bf[1], u0.y, t);
+        t = fmaf(bf[2], u0.z, t);
+        t = fmaf(bf[3], u0.w, t);
+        t = fmaf(bf[4], u1.x, t);
+        t = fmaf(bf[5], u1.y, t);
+        t = fmaf(bf[6], u1.z, t);
+        t = fmaf(bf[7], u1.w, t);
+        acc[p] = t;
+      }
+    }
+    dst[2 * ph] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[2 * ph + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
 template <bool I8, int BITS>
 __global__ void __launch_bounds__(kDThreads, 1)
-    k_qdec(const __grid_constant__ CUtensorMap tm_x, const DecArgs a) {
+    k_qdec(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ DecArgs a) {
   using C = DCfg<I8, BITS>;
-  constexpr int NW = C::kWStages, NX = C::kXStages, NSS = C::kSStages, NA = C::kASlots;
+  constexpr int NW = C::kWStages, NA = C::kASlots, NX = C::kXSlots, NBUF = C::kBufs, NBATCH = C::kBatch;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xring = smem;                              // [NX][kXTile], 1024-aligned (128B swizzle)
   uint8_t* wring = xring + NX * C::kXTile;            // [NW][kWBlock]
-  uint8_t* sring = wring + NW * C::kWBlock;           // [NSS][2 groups][128 rows] group scales
-  __half* ucat_s = reinterpret_cast<__half*>(sring + NSS * C::kSBlock);  // [16][R_pad]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ucat_s) + C::kUcatBytes);
-  uint64_t* wfull = bars;                  // [NW] packed block landed (1 + bytes)
-  uint64_t* wempty = wfull + NW;           // [NW] the unpack team has used it (4 warps)
-  uint64_t* xfull = wempty + NW;           // [NX] activation tile landed (1 + bytes)
-  uint64_t* xempty = xfull + NX;           // [NX] the block's MMAs are done
-  uint64_t* sfull = xempty + NX;           // [NSS] scale slabs landed (1 + bytes)
-  uint64_t* sempty = sfull + NSS;          // [NSS] the epilogue read them (4 warps)
-  uint64_t* afull = sempty + NSS;          // [NA] A unpacked into TMEM (the 4 warps of a team)
-  uint64_t* aempty = afull + NA;           // [NA] the MMAs of the block are done (A slot free)
-  uint64_t* accf = aempty + NA;            // [kAccSlots] group sum ready
-  uint64_t* acce = accf + C::kAccSlots;    // [kAccSlots] group sum read (4 epilogue warps)
-  uint64_t* done = acce + C::kAccSlots;    // teardown
+  float* u_s = reinterpret_cast<float*>(wring + NW * C::kWBlock);  // U_cat as fp32 [16][R_pad]
+  uint32_t* sc_s = reinterpret_cast<uint32_t*>(u_s + kDN * kMaxRpad);  // [3][NBATCH][128] scale words
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sc_s + C::kScaleBatches * NBATCH * kTileN);
+  uint64_t* wfull = bars;          // [NW] packed block landed (1 + bytes)
+  uint64_t* wempty = wfull + NW;   // [NW] the unpack team has read it (4 warps)
+  uint64_t* xfull = wempty + NW;   // [NX] activation tile landed (1 + bytes)
+  uint64_t* afull = xfull + NX;    // [NA] block unpacked into TMEM (the 4 warps of a team)
+  uint64_t* mdone = afull + NA;    // [NA] the block's MMAs are done: its A slot is free
+  uint64_t* accf = mdone + NA;     // [NBUF] batch of group sums ready (one commit per issuer)
+  uint64_t* acce = accf + NBUF;    // [NBUF] batch read (4 epilogue warps)
+  uint64_t* done = acce + NBUF;    // teardown
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   int* flag_s = reinterpret_cast<int*>(tmem_slot + 1);
-  volatile int* ad_done = reinterpret_cast<volatile int*>(tmem_slot + 2);  // adapter tiles written so far
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
@@ -263,36 +322,30 @@ __global__ void __launch_bounds__(kDThreads, 1)
   const int nblk = static_cast<int>(b1 - b0);
   const int gpb = kTileK / a.group;
   const BlockPos pos0{static_cast<int>(b0 / a.KB), static_cast<int>(b0 % a.KB)};
+  // groups of this CTA's blocks (with a ragged K the last K block of each tile holds fewer) and
+  // the epilogue batches they form
+  const bool ragged = a.G_total < a.KB * gpb;
+  const int ngroups = nblk * gpb - (ragged ? static_cast<int>(b1 / a.KB - b0 / a.KB) : 0);
+  const int nbatch = (ngroups + NBATCH - 1) / NBATCH;
   int* const a_err = a.err;
-  // tiles whose first block lies in this CTA's range: their adapter terms are computed here
-  const int nt_ad0 = static_cast<int>((b0 + a.KB - 1) / a.KB), nt_ad1 = static_cast<int>((b1 - 1) / a.KB);
-  const bool any_ad = a.su_sorted != nullptr && nt_ad0 <= nt_ad1;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NW; ++s) {
-      mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 4);
+  {
+    // one barrier per thread (the arrays are contiguous: wfull, wempty, xfull, afull, mdone, accf,
+    // acce, done)
+    constexpr int kBars = 2 * NW + NX + 2 * NA + 2 * NBUF + 1;
+    static_assert(kBars <= kDThreads, "one thread per barrier");
+    const int t = threadIdx.x;
+    if (t < kBars) {
+      int count = 1;  // wfull, xfull, mdone: one arrival (+ bytes / commit)
+      if ((t >= NW && t < 2 * NW) || (t >= 2 * NW + NX && t < 2 * NW + NX + NA)) count = 4;  // wempty, afull
+      if (t >= 2 * NW + NX + 2 * NA) {
+        const int u = t - (2 * NW + NX + 2 * NA);  // accf[NBUF], acce[NBUF], done
+        count = (u < NBUF) ? kIssuers : (u < 2 * NBUF) ? 4 : kIssuers;
+      }
+      mbar_init(&bars[t], static_cast<uint32_t>(count));
+      mbar_fence_init();
     }
-    for (int s = 0; s < NX; ++s) {
-      mbar_init(&xfull[s], 1);
-      mbar_init(&xempty[s], 1);
-    }
-    for (int s = 0; s < NSS; ++s) {
-      mbar_init(&sfull[s], 1);
-      mbar_init(&sempty[s], 4);
-    }
-    *ad_done = 0;
-    for (int s = 0; s < NA; ++s) {
-      mbar_init(&afull[s], 4);
-      mbar_init(&aempty[s], 1);
-    }
-    for (int b = 0; b < C::kAccSlots; ++b) {
-      mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], 4);
-    }
-    mbar_init(done, 2);
-    mbar_fence_init();
-    prefetch_tmap(&tm_x);
+    if (t == kBars) prefetch_tmap(&tm_x);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kDTmemCols);
@@ -301,88 +354,99 @@ __global__ void __launch_bounds__(kDThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t colA = 0, colAcc = NA * C::kACols;
-  grid_dep_wait();
+  const uint32_t colA = 0, colAcc = NA * C::kACols;  // A slots, then the batch buffers
   grid_dep_launch();
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // per block: the packed block, its activation tile and its scale slabs, each into its own ring
+    // ------------------------------------------------------------ packed blocks
+    // No earlier kernel writes the packed weights, so this warp streams them without waiting for
+    // the previous grid.
     if (lane == 0) {
       int i = 0;
-      BlockPos bp = pos0;
-      bool ok = true;
-      for (; i < nblk; ++i, bp.next(a.KB)) {
-        const int kb = bp.kb;
-        const int sw = i % NW, sx = i % NX, ss = i % NSS;
-        if (!mbar_wait(&wempty[sw], ((i / NW) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&wfull[sw], C::kWBlock);
-        bulk_load(wring + sw * C::kWBlock, a.w_packed + (b0 + i) * C::kWBlock, C::kWBlock, &wfull[sw]);
-        if (!mbar_wait(&xempty[sx], ((i / NX) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) {
-          ok = false;
-          ++i;
-          break;
-        }
-        mbar_arrive_expect_tx(&xfull[sx], C::kXTile);
-        tma_load_2d(xring + sx * C::kXTile, &tm_x, kb * kTileK, 0, &xfull[sx]);
-        if constexpr (!I8) tma_load_2d(xring + sx * C::kXTile + C::kXAtom, &tm_x, kb * kTileK + 64, 0, &xfull[sx]);
-        if (!mbar_wait(&sempty[ss], ((i / NSS) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) {
-          ok = false;
-          ++i;
-          break;
-        }
-        // the 128-row scale slab of each of the block's groups (contiguous: group-major [G][N]);
-        // with a row pitch that is not a multiple of 16 bytes the epilogue reads its scales itself
-        const int ng = min(gpb, a.G_total - kb * gpb);
-        const int o0 = bp.nt * kTileN;
-        const uint32_t scopy = a.sw_vec ? static_cast<uint32_t>(min(128, a.N - o0) * a.sw_elem) : 0u;
-        mbar_arrive_expect_tx(&sfull[ss], ng * scopy);
-        for (int gi = 0; gi < (scopy ? ng : 0); ++gi)
-          bulk_load(sring + ss * C::kSBlock + gi * 512,
-                    reinterpret_cast<const uint8_t*>(a.w_scale) +
-                        (static_cast<size_t>(kb * gpb + gi) * a.N + o0) * a.sw_elem,
-                    scopy, &sfull[ss]);
+      for (; i < nblk; ++i) {
+        const int s = i % NW;
+        if (!mbar_wait(&wempty[s], ((i / NW) & 1) ^ 1, a_err, DEVERR_WAIT_PRODUCER)) break;
+        mbar_arrive_expect_tx(&wfull[s], C::kWBlock);
+        bulk_load(wring + s * C::kWBlock, a.w_packed + (b0 + i) * C::kWBlock, C::kWBlock, &wfull[s]);
       }
-      (void)ok;
       drain_ring(wfull, NW, i);
-      drain_ring(xfull, NX, i);
-      drain_ring(sfull, NSS, i);
     }
-  } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------------------------ MMA issuers (alternate blocks)
+  } else if (warp >= 1 && warp <= kIssuers) {
+    // ------------------------------------------------------------ MMA issuers (every third block)
     const int qi = warp - 1;
+    grid_dep_wait();  // the activation tiles are the previous grid's output
     if (lane == 0) {
+      // Each issuer loads the activation tiles of its own blocks, NA blocks ahead. Block j's tile
+      // goes to slot j % NX, which last held block j - NX's; it is requested once this issuer has
+      // seen afull of block j - NA, whose A slot the unpack team refilled only after the MMAs of
+      // block j - 2 NA = j - NX were done. Blocks j and j - NA have the same issuer.
+      int ix = qi;             // next own block whose tile is requested
+      BlockPos xb = pos0;      // position of block ix
+      for (int t = 0; t < qi; ++t) xb.next(a.KB);
+      auto request_tile = [&]() {
+        const int s = ix % NX;
+        mbar_arrive_expect_tx(&xfull[s], C::kXTile);
+        tma_load_2d(xring + s * C::kXTile, &tm_x, xb.kb * kTileK, 0, &xfull[s]);
+        if constexpr (!I8) tma_load_2d(xring + s * C::kXTile + C::kXAtom, &tm_x, xb.kb * kTileK + 64, 0, &xfull[s]);
+        ix += kIssuers;
+        for (int t = 0; t < kIssuers; ++t) xb.next(a.KB);
+      };
+      while (ix < nblk && ix < NA) request_tile();  // the first NA blocks' tiles: slots never used
       const uint32_t idesc = I8 ? idesc_i8(128, kDN) : idesc_bf16(128, kDN);
       const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xring));
-      int own = 0;
       bool ok = true;
+      int acquired = 0;   // batches whose buffer this issuer has waited for (in order)
+      int committed = 0;  // batches this issuer has committed (in order)
+      // the buffer of batch b is free once the epilogue has drained batch b - NBUF
+      auto acquire = [&](int b) {
+        while (ok && acquired <= b) {
+          ok = mbar_wait(&acce[acquired % NBUF], ((acquired / NBUF) & 1) ^ 1, a_err, DEVERR_WAIT_MMA);
+          if (ok) {
+            tc_fence_after();
+            ++acquired;
+          }
+        }
+      };
+      // this issuer has issued all its groups of the batches before b: one commit each (a batch
+      // is committed only after its buffer was acquired, so an arrival never lands in the
+      // barrier's previous phase)
+      auto commit_before = [&](int b) {
+        while (ok && committed < b) {
+          acquire(committed);
+          if (!ok) break;
+          tc_commit(&accf[committed % NBUF]);
+          ++committed;
+        }
+      };
       BlockPos bp = pos0;
-      if (qi) bp.next(a.KB);
-      for (int i = qi; i < nblk && ok; i += 2, bp.next(a.KB), bp.next(a.KB)) {
-        const int sx = i % NX, as = i % NA;
-        const int kb = bp.kb;
-        const int ng = min(gpb, a.G_total - kb * gpb);
-        if (!mbar_wait(&afull[as], (i / NA) & 1, a_err, DEVERR_WAIT_MMA) ||
-            !mbar_wait(&xfull[sx], (i / NX) & 1, a_err, DEVERR_WAIT_MMA)) {
+      int gidx = 0;  // first group of block i in this CTA's group sequence
+      for (int i = 0; i < nblk && ok; ++i, bp.next(a.KB)) {
+        const int ng = min(gpb, a.G_total - bp.kb * gpb);
+        if (i % kIssuers != qi) {
+          gidx += ng;
+          continue;
+        }
+        const int s = i % NA, sx = i % NX;
+        if (!mbar_wait(&afull[s], (i / NA) & 1, a_err, DEVERR_WAIT_MMA)) {
+          ok = false;
+          break;
+        }
+        // block i's A slot held block i - NA before: that block's MMAs are done (the unpack team
+        // waited for them), so the tile slot of block i + NA (= block i - NA's) is free
+        while (ix < nblk && ix <= i + NA) request_tile();
+        if (!mbar_wait(&xfull[sx], (i / NX) & 1, a_err, DEVERR_WAIT_MMA)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint64_t xdesc = xdesc0 + static_cast<uint64_t>((sx * C::kXTile) >> 4);
-        const uint32_t a_col = tmem + colA + as * C::kACols;
-        for (int gi = 0; gi < ng; ++gi) {
-          const int slot = qi + 2 * (own % C::kOwn);
-          const uint32_t use = static_cast<uint32_t>(own / C::kOwn);
-          ++own;
-          if (!mbar_wait(&acce[slot], (use & 1u) ^ 1u, a_err, DEVERR_WAIT_MMA)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d = tmem + colAcc + slot * kDN;
+        const uint32_t a_col = tmem + colA + s * C::kACols;
+        for (int gi = 0; gi < ng; ++gi, ++gidx) {
+          const int bt = gidx / NBATCH;
+          commit_before(bt);
+          acquire(bt);
+          if (!ok) break;
+          const uint32_t d = tmem + colAcc + (bt % NBUF) * (NBATCH * kDN) + (gidx % NBATCH) * kDN;
           const int k0 = (gpb == 1) ? 0 : gi * (C::kKSteps / 2);
           const int nk = (gpb == 1) ? C::kKSteps : C::kKSteps / 2;
           for (int kk = 0; kk < nk; ++kk) {
@@ -396,152 +460,89 @@ __global__ void __launch_bounds__(kDThreads, 1)
               mma_f16_ta(d, a_col + ks * 8, xdesc + offb, idesc, kk > 0 ? 1u : 0u);
             }
           }
-          tc_commit(&accf[slot]);
         }
-        tc_commit(&aempty[as]);
-        tc_commit(&xempty[sx]);
+        if (!ok) break;
+        tc_commit(&mdone[s]);
       }
+      commit_before(nbatch);
+      // tiles still in flight after a wait ran out must land before the CTA exits
+      for (int j = ix - kIssuers; j >= 0 && j >= ix - NX; j -= kIssuers)
+        mbar_wait_for(&xfull[j % NX], static_cast<uint32_t>((j / NX) & 1), nullptr, 0, kDrainLimitNs);
       tc_commit(done);
       mbar_wait(done, 0, a_err, DEVERR_WAIT_TEARDOWN);
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ adapter terms (CUDA cores)
-    // ad[nt][r][p] = sum_j B_catT[o][j] * U_cat[p][j] (fp16 inputs, fp32 sums) for every tile whose
-    // first block this CTA streams; lane l takes rows l, l+32, l+64, l+96. Off the epilogue's path:
-    // the segment holding a tile's first block waits for that tile's term (the count ad_done)
-    // only when it finishes.
-    if (any_ad) {
-      const int rp = a.R_pad, T = a.T;
-      for (int e = lane; e < kDN * rp / 8; e += 32) {
-        const int p = e / (rp / 8), c8 = e % (rp / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (p < T) v = __ldg(reinterpret_cast<const uint4*>(a.ucat + static_cast<size_t>(p) * rp) + c8);
-        *reinterpret_cast<uint4*>(ucat_s + static_cast<size_t>(p) * rp + c8 * 8) = v;
-      }
-      __syncwarp();
-      for (int nt = nt_ad0; nt <= nt_ad1; ++nt) {
-        for (int rr = 0; rr < 4; ++rr) {
-          const int r = lane + 32 * rr;
-          const int o = nt * kTileN + r;
-          float adr[kDN];
-#pragma unroll
-          for (int p = 0; p < kDN; ++p) adr[p] = 0.0f;
-          if (o < a.N) {
-            const uint4* brow = reinterpret_cast<const uint4*>(a.bcat + static_cast<size_t>(o) * rp);
-            for (int c0 = 0; c0 < rp / 8; c0 += 8) {
-              uint4 bv[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k) bv[k] = (c0 + k < rp / 8) ? __ldg(brow + c0 + k) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                if (c0 + k >= rp / 8) break;
-                const __half2* bh = reinterpret_cast<const __half2*>(&bv[k]);
-                float2 bf[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) bf[q] = __half22float2(bh[q]);
-#pragma unroll
-                for (int p = 0; p < kDN; ++p) {
-                  if (p >= T) break;
-                  const uint4 uv = *reinterpret_cast<const uint4*>(ucat_s + static_cast<size_t>(p) * rp + (c0 + k) * 8);
-                  const __half2* uh = reinterpret_cast<const __half2*>(&uv);
-                  float sacc = adr[p];
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    const float2 uf = __half22float2(uh[q]);
-                    sacc = fmaf(bf[q].x, uf.x, sacc);
-                    sacc = fmaf(bf[q].y, uf.y, sacc);
-                  }
-                  adr[p] = sacc;
-                }
-              }
-            }
-          }
-          float4* dst = reinterpret_cast<float4*>(a.ad + (static_cast<size_t>(nt) * kTileN + r) * kDN);
-#pragma unroll
-          for (int k = 0; k < kDN / 4; ++k) dst[k] = make_float4(adr[4 * k], adr[4 * k + 1], adr[4 * k + 2], adr[4 * k + 3]);
-        }
-        // this tile's term is in memory: the epilogue can finish the tile's first segment
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) *ad_done = nt - nt_ad0 + 1;
-      }
-    }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ unpack into TMEM
-    // Two teams of four warps (one per TMEM lane quarter) take alternate blocks, so two blocks are
-    // in flight; each thread unpacks one full row of the block.
+    // Two teams of four warps (one per TMEM lane quarter) take alternate blocks; each thread
+    // unpacks one full row of the block. Only this kernel's shared memory is read: no wait for
+    // the previous grid.
     const int q4 = warp & 3, team = (warp - 4) >> 2;
     const int r = 32 * q4 + lane;  // block row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
     for (int i = team; i < nblk; i += 2) {
-      const int sw = i % NW, as = i % NA;
+      const int sw = i % NW, s = i % NA;
       if (!mbar_wait(&wfull[sw], (i / NW) & 1, a_err, DEVERR_WAIT_UNPACK) ||
-          !mbar_wait(&aempty[as], ((i / NA) & 1) ^ 1, a_err, DEVERR_WAIT_UNPACK))
+          !mbar_wait(&mdone[s], ((i / NA) & 1) ^ 1, a_err, DEVERR_WAIT_UNPACK))
         break;
       tc_fence_after();
-      const uint32_t ta = tmem + lane_base + colA + as * C::kACols;
+      const uint32_t ta = tmem + lane_base + colA + s * C::kACols;
       unpack_half_row<I8, BITS>(wring + sw * C::kWBlock, r, 0, ta);
       unpack_half_row<I8, BITS>(wring + sw * C::kWBlock, r, 1, ta + C::kACols / 2);
-      // the packed block's values have been used (the stores below hold them): free its slot now,
-      // so the next load can land while this block goes through the MMA
+      // the packed block's values have been read (the stores below hold them): free its slot now
       __syncwarp();
       if (lane == 0) mbar_arrive(&wempty[sw]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[as]);
+      if (lane == 0) mbar_arrive(&afull[s]);
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------------ epilogue, one output row per thread
-    // Control flow follows the block schedule only; after a wait ran out, `ok` turns off every
+    // Control flow follows the group schedule only; after a wait ran out, `ok` turns off every
     // later wait and TMEM access, and the named barriers are still reached by all four warps.
+    grid_dep_wait();
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;
     const int et = threadIdx.x - 384;  // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
     const int T = a.T;
-    // the group scales of block i: the 128-row slab(s) the producer copied into ring slot i % NS
-    // (or, when a row of scales is not a multiple of 16 bytes, this thread's own scale from memory)
-    auto scale_at = [&](int s, int gi, int nt, int j) -> float {
-      if (a.sw_vec) {
-        const uint8_t* slab = sring + s * C::kSBlock + gi * 512;
-        if (a.sw_f16) return __half2float(*reinterpret_cast<const __half*>(slab + r * 2));
-        return *reinterpret_cast<const float*>(slab + r * 4);
+
+    // U_cat as fp32 for the adapter terms (computed when this CTA publishes the first segment of a
+    // tile: any CTA's fix-up of the tile reads them only after that)
+    if (a.su_sorted) {
+      const int nv = kDN * a.R_pad / 8;  // 8 halves per vector; R_pad is a multiple of 8
+      for (int v = et; v < nv; v += 128) {
+        const int p = (v * 8) / a.R_pad, j = v * 8 - p * a.R_pad;
+        float4 lo = make_float4(0.0f, 0.0f, 0.0f, 0.0f), hi = lo;
+        if (p < T) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.ucat + static_cast<size_t>(p) * a.R_pad + j));
+          const __half2* h = reinterpret_cast<const __half2*>(&u);
+          const float2 f0 = __half22float2(h[0]), f1 = __half22float2(h[1]), f2 = __half22float2(h[2]),
+                       f3 = __half22float2(h[3]);
+          lo = make_float4(f0.x, f0.y, f1.x, f1.y);
+          hi = make_float4(f2.x, f2.y, f3.x, f3.y);
+        }
+        *reinterpret_cast<float4*>(u_s + v * 8) = lo;
+        *reinterpret_cast<float4*>(u_s + v * 8 + 4) = hi;
       }
-      const int o = nt * kTileN + r;
-      return (o < a.N) ? load_scale(a.w_scale, static_cast<size_t>(j) * a.N + o, a.sw_f16) : 0.0f;
-    };
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
 
     bool ok = true;
-    int cnt0 = 0, cnt1 = 0;  // groups drained from issuer 0 / 1
     float acc[kDN];
 #pragma unroll
     for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
     int cur_nt = -1;
-    bool cur_ad = false;     // this segment holds its tile's first block
 
     // End of a segment of tile nt: a tile held by this CTA alone is written at once; otherwise the
     // partial goes to its slot and the last CTA to finish the tile adds the partials in segment order.
-    auto finish_segment = [&](int nt, bool has_first) {
+    auto finish_segment = [&](int nt) {
       const int64_t f0 = static_cast<int64_t>(nt) * a.KB;
       const int c_first = cta_of(f0, a.NB, G);
       const int nseg = cta_of(f0 + a.KB - 1, a.NB, G) - c_first + 1;
       const int seg = c - c_first;
       const int o = nt * kTileN + r;
       const size_t tile_row = (static_cast<size_t>(nt) * kTileN + r) * kDN;
-      // the adapter term of this tile was computed by warp 3 of this CTA
-      if (has_first && a.su_sorted && ok) {
-        // warp 3 writes the terms in tile order; this is tile nt - nt_ad0 of that list
-        const int need = nt - nt_ad0 + 1;
-        bool got = *ad_done >= need;
-        if (!got) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!(got = (*ad_done >= need)) && globaltimer_ns() - t0 < kWaitLimitNs) __nanosleep(256);
-        }
-        if (!got) record_error(a_err, DEVERR_WAIT_EPILOGUE);
-        __threadfence_block();
-        ok = __all_sync(0xffffffffu, got);
-      }
       bool last = true;
       if (nseg > 1) {
         float4* dst = reinterpret_cast<float4*>(a.part + (static_cast<size_t>(nt) * a.maxseg + seg) * kTileN * kDN +
@@ -608,66 +609,130 @@ __global__ void __launch_bounds__(kDThreads, 1)
       }
     };
 
-    BlockPos bp = pos0;
-    for (int i = 0; i < nblk; ++i, bp.next(a.KB)) {
-      const int nt = bp.nt, kb = bp.kb;
-      if (nt != cur_nt) {
-        if (cur_nt >= 0) finish_segment(cur_nt, cur_ad);
-        cur_nt = nt;
-        cur_ad = kb == 0;
-#pragma unroll
-        for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
+    // group scales, one per group and row, copied by the thread itself (cp.async) into its own
+    // column of a four-batch ring: batch bt + 3 is requested when batch bt starts. An fp16 scale
+    // travels in the aligned 4-byte pair that holds it.
+    GroupPos pf;
+    pf.init(pos0, gpb, a.G_total);
+    int pf_left = ngroups;
+    const size_t sc_total = static_cast<size_t>(a.G_total) * a.N;
+    auto request_batch_scales = [&](int bt) {
+      uint32_t* dst = sc_s + (bt % C::kScaleBatches) * NBATCH * kTileN + et;
+      for (int k = 0; k < NBATCH && pf_left > 0; ++k, --pf_left, pf.next(a.KB, gpb, a.G_total)) {
+        const int o = pf.bp.nt * kTileN + r;
+        if (o >= a.N) continue;
+        const size_t idx = static_cast<size_t>(pf.bp.kb * gpb + pf.gi) * a.N + o;
+        if (a.sw_f16) {
+          const size_t e0 = idx & ~size_t(1);
+          cp_async4_n(dst + k * kTileN, reinterpret_cast<const unsigned short*>(a.w_scale) + e0,
+                      (e0 + 1 < sc_total) ? 4u : 2u);
+        } else {
+          cp_async4_n(dst + k * kTileN, a.w_scale + idx, 4u);
+        }
       }
-      // this block's scale slabs (the phase cannot move on before this epilogue frees the slot,
-      // so the parity wait is exact)
-      const int ss = i % NSS;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sfull[ss], (i / NSS) & 1, a_err, DEVERR_WAIT_EPILOGUE));
-      const float s0 = scale_at(ss, 0, nt, kb * gpb);
-      const float s1 = (gpb == 2) ? scale_at(ss, 1, nt, kb * gpb + 1) : 0.0f;
-      const int q = i & 1;
-      const int ng = min(gpb, a.G_total - kb * gpb);
-      for (int gi = 0; gi < ng; ++gi) {
-        const int n_q = q ? cnt1 : cnt0;
-        const int slot = q + 2 * (n_q % C::kOwn);
-        const uint32_t use = static_cast<uint32_t>(n_q / C::kOwn);
-        if (q) ++cnt1;
-        else ++cnt0;
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[slot], use & 1u, a_err, DEVERR_WAIT_EPILOGUE));
-        if (!ok) continue;
-        tc_fence_after();
-        uint32_t v[kDN];
-        tmem_ld16(tmem + lane_base + colAcc + slot * kDN, v);
-        tmem_wait_ld();
-        reg_fence(v);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acce[slot]);
-        const float sw = gi ? s1 : s0;
-        if constexpr (I8) {
-          const float swq = sw * 0.0625f;  // codes entered the MMA as 16*q
+      cp_async_commit();
+    };
+    // the scale of group k of batch bt (j = its group index in the weight's group order, o its row)
+    auto scale_of = [&](int bt, int k, int j, int o) -> float {
+      const uint32_t w = sc_s[((bt % C::kScaleBatches) * NBATCH + k) * kTileN + et];
+      if (a.sw_f16) {
+        const bool high = ((static_cast<int64_t>(j) * a.N + o) & 1) != 0;
+        const unsigned short h = static_cast<unsigned short>(high ? (w >> 16) : (w & 0xFFFFu));
+        float f;
+        asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
+        return f;
+      }
+      return __uint_as_float(w);
+    };
+    for (int b = 0; b < C::kScaleBatches - 1; ++b) request_batch_scales(b);
+
+    // A new tile starts in the group sequence: finish the previous one; when this CTA streams the
+    // tile's first block, compute the tile's adapter term now (it goes out with this CTA's segment,
+    // before any fix-up of the tile can read it)
+    auto enter_tile = [&](int nt, int kb) {
+      if (cur_nt >= 0) finish_segment(cur_nt);
+      cur_nt = nt;
 #pragma unroll
-          for (int p = 0; p < kDN; ++p) acc[p] = fmaf(static_cast<float>(static_cast<int32_t>(v[p])), swq, acc[p]);
-          if (a.dbg_acc) {
-            const int o = nt * kTileN + r;
-            if (o < a.N) {
+      for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
+      if (a.su_sorted && kb == 0) adapter_row(a, u_s, nt, r);
+    };
+
+    GroupPos gp;
+    gp.init(pos0, gpb, a.G_total);
+    int gleft = ngroups;
+    for (int bt = 0; bt < nbatch; ++bt) {
+      request_batch_scales(bt + C::kScaleBatches - 1);
+      cp_async_wait_group<C::kScaleBatches - 1>();  // batch bt's scales have landed (this thread's own copies)
+      const int buf = bt % NBUF;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (bt / NBUF) & 1, a_err, DEVERR_WAIT_EPILOGUE));
+      if (ok) tc_fence_after();
+      const int nb = min(NBATCH, gleft);
+      gleft -= nb;
+      const uint32_t bcol = tmem + lane_base + colAcc + buf * (NBATCH * kDN);
+      if (gp.bp.nt != cur_nt) enter_tile(gp.bp.nt, gp.bp.kb);
+      const int j0 = gp.bp.kb * gpb + gp.gi;
+      if (ok && nb == NBATCH && nb <= a.G_total - j0 && !a.dbg_acc) {
+        // the whole batch lies in the current tile: its groups are consecutive in the weight's
+        // group order (j0 .. j0 + 7), read two at a time
+        const int o = cur_nt * kTileN + r;
+#pragma unroll
+        for (int h = 0; h < NBATCH / 2; ++h) {
+          uint32_t v[2 * kDN];
+          tmem_ld32(bcol + h * 2 * kDN, v);
+          tmem_wait_ld();
+          reg_fence(v);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const float sw = scale_of(bt, 2 * h + k, j0 + 2 * h + k, o);
+            if constexpr (I8) {
+              const float swq = sw * 0.0625f;  // codes entered the MMA as 16*q
+#pragma unroll
+              for (int p = 0; p < kDN; ++p)
+                acc[p] = fmaf(static_cast<float>(static_cast<int32_t>(v[k * kDN + p])), swq, acc[p]);
+            } else {
+#pragma unroll
+              for (int p = 0; p < kDN; ++p) acc[p] = fmaf(__uint_as_float(v[k * kDN + p]), sw, acc[p]);
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < NBATCH; ++k) gp.next(a.KB, gpb, a.G_total);
+      } else {
+        for (int k = 0; k < nb; ++k, gp.next(a.KB, gpb, a.G_total)) {
+          const int nt = gp.bp.nt;
+          if (nt != cur_nt) enter_tile(nt, gp.bp.kb);
+          if (!ok) continue;
+          uint32_t v[kDN];
+          tmem_ld16(bcol + k * kDN, v);
+          tmem_wait_ld();
+          reg_fence(v);
+          const int j = gp.bp.kb * gpb + gp.gi, o = nt * kTileN + r;
+          const float sw = (o < a.N) ? scale_of(bt, k, j, o) : 0.0f;
+          if constexpr (I8) {
+            const float swq = sw * 0.0625f;  // codes entered the MMA as 16*q
+#pragma unroll
+            for (int p = 0; p < kDN; ++p) acc[p] = fmaf(static_cast<float>(static_cast<int32_t>(v[p])), swq, acc[p]);
+            if (a.dbg_acc && o < a.N) {
 #pragma unroll
               for (int p = 0; p < kDN; ++p) {
                 if (p >= T) break;
-                a.dbg_acc[(static_cast<size_t>(__ldg(a.perm + p)) * a.N + o) * a.G_total + kb * gpb + gi] =
+                a.dbg_acc[(static_cast<size_t>(__ldg(a.perm + p)) * a.N + o) * a.G_total + j] =
                     static_cast<int32_t>(v[p]) / 16;
               }
             }
-          }
-        } else {
+          } else {
 #pragma unroll
-          for (int p = 0; p < kDN; ++p) acc[p] = fmaf(__uint_as_float(v[p]), sw, acc[p]);
+            for (int p = 0; p < kDN; ++p) acc[p] = fmaf(__uint_as_float(v[p]), sw, acc[p]);
+          }
         }
       }
-      // the block's scales have been read: the slot can take a later block's
+      // the batch's sums are in registers: the buffer can take batch bt + NBUF
+      if (ok) tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sempty[ss]);
+      if (ok && lane == 0) mbar_arrive(&acce[buf]);
     }
-    if (cur_nt >= 0) finish_segment(cur_nt, cur_ad);
+    if (cur_nt >= 0) finish_segment(cur_nt);
+    cp_async_wait_group<0>();
     tc_fence_before();
   }
   __syncthreads();
@@ -733,8 +798,6 @@ cudaError_t launch_qdec(int w_bits, bool int8, const CUtensorMap& tm_x, const De
   a.w_packed = q.w_packed;
   a.w_scale = q.w_scale;
   a.sw_f16 = q.sw_f16;
-  a.sw_elem = q.sw_f16 ? 2 : 4;
-  a.sw_vec = ((static_cast<int64_t>(q.N) * a.sw_elem) % 16) == 0 ? 1 : 0;
   a.sa_sorted = q.sa_sorted;
   a.su_sorted = q.su_sorted;
   a.perm = q.perm;
@@ -757,7 +820,7 @@ cudaError_t launch_qdec(int w_bits, bool int8, const CUtensorMap& tm_x, const De
   a.cnt = cnt;
   a.dbg_acc = q.dbg_acc;
   a.err = q.err;
-  if (q.T > kDN || q.T < 1 || R_pad > 512) return cudaErrorInvalidValue;
+  if (q.T > kDN || q.T < 1 || R_pad > kMaxRpad || R_pad % 8 != 0) return cudaErrorInvalidValue;
   if (int8) {
     if (w_bits != 4) return cudaErrorInvalidValue;
     return launch_qdec_t<true, 4>(tm_x, a, plan.grid, st);

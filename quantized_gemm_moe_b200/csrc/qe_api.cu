@@ -84,7 +84,7 @@ Plan make_plan(const qe_layer_desc* d, int T, bool x_bf16) {
   p.has_ad = p.g.R_a > 0;
   const int Tm = std::max(T, 1);
   p.up = plan_ugemm(Tm, p.K, p.g.R_tot);
-  p.dec = Tm <= kDecodeMaxT;
+  p.dec = Tm <= kDecodeMaxT && (!p.has_ad || p.g.R_pad <= kDecodeMaxRpad);
   if (p.dec) {
     p.dp = plan_decode(p.N, p.K, decode_grid_sms());
     p.bn = 16;

@@ -199,6 +199,7 @@ cudaError_t launch_qdec(int w_bits, bool int8, const CUtensorMap& tm_x, const De
                         const uint16_t* ucat, const uint16_t* bcat, int R_pad, float* part, float* ad,
                         unsigned* cnt, cudaStream_t st);
 constexpr int kDecodeMaxT = 16;
+constexpr int kDecodeMaxRpad = 384;  // the decode product stages U_cat in shared memory
 
 // Weight-only (W3A16 / W4A16) product on the tensor cores: codes unpacked to bf16, bf16
 // activations (act16, bucket order), per-group fp32 sums scaled by sw, adapter epilogue.

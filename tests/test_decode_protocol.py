@@ -6,13 +6,15 @@
    segments than the workspace holds (the partial slot index stays in bounds), and that the
    per-tile fix-up (the last of the tile's segments to arrive adds them in segment order) runs
    exactly once per tile, whatever order the CTAs finish in.
-2. The mbarrier protocol: a producer fills the packed-block ring in order, two teams of four
-   unpack warps take alternate blocks and put each into one of four TMEM A slots, two issuers take
-   alternate blocks (issuer q owns accumulator slots q, q+2, ...), four epilogue warps drain the
-   groups in block order. Three rings: packed blocks (freed by the unpack team once used),
-   activation tiles (freed by the MMA commit) and scale slabs (freed by the epilogue). Random
-   interleavings; every parity wait must be sound (the barrier has completed n or n+1 phases
-   when a wait for phase n passes) and everything must finish.
+2. The mbarrier protocol: one thread streams the packed blocks into a ring that the unpack team
+   frees as soon as it has read a block; two teams of four unpack warps take alternate blocks;
+   three issuers take every third block, each loading the activation tiles of its own blocks NA
+   blocks ahead into a 2 NA ring (the tile of block j is requested after afull of block j - NA,
+   which implies that block j - 2 NA's MMAs, the slot's previous user, are done), and commit once
+   per block (freeing the A slot) and once per batch of groups (two batch buffers); four epilogue
+   warps drain the batches in order. Random interleavings and random commit delays; every parity wait
+   must be sound (the barrier has completed n or n+1 phases when a wait for phase n passes),
+   every commit must land in the phase it is meant for, and everything must finish.
 """
 import random
 
@@ -108,82 +110,125 @@ def test_fixup_runs_once_per_tile_in_segment_order(N, K):
         assert all(v == 0 for v in cnt)                             # counters left at zero
 
 
-def run_decode_model(nblk, gpb_of, NW, NX, NSS, NA, n_slots, rng, n_unpack=8, n_epi=4):
-    """nblk blocks; gpb_of(i) = groups of block i (1, or 2 at g = 64)."""
+class TaggedBarrier(Barrier):
+    """A barrier whose arrivals say which phase they belong to (a commit must never land in an
+    earlier phase that is still open)."""
+
+    def arrive_for(self, phase, who):
+        if phase != self.done:
+            raise Unsound(f"{who}: arrival for phase {phase} of {self.name} landed in phase {self.done}")
+        self.arrive()
+
+
+def run_decode_model(nblk, gpb_of, NW, NA, rng, NBUF=2, NBATCH=8, n_epi=4, n_iss=3):
+    """nblk blocks; gpb_of(i) = groups of block i (1, or 2 at g = 64, 1 for the ragged last K block)."""
     wfull = [Barrier(f"wfull{i}", 1) for i in range(NW)]
-    wempty = [Barrier(f"wempty{i}", n_unpack // 2) for i in range(NW)]
-    xfull = [Barrier(f"xfull{i}", 1) for i in range(NX)]
-    xempty = [Barrier(f"xempty{i}", 1) for i in range(NX)]
-    sfull = [Barrier(f"sfull{i}", 1) for i in range(NSS)]
-    sempty = [Barrier(f"sempty{i}", n_epi) for i in range(NSS)]
-    afull = [Barrier(f"afull{i}", n_unpack // 2) for i in range(NA)]
-    aempty = [Barrier(f"aempty{i}", 1) for i in range(NA)]
-    accf = [Barrier(f"accf{i}", 1) for i in range(n_slots)]
-    acce = [Barrier(f"acce{i}", n_epi) for i in range(n_slots)]
-    own_n = n_slots // 2
+    wempty = [Barrier(f"wempty{i}", 4) for i in range(NW)]
+    NX = 2 * NA
+    xfull = [TaggedBarrier(f"xfull{i}", 1) for i in range(NX)]
+    x_reader_done = {}   # block -> its tile has been consumed by an issued MMA that completed
+    afull = [Barrier(f"afull{i}", 4) for i in range(NA)]
+    mdone = [TaggedBarrier(f"mdone{i}", 1) for i in range(NA)]
+    accf = [TaggedBarrier(f"accf{i}", n_iss) for i in range(NBUF)]
+    acce = [Barrier(f"acce{i}", n_epi) for i in range(NBUF)]
+    ngroups = sum(gpb_of(i) for i in range(nblk))
+    nbatch = -(-ngroups // NBATCH)
     pending = []
 
-    def producer():
+    def later(fn, *args):
+        pending.append([rng.randint(1, 6), lambda: fn(*args)])
+
+    def w_producer():
         for i in range(nblk):
-            for full, empty, depth in ((wfull, wempty, NW), (xfull, xempty, NX), (sfull, sempty, NSS)):
-                s, n = i % depth, i // depth
-                if n > 0:
-                    yield from _wait(empty[s], n - 1, "producer")
-                pending.append([rng.randint(1, 8), full[s].arrive])
-                yield
+            s, n = i % NW, i // NW
+            if n > 0:
+                yield from _wait(wempty[s], n - 1, "w_producer")
+            later(wfull[s].arrive)
+            yield
 
     def unpack(k):
-        team = k // 4          # two teams of four warps take alternate blocks
+        team = k // 4
         for i in range(team, nblk, 2):
-            s, a = i % NW, i % NA
-            yield from _wait(wfull[s], i // NW, f"unpack{k}")
+            sw, s = i % NW, i % NA
+            yield from _wait(wfull[sw], i // NW, f"unpack{k}")
             if i // NA > 0:
-                yield from _wait(aempty[a], i // NA - 1, f"unpack{k}")
+                yield from _wait(mdone[s], i // NA - 1, f"unpack{k}")
             for _ in range(rng.randint(0, 3)):
                 yield
-            wempty[s].arrive()     # the packed block has been used
-            afull[a].arrive()
+            wempty[sw].arrive()
+            yield
+            afull[s].arrive()
 
     def issuer(q):
-        own = 0
-        for i in range(q, nblk, 2):
-            a, sx = i % NA, i % NX
-            yield from _wait(afull[a], i // NA, f"issuer{q}")
-            yield from _wait(xfull[sx], i // NX, f"issuer{q}")
-            for _ in range(gpb_of(i)):
-                slot, use = q + 2 * (own % own_n), own // own_n
-                own += 1
-                if use > 0:
-                    yield from _wait(acce[slot], use - 1, f"issuer{q}")
+        st = {"acq": 0, "com": 0}
+
+        def acquire(b):
+            while st["acq"] <= b:
+                a = st["acq"]
+                if a // NBUF > 0:
+                    yield from _wait(acce[a % NBUF], a // NBUF - 1, f"issuer{q}")
+                st["acq"] += 1
+
+        def commit_before(b):
+            while st["com"] < b:
+                cb = st["com"]
+                yield from acquire(cb)
+                later(accf[cb % NBUF].arrive_for, cb // NBUF, f"issuer{q}")
+                st["com"] += 1
+
+        st["ix"] = q
+
+        def request_tiles(upto):
+            while st["ix"] < nblk and st["ix"] <= upto:
+                j = st["ix"]
+                if j >= NX and not x_reader_done.get(j - NX, False):
+                    raise Unsound(f"issuer{q}: tile of block {j} requested while block {j - NX} may still read the slot")
+                later(xfull[j % NX].arrive_for, j // NX, f"issuer{q}")
+                st["ix"] += n_iss
+
+        request_tiles(NA - 1)
+        gidx = 0
+        for i in range(nblk):
+            ng = gpb_of(i)
+            if i % n_iss != q:
+                gidx += ng
+                continue
+            s = i % NA
+            yield from _wait(afull[s], i // NA, f"issuer{q}")
+            request_tiles(i + NA)
+            yield from _wait(xfull[i % NX], i // NX, f"issuer{q}")
+            for _ in range(ng):
+                bt = gidx // NBATCH
+                yield from commit_before(bt)
+                yield from acquire(bt)
                 yield
-                pending.append([rng.randint(1, 5), accf[slot].arrive])
-            pending.append([rng.randint(1, 5), aempty[a].arrive])
-            pending.append([rng.randint(1, 5), xempty[sx].arrive])
+                gidx += 1
+            def mma_done(i=i, s=s):
+                x_reader_done[i] = True
+                mdone[s].arrive_for(i // NA, f"issuer{q}")
+            later(mma_done)
+        yield from commit_before(nbatch)
 
     def epilogue(k):
-        n = [0, 0]
-        for i in range(nblk):
-            q, ss = i & 1, i % NSS
-            yield from _wait(sfull[ss], i // NSS, f"epilogue{k}")   # the block's scale slabs
-            for _ in range(gpb_of(i)):
-                slot, use = q + 2 * (n[q] % own_n), n[q] // own_n
-                n[q] += 1
-                yield from _wait(accf[slot], use, f"epilogue{k}")
-                for _ in range(rng.randint(0, 6)):
-                    yield
-                acce[slot].arrive()
-            sempty[ss].arrive()    # scales read: the slot is free
+        for bt in range(nbatch):
+            yield from _wait(accf[bt % NBUF], bt // NBUF, f"epilogue{k}")
+            for _ in range(rng.randint(0, 4)):
+                yield
+            acce[bt % NBUF].arrive()
 
-    roles = [producer(), issuer(0), issuer(1)] + [unpack(k) for k in range(n_unpack)]
+    roles = [w_producer()] + [issuer(q) for q in range(n_iss)] + [unpack(k) for k in range(8)]
     roles += [epilogue(k) for k in range(n_epi)]
     for _ in range(2000000):
-        if not roles:
+        if not roles and not pending:
+            assert all(b.done == -(-max(nblk - i, 0) // NA) for i, b in enumerate(mdone))
             return
         for p in list(pending):
             p[0] -= 1
             if p[0] <= 0:
                 pending.remove(p)
                 p[1]()
+        if not roles:
+            continue
         r = rng.choice(roles)
         try:
             for _ in range(rng.randint(1, 3)):
@@ -193,18 +238,35 @@ def run_decode_model(nblk, gpb_of, NW, NX, NSS, NA, n_slots, rng, n_unpack=8, n_
     raise Unsound("no progress (deadlock)")
 
 
-# rings (packed, tile, scales), A slots, accumulator slots of the three instances:
-# int8 (16, 24, 24, 8, 16); W4 bf16 (12, 16, 16, 6, 8); W3 bf16 (16, 16, 16, 6, 8)
-@pytest.mark.parametrize("NW,NX,NSS,NA,n_slots", [(16, 24, 24, 8, 16), (12, 16, 16, 6, 8), (16, 16, 16, 6, 8)])
-@pytest.mark.parametrize("kind", ["g128", "g64", "ragged_g64", "one", "two"])
-def test_decode_barrier_protocol_is_sound(NW, NX, NSS, NA, n_slots, kind):
+# packed-block ring, A slots, groups per batch of the three instances: int8 (20, 6, 8);
+# W4 bf16 (20, 6, 4); W3 bf16 (24, 6, 4)
+@pytest.mark.parametrize("NW,NA,NBATCH", [(20, 6, 8), (20, 6, 4), (24, 6, 4)])
+@pytest.mark.parametrize("kind", ["g128", "g64", "ragged_g64", "one", "two", "three_g64", "seven"])
+def test_decode_barrier_protocol_is_sound(NW, NA, NBATCH, kind):
     shapes = {
         "g128": (100, lambda i: 1),
         "g64": (60, lambda i: 2),
         "ragged_g64": (45, lambda i: 1 if i % 5 == 4 else 2),   # the last block of each tile holds one group
         "one": (1, lambda i: 1),
         "two": (2, lambda i: 2),
+        "three_g64": (3, lambda i: 2),
+        "seven": (7, lambda i: 1),
     }
     nblk, gpb_of = shapes[kind]
     for seed in range(3):
-        run_decode_model(nblk, gpb_of, NW, NX, NSS, NA, n_slots, random.Random(seed))
+        run_decode_model(nblk, gpb_of, NW, NA, random.Random(seed), NBATCH=NBATCH)
+
+
+@pytest.mark.parametrize("N,K,group", [(29568, 8192, 128), (8192, 29568, 128), (640, 1088, 64), (136, 320, 64)])
+def test_group_count_closed_form(N, K, group):
+    """The kernel counts a CTA's groups as nblk * gpb minus one per tile end in its range when the
+    last K block of a tile holds one group (K = 64 mod 128 at g = 64)."""
+    NT, KB, NB, G, _ = plan(N, K)
+    gpb = 128 // group
+    G_total = -(-K // group)
+    for c in range(G):
+        b0, b1 = range_begin(c, NB, G), range_begin(c + 1, NB, G)
+        walk = sum(min(gpb, G_total - (f % KB) * gpb) for f in range(b0, b1))
+        ragged = G_total < KB * gpb
+        closed = (b1 - b0) * gpb - ((b1 // KB - b0 // KB) if ragged else 0)
+        assert walk == closed
