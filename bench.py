@@ -483,7 +483,7 @@ def product_roofline(cfg, layers, T, prod_ms, peaks, int8, traffic):
     """Roofline of the dominant kernel (the main product) for one timed layer set."""
     from quantized_gemm_moe_b200 import roofline
     wonly = cfg.a_bits == 16
-    kernel = "wgemm" if wonly else "qgemm"
+    kernel = "qdec" if T <= 16 else ("wgemm" if wonly else "qgemm")
     if T <= 16:
         # decode: HBM bound; the product streams the packed codes, the scales and the adapters
         by = sum(roofline.layer_bytes(T, L["proj"].d_in, L["proj"].d_out, cfg.group, cfg.w_bits, cfg.rank_shared,
@@ -597,8 +597,13 @@ def run_ours(args, workload):
                                       cfg.n_routed, cfg.rank_routed, xb, 2, 2 if cfg.scale_fp16 else 4)
                  for L in layers)
     prod_ms = stage_ms[:, :, 2].sum(axis=1).mean()  # the product kernels of one step
-    kernel_file = "quantized_gemm_moe_b200/csrc/k_wgemm.cu" if wonly else "quantized_gemm_moe_b200/csrc/k_gemm.cu"
-    traffic = read_traffic(kernel_file, ("wgemm_" if wonly else "qgemm_") + workload) if not args.tokens else None
+    if T <= 16:
+        kernel_file, kname = "quantized_gemm_moe_b200/csrc/k_decode.cu", "qdec_"
+    elif wonly:
+        kernel_file, kname = "quantized_gemm_moe_b200/csrc/k_wgemm.cu", "wgemm_"
+    else:
+        kernel_file, kname = "quantized_gemm_moe_b200/csrc/k_gemm.cu", "qgemm_"
+    traffic = read_traffic(kernel_file, kname + workload) if not args.tokens else None
     roof = product_roofline(cfg, layers, T, prod_ms, peaks, int8, traffic)
     per_proj = per_projection(cfg, layers, T, stage_ms)
 
@@ -654,8 +659,7 @@ def run_ours(args, workload):
                 s_ms, st_ms, dclk = time_layer_set(qe, dl, dT, args, flush, pg, stages)
                 tot = max_over_ranks(float(s_ms.sum()), pg, dev)
                 pm = st_ms[:, :, 2].sum(axis=1).mean()
-                dfile = "quantized_gemm_moe_b200/csrc/" + ("k_wgemm.cu" if dcfg.a_bits == 16 else "k_gemm.cu")
-                dtraffic = read_traffic(dfile, ("wgemm_" if dcfg.a_bits == 16 else "qgemm_") + f"{dname}_t{dT}")
+                dtraffic = read_traffic("quantized_gemm_moe_b200/csrc/k_decode.cu", f"qdec_{dname}_t{dT}")
                 decode.append({
                     "workload": dname, "T": dT,
                     "description": f"72B decode gate/up/down, T={dT}, {'W3A16' if dcfg.w_bits == 3 else 'W4A8'} g128"

@@ -249,21 +249,21 @@ struct GroupPos {
 
 // ad[nt][r][p] = sum_j B_catT[nt*128 + r][j] * U_cat[p][j] for p < T (zero for p >= T and rows past
 // d_out): the adapter term of row r of tile nt, fp16 inputs (U_cat staged as fp32 in u_s) and fp32
-// sums. Two passes of eight tokens keep the register footprint small (the row's second read hits L1).
+// sums. The row is read eight 16-byte pieces at a time, all in flight together.
 __device__ __forceinline__ void adapter_row(const DecArgs& a, const float* u_s, int nt, int r) {
   const int o = nt * kTileN + r;
-  float4* dst = reinterpret_cast<float4*>(a.ad + (static_cast<size_t>(nt) * kTileN + r) * kDN);
+  float acc[kDN];
+#pragma unroll
+  for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
   const uint4* brow = reinterpret_cast<const uint4*>(a.bcat + static_cast<size_t>(o) * a.R_pad);
   const int n8 = (o < a.N) ? a.R_pad / 8 : 0;
-#pragma unroll 1
-  for (int ph = 0; ph < 2; ++ph) {
-    float acc[8];
+  for (int c0 = 0; c0 < n8; c0 += 8) {
+    uint4 bv[8];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) acc[p] = 0.0f;
-#pragma unroll 2
-    for (int c = 0; c < n8; ++c) {
-      const uint4 bv = __ldg(brow + c);
-      const __half2* bh = reinterpret_cast<const __half2*>(&bv);
+    for (int k = 0; k < 8; ++k) bv[k] = (c0 + k < n8) ? __ldg(brow + c0 + k) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const __half2* bh = reinterpret_cast<const __half2*>(&bv[k]);
       float bf[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -271,11 +271,11 @@ __device__ __forceinline__ void adapter_row(const DecArgs& a, const float* u_s, 
         bf[2 * q] = f.x;
         bf[2 * q + 1] = f.y;
       }
+      const int j0 = min(c0 + k, n8 - 1) * 8;  // pieces past the row are zero: any in-range U column
 #pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const float* u = u_s + (8 * ph + p) * a.R_pad + c * 8;
-        const float4 u0 = *reinterpret_cast<const float4*>(u);
-        const float4 u1 = *reinterpret_cast<const float4*>(u + 4);
+      for (int p = 0; p < kDN; ++p) {
+        const float4 u0 = *reinterpret_cast<const float4*>(u_s + p * a.R_pad + j0);
+        const float4 u1 = *reinterpret_cast<const float4*>(u_s + p * a.R_pad + j0 + 4);
         float t = acc[p];
         t = fmaf(bf[0], u0.x, t);
         t = fmaf(bf[1], u0.y, t);
@@ -288,9 +288,10 @@ __device__ __forceinline__ void adapter_row(const DecArgs& a, const float* u_s, 
         acc[p] = t;
       }
     }
-    dst[2 * ph] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    dst[2 * ph + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
+  float4* dst = reinterpret_cast<float4*>(a.ad + (static_cast<size_t>(nt) * kTileN + r) * kDN);
+#pragma unroll
+  for (int k = 0; k < kDN / 4; ++k) dst[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
 }
 
 template <bool I8, int BITS>
@@ -507,8 +508,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(32 * q4) << 16;
     const int T = a.T;
 
-    // U_cat as fp32 for the adapter terms (computed when this CTA publishes the first segment of a
-    // tile: any CTA's fix-up of the tile reads them only after that)
+    // adapter terms of the tiles whose first block this CTA streams, computed while the pipeline
+    // fills (any CTA's fix-up of such a tile reads them only after this CTA has published its
+    // segment of the tile); U_cat is staged as fp32 first
     if (a.su_sorted) {
       const int nv = kDN * a.R_pad / 8;  // 8 halves per vector; R_pad is a multiple of 8
       for (int v = et; v < nv; v += 128) {
@@ -526,6 +528,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
         *reinterpret_cast<float4*>(u_s + v * 8 + 4) = hi;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int nt_a0 = static_cast<int>((b0 + a.KB - 1) / a.KB), nt_a1 = static_cast<int>((b1 - 1) / a.KB);
+      for (int nt = nt_a0; nt <= nt_a1; ++nt) adapter_row(a, u_s, nt, r);
     }
 
     bool ok = true;
@@ -646,15 +650,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
     };
     for (int b = 0; b < C::kScaleBatches - 1; ++b) request_batch_scales(b);
 
-    // A new tile starts in the group sequence: finish the previous one; when this CTA streams the
-    // tile's first block, compute the tile's adapter term now (it goes out with this CTA's segment,
-    // before any fix-up of the tile can read it)
-    auto enter_tile = [&](int nt, int kb) {
+    // a new tile starts in the group sequence: finish the previous one
+    auto enter_tile = [&](int nt) {
       if (cur_nt >= 0) finish_segment(cur_nt);
       cur_nt = nt;
 #pragma unroll
       for (int p = 0; p < kDN; ++p) acc[p] = 0.0f;
-      if (a.su_sorted && kb == 0) adapter_row(a, u_s, nt, r);
     };
 
     GroupPos gp;
@@ -669,7 +670,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const int nb = min(NBATCH, gleft);
       gleft -= nb;
       const uint32_t bcol = tmem + lane_base + colAcc + buf * (NBATCH * kDN);
-      if (gp.bp.nt != cur_nt) enter_tile(gp.bp.nt, gp.bp.kb);
+      if (gp.bp.nt != cur_nt) enter_tile(gp.bp.nt);
       const int j0 = gp.bp.kb * gpb + gp.gi;
       if (ok && nb == NBATCH && nb <= a.G_total - j0 && !a.dbg_acc) {
         // the whole batch lies in the current tile: its groups are consecutive in the weight's
@@ -700,7 +701,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
       } else {
         for (int k = 0; k < nb; ++k, gp.next(a.KB, gpb, a.G_total)) {
           const int nt = gp.bp.nt;
-          if (nt != cur_nt) enter_tile(nt, gp.bp.kb);
+          if (nt != cur_nt) enter_tile(nt);
           if (!ok) continue;
           uint32_t v[kDN];
           tmem_ld16(bcol + k * kDN, v);
