@@ -99,7 +99,7 @@ def parse_args(argv=None):
                     help="leave out the decode-shaped 72B layers measured beside the default workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-mode", choices=["serial", "overlap"], default="serial",
+    ap.add_argument("--e2e-mode", choices=["serial", "overlap"], default="overlap",
                     help="serial: each layer's copy in, forward and copy out on one stream; overlap: copies "
                          "on their own streams, so layer i+1's input and layer i-1's output cross PCIe while "
                          "layer i computes")

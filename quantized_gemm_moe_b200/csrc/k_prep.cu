@@ -594,6 +594,23 @@ __device__ __forceinline__ float slot_sum(const float* __restrict__ p, size_t sl
   return acc;
 }
 
+// Sum of slots j, j + g, j + 2g, ... of one column, in that order, eight loads in flight.
+__device__ __forceinline__ float slot_sum_strided(const float* __restrict__ p, size_t slot_stride, int nslots, int j,
+                                                  int g) {
+  float acc = 0.0f;
+  for (int s0 = j; s0 < nslots; s0 += 8 * g) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int s = s0 + i * g;
+      v[i] = (s < nslots) ? __ldg(p + static_cast<size_t>(s) * slot_stride) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc += v[i];
+  }
+  return acc;
+}
+
 // Grid-wide barrier for a cooperative launch: every CTA is resident, so each waits until all
 // have arrived. *ctr must be 0 when the kernel starts. The wait gives up after about two
 // seconds of clock cycles, records an error and returns false.
@@ -726,6 +743,8 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
   constexpr int kB = RowBatch<BF16>::kIters;
   __shared__ int wcnt[kWarps][kMaxRouted], wbase[kWarps][kMaxRouted];
   __shared__ int tot_s[kMaxRouted], before_s[kMaxRouted], run_s[kMaxRouted];
+  __shared__ float lpart_s[kRQThreads];  // router-logit partials of the token groups ([group][g][n_r])
+  __shared__ float gmx_s[kWarps];        // per-warp maxima of a group's adapter row
   extern __shared__ float4 rq_dyn[];
   float* s_inv_s = reinterpret_cast<float*>(rq_dyn);
   float* u_w = s_inv_s + a.K;
@@ -740,6 +759,9 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
   int wpt = 1;
   while (wpt * 2 * a.chunk <= kWarps) wpt *= 2;
   const int sub = warp % wpt, slot = warp / wpt, nslot_w = kWarps / wpt;
+  // A token's wpt warps meet at named barrier 1 + slot when they share its slot sums (wpt >= 2).
+  const int gthr = wpt * 32, gtid = sub * 32 + lane;
+  auto group_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + slot), "r"(gthr) : "memory"); };
   for (int i = threadIdx.x; i < a.K / 4; i += kRQThreads)
     reinterpret_cast<float4*>(s_inv_s)[i] = __ldg(reinterpret_cast<const float4*>(a.s_inv) + i);
   for (int i = threadIdx.x; i < t1 - t0; i += kRQThreads) mx_s[i] = 0;
@@ -751,10 +773,25 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
   if (a.do_route) {
     // ---- per token: logits, argmin (the token's first warp), absmax (all of its warps)
     for (int t = t0 + slot; t < t1; t += nslot_w) {
+      // with several warps per token, they split each logit's slot sum: thread (j, e) adds slots
+      // j, j + g, ... of column e, and the token's first warp adds the g partials in order
+      const int lg = gthr / n_r;
+      float* lp = lpart_s + slot * gthr;
+      if (wpt > 1) {
+        if (gtid < lg * n_r)
+          lp[gtid] = slot_sum_strided(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_rt + gtid % n_r, slot_stride,
+                                      a.nslots, gtid / n_r, lg);
+        group_sync();
+      }
       if (sub == 0) {
-        const float L = (lane < n_r) ? slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_rt + lane,
-                                                slot_stride, a.nslots)
-                                     : 0.0f;
+        float L = 0.0f;
+        if (lane < n_r) {
+          if (wpt > 1) {
+            for (int j = 0; j < lg; ++j) L += lp[j * n_r + lane];
+          } else {
+            L = slot_sum(a.partial + static_cast<size_t>(t) * a.R_tot + a.R_rt + lane, slot_stride, a.nslots);
+          }
+        }
         float best = (lane < n_r) ? L : INFINITY;
         int bi = (lane < n_r) ? lane : 0x7fffffff;
 #pragma unroll
@@ -929,6 +966,50 @@ __global__ void __launch_bounds__(kRQThreads) k_route_quant(const RouteQuantArgs
           *reinterpret_cast<uint4*>(a.act16 + p * a.K + k) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
+    }
+    if (wpt > 1 && a.kc == 0 && a.R_pad > 0) {
+      // the token's wpt warps build its adapter row together: thread (j, c) adds slots j, j + g,
+      // ... of column c into a partial row, then column c's g partials are added in order
+      if (sub == 0 && a.codes && lane == 0) a.sa_sorted[p] = sa;
+      const int e = e_s[t - t0];
+      const int g = max(1, gthr / a.R_pad);
+      float* part = u_w + static_cast<size_t>(slot) * wpt * a.R_pad;  // the group's wpt rows: [g][R_pad]
+      float* row = part + static_cast<size_t>(g) * a.R_pad;           // then the summed row (g + 1 <= wpt)
+      const float* prow = a.partial + static_cast<size_t>(t) * a.R_tot;
+      for (int idx = gtid; idx < g * a.R_pad; idx += gthr) {
+        const int c = idx % a.R_pad, j = idx / a.R_pad;
+        float v = 0.0f;
+        if (c < a.R_a && (c < a.r_s || (c - a.r_s) / a.r_r == e)) v = slot_sum_strided(prow + c, slot_stride, a.nslots, j, g);
+        part[idx] = v;
+      }
+      group_sync();
+      float mx = 0.0f;
+      for (int c = gtid; c < a.R_pad; c += gthr) {
+        float v = 0.0f;
+        for (int j = 0; j < g; ++j) v += part[j * a.R_pad + c];
+        row[c] = v;
+        mx = fmaxf(mx, fabsf(v));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      if (lane == 0) gmx_s[warp] = mx;
+      group_sync();
+      mx = 0.0f;
+      for (int w = 0; w < wpt; ++w) mx = fmaxf(mx, gmx_s[slot * wpt + w]);
+      float su = 1.0f;
+      if (mx > 0.0f) {
+        int ex;
+        frexpf(mx, &ex);  // mx = m * 2^ex, m in [0.5, 1)
+        su = ldexpf(1.0f, ex - 14);
+      }
+      const float inv_su = 1.0f / su;  // exact: su is a power of two
+      for (int c = gtid; c < a.R_pad; c += gthr) {
+        __half h = __float2half_rn(row[c] * inv_su);
+        a.ucat[p * a.R_pad + c] = *reinterpret_cast<uint16_t*>(&h);
+      }
+      if (gtid == 0) a.su_sorted[p] = su;
+      group_sync();  // the rows are free for the group's next token
+      continue;
     }
     if (sub != 0) continue;
     if (a.codes && lane == 0) a.sa_sorted[p] = sa;
