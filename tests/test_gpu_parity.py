@@ -577,3 +577,39 @@ def test_forward_full_size_is_deterministic(proj_index):
     for y in ys[1:]:
         bad = (~(y == ys[0]).all(dim=1)).nonzero().flatten().tolist()
         assert not bad, f"rows differing between runs: {bad[:10]}"
+
+
+# ---------------------------------------------------------------- fp16 range of the packed up-projections
+
+def test_adapter_up_projection_beyond_fp16_range_is_reported():
+    # The packed up-projections are fp16 (qe.h, qe_pack_adapters). A bf16 value beyond 65504 is
+    # stored as 65504 and reported through the device error word (0x201); values inside the
+    # range leave the word clear.
+    cfg = _cfg(T=16)
+    proj = cfg.projections[0]
+    inp = qi.layer_inputs(cfg, proj, T=16)
+    assert qe.device_error() == 0
+    Case(cfg, proj, 16, inp=inp)
+    assert qe.device_error() == 0
+    big = dict(inp)
+    B = inp["B_s"].clone()
+    B[0, 5] = 1.0e5
+    big["B_s"] = B
+    Case(cfg, proj, 16, inp=big)
+    assert qe.device_error() == 0x201
+    assert qe.device_error() == 0  # reading the word cleared it
+
+
+@pytest.mark.parametrize("T", [16, 300])
+def test_adapter_up_projection_below_fp16_normal_range(T):
+    # Up-projection entries around 2e-6 sit in fp16's subnormal range (below 2^-14), where the
+    # packed values keep fewer significant bits. The forward (decode product at T = 16, the int8
+    # GEMM at T = 300) still meets the output tolerance against the oracle, which uses the bf16
+    # values exactly.
+    cfg = _cfg(T=T)
+    proj = cfg.projections[0]
+    inp = qi.layer_inputs(cfg, proj, T=T)
+    small = dict(inp)
+    small["B_s"] = (inp["B_s"].float() * 1e-4).to(torch.bfloat16)
+    small["B_r"] = (inp["B_r"].float() * 1e-4).to(torch.bfloat16)
+    _forward_check(Case(cfg, proj, T, inp=small))
