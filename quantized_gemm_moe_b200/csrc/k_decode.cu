@@ -14,22 +14,24 @@
 // hand-off decides the speed: an MMA or a commit keeps its issuing thread ~140 cycles whatever N
 // is (several issuing threads overlap), and every dependent barrier step of a role costs a few
 // hundred cycles. The roles are laid out to keep those steps few per byte:
-//   warp 0      bulk copy of each packed block into a 20-24 deep ring (~150 KB in flight per SM),
-//               freed by the unpack team as soon as it has read the block; and TMA of each
-//               block's activation tile (16 tokens x 128 channels) into the slot of the block's
-//               unpacked weights, free again once the block's MMAs are done. One thread polls both.
+//   warp 0      bulk copy of each packed block into a 16-20 deep ring (120-160 KB in flight per
+//               SM), freed by the unpack team as soon as it has read the block. No earlier kernel
+//               writes the weights, so the stream starts before the previous grid has finished.
 //   warps 4-11  unpack the block straight into tensor memory with tcgen05.st: the MMA takes its
 //               A operand (the weights, M = 128 output rows = TMEM lanes, K along the columns)
 //               from TMEM, so the unpacked weights never pass through shared memory. Two teams of
 //               four warps (one per TMEM lane quarter) take alternate blocks, a row per thread.
 //   warps 1-3   one thread each issues the MMAs of every third block: kind::i8 (codes x16 against
 //               int8 activation codes, 4 K steps) or kind::f16 (bf16 weights against bf16
-//               activations, 8 K steps), one commit per block (frees the A slot and the tile).
+//               activations, 8 K steps), one commit per block (frees the block's A slot). Each
+//               also loads the activation tiles (16 tokens x 128 channels, TMA) of its own blocks
+//               six blocks ahead, into a 12-slot ring.
 //               Every quantization group gets a fresh 16-column accumulator; eight (bf16: four)
 //               consecutive groups share one batch buffer (two buffers), committed once per batch.
 //   warps 12-15 epilogue, one output row per thread, a batch of groups at a time: the group
-//               sums (int8 sums converted exactly) times the group scales (loaded by the thread a
-//               batch ahead), the segment partials and the per-tile fix-up, which adds su times
+//               sums (int8 sums converted exactly) times the group scales (each thread copies its
+//               own with cp.async, three batches ahead), the segment partials and the per-tile
+//               fix-up, which adds su times
 //               the adapter term U_cat . B_catT of the tile. The adapter terms of the tiles whose
 //               first block this CTA streams are computed by these threads while the pipeline fills.
 #include <cuda_bf16.h>
@@ -56,9 +58,8 @@ struct DCfg {
   static constexpr int kXTile = I8 ? kXAtom : 2 * kXAtom;  // 128 input channels: int8 codes or bf16
   static constexpr int kACols = I8 ? 32 : 64;             // TMEM columns of one unpacked block
   static constexpr int kKSteps = I8 ? 4 : 8;              // MMA K steps per block (32 int8 / 16 bf16)
-  // unpacked blocks in TMEM (the activation tile of a block sits in the shared-memory slot of the
-  // same index): unpack -> MMA -> slot free spans this many blocks. A multiple of 6, so that each
-  // of the two unpack teams and each of the three issuers keeps its own slots.
+  // unpacked blocks in TMEM: unpack -> MMA -> slot free spans this many blocks. A multiple of 6,
+  // so that each of the two unpack teams and each of the three issuers keeps its own slots.
   static constexpr int kASlots = 6;
   static constexpr int kBatch = I8 ? 8 : 4;               // groups per epilogue batch (16 columns each)
   static constexpr int kBufs = 2;                         // batch buffers
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
   uint8_t* xring = smem;                              // [NX][kXTile], 1024-aligned (128B swizzle)
   uint8_t* wring = xring + NX * C::kXTile;            // [NW][kWBlock]
   float* u_s = reinterpret_cast<float*>(wring + NW * C::kWBlock);  // U_cat as fp32 [16][R_pad]
-  uint32_t* sc_s = reinterpret_cast<uint32_t*>(u_s + kDN * kMaxRpad);  // [3][NBATCH][128] scale words
+  uint32_t* sc_s = reinterpret_cast<uint32_t*>(u_s + kDN * kMaxRpad);  // [4][NBATCH][128] scale words
   uint64_t* bars = reinterpret_cast<uint64_t*>(sc_s + C::kScaleBatches * NBATCH * kTileN);
   uint64_t* wfull = bars;          // [NW] packed block landed (1 + bytes)
   uint64_t* wempty = wfull + NW;   // [NW] the unpack team has read it (4 warps)
@@ -489,7 +490,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const uint32_t ta = tmem + lane_base + colA + s * C::kACols;
       unpack_half_row<I8, BITS>(wring + sw * C::kWBlock, r, 0, ta);
       unpack_half_row<I8, BITS>(wring + sw * C::kWBlock, r, 1, ta + C::kACols / 2);
-      // the packed block's values have been read (the stores below hold them): free its slot now
+      // the packed block's values are in registers, handed to the tcgen05.st above: free its slot now
       __syncwarp();
       if (lane == 0) mbar_arrive(&wempty[sw]);
       tmem_wait_st();
