@@ -280,12 +280,18 @@ QE_API int32_t qe_linear_kernel_launches(const qe_layer_desc* desc, int32_t T, q
  *   weight_only          1 for a_bits = 16 (the weight-only product)
  *   workspace_bytes      the scratch this call needs for this x_dtype (qe_linear_workspace_bytes
  *                        is the larger of the fp32 and bf16 needs)
+ *   decode_product       1 when the product is the decode-batch kernel (T <= 16 and, with
+ *                        adapters, R_pad <= 384): the (128-row tile, 128-channel block) sequence
+ *                        split evenly over decode_ctas CTAs, at most decode_max_segments
+ *                        pieces per output tile; 0 (and 0, 0) otherwise. The CTA count is
+ *                        the current device's SM count (148 when no device is visible).
  * Returns QE_ERR_INVALID_ARG for a null pointer or T < 1, and check errors of desc.
  */
 typedef struct {
   int32_t product_tile_tokens, product_k_splits, adapter_atoms, adapter_gemm_width, adapter_gemm_tile,
       adapter_gemm_splits, weight_only;
   int64_t workspace_bytes;
+  int32_t decode_product, decode_ctas, decode_max_segments;
 } qe_linear_plan_info;
 QE_API qe_status qe_linear_plan(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype, qe_linear_plan_info* out);
 

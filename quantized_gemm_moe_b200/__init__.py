@@ -56,7 +56,8 @@ class LayerDesc(ctypes.Structure):
 class LinearPlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("product_tile_tokens", "product_k_splits", "adapter_atoms",
                                               "adapter_gemm_width", "adapter_gemm_tile", "adapter_gemm_splits",
-                                              "weight_only")] + [("workspace_bytes", ctypes.c_int64)]
+                                              "weight_only")] + [("workspace_bytes", ctypes.c_int64)] + [
+        (n, ctypes.c_int32) for n in ("decode_product", "decode_ctas", "decode_max_segments")]
 
 
 class LayerWeights(ctypes.Structure):

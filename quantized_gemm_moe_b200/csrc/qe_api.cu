@@ -514,6 +514,9 @@ qe_status qe_linear_plan(const qe_layer_desc* desc, int32_t T, qe_dtype x_dtype,
   out->adapter_gemm_splits = p.uslots;
   out->weight_only = desc->a_bits == 16 ? 1 : 0;
   out->workspace_bytes = static_cast<int64_t>(p.bytes);
+  out->decode_product = p.dec ? 1 : 0;
+  out->decode_ctas = p.dec ? p.dp.grid : 0;
+  out->decode_max_segments = p.dec ? p.dp.maxseg : 0;
   return QE_OK;
 }
 

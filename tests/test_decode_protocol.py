@@ -270,3 +270,42 @@ def test_group_count_closed_form(N, K, group):
         ragged = G_total < KB * gpb
         closed = (b1 - b0) * gpb - ((b1 // KB - b0 // KB) if ragged else 0)
         assert walk == closed
+
+
+# (T, K, N, group, a_bits, w_bits, r_s, N_r, r_r): the 72B decode projections, the decode parity
+# shapes' corners, and a rank that takes the adapters past the decode product's 384 columns
+PLAN_SHAPES = [
+    (16, 8192, 29568, 128, 8, 4, 32, 8, 4), (16, 29568, 8192, 128, 8, 4, 32, 8, 4), (1, 8192, 29568, 128, 16, 3, 32, 8, 4),
+    (2, 320, 200, 64, 16, 3, 8, 4, 4), (7, 8192, 128, 128, 8, 4, 32, 8, 4), (16, 29568, 256, 128, 6, 4, 32, 8, 4),
+    (16, 1024, 1000, 128, 8, 4, 0, 1, 0), (13, 1024, 640, 128, 6, 4, 32, 8, 32),
+]
+
+
+@pytest.mark.parametrize("T,K,N,group,a_bits,w_bits,rs,nr,rr", PLAN_SHAPES)
+def test_library_decode_plan_matches_the_model(T, K, N, group, a_bits, w_bits, rs, nr, rr):
+    """The schedule these models check is the one the library plans: qe_linear_plan reports the
+    decode product's CTA count and segment bound, computed by the C code, host only."""
+    import quantized_gemm_moe_b200 as qe
+    try:
+        qe.load()
+    except Exception as e:  # pragma: no cover - the build step makes the library
+        pytest.skip(f"libqe.so not built: {e}")
+    p = qe.linear_plan(qe.make_desc(K, N, group, w_bits, a_bits, rs, nr, rr), T, qe.QE_BF16)
+    assert p["decode_product"] == 1
+    NT, KB, NB, G, maxseg = plan(N, K, p["decode_ctas"])
+    assert p["decode_ctas"] == G
+    assert p["decode_max_segments"] == maxseg
+    assert p["product_tile_tokens"] == 16 and p["product_k_splits"] == 1
+
+
+def test_library_decode_plan_limits():
+    import quantized_gemm_moe_b200 as qe
+    try:
+        qe.load()
+    except Exception as e:  # pragma: no cover
+        pytest.skip(f"libqe.so not built: {e}")
+    # 17 tokens, and adapters wider than 384 columns (R_pad = 448), run on the GEMM instead
+    assert qe.linear_plan(qe.make_desc(8192, 4096, 128, 4, 8, 32, 8, 4), 17)["decode_product"] == 0
+    wide = qe.linear_plan(qe.make_desc(8192, 4096, 128, 4, 8, 64, 8, 48), 16)
+    assert wide["decode_product"] == 0 and wide["decode_ctas"] == 0 and wide["decode_max_segments"] == 0
+    assert qe.linear_plan(qe.make_desc(8192, 4096, 128, 4, 8, 64, 8, 40), 16)["decode_product"] == 1  # R_pad 384
