@@ -120,8 +120,10 @@ class TaggedBarrier(Barrier):
         self.arrive()
 
 
-def run_decode_model(nblk, gpb_of, NW, NA, rng, NBUF=2, NBATCH=8, n_epi=4, n_iss=3):
-    """nblk blocks; gpb_of(i) = groups of block i (1, or 2 at g = 64, 1 for the ragged last K block)."""
+def run_decode_model(nblk, gpb_of, NW, NA, rng, NBUF=2, NBATCH=8, n_epi=4, n_iss=3, tiles_ahead=None):
+    """nblk blocks; gpb_of(i) = groups of block i (1, or 2 at g = 64, 1 for the ragged last K block).
+    tiles_ahead: how far ahead (in blocks) an issuer requests activation tiles; the kernel's NA."""
+    ahead = NA if tiles_ahead is None else tiles_ahead
     wfull = [Barrier(f"wfull{i}", 1) for i in range(NW)]
     wempty = [Barrier(f"wempty{i}", 4) for i in range(NW)]
     NX = 2 * NA
@@ -195,7 +197,7 @@ def run_decode_model(nblk, gpb_of, NW, NA, rng, NBUF=2, NBATCH=8, n_epi=4, n_iss
                 continue
             s = i % NA
             yield from _wait(afull[s], i // NA, f"issuer{q}")
-            request_tiles(i + NA)
+            request_tiles(i + ahead)
             yield from _wait(xfull[i % NX], i // NX, f"issuer{q}")
             for _ in range(ng):
                 bt = gidx // NBATCH
@@ -309,3 +311,15 @@ def test_library_decode_plan_limits():
     wide = qe.linear_plan(qe.make_desc(8192, 4096, 128, 4, 8, 64, 8, 48), 16)
     assert wide["decode_product"] == 0 and wide["decode_ctas"] == 0 and wide["decode_max_segments"] == 0
     assert qe.linear_plan(qe.make_desc(8192, 4096, 128, 4, 8, 64, 8, 40), 16)["decode_product"] == 1  # R_pad 384
+
+
+def test_decode_model_catches_early_tile_requests():
+    """Control: requesting the activation tiles three blocks further ahead than the kernel does
+    reuses a tile slot whose MMAs may still be reading it; the model must see that."""
+    caught = 0
+    for seed in range(10):
+        try:
+            run_decode_model(100, lambda i: 1, 20, 6, random.Random(seed), NBATCH=8, tiles_ahead=6 + 3)
+        except Unsound:
+            caught += 1
+    assert caught >= 8
