@@ -323,3 +323,57 @@ def test_decode_model_catches_early_tile_requests():
         except Unsound:
             caught += 1
     assert caught >= 8
+
+
+@pytest.mark.parametrize("nbatch", [1, 2, 3, 4, 5, 13, 40])
+def test_scale_ring_reads_landed_slots_that_are_not_being_rewritten(nbatch):
+    """The epilogue's group scales: each thread requests batch b's scales into slot b % R (R = 4)
+    as one cp.async group, R - 1 batches ahead, and before reading batch b waits with
+    cp.async.wait_group R - 1: every group except the R - 1 most recently committed has landed.
+    Other groups land in any order."""
+    R = 4
+    rng = random.Random(nbatch)
+    slot_owner = {}      # slot -> batch whose copy last went into it
+    committed = []       # groups in commit order: batch, or None for an empty group
+    landed = set()
+
+    def request(b):
+        if b < nbatch:
+            slot_owner[b % R] = b
+        committed.append(b if b < nbatch else None)   # an empty group is committed all the same
+
+    for b in range(R - 1):
+        request(b)
+    for bt in range(nbatch):
+        request(bt + R - 1)
+        for g in committed:                  # some copies land early, in any order
+            if g is not None and rng.random() < 0.3:
+                landed.add(g)
+        for g in committed[:-(R - 1)]:       # cp.async.wait_group R - 1
+            if g is not None:
+                landed.add(g)
+        assert bt in landed                  # this batch's scales are there
+        assert slot_owner[bt % R] == bt      # and no later batch has been requested into its slot
+
+
+@pytest.mark.parametrize("R_pad", [64, 128, 192, 320, 384, 512])
+@pytest.mark.parametrize("chunk", [1, 2, 3, 5, 8, 16, 100])
+def test_route_quant_group_sum_layout_fits(R_pad, chunk):
+    """k_route_quant with several warps per token: the token group's partial rows [g][R_pad] and
+    its summed row fit in the group's wpt adapter rows, the logit partials in the static buffer,
+    and the named barrier ids stay in 1..15."""
+    kWarps, kThreads, kMaxRouted = 16, 512, 16
+    wpt = 1
+    while wpt * 2 * chunk <= kWarps:
+        wpt *= 2
+    nslot_w = kWarps // wpt
+    if wpt == 1:
+        return                                   # one warp per token: the per-warp path
+    gthr = wpt * 32
+    g = max(1, gthr // R_pad)
+    assert (g + 1) * R_pad <= wpt * R_pad        # partials + summed row inside the group's rows
+    for n_r in range(1, kMaxRouted + 1):
+        lg = gthr // n_r
+        assert lg >= 1 and lg * n_r <= gthr      # this group's share of the logit buffer
+        assert (nslot_w - 1) * gthr + gthr <= kThreads
+    assert 1 <= 1 + (nslot_w - 1) <= 15
